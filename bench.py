@@ -1,0 +1,410 @@
+#!/usr/bin/env python
+"""Benchmark of the MPQ row solve on B200.
+
+One step = one whole solve of a layer (init, T_vamp VAMP iterations, marginal
+MAP, <= 3 CD sweeps, energies) through the C ABI with W already resident in
+HBM.  Default workload: the 4096x4096 q_proj-shaped layer, 4-bit scalar grid,
+T_vamp = 16, 3 CD sweeps, X 8192x4096 (synthetic, seeded).  Setup (the
+compact SVD of X on the device) is timed separately and not part of a step.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mpq|reference]
+
+With N > 1 (torchrun, one rank per GPU) every rank solves its own rows of a
+layer with N*m_out rows (weak scaling, no data-path collective); the time is
+the max over ranks.  `--impl reference` times the float64 CPU oracle on a
+bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MPQ solve weights/sec (VAMP+3 CD sweeps) per layer; % of roofline"
+UNIT = "weights/s"
+FP32_ALU_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12  # FMA lanes x 2 x max SM clock
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="mpq", choices=["mpq", "reference"])
+    ap.add_argument("--config", default="q4096")
+    ap.add_argument("--cpu-rows", type=int, default=8, help="oracle sample size (rows)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ dist ---
+
+def dist_init(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    return world, rank, local
+
+
+def allreduce_max(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------- clocks ---
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.lines = []
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.dev), "-lms", "200"], stdout=subprocess.PIPE,
+                stderr=subprocess.DEVNULL, text=True)
+            threading.Thread(target=self._read, daemon=True).start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------- algorithmic work ---
+
+def kernel_work(name, m, n, r, d, K, L):
+    """(bound, unit, work per launch) -- algorithmic flops or bytes."""
+    if name in ("gemm_project", "gemm_energy", "gemm_expand"):
+        return "alu", "TFLOP/s", 2.0 * m * n * r
+    if name == "gemm_hessian":
+        return "alu", "TFLOP/s", 2.0 * m * n * n
+    if name == "k_denoise_scalar":      # read r1, write xhat1 (+ v per element)
+        return "hbm", "GB/s", 8.0 * m * n
+    if name == "k_extrinsic_d2l":        # read w, r1, xhat1; write r2, A
+        return "hbm", "GB/s", 20.0 * m * n
+    if name == "k_extrinsic_l2d":        # read r2, D; write r1
+        return "hbm", "GB/s", 12.0 * m * n
+    if name == "k_linear_rows":          # read/write U' (m x r)
+        return "hbm", "GB/s", 8.0 * m * r
+    if name == "k_denoise_vec":          # candidate evaluations (exp-bound)
+        return "sfu", "Gexp/s", float(m) * (n // 8) * K
+    return None
+
+
+def source_sha():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "post_weight_quantization_row_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel, workload):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    sha = source_sha()
+    for line in open(path):
+        parts = line.split()
+        if len(parts) == 4 and not line.startswith("#") and parts[0] == kernel and parts[1] == workload:
+            return float(parts[2]) if parts[3] == sha else None
+    return None
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+# ------------------------------------------------------------ workloads ---
+
+def workload(cfg, rank=0):
+    import mpq_inputs as mi
+    p = mi.make_problem(cfg)
+    if rank > 0:
+        # weak scaling: rank k solves other rows of an N*m_out-row layer
+        cfgno = mi.WORKLOADS[cfg][0]
+        g = np.random.default_rng(mi.SEED_BASE + 10 * cfgno + 1000 * rank)
+        W = mi.lognormal_rows_w(g, p.m_out, p.n)
+        if p.d == 8:
+            signs = np.where(mi.rng_for(cfgno, 3).random(p.n) < 0.5, -1.0, 1.0)
+            W = mi.random_hadamard_apply(W, signs)
+        p.W = np.ascontiguousarray(W, dtype=np.float32)
+    return p
+
+
+def describe(p, cfg):
+    bits = {8: 3, 16: 4}.get(p.levels, None) if p.d == 1 else 2
+    return {"workload": f"{cfg}: W {p.m_out}x{p.n}, X {p.X.shape[0]}x{p.n}, "
+                        + (f"{bits}-bit per-row min-max grid" if p.d == 1 else
+                           f"offset-E8 d=8 K={p.levels}, RHT")
+                        + f", T_vamp={p.T_vamp}, CD sweeps<={p.cd_sweeps}",
+            "m_out": p.m_out, "n": p.n, "m_calib": int(p.X.shape[0]), "d": p.d,
+            "levels_or_K": p.levels, "T_vamp": p.T_vamp, "cd_sweeps": p.cd_sweeps,
+            "seeds": p.seeds, "l2": "flushed between timed steps (512 MiB write)"}
+
+
+def oracle_sample(p, rows, steps=1):
+    """Time the float64 oracle on `rows` rows of the layer (spectrum excluded)."""
+    from oracle import mpq_oracle as orc
+    t0 = time.time()
+    s, V = orc.spectrum(p.X)
+    t_spec = time.time() - t0
+    cb = orc.scalar_levels(p.levels) if p.d == 1 else p.codebook.astype(np.float64)
+    times = []
+    for k in range(steps):
+        sel = slice((k * rows) % p.m_out, (k * rows) % p.m_out + rows)
+        t0 = time.perf_counter()
+        orc.solve(p.W[sel], cb, s, V, p.T_vamp, p.cd_sweeps)
+        times.append(time.perf_counter() - t0)
+    return times, t_spec
+
+
+# ------------------------------------------------------------ reference ---
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    p = workload(args.config)
+    rows = max(1, args.cpu_rows // 2)
+    times, t_spec = oracle_sample(p, rows, args.warmup + args.steps)
+    timed = times[args.warmup:]
+    sec = sum(timed) / len(timed)
+    value = rows * p.n / sec
+    cores = len(os.sched_getaffinity(0))
+    cfgd = describe(p, args.config)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": cfgd,
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": f"{rows} rows of the layer per step (rows are independent "
+                                       f"problems), full T_vamp and CD; spectrum "
+                                       f"({t_spec:.1f} s) excluded"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ mpq ---
+
+def run_mpq(args, world, rank, local):
+    import torch
+
+    import post_weight_quantization_row_b200 as mpq
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    p = workload(args.config, rank)
+    cfgd = describe(p, args.config)
+    m, n = p.m_out, p.n
+    X = torch.from_numpy(p.X).to(dev)
+    torch.cuda.synchronize()
+    t0 = time.time()
+    plan = mpq.Plan.from_x(X, p.d, p.levels, codebook=p.codebook if p.d == 8 else None)
+    torch.cuda.synchronize()
+    setup_s = time.time() - t0
+    del X
+    r = plan.r
+    W = torch.from_numpy(p.W).to(dev)
+    out = {"idx": torch.empty(m, plan.B, dtype=torch.int16, device=dev),
+           "w_hat": torch.empty(m, n, dtype=torch.float32, device=dev),
+           "energy": torch.empty(m, dtype=torch.float32, device=dev)}
+    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        plan.solve(W, p.T_vamp, p.cd_sweeps, out=out, check_status=False)
+
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        step()
+    plan.status()
+    torch.cuda.synchronize()
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    launches0 = mpq.kernel_launch_count()
+    with ClockSampler(local) as clk:
+        mpq.profile_start()
+        for i in range(args.steps):
+            flush.fill_(float(i))
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        prof = mpq.profile_stop()
+    launches = mpq.kernel_launch_count() - launches0
+    plan.status()
+    barrier(world)
+    total_ms = sum(a.elapsed_time(b) for a, b in ev)
+    total_ms = allreduce_max(total_ms, world)
+    ms_per_step = total_ms / args.steps
+    value = world * m * n / (ms_per_step / 1e3)
+
+    # roofline of the dominant kernel (largest share of device time)
+    peaks, peak_src = load_peaks()
+    dom = max(prof.items(), key=lambda kv: kv[1][1])
+    name, (cnt, kms) = dom
+    roof = None
+    wk = kernel_work(name, m, n, r, p.d, p.levels, p.levels)
+    if wk:
+        bound, unit, work = wk
+        avg_s = kms / cnt / 1e3
+        if unit == "TFLOP/s":
+            achieved = work / avg_s / 1e12
+            peak = FP32_ALU_PEAK_TFLOPS if bound == "alu" else peaks["bf16_tflops"]
+        elif unit == "GB/s":
+            achieved = work / avg_s / 1e9
+            peak = peaks["hbm_gbs"]
+        else:
+            achieved = work / avg_s / 1e9
+            peak = 148 * 16 * 1.965  # MUFU ex2 per clock per SM x SMs x GHz -> Gexp/s
+        roof = {"bound": bound, "kernel": name, "achieved": achieved, "peak": peak, "unit": unit,
+                "frac": achieved / peak, "traffic": recorded_traffic(name, args.config),
+                "peak_source": ("derived: 148 SMs x 128 FP32 lanes x 2 x 1965 MHz"
+                                if bound == "alu" else f"{peak_src} MEASURED_PEAKS.json"),
+                "work_per_launch": work, "launches": cnt, "avg_launch_ms": kms / cnt}
+    total_prof = sum(v[1] for v in prof.values())
+    kernels = {k: {"launches": v[0], "ms": round(v[1], 4), "share": round(v[1] / total_prof, 4)}
+               for k, v in sorted(prof.items(), key=lambda kv: -kv[1][1])}
+
+    # end to end through the C ABI with host buffers
+    e2e = None
+    if not args.no_e2e:
+        Wh = torch.from_numpy(p.W).pin_memory()
+        ho = {"idx": torch.empty(m, plan.B, dtype=torch.int16, pin_memory=True),
+              "w_hat": torch.empty(m, n, dtype=torch.float32, pin_memory=True),
+              "energy": torch.empty(m, dtype=torch.float32, pin_memory=True)}
+        plan.solve_host(Wh, p.T_vamp, p.cd_sweeps, out=ho)  # warm the staging buffers
+        barrier(world)
+        torch.cuda.synchronize()
+        e2e_ms = 0.0
+        for i in range(args.steps):
+            flush.fill_(float(i))
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            plan.solve_host(Wh, p.T_vamp, p.cd_sweeps, out=ho)
+            b.record(stream)
+            torch.cuda.synchronize()
+            e2e_ms += a.elapsed_time(b)
+        e2e_ms = allreduce_max(e2e_ms, world) / args.steps
+        e2e = {"value": world * m * n / (e2e_ms / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": m * n * 4,
+               "d2h_bytes_per_step": m * plan.B * 2 + m * n * 4 + m * 4,
+               "ms_per_step": e2e_ms}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        times, t_spec = oracle_sample(p, args.cpu_rows)
+        cpu = {"value": args.cpu_rows * n / times[0], "unit": UNIT,
+               "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
+               "sample": f"rows 0..{args.cpu_rows - 1} of the layer (independent problems), "
+                         f"full T_vamp and CD; spectrum ({t_spec:.1f} s) excluded"}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+                "data": "synthetic", "config": dict(cfgd, setup_s=round(setup_s, 3), rank=r,
+                                                    parallelism=f"rows sharded over {world} GPU(s)"),
+                "rows_per_s": world * m / (ms_per_step / 1e3),
+                "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk.summary(),
+                "gpu_launches": launches, "kernels": kernels}
+        print(json.dumps(line), flush=True)
+    plan.close()
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_init(args.gpus)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_mpq(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

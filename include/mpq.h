@@ -1,0 +1,237 @@
+/*
+ * mpq.h -- C ABI of libmpq, a B200 (sm_100a) implementation of the MPQ
+ * row-batched post-training-quantisation solver.
+ *
+ * Source of every operation: "MPQ: A Message-Passing View of Post-Training
+ * Quantization" (papernotes.org NeurIPS 2026 note).  Sections cited below:
+ *   [Overall framework]  row objective 1/2 |Xw - X w_hat|^2 over the product
+ *                        of block codebooks C_1 x ... x C_B, B = n/d;
+ *   [Flowchart]          A = X, y = Xw -> compact SVD (T = Sigma V^T,
+ *                        y~ = U^T y) -> T_vamp x (VAMP soft messages, beta
+ *                        M-step) -> marginal MAP -> Mahalanobis CD;
+ *   [Key design 1]       blockwise denoiser q_b(c) ~ rho_b(c) exp(-gamma1/2
+ *                        |c - r1_b|^2), extrinsic updates, Gaussian linear
+ *                        module solved in rank space;
+ *   [Key design 2]       empirical-Bayes M-step for beta, damped;
+ *   [Key design 3]       marginal-MAP argmax and exact block CD in the metric
+ *                        G_b = T_b^T T_b;
+ *   [Hyper-parameters]   (loss / training strategy section) T_vamp = 16,
+ *                        rho_damp = 0.5, tau, S_CD = 3 with early stop,
+ *                        gamma1_0 = 1/MSE(w, w_rtn), E8 d = 8, M_b = 2^16.
+ * The min-max scalar grid follows the NeUQI note ("Near-Optimal Uniform
+ * Quantization Parameter Initialization for Low-Bit LLMs"), existing pain
+ * points section: s = (max - min)/(2^k - 1), z = -round(min/s).
+ *
+ * Conventions for every entry point:
+ *  - Pointers are DEVICE pointers (memory the caller allocated on the
+ *    plan's device) unless the argument says HOST.  The caller owns every
+ *    buffer it passes and keeps it alive until the stream has finished the
+ *    call.  Row-major layouts throughout.
+ *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream) and the call returns without synchronising, except where noted.
+ *  - Arguments are validated before anything is launched; a rejected call
+ *    launches nothing and returns MPQ_ERR_INVALID_ARG.  Kernels that meet a
+ *    non-finite input or hit an iteration cap set a device status word that
+ *    mpq_plan_status() reads.  Outputs are defined only when both the call
+ *    and the following mpq_plan_status() return MPQ_OK.
+ *  - mpq_last_error() gives a thread-local message for the last failure.
+ *  - No entry point throws; all are thread-compatible per plan (one thread
+ *    at a time per plan).
+ */
+#ifndef MPQ_H_
+#define MPQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MPQ_API __attribute__((visibility("default")))
+#else
+#define MPQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct mpq_plan_s* mpq_plan_t;
+typedef void* mpq_stream_t; /* cudaStream_t */
+
+typedef enum {
+  MPQ_OK = 0,
+  MPQ_ERR_INVALID_ARG = 1, /* bad size, NULL pointer, unsupported parameter */
+  MPQ_ERR_CUDA = 2,        /* a CUDA runtime call failed (message has it)   */
+  MPQ_ERR_OOM = 3,         /* device allocation failed / over the cap       */
+  MPQ_ERR_NONFINITE = 4,   /* NaN/Inf met in an input on the device         */
+  MPQ_ERR_RANK = 5,        /* setup found rank 0                            */
+  MPQ_ERR_TIMEOUT = 6,     /* a bounded device loop reached its cap         */
+  MPQ_ERR_UNSUPPORTED = 7
+} mpq_status;
+
+/* Solver parameters ([Hyper-parameters]).  Fill with mpq_params_default. */
+typedef struct {
+  int32_t d;              /* block size: 1 (scalar grid) or 8 (vector codebook) */
+  int32_t K;              /* d = 1: grid levels L, 2..256; d = 8: codebook size 1..65536 */
+  const float* codebook;  /* d = 8: HOST pointer, K x 8 row-major, copied at plan
+                             creation; d = 1: must be NULL (levels are 0..L-1,
+                             mapped per row by scale * k + offset) */
+  double beta0;           /* initial inverse temperature, default 1 */
+  double damping;         /* rho_damp: beta <- (1-rho) beta + rho beta_hat, default 0.5 */
+  double tau;             /* prior anchor scale; INFINITY (default) = uniform rho_b.
+                             Finite tau: rho_b(c) = exp(-(gamma1_0/tau^2)/2 |c - w_b|^2) */
+  double gamma_lo_rel;    /* extrinsic precisions are clipped into        */
+  double gamma_hi_rel;    /*   [lo, hi] * gamma1_0 (defaults 1e-10, 1e10) */
+  double alpha_min;       /* mean divergences are clipped into            */
+  double alpha_max;       /*   [alpha_min, alpha_max] (1e-10, 1 - 1e-5)   */
+} mpq_params;
+
+/* Fill `p` with the defaults above for block size d and codebook size K. */
+MPQ_API void mpq_params_default(mpq_params* p, int32_t d, int32_t K);
+
+/* ---------------------------------------------------------------- plans --- */
+
+/* Create a plan from a precomputed spectrum ([Flowchart]: T = diag(s) V^T).
+ *   s: r doubles, descending, > 0.   V: n x r doubles, orthonormal columns.
+ *   n must be a multiple of params->d; 1 <= r <= n.
+ * The plan copies s and V (fp32 + fp64 copies, both layouts), builds
+ * H = V diag(s^2) V^T and, for d = 8, the per-block tables 1/2 c^T H_bb c.
+ * Synchronises `stream` before returning. */
+MPQ_API mpq_status mpq_plan_create_from_spectrum(const double* s, const double* V, int64_t n, int64_t r,
+                                         const mpq_params* params, mpq_stream_t stream,
+                                         mpq_plan_t* plan);
+
+/* Create a plan from calibration activations X (m x n fp32, device):
+ * the compact SVD of X through the smaller Gram matrix (X^T X if n <= m,
+ * else X X^T), computed on the device in fp64 by cyclic Jacobi; rank cut at
+ * lambda > lambda_max * max(m, n) * 2^-52 ([Key design 1]: T in the rank
+ * space r = rank(X)).  Synchronises `stream`.  MPQ_ERR_RANK if X == 0. */
+MPQ_API mpq_status mpq_plan_create_from_x(const float* X, int64_t m, int64_t n, const mpq_params* params,
+                                  mpq_stream_t stream, mpq_plan_t* plan);
+
+/* Release every device buffer the plan owns.  NULL is a no-op. */
+MPQ_API mpq_status mpq_plan_destroy(mpq_plan_t plan);
+
+/* HOST outputs (any may be NULL): n, rank r, d, K. */
+MPQ_API mpq_status mpq_plan_info(mpq_plan_t plan, int64_t* n, int64_t* r, int32_t* d, int32_t* K);
+
+/* Copy the plan's spectrum out: s (r doubles) and V (n x r doubles), device. */
+MPQ_API mpq_status mpq_plan_get_spectrum(mpq_plan_t plan, double* s, double* V, mpq_stream_t stream);
+
+/* Synchronise `stream`, read and clear the plan's device status word.
+ * Returns MPQ_OK, MPQ_ERR_NONFINITE or MPQ_ERR_TIMEOUT. */
+MPQ_API mpq_status mpq_plan_status(mpq_plan_t plan, mpq_stream_t stream);
+
+/* Upper bound on the workspace (bytes) that a solve of m_out rows allocates
+ * inside the plan, and an optional cap: a solve that would need more than
+ * `cap_bytes` fails with MPQ_ERR_OOM before launching (0 = no cap). */
+MPQ_API int64_t mpq_plan_workspace_bytes(mpq_plan_t plan, int64_t m_out);
+MPQ_API mpq_status mpq_plan_set_workspace_cap(mpq_plan_t plan, int64_t cap_bytes);
+
+/* --------------------------------------------------------------- solve --- */
+
+/* Optional per-row outputs of a solve (device pointers, each may be NULL). */
+typedef struct {
+  double* gamma1;     /* m_out: terminal denoiser precision gamma1^T          */
+  double* beta;       /* m_out: terminal inverse temperature                  */
+  int32_t* clamps;    /* m_out: number of clips applied over the VAMP loop    */
+  int32_t* cd_changes;/* m_out x cd_sweeps: blocks changed in each CD sweep   */
+} mpq_row_stats;
+
+/* The whole MPQ solve of every row of W ([Flowchart]):
+ * init (per-row scale/offset, round-to-nearest, gamma1_0 = 1/MSE, r1 = w,
+ * beta = beta0) -> T_vamp iterations of {denoiser, extrinsic update, rank-
+ * space linear module, beta M-step} -> marginal-MAP argmax -> at most
+ * cd_sweeps sweeps of exact block CD (stop after a sweep without change)
+ * -> w_hat and energies E = 1/2 |T (w - w_hat)|^2.
+ *   W: m_out x n fp32.
+ *   row_scale/row_offset: m_out floats each, or both NULL for the built-in
+ *     choice (d = 1: per-row min-max grid; d = 8: scale = RMS(w), offset 0).
+ *   T_vamp >= 0, 0 <= cd_sweeps <= 64.
+ *   idx: m_out x B uint16 codeword indices (out).  w_hat: m_out x n fp32
+ *   (out, may be NULL).  energy: m_out fp32 (out, may be NULL).
+ *   stats: HOST struct of optional device outputs, may be NULL.
+ * Asynchronous; may allocate plan workspace on first use for a row count
+ * (which synchronises the device). */
+MPQ_API mpq_status mpq_solve(mpq_plan_t plan, const float* W, int64_t m_out, const float* row_scale,
+                     const float* row_offset, int32_t T_vamp, int32_t cd_sweeps, uint16_t* idx,
+                     float* w_hat, float* energy, const mpq_row_stats* stats,
+                     mpq_stream_t stream);
+
+/* Same as mpq_solve with HOST buffers for W, idx, w_hat and energy (pinned
+ * memory gives the fastest copies).  Copies W to plan-owned device memory,
+ * solves, copies the results back, synchronises `stream` and returns the
+ * device status (as mpq_plan_status). */
+MPQ_API mpq_status mpq_solve_host(mpq_plan_t plan, const float* W_host, int64_t m_out, int32_t T_vamp,
+                          int32_t cd_sweeps, uint16_t* idx_host, float* w_hat_host,
+                          float* energy_host, mpq_stream_t stream);
+
+/* -------------------------------------------------- stage entry points --- */
+/* Each runs exactly the kernels that mpq_solve runs for one stage, on state
+ * the caller injects, so that every stage can be compared on identical
+ * inputs.  B = n/d.  Per-row scalars are fp64, vectors fp32. */
+
+/* Init ([Hyper-parameters]): if `given` == 0, compute scale/offset (built-in
+ * rule) into scale/offset; else read them.  idx_rtn: m x B nearest codeword
+ * (lowest index on ties); gamma1_0: m doubles, 1/max(MSE(w, w_rtn), 1e-30). */
+MPQ_API mpq_status mpq_stage_init(mpq_plan_t plan, const float* W, int64_t m, int32_t given, float* scale,
+                          float* offset, uint16_t* idx_rtn, double* gamma1_0, mpq_stream_t stream);
+
+/* Denoiser ([Key design 1]): for every block the posterior over the row's
+ * codewords scale*c + offset.  Inputs R1 (m x n), gamma1 (m), scale/offset
+ * (m); for a finite-tau plan also W (m x n) and gamma1_0 (m), else NULL.
+ * Outputs xhat1 (m x n posterior means), vblock (m x B traces of the
+ * posterior covariances, may be NULL), vsum (m, fp64 sums of vblock),
+ * idx (m x B argmax, lowest index on ties, may be NULL). */
+MPQ_API mpq_status mpq_stage_denoise(mpq_plan_t plan, const float* R1, const double* gamma1,
+                             const float* scale, const float* offset, int64_t m, const float* W,
+                             const double* gamma1_0, float* xhat1, float* vblock, double* vsum,
+                             uint16_t* idx, mpq_stream_t stream);
+
+/* Extrinsic update, linear module and M-step ([Key design 1], [Key design
+ * 2]).  Inputs W, R1, xhat1 (m x n), gamma1, vsum, gamma1_0 (m); beta (m)
+ * is read and overwritten with the damped update.  Outputs R1_out (m x n),
+ * gamma1_out (m).  Diagnostics (each may be NULL): R2 (m x n), gamma2 (m),
+ * Uprime (m x r, D*u), xhat2 (m x n), alpha2 (m, before clipping),
+ * beta_hat (m), clamps (m, added to). */
+MPQ_API mpq_status mpq_stage_linear(mpq_plan_t plan, const float* W, int64_t m, const float* R1,
+                            const double* gamma1, const float* xhat1, const double* vsum,
+                            const double* gamma1_0, double* beta, float* R1_out,
+                            double* gamma1_out, float* R2, double* gamma2, float* Uprime,
+                            float* xhat2, double* alpha2, double* beta_hat, int32_t* clamps,
+                            mpq_stream_t stream);
+
+/* Exact block CD ([Key design 3]) from the codewords in idx (m x B, read
+ * and overwritten): h = H (w - x), then at most `sweeps` sweeps over the
+ * blocks in order; each block takes the codeword of least energy (lowest
+ * index on ties) when that lowers the energy; a row stops after a sweep
+ * without change.  changes: m x sweeps ints (may be NULL). */
+MPQ_API mpq_status mpq_stage_cd(mpq_plan_t plan, const float* W, int64_t m, const float* scale,
+                        const float* offset, uint16_t* idx, int32_t sweeps, int32_t* changes,
+                        mpq_stream_t stream);
+
+/* Output ([Overall framework]): w_hat = scale * C[idx] + offset (m x n, may
+ * be NULL) and E = 1/2 |diag(s) V^T (w - w_hat)|^2 (m floats). */
+MPQ_API mpq_status mpq_stage_energy(mpq_plan_t plan, const float* W, int64_t m, const float* scale,
+                            const float* offset, const uint16_t* idx, float* w_hat, float* energy,
+                            mpq_stream_t stream);
+
+/* ----------------------------------------------------------- profiling --- */
+/* Per-kernel timing with CUDA events recorded on the launching stream around
+ * every kernel the library launches while profiling is on.  start clears
+ * earlier records; stop synchronises on the recorded events and writes one
+ * line per kernel name into the HOST buffer `buf` (NUL-terminated):
+ *   "<name> <launches> <total milliseconds>\n"
+ * Returns MPQ_ERR_INVALID_ARG if the text does not fit in `buflen`. */
+MPQ_API mpq_status mpq_profile_start(void);
+MPQ_API mpq_status mpq_profile_stop(char* buf, int64_t buflen);
+
+/* Thread-local text of the last error (never NULL). */
+MPQ_API const char* mpq_last_error(void);
+
+/* Number of kernels this library has launched in the calling process. */
+MPQ_API int64_t mpq_kernel_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MPQ_H_ */

@@ -1,0 +1,727 @@
+// Row kernels of the MPQ solve: init, blockwise denoisers, extrinsic
+// updates, the per-row epilogue of the rank-space linear module with the
+// beta M-step, residuals and energies.
+//
+// Source: "MPQ: A Message-Passing View of Post-Training Quantization"
+// (papernotes.org note), Key design 1 (denoiser, extrinsic updates, linear
+// module in rank space), Key design 2 (beta M-step), hyper-parameter
+// section (gamma1_0 = 1/MSE(w, w_rtn), rho_damp); the min-max grid follows
+// the NeUQI note, existing pain points section.
+#include <math.h>
+
+#include "mpq_internal.cuh"
+
+namespace mpq {
+namespace {
+
+constexpr int ROW_THREADS = 256;
+
+// ------------------------------------------------------------ reductions ---
+template <typename T, typename Op>
+__device__ __forceinline__ T warp_reduce(T v, Op op) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = op(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Deterministic block reduction (fixed tree), result broadcast to all threads.
+template <typename T, typename Op>
+__device__ T block_reduce(T v, Op op, T* smem /* >= 32 */) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int nw = (blockDim.x + 31) >> 5;
+  v = warp_reduce(v, op);
+  __syncthreads();
+  if (lane == 0) smem[wid] = v;
+  __syncthreads();
+  if (wid == 0) {
+    T x = lane < nw ? smem[lane] : smem[0];
+    if (lane >= nw) x = smem[0];
+    // lanes >= nw duplicate element 0; op must be idempotent for those
+    // (min/max) or we mask them explicitly for sums below
+    x = warp_reduce(x, op);
+    if (lane == 0) smem[32] = x;
+  }
+  __syncthreads();
+  return smem[32];
+}
+
+struct SumD {
+  __device__ double operator()(double a, double b) const { return a + b; }
+};
+struct MinF {
+  __device__ float operator()(float a, float b) const { return fminf(a, b); }
+};
+struct MaxF {
+  __device__ float operator()(float a, float b) const { return fmaxf(a, b); }
+};
+
+__device__ double block_sum(double v, double* smem) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int nw = (blockDim.x + 31) >> 5;
+  v = warp_reduce(v, SumD());
+  __syncthreads();
+  if (lane == 0) smem[wid] = v;
+  __syncthreads();
+  if (wid == 0) {
+    double x = lane < nw ? smem[lane] : 0.0;
+    x = warp_reduce(x, SumD());
+    if (lane == 0) smem[32] = x;
+  }
+  __syncthreads();
+  return smem[32];
+}
+
+__device__ __forceinline__ double clip_count(double v, double lo, double hi, int* cnt) {
+  double c = isnan(v) ? lo : fmin(fmax(v, lo), hi);
+  if (c != v) ++*cnt;
+  return c;
+}
+
+// ------------------------------------------------------------------ init ---
+// d = 1: per-row min-max grid (unless given), nearest level, gamma1_0.
+__global__ void __launch_bounds__(ROW_THREADS)
+    k_init_scalar(const float* __restrict__ W, int64_t n, int L, int given,
+                  float* __restrict__ scale, float* __restrict__ offset,
+                  uint16_t* __restrict__ idx, double* __restrict__ gamma1_0, int* status) {
+  __shared__ float fs[33];
+  __shared__ double ds[33];
+  const int64_t row = blockIdx.x;
+  const float* w = W + row * n;
+  if (!given) {
+    float lo = INFINITY, hi = -INFINITY;
+    bool bad = false;
+    for (int64_t j = threadIdx.x; j < n; j += blockDim.x) {
+      const float x = w[j];
+      bad |= !isfinite(x);
+      lo = fminf(lo, x);
+      hi = fmaxf(hi, x);
+    }
+    if (bad) atomicOr(status, STATUS_NONFINITE);
+    lo = block_reduce(lo, MinF(), fs);
+    hi = block_reduce(hi, MaxF(), fs);
+    if (threadIdx.x == 0) {
+      double s = ((double)hi - (double)lo) / (double)(L - 1);
+      if (!(hi > lo)) s = (hi != 0.0f) ? fabs((double)hi) : 1.0;
+      double z = rint(-(double)lo / s);
+      z = fmin(fmax(z, 0.0), (double)(L - 1));
+      scale[row] = (float)s;
+      offset[row] = (float)(-s * z);
+    }
+    __syncthreads();
+  }
+  const double sc = scale[row], off = offset[row];
+  double se = 0.0;
+  for (int64_t j = threadIdx.x; j < n; j += blockDim.x) {
+    const double x = w[j];
+    double t = (x - off) / sc;
+    double k0 = fmin(fmax(floor(t), 0.0), (double)(L - 1));
+    double k1 = fmin(k0 + 1.0, (double)(L - 1));
+    const double d0 = fabs(sc * k0 + off - x), d1 = fabs(sc * k1 + off - x);
+    const double k = (d1 < d0) ? k1 : k0;
+    idx[row * n + j] = (uint16_t)k;
+    const double e = x - (sc * k + off);
+    se += e * e;
+  }
+  se = block_sum(se, ds);
+  if (threadIdx.x == 0) gamma1_0[row] = 1.0 / fmax(se / (double)n, 1e-30);
+}
+
+// d = 8: per-row RMS scale (unless given), offset 0.
+__global__ void __launch_bounds__(ROW_THREADS)
+    k_init_rms(const float* __restrict__ W, int64_t n, int given, float* __restrict__ scale,
+               float* __restrict__ offset, int* status) {
+  __shared__ double ds[33];
+  const int64_t row = blockIdx.x;
+  const float* w = W + row * n;
+  double ss = 0.0;
+  bool bad = false;
+  for (int64_t j = threadIdx.x; j < n; j += blockDim.x) {
+    const double x = w[j];
+    bad |= !isfinite(w[j]);
+    ss += x * x;
+  }
+  if (bad) atomicOr(status, STATUS_NONFINITE);
+  ss = block_sum(ss, ds);
+  if (!given && threadIdx.x == 0) {
+    double rho = sqrt(ss / (double)n);
+    if (!(rho > 0.0)) rho = 1.0;
+    scale[row] = (float)rho;
+    offset[row] = 0.0f;
+  }
+}
+
+// d = 8: gamma1_0 from the nearest codewords already in idx.
+__global__ void __launch_bounds__(ROW_THREADS)
+    k_gamma0_vec(const float* __restrict__ W, int64_t n, const float* __restrict__ cb,
+                 const float* __restrict__ scale, const float* __restrict__ offset,
+                 const uint16_t* __restrict__ idx, double* __restrict__ gamma1_0) {
+  __shared__ double ds[33];
+  const int64_t row = blockIdx.x;
+  const double sc = scale[row], off = offset[row];
+  double se = 0.0;
+  for (int64_t j = threadIdx.x; j < n; j += blockDim.x) {
+    const int k = idx[row * (n / 8) + j / 8];
+    const double e = (double)W[row * n + j] - (sc * cb[k * 8 + (j & 7)] + off);
+    se += e * e;
+  }
+  se = block_sum(se, ds);
+  if (threadIdx.x == 0) gamma1_0[row] = 1.0 / fmax(se / (double)n, 1e-30);
+}
+
+// ------------------------------------------------------- scalar denoiser ---
+// Posterior over levels k = 0..L-1 (weights scale*k + offset) of
+// q(k) ~ exp(-gamma1/2 (scale k + offset - r)^2) [* anchor]; in level units
+// t = (r - offset)/scale, g = gamma1 scale^2, logit_k = -g/2 (k - t)^2.
+__global__ void __launch_bounds__(ROW_THREADS)
+    k_denoise_scalar(const float* __restrict__ R1, const double* __restrict__ gamma1,
+                     const float* __restrict__ scale, const float* __restrict__ offset,
+                     int64_t n, int L, const float* __restrict__ W,
+                     const double* __restrict__ gamma1_0, double inv_tau2,
+                     float* __restrict__ xhat, float* __restrict__ vblock,
+                     double* __restrict__ vsum, uint16_t* __restrict__ idx) {
+  __shared__ double ds[33];
+  const int64_t row = blockIdx.x;
+  const float sc = scale[row], off = offset[row];
+  const double dsc = sc, doff = off;
+  const double sc2 = dsc * dsc;
+  const double g = fmin(gamma1[row] * sc2, 1e30);
+  const bool anchored = (W != nullptr);
+  const double ga = anchored ? fmin(gamma1_0[row] * inv_tau2 * sc2, 1e30) : 0.0;
+  const double geff = g + ga;
+  const double Lm1 = (double)(L - 1);
+  double acc = 0.0;
+  for (int64_t j = threadIdx.x; j < n; j += blockDim.x) {
+    const int64_t o = row * n + j;
+    // level coordinate and logit arguments in fp64: the fp32 inputs are
+    // exact there, so only the exponentials and sums round in fp32
+    double t = ((double)R1[o] - doff) / dsc;
+    if (anchored) {
+      const double tw = ((double)W[o] - doff) / dsc;
+      t = (g * t + ga * tw) / geff;
+    }
+    // argmax of -(k - t)^2, lowest k on ties
+    const double ks = fmin(fmax(ceil(t - 0.5), 0.0), Lm1);
+    const double dt = t - ks;
+    float S0 = 0.0f, S1 = 0.0f, S2 = 0.0f;
+    for (int k = 0; k < L; ++k) {
+      const double dk = (double)k - ks;
+      const float e = __expf((float)(-0.5 * geff * dk * (dk - 2.0 * dt)));
+      const float dkf = (float)dk;
+      S0 += e;
+      S1 = fmaf(e, dkf, S1);
+      S2 = fmaf(e * dkf, dkf, S2);
+    }
+    const float m1 = S1 / S0;
+    const float var = fmaxf(S2 / S0 - m1 * m1, 0.0f);
+    xhat[o] = (float)(dsc * (ks + (double)m1) + doff);
+    const float v = (float)(sc2 * (double)var);
+    if (vblock) vblock[o] = v;
+    if (idx) idx[o] = (uint16_t)ks;
+    acc += (double)v;
+  }
+  acc = block_sum(acc, ds);
+  if (threadIdx.x == 0) vsum[row] = acc;
+}
+
+// ------------------------------------------------------- vector denoiser ---
+// One thread per block of 8 weights; the codebook streams through shared
+// memory in chunks that every thread of the CTA reads in lock step.
+constexpr int VEC_THREADS = 128;
+constexpr int VEC_CHUNK = 512;
+
+struct VecDenoiseArgs {
+  const float* R1;
+  const double* gamma1;
+  const float* scale;
+  const float* offset;
+  int64_t m, n;
+  int K;
+  const float* cb;       // K x 8
+  const float* cb_norm;  // K
+  const float* W;        // anchor (nullable)
+  const double* gamma1_0;
+  double inv_tau2;
+  float* xhat;
+  float* vblock;
+  uint16_t* idx;
+  int nearest_only;      // 1: only the argmax (nearest codeword) into idx
+};
+
+__global__ void __launch_bounds__(VEC_THREADS) k_denoise_vec(VecDenoiseArgs a) {
+  __shared__ float scb[VEC_CHUNK][9];
+  const int64_t B = a.n / 8;
+  const int64_t blk = (int64_t)blockIdx.x * VEC_THREADS + threadIdx.x;
+  const bool active = blk < a.m * B;
+  const int64_t row = active ? blk / B : 0;
+  float t[8];
+  double t64[8];
+  float g = 0.0f;
+  if (active) {
+    const double sc = a.scale[row];
+    const double sc2 = sc * sc;
+    const float* r = a.R1 + blk * 8;
+    double gg = 1.0, ga = 0.0;
+    if (!a.nearest_only) {
+      gg = a.gamma1[row] * sc2;
+      ga = a.W ? a.gamma1_0[row] * a.inv_tau2 * sc2 : 0.0;
+    }
+    g = (float)fmin(gg + ga, 1e30);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      double ti = (double)r[i] / sc;
+      if (a.W && !a.nearest_only) ti = (gg * ti + ga * ((double)a.W[blk * 8 + i] / sc)) / (gg + ga);
+      t64[i] = ti;
+      t[i] = (float)ti;
+    }
+  }
+  // pass 1: best score  s(c) = c.t - |c|^2/2  (logit = g s + const)
+  float best = -INFINITY;
+  int bidx = 0;
+  for (int c0 = 0; c0 < a.K; c0 += VEC_CHUNK) {
+    const int cn = min(VEC_CHUNK, a.K - c0);
+    __syncthreads();
+    for (int e = threadIdx.x; e < cn * 9; e += VEC_THREADS) {
+      const int c = e / 9, i = e % 9;
+      scb[c][i] = (i < 8) ? a.cb[(int64_t)(c0 + c) * 8 + i] : a.cb_norm[c0 + c];
+    }
+    __syncthreads();
+    if (active) {
+      for (int c = 0; c < cn; ++c) {
+        float s = -0.5f * scb[c][8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) s = fmaf(scb[c][i], t[i], s);
+        if (s > best) {
+          best = s;
+          bidx = c0 + c;
+        }
+      }
+    }
+  }
+  if (a.nearest_only) {
+    if (active) a.idx[blk] = (uint16_t)bidx;
+    return;
+  }
+  // pass 2: moments centred on the argmax codeword c*.  With dc = c - c*
+  // (exact for lattice codebooks) and tp = t - c*, the logit relative to
+  // the best is g (dc.tp - |dc|^2/2), which keeps fp32 cancellation small.
+  float cs[8], tp[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    cs[i] = active ? a.cb[(int64_t)bidx * 8 + i] : 0.0f;
+    tp[i] = (float)(t64[i] - (double)cs[i]);
+  }
+  float S0 = 0.0f, m2 = 0.0f, m1[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m1[i] = 0.0f;
+  for (int c0 = 0; c0 < a.K; c0 += VEC_CHUNK) {
+    const int cn = min(VEC_CHUNK, a.K - c0);
+    __syncthreads();
+    for (int e = threadIdx.x; e < cn * 9; e += VEC_THREADS) {
+      const int c = e / 9, i = e % 9;
+      scb[c][i] = (i < 8) ? a.cb[(int64_t)(c0 + c) * 8 + i] : a.cb_norm[c0 + c];
+    }
+    __syncthreads();
+    if (active) {
+      for (int c = 0; c < cn; ++c) {
+        float dc[8];
+        float dot = 0.0f, nn = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          dc[i] = scb[c][i] - cs[i];
+          dot = fmaf(dc[i], tp[i], dot);
+          nn = fmaf(dc[i], dc[i], nn);
+        }
+        const float q = __expf(g * (dot - 0.5f * nn));
+        S0 += q;
+        m2 = fmaf(q, nn, m2);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m1[i] = fmaf(q, dc[i], m1[i]);
+      }
+    }
+  }
+  if (!active) return;
+  const float sc = a.scale[row], off = a.offset[row];
+  const float inv = 1.0f / S0;
+  float mm = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float mi = m1[i] * inv;
+    mm = fmaf(mi, mi, mm);
+    a.xhat[blk * 8 + i] = fmaf(sc, cs[i] + mi, off);
+  }
+  const float var = fmaxf(m2 * inv - mm, 0.0f);
+  a.vblock[blk] = (float)((double)sc * sc * var);
+  if (a.idx) a.idx[blk] = (uint16_t)bidx;
+}
+
+// per-row sum of the block variances (deterministic)
+__global__ void __launch_bounds__(ROW_THREADS)
+    k_row_sum(const float* __restrict__ v, int64_t B, double* __restrict__ out) {
+  __shared__ double ds[33];
+  const int64_t row = blockIdx.x;
+  double acc = 0.0;
+  for (int64_t j = threadIdx.x; j < B; j += blockDim.x) acc += (double)v[row * B + j];
+  acc = block_sum(acc, ds);
+  if (threadIdx.x == 0) out[row] = acc;
+}
+
+// ------------------------------------------------- extrinsic d -> linear ---
+// alpha1 = gamma1 vsum / n (clipped), gamma2 = gamma1 (1 - alpha1)/alpha1
+// (clipped), r2 = r1 + (xhat1 - r1)/(1 - alpha1)  [= (xhat1 - alpha1 r1)/
+// (1 - alpha1) = (eta1 xhat1 - gamma1 r1)/gamma2], A = w - r2.
+__global__ void __launch_bounds__(ROW_THREADS)
+    k_extrinsic_d2l(const float* __restrict__ W, int64_t n, const float* __restrict__ R1,
+                    const double* __restrict__ gamma1, const float* __restrict__ X1,
+                    const double* __restrict__ vsum, const double* __restrict__ gamma1_0,
+                    double glo, double ghi, double amin, double amax, float* __restrict__ R2,
+                    float* __restrict__ A, double* __restrict__ gamma2,
+                    int32_t* __restrict__ clamps) {
+  __shared__ float cf;
+  const int64_t row = blockIdx.x;
+  if (threadIdx.x == 0) {
+    int cnt = 0;
+    const double g1 = gamma1[row];
+    const double a1 = clip_count(g1 * vsum[row] / (double)n, amin, amax, &cnt);
+    const double g0 = gamma1_0[row];
+    const double g2 = clip_count(g1 * (1.0 - a1) / a1, glo * g0, ghi * g0, &cnt);
+    gamma2[row] = g2;
+    cf = (float)(1.0 / (1.0 - a1));
+    if (clamps) clamps[row] += cnt;
+  }
+  __syncthreads();
+  const float c = cf;
+  for (int64_t j = threadIdx.x; j < n; j += blockDim.x) {
+    const int64_t o = row * n + j;
+    const float r1 = R1[o];
+    const float r2 = fmaf(c, X1[o] - r1, r1);
+    R2[o] = r2;
+    A[o] = W[o] - r2;
+  }
+}
+
+// -------------------------------------- linear module epilogue + M-step ---
+// P holds p' = V^T (w - r2) (m x r).  u = s p', F = gamma2/(beta s^2 +
+// gamma2), D u = (1 - F) p', alpha2 = [sum F + n - r]/n,
+// 1/beta_hat = (1/r) sum[F^2 u^2 + s^2/(beta s^2 + gamma2)],
+// beta <- (1-rho) beta + rho beta_hat, gamma1' = gamma2 (1-alpha2)/alpha2
+// (clipped), coef = 1/(1 - alpha2), kappa = alpha2/(1 - alpha2).
+// GEMM2 operand written back into P:
+//   r < n: (1 - F) p'            -> G = V (D u) = xhat2 - r2
+//   r = n: -F p'                 -> G = xhat2 - w  (V V^T = I), which avoids
+//          forming r2 + V V^T (w - r2) when r2 is far from w.
+__global__ void __launch_bounds__(ROW_THREADS)
+    k_linear_rows(float* __restrict__ P, int64_t n, int64_t r, const double* __restrict__ s,
+                  const double* __restrict__ gamma2, const double* __restrict__ gamma1_0,
+                  double* __restrict__ beta, double damping, double glo, double ghi,
+                  double amin, double amax, int full_rank, double* __restrict__ gamma1_out,
+                  double* __restrict__ coef, double* __restrict__ kappa,
+                  double* __restrict__ alpha2_out, double* __restrict__ beta_hat_out,
+                  int32_t* __restrict__ clamps, float* __restrict__ Uprime) {
+  __shared__ double ds[33];
+  const int64_t row = blockIdx.x;
+  const double b = beta[row], g2 = gamma2[row];
+  double a2s = 0.0, bs = 0.0;
+  for (int64_t l = threadIdx.x; l < r; l += blockDim.x) {
+    const double sl = s[l];
+    const double pl = (double)P[row * r + l];
+    const double u = sl * pl;
+    const double den = b * sl * sl + g2;
+    const double f = g2 / den;
+    a2s += f;
+    bs += f * f * u * u + sl * sl / den;
+    if (Uprime) Uprime[row * r + l] = (float)((1.0 - f) * pl);
+    P[row * r + l] = (float)(full_rank ? -f * pl : (1.0 - f) * pl);
+  }
+  a2s = block_sum(a2s, ds);
+  bs = block_sum(bs, ds);
+  if (threadIdx.x == 0) {
+    int cnt = 0;
+    const double alpha2 = (a2s + (double)(n - r)) / (double)n;
+    const double bhat = (double)r / bs;
+    beta[row] = (1.0 - damping) * b + damping * bhat;
+    const double a2 = clip_count(alpha2, amin, amax, &cnt);
+    const double g0 = gamma1_0[row];
+    gamma1_out[row] = clip_count(g2 * (1.0 - a2) / a2, glo * g0, ghi * g0, &cnt);
+    coef[row] = 1.0 / (1.0 - a2);
+    kappa[row] = a2 / (1.0 - a2);
+    if (alpha2_out) alpha2_out[row] = alpha2;
+    if (beta_hat_out) beta_hat_out[row] = bhat;
+    if (clamps) clamps[row] += cnt;
+  }
+}
+
+// ------------------------------------------------- extrinsic linear -> d ---
+// r1' = (xhat2 - alpha2 r2)/(1 - alpha2) = (eta2 xhat2 - gamma2 r2)/gamma1'.
+//   r < n: G = xhat2 - r2:  r1' = r2 + coef G,            xhat2 = r2 + G
+//   r = n: G = xhat2 - w:   r1' = w + kappa e + coef G,  xhat2 = w + G,
+//          with e = w - r2 (the GEMM1 operand).
+__global__ void __launch_bounds__(ROW_THREADS)
+    k_extrinsic_l2d(const float* __restrict__ W, const float* __restrict__ R2,
+                    const float* __restrict__ E, const float* __restrict__ G, int64_t n,
+                    const double* __restrict__ coef, const double* __restrict__ kappa,
+                    int full_rank, float* __restrict__ R1, float* __restrict__ xhat2) {
+  const int64_t row = blockIdx.x;
+  const float c = (float)coef[row];
+  const float k = (float)kappa[row];
+  for (int64_t j = threadIdx.x; j < n; j += blockDim.x) {
+    const int64_t o = row * n + j;
+    const float g = G[o];
+    if (full_rank) {
+      const float w = W[o];
+      R1[o] = fmaf(c, g, fmaf(k, E[o], w));
+      if (xhat2) xhat2[o] = w + g;
+    } else {
+      const float r2 = R2[o];
+      R1[o] = fmaf(c, g, r2);
+      if (xhat2) xhat2[o] = r2 + g;
+    }
+  }
+}
+
+// --------------------------------------------------- residual / energies ---
+__global__ void __launch_bounds__(ROW_THREADS)
+    k_residual(const float* __restrict__ W, int64_t n, int d, const float* __restrict__ cb,
+               const float* __restrict__ scale, const float* __restrict__ offset,
+               const uint16_t* __restrict__ idx, float* __restrict__ E,
+               float* __restrict__ w_hat) {
+  const int64_t row = blockIdx.x;
+  const float sc = scale[row], off = offset[row];
+  const int64_t B = n / d;
+  for (int64_t j = threadIdx.x; j < n; j += blockDim.x) {
+    const int k = idx[row * B + j / d];  // in range: sanitised on entry
+    const float c = (d == 1) ? (float)k : cb[(int64_t)k * d + (j % d)];
+    const float wh = fmaf(sc, c, off);
+    E[row * n + j] = W[row * n + j] - wh;
+    if (w_hat) w_hat[row * n + j] = wh;
+  }
+}
+
+__global__ void __launch_bounds__(ROW_THREADS)
+    k_energy_rows(const float* __restrict__ P, int64_t r, const double* __restrict__ s,
+                  float* __restrict__ energy) {
+  __shared__ double ds[33];
+  const int64_t row = blockIdx.x;
+  double acc = 0.0;
+  for (int64_t l = threadIdx.x; l < r; l += blockDim.x) {
+    const double u = s[l] * (double)P[row * r + l];
+    acc += u * u;
+  }
+  acc = block_sum(acc, ds);
+  if (threadIdx.x == 0) energy[row] = (float)(0.5 * acc);
+}
+
+__global__ void k_sanitize_idx(uint16_t* __restrict__ idx, int64_t count, int K, int* status) {
+  bool bad = false;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < count;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    if (idx[i] >= K) {
+      idx[i] = (uint16_t)(K - 1);
+      bad = true;
+    }
+  }
+  if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) atomicOr(status, STATUS_BADINDEX);
+}
+
+__global__ void k_check_finite(const float* __restrict__ x, int64_t count, int* status) {
+  bool bad = false;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < count;
+       i += (int64_t)gridDim.x * blockDim.x)
+    bad |= !isfinite(x[i]);
+  if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) atomicOr(status, STATUS_NONFINITE);
+}
+
+inline unsigned rows_grid(int64_t m) { return (unsigned)m; }
+
+}  // namespace
+
+// =============================================================== launchers ==
+
+mpq_status launch_init(const mpq_plan_s* p, const float* W, int64_t m, int given, float* scale,
+                       float* offset, uint16_t* idx, double* gamma1_0, cudaStream_t st) {
+  if (m <= 0) return MPQ_OK;
+  if (p->d == 1) {
+    {
+      ProfScope ps_("k_init_scalar", st);
+      k_init_scalar<<<rows_grid(m), ROW_THREADS, 0, st>>>(W, p->n, p->K, given, scale, offset, idx,
+                                                          gamma1_0, p->status);
+    }
+    count_launch();
+    return check_launch("k_init_scalar");
+  }
+  {
+    ProfScope ps_("k_init_rms", st);
+    k_init_rms<<<rows_grid(m), ROW_THREADS, 0, st>>>(W, p->n, given, scale, offset, p->status);
+  }
+  count_launch();
+  MPQ_TRY(check_launch("k_init_rms"));
+  VecDenoiseArgs a{};
+  a.R1 = W;
+  a.scale = scale;
+  a.offset = offset;
+  a.m = m;
+  a.n = p->n;
+  a.K = p->K;
+  a.cb = p->cb;
+  a.cb_norm = p->cb_norm;
+  a.idx = idx;
+  a.nearest_only = 1;
+  const int64_t nb = m * (p->n / 8);
+  {
+    ProfScope ps_("k_denoise_vec", st);
+    k_denoise_vec<<<(unsigned)cdiv(nb, VEC_THREADS), VEC_THREADS, 0, st>>>(a);
+  }
+  count_launch();
+  MPQ_TRY(check_launch("k_denoise_vec(nearest)"));
+  {
+    ProfScope ps_("k_gamma0_vec", st);
+    k_gamma0_vec<<<rows_grid(m), ROW_THREADS, 0, st>>>(W, p->n, p->cb, scale, offset, idx, gamma1_0);
+  }
+  count_launch();
+  return check_launch("k_gamma0_vec");
+}
+
+mpq_status launch_denoise(const mpq_plan_s* p, const float* R1, const double* gamma1,
+                          const float* scale, const float* offset, int64_t m, const float* W,
+                          const double* gamma1_0, float* xhat1, float* vblock, double* vsum,
+                          uint16_t* idx, cudaStream_t st) {
+  if (m <= 0) return MPQ_OK;
+  const bool anchored = std::isfinite(p->params.tau);
+  const double inv_tau2 = anchored ? 1.0 / (p->params.tau * p->params.tau) : 0.0;
+  if (p->d == 1) {
+    {
+      ProfScope ps_("k_denoise_scalar", st);
+      k_denoise_scalar<<<rows_grid(m), ROW_THREADS, 0, st>>>(
+          R1, gamma1, scale, offset, p->n, p->K, anchored ? W : nullptr, gamma1_0, inv_tau2, xhat1,
+          vblock, vsum, idx);
+    }
+    count_launch();
+    return check_launch("k_denoise_scalar");
+  }
+  if (vblock == nullptr) return fail(MPQ_ERR_INVALID_ARG, "vector denoiser needs vblock");
+  VecDenoiseArgs a{};
+  a.R1 = R1;
+  a.gamma1 = gamma1;
+  a.scale = scale;
+  a.offset = offset;
+  a.m = m;
+  a.n = p->n;
+  a.K = p->K;
+  a.cb = p->cb;
+  a.cb_norm = p->cb_norm;
+  a.W = anchored ? W : nullptr;
+  a.gamma1_0 = gamma1_0;
+  a.inv_tau2 = inv_tau2;
+  a.xhat = xhat1;
+  a.vblock = vblock;
+  a.idx = idx;
+  a.nearest_only = 0;
+  const int64_t nb = m * (p->n / 8);
+  {
+    ProfScope ps_("k_denoise_vec", st);
+    k_denoise_vec<<<(unsigned)cdiv(nb, VEC_THREADS), VEC_THREADS, 0, st>>>(a);
+  }
+  count_launch();
+  MPQ_TRY(check_launch("k_denoise_vec"));
+  {
+    ProfScope ps_("k_row_sum", st);
+    k_row_sum<<<rows_grid(m), ROW_THREADS, 0, st>>>(vblock, p->n / 8, vsum);
+  }
+  count_launch();
+  return check_launch("k_row_sum");
+}
+
+mpq_status launch_extrinsic_d2l(const mpq_plan_s* p, const float* W, int64_t m, const float* R1,
+                                const double* gamma1, const float* xhat1, const double* vsum,
+                                const double* gamma1_0, float* R2, float* A, double* gamma2,
+                                int32_t* clamps, cudaStream_t st) {
+  if (m <= 0) return MPQ_OK;
+  const mpq_params& q = p->params;
+  {
+    ProfScope ps_("k_extrinsic_d2l", st);
+    k_extrinsic_d2l<<<rows_grid(m), ROW_THREADS, 0, st>>>(W, p->n, R1, gamma1, xhat1, vsum,
+                                                          gamma1_0, q.gamma_lo_rel, q.gamma_hi_rel,
+                                                          q.alpha_min, q.alpha_max, R2, A, gamma2,
+                                                          clamps);
+  }
+  count_launch();
+  return check_launch("k_extrinsic_d2l");
+}
+
+mpq_status launch_linear_rows(const mpq_plan_s* p, int64_t m, float* P, const double* gamma2,
+                              const double* gamma1_0, double* beta, double* gamma1_out,
+                              double* coef, double* kappa, double* alpha2, double* beta_hat,
+                              int32_t* clamps, float* Uprime, cudaStream_t st) {
+  if (m <= 0) return MPQ_OK;
+  const mpq_params& q = p->params;
+  {
+    ProfScope ps_("k_linear_rows", st);
+    k_linear_rows<<<rows_grid(m), ROW_THREADS, 0, st>>>(
+        P, p->n, p->r, p->s64, gamma2, gamma1_0, beta, q.damping, q.gamma_lo_rel, q.gamma_hi_rel,
+        q.alpha_min, q.alpha_max, p->r == p->n ? 1 : 0, gamma1_out, coef, kappa, alpha2, beta_hat,
+        clamps, Uprime);
+  }
+  count_launch();
+  return check_launch("k_linear_rows");
+}
+
+mpq_status launch_extrinsic_l2d(const mpq_plan_s* p, const float* W, int64_t m, const float* R2,
+                                const float* E, const float* G, const double* coef,
+                                const double* kappa, float* R1_out, float* xhat2,
+                                cudaStream_t st) {
+  if (m <= 0) return MPQ_OK;
+  {
+    ProfScope ps_("k_extrinsic_l2d", st);
+    k_extrinsic_l2d<<<rows_grid(m), ROW_THREADS, 0, st>>>(W, R2, E, G, p->n, coef, kappa,
+                                                          p->r == p->n ? 1 : 0, R1_out, xhat2);
+  }
+  count_launch();
+  return check_launch("k_extrinsic_l2d");
+}
+
+mpq_status launch_residual(const mpq_plan_s* p, const float* W, int64_t m, const float* scale,
+                           const float* offset, const uint16_t* idx, float* E, float* w_hat,
+                           cudaStream_t st) {
+  if (m <= 0) return MPQ_OK;
+  {
+    ProfScope ps_("k_residual", st);
+    k_residual<<<rows_grid(m), ROW_THREADS, 0, st>>>(W, p->n, p->d, p->cb, scale, offset, idx, E,
+                                                     w_hat);
+  }
+  count_launch();
+  return check_launch("k_residual");
+}
+
+mpq_status launch_energy_rows(const mpq_plan_s* p, int64_t m, const float* P, float* energy,
+                              cudaStream_t st) {
+  if (m <= 0) return MPQ_OK;
+  {
+    ProfScope ps_("k_energy_rows", st);
+    k_energy_rows<<<rows_grid(m), ROW_THREADS, 0, st>>>(P, p->r, p->s64, energy);
+  }
+  count_launch();
+  return check_launch("k_energy_rows");
+}
+
+mpq_status launch_sanitize_idx(const mpq_plan_s* p, uint16_t* idx, int64_t count, cudaStream_t st) {
+  if (count <= 0) return MPQ_OK;
+  const unsigned blocks = (unsigned)std::min<int64_t>(cdiv(count, 256), 148 * 8);
+  {
+    ProfScope ps_("k_sanitize_idx", st);
+    k_sanitize_idx<<<blocks, 256, 0, st>>>(idx, count, p->K, p->status);
+  }
+  count_launch();
+  return check_launch("k_sanitize_idx");
+}
+
+mpq_status launch_check_finite(const float* x, int64_t count, int* status, cudaStream_t st) {
+  if (count <= 0) return MPQ_OK;
+  const unsigned blocks = (unsigned)std::min<int64_t>(cdiv(count, 256), 148 * 8);
+  {
+    ProfScope ps_("k_check_finite", st);
+    k_check_finite<<<blocks, 256, 0, st>>>(x, count, status);
+  }
+  count_launch();
+  return check_launch("k_check_finite");
+}
+
+}  // namespace mpq

@@ -1,0 +1,672 @@
+// C ABI of libmpq: plans, workspace, the solve pipeline and the stage entry
+// points.  The order of the pipeline follows the flowchart of "MPQ: A
+// Message-Passing View of Post-Training Quantization" (papernotes.org note):
+// init -> T_vamp x (denoiser, extrinsic update, rank-space linear module,
+// beta M-step) -> marginal-MAP argmax -> exact block CD -> energies.
+#include <math.h>
+#include <string.h>
+
+#include <algorithm>
+#include <atomic>
+#include <map>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "mpq_internal.cuh"
+
+namespace mpq {
+
+static thread_local std::string g_last_error = "no error";
+static std::atomic<int64_t> g_launches{0};
+
+void set_error(const std::string& msg) { g_last_error = msg; }
+
+mpq_status fail(mpq_status st, const std::string& msg) {
+  set_error(msg);
+  return st;
+}
+
+mpq_status cuda_fail(cudaError_t e, const char* what) {
+  set_error(std::string(what) + ": " + cudaGetErrorString(e));
+  return e == cudaErrorMemoryAllocation ? MPQ_ERR_OOM : MPQ_ERR_CUDA;
+}
+
+void count_launch(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+mpq_status check_launch(const char* name) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, name);
+  return MPQ_OK;
+}
+
+// ------------------------------------------------------------- profiling --
+namespace {
+struct ProfRec {
+  const char* name;
+  cudaEvent_t a, b;
+};
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+std::vector<ProfRec> g_prof;
+std::vector<cudaEvent_t> g_event_pool;
+
+cudaEvent_t pool_event() {
+  if (!g_event_pool.empty()) {
+    cudaEvent_t e = g_event_pool.back();
+    g_event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  return e;
+}
+}  // namespace
+
+ProfScope::ProfScope(const char* name, cudaStream_t stream) : st(stream) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  if (!g_prof_on) return;
+  ProfRec r{name, pool_event(), pool_event()};
+  if (!r.a || !r.b) return;
+  cudaEventRecord(r.a, st);
+  slot = (int)g_prof.size();
+  g_prof.push_back(r);
+}
+
+ProfScope::~ProfScope() {
+  if (slot < 0) return;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  if (slot < (int)g_prof.size()) cudaEventRecord(g_prof[slot].b, st);
+}
+
+namespace {
+
+struct DeviceGuard {
+  int prev = -1;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) == cudaSuccess && prev != dev) cudaSetDevice(dev);
+  }
+  ~DeviceGuard() {
+    int cur = -1;
+    if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+  }
+};
+
+__global__ void k_fill_f64(double* x, int64_t count, double v) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < count;
+       i += (int64_t)gridDim.x * blockDim.x)
+    x[i] = v;
+}
+
+mpq_status fill_f64(double* x, int64_t count, double v, cudaStream_t st) {
+  if (count <= 0) return MPQ_OK;
+  {
+    ProfScope ps_("k_fill_f64", st);
+    k_fill_f64<<<(unsigned)std::min<int64_t>(cdiv(count, 256), 1024), 256, 0, st>>>(x, count, v);
+  }
+  count_launch();
+  return check_launch("k_fill_f64");
+}
+
+mpq_status validate_params(const mpq_params* q, int64_t n) {
+  if (!q) return fail(MPQ_ERR_INVALID_ARG, "params is NULL");
+  if (q->d == 1) {
+    if (q->K < 2 || q->K > 256) return fail(MPQ_ERR_INVALID_ARG, "d=1 needs 2 <= K <= 256");
+    if (q->codebook) return fail(MPQ_ERR_INVALID_ARG, "d=1 takes no codebook (levels 0..K-1)");
+  } else if (q->d == 8) {
+    if (q->K < 1 || q->K > 65536) return fail(MPQ_ERR_INVALID_ARG, "d=8 needs 1 <= K <= 65536");
+    if (!q->codebook) return fail(MPQ_ERR_INVALID_ARG, "d=8 needs a codebook");
+  } else {
+    return fail(MPQ_ERR_INVALID_ARG, "d must be 1 or 8");
+  }
+  if (n <= 0 || n % q->d != 0) return fail(MPQ_ERR_INVALID_ARG, "n must be a positive multiple of d");
+  if (!(q->beta0 > 0.0) || !isfinite(q->beta0)) return fail(MPQ_ERR_INVALID_ARG, "beta0 must be > 0");
+  if (!(q->damping >= 0.0 && q->damping <= 1.0)) return fail(MPQ_ERR_INVALID_ARG, "damping must be in [0,1]");
+  if (!(q->tau > 0.0)) return fail(MPQ_ERR_INVALID_ARG, "tau must be > 0 (INFINITY = uniform prior)");
+  if (!(q->gamma_lo_rel > 0.0 && q->gamma_lo_rel < q->gamma_hi_rel && isfinite(q->gamma_hi_rel)))
+    return fail(MPQ_ERR_INVALID_ARG, "need 0 < gamma_lo_rel < gamma_hi_rel < inf");
+  if (!(q->alpha_min > 0.0 && q->alpha_min < q->alpha_max && q->alpha_max < 1.0))
+    return fail(MPQ_ERR_INVALID_ARG, "need 0 < alpha_min < alpha_max < 1");
+  return MPQ_OK;
+}
+
+template <typename T>
+mpq_status dalloc(T** p, int64_t count) {
+  *p = nullptr;
+  if (count <= 0) return MPQ_OK;
+  cudaError_t e = cudaMalloc((void**)p, sizeof(T) * (size_t)count);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    *p = nullptr;
+    return fail(MPQ_ERR_OOM, std::string("cudaMalloc of ") + std::to_string(sizeof(T) * count) +
+                                 " bytes failed: " + cudaGetErrorString(e));
+  }
+  return MPQ_OK;
+}
+
+template <typename T>
+void dfree(T*& p) {
+  if (p) cudaFree(p);
+  p = nullptr;
+}
+
+void free_workspace(Workspace& w) {
+  dfree(w.R1); dfree(w.X1); dfree(w.R2); dfree(w.A); dfree(w.P); dfree(w.idx);
+  dfree(w.scale); dfree(w.offset); dfree(w.gamma1); dfree(w.gamma1_0); dfree(w.gamma2);
+  dfree(w.beta); dfree(w.vsum); dfree(w.coef); dfree(w.kappa); dfree(w.clamps); dfree(w.W); dfree(w.w_hat);
+  dfree(w.energy); dfree(w.idx_stage);
+  w.rows = 0;
+  w.bytes = 0;
+}
+
+constexpr int MAX_SWEEPS = 64;
+
+int64_t ws_bytes_per_row(const mpq_plan_s* p) {
+  return 4 * p->n * 4 + p->r * 4 + p->B * 2 + 2 * 4 + 8 * 8 + 4 + MAX_SWEEPS * 4;
+}
+
+// changes buffer rides in the tail of `clamps`: rows x (1 + MAX_SWEEPS) ints
+mpq_status ensure_workspace(mpq_plan_s* p, int64_t rows) {
+  if (rows <= p->ws.rows) return MPQ_OK;
+  const int64_t need = rows * ws_bytes_per_row(p);
+  if (p->ws_cap > 0 && need > p->ws_cap)
+    return fail(MPQ_ERR_OOM, "workspace of " + std::to_string(need) + " bytes exceeds the cap");
+  MPQ_CUDA(cudaDeviceSynchronize());
+  free_workspace(p->ws);
+  Workspace& w = p->ws;
+  const int64_t mn = rows * p->n;
+  mpq_status st = MPQ_OK;
+  auto chk = [&](mpq_status s) { if (st == MPQ_OK) st = s; };
+  chk(dalloc(&w.R1, mn)); chk(dalloc(&w.X1, mn)); chk(dalloc(&w.R2, mn)); chk(dalloc(&w.A, mn));
+  chk(dalloc(&w.P, rows * p->r)); chk(dalloc(&w.idx, rows * p->B));
+  chk(dalloc(&w.scale, rows)); chk(dalloc(&w.offset, rows));
+  chk(dalloc(&w.gamma1, rows)); chk(dalloc(&w.gamma1_0, rows)); chk(dalloc(&w.gamma2, rows));
+  chk(dalloc(&w.beta, rows)); chk(dalloc(&w.vsum, rows)); chk(dalloc(&w.coef, rows));
+  chk(dalloc(&w.kappa, rows));
+  chk(dalloc(&w.clamps, rows * (1 + MAX_SWEEPS)));
+  if (st != MPQ_OK) {
+    free_workspace(w);
+    return st;
+  }
+  w.rows = rows;
+  w.bytes = need;
+  return MPQ_OK;
+}
+
+mpq_status ensure_host_staging(mpq_plan_s* p, int64_t rows) {
+  Workspace& w = p->ws;
+  // staging buffers follow the workspace row count
+  if (w.W) return MPQ_OK;
+  mpq_status st = MPQ_OK;
+  auto chk = [&](mpq_status s) { if (st == MPQ_OK) st = s; };
+  chk(dalloc(&w.W, rows * p->n));
+  chk(dalloc(&w.w_hat, rows * p->n));
+  chk(dalloc(&w.energy, rows));
+  chk(dalloc(&w.idx_stage, rows * p->B));
+  return st;
+}
+
+// --------------------------------------------------------- pipeline ------
+
+struct SolveIO {
+  const float* W;
+  int64_t m;
+  const float* row_scale;
+  const float* row_offset;
+  int T_vamp;
+  int sweeps;
+  uint16_t* idx;
+  float* w_hat;
+  float* energy;
+  const mpq_row_stats* stats;
+};
+
+// linear half-iteration on workspace state (R1 may alias W on the first call)
+mpq_status run_linear(mpq_plan_s* p, const float* W, int64_t m, const float* R1,
+                      const double* gamma1, const float* X1, const double* vsum,
+                      const double* gamma1_0, double* beta, float* R1_out, double* gamma1_out,
+                      float* R2, double* gamma2, float* Uprime, float* xhat2, double* alpha2,
+                      double* beta_hat, int32_t* clamps, cudaStream_t st) {
+  Workspace& w = p->ws;
+  const int64_t n = p->n, r = p->r;
+  MPQ_TRY(launch_extrinsic_d2l(p, W, m, R1, gamma1, X1, vsum, gamma1_0, R2, w.A, gamma2, clamps, st));
+  MPQ_TRY(gemm_nt_f32(w.A, n, p->Vt32, n, w.P, r, m, r, n, st, "gemm_project"));
+  MPQ_TRY(launch_linear_rows(p, m, w.P, gamma2, gamma1_0, beta, gamma1_out, w.coef, w.kappa,
+                             alpha2, beta_hat, clamps, Uprime, st));
+  // G into X1: the denoiser output is consumed by now, A (= w - r2) is still needed
+  MPQ_TRY(gemm_nt_f32(w.P, r, p->V32, r, w.X1, n, m, n, r, st, "gemm_expand"));
+  return launch_extrinsic_l2d(p, W, m, R2, w.A, w.X1, w.coef, w.kappa, R1_out, xhat2, st);
+}
+
+mpq_status run_cd(mpq_plan_s* p, const float* W, int64_t m, const float* scale,
+                  const float* offset, uint16_t* idx, int sweeps, int32_t* changes,
+                  cudaStream_t st) {
+  Workspace& w = p->ws;
+  const int64_t n = p->n;
+  MPQ_TRY(launch_residual(p, W, m, scale, offset, idx, w.A, nullptr, st));
+  MPQ_TRY(gemm_nt_f32(w.A, n, p->H32, n, w.X1, n, m, n, n, st, "gemm_hessian"));  // h = H (w - x)
+  return launch_cd(p, W, m, scale, offset, idx, w.X1, sweeps, changes, st);
+}
+
+mpq_status run_energy(mpq_plan_s* p, const float* W, int64_t m, const float* scale,
+                      const float* offset, const uint16_t* idx, float* w_hat, float* energy,
+                      cudaStream_t st) {
+  Workspace& w = p->ws;
+  const int64_t n = p->n, r = p->r;
+  MPQ_TRY(launch_residual(p, W, m, scale, offset, idx, w.A, w_hat, st));
+  if (!energy) return MPQ_OK;
+  MPQ_TRY(gemm_nt_f32(w.A, n, p->Vt32, n, w.P, r, m, r, n, st, "gemm_energy"));
+  return launch_energy_rows(p, m, w.P, energy, st);
+}
+
+// one batch of rows, all device pointers
+mpq_status solve_batch(mpq_plan_s* p, const SolveIO& io, int64_t row0, int64_t mb,
+                       cudaStream_t st) {
+  Workspace& w = p->ws;
+  const int64_t n = p->n, B = p->B;
+  const float* W = io.W + row0 * n;
+  uint16_t* idx = io.idx + row0 * B;
+  const int given = io.row_scale != nullptr;
+  if (given) {
+    MPQ_CUDA(cudaMemcpyAsync(w.scale, io.row_scale + row0, sizeof(float) * mb, cudaMemcpyDeviceToDevice, st));
+    MPQ_CUDA(cudaMemcpyAsync(w.offset, io.row_offset + row0, sizeof(float) * mb, cudaMemcpyDeviceToDevice, st));
+  }
+  int32_t* clamps = w.clamps;
+  int32_t* changes = w.clamps + w.rows;  // rows x MAX_SWEEPS
+  MPQ_CUDA(cudaMemsetAsync(clamps, 0, sizeof(int32_t) * mb, st));
+  // init: scale/offset, round-to-nearest (into idx), gamma1_0
+  MPQ_TRY(launch_init(p, W, mb, given, w.scale, w.offset, idx, w.gamma1_0, st));
+  MPQ_CUDA(cudaMemcpyAsync(w.gamma1, w.gamma1_0, sizeof(double) * mb, cudaMemcpyDeviceToDevice, st));
+  MPQ_TRY(fill_f64(w.beta, mb, p->params.beta0, st));
+  const float* R1 = W;  // cavity r1_0 = w
+  float* vblock = (p->d == 8) ? w.R2 : nullptr;  // R2 is free while the denoiser runs
+  for (int t = 0; t < io.T_vamp; ++t) {
+    MPQ_TRY(launch_denoise(p, R1, w.gamma1, w.scale, w.offset, mb, W, w.gamma1_0, w.X1, vblock,
+                           w.vsum, nullptr, st));
+    MPQ_TRY(run_linear(p, W, mb, R1, w.gamma1, w.X1, w.vsum, w.gamma1_0, w.beta, w.R1, w.gamma1,
+                       w.R2, w.gamma2, nullptr, nullptr, nullptr, nullptr, clamps, st));
+    R1 = w.R1;
+  }
+  // marginal MAP: argmax of one more denoiser call
+  if (io.T_vamp > 0)
+    MPQ_TRY(launch_denoise(p, R1, w.gamma1, w.scale, w.offset, mb, W, w.gamma1_0, w.X1, vblock,
+                           w.vsum, idx, st));
+  if (io.sweeps > 0) MPQ_TRY(run_cd(p, W, mb, w.scale, w.offset, idx, io.sweeps, changes, st));
+  MPQ_TRY(run_energy(p, W, mb, w.scale, w.offset, idx, io.w_hat ? io.w_hat + row0 * n : nullptr,
+                     io.energy ? io.energy + row0 : nullptr, st));
+  if (io.stats) {
+    const mpq_row_stats* s = io.stats;
+    if (s->gamma1) MPQ_CUDA(cudaMemcpyAsync(s->gamma1 + row0, w.gamma1, sizeof(double) * mb, cudaMemcpyDeviceToDevice, st));
+    if (s->beta) MPQ_CUDA(cudaMemcpyAsync(s->beta + row0, w.beta, sizeof(double) * mb, cudaMemcpyDeviceToDevice, st));
+    if (s->clamps) MPQ_CUDA(cudaMemcpyAsync(s->clamps + row0, clamps, sizeof(int32_t) * mb, cudaMemcpyDeviceToDevice, st));
+    if (s->cd_changes && io.sweeps > 0)
+      MPQ_CUDA(cudaMemcpyAsync(s->cd_changes + row0 * io.sweeps, changes, sizeof(int32_t) * mb * io.sweeps, cudaMemcpyDeviceToDevice, st));
+  }
+  return MPQ_OK;
+}
+
+mpq_status solve_device(mpq_plan_s* p, const SolveIO& io, cudaStream_t st) {
+  if (io.m <= 0) return MPQ_OK;
+  int64_t rows = io.m;
+  if (p->ws_cap > 0) {
+    const int64_t fit = p->ws_cap / ws_bytes_per_row(p);
+    if (fit < 1) return fail(MPQ_ERR_OOM, "workspace cap is below one row");
+    rows = std::min(rows, fit);
+  }
+  MPQ_TRY(ensure_workspace(p, rows));
+  for (int64_t r0 = 0; r0 < io.m; r0 += rows) {
+    MPQ_TRY(solve_batch(p, io, r0, std::min(rows, io.m - r0), st));
+  }
+  return MPQ_OK;
+}
+
+mpq_status finish_plan(mpq_plan_s* p, cudaStream_t st) {
+  const int64_t n = p->n, r = p->r;
+  MPQ_TRY(dalloc(&p->s32, r));
+  MPQ_TRY(dalloc(&p->V32, n * r));
+  MPQ_TRY(dalloc(&p->Vt32, r * n));
+  MPQ_TRY(dalloc(&p->H32, n * n));
+  MPQ_TRY(dalloc(&p->Hdiag, n));
+  MPQ_TRY(dalloc(&p->status, 1));
+  MPQ_CUDA(cudaMemsetAsync(p->status, 0, sizeof(int), st));
+  MPQ_TRY(build_hessian(p, st));
+  if (p->d == 8) {
+    MPQ_TRY(dalloc(&p->cb_norm, p->K));
+    MPQ_TRY(dalloc(&p->qtab, p->B * (int64_t)p->K));
+    MPQ_TRY(build_codebook_tables(p, st));
+  }
+  MPQ_CUDA(cudaStreamSynchronize(st));
+  return MPQ_OK;
+}
+
+void destroy_plan(mpq_plan_s* p) {
+  if (!p) return;
+  DeviceGuard g(p->device);
+  free_workspace(p->ws);
+  dfree(p->s64); dfree(p->V64); dfree(p->s32); dfree(p->V32); dfree(p->Vt32); dfree(p->H32);
+  dfree(p->Hdiag); dfree(p->cb); dfree(p->cb_norm); dfree(p->qtab); dfree(p->status);
+  delete p;
+}
+
+mpq_status new_plan(const mpq_params* params, int64_t n, mpq_plan_s** out) {
+  MPQ_TRY(validate_params(params, n));
+  mpq_plan_s* p = new mpq_plan_s();
+  MPQ_CUDA(cudaGetDevice(&p->device));
+  p->params = *params;
+  p->params.codebook = nullptr;
+  p->n = n;
+  p->d = params->d;
+  p->K = params->K;
+  p->B = n / params->d;
+  if (p->d == 8) {
+    mpq_status st = dalloc(&p->cb, (int64_t)p->K * 8);
+    if (st == MPQ_OK) {
+      cudaError_t e = cudaMemcpy(p->cb, params->codebook, sizeof(float) * p->K * 8, cudaMemcpyHostToDevice);
+      if (e != cudaSuccess) st = cuda_fail(e, "codebook copy");
+    }
+    if (st != MPQ_OK) {
+      destroy_plan(p);
+      return st;
+    }
+  }
+  *out = p;
+  return MPQ_OK;
+}
+
+#define PLAN_CHECK(p)                                                      \
+  do {                                                                     \
+    if (!(p)) return ::mpq::fail(MPQ_ERR_INVALID_ARG, "plan is NULL");     \
+  } while (0)
+
+}  // namespace
+}  // namespace mpq
+
+using namespace mpq;
+
+extern "C" {
+
+void mpq_params_default(mpq_params* p, int32_t d, int32_t K) {
+  if (!p) return;
+  memset(p, 0, sizeof(*p));
+  p->d = d;
+  p->K = K;
+  p->codebook = nullptr;
+  p->beta0 = 1.0;
+  p->damping = 0.5;
+  p->tau = INFINITY;
+  p->gamma_lo_rel = 1e-10;
+  p->gamma_hi_rel = 1e10;
+  p->alpha_min = 1e-10;
+  p->alpha_max = 1.0 - 1e-5;
+}
+
+mpq_status mpq_plan_create_from_spectrum(const double* s, const double* V, int64_t n, int64_t r,
+                                         const mpq_params* params, mpq_stream_t stream,
+                                         mpq_plan_t* plan) {
+  if (!plan) return fail(MPQ_ERR_INVALID_ARG, "plan out-pointer is NULL");
+  *plan = nullptr;
+  if (!s || !V) return fail(MPQ_ERR_INVALID_ARG, "s and V must be device pointers");
+  if (r < 1 || r > n) return fail(MPQ_ERR_INVALID_ARG, "need 1 <= r <= n");
+  cudaStream_t st = (cudaStream_t)stream;
+  mpq_plan_s* p = nullptr;
+  MPQ_TRY(new_plan(params, n, &p));
+  p->r = r;
+  mpq_status rc = dalloc(&p->s64, r);
+  if (rc == MPQ_OK) rc = dalloc(&p->V64, n * r);
+  if (rc == MPQ_OK) {
+    cudaError_t e = cudaMemcpyAsync(p->s64, s, sizeof(double) * r, cudaMemcpyDeviceToDevice, st);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(p->V64, V, sizeof(double) * n * r, cudaMemcpyDeviceToDevice, st);
+    if (e != cudaSuccess) rc = cuda_fail(e, "spectrum copy");
+  }
+  if (rc == MPQ_OK) {
+    std::vector<double> hs(r);
+    cudaError_t e = cudaMemcpyAsync(hs.data(), p->s64, sizeof(double) * r, cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) rc = cuda_fail(e, "spectrum read-back");
+    for (int64_t l = 0; rc == MPQ_OK && l < r; ++l)
+      if (!(hs[l] > 0.0) || !isfinite(hs[l]))
+        rc = fail(MPQ_ERR_INVALID_ARG, "singular values must be finite and > 0");
+  }
+  if (rc == MPQ_OK) rc = finish_plan(p, st);
+  if (rc != MPQ_OK) {
+    destroy_plan(p);
+    return rc;
+  }
+  *plan = p;
+  return MPQ_OK;
+}
+
+mpq_status mpq_plan_create_from_x(const float* X, int64_t m, int64_t n, const mpq_params* params,
+                                  mpq_stream_t stream, mpq_plan_t* plan) {
+  if (!plan) return fail(MPQ_ERR_INVALID_ARG, "plan out-pointer is NULL");
+  *plan = nullptr;
+  if (!X || m < 1 || n < 1) return fail(MPQ_ERR_INVALID_ARG, "X must be a device m x n matrix");
+  cudaStream_t st = (cudaStream_t)stream;
+  mpq_plan_s* p = nullptr;
+  MPQ_TRY(new_plan(params, n, &p));
+  mpq_status rc = setup_spectrum_from_x(p, X, m, n, st);
+  if (rc == MPQ_OK) rc = finish_plan(p, st);
+  if (rc != MPQ_OK) {
+    destroy_plan(p);
+    return rc;
+  }
+  *plan = p;
+  return MPQ_OK;
+}
+
+mpq_status mpq_plan_destroy(mpq_plan_t plan) {
+  destroy_plan(plan);
+  return MPQ_OK;
+}
+
+mpq_status mpq_plan_info(mpq_plan_t p, int64_t* n, int64_t* r, int32_t* d, int32_t* K) {
+  PLAN_CHECK(p);
+  if (n) *n = p->n;
+  if (r) *r = p->r;
+  if (d) *d = p->d;
+  if (K) *K = p->K;
+  return MPQ_OK;
+}
+
+mpq_status mpq_plan_get_spectrum(mpq_plan_t p, double* s, double* V, mpq_stream_t stream) {
+  PLAN_CHECK(p);
+  DeviceGuard g(p->device);
+  cudaStream_t st = (cudaStream_t)stream;
+  if (s) MPQ_CUDA(cudaMemcpyAsync(s, p->s64, sizeof(double) * p->r, cudaMemcpyDeviceToDevice, st));
+  if (V) MPQ_CUDA(cudaMemcpyAsync(V, p->V64, sizeof(double) * p->n * p->r, cudaMemcpyDeviceToDevice, st));
+  return MPQ_OK;
+}
+
+mpq_status mpq_plan_status(mpq_plan_t p, mpq_stream_t stream) {
+  PLAN_CHECK(p);
+  DeviceGuard g(p->device);
+  MPQ_CUDA(cudaStreamSynchronize((cudaStream_t)stream));
+  int word = 0;
+  MPQ_CUDA(cudaMemcpy(&word, p->status, sizeof(int), cudaMemcpyDeviceToHost));
+  MPQ_CUDA(cudaMemset(p->status, 0, sizeof(int)));
+  if (word & STATUS_NONFINITE) return fail(MPQ_ERR_NONFINITE, "non-finite value in an input row");
+  if (word & STATUS_TIMEOUT) return fail(MPQ_ERR_TIMEOUT, "a bounded device loop reached its cap");
+  if (word & STATUS_BADINDEX) return fail(MPQ_ERR_INVALID_ARG, "a codeword index was >= K (clamped)");
+  return MPQ_OK;
+}
+
+int64_t mpq_plan_workspace_bytes(mpq_plan_t p, int64_t m_out) {
+  if (!p || m_out < 0) return -1;
+  return m_out * ws_bytes_per_row(p);
+}
+
+mpq_status mpq_plan_set_workspace_cap(mpq_plan_t p, int64_t cap_bytes) {
+  PLAN_CHECK(p);
+  if (cap_bytes < 0) return fail(MPQ_ERR_INVALID_ARG, "cap must be >= 0");
+  p->ws_cap = cap_bytes;
+  return MPQ_OK;
+}
+
+mpq_status mpq_solve(mpq_plan_t p, const float* W, int64_t m_out, const float* row_scale,
+                     const float* row_offset, int32_t T_vamp, int32_t cd_sweeps, uint16_t* idx,
+                     float* w_hat, float* energy, const mpq_row_stats* stats,
+                     mpq_stream_t stream) {
+  PLAN_CHECK(p);
+  if (m_out < 0) return fail(MPQ_ERR_INVALID_ARG, "m_out must be >= 0");
+  if (m_out > 0 && (!W || !idx)) return fail(MPQ_ERR_INVALID_ARG, "W and idx are required");
+  if ((row_scale == nullptr) != (row_offset == nullptr))
+    return fail(MPQ_ERR_INVALID_ARG, "row_scale and row_offset go together");
+  if (T_vamp < 0) return fail(MPQ_ERR_INVALID_ARG, "T_vamp must be >= 0");
+  if (cd_sweeps < 0 || cd_sweeps > MAX_SWEEPS) return fail(MPQ_ERR_INVALID_ARG, "cd_sweeps must be in [0, 64]");
+  if (m_out > 2147483647LL) return fail(MPQ_ERR_INVALID_ARG, "m_out too large");
+  DeviceGuard g(p->device);
+  SolveIO io{W, m_out, row_scale, row_offset, T_vamp, cd_sweeps, idx, w_hat, energy, stats};
+  return solve_device(p, io, (cudaStream_t)stream);
+}
+
+mpq_status mpq_solve_host(mpq_plan_t p, const float* W_host, int64_t m_out, int32_t T_vamp,
+                          int32_t cd_sweeps, uint16_t* idx_host, float* w_hat_host,
+                          float* energy_host, mpq_stream_t stream) {
+  PLAN_CHECK(p);
+  if (m_out < 0) return fail(MPQ_ERR_INVALID_ARG, "m_out must be >= 0");
+  if (m_out == 0) return MPQ_OK;
+  if (!W_host || !idx_host) return fail(MPQ_ERR_INVALID_ARG, "W and idx are required");
+  if (T_vamp < 0 || cd_sweeps < 0 || cd_sweeps > MAX_SWEEPS)
+    return fail(MPQ_ERR_INVALID_ARG, "bad T_vamp / cd_sweeps");
+  if (p->ws_cap > 0) return fail(MPQ_ERR_UNSUPPORTED, "host solve does not batch under a cap");
+  DeviceGuard g(p->device);
+  cudaStream_t st = (cudaStream_t)stream;
+  if (p->ws.rows < m_out) MPQ_TRY(ensure_workspace(p, m_out));
+  MPQ_TRY(ensure_host_staging(p, p->ws.rows));
+  Workspace& w = p->ws;
+  const int64_t n = p->n, B = p->B;
+  MPQ_CUDA(cudaMemcpyAsync(w.W, W_host, sizeof(float) * m_out * n, cudaMemcpyHostToDevice, st));
+  SolveIO io{w.W, m_out, nullptr, nullptr, T_vamp, cd_sweeps, w.idx_stage,
+             w_hat_host ? w.w_hat : nullptr, energy_host ? w.energy : nullptr, nullptr};
+  MPQ_TRY(solve_device(p, io, st));
+  MPQ_CUDA(cudaMemcpyAsync(idx_host, w.idx_stage, sizeof(uint16_t) * m_out * B, cudaMemcpyDeviceToHost, st));
+  if (w_hat_host)
+    MPQ_CUDA(cudaMemcpyAsync(w_hat_host, w.w_hat, sizeof(float) * m_out * n, cudaMemcpyDeviceToHost, st));
+  if (energy_host)
+    MPQ_CUDA(cudaMemcpyAsync(energy_host, w.energy, sizeof(float) * m_out, cudaMemcpyDeviceToHost, st));
+  return mpq_plan_status(p, stream);
+}
+
+mpq_status mpq_stage_init(mpq_plan_t p, const float* W, int64_t m, int32_t given, float* scale,
+                          float* offset, uint16_t* idx_rtn, double* gamma1_0,
+                          mpq_stream_t stream) {
+  PLAN_CHECK(p);
+  if (m < 0 || (m > 0 && (!W || !scale || !offset || !idx_rtn || !gamma1_0)))
+    return fail(MPQ_ERR_INVALID_ARG, "init: missing buffer");
+  DeviceGuard g(p->device);
+  return launch_init(p, W, m, given ? 1 : 0, scale, offset, idx_rtn, gamma1_0, (cudaStream_t)stream);
+}
+
+mpq_status mpq_stage_denoise(mpq_plan_t p, const float* R1, const double* gamma1,
+                             const float* scale, const float* offset, int64_t m, const float* W,
+                             const double* gamma1_0, float* xhat1, float* vblock, double* vsum,
+                             uint16_t* idx, mpq_stream_t stream) {
+  PLAN_CHECK(p);
+  if (m < 0 || (m > 0 && (!R1 || !gamma1 || !scale || !offset || !xhat1 || !vsum)))
+    return fail(MPQ_ERR_INVALID_ARG, "denoise: missing buffer");
+  if (isfinite(p->params.tau) && m > 0 && (!W || !gamma1_0))
+    return fail(MPQ_ERR_INVALID_ARG, "denoise: an anchored plan needs W and gamma1_0");
+  DeviceGuard g(p->device);
+  cudaStream_t st = (cudaStream_t)stream;
+  if (p->d == 8 && vblock == nullptr) {
+    MPQ_TRY(ensure_workspace(p, m));
+    vblock = p->ws.R2;
+  }
+  return launch_denoise(p, R1, gamma1, scale, offset, m, W, gamma1_0, xhat1, vblock, vsum, idx, st);
+}
+
+mpq_status mpq_stage_linear(mpq_plan_t p, const float* W, int64_t m, const float* R1,
+                            const double* gamma1, const float* xhat1, const double* vsum,
+                            const double* gamma1_0, double* beta, float* R1_out,
+                            double* gamma1_out, float* R2, double* gamma2, float* Uprime,
+                            float* xhat2, double* alpha2, double* beta_hat, int32_t* clamps,
+                            mpq_stream_t stream) {
+  PLAN_CHECK(p);
+  if (m < 0 || (m > 0 && (!W || !R1 || !gamma1 || !xhat1 || !vsum || !gamma1_0 || !beta ||
+                          !R1_out || !gamma1_out)))
+    return fail(MPQ_ERR_INVALID_ARG, "linear: missing buffer");
+  if (m == 0) return MPQ_OK;
+  DeviceGuard g(p->device);
+  MPQ_TRY(ensure_workspace(p, m));
+  Workspace& w = p->ws;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (!R2) R2 = w.R2;
+  if (!gamma2) gamma2 = w.gamma2;
+  return run_linear(p, W, m, R1, gamma1, xhat1, vsum, gamma1_0, beta, R1_out, gamma1_out, R2,
+                    gamma2, Uprime, xhat2, alpha2, beta_hat, clamps, st);
+}
+
+mpq_status mpq_stage_cd(mpq_plan_t p, const float* W, int64_t m, const float* scale,
+                        const float* offset, uint16_t* idx, int32_t sweeps, int32_t* changes,
+                        mpq_stream_t stream) {
+  PLAN_CHECK(p);
+  if (m < 0 || (m > 0 && (!W || !scale || !offset || !idx)))
+    return fail(MPQ_ERR_INVALID_ARG, "cd: missing buffer");
+  if (sweeps < 0 || sweeps > MAX_SWEEPS) return fail(MPQ_ERR_INVALID_ARG, "sweeps must be in [0, 64]");
+  if (m == 0 || sweeps == 0) return MPQ_OK;
+  DeviceGuard g(p->device);
+  MPQ_TRY(ensure_workspace(p, m));
+  if (!changes) changes = p->ws.clamps + p->ws.rows;
+  MPQ_TRY(launch_sanitize_idx(p, idx, m * p->B, (cudaStream_t)stream));
+  return run_cd(p, W, m, scale, offset, idx, sweeps, changes, (cudaStream_t)stream);
+}
+
+mpq_status mpq_stage_energy(mpq_plan_t p, const float* W, int64_t m, const float* scale,
+                            const float* offset, const uint16_t* idx, float* w_hat, float* energy,
+                            mpq_stream_t stream) {
+  PLAN_CHECK(p);
+  if (m < 0 || (m > 0 && (!W || !scale || !offset || !idx || !energy)))
+    return fail(MPQ_ERR_INVALID_ARG, "energy: missing buffer");
+  if (m == 0) return MPQ_OK;
+  DeviceGuard g(p->device);
+  MPQ_TRY(ensure_workspace(p, m));
+  // the caller's indices are copied and sanitised before any codebook lookup
+  uint16_t* safe = p->ws.idx;
+  MPQ_CUDA(cudaMemcpyAsync(safe, idx, sizeof(uint16_t) * m * p->B, cudaMemcpyDeviceToDevice, (cudaStream_t)stream));
+  MPQ_TRY(launch_sanitize_idx(p, safe, m * p->B, (cudaStream_t)stream));
+  return run_energy(p, W, m, scale, offset, safe, w_hat, energy, (cudaStream_t)stream);
+}
+
+mpq_status mpq_profile_start(void) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  for (auto& r : g_prof) {
+    g_event_pool.push_back(r.a);
+    g_event_pool.push_back(r.b);
+  }
+  g_prof.clear();
+  g_prof_on = true;
+  return MPQ_OK;
+}
+
+mpq_status mpq_profile_stop(char* buf, int64_t buflen) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  g_prof_on = false;
+  std::map<std::string, std::pair<int64_t, double>> agg;
+  for (auto& r : g_prof) {
+    MPQ_CUDA(cudaEventSynchronize(r.b));
+    float ms = 0.0f;
+    MPQ_CUDA(cudaEventElapsedTime(&ms, r.a, r.b));
+    auto& e = agg[r.name];
+    e.first += 1;
+    e.second += ms;
+  }
+  std::string out;
+  for (auto& kv : agg) {
+    char line[256];
+    snprintf(line, sizeof(line), "%s %lld %.6f\n", kv.first.c_str(), (long long)kv.second.first,
+             kv.second.second);
+    out += line;
+  }
+  if (!buf || (int64_t)out.size() + 1 > buflen) return fail(MPQ_ERR_INVALID_ARG, "profile buffer too small");
+  memcpy(buf, out.c_str(), out.size() + 1);
+  return MPQ_OK;
+}
+
+const char* mpq_last_error(void) { return g_last_error.c_str(); }
+
+int64_t mpq_kernel_launch_count(void) { return g_launches.load(); }
+
+}  // extern "C"

@@ -1,0 +1,153 @@
+// Internal declarations shared by the libmpq translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+
+#include "../../include/mpq.h"
+
+namespace mpq {
+
+// ---------------------------------------------------------------- errors ---
+void set_error(const std::string& msg);
+mpq_status fail(mpq_status st, const std::string& msg);
+mpq_status cuda_fail(cudaError_t e, const char* what);
+
+#define MPQ_CUDA(call)                                              \
+  do {                                                              \
+    cudaError_t e_ = (call);                                        \
+    if (e_ != cudaSuccess) return ::mpq::cuda_fail(e_, #call);      \
+  } while (0)
+
+#define MPQ_TRY(call)                                               \
+  do {                                                              \
+    mpq_status s_ = (call);                                         \
+    if (s_ != MPQ_OK) return s_;                                    \
+  } while (0)
+
+// Event pair around one kernel launch when profiling is on (mpq_profile_*).
+struct ProfScope {
+  int slot = -1;
+  cudaStream_t st = nullptr;
+  ProfScope(const char* name, cudaStream_t stream);
+  ~ProfScope();
+};
+
+// Every kernel launch goes through this counter (see mpq_kernel_launch_count).
+void count_launch(int n = 1);
+mpq_status check_launch(const char* name);
+
+// Device status word bits (set by kernels, read by mpq_plan_status).
+enum : int { STATUS_NONFINITE = 1, STATUS_TIMEOUT = 2, STATUS_BADINDEX = 4 };
+
+// --------------------------------------------------------------- workspace --
+struct Workspace {
+  int64_t rows = 0;       // rows the buffers are sized for
+  int64_t bytes = 0;
+  // m x n fp32
+  float* R1 = nullptr;
+  float* X1 = nullptr;
+  float* R2 = nullptr;
+  float* A = nullptr;     // GEMM1 operand / GEMM2 output / CD gradient
+  // m x r fp32
+  float* P = nullptr;
+  // m x B
+  uint16_t* idx = nullptr;
+  // per-row
+  float* scale = nullptr;
+  float* offset = nullptr;
+  double* gamma1 = nullptr;
+  double* gamma1_0 = nullptr;
+  double* gamma2 = nullptr;
+  double* beta = nullptr;
+  double* vsum = nullptr;
+  double* coef = nullptr;   // 1/(1 - alpha2) of the last linear step
+  double* kappa = nullptr;  // alpha2/(1 - alpha2)
+  int32_t* clamps = nullptr;
+  // host-buffer solve staging (m x n W, outputs)
+  float* W = nullptr;
+  float* w_hat = nullptr;
+  float* energy = nullptr;
+  uint16_t* idx_stage = nullptr;
+};
+
+}  // namespace mpq
+
+struct mpq_plan_s {
+  int device = 0;
+  int64_t n = 0, r = 0;
+  int32_t d = 1, K = 2;
+  int64_t B = 0;
+  mpq_params params{};
+  // spectrum
+  double* s64 = nullptr;   // r
+  double* V64 = nullptr;   // n x r
+  float* s32 = nullptr;    // r
+  float* V32 = nullptr;    // n x r  (operand of x2 = r2 + V u')
+  float* Vt32 = nullptr;   // r x n  (operand of p = V^T (w - r2))
+  float* H32 = nullptr;    // n x n  H = V diag(s^2) V^T
+  float* Hdiag = nullptr;  // n
+  // vector codebook (d = 8)
+  float* cb = nullptr;       // K x 8
+  float* cb_norm = nullptr;  // K  |c|^2
+  float* qtab = nullptr;     // B x K  1/2 c^T H_bb c
+  // status
+  int* status = nullptr;     // device word
+  int64_t ws_cap = 0;
+  mpq::Workspace ws;
+};
+
+namespace mpq {
+
+// ------------------------------------------------------------- launchers ---
+// GEMM  C[M x N] = A[M x K] * B[N x K]^T  (row-major, K contiguous), fp32.
+// `tag` names the launch in the profiler (one name per GEMM role).
+mpq_status gemm_nt_f32(const float* A, int64_t lda, const float* B, int64_t ldb, float* C,
+                       int64_t ldc, int64_t M, int64_t N, int64_t K, cudaStream_t st,
+                       const char* tag = "gemm_f32");
+// Same with fp64 operands and accumulation (setup).
+mpq_status gemm_nt_f64(const double* A, int64_t lda, const double* B, int64_t ldb, double* C,
+                       int64_t ldc, int64_t M, int64_t N, int64_t K, cudaStream_t st);
+
+mpq_status launch_init(const mpq_plan_s* p, const float* W, int64_t m, int given, float* scale,
+                       float* offset, uint16_t* idx, double* gamma1_0, cudaStream_t st);
+mpq_status launch_denoise(const mpq_plan_s* p, const float* R1, const double* gamma1,
+                          const float* scale, const float* offset, int64_t m, const float* W,
+                          const double* gamma1_0, float* xhat1, float* vblock, double* vsum,
+                          uint16_t* idx, cudaStream_t st);
+mpq_status launch_extrinsic_d2l(const mpq_plan_s* p, const float* W, int64_t m, const float* R1,
+                                const double* gamma1, const float* xhat1, const double* vsum,
+                                const double* gamma1_0, float* R2, float* A, double* gamma2,
+                                int32_t* clamps, cudaStream_t st);
+mpq_status launch_linear_rows(const mpq_plan_s* p, int64_t m, float* P, const double* gamma2,
+                              const double* gamma1_0, double* beta, double* gamma1_out,
+                              double* coef, double* kappa, double* alpha2, double* beta_hat,
+                              int32_t* clamps, float* Uprime, cudaStream_t st);
+mpq_status launch_extrinsic_l2d(const mpq_plan_s* p, const float* W, int64_t m, const float* R2,
+                                const float* E, const float* G, const double* coef,
+                                const double* kappa, float* R1_out, float* xhat2,
+                                cudaStream_t st);
+mpq_status launch_residual(const mpq_plan_s* p, const float* W, int64_t m, const float* scale,
+                           const float* offset, const uint16_t* idx, float* E, float* w_hat,
+                           cudaStream_t st);
+// Clamp caller-supplied codeword indices into [0, K) in place, flagging any
+// that were out of range in the status word (STATUS_BADINDEX).
+mpq_status launch_sanitize_idx(const mpq_plan_s* p, uint16_t* idx, int64_t count, cudaStream_t st);
+mpq_status launch_energy_rows(const mpq_plan_s* p, int64_t m, const float* P, float* energy,
+                              cudaStream_t st);
+mpq_status launch_cd(const mpq_plan_s* p, const float* W, int64_t m, const float* scale,
+                     const float* offset, uint16_t* idx, float* h, int32_t sweeps,
+                     int32_t* changes, cudaStream_t st);
+mpq_status launch_check_finite(const float* x, int64_t count, int* status, cudaStream_t st);
+
+// plan-time builders
+mpq_status build_hessian(mpq_plan_s* p, cudaStream_t st);
+mpq_status build_codebook_tables(mpq_plan_s* p, cudaStream_t st);
+mpq_status setup_spectrum_from_x(mpq_plan_s* p, const float* X, int64_t m, int64_t n,
+                                 cudaStream_t st);
+
+inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+}  // namespace mpq

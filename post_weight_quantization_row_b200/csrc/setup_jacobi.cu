@@ -1,0 +1,365 @@
+// Setup: the compact SVD of the calibration activations X through the
+// smaller Gram matrix, on the device, in fp64.
+//
+// Source: "MPQ: A Message-Passing View of Post-Training Quantization"
+// (papernotes.org note), key design 1 and the flowchart: A = X = U Sigma V^T
+// (compact), T = Sigma V^T in the rank space r = rank(A).
+//
+// Eigensolver: the cyclic Jacobi method for symmetric matrices with the
+// parallel round-robin ("tournament") ordering of Brent and Luk; each 2x2
+// rotation is the symmetric Schur decomposition of Golub & Van Loan,
+// Matrix Computations, section 8.5 (Jacobi methods).  In round k the pairs
+// are (0, 1 + k) and (1 + (k+i) mod (N-1), 1 + (k-i) mod (N-1)); both index
+// runs are contiguous in i, so every round streams the matrix with coalesced
+// accesses.  Rank cut: lambda > lambda_max * max(m, n) * 2^-52.
+#include <math.h>
+
+#include <vector>
+
+#include "mpq_internal.cuh"
+
+namespace mpq {
+namespace {
+
+constexpr int JACOBI_MAX_SWEEPS = 40;
+
+__device__ __forceinline__ void rr_pair(int64_t N, int64_t k, int64_t i, int64_t* p, int64_t* q) {
+  if (i == 0) {
+    *p = 0;
+    *q = 1 + k;
+  } else {
+    const int64_t M = N - 1;
+    *p = 1 + (k + i) % M;
+    *q = 1 + ((k - i) % M + M) % M;
+  }
+}
+
+__global__ void k_jacobi_rot(const double* __restrict__ A, int64_t N, int64_t k,
+                             double* __restrict__ cs) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= N / 2) return;
+  int64_t p, q;
+  rr_pair(N, k, i, &p, &q);
+  const double app = A[p * N + p], aqq = A[q * N + q], apq = A[p * N + q];
+  double c = 1.0, s = 0.0;
+  if (apq != 0.0 && fabs(apq) > 1e-300) {
+    const double tau = (aqq - app) / (2.0 * apq);
+    const double t = (tau >= 0.0) ? 1.0 / (tau + sqrt(1.0 + tau * tau))
+                                   : -1.0 / (-tau + sqrt(1.0 + tau * tau));
+    c = 1.0 / sqrt(1.0 + t * t);
+    s = t * c;
+  }
+  cs[2 * i] = c;
+  cs[2 * i + 1] = s;
+}
+
+// A <- J^T A J on all 2x2 blocks (pair I rows, pair J cols)
+__global__ void k_jacobi_apply(double* __restrict__ A, int64_t N, int64_t k,
+                               const double* __restrict__ cs) {
+  const int64_t half = N / 2;
+  const int64_t J = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t I = blockIdx.y;
+  if (J >= half) return;
+  int64_t pI, qI, pJ, qJ;
+  rr_pair(N, k, I, &pI, &qI);
+  rr_pair(N, k, J, &pJ, &qJ);
+  const double cI = cs[2 * I], sI = cs[2 * I + 1];
+  const double cJ = cs[2 * J], sJ = cs[2 * J + 1];
+  const double m00 = A[pI * N + pJ], m01 = A[pI * N + qJ];
+  const double m10 = A[qI * N + pJ], m11 = A[qI * N + qJ];
+  // M R_J
+  const double a00 = cJ * m00 - sJ * m01, a01 = sJ * m00 + cJ * m01;
+  const double a10 = cJ * m10 - sJ * m11, a11 = sJ * m10 + cJ * m11;
+  // R_I^T (M R_J)
+  double b00 = cI * a00 - sI * a10, b01 = cI * a01 - sI * a11;
+  double b10 = sI * a00 + cI * a10, b11 = sI * a01 + cI * a11;
+  if (I == J) {
+    b01 = 0.0;
+    b10 = 0.0;
+  }
+  A[pI * N + pJ] = b00;
+  A[pI * N + qJ] = b01;
+  A[qI * N + pJ] = b10;
+  A[qI * N + qJ] = b11;
+}
+
+// V <- V J  (columns p, q of every row)
+__global__ void k_jacobi_vec(double* __restrict__ V, int64_t N, int64_t k,
+                             const double* __restrict__ cs) {
+  const int64_t J = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t row = blockIdx.y;
+  if (J >= N / 2) return;
+  int64_t p, q;
+  rr_pair(N, k, J, &p, &q);
+  const double c = cs[2 * J], s = cs[2 * J + 1];
+  const double vp = V[row * N + p], vq = V[row * N + q];
+  V[row * N + p] = c * vp - s * vq;
+  V[row * N + q] = s * vp + c * vq;
+}
+
+__global__ void k_offdiag(const double* __restrict__ A, int64_t N, double* __restrict__ out) {
+  __shared__ double so[256], sd[256];
+  double off = 0.0, dg = 0.0;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < N * N;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const double v = A[e];
+    if (e / N == e % N) dg += v * v;
+    else off += v * v;
+  }
+  so[threadIdx.x] = off;
+  sd[threadIdx.x] = dg;
+  __syncthreads();
+  for (int s = 128; s > 0; s >>= 1) {
+    if (threadIdx.x < s) {
+      so[threadIdx.x] += so[threadIdx.x + s];
+      sd[threadIdx.x] += sd[threadIdx.x + s];
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    out[2 * blockIdx.x] = so[0];
+    out[2 * blockIdx.x + 1] = sd[0];
+  }
+}
+
+__global__ void k_eye(double* V, int64_t N) {
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < N * N;
+       e += (int64_t)gridDim.x * blockDim.x)
+    V[e] = (e / N == e % N) ? 1.0 : 0.0;
+}
+
+// fp32 m x n -> fp64, optionally transposed (out n x m), zero-padded to Np
+__global__ void k_x_to_f64(const float* __restrict__ X, int64_t m, int64_t n, int transpose,
+                           double* __restrict__ out) {
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < m * n;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t i = e / n, j = e % n;
+    if (transpose) out[j * m + i] = (double)X[e];
+    else out[e] = (double)X[e];
+  }
+}
+
+// copy the N0 x N0 Gram into an N x N zero-padded matrix
+__global__ void k_pad(const double* __restrict__ G, int64_t N0, int64_t N, double* __restrict__ A) {
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < N * N;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t i = e / N, j = e % N;
+    A[e] = (i < N0 && j < N0) ? G[i * N0 + j] : 0.0;
+  }
+}
+
+// descending rank of each eigenvalue (ties by index): rank_i = #{j: l_j > l_i or (l_j == l_i and j < i)}
+__global__ void k_rank(const double* __restrict__ A, int64_t N, int64_t N0, int* __restrict__ rank) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= N0) return;
+  const double li = A[i * N + i];
+  int r = 0;
+  for (int64_t j = 0; j < N0; ++j) {
+    const double lj = A[j * N + j];
+    r += (lj > li) || (lj == li && j < i);
+  }
+  rank[i] = r;
+}
+
+// eigen-pairs in descending order: lam[rank] and vectors E[:, rank] (E N0 x N0)
+__global__ void k_gather_sorted(const double* __restrict__ A, const double* __restrict__ V,
+                                int64_t N, int64_t N0, const int* __restrict__ rank,
+                                double* __restrict__ lam, double* __restrict__ E) {
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= N0 * N0) return;
+  const int64_t row = e / N0, col = e % N0;
+  const int rk = rank[col];
+  E[row * N0 + rk] = V[row * N + col];
+  if (row == 0) lam[rk] = A[col * N + col];
+}
+
+__global__ void k_sqrt_first(const double* __restrict__ lam, int64_t r, double* __restrict__ s) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < r) s[i] = sqrt(fmax(lam[i], 0.0));
+}
+
+// first r columns of E (N0 x N0) -> out (N0 x r)
+__global__ void k_take_cols(const double* __restrict__ E, int64_t N0, int64_t r, double* __restrict__ out) {
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= N0 * r) return;
+  out[e] = E[(e / r) * N0 + e % r];
+}
+
+// Ut (r x m) = E[:, :r]^T
+__global__ void k_take_cols_t(const double* __restrict__ E, int64_t N0, int64_t r, double* __restrict__ out) {
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= N0 * r) return;
+  const int64_t l = e / N0, i = e % N0;
+  out[e] = E[i * N0 + l];
+}
+
+__global__ void k_div_cols(double* __restrict__ V, int64_t n, int64_t r, const double* __restrict__ s) {
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n * r;
+       e += (int64_t)gridDim.x * blockDim.x)
+    V[e] /= s[e % r];
+}
+
+unsigned g1(int64_t count) { return (unsigned)std::min<int64_t>(cdiv(count, 256), 148 * 32); }
+
+template <typename T>
+struct DevBuf {
+  T* p = nullptr;
+  ~DevBuf() {
+    if (p) cudaFree(p);
+  }
+  mpq_status alloc(int64_t count) {
+    cudaError_t e = cudaMalloc((void**)&p, sizeof(T) * (size_t)std::max<int64_t>(count, 1));
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      p = nullptr;
+      return fail(MPQ_ERR_OOM, "setup allocation failed");
+    }
+    return MPQ_OK;
+  }
+};
+
+// Symmetric eigendecomposition of the N0 x N0 matrix G (device, fp64):
+// descending eigenvalues lam (N0) and eigenvectors E (N0 x N0, columns).
+mpq_status jacobi_eig(const double* G, int64_t N0, double* lam, double* E, cudaStream_t st) {
+  const int64_t N = N0 + (N0 & 1);  // even; the pad row/col is zero
+  DevBuf<double> A, V, cs, red;
+  DevBuf<int> rank;
+  MPQ_TRY(A.alloc(N * N));
+  MPQ_TRY(V.alloc(N * N));
+  MPQ_TRY(cs.alloc(N));
+  const int red_blocks = 256;
+  MPQ_TRY(red.alloc(2 * red_blocks));
+  MPQ_TRY(rank.alloc(N0));
+  {
+    ProfScope ps_("k_pad", st);
+    k_pad<<<g1(N * N), 256, 0, st>>>(G, N0, N, A.p);
+  }
+  {
+    ProfScope ps_("k_eye", st);
+    k_eye<<<g1(N * N), 256, 0, st>>>(V.p, N);
+  }
+  count_launch(2);
+  MPQ_TRY(check_launch("jacobi init"));
+  std::vector<double> h(2 * red_blocks);
+  const int64_t half = N / 2;
+  bool converged = (N <= 1);
+  for (int sweep = 0; sweep < JACOBI_MAX_SWEEPS && !converged; ++sweep) {
+    for (int64_t k = 0; k < N - 1; ++k) {
+      {
+        ProfScope ps_("k_jacobi_rot", st);
+        k_jacobi_rot<<<(unsigned)cdiv(half, 256), 256, 0, st>>>(A.p, N, k, cs.p);
+      }
+      dim3 ga((unsigned)cdiv(half, 128), (unsigned)half);
+      {
+        ProfScope ps_("k_jacobi_apply", st);
+        k_jacobi_apply<<<ga, 128, 0, st>>>(A.p, N, k, cs.p);
+      }
+      dim3 gv((unsigned)cdiv(half, 128), (unsigned)N);
+      {
+        ProfScope ps_("k_jacobi_vec", st);
+        k_jacobi_vec<<<gv, 128, 0, st>>>(V.p, N, k, cs.p);
+      }
+      count_launch(3);
+    }
+    MPQ_TRY(check_launch("jacobi sweep"));
+    {
+      ProfScope ps_("k_offdiag", st);
+      k_offdiag<<<red_blocks, 256, 0, st>>>(A.p, N, red.p);
+    }
+    count_launch();
+    MPQ_CUDA(cudaMemcpyAsync(h.data(), red.p, sizeof(double) * 2 * red_blocks, cudaMemcpyDeviceToHost, st));
+    MPQ_CUDA(cudaStreamSynchronize(st));
+    double off = 0.0, dg = 0.0;
+    for (int b = 0; b < red_blocks; ++b) {
+      off += h[2 * b];
+      dg += h[2 * b + 1];
+    }
+    converged = !(off > 1e-28 * dg) || dg == 0.0;
+  }
+  if (!converged) return fail(MPQ_ERR_TIMEOUT, "Jacobi eigensolver did not converge in 40 sweeps");
+  {
+    ProfScope ps_("k_rank", st);
+    k_rank<<<(unsigned)cdiv(N0, 256), 256, 0, st>>>(A.p, N, N0, rank.p);
+  }
+  {
+    ProfScope ps_("k_gather_sorted", st);
+    k_gather_sorted<<<(unsigned)cdiv(N0 * N0, 256), 256, 0, st>>>(A.p, V.p, N, N0, rank.p, lam, E);
+  }
+  count_launch(2);
+  return check_launch("jacobi sort");
+}
+
+}  // namespace
+
+mpq_status setup_spectrum_from_x(mpq_plan_s* p, const float* X, int64_t m, int64_t n,
+                                 cudaStream_t st) {
+  const bool right = n <= m;  // Gram X^T X (n x n); else X X^T (m x m)
+  const int64_t N0 = right ? n : m;
+  DevBuf<double> Xd, G, lam, E;
+  MPQ_TRY(Xd.alloc(m * n));
+  MPQ_TRY(G.alloc(N0 * N0));
+  MPQ_TRY(lam.alloc(N0));
+  MPQ_TRY(E.alloc(N0 * N0));
+  {
+    ProfScope ps_("k_x_to_f64", st);
+    k_x_to_f64<<<g1(m * n), 256, 0, st>>>(X, m, n, right ? 1 : 0, Xd.p);
+  }
+  count_launch();
+  MPQ_TRY(check_launch("k_x_to_f64"));
+  if (right) MPQ_TRY(gemm_nt_f64(Xd.p, m, Xd.p, m, G.p, n, n, n, m, st));   // (X^T)(X^T)^T
+  else MPQ_TRY(gemm_nt_f64(Xd.p, n, Xd.p, n, G.p, m, m, m, n, st));          // X X^T
+  MPQ_TRY(jacobi_eig(G.p, N0, lam.p, E.p, st));
+  // rank cut on the host from the sorted eigenvalues (N0 values)
+  std::vector<double> hl(N0);
+  MPQ_CUDA(cudaMemcpyAsync(hl.data(), lam.p, sizeof(double) * N0, cudaMemcpyDeviceToHost, st));
+  MPQ_CUDA(cudaStreamSynchronize(st));
+  const double tol = (N0 > 0 ? hl[0] : 0.0) * (double)std::max(m, n) * ldexp(1.0, -52);
+  int64_t r = 0;
+  while (r < N0 && hl[r] > tol) ++r;
+  if (r == 0) return fail(MPQ_ERR_RANK, "X has rank 0");
+  p->r = r;
+  cudaError_t e1 = cudaMalloc((void**)&p->s64, sizeof(double) * r);
+  cudaError_t e2 = cudaMalloc((void**)&p->V64, sizeof(double) * n * r);
+  if (e1 != cudaSuccess || e2 != cudaSuccess) {
+    cudaGetLastError();
+    return fail(MPQ_ERR_OOM, "spectrum allocation failed");
+  }
+  {
+    ProfScope ps_("k_sqrt_first", st);
+    k_sqrt_first<<<(unsigned)cdiv(r, 256), 256, 0, st>>>(lam.p, r, p->s64);
+  }
+  count_launch();
+  if (right) {
+    {
+      ProfScope ps_("k_take_cols", st);
+      k_take_cols<<<(unsigned)cdiv(N0 * r, 256), 256, 0, st>>>(E.p, N0, r, p->V64);
+    }
+    count_launch();
+    return check_launch("setup gather");
+  }
+  // V = X^T U diag(1/s): (n x r) = Xt (n x m) * Ut (r x m)^T
+  DevBuf<double> Xt, Ut;
+  MPQ_TRY(Xt.alloc(n * m));
+  MPQ_TRY(Ut.alloc(r * m));
+  {
+    ProfScope ps_("k_x_to_f64", st);
+    k_x_to_f64<<<g1(m * n), 256, 0, st>>>(X, m, n, 1, Xt.p);
+  }
+  {
+    ProfScope ps_("k_take_cols_t", st);
+    k_take_cols_t<<<(unsigned)cdiv(N0 * r, 256), 256, 0, st>>>(E.p, N0, r, Ut.p);
+  }
+  count_launch(2);
+  MPQ_TRY(check_launch("setup transposes"));
+  MPQ_TRY(gemm_nt_f64(Xt.p, m, Ut.p, m, p->V64, r, n, r, m, st));
+  {
+    ProfScope ps_("k_div_cols", st);
+    k_div_cols<<<g1(n * r), 256, 0, st>>>(p->V64, n, r, p->s64);
+  }
+  count_launch();
+  MPQ_TRY(check_launch("k_div_cols"));
+  MPQ_CUDA(cudaStreamSynchronize(st));
+  return MPQ_OK;
+}
+
+}  // namespace mpq

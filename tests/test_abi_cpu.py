@@ -1,0 +1,69 @@
+"""CPU checks of the C ABI: the library loads, exports every symbol that
+include/mpq.h declares, and rejects bad arguments before touching the GPU."""
+import ctypes as C
+import math
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def mpq():
+    from post_weight_quantization_row_b200 import _lib
+    return _lib
+
+
+def declared_symbols():
+    txt = open(os.path.join(ROOT, "include", "mpq.h")).read()
+    return sorted(set(re.findall(r"^MPQ_API\s+[\w\s\*]+?\b(mpq_\w+)\s*\(", txt, flags=re.M)))
+
+
+def test_header_declares_the_abi():
+    syms = declared_symbols()
+    assert "mpq_solve" in syms and "mpq_plan_create_from_x" in syms
+    assert len(syms) >= 18
+
+
+def test_library_exports_every_declared_symbol(mpq):
+    for name in declared_symbols():
+        assert hasattr(mpq.lib, name), name
+    assert set(declared_symbols()) == set(mpq.EXPORTED)
+
+
+def test_params_default(mpq):
+    p = mpq.Params()
+    mpq.lib.mpq_params_default(C.byref(p), 1, 8)
+    assert p.d == 1 and p.K == 8 and p.beta0 == 1.0 and p.damping == 0.5
+    assert math.isinf(p.tau) and p.gamma_lo_rel == 1e-10 and p.gamma_hi_rel == 1e10
+    assert p.alpha_min == 1e-10 and abs(p.alpha_max - (1 - 1e-5)) < 1e-15
+
+
+@pytest.mark.parametrize("field,value", [("d", 3), ("K", 1), ("damping", 1.5), ("beta0", -1.0),
+                                         ("tau", 0.0), ("alpha_max", 1.0)])
+def test_bad_params_rejected_without_a_device(mpq, field, value):
+    p = mpq.Params()
+    mpq.lib.mpq_params_default(C.byref(p), 1, 8)
+    setattr(p, field, value)
+    h = C.c_void_p()
+    dummy = C.c_void_p(16)
+    st = mpq.lib.mpq_plan_create_from_spectrum(dummy, dummy, 64, 8, C.byref(p), None, C.byref(h))
+    assert st == 1, mpq.lib.mpq_last_error()
+    assert h.value is None
+
+
+def test_null_plan_rejected(mpq):
+    assert mpq.lib.mpq_solve(None, None, 0, None, None, 1, 1, None, None, None, None, None) == 1
+    assert b"plan" in mpq.lib.mpq_last_error()
+    assert mpq.lib.mpq_plan_destroy(None) == 0
+
+
+def test_codebook_required_for_vector_plans(mpq):
+    p = mpq.Params()
+    mpq.lib.mpq_params_default(C.byref(p), 8, 16)
+    h = C.c_void_p()
+    st = mpq.lib.mpq_plan_create_from_spectrum(C.c_void_p(16), C.c_void_p(16), 64, 8, C.byref(p),
+                                               None, C.byref(h))
+    assert st == 1
