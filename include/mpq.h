@@ -215,6 +215,32 @@ MPQ_API mpq_status mpq_stage_energy(mpq_plan_t plan, const float* W, int64_t m, 
                             const float* offset, const uint16_t* idx, float* w_hat, float* energy,
                             mpq_stream_t stream);
 
+/* Allocation-free variant of mpq_stage_energy (the paper has no counterpart;
+ * this exists for integration).  Some callers cannot let a library allocate
+ * device memory: a framework whose allocator owns all of the GPU's memory, a
+ * serving loop that must never stall on the device-wide synchronisation an
+ * allocation or free can cause, or a process whose memory budget is fixed at
+ * start-up.  This entry point uses no plan workspace and calls no allocator:
+ * its intermediates (the residual w - w_hat, its projection V^T (w - w_hat)
+ * and a sanitised copy of idx) live in one static device array of
+ * MPQ_NOALLOC_SCRATCH_BYTES bytes that every GPU loading the library holds
+ * until the process exits.
+ *   Same arguments, layouts and results as mpq_stage_energy.
+ *   Limit: m * (4 n + 4 r + 2 B) bytes (each part rounded up to 256) must
+ *   fit in MPQ_NOALLOC_SCRATCH_BYTES; larger calls return
+ *   MPQ_ERR_INVALID_ARG without launching -- split the rows.
+ *   The plan's device must be current.  The first call on a device looks
+ *   up the array's device address (cudaGetSymbolAddress) and caches it;
+ *   make that first call before any stream capture.
+ *   All calls on a device share the one array and it keeps the last call's
+ *   contents; two calls whose work overlaps on the GPU (different streams,
+ *   no ordering between them) race on it, so order them on one stream. */
+#define MPQ_NOALLOC_SCRATCH_BYTES (16u << 20)
+MPQ_API mpq_status mpq_stage_energy_noalloc(mpq_plan_t plan, const float* W, int64_t m,
+                                            const float* scale, const float* offset,
+                                            const uint16_t* idx, float* w_hat, float* energy,
+                                            mpq_stream_t stream);
+
 /* ----------------------------------------------------------- profiling --- */
 /* Per-kernel timing with CUDA events recorded on the launching stream around
  * every kernel the library launches while profiling is on.  start clears

@@ -78,6 +78,7 @@ _sig("mpq_stage_denoise", ST, P, P, P, P, P, I64, P, P, P, P, P, P, P)
 _sig("mpq_stage_linear", ST, P, P, I64, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P)
 _sig("mpq_stage_cd", ST, P, P, I64, P, P, P, I32, P, P)
 _sig("mpq_stage_energy", ST, P, P, I64, P, P, P, P, P, P)
+_sig("mpq_stage_energy_noalloc", ST, P, P, I64, P, P, P, P, P, P)
 _sig("mpq_profile_start", ST)
 _sig("mpq_profile_stop", ST, C.c_char_p, I64)
 _sig("mpq_last_error", C.c_char_p)
@@ -87,7 +88,8 @@ EXPORTED = ["mpq_params_default", "mpq_plan_create_from_spectrum", "mpq_plan_cre
             "mpq_plan_destroy", "mpq_plan_info", "mpq_plan_get_spectrum", "mpq_plan_status",
             "mpq_plan_workspace_bytes", "mpq_plan_set_workspace_cap", "mpq_solve",
             "mpq_solve_host", "mpq_stage_init", "mpq_stage_denoise", "mpq_stage_linear",
-            "mpq_stage_cd", "mpq_stage_energy", "mpq_profile_start", "mpq_profile_stop",
+            "mpq_stage_cd", "mpq_stage_energy", "mpq_stage_energy_noalloc",
+            "mpq_profile_start", "mpq_profile_stop",
             "mpq_last_error", "mpq_kernel_launch_count"]
 
 
@@ -346,6 +348,27 @@ class Plan:
                                    _ptr(idx, torch.int16, (m, self.B), "idx"), _ptr(w_hat),
                                    _ptr(energy), _stream()), "mpq_stage_energy")
         return {"w_hat": w_hat, "energy": energy}
+
+
+    def stage_energy_noalloc(self, W, scale, offset, idx, w_hat=None, energy=None):
+        """mpq_stage_energy_noalloc: the energy stage without any allocation in
+        the library (its scratch is a static device array).  Output tensors
+        are allocated here by the caller side unless given."""
+        m = W.shape[0]
+        if w_hat is None:
+            w_hat = torch.empty(m, self.n, dtype=torch.float32, device=W.device)
+        if energy is None:
+            energy = torch.empty(m, dtype=torch.float32, device=W.device)
+        check(lib.mpq_stage_energy_noalloc(self._h, _ptr(W, torch.float32, (m, self.n), "W"), m,
+                                           _ptr(scale, torch.float32, (m,), "scale"),
+                                           _ptr(offset, torch.float32, (m,), "offset"),
+                                           _ptr(idx, torch.int16, (m, self.B), "idx"),
+                                           _ptr(w_hat), _ptr(energy), _stream()),
+              "mpq_stage_energy_noalloc")
+        return {"w_hat": w_hat, "energy": energy}
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 def idx_to_numpy(idx: torch.Tensor) -> np.ndarray:
