@@ -1,0 +1,357 @@
+// Tensor-core GEMM for the fp32 contractions of the solve (sm_100a tcgen05).
+//
+//   C[M x N] = diag(row_scale) * (A_hi B_hi^T + A_hi B_lo^T + A_lo B_hi^T) * b_scale
+//
+// A and B are fp32 matrices stored as power-of-two-scaled fp16 pairs
+// (x * 2^-e = hi + lo, hi = fp16(x * 2^-e), lo = fp16(x * 2^-e - hi)), so
+// hi + lo carries ~22 significand bits and the three products recover an
+// fp32-accurate contraction (the dropped lo*lo term is ~2^-22 relative).
+// Both operands are K-major (K contiguous).  Tiles: 128 x 256 x 64, fp16
+// kind::f16 MMAs with the fp32 accumulator in TMEM (256 columns), operands
+// staged by TMA (128-byte swizzle, no multicast) through a 2-stage mbarrier
+// pipeline.  Warp 0 issues TMA, warp 1 owns TMEM and issues the MMAs from one
+// thread, warps 2-5 read the accumulator back (tcgen05.ld) and store C.
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "mpq_internal.cuh"
+
+namespace mpq {
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 2;
+constexpr int A_TILE = BM * BK * 2;                 // 16 KiB
+constexpr int B_TILE = BN * BK * 2;                 // 32 KiB
+constexpr int STAGE_BYTES = 2 * A_TILE + 2 * B_TILE;  // 96 KiB
+constexpr int TC_THREADS = 192;
+constexpr uint32_t TMEM_COLS = 256;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /* alignment slack */ + 128;
+
+// instruction descriptor, kind::f16: fp32 accumulate (bits 4-5 = 1), A and
+// B fp16 (format 0), both K-major, N >> 3 at bits 17-22, M >> 4 at bits 24-28
+constexpr uint32_t IDESC = (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait (>= about a second of polling); false on timeout.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  for (uint32_t i = 0; i < (1u << 25); ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (i > 256) __nanosleep(64);
+  }
+  return false;
+}
+
+__device__ __forceinline__ void tma_load_2d(const CUtensorMap* tm, uint64_t* bar, void* dst,
+                                            int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"((uint64_t)tm), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// K-major operand tile of `rows` x 64 fp16 written by TMA with 128-byte
+// swizzle: rows of 128 B, 8-row groups 1024 B apart (SBO), layout type 2
+// (SWIZZLE_128B), descriptor version 1.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1 << 16;
+  d |= (uint64_t)(1024 >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
+__device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(IDESC), "r"(accum));
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+        "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]),
+        "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]),
+        "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__global__ void __launch_bounds__(TC_THREADS, 1)
+    k_gemm_tc(const __grid_constant__ CUtensorMap ta_hi, const __grid_constant__ CUtensorMap ta_lo,
+              const __grid_constant__ CUtensorMap tb_hi, const __grid_constant__ CUtensorMap tb_lo,
+              float* __restrict__ C, int64_t ldc, int M, int N, int K,
+              const float* __restrict__ row_scale, float b_scale, int* status) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint64_t* full = (uint64_t*)(smem + STAGES * STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* done = empty + STAGES;
+  uint32_t* tmem_slot = (uint32_t*)(done + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
+  const int KT = (K + BK - 1) / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(done, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(TMEM_COLS));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------------------------------------------------- producer
+    for (int kt = 0; kt < KT; ++kt) {
+      const int s = kt % STAGES, it = kt / STAGES;
+      if (kt >= STAGES && !mbar_wait(&empty[s], (it - 1) & 1)) {
+        atomicOr(status, STATUS_TIMEOUT);
+        break;
+      }
+      uint8_t* base = smem + s * STAGE_BYTES;
+      mbar_expect_tx(&full[s], STAGE_BYTES);
+      tma_load_2d(&ta_hi, &full[s], base, kt * BK, m0);
+      tma_load_2d(&ta_lo, &full[s], base + A_TILE, kt * BK, m0);
+      tma_load_2d(&tb_hi, &full[s], base + 2 * A_TILE, kt * BK, n0);
+      tma_load_2d(&tb_lo, &full[s], base + 2 * A_TILE + B_TILE, kt * BK, n0);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------- MMA issuer
+    bool ok = true;
+    for (int kt = 0; kt < KT && ok; ++kt) {
+      const int s = kt % STAGES, it = kt / STAGES;
+      if (!mbar_wait(&full[s], it & 1)) {
+        atomicOr(status, STATUS_TIMEOUT);
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t a_hi = smem_u32(smem + s * STAGE_BYTES);
+      const uint32_t a_lo = a_hi + A_TILE;
+      const uint32_t b_hi = a_hi + 2 * A_TILE;
+      const uint32_t b_lo = b_hi + B_TILE;
+#pragma unroll
+      for (int kk = 0; kk < BK / 16; ++kk) {
+        const uint32_t off = kk * 32;  // 16 fp16 along K inside the 128-byte row
+        const uint64_t dah = sw128_desc(a_hi + off), dal = sw128_desc(a_lo + off);
+        const uint64_t dbh = sw128_desc(b_hi + off), dbl = sw128_desc(b_lo + off);
+        umma_f16(tmem, dah, dbh, (kt | kk) != 0 ? 1u : 0u);
+        umma_f16(tmem, dah, dbl, 1u);
+        umma_f16(tmem, dal, dbh, 1u);
+      }
+      umma_commit(&empty[s]);
+    }
+    umma_commit(done);
+  } else if (warp >= 2) {
+    // --------------------------------------------------------- epilogue
+    // warp-uniform outcome: the TMEM loads below are .sync.aligned
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(done, 0));
+    if (!ok && lane == 0) atomicOr(status, STATUS_TIMEOUT);
+    tc_fence_after();
+    const int q = warp & 3;  // TMEM lane quadrant this warp may read
+    const int row = m0 + q * 32 + lane;
+    const float rs = (row < M) ? row_scale[row] * b_scale : 0.0f;
+    for (int c0 = 0; c0 < BN && ok; c0 += 32) {
+      if (n0 + c0 >= N) break;
+      uint32_t v[32];
+      tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c0, v);
+      if (row < M) {
+        float* crow = C + (int64_t)row * ldc + n0 + c0;
+        if (n0 + c0 + 32 <= N && (ldc & 3) == 0) {
+#pragma unroll
+          for (int j = 0; j < 32; j += 4) {
+            float4 o = make_float4(__uint_as_float(v[j]) * rs, __uint_as_float(v[j + 1]) * rs,
+                                   __uint_as_float(v[j + 2]) * rs, __uint_as_float(v[j + 3]) * rs);
+            *reinterpret_cast<float4*>(crow + j) = o;
+          }
+        } else {
+          for (int j = 0; j < 32 && n0 + c0 + j < N; ++j) crow[j] = __uint_as_float(v[j]) * rs;
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(TMEM_COLS));
+  }
+}
+
+// --------------------------------------------------------------- splitting --
+// Global-scale split of a fp32 matrix (plan-time operands V, V^T, H):
+// dst = src * 2^-e as fp16 hi/lo, rows x ld (zero beyond K), e from max|src|.
+__global__ void k_absmax(const float* __restrict__ x, int64_t count, unsigned* out) {
+  float m = 0.0f;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < count;
+       i += (int64_t)gridDim.x * blockDim.x)
+    m = fmaxf(m, fabsf(x[i]));
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) atomicMax(out, __float_as_uint(m));  // m >= 0: order-preserving
+}
+
+__global__ void k_split_global(const float* __restrict__ src, int64_t rows, int64_t K,
+                               int64_t ld, const unsigned* __restrict__ amax_bits,
+                               __half* __restrict__ hi, __half* __restrict__ lo,
+                               float* __restrict__ unscale) {
+  const float amax = __uint_as_float(*amax_bits);
+  int ex = 0;
+  frexpf(amax, &ex);
+  const int e = (amax > 0.0f) ? ex - 14 : 0;  // scaled |x| < 2^14
+  const float down = ldexpf(1.0f, -e);
+  if (blockIdx.x == 0 && threadIdx.x == 0) *unscale = ldexpf(1.0f, e);
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < rows * ld;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = i / ld, c = i % ld;
+    const float x = (c < K) ? src[r * K + c] * down : 0.0f;
+    const __half h = __float2half_rn(x);
+    hi[i] = h;
+    lo[i] = __float2half_rn(x - __half2float(h));
+  }
+}
+
+// ---------------------------------------------------- tensor-map encoding --
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::mutex g_encode_mu;
+
+mpq_status get_encoder() {
+  std::lock_guard<std::mutex> lk(g_encode_mu);
+  if (g_encode) return MPQ_OK;
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q{};
+  cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+  if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn)
+    return fail(MPQ_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  return MPQ_OK;
+}
+
+bool g_smem_attr_set[64] = {};
+
+}  // namespace
+
+mpq_status make_tmap_f16(CUtensorMap* tm, const void* base, int64_t inner, int64_t rows,
+                         int64_t ld_elems, int box_rows) {
+  MPQ_TRY(get_encoder());
+  if (((uintptr_t)base & 15) || (ld_elems * 2) % 16 || inner % 64 || rows < box_rows)
+    return fail(MPQ_ERR_INVALID_ARG, "tensor map: misaligned operand");
+  cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(ld_elems * 2)};
+  cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims,
+                        strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(MPQ_ERR_CUDA, "cuTensorMapEncodeTiled failed with code " + std::to_string((int)r));
+  return MPQ_OK;
+}
+
+mpq_status split_global(const float* src, int64_t rows, int64_t K, SplitOperand* dst,
+                        cudaStream_t st) {
+  unsigned* amax = nullptr;
+  MPQ_CUDA(cudaMallocAsync(&amax, sizeof(unsigned), st));
+  MPQ_CUDA(cudaMemsetAsync(amax, 0, sizeof(unsigned), st));
+  {
+    ProfScope ps_("k_absmax", st);
+    k_absmax<<<(unsigned)std::min<int64_t>(cdiv(rows * K, 256), 148 * 8), 256, 0, st>>>(src, rows * K, amax);
+  }
+  {
+    ProfScope ps_("k_split_global", st);
+    k_split_global<<<(unsigned)std::min<int64_t>(cdiv(dst->rows_pad * dst->ld, 256), 148 * 16), 256, 0, st>>>(
+        src, rows, K, dst->ld, amax, dst->hi, dst->lo, dst->unscale);
+  }
+  count_launch(2);
+  MPQ_TRY(check_launch("split_global"));
+  cudaFreeAsync(amax, st);
+  return MPQ_OK;
+}
+
+mpq_status gemm_tc(const SplitOperand& A, const CUtensorMap& ta_hi, const CUtensorMap& ta_lo,
+                   const SplitOperand& B, const CUtensorMap& tb_hi, const CUtensorMap& tb_lo,
+                   float* C, int64_t ldc, int64_t M, int64_t N, int64_t K, float b_scale_host,
+                   int* status, cudaStream_t st, const char* tag) {
+  if (M <= 0 || N <= 0) return MPQ_OK;
+  if (M > A.rows_pad || N > B.rows_pad || K > A.ld || K > B.ld)
+    return fail(MPQ_ERR_INVALID_ARG, "gemm_tc: operand smaller than the problem");
+  int dev = 0;
+  MPQ_CUDA(cudaGetDevice(&dev));
+  if (dev >= 0 && dev < 64 && !g_smem_attr_set[dev]) {
+    MPQ_CUDA(cudaFuncSetAttribute(k_gemm_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES));
+    g_smem_attr_set[dev] = true;
+  }
+  dim3 grid((unsigned)cdiv(N, BN), (unsigned)cdiv(M, BM));
+  {
+    ProfScope ps_(tag, st);
+    k_gemm_tc<<<grid, TC_THREADS, SMEM_BYTES, st>>>(ta_hi, ta_lo, tb_hi, tb_lo, C, ldc, (int)M,
+                                                    (int)N, (int)K, A.row_unscale, b_scale_host,
+                                                    status);
+  }
+  count_launch();
+  return check_launch("k_gemm_tc");
+}
+
+}  // namespace mpq

@@ -77,6 +77,21 @@ __device__ __forceinline__ double clip_count(double v, double lo, double hi, int
   return c;
 }
 
+// Split of a row for the tensor-core GEMM: a per-row power of two e with
+// max|x| * 2^-e < 2^14, then hi = fp16(x 2^-e), lo = fp16(x 2^-e - hi).
+__device__ __forceinline__ int split_exponent(float amax) {
+  int ex = 0;
+  frexpf(amax, &ex);
+  return (amax > 0.0f) ? ex - 14 : 0;
+}
+
+__device__ __forceinline__ void split_store(float xs, __half* __restrict__ hi,
+                                            __half* __restrict__ lo, int64_t o) {
+  const __half h = __float2half_rn(xs);
+  hi[o] = h;
+  lo[o] = __float2half_rn(xs - __half2float(h));
+}
+
 // ------------------------------------------------------------------ init ---
 // d = 1: per-row min-max grid (unless given), nearest level, gamma1_0.
 __global__ void __launch_bounds__(ROW_THREADS)
@@ -368,15 +383,18 @@ __global__ void __launch_bounds__(ROW_THREADS)
 // ------------------------------------------------- extrinsic d -> linear ---
 // alpha1 = gamma1 vsum / n (clipped), gamma2 = gamma1 (1 - alpha1)/alpha1
 // (clipped), r2 = r1 + (xhat1 - r1)/(1 - alpha1)  [= (xhat1 - alpha1 r1)/
-// (1 - alpha1) = (eta1 xhat1 - gamma1 r1)/gamma2], A = w - r2.
+// (1 - alpha1) = (eta1 xhat1 - gamma1 r1)/gamma2].  Also writes the GEMM1
+// operand w - r2 split for the tensor cores (K = n view, zero up to ldn).
 __global__ void __launch_bounds__(ROW_THREADS)
     k_extrinsic_d2l(const float* __restrict__ W, int64_t n, const float* __restrict__ R1,
                     const double* __restrict__ gamma1, const float* __restrict__ X1,
                     const double* __restrict__ vsum, const double* __restrict__ gamma1_0,
                     double glo, double ghi, double amin, double amax, float* __restrict__ R2,
-                    float* __restrict__ A, double* __restrict__ gamma2,
+                    __half* __restrict__ ahi, __half* __restrict__ alo, int64_t lda, int64_t ldn,
+                    float* __restrict__ a_unscale, double* __restrict__ gamma2,
                     int32_t* __restrict__ clamps) {
   __shared__ float cf;
+  __shared__ float fs[33];
   const int64_t row = blockIdx.x;
   if (threadIdx.x == 0) {
     int cnt = 0;
@@ -390,13 +408,22 @@ __global__ void __launch_bounds__(ROW_THREADS)
   }
   __syncthreads();
   const float c = cf;
+  float mx = 0.0f;
   for (int64_t j = threadIdx.x; j < n; j += blockDim.x) {
     const int64_t o = row * n + j;
     const float r1 = R1[o];
     const float r2 = fmaf(c, X1[o] - r1, r1);
     R2[o] = r2;
-    A[o] = W[o] - r2;
+    mx = fmaxf(mx, fabsf(W[o] - r2));
   }
+  mx = block_reduce(mx, MaxF(), fs);
+  const int ex = split_exponent(mx);
+  const float down = ldexpf(1.0f, -ex);
+  for (int64_t j = threadIdx.x; j < ldn; j += blockDim.x) {
+    const float x = (j < n) ? (W[row * n + j] - R2[row * n + j]) * down : 0.0f;
+    split_store(x, ahi, alo, row * lda + j);
+  }
+  if (threadIdx.x == 0) a_unscale[row] = ldexpf(1.0f, ex);
 }
 
 // -------------------------------------- linear module epilogue + M-step ---
@@ -405,7 +432,7 @@ __global__ void __launch_bounds__(ROW_THREADS)
 // 1/beta_hat = (1/r) sum[F^2 u^2 + s^2/(beta s^2 + gamma2)],
 // beta <- (1-rho) beta + rho beta_hat, gamma1' = gamma2 (1-alpha2)/alpha2
 // (clipped), coef = 1/(1 - alpha2), kappa = alpha2/(1 - alpha2).
-// GEMM2 operand written back into P:
+// GEMM2 operand (written into P, then split for the tensor cores, K = r):
 //   r < n: (1 - F) p'            -> G = V (D u) = xhat2 - r2
 //   r = n: -F p'                 -> G = xhat2 - w  (V V^T = I), which avoids
 //          forming r2 + V V^T (w - r2) when r2 is far from w.
@@ -416,11 +443,15 @@ __global__ void __launch_bounds__(ROW_THREADS)
                   double amin, double amax, int full_rank, double* __restrict__ gamma1_out,
                   double* __restrict__ coef, double* __restrict__ kappa,
                   double* __restrict__ alpha2_out, double* __restrict__ beta_hat_out,
-                  int32_t* __restrict__ clamps, float* __restrict__ Uprime) {
+                  int32_t* __restrict__ clamps, float* __restrict__ Uprime,
+                  __half* __restrict__ ahi, __half* __restrict__ alo, int64_t lda, int64_t ldr,
+                  float* __restrict__ a_unscale) {
   __shared__ double ds[33];
+  __shared__ float fs[33];
   const int64_t row = blockIdx.x;
   const double b = beta[row], g2 = gamma2[row];
   double a2s = 0.0, bs = 0.0;
+  float mx = 0.0f;
   for (int64_t l = threadIdx.x; l < r; l += blockDim.x) {
     const double sl = s[l];
     const double pl = (double)P[row * r + l];
@@ -430,11 +461,21 @@ __global__ void __launch_bounds__(ROW_THREADS)
     a2s += f;
     bs += f * f * u * u + sl * sl / den;
     if (Uprime) Uprime[row * r + l] = (float)((1.0 - f) * pl);
-    P[row * r + l] = (float)(full_rank ? -f * pl : (1.0 - f) * pl);
+    const float q = (float)(full_rank ? -f * pl : (1.0 - f) * pl);
+    P[row * r + l] = q;
+    mx = fmaxf(mx, fabsf(q));
   }
   a2s = block_sum(a2s, ds);
   bs = block_sum(bs, ds);
+  mx = block_reduce(mx, MaxF(), fs);
+  const int ex = split_exponent(mx);
+  const float down = ldexpf(1.0f, -ex);
+  for (int64_t l = threadIdx.x; l < ldr; l += blockDim.x) {
+    const float x = (l < r) ? P[row * r + l] * down : 0.0f;
+    split_store(x, ahi, alo, row * lda + l);
+  }
   if (threadIdx.x == 0) {
+    a_unscale[row] = ldexpf(1.0f, ex);
     int cnt = 0;
     const double alpha2 = (a2s + (double)(n - r)) / (double)n;
     const double bhat = (double)r / bs;
@@ -452,26 +493,24 @@ __global__ void __launch_bounds__(ROW_THREADS)
 
 // ------------------------------------------------- extrinsic linear -> d ---
 // r1' = (xhat2 - alpha2 r2)/(1 - alpha2) = (eta2 xhat2 - gamma2 r2)/gamma1'.
-//   r < n: G = xhat2 - r2:  r1' = r2 + coef G,            xhat2 = r2 + G
-//   r = n: G = xhat2 - w:   r1' = w + kappa e + coef G,  xhat2 = w + G,
-//          with e = w - r2 (the GEMM1 operand).
+//   r < n: G = xhat2 - r2:  r1' = r2 + coef G,              xhat2 = r2 + G
+//   r = n: G = xhat2 - w:   r1' = w + kappa (w - r2) + coef G,  xhat2 = w + G
 __global__ void __launch_bounds__(ROW_THREADS)
     k_extrinsic_l2d(const float* __restrict__ W, const float* __restrict__ R2,
-                    const float* __restrict__ E, const float* __restrict__ G, int64_t n,
-                    const double* __restrict__ coef, const double* __restrict__ kappa,
-                    int full_rank, float* __restrict__ R1, float* __restrict__ xhat2) {
+                    const float* __restrict__ G, int64_t n, const double* __restrict__ coef,
+                    const double* __restrict__ kappa, int full_rank, float* __restrict__ R1,
+                    float* __restrict__ xhat2) {
   const int64_t row = blockIdx.x;
   const float c = (float)coef[row];
   const float k = (float)kappa[row];
   for (int64_t j = threadIdx.x; j < n; j += blockDim.x) {
     const int64_t o = row * n + j;
-    const float g = G[o];
+    const float g = G[o], r2 = R2[o];
     if (full_rank) {
       const float w = W[o];
-      R1[o] = fmaf(c, g, fmaf(k, E[o], w));
+      R1[o] = fmaf(c, g, fmaf(k, w - r2, w));
       if (xhat2) xhat2[o] = w + g;
     } else {
-      const float r2 = R2[o];
       R1[o] = fmaf(c, g, r2);
       if (xhat2) xhat2[o] = r2 + g;
     }
@@ -494,6 +533,40 @@ __global__ void __launch_bounds__(ROW_THREADS)
     E[row * n + j] = W[row * n + j] - wh;
     if (w_hat) w_hat[row * n + j] = wh;
   }
+}
+
+// residual w - w_hat split for the tensor cores (K = n view), w_hat optional
+__global__ void __launch_bounds__(ROW_THREADS)
+    k_residual_split(const float* __restrict__ W, int64_t n, int d, const float* __restrict__ cb,
+                     const float* __restrict__ scale, const float* __restrict__ offset,
+                     const uint16_t* __restrict__ idx, float* __restrict__ w_hat,
+                     __half* __restrict__ ahi, __half* __restrict__ alo, int64_t lda, int64_t ldn,
+                     float* __restrict__ a_unscale) {
+  __shared__ float fs[33];
+  const int64_t row = blockIdx.x;
+  const float sc = scale[row], off = offset[row];
+  const int64_t B = n / d;
+  float mx = 0.0f;
+  for (int64_t j = threadIdx.x; j < n; j += blockDim.x) {
+    const int k = idx[row * B + j / d];
+    const float c = (d == 1) ? (float)k : cb[(int64_t)k * d + (j % d)];
+    const float wh = fmaf(sc, c, off);
+    if (w_hat) w_hat[row * n + j] = wh;
+    mx = fmaxf(mx, fabsf(W[row * n + j] - wh));
+  }
+  mx = block_reduce(mx, MaxF(), fs);
+  const int ex = split_exponent(mx);
+  const float down = ldexpf(1.0f, -ex);
+  for (int64_t j = threadIdx.x; j < ldn; j += blockDim.x) {
+    float x = 0.0f;
+    if (j < n) {
+      const int k = idx[row * B + j / d];
+      const float c = (d == 1) ? (float)k : cb[(int64_t)k * d + (j % d)];
+      x = (W[row * n + j] - fmaf(sc, c, off)) * down;
+    }
+    split_store(x, ahi, alo, row * lda + j);
+  }
+  if (threadIdx.x == 0) a_unscale[row] = ldexpf(1.0f, ex);
 }
 
 __global__ void __launch_bounds__(ROW_THREADS)
@@ -632,50 +705,65 @@ mpq_status launch_denoise(const mpq_plan_s* p, const float* R1, const double* ga
 
 mpq_status launch_extrinsic_d2l(const mpq_plan_s* p, const float* W, int64_t m, const float* R1,
                                 const double* gamma1, const float* xhat1, const double* vsum,
-                                const double* gamma1_0, float* R2, float* A, double* gamma2,
-                                int32_t* clamps, cudaStream_t st) {
+                                const double* gamma1_0, float* R2, SplitOperand* As,
+                                double* gamma2, int32_t* clamps, cudaStream_t st) {
   if (m <= 0) return MPQ_OK;
   const mpq_params& q = p->params;
   {
     ProfScope ps_("k_extrinsic_d2l", st);
-    k_extrinsic_d2l<<<rows_grid(m), ROW_THREADS, 0, st>>>(W, p->n, R1, gamma1, xhat1, vsum,
-                                                          gamma1_0, q.gamma_lo_rel, q.gamma_hi_rel,
-                                                          q.alpha_min, q.alpha_max, R2, A, gamma2,
-                                                          clamps);
+    k_extrinsic_d2l<<<rows_grid(m), ROW_THREADS, 0, st>>>(
+        W, p->n, R1, gamma1, xhat1, vsum, gamma1_0, q.gamma_lo_rel, q.gamma_hi_rel, q.alpha_min,
+        q.alpha_max, R2, As->hi, As->lo, As->ld, round_up(p->n, 64), As->row_unscale, gamma2,
+        clamps);
   }
   count_launch();
   return check_launch("k_extrinsic_d2l");
 }
 
-mpq_status launch_linear_rows(const mpq_plan_s* p, int64_t m, float* P, const double* gamma2,
-                              const double* gamma1_0, double* beta, double* gamma1_out,
-                              double* coef, double* kappa, double* alpha2, double* beta_hat,
-                              int32_t* clamps, float* Uprime, cudaStream_t st) {
+mpq_status launch_linear_rows(const mpq_plan_s* p, int64_t m, const float* P,
+                              const double* gamma2, const double* gamma1_0, double* beta,
+                              double* gamma1_out, double* coef, double* kappa, double* alpha2,
+                              double* beta_hat, int32_t* clamps, float* Uprime, SplitOperand* As,
+                              cudaStream_t st) {
   if (m <= 0) return MPQ_OK;
   const mpq_params& q = p->params;
   {
     ProfScope ps_("k_linear_rows", st);
     k_linear_rows<<<rows_grid(m), ROW_THREADS, 0, st>>>(
-        P, p->n, p->r, p->s64, gamma2, gamma1_0, beta, q.damping, q.gamma_lo_rel, q.gamma_hi_rel,
-        q.alpha_min, q.alpha_max, p->r == p->n ? 1 : 0, gamma1_out, coef, kappa, alpha2, beta_hat,
-        clamps, Uprime);
+        const_cast<float*>(P), p->n, p->r, p->s64, gamma2, gamma1_0, beta, q.damping,
+        q.gamma_lo_rel, q.gamma_hi_rel, q.alpha_min, q.alpha_max, p->r == p->n ? 1 : 0,
+        gamma1_out, coef, kappa, alpha2, beta_hat, clamps, Uprime, As->hi, As->lo, As->ld,
+        round_up(p->r, 64), As->row_unscale);
   }
   count_launch();
   return check_launch("k_linear_rows");
 }
 
 mpq_status launch_extrinsic_l2d(const mpq_plan_s* p, const float* W, int64_t m, const float* R2,
-                                const float* E, const float* G, const double* coef,
-                                const double* kappa, float* R1_out, float* xhat2,
-                                cudaStream_t st) {
+                                const float* G, const double* coef, const double* kappa,
+                                float* R1_out, float* xhat2, cudaStream_t st) {
   if (m <= 0) return MPQ_OK;
   {
     ProfScope ps_("k_extrinsic_l2d", st);
-    k_extrinsic_l2d<<<rows_grid(m), ROW_THREADS, 0, st>>>(W, R2, E, G, p->n, coef, kappa,
+    k_extrinsic_l2d<<<rows_grid(m), ROW_THREADS, 0, st>>>(W, R2, G, p->n, coef, kappa,
                                                           p->r == p->n ? 1 : 0, R1_out, xhat2);
   }
   count_launch();
   return check_launch("k_extrinsic_l2d");
+}
+
+mpq_status launch_residual_split(const mpq_plan_s* p, const float* W, int64_t m,
+                                 const float* scale, const float* offset, const uint16_t* idx,
+                                 SplitOperand* As, float* w_hat, cudaStream_t st) {
+  if (m <= 0) return MPQ_OK;
+  {
+    ProfScope ps_("k_residual_split", st);
+    k_residual_split<<<rows_grid(m), ROW_THREADS, 0, st>>>(W, p->n, p->d, p->cb, scale, offset,
+                                                           idx, w_hat, As->hi, As->lo, As->ld,
+                                                           round_up(p->n, 64), As->row_unscale);
+  }
+  count_launch();
+  return check_launch("k_residual_split");
 }
 
 mpq_status launch_residual(const mpq_plan_s* p, const float* W, int64_t m, const float* scale,

@@ -153,8 +153,31 @@ void dfree(T*& p) {
   p = nullptr;
 }
 
+void free_split(SplitOperand& s) {
+  dfree(s.hi); dfree(s.lo); dfree(s.row_unscale); dfree(s.unscale);
+  s = SplitOperand();
+}
+
+// fp16 hi/lo buffers: rows padded to 256, K to 64, zero-filled
+mpq_status alloc_split(SplitOperand& s, int64_t rows, int64_t K, bool per_row) {
+  s.rows = rows;
+  s.rows_pad = round_up(std::max<int64_t>(rows, 1), 256);
+  s.K = K;
+  s.ld = round_up(K, 64);
+  mpq_status st = dalloc(&s.hi, s.rows_pad * s.ld);
+  if (st == MPQ_OK) st = dalloc(&s.lo, s.rows_pad * s.ld);
+  if (st == MPQ_OK && per_row) st = dalloc(&s.row_unscale, s.rows_pad);
+  if (st == MPQ_OK && !per_row) st = dalloc(&s.unscale, 1);
+  if (st != MPQ_OK) return st;
+  MPQ_CUDA(cudaMemset(s.hi, 0, sizeof(__half) * s.rows_pad * s.ld));
+  MPQ_CUDA(cudaMemset(s.lo, 0, sizeof(__half) * s.rows_pad * s.ld));
+  if (per_row) MPQ_CUDA(cudaMemset(s.row_unscale, 0, sizeof(float) * s.rows_pad));
+  return MPQ_OK;
+}
+
 void free_workspace(Workspace& w) {
-  dfree(w.R1); dfree(w.X1); dfree(w.R2); dfree(w.A); dfree(w.P); dfree(w.idx);
+  dfree(w.R1); dfree(w.X1); dfree(w.R2); dfree(w.P); dfree(w.idx);
+  free_split(w.As);
   dfree(w.scale); dfree(w.offset); dfree(w.gamma1); dfree(w.gamma1_0); dfree(w.gamma2);
   dfree(w.beta); dfree(w.vsum); dfree(w.coef); dfree(w.kappa); dfree(w.clamps); dfree(w.W); dfree(w.w_hat);
   dfree(w.energy); dfree(w.idx_stage);
@@ -165,7 +188,8 @@ void free_workspace(Workspace& w) {
 constexpr int MAX_SWEEPS = 64;
 
 int64_t ws_bytes_per_row(const mpq_plan_s* p) {
-  return 4 * p->n * 4 + p->r * 4 + p->B * 2 + 2 * 4 + 8 * 8 + 4 + MAX_SWEEPS * 4;
+  return 3 * p->n * 4 + p->r * 4 + 4 * round_up(std::max(p->n, p->r), 64) + p->B * 2 + 3 * 4 +
+         8 * 8 + 4 + MAX_SWEEPS * 4;
 }
 
 // changes buffer rides in the tail of `clamps`: rows x (1 + MAX_SWEEPS) ints
@@ -180,7 +204,16 @@ mpq_status ensure_workspace(mpq_plan_s* p, int64_t rows) {
   const int64_t mn = rows * p->n;
   mpq_status st = MPQ_OK;
   auto chk = [&](mpq_status s) { if (st == MPQ_OK) st = s; };
-  chk(dalloc(&w.R1, mn)); chk(dalloc(&w.X1, mn)); chk(dalloc(&w.R2, mn)); chk(dalloc(&w.A, mn));
+  chk(dalloc(&w.R1, mn)); chk(dalloc(&w.X1, mn)); chk(dalloc(&w.R2, mn));
+  if (st == MPQ_OK) chk(alloc_split(w.As, rows, std::max(p->n, p->r), true));
+  if (st == MPQ_OK)
+    chk(make_tmap_f16(&w.tm_an_hi, w.As.hi, round_up(p->n, 64), w.As.rows_pad, w.As.ld, 128));
+  if (st == MPQ_OK)
+    chk(make_tmap_f16(&w.tm_an_lo, w.As.lo, round_up(p->n, 64), w.As.rows_pad, w.As.ld, 128));
+  if (st == MPQ_OK)
+    chk(make_tmap_f16(&w.tm_ar_hi, w.As.hi, round_up(p->r, 64), w.As.rows_pad, w.As.ld, 128));
+  if (st == MPQ_OK)
+    chk(make_tmap_f16(&w.tm_ar_lo, w.As.lo, round_up(p->r, 64), w.As.rows_pad, w.As.ld, 128));
   chk(dalloc(&w.P, rows * p->r)); chk(dalloc(&w.idx, rows * p->B));
   chk(dalloc(&w.scale, rows)); chk(dalloc(&w.offset, rows));
   chk(dalloc(&w.gamma1, rows)); chk(dalloc(&w.gamma1_0, rows)); chk(dalloc(&w.gamma2, rows));
@@ -232,13 +265,16 @@ mpq_status run_linear(mpq_plan_s* p, const float* W, int64_t m, const float* R1,
                       double* beta_hat, int32_t* clamps, cudaStream_t st) {
   Workspace& w = p->ws;
   const int64_t n = p->n, r = p->r;
-  MPQ_TRY(launch_extrinsic_d2l(p, W, m, R1, gamma1, X1, vsum, gamma1_0, R2, w.A, gamma2, clamps, st));
-  MPQ_TRY(gemm_nt_f32(w.A, n, p->Vt32, n, w.P, r, m, r, n, st, "gemm_project"));
+  MPQ_TRY(launch_extrinsic_d2l(p, W, m, R1, gamma1, X1, vsum, gamma1_0, R2, &w.As, gamma2, clamps, st));
+  // p' = V^T (w - r2)
+  MPQ_TRY(gemm_tc(w.As, w.tm_an_hi, w.tm_an_lo, p->Vt_s, p->tm_vt_hi, p->tm_vt_lo, w.P, r, m, r, n,
+                  p->Vt_s.unscale_host, p->status, st, "gemm_project"));
   MPQ_TRY(launch_linear_rows(p, m, w.P, gamma2, gamma1_0, beta, gamma1_out, w.coef, w.kappa,
-                             alpha2, beta_hat, clamps, Uprime, st));
-  // G into X1: the denoiser output is consumed by now, A (= w - r2) is still needed
-  MPQ_TRY(gemm_nt_f32(w.P, r, p->V32, r, w.X1, n, m, n, r, st, "gemm_expand"));
-  return launch_extrinsic_l2d(p, W, m, R2, w.A, w.X1, w.coef, w.kappa, R1_out, xhat2, st);
+                             alpha2, beta_hat, clamps, Uprime, &w.As, st));
+  // G into X1: the denoiser output is consumed by now
+  MPQ_TRY(gemm_tc(w.As, w.tm_ar_hi, w.tm_ar_lo, p->V_s, p->tm_v_hi, p->tm_v_lo, w.X1, n, m, n, r,
+                  p->V_s.unscale_host, p->status, st, "gemm_expand"));
+  return launch_extrinsic_l2d(p, W, m, R2, w.X1, w.coef, w.kappa, R1_out, xhat2, st);
 }
 
 mpq_status run_cd(mpq_plan_s* p, const float* W, int64_t m, const float* scale,
@@ -246,8 +282,10 @@ mpq_status run_cd(mpq_plan_s* p, const float* W, int64_t m, const float* scale,
                   cudaStream_t st) {
   Workspace& w = p->ws;
   const int64_t n = p->n;
-  MPQ_TRY(launch_residual(p, W, m, scale, offset, idx, w.A, nullptr, st));
-  MPQ_TRY(gemm_nt_f32(w.A, n, p->H32, n, w.X1, n, m, n, n, st, "gemm_hessian"));  // h = H (w - x)
+  MPQ_TRY(launch_residual_split(p, W, m, scale, offset, idx, &w.As, nullptr, st));
+  // h = H (w - x)
+  MPQ_TRY(gemm_tc(w.As, w.tm_an_hi, w.tm_an_lo, p->H_s, p->tm_h_hi, p->tm_h_lo, w.X1, n, m, n, n,
+                  p->H_s.unscale_host, p->status, st, "gemm_hessian"));
   return launch_cd(p, W, m, scale, offset, idx, w.X1, sweeps, changes, st);
 }
 
@@ -256,9 +294,10 @@ mpq_status run_energy(mpq_plan_s* p, const float* W, int64_t m, const float* sca
                       cudaStream_t st) {
   Workspace& w = p->ws;
   const int64_t n = p->n, r = p->r;
-  MPQ_TRY(launch_residual(p, W, m, scale, offset, idx, w.A, w_hat, st));
+  MPQ_TRY(launch_residual_split(p, W, m, scale, offset, idx, &w.As, w_hat, st));
   if (!energy) return MPQ_OK;
-  MPQ_TRY(gemm_nt_f32(w.A, n, p->Vt32, n, w.P, r, m, r, n, st, "gemm_energy"));
+  MPQ_TRY(gemm_tc(w.As, w.tm_an_hi, w.tm_an_lo, p->Vt_s, p->tm_vt_hi, p->tm_vt_lo, w.P, r, m, r, n,
+                  p->Vt_s.unscale_host, p->status, st, "gemm_energy"));
   return launch_energy_rows(p, m, w.P, energy, st);
 }
 
@@ -333,6 +372,21 @@ mpq_status finish_plan(mpq_plan_s* p, cudaStream_t st) {
   MPQ_TRY(dalloc(&p->status, 1));
   MPQ_CUDA(cudaMemsetAsync(p->status, 0, sizeof(int), st));
   MPQ_TRY(build_hessian(p, st));
+  MPQ_TRY(alloc_split(p->Vt_s, r, n, false));
+  MPQ_TRY(alloc_split(p->V_s, n, r, false));
+  MPQ_TRY(alloc_split(p->H_s, n, n, false));
+  MPQ_TRY(split_global(p->Vt32, r, n, &p->Vt_s, st));
+  MPQ_TRY(split_global(p->V32, n, r, &p->V_s, st));
+  MPQ_TRY(split_global(p->H32, n, n, &p->H_s, st));
+  MPQ_CUDA(cudaMemcpyAsync(&p->Vt_s.unscale_host, p->Vt_s.unscale, sizeof(float), cudaMemcpyDeviceToHost, st));
+  MPQ_CUDA(cudaMemcpyAsync(&p->V_s.unscale_host, p->V_s.unscale, sizeof(float), cudaMemcpyDeviceToHost, st));
+  MPQ_CUDA(cudaMemcpyAsync(&p->H_s.unscale_host, p->H_s.unscale, sizeof(float), cudaMemcpyDeviceToHost, st));
+  MPQ_TRY(make_tmap_f16(&p->tm_vt_hi, p->Vt_s.hi, p->Vt_s.ld, p->Vt_s.rows_pad, p->Vt_s.ld, 256));
+  MPQ_TRY(make_tmap_f16(&p->tm_vt_lo, p->Vt_s.lo, p->Vt_s.ld, p->Vt_s.rows_pad, p->Vt_s.ld, 256));
+  MPQ_TRY(make_tmap_f16(&p->tm_v_hi, p->V_s.hi, p->V_s.ld, p->V_s.rows_pad, p->V_s.ld, 256));
+  MPQ_TRY(make_tmap_f16(&p->tm_v_lo, p->V_s.lo, p->V_s.ld, p->V_s.rows_pad, p->V_s.ld, 256));
+  MPQ_TRY(make_tmap_f16(&p->tm_h_hi, p->H_s.hi, p->H_s.ld, p->H_s.rows_pad, p->H_s.ld, 256));
+  MPQ_TRY(make_tmap_f16(&p->tm_h_lo, p->H_s.lo, p->H_s.ld, p->H_s.rows_pad, p->H_s.ld, 256));
   if (p->d == 8) {
     MPQ_TRY(dalloc(&p->cb_norm, p->K));
     MPQ_TRY(dalloc(&p->qtab, p->B * (int64_t)p->K));
@@ -348,6 +402,7 @@ void destroy_plan(mpq_plan_s* p) {
   free_workspace(p->ws);
   dfree(p->s64); dfree(p->V64); dfree(p->s32); dfree(p->V32); dfree(p->Vt32); dfree(p->H32);
   dfree(p->Hdiag); dfree(p->cb); dfree(p->cb_norm); dfree(p->qtab); dfree(p->status);
+  free_split(p->Vt_s); free_split(p->V_s); free_split(p->H_s);
   delete p;
 }
 

@@ -1,6 +1,8 @@
 // Internal declarations shared by the libmpq translation units.
 #pragma once
 
+#include <cuda.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -42,6 +44,20 @@ mpq_status check_launch(const char* name);
 // Device status word bits (set by kernels, read by mpq_plan_status).
 enum : int { STATUS_NONFINITE = 1, STATUS_TIMEOUT = 2, STATUS_BADINDEX = 4 };
 
+// A fp32 matrix stored for the tensor-core GEMM as fp16 hi/lo pairs of its
+// power-of-two-scaled values: x = (hi + lo) * unscale, rows padded to a
+// multiple of 256 and K to a multiple of 64 (zero padding), K contiguous.
+struct SplitOperand {
+  __half* hi = nullptr;
+  __half* lo = nullptr;
+  int64_t rows = 0, rows_pad = 0, K = 0, ld = 0;
+  float* row_unscale = nullptr;  // per-row 2^e (A operands), rows_pad floats
+  float* unscale = nullptr;      // device scalar 2^e (B operands)
+  float unscale_host = 1.0f;     // host copy of *unscale
+};
+
+inline int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
+
 // --------------------------------------------------------------- workspace --
 struct Workspace {
   int64_t rows = 0;       // rows the buffers are sized for
@@ -50,7 +66,10 @@ struct Workspace {
   float* R1 = nullptr;
   float* X1 = nullptr;
   float* R2 = nullptr;
-  float* A = nullptr;     // GEMM1 operand / GEMM2 output / CD gradient
+  // A operand of the tensor-core GEMMs (w - r2, the GEMM2 operand, residuals)
+  SplitOperand As;
+  CUtensorMap tm_an_hi, tm_an_lo;  // K = n view
+  CUtensorMap tm_ar_hi, tm_ar_lo;  // K = r view
   // m x r fp32
   float* P = nullptr;
   // m x B
@@ -89,6 +108,9 @@ struct mpq_plan_s {
   float* Vt32 = nullptr;   // r x n  (operand of p = V^T (w - r2))
   float* H32 = nullptr;    // n x n  H = V diag(s^2) V^T
   float* Hdiag = nullptr;  // n
+  // B operands of the tensor-core GEMMs
+  mpq::SplitOperand Vt_s, V_s, H_s;
+  CUtensorMap tm_vt_hi, tm_vt_lo, tm_v_hi, tm_v_lo, tm_h_hi, tm_h_lo;
   // vector codebook (d = 8)
   float* cb = nullptr;       // K x 8
   float* cb_norm = nullptr;  // K  |c|^2
@@ -117,18 +139,24 @@ mpq_status launch_denoise(const mpq_plan_s* p, const float* R1, const double* ga
                           const float* scale, const float* offset, int64_t m, const float* W,
                           const double* gamma1_0, float* xhat1, float* vblock, double* vsum,
                           uint16_t* idx, cudaStream_t st);
+// writes r2 and the A operand w - r2 (split, K = n)
 mpq_status launch_extrinsic_d2l(const mpq_plan_s* p, const float* W, int64_t m, const float* R1,
                                 const double* gamma1, const float* xhat1, const double* vsum,
-                                const double* gamma1_0, float* R2, float* A, double* gamma2,
-                                int32_t* clamps, cudaStream_t st);
-mpq_status launch_linear_rows(const mpq_plan_s* p, int64_t m, float* P, const double* gamma2,
-                              const double* gamma1_0, double* beta, double* gamma1_out,
-                              double* coef, double* kappa, double* alpha2, double* beta_hat,
-                              int32_t* clamps, float* Uprime, cudaStream_t st);
+                                const double* gamma1_0, float* R2, SplitOperand* As,
+                                double* gamma2, int32_t* clamps, cudaStream_t st);
+// reads p' from P, writes the GEMM2 A operand (split, K = r)
+mpq_status launch_linear_rows(const mpq_plan_s* p, int64_t m, const float* P,
+                              const double* gamma2, const double* gamma1_0, double* beta,
+                              double* gamma1_out, double* coef, double* kappa, double* alpha2,
+                              double* beta_hat, int32_t* clamps, float* Uprime, SplitOperand* As,
+                              cudaStream_t st);
 mpq_status launch_extrinsic_l2d(const mpq_plan_s* p, const float* W, int64_t m, const float* R2,
-                                const float* E, const float* G, const double* coef,
-                                const double* kappa, float* R1_out, float* xhat2,
-                                cudaStream_t st);
+                                const float* G, const double* coef, const double* kappa,
+                                float* R1_out, float* xhat2, cudaStream_t st);
+// residual w - w_hat as the split A operand (K = n); w_hat optional
+mpq_status launch_residual_split(const mpq_plan_s* p, const float* W, int64_t m,
+                                 const float* scale, const float* offset, const uint16_t* idx,
+                                 SplitOperand* As, float* w_hat, cudaStream_t st);
 mpq_status launch_residual(const mpq_plan_s* p, const float* W, int64_t m, const float* scale,
                            const float* offset, const uint16_t* idx, float* E, float* w_hat,
                            cudaStream_t st);
@@ -141,6 +169,16 @@ mpq_status launch_cd(const mpq_plan_s* p, const float* W, int64_t m, const float
                      const float* offset, uint16_t* idx, float* h, int32_t sweeps,
                      int32_t* changes, cudaStream_t st);
 mpq_status launch_check_finite(const float* x, int64_t count, int* status, cudaStream_t st);
+
+// tensor-core GEMM (gemm_tc.cu): C = diag(A.row_unscale) (A B^T) * b_scale
+mpq_status make_tmap_f16(CUtensorMap* tm, const void* base, int64_t inner, int64_t rows,
+                         int64_t ld_elems, int box_rows);
+mpq_status split_global(const float* src, int64_t rows, int64_t K, SplitOperand* dst,
+                        cudaStream_t st);
+mpq_status gemm_tc(const SplitOperand& A, const CUtensorMap& ta_hi, const CUtensorMap& ta_lo,
+                   const SplitOperand& B, const CUtensorMap& tb_hi, const CUtensorMap& tb_lo,
+                   float* C, int64_t ldc, int64_t M, int64_t N, int64_t K, float b_scale_host,
+                   int* status, cudaStream_t st, const char* tag);
 
 // plan-time builders
 mpq_status build_hessian(mpq_plan_s* p, cudaStream_t st);
