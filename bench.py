@@ -145,12 +145,18 @@ class ClockSampler:
 
 # ------------------------------------------------------- algorithmic work ---
 
+# fp32-accurate contractions are issued as fp16 tensor-core MMAs on hi/lo
+# splits: 3 passes per product (2 when the A operand is exact in fp16)
+GEMM_PASSES = {"gemm_project": 3, "gemm_expand": 3, "gemm_energy": 3, "gemm_hessian": 3,
+               "gemm_cd_update": 2}
+
+
 def kernel_work(name, m, n, r, d, K, L):
     """(bound, unit, work per launch) -- algorithmic flops or bytes."""
     if name in ("gemm_project", "gemm_energy", "gemm_expand"):
-        return "alu", "TFLOP/s", 2.0 * m * n * r
+        return "tensor", "TFLOP/s", 2.0 * m * n * r
     if name == "gemm_hessian":
-        return "alu", "TFLOP/s", 2.0 * m * n * n
+        return "tensor", "TFLOP/s", 2.0 * m * n * n
     if name == "k_denoise_scalar":      # read r1, write xhat1 (+ v per element)
         return "hbm", "GB/s", 8.0 * m * n
     if name == "k_extrinsic_d2l":        # read w, r1, xhat1; write r2, A
@@ -341,20 +347,27 @@ def run_mpq(args, world, rank, local):
     if wk:
         bound, unit, work = wk
         avg_s = kms / cnt / 1e3
+        passes = GEMM_PASSES.get(name, 1)
         if unit == "TFLOP/s":
             achieved = work / avg_s / 1e12
-            peak = FP32_ALU_PEAK_TFLOPS if bound == "alu" else peaks["bf16_tflops"]
+            # fp32-accurate work: the fp16 dense peak divided by the MMA passes
+            peak = FP32_ALU_PEAK_TFLOPS if bound == "alu" else peaks["bf16_tflops"] / passes
         elif unit == "GB/s":
             achieved = work / avg_s / 1e9
             peak = peaks["hbm_gbs"]
         else:
             achieved = work / avg_s / 1e9
             peak = 148 * 16 * 1.965  # MUFU ex2 per clock per SM x SMs x GHz -> Gexp/s
+        src = {"alu": "derived: 148 SMs x 128 FP32 lanes x 2 x 1965 MHz",
+               "tensor": f"{peak_src} bf16/fp16 dense {peaks['bf16_tflops']} TFLOP/s "
+                         f"(MEASURED_PEAKS.json) / {passes} fp16 MMA passes per fp32-accurate product",
+               }.get(bound, f"{peak_src} MEASURED_PEAKS.json")
         roof = {"bound": bound, "kernel": name, "achieved": achieved, "peak": peak, "unit": unit,
                 "frac": achieved / peak, "traffic": recorded_traffic(name, args.config),
-                "peak_source": ("derived: 148 SMs x 128 FP32 lanes x 2 x 1965 MHz"
-                                if bound == "alu" else f"{peak_src} MEASURED_PEAKS.json"),
-                "work_per_launch": work, "launches": cnt, "avg_launch_ms": kms / cnt}
+                "peak_source": src, "work_per_launch": work, "launches": cnt,
+                "avg_launch_ms": kms / cnt}
+        if bound == "tensor":
+            roof["tensor_pipe_frac"] = achieved * passes / peaks["bf16_tflops"]
     total_prof = sum(v[1] for v in prof.values())
     kernels = {k: {"launches": v[0], "ms": round(v[1], 4), "share": round(v[1] / total_prof, 4)}
                for k, v in sorted(prof.items(), key=lambda kv: -kv[1][1])}

@@ -129,8 +129,11 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
 __global__ void __launch_bounds__(TC_THREADS, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap ta_hi, const __grid_constant__ CUtensorMap ta_lo,
               const __grid_constant__ CUtensorMap tb_hi, const __grid_constant__ CUtensorMap tb_lo,
-              float* __restrict__ C, int64_t ldc, int M, int N, int K,
-              const float* __restrict__ row_scale, float b_scale, int* status) {
+              float* __restrict__ C, int64_t ldc, int M, int N, int K, int b_k0,
+              const float* __restrict__ row_scale, float b_scale, int accumulate, int a_exact,
+              const int* __restrict__ gate, int* status) {
+  // a zero gate means there is nothing to add: skip the whole tile
+  if (gate != nullptr && *gate == 0) return;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint64_t* full = (uint64_t*)(smem + STAGES * STAGE_BYTES);
@@ -171,11 +174,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         break;
       }
       uint8_t* base = smem + s * STAGE_BYTES;
-      mbar_expect_tx(&full[s], STAGE_BYTES);
+      mbar_expect_tx(&full[s], a_exact ? STAGE_BYTES - A_TILE : STAGE_BYTES);
       tma_load_2d(&ta_hi, &full[s], base, kt * BK, m0);
-      tma_load_2d(&ta_lo, &full[s], base + A_TILE, kt * BK, m0);
-      tma_load_2d(&tb_hi, &full[s], base + 2 * A_TILE, kt * BK, n0);
-      tma_load_2d(&tb_lo, &full[s], base + 2 * A_TILE + B_TILE, kt * BK, n0);
+      if (!a_exact) tma_load_2d(&ta_lo, &full[s], base + A_TILE, kt * BK, m0);
+      tma_load_2d(&tb_hi, &full[s], base + 2 * A_TILE, b_k0 + kt * BK, n0);
+      tma_load_2d(&tb_lo, &full[s], base + 2 * A_TILE + B_TILE, b_k0 + kt * BK, n0);
     }
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------- MMA issuer
@@ -199,7 +202,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const uint64_t dbh = sw128_desc(b_hi + off), dbl = sw128_desc(b_lo + off);
         umma_f16(tmem, dah, dbh, (kt | kk) != 0 ? 1u : 0u);
         umma_f16(tmem, dah, dbl, 1u);
-        umma_f16(tmem, dal, dbh, 1u);
+        if (!a_exact) umma_f16(tmem, dal, dbh, 1u);
       }
       umma_commit(&empty[s]);
     }
@@ -213,23 +216,35 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const int q = warp & 3;  // TMEM lane quadrant this warp may read
     const int row = m0 + q * 32 + lane;
     const float rs = (row < M) ? row_scale[row] * b_scale : 0.0f;
+    // the pipeline buffers are idle now: a 32 x 33 staging tile per warp turns
+    // the lane-per-row TMEM layout into row-contiguous, coalesced accesses
+    float* stage = reinterpret_cast<float*>(smem) + (warp - 2) * (32 * 33);
     for (int c0 = 0; c0 < BN && ok; c0 += 32) {
       if (n0 + c0 >= N) break;
       uint32_t v[32];
       tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c0, v);
-      if (row < M) {
-        float* crow = C + (int64_t)row * ldc + n0 + c0;
-        if (n0 + c0 + 32 <= N && (ldc & 3) == 0) {
 #pragma unroll
-          for (int j = 0; j < 32; j += 4) {
-            float4 o = make_float4(__uint_as_float(v[j]) * rs, __uint_as_float(v[j + 1]) * rs,
-                                   __uint_as_float(v[j + 2]) * rs, __uint_as_float(v[j + 3]) * rs);
-            *reinterpret_cast<float4*>(crow + j) = o;
-          }
+      for (int j = 0; j < 32; ++j) stage[lane * 33 + j] = __uint_as_float(v[j]) * rs;
+      __syncwarp();
+      const int col = n0 + c0 + lane;
+      const int nrow = min(32, M - (m0 + q * 32));
+      float* cbase = C + (int64_t)(m0 + q * 32) * ldc + col;
+      if (col < N) {
+        if (accumulate) {
+          float prev[32];
+#pragma unroll
+          for (int rr = 0; rr < 32; ++rr)  // all loads in flight before any store
+            prev[rr] = (rr < nrow) ? cbase[(int64_t)rr * ldc] : 0.0f;
+#pragma unroll
+          for (int rr = 0; rr < 32; ++rr)
+            if (rr < nrow) cbase[(int64_t)rr * ldc] = prev[rr] + stage[rr * 33 + lane];
         } else {
-          for (int j = 0; j < 32 && n0 + c0 + j < N; ++j) crow[j] = __uint_as_float(v[j]) * rs;
+#pragma unroll
+          for (int rr = 0; rr < 32; ++rr)
+            if (rr < nrow) cbase[(int64_t)rr * ldc] = stage[rr * 33 + lane];
         }
       }
+      __syncwarp();
     }
   }
   tc_fence_before();
@@ -333,9 +348,9 @@ mpq_status split_global(const float* src, int64_t rows, int64_t K, SplitOperand*
 mpq_status gemm_tc(const SplitOperand& A, const CUtensorMap& ta_hi, const CUtensorMap& ta_lo,
                    const SplitOperand& B, const CUtensorMap& tb_hi, const CUtensorMap& tb_lo,
                    float* C, int64_t ldc, int64_t M, int64_t N, int64_t K, float b_scale_host,
-                   int* status, cudaStream_t st, const char* tag) {
+                   int* status, cudaStream_t st, const char* tag, const GemmOpts& o) {
   if (M <= 0 || N <= 0) return MPQ_OK;
-  if (M > A.rows_pad || N > B.rows_pad || K > A.ld || K > B.ld)
+  if (M > A.rows_pad || N > B.rows_pad || K > A.ld || o.b_k0 + K > B.ld || o.b_k0 % 64)
     return fail(MPQ_ERR_INVALID_ARG, "gemm_tc: operand smaller than the problem");
   int dev = 0;
   MPQ_CUDA(cudaGetDevice(&dev));
@@ -346,9 +361,9 @@ mpq_status gemm_tc(const SplitOperand& A, const CUtensorMap& ta_hi, const CUtens
   dim3 grid((unsigned)cdiv(N, BN), (unsigned)cdiv(M, BM));
   {
     ProfScope ps_(tag, st);
-    k_gemm_tc<<<grid, TC_THREADS, SMEM_BYTES, st>>>(ta_hi, ta_lo, tb_hi, tb_lo, C, ldc, (int)M,
-                                                    (int)N, (int)K, A.row_unscale, b_scale_host,
-                                                    status);
+    k_gemm_tc<<<grid, TC_THREADS, SMEM_BYTES, st>>>(
+        ta_hi, ta_lo, tb_hi, tb_lo, C, ldc, (int)M, (int)N, (int)K, (int)o.b_k0, A.row_unscale,
+        b_scale_host, o.accumulate ? 1 : 0, o.a_exact ? 1 : 0, o.gate, status);
   }
   count_launch();
   return check_launch("k_gemm_tc");

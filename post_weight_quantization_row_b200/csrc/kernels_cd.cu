@@ -16,102 +16,114 @@ namespace mpq {
 namespace {
 
 // ------------------------------------------------------------------ d = 1 --
-// One warp per row, all sweeps in one launch.  Columns are visited in tiles
-// of CD1_TILE.  Inside a tile the gradient of the tile's own columns lives in
-// shared memory: the 32 lanes evaluate 32 consecutive columns against it;
-// the decisions are exact up to the first lane that accepts a change, so the
-// warp commits that change, updates the tile-local gradient with the row of
-// H and resumes right after it (identical to visiting columns one by one).
-// When the tile is done its changes are applied to the rest of h in one pass
-// (h_i -= sum_changes H[c, i] delta_c), so h is read and written once per
-// tile instead of once per change.
-constexpr int CD1_WARPS = 8;
-constexpr int CD1_TILE = 128;
+// A sweep visits the columns in tiles of CD_TILE.  For tile j the decide
+// kernel runs one warp per row on the tile's own gradient (shared memory):
+// the 32 lanes evaluate 32 consecutive columns, which is exact up to the
+// first lane that accepts a change; the warp commits that change, updates
+// the tile-local gradient with the row of H, and resumes right after it --
+// identical to visiting the columns one by one.  The tile's changes leave as
+// Delta/scale (small integers, exact in fp16) in the A operand of a tensor-
+// core update  h += (-scale) Delta H[tile, :]  over all columns, which also
+// reproduces the in-tile updates for the next tile and the next sweep.
+constexpr int CD1_WARPS = 16;
+constexpr int CD1_SMEM = (CD_TILE * CD_TILE + CD1_WARPS * CD_TILE) * 4 + CD1_WARPS * CD_TILE * 2;
 
 __global__ void __launch_bounds__(CD1_WARPS * 32)
-    k_cd_scalar(int64_t m, int64_t n, int L, const float* __restrict__ scale,
-                const float* __restrict__ H, const float* __restrict__ Hdiag,
-                uint16_t* __restrict__ idx, float* __restrict__ h, int sweeps,
-                int32_t* __restrict__ changes) {
-  __shared__ float s_h[CD1_WARPS][CD1_TILE];
-  __shared__ int s_col[CD1_WARPS][CD1_TILE];
-  __shared__ float s_dl[CD1_WARPS][CD1_TILE];
+    k_cd_tile_decide(int64_t m, int64_t n, int L, int64_t t0, int tw, int tile, int ntiles,
+                     const float* __restrict__ scale, const float* __restrict__ H,
+                     uint16_t* __restrict__ idx, const float* __restrict__ h, int sweeps, int sw,
+                     int32_t* __restrict__ changes, __half* __restrict__ dhi,
+                     __half* __restrict__ dlo, int64_t lda, float* __restrict__ d_unscale,
+                     int* __restrict__ tile_count) {
+  extern __shared__ float cd_smem[];
+  float* sH = cd_smem;                                  // H[tile, tile]
+  float* s_h_all = sH + CD_TILE * CD_TILE;              // per-warp gradient of the tile
+  uint16_t* s_i_all = (uint16_t*)(s_h_all + CD1_WARPS * CD_TILE);  // per-warp indices
+  for (int e = threadIdx.x; e < tw * tw; e += blockDim.x) {
+    const int i = e / tw, j = e - i * tw;
+    sH[i * CD_TILE + j] = H[(t0 + i) * n + t0 + j];
+  }
+  __syncthreads();
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int64_t row = (int64_t)blockIdx.x * CD1_WARPS + wid;
   if (row >= m) return;
+  __half* drow_hi = dhi + row * lda;
+  __half* drow_lo = dlo + row * lda;
+  for (int i = lane; i < CD_TILE; i += 32) {
+    drow_hi[i] = __float2half_rn(0.0f);
+    drow_lo[i] = __float2half_rn(0.0f);
+  }
   const float sc = scale[row];
-  float* hr = h + row * n;
-  uint16_t* ir = idx + row * n;
-  float* sh = s_h[wid];
-  int* scol = s_col[wid];
-  float* sdl = s_dl[wid];
-  for (int sw = 0; sw < sweeps; ++sw) {
-    int nchg = 0;
-    for (int64_t t0 = 0; t0 < n; t0 += CD1_TILE) {
-      const int tw = (int)((n - t0) < CD1_TILE ? (n - t0) : CD1_TILE);
-      for (int i = lane; i < tw; i += 32) sh[i] = hr[t0 + i];
-      __syncwarp();
-      int ntile = 0;  // changes in this tile
-      int c = 0;
-      while (c < tw) {
-        const int j = c + lane;
-        bool acc = false;
-        int kb = 0, kc = 0;
-        if (j < tw) {
-          const float hj = sh[j], g = Hdiag[t0 + j];
-          kc = ir[t0 + j];
-          float best = 0.0f;  // staying put
-          for (int k = 0; k < L; ++k) {
-            const float dl = sc * (float)(k - kc);
-            const float dE = dl * fmaf(0.5f * dl, g, -hj);
-            if (dE < best) {
-              best = dE;
-              kb = k;
-            }
-          }
-          acc = best < 0.0f;
-        }
-        const unsigned mask = __ballot_sync(0xffffffffu, acc);
-        if (mask == 0u) {
-          c += 32;
-          continue;
-        }
-        const int first = __ffs(mask) - 1;
-        const int jj = c + first;
-        const int knew = __shfl_sync(0xffffffffu, kb, first);
-        const int kold = __shfl_sync(0xffffffffu, kc, first);
-        const float dl = sc * (float)(knew - kold);
-        if (lane == first) {
-          ir[t0 + jj] = (uint16_t)knew;
-          scol[ntile] = (int)(t0 + jj);
-          sdl[ntile] = dl;
-        }
-        ++ntile;
-        const float* Hj = H + (t0 + jj) * n + t0;
-        for (int i = lane; i < tw; i += 32) sh[i] = fmaf(-Hj[i], dl, sh[i]);
-        __syncwarp();
-        c = jj + 1;
+  if (lane == 0) d_unscale[row] = -sc;
+  // a row stops after a sweep without change (its Delta row stays zero)
+  if (sw > 0 && changes[row * sweeps + sw - 1] == 0) return;
+  float* sh = s_h_all + wid * CD_TILE;
+  uint16_t* si = s_i_all + wid * CD_TILE;
+  const float* hr = h + row * n + t0;
+  uint16_t* ir = idx + row * n + t0;
+  for (int i = lane; i < tw; i += 32) {
+    sh[i] = hr[i];
+    si[i] = ir[i];
+  }
+  __syncwarp();
+  int ntile = 0;
+  int c = 0;
+  while (c < tw) {
+    const int j = c + lane;
+    bool acc = false;
+    int kb = 0, kc = 0;
+    if (j < tw) {
+      const float hj = sh[j], g = sH[j * CD_TILE + j];
+      kc = si[j];
+      // dE(k) = d (d g/2 - h), d = scale (k - kc), is a convex quadratic in k:
+      // its integer minimiser is one of the two levels around the continuous
+      // one (the grid ends when g <= 0), lowest index on ties
+      int k0, k1;
+      if (g > 0.0f) {
+        const float kcont = (float)kc + hj / (sc * g);
+        k0 = (int)fminf(fmaxf(floorf(kcont), 0.0f), (float)(L - 1));
+        k1 = min(k0 + 1, L - 1);
+      } else {
+        k0 = 0;
+        k1 = L - 1;
       }
-      __syncwarp();
-      nchg += ntile;
-      // write the tile back and apply its changes to every other column
-      for (int i = lane; i < tw; i += 32) hr[t0 + i] = sh[i];
-      if (ntile > 0) {
-        for (int64_t i = lane; i < n; i += 32) {
-          if (i >= t0 && i < t0 + tw) continue;
-          float a = hr[i];
-          for (int q = 0; q < ntile; ++q) a = fmaf(-H[(int64_t)scol[q] * n + i], sdl[q], a);
-          hr[i] = a;
-        }
+      const float d0 = sc * (float)(k0 - kc), d1 = sc * (float)(k1 - kc);
+      const float e0 = d0 * fmaf(0.5f * d0, g, -hj), e1 = d1 * fmaf(0.5f * d1, g, -hj);
+      float best = 0.0f;  // staying put
+      if (e0 < best) {
+        best = e0;
+        kb = k0;
       }
-      __syncwarp();
+      if (e1 < best) {
+        best = e1;
+        kb = k1;
+      }
+      acc = best < 0.0f;
     }
-    if (lane == 0 && changes) changes[row * sweeps + sw] = nchg;
-    if (nchg == 0) {
-      if (lane == 0 && changes)
-        for (int s2 = sw + 1; s2 < sweeps; ++s2) changes[row * sweeps + s2] = 0;
-      break;
+    const unsigned mask = __ballot_sync(0xffffffffu, acc);
+    if (mask == 0u) {
+      c += 32;
+      continue;
     }
+    const int first = __ffs(mask) - 1;
+    const int jj = c + first;
+    const int knew = __shfl_sync(0xffffffffu, kb, first);
+    const int kold = __shfl_sync(0xffffffffu, kc, first);
+    const float dl = sc * (float)(knew - kold);
+    if (lane == first) {
+      ir[jj] = (uint16_t)knew;
+      si[jj] = (uint16_t)knew;
+      drow_hi[jj] = __float2half_rn((float)(knew - kold));
+    }
+    ++ntile;
+    const float* Hj = sH + jj * CD_TILE;
+    for (int i = lane; i < tw; i += 32) sh[i] = fmaf(-Hj[i], dl, sh[i]);
+    __syncwarp();
+    c = jj + 1;
+  }
+  if (lane == 0 && ntile > 0) {
+    changes[row * sweeps + sw] += ntile;
+    tile_count[sw * ntiles + tile] = 1;  // gate of the update: some row changed
   }
 }
 
@@ -289,23 +301,44 @@ __global__ void __launch_bounds__(256)
 
 }  // namespace
 
-mpq_status launch_cd(const mpq_plan_s* p, const float* W, int64_t m, const float* scale,
+mpq_status launch_cd(mpq_plan_s* p, const float* W, int64_t m, const float* scale,
                      const float* offset, uint16_t* idx, float* h, int32_t sweeps,
                      int32_t* changes, cudaStream_t st) {
   (void)W;
   (void)offset;
   if (m <= 0 || sweeps <= 0) return MPQ_OK;
+  if (changes == nullptr) return fail(MPQ_ERR_INVALID_ARG, "CD needs a changes buffer");
+  MPQ_CUDA(cudaMemsetAsync(changes, 0, sizeof(int32_t) * m * sweeps, st));
   if (p->d == 1) {
-    {
-      ProfScope ps_("k_cd_scalar", st);
-      k_cd_scalar<<<(unsigned)cdiv(m, CD1_WARPS), CD1_WARPS * 32, 0, st>>>(
-          m, p->n, p->K, scale, p->H32, p->Hdiag, idx, h, sweeps, changes);
+    Workspace& w = p->ws;
+    const int64_t n = p->n;
+    const int nt = (int)cdiv(n, CD_TILE);
+    MPQ_CUDA(cudaFuncSetAttribute(k_cd_tile_decide, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  CD1_SMEM));
+    MPQ_CUDA(cudaMemsetAsync(w.tile_count, 0, sizeof(int) * sweeps * nt, st));
+    for (int sw = 0; sw < sweeps; ++sw) {
+      for (int j = 0; j < nt; ++j) {
+        const int64_t t0 = (int64_t)j * CD_TILE;
+        const int tw = (int)std::min<int64_t>(CD_TILE, n - t0);
+        {
+          ProfScope ps_("k_cd_tile_decide", st);
+          k_cd_tile_decide<<<(unsigned)cdiv(m, CD1_WARPS), CD1_WARPS * 32, CD1_SMEM, st>>>(
+              m, n, p->K, t0, tw, j, nt, scale, p->H32, idx, h, sweeps, sw, changes, w.As.hi,
+              w.As.lo, w.As.ld, w.As.row_unscale, w.tile_count);
+        }
+        count_launch();
+        MPQ_TRY(check_launch("k_cd_tile_decide"));
+        GemmOpts o;
+        o.b_k0 = t0;
+        o.accumulate = true;
+        o.a_exact = true;
+        o.gate = w.tile_count + sw * nt + j;
+        MPQ_TRY(gemm_tc(w.As, w.tm_at_hi, w.tm_at_lo, p->H_s, p->tm_h_hi, p->tm_h_lo, h, n, m, n,
+                        tw, p->H_s.unscale_host, p->status, st, "gemm_cd_update", o));
+      }
     }
-    count_launch();
-    return check_launch("k_cd_scalar");
+    return MPQ_OK;
   }
-  // d = 8 needs the change counters for its early stop
-  if (changes == nullptr) return fail(MPQ_ERR_INVALID_ARG, "vector CD needs a changes buffer");
   const int nchunks = (int)cdiv(p->K, CD8_CHUNK);
   float* part_val = nullptr;
   int* part_idx = nullptr;

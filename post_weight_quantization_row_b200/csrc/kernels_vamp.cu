@@ -197,41 +197,65 @@ __global__ void __launch_bounds__(ROW_THREADS)
   __shared__ double ds[33];
   const int64_t row = blockIdx.x;
   const float sc = scale[row], off = offset[row];
-  const double dsc = sc, doff = off;
+  const double dsc = sc, doff = off, inv_dsc = 1.0 / dsc;
   const double sc2 = dsc * dsc;
   const double g = fmin(gamma1[row] * sc2, 1e30);
   const bool anchored = (W != nullptr);
   const double ga = anchored ? fmin(gamma1_0[row] * inv_tau2 * sc2, 1e30) : 0.0;
   const double geff = g + ga;
+  const float decay = (float)exp(-geff);
   const double Lm1 = (double)(L - 1);
   double acc = 0.0;
   for (int64_t j = threadIdx.x; j < n; j += blockDim.x) {
     const int64_t o = row * n + j;
-    // level coordinate and logit arguments in fp64: the fp32 inputs are
-    // exact there, so only the exponentials and sums round in fp32
-    double t = ((double)R1[o] - doff) / dsc;
+    // the level coordinate is formed in fp64 (the fp32 inputs are exact
+    // there) so that its offset from the nearest level, |dt| <= 1/2 inside
+    // the grid, is accurate to fp32 rounding; the 16 logits then only lose
+    // fp32 relative precision of their own size
+    double t = ((double)R1[o] - doff) * inv_dsc;
     if (anchored) {
-      const double tw = ((double)W[o] - doff) / dsc;
+      const double tw = ((double)W[o] - doff) * inv_dsc;
       t = (g * t + ga * tw) / geff;
     }
     // argmax of -(k - t)^2, lowest k on ties
     const double ks = fmin(fmax(ceil(t - 0.5), 0.0), Lm1);
-    const double dt = t - ks;
-    float S0 = 0.0f, S1 = 0.0f, S2 = 0.0f;
-    for (int k = 0; k < L; ++k) {
-      const double dk = (double)k - ks;
-      const float e = __expf((float)(-0.5 * geff * dk * (dk - 2.0 * dt)));
-      const float dkf = (float)dk;
-      S0 += e;
-      S1 = fmaf(e, dkf, S1);
-      S2 = fmaf(e * dkf, dkf, S2);
+    const double dt = t - ks;  // |dt| <= 1/2 inside the grid
+    const int kstar = (int)ks;
+    // q_k / q_k* = exp(-geff/2 ((k - t)^2 - (k* - t)^2)).  On a uniform grid
+    // consecutive ratios differ by the constant factor exp(-geff), so the L
+    // weights follow from three exponentials and a product recurrence
+    // (relative error ~|k - k*| ulp) instead of L exponentials.
+    const float up0 = __expf(-(float)(geff * (0.5 - dt)));  // q_{k*+1}/q_{k*} <= 1
+    const float dn0 = __expf(-(float)(geff * (0.5 + dt)));  // q_{k*-1}/q_{k*} <= 1
+    float S0 = 1.0f, S1 = 0.0f, S2 = 0.0f;
+    {
+      float e = 1.0f, ratio = up0, dk = 0.0f;
+      for (int k = kstar + 1; k < L; ++k) {
+        e *= ratio;
+        ratio *= decay;
+        dk += 1.0f;
+        S0 += e;
+        S1 = fmaf(e, dk, S1);
+        S2 = fmaf(e * dk, dk, S2);
+      }
+    }
+    {
+      float e = 1.0f, ratio = dn0, dk = 0.0f;
+      for (int k = kstar - 1; k >= 0; --k) {
+        e *= ratio;
+        ratio *= decay;
+        dk -= 1.0f;
+        S0 += e;
+        S1 = fmaf(e, dk, S1);
+        S2 = fmaf(e * dk, dk, S2);
+      }
     }
     const float m1 = S1 / S0;
     const float var = fmaxf(S2 / S0 - m1 * m1, 0.0f);
-    xhat[o] = (float)(dsc * (ks + (double)m1) + doff);
+    xhat[o] = fmaf(sc, (float)kstar + m1, off);
     const float v = (float)(sc2 * (double)var);
     if (vblock) vblock[o] = v;
-    if (idx) idx[o] = (uint16_t)ks;
+    if (idx) idx[o] = (uint16_t)kstar;
     acc += (double)v;
   }
   acc = block_sum(acc, ds);
@@ -437,7 +461,7 @@ __global__ void __launch_bounds__(ROW_THREADS)
 //   r = n: -F p'                 -> G = xhat2 - w  (V V^T = I), which avoids
 //          forming r2 + V V^T (w - r2) when r2 is far from w.
 __global__ void __launch_bounds__(ROW_THREADS)
-    k_linear_rows(float* __restrict__ P, int64_t n, int64_t r, const double* __restrict__ s,
+    k_linear_rows(float* __restrict__ P, int64_t n, int64_t r, const float* __restrict__ s32,
                   const double* __restrict__ gamma2, const double* __restrict__ gamma1_0,
                   double* __restrict__ beta, double damping, double glo, double ghi,
                   double amin, double amax, int full_rank, double* __restrict__ gamma1_out,
@@ -452,16 +476,19 @@ __global__ void __launch_bounds__(ROW_THREADS)
   const double b = beta[row], g2 = gamma2[row];
   double a2s = 0.0, bs = 0.0;
   float mx = 0.0f;
+  const float bf = (float)b, g2f = (float)g2;
   for (int64_t l = threadIdx.x; l < r; l += blockDim.x) {
-    const double sl = s[l];
-    const double pl = (double)P[row * r + l];
-    const double u = sl * pl;
-    const double den = b * sl * sl + g2;
-    const double f = g2 / den;
-    a2s += f;
-    bs += f * f * u * u + sl * sl / den;
-    if (Uprime) Uprime[row * r + l] = (float)((1.0 - f) * pl);
-    const float q = (float)(full_rank ? -f * pl : (1.0 - f) * pl);
+    // per element in fp32 (relative error ~1e-7), sums in fp64
+    const float sl = s32[l];
+    const float pl = P[row * r + l];
+    const float u = sl * pl;
+    const float den = fmaf(bf * sl, sl, g2f);
+    const float inv = 1.0f / den;
+    const float f = g2f * inv;
+    a2s += (double)f;
+    bs += (double)(f * f * u * u) + (double)(sl * sl * inv);
+    if (Uprime) Uprime[row * r + l] = (1.0f - f) * pl;
+    const float q = full_rank ? -f * pl : (1.0f - f) * pl;
     P[row * r + l] = q;
     mx = fmaxf(mx, fabsf(q));
   }
@@ -730,7 +757,7 @@ mpq_status launch_linear_rows(const mpq_plan_s* p, int64_t m, const float* P,
   {
     ProfScope ps_("k_linear_rows", st);
     k_linear_rows<<<rows_grid(m), ROW_THREADS, 0, st>>>(
-        const_cast<float*>(P), p->n, p->r, p->s64, gamma2, gamma1_0, beta, q.damping,
+        const_cast<float*>(P), p->n, p->r, p->s32, gamma2, gamma1_0, beta, q.damping,
         q.gamma_lo_rel, q.gamma_hi_rel, q.alpha_min, q.alpha_max, p->r == p->n ? 1 : 0,
         gamma1_out, coef, kappa, alpha2, beta_hat, clamps, Uprime, As->hi, As->lo, As->ld,
         round_up(p->r, 64), As->row_unscale);

@@ -178,6 +178,7 @@ mpq_status alloc_split(SplitOperand& s, int64_t rows, int64_t K, bool per_row) {
 void free_workspace(Workspace& w) {
   dfree(w.R1); dfree(w.X1); dfree(w.R2); dfree(w.P); dfree(w.idx);
   free_split(w.As);
+  dfree(w.tile_count);
   dfree(w.scale); dfree(w.offset); dfree(w.gamma1); dfree(w.gamma1_0); dfree(w.gamma2);
   dfree(w.beta); dfree(w.vsum); dfree(w.coef); dfree(w.kappa); dfree(w.clamps); dfree(w.W); dfree(w.w_hat);
   dfree(w.energy); dfree(w.idx_stage);
@@ -188,7 +189,8 @@ void free_workspace(Workspace& w) {
 constexpr int MAX_SWEEPS = 64;
 
 int64_t ws_bytes_per_row(const mpq_plan_s* p) {
-  return 3 * p->n * 4 + p->r * 4 + 4 * round_up(std::max(p->n, p->r), 64) + p->B * 2 + 3 * 4 +
+  return 3 * p->n * 4 + p->r * 4 +
+         4 * round_up(std::max<int64_t>(std::max(p->n, p->r), CD_TILE), 64) + p->B * 2 + 3 * 4 +
          8 * 8 + 4 + MAX_SWEEPS * 4;
 }
 
@@ -205,7 +207,9 @@ mpq_status ensure_workspace(mpq_plan_s* p, int64_t rows) {
   mpq_status st = MPQ_OK;
   auto chk = [&](mpq_status s) { if (st == MPQ_OK) st = s; };
   chk(dalloc(&w.R1, mn)); chk(dalloc(&w.X1, mn)); chk(dalloc(&w.R2, mn));
-  if (st == MPQ_OK) chk(alloc_split(w.As, rows, std::max(p->n, p->r), true));
+  if (st == MPQ_OK)
+    chk(alloc_split(w.As, rows, std::max<int64_t>(std::max(p->n, p->r), CD_TILE), true));
+  chk(dalloc(&w.tile_count, (int64_t)MAX_SWEEPS * cdiv(p->n, CD_TILE)));
   if (st == MPQ_OK)
     chk(make_tmap_f16(&w.tm_an_hi, w.As.hi, round_up(p->n, 64), w.As.rows_pad, w.As.ld, 128));
   if (st == MPQ_OK)
@@ -214,6 +218,10 @@ mpq_status ensure_workspace(mpq_plan_s* p, int64_t rows) {
     chk(make_tmap_f16(&w.tm_ar_hi, w.As.hi, round_up(p->r, 64), w.As.rows_pad, w.As.ld, 128));
   if (st == MPQ_OK)
     chk(make_tmap_f16(&w.tm_ar_lo, w.As.lo, round_up(p->r, 64), w.As.rows_pad, w.As.ld, 128));
+  if (st == MPQ_OK)
+    chk(make_tmap_f16(&w.tm_at_hi, w.As.hi, CD_TILE, w.As.rows_pad, w.As.ld, 128));
+  if (st == MPQ_OK)
+    chk(make_tmap_f16(&w.tm_at_lo, w.As.lo, CD_TILE, w.As.rows_pad, w.As.ld, 128));
   chk(dalloc(&w.P, rows * p->r)); chk(dalloc(&w.idx, rows * p->B));
   chk(dalloc(&w.scale, rows)); chk(dalloc(&w.offset, rows));
   chk(dalloc(&w.gamma1, rows)); chk(dalloc(&w.gamma1_0, rows)); chk(dalloc(&w.gamma2, rows));

@@ -70,6 +70,8 @@ struct Workspace {
   SplitOperand As;
   CUtensorMap tm_an_hi, tm_an_lo;  // K = n view
   CUtensorMap tm_ar_hi, tm_ar_lo;  // K = r view
+  CUtensorMap tm_at_hi, tm_at_lo;  // K = CD tile view
+  int* tile_count = nullptr;       // CD: changes per (sweep, tile)
   // m x r fp32
   float* P = nullptr;
   // m x B
@@ -165,9 +167,11 @@ mpq_status launch_residual(const mpq_plan_s* p, const float* W, int64_t m, const
 mpq_status launch_sanitize_idx(const mpq_plan_s* p, uint16_t* idx, int64_t count, cudaStream_t st);
 mpq_status launch_energy_rows(const mpq_plan_s* p, int64_t m, const float* P, float* energy,
                               cudaStream_t st);
-mpq_status launch_cd(const mpq_plan_s* p, const float* W, int64_t m, const float* scale,
+// CD sweeps; h (m x n) holds H (w - x) on entry and is updated in place
+mpq_status launch_cd(mpq_plan_s* p, const float* W, int64_t m, const float* scale,
                      const float* offset, uint16_t* idx, float* h, int32_t sweeps,
                      int32_t* changes, cudaStream_t st);
+constexpr int CD_TILE = 128;  // columns per scalar CD tile (multiple of 64)
 mpq_status launch_check_finite(const float* x, int64_t count, int* status, cudaStream_t st);
 
 // tensor-core GEMM (gemm_tc.cu): C = diag(A.row_unscale) (A B^T) * b_scale
@@ -175,10 +179,16 @@ mpq_status make_tmap_f16(CUtensorMap* tm, const void* base, int64_t inner, int64
                          int64_t ld_elems, int box_rows);
 mpq_status split_global(const float* src, int64_t rows, int64_t K, SplitOperand* dst,
                         cudaStream_t st);
+struct GemmOpts {
+  int64_t b_k0 = 0;         // K offset into B (a multiple of 64)
+  bool accumulate = false;  // C += result instead of C = result
+  bool a_exact = false;     // A_lo is zero: skip its load and product
+  const int* gate = nullptr;  // device int; 0 -> the launch does nothing
+};
 mpq_status gemm_tc(const SplitOperand& A, const CUtensorMap& ta_hi, const CUtensorMap& ta_lo,
                    const SplitOperand& B, const CUtensorMap& tb_hi, const CUtensorMap& tb_lo,
                    float* C, int64_t ldc, int64_t M, int64_t N, int64_t K, float b_scale_host,
-                   int* status, cudaStream_t st, const char* tag);
+                   int* status, cudaStream_t st, const char* tag, const GemmOpts& o = GemmOpts());
 
 // plan-time builders
 mpq_status build_hessian(mpq_plan_s* p, cudaStream_t st);
