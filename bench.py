@@ -170,10 +170,15 @@ def kernel_work(name, m, n, r, d, K, L):
     return None
 
 
-def source_sha():
-    h = hashlib.sha256()
+KERNEL_SOURCE = {"gemm": "gemm_tc.cu", "k_cd": "kernels_cd.cu", "k_": "kernels_vamp.cu"}
+
+
+def source_sha(kernel):
+    """Hash of the source file that defines `kernel` plus the shared header."""
     csrc = os.path.join(ROOT, "post_weight_quantization_row_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    fname = next(v for k, v in KERNEL_SOURCE.items() if kernel.startswith(k))
+    h = hashlib.sha256()
+    for f in (fname, "mpq_internal.cuh"):
         h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 
@@ -184,7 +189,7 @@ def recorded_traffic(kernel, workload):
     path = os.path.join(ROOT, "profiles", "traffic.txt")
     if not os.path.exists(path):
         return None
-    sha = source_sha()
+    sha = source_sha(kernel)
     for line in open(path):
         parts = line.split()
         if len(parts) == 4 and not line.startswith("#") and parts[0] == kernel and parts[1] == workload:
