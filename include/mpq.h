@@ -82,7 +82,7 @@ typedef struct {
   double gamma_lo_rel;    /* extrinsic precisions are clipped into        */
   double gamma_hi_rel;    /*   [lo, hi] * gamma1_0 (defaults 1e-10, 1e10) */
   double alpha_min;       /* mean divergences are clipped into            */
-  double alpha_max;       /*   [alpha_min, alpha_max] (1e-10, 1 - 1e-5)   */
+  double alpha_max;       /*   [alpha_min, alpha_max] (1e-10, 0.99)       */
 } mpq_params;
 
 /* Fill `p` with the defaults above for block size d and codebook size K. */

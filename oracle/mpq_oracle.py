@@ -26,7 +26,7 @@ Readings where the pages are silent (each also listed in the design doc):
       Finite tau adds the anchor log rho_b(c) = -(gamma1_0/tau^2)/2 |c-w_b|^2.
   R5  extrinsic updates use the divergence form (identical to the pages'
       eta form when nothing is clipped): mean divergences alpha are clipped
-      into [1e-10, 1 - 1e-5] before the extrinsic mean is formed, and the
+      into [1e-10, 0.99] before the extrinsic mean is formed, and the
       extrinsic precisions into [1e-10, 1e10] * gamma1_0.
   R6  alpha2 counts null-space directions (n - r) as passing r2 through.
   R7  damping acts on beta (not 1/beta): beta <- (1-rho) beta + rho beta_hat.
@@ -47,7 +47,7 @@ import numpy as np
 GAMMA_LO_REL = 1e-10
 GAMMA_HI_REL = 1e10
 ALPHA_MIN = 1e-10
-ALPHA_MAX = 1.0 - 1e-5
+ALPHA_MAX = 0.99
 
 
 # ----------------------------------------------------------------------------

@@ -78,6 +78,17 @@ __device__ __forceinline__ void tma_load_2d(const CUtensorMap* tm, uint64_t* bar
       : "memory");
 }
 
+// reduce-add of a 32 x 32 fp32 box (128B-swizzled in shared memory) into global
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* tm, const void* src, int c0,
+                                                  int c1) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group"
+      " [%0, {%2, %3}], [%1];" ::"l"((uint64_t)tm),
+      "r"(smem_u32(src)), "r"(c0), "r"(c1)
+      : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
@@ -131,7 +142,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
               const __grid_constant__ CUtensorMap tb_hi, const __grid_constant__ CUtensorMap tb_lo,
               float* __restrict__ C, int64_t ldc, int M, int N, int K, int b_k0,
               const float* __restrict__ row_scale, float b_scale, int accumulate, int a_exact,
-              const int* __restrict__ gate, int* status) {
+              const int* __restrict__ gate, const __grid_constant__ CUtensorMap tc_out,
+              int use_reduce, int* status) {
   // a zero gate means there is nothing to add: skip the whole tile
   if (gate != nullptr && *gate == 0) return;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -216,6 +228,33 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const int q = warp & 3;  // TMEM lane quadrant this warp may read
     const int row = m0 + q * 32 + lane;
     const float rs = (row < M) ? row_scale[row] * b_scale : 0.0f;
+    if (use_reduce) {
+      // accumulate through the TMA unit: each warp stages its 32 x 32 block in
+      // a 128B-swizzled buffer (two per warp, alternating) and issues a
+      // tensor reduce-add into C; L2 performs the read-modify-write
+      uint8_t* stg0 = smem + (warp - 2) * 8192;
+      int nb = 0;
+      for (int c0 = 0; c0 < BN && ok; c0 += 32) {
+        if (n0 + c0 >= N) break;
+        uint32_t v[32];
+        tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c0, v);
+        uint8_t* stg = stg0 + (nb & 1) * 4096;
+        if (lane == 0 && nb >= 2) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          float4 o = make_float4(__uint_as_float(v[4 * k]) * rs, __uint_as_float(v[4 * k + 1]) * rs,
+                                 __uint_as_float(v[4 * k + 2]) * rs, __uint_as_float(v[4 * k + 3]) * rs);
+          *reinterpret_cast<float4*>(stg + lane * 128 + ((k ^ (lane & 7)) * 16)) = o;
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) tma_reduce_add_2d(&tc_out, stg, n0 + c0, m0 + q * 32);
+        ++nb;
+      }
+      if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+      __syncwarp();
+    } else {
     // the pipeline buffers are idle now: a 32 x 33 staging tile per warp turns
     // the lane-per-row TMEM layout into row-contiguous, coalesced accesses
     float* stage = reinterpret_cast<float*>(smem) + (warp - 2) * (32 * 33);
@@ -245,6 +284,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
       }
       __syncwarp();
+    }
     }
   }
   tc_fence_before();
@@ -325,6 +365,23 @@ mpq_status make_tmap_f16(CUtensorMap* tm, const void* base, int64_t inner, int64
   return MPQ_OK;
 }
 
+mpq_status make_tmap_f32_out(CUtensorMap* tm, const float* base, int64_t cols, int64_t rows,
+                             int64_t ld_elems) {
+  MPQ_TRY(get_encoder());
+  if (((uintptr_t)base & 127) || (ld_elems * 4) % 16 || cols < 32 || rows < 32)
+    return fail(MPQ_ERR_INVALID_ARG, "tensor map: misaligned output");
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(ld_elems * 4)};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims,
+                        strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(MPQ_ERR_CUDA, "cuTensorMapEncodeTiled (fp32) failed with code " + std::to_string((int)r));
+  return MPQ_OK;
+}
+
 mpq_status split_global(const float* src, int64_t rows, int64_t K, SplitOperand* dst,
                         cudaStream_t st) {
   unsigned* amax = nullptr;
@@ -358,12 +415,16 @@ mpq_status gemm_tc(const SplitOperand& A, const CUtensorMap& ta_hi, const CUtens
     MPQ_CUDA(cudaFuncSetAttribute(k_gemm_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES));
     g_smem_attr_set[dev] = true;
   }
+  if (o.c_reduce && !o.accumulate)
+    return fail(MPQ_ERR_INVALID_ARG, "gemm_tc: reduce output needs accumulate");
   dim3 grid((unsigned)cdiv(N, BN), (unsigned)cdiv(M, BM));
+  const CUtensorMap& cmap = o.c_reduce ? *o.c_reduce : tb_hi;  // unused unless reducing
   {
     ProfScope ps_(tag, st);
     k_gemm_tc<<<grid, TC_THREADS, SMEM_BYTES, st>>>(
         ta_hi, ta_lo, tb_hi, tb_lo, C, ldc, (int)M, (int)N, (int)K, (int)o.b_k0, A.row_unscale,
-        b_scale_host, o.accumulate ? 1 : 0, o.a_exact ? 1 : 0, o.gate, status);
+        b_scale_host, o.accumulate ? 1 : 0, o.a_exact ? 1 : 0, o.gate, cmap, o.c_reduce ? 1 : 0,
+        status);
   }
   count_launch();
   return check_launch("k_gemm_tc");

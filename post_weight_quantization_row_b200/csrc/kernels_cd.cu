@@ -31,7 +31,8 @@ constexpr int CD1_SMEM = (CD_TILE * CD_TILE + CD1_WARPS * CD_TILE) * 4 + CD1_WAR
 __global__ void __launch_bounds__(CD1_WARPS * 32)
     k_cd_tile_decide(int64_t m, int64_t n, int L, int64_t t0, int tw, int tile, int ntiles,
                      const float* __restrict__ scale, const float* __restrict__ H,
-                     uint16_t* __restrict__ idx, const float* __restrict__ h, int sweeps, int sw,
+                     uint16_t* __restrict__ idx, const float* __restrict__ h, int64_t ldh,
+                     int sweeps, int sw,
                      int32_t* __restrict__ changes, __half* __restrict__ dhi,
                      __half* __restrict__ dlo, int64_t lda, float* __restrict__ d_unscale,
                      int* __restrict__ tile_count) {
@@ -39,9 +40,21 @@ __global__ void __launch_bounds__(CD1_WARPS * 32)
   float* sH = cd_smem;                                  // H[tile, tile]
   float* s_h_all = sH + CD_TILE * CD_TILE;              // per-warp gradient of the tile
   uint16_t* s_i_all = (uint16_t*)(s_h_all + CD1_WARPS * CD_TILE);  // per-warp indices
-  for (int e = threadIdx.x; e < tw * tw; e += blockDim.x) {
-    const int i = e / tw, j = e - i * tw;
-    sH[i * CD_TILE + j] = H[(t0 + i) * n + t0 + j];
+  // H[tile, tile] into shared memory: each warp copies rows with coalesced
+  // loads, all of a row's loads in flight together
+  {
+    const int wid0 = threadIdx.x >> 5, lane0 = threadIdx.x & 31;
+    for (int i = wid0; i < tw; i += CD1_WARPS) {
+      const float* src = H + (t0 + i) * n + t0;
+      float v[CD_TILE / 32];
+#pragma unroll
+      for (int q = 0; q < CD_TILE / 32; ++q) {
+        const int j = lane0 + 32 * q;
+        v[q] = (j < tw) ? src[j] : 0.0f;
+      }
+#pragma unroll
+      for (int q = 0; q < CD_TILE / 32; ++q) sH[i * CD_TILE + lane0 + 32 * q] = v[q];
+    }
   }
   __syncthreads();
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
@@ -59,7 +72,7 @@ __global__ void __launch_bounds__(CD1_WARPS * 32)
   if (sw > 0 && changes[row * sweeps + sw - 1] == 0) return;
   float* sh = s_h_all + wid * CD_TILE;
   uint16_t* si = s_i_all + wid * CD_TILE;
-  const float* hr = h + row * n + t0;
+  const float* hr = h + row * ldh + t0;
   uint16_t* ir = idx + row * n + t0;
   for (int i = lane; i < tw; i += 32) {
     sh[i] = hr[i];
@@ -163,7 +176,7 @@ __global__ void __launch_bounds__(256)
     k_cd_vec_eval(int64_t m, int64_t n, int K, int64_t b, const float* __restrict__ cb,
                   const float* __restrict__ qtab, const float* __restrict__ H,
                   const float* __restrict__ scale, const uint16_t* __restrict__ idx,
-                  const float* __restrict__ h, int sweeps, int sw,
+                  const float* __restrict__ h, int64_t ldh, int sweeps, int sw,
                   const int32_t* __restrict__ changes, float* __restrict__ part_val,
                   int* __restrict__ part_idx, int nchunks) {
   __shared__ float scb[CD8_CHUNK][8];
@@ -181,7 +194,7 @@ __global__ void __launch_bounds__(256)
     const bool act = row < m && row_active(changes, row, sweeps, sw);
     if (act) {
       float g[8];
-      block_gradient(H, n, h + row * n, cb, idx[row * B + b], scale[row], b, g);
+      block_gradient(H, n, h + row * ldh, cb, idx[row * B + b], scale[row], b, g);
 #pragma unroll
       for (int i = 0; i < 8; ++i) sg[threadIdx.x][i] = g[i];
     } else {
@@ -245,7 +258,8 @@ __global__ void __launch_bounds__(256)
     k_cd_vec_apply(int64_t m, int64_t n, int K, int64_t b, const float* __restrict__ cb,
                    const float* __restrict__ qtab, const float* __restrict__ H,
                    const float* __restrict__ scale, uint16_t* __restrict__ idx,
-                   float* __restrict__ h, int sweeps, int sw, int32_t* __restrict__ changes,
+                   float* __restrict__ h, int64_t ldh, int sweeps, int sw,
+                   int32_t* __restrict__ changes,
                    const float* __restrict__ part_val, const int* __restrict__ part_idx,
                    int nchunks) {
   __shared__ float sdelta[8];
@@ -271,7 +285,7 @@ __global__ void __launch_bounds__(256)
     const int kcur = idx[row * B + b];
     const float sc = scale[row];
     float g[8];
-    block_gradient(H, n, h + row * n, cb, kcur, sc, b, g);
+    block_gradient(H, n, h + row * ldh, cb, kcur, sc, b, g);
     float scur = qtab[b * K + kcur];
 #pragma unroll
     for (int i = 0; i < 8; ++i) scur = fmaf(-cb[(int64_t)kcur * 8 + i], g[i], scur);
@@ -289,7 +303,7 @@ __global__ void __launch_bounds__(256)
   float dl[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) dl[j] = sdelta[j];
-  float* hr = h + row * n;
+  float* hr = h + row * ldh;
   for (int64_t i = threadIdx.x; i < n; i += blockDim.x) {
     const float* Hi = H + i * n + 8 * b;
     float acc = hr[i];
@@ -302,7 +316,7 @@ __global__ void __launch_bounds__(256)
 }  // namespace
 
 mpq_status launch_cd(mpq_plan_s* p, const float* W, int64_t m, const float* scale,
-                     const float* offset, uint16_t* idx, float* h, int32_t sweeps,
+                     const float* offset, uint16_t* idx, float* h, int64_t ldh, int32_t sweeps,
                      int32_t* changes, cudaStream_t st) {
   (void)W;
   (void)offset;
@@ -323,8 +337,8 @@ mpq_status launch_cd(mpq_plan_s* p, const float* W, int64_t m, const float* scal
         {
           ProfScope ps_("k_cd_tile_decide", st);
           k_cd_tile_decide<<<(unsigned)cdiv(m, CD1_WARPS), CD1_WARPS * 32, CD1_SMEM, st>>>(
-              m, n, p->K, t0, tw, j, nt, scale, p->H32, idx, h, sweeps, sw, changes, w.As.hi,
-              w.As.lo, w.As.ld, w.As.row_unscale, w.tile_count);
+              m, n, p->K, t0, tw, j, nt, scale, p->H32, idx, h, ldh, sweeps, sw, changes,
+              w.As.hi, w.As.lo, w.As.ld, w.As.row_unscale, w.tile_count);
         }
         count_launch();
         MPQ_TRY(check_launch("k_cd_tile_decide"));
@@ -333,7 +347,8 @@ mpq_status launch_cd(mpq_plan_s* p, const float* W, int64_t m, const float* scal
         o.accumulate = true;
         o.a_exact = true;
         o.gate = w.tile_count + sw * nt + j;
-        MPQ_TRY(gemm_tc(w.As, w.tm_at_hi, w.tm_at_lo, p->H_s, p->tm_h_hi, p->tm_h_lo, h, n, m, n,
+        o.c_reduce = (h == w.Hg) ? &w.tm_hg : nullptr;
+        MPQ_TRY(gemm_tc(w.As, w.tm_at_hi, w.tm_at_lo, p->H_s, p->tm_h_hi, p->tm_h_lo, h, ldh, m, n,
                         tw, p->H_s.unscale_host, p->status, st, "gemm_cd_update", o));
       }
     }
@@ -352,13 +367,13 @@ mpq_status launch_cd(mpq_plan_s* p, const float* W, int64_t m, const float* scal
       {
         ProfScope ps_("k_cd_vec_eval", st);
         k_cd_vec_eval<<<ga, 256, 0, st>>>(m, p->n, p->K, b, p->cb, p->qtab, p->H32, scale, idx, h,
-                                          sweeps, sw, changes, part_val, part_idx, nchunks);
+                                          ldh, sweeps, sw, changes, part_val, part_idx, nchunks);
       }
       {
         ProfScope ps_("k_cd_vec_apply", st);
         k_cd_vec_apply<<<(unsigned)m, 256, 0, st>>>(m, p->n, p->K, b, p->cb, p->qtab, p->H32,
-                                                    scale, idx, h, sweeps, sw, changes, part_val,
-                                                    part_idx, nchunks);
+                                                    scale, idx, h, ldh, sweeps, sw, changes,
+                                                    part_val, part_idx, nchunks);
       }
       count_launch(2);
       rc = check_launch("k_cd_vec");

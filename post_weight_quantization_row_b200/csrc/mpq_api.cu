@@ -179,6 +179,7 @@ void free_workspace(Workspace& w) {
   dfree(w.R1); dfree(w.X1); dfree(w.R2); dfree(w.P); dfree(w.idx);
   free_split(w.As);
   dfree(w.tile_count);
+  dfree(w.Hg);
   dfree(w.scale); dfree(w.offset); dfree(w.gamma1); dfree(w.gamma1_0); dfree(w.gamma2);
   dfree(w.beta); dfree(w.vsum); dfree(w.coef); dfree(w.kappa); dfree(w.clamps); dfree(w.W); dfree(w.w_hat);
   dfree(w.energy); dfree(w.idx_stage);
@@ -189,7 +190,7 @@ void free_workspace(Workspace& w) {
 constexpr int MAX_SWEEPS = 64;
 
 int64_t ws_bytes_per_row(const mpq_plan_s* p) {
-  return 3 * p->n * 4 + p->r * 4 +
+  return 3 * p->n * 4 + round_up(p->n, 32) * 4 + p->r * 4 +
          4 * round_up(std::max<int64_t>(std::max(p->n, p->r), CD_TILE), 64) + p->B * 2 + 3 * 4 +
          8 * 8 + 4 + MAX_SWEEPS * 4;
 }
@@ -210,6 +211,11 @@ mpq_status ensure_workspace(mpq_plan_s* p, int64_t rows) {
   if (st == MPQ_OK)
     chk(alloc_split(w.As, rows, std::max<int64_t>(std::max(p->n, p->r), CD_TILE), true));
   chk(dalloc(&w.tile_count, (int64_t)MAX_SWEEPS * cdiv(p->n, CD_TILE)));
+  w.ldh = round_up(p->n, 32);
+  chk(dalloc(&w.Hg, round_up(std::max<int64_t>(rows, 32), 32) * w.ldh));
+  if (st == MPQ_OK)
+    chk(make_tmap_f32_out(&w.tm_hg, w.Hg, std::max<int64_t>(p->n, 32),
+                          round_up(std::max<int64_t>(rows, 32), 32), w.ldh));
   if (st == MPQ_OK)
     chk(make_tmap_f16(&w.tm_an_hi, w.As.hi, round_up(p->n, 64), w.As.rows_pad, w.As.ld, 128));
   if (st == MPQ_OK)
@@ -291,10 +297,10 @@ mpq_status run_cd(mpq_plan_s* p, const float* W, int64_t m, const float* scale,
   Workspace& w = p->ws;
   const int64_t n = p->n;
   MPQ_TRY(launch_residual_split(p, W, m, scale, offset, idx, &w.As, nullptr, st));
-  // h = H (w - x)
-  MPQ_TRY(gemm_tc(w.As, w.tm_an_hi, w.tm_an_lo, p->H_s, p->tm_h_hi, p->tm_h_lo, w.X1, n, m, n, n,
-                  p->H_s.unscale_host, p->status, st, "gemm_hessian"));
-  return launch_cd(p, W, m, scale, offset, idx, w.X1, sweeps, changes, st);
+  // h = H (w - x), in its own padded buffer (the CD updates reduce into it)
+  MPQ_TRY(gemm_tc(w.As, w.tm_an_hi, w.tm_an_lo, p->H_s, p->tm_h_hi, p->tm_h_lo, w.Hg, w.ldh, m, n,
+                  n, p->H_s.unscale_host, p->status, st, "gemm_hessian"));
+  return launch_cd(p, W, m, scale, offset, idx, w.Hg, w.ldh, sweeps, changes, st);
 }
 
 mpq_status run_energy(mpq_plan_s* p, const float* W, int64_t m, const float* scale,
@@ -463,7 +469,7 @@ void mpq_params_default(mpq_params* p, int32_t d, int32_t K) {
   p->gamma_lo_rel = 1e-10;
   p->gamma_hi_rel = 1e10;
   p->alpha_min = 1e-10;
-  p->alpha_max = 1.0 - 1e-5;
+  p->alpha_max = 0.99;
 }
 
 mpq_status mpq_plan_create_from_spectrum(const double* s, const double* V, int64_t n, int64_t r,

@@ -72,6 +72,10 @@ struct Workspace {
   CUtensorMap tm_ar_hi, tm_ar_lo;  // K = r view
   CUtensorMap tm_at_hi, tm_at_lo;  // K = CD tile view
   int* tile_count = nullptr;       // CD: changes per (sweep, tile)
+  // CD gradient h = H (w - x), rows x ldh (ldh = n rounded up to 32)
+  float* Hg = nullptr;
+  int64_t ldh = 0;
+  CUtensorMap tm_hg;               // reduce-add target of the CD updates
   // m x r fp32
   float* P = nullptr;
   // m x B
@@ -167,9 +171,9 @@ mpq_status launch_residual(const mpq_plan_s* p, const float* W, int64_t m, const
 mpq_status launch_sanitize_idx(const mpq_plan_s* p, uint16_t* idx, int64_t count, cudaStream_t st);
 mpq_status launch_energy_rows(const mpq_plan_s* p, int64_t m, const float* P, float* energy,
                               cudaStream_t st);
-// CD sweeps; h (m x n) holds H (w - x) on entry and is updated in place
+// CD sweeps; h (m x ldh) holds H (w - x) on entry and is updated in place
 mpq_status launch_cd(mpq_plan_s* p, const float* W, int64_t m, const float* scale,
-                     const float* offset, uint16_t* idx, float* h, int32_t sweeps,
+                     const float* offset, uint16_t* idx, float* h, int64_t ldh, int32_t sweeps,
                      int32_t* changes, cudaStream_t st);
 constexpr int CD_TILE = 128;  // columns per scalar CD tile (multiple of 64)
 mpq_status launch_check_finite(const float* x, int64_t count, int* status, cudaStream_t st);
@@ -184,7 +188,12 @@ struct GemmOpts {
   bool accumulate = false;  // C += result instead of C = result
   bool a_exact = false;     // A_lo is zero: skip its load and product
   const int* gate = nullptr;  // device int; 0 -> the launch does nothing
+  // accumulate through TMA reduce-add into the fp32 matrix this map
+  // describes (box 32 x 32, 128B swizzle) instead of a read-modify-write
+  const CUtensorMap* c_reduce = nullptr;
 };
+mpq_status make_tmap_f32_out(CUtensorMap* tm, const float* base, int64_t cols, int64_t rows,
+                             int64_t ld_elems);
 mpq_status gemm_tc(const SplitOperand& A, const CUtensorMap& ta_hi, const CUtensorMap& ta_lo,
                    const SplitOperand& B, const CUtensorMap& tb_hi, const CUtensorMap& tb_lo,
                    float* C, int64_t ldc, int64_t M, int64_t N, int64_t K, float b_scale_host,

@@ -38,7 +38,7 @@ def test_params_default(mpq):
     mpq.lib.mpq_params_default(C.byref(p), 1, 8)
     assert p.d == 1 and p.K == 8 and p.beta0 == 1.0 and p.damping == 0.5
     assert math.isinf(p.tau) and p.gamma_lo_rel == 1e-10 and p.gamma_hi_rel == 1e10
-    assert p.alpha_min == 1e-10 and abs(p.alpha_max - (1 - 1e-5)) < 1e-15
+    assert p.alpha_min == 1e-10 and p.alpha_max == 0.99
 
 
 @pytest.mark.parametrize("field,value", [("d", 3), ("K", 1), ("damping", 1.5), ("beta0", -1.0),
