@@ -58,7 +58,7 @@ def parse():
 
 # ------------------------------------------------------------------ dist ---
 
-def dist_init(n_gpus):
+def dist_init(n_gpus, backend="nccl"):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -66,18 +66,28 @@ def dist_init(n_gpus):
         import datetime
 
         import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
     return world, rank, local
 
 
 def allreduce_max(x: float, world: int) -> float:
+    """Max over ranks (the job's time is that of its slowest rank)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(local_total_ms: float, steps: int, m_out: int, n: int, world: int):
+    """Weak scaling: every rank solves its own m_out rows; the job's step time
+    is the slowest rank's, and the value counts the weights of all ranks."""
+    total_ms = allreduce_max(local_total_ms, world)
+    ms_per_step = total_ms / steps
+    return world * m_out * n / (ms_per_step / 1e3), ms_per_step
 
 
 def barrier(world):
@@ -338,10 +348,8 @@ def run_mpq(args, world, rank, local):
     launches = mpq.kernel_launch_count() - launches0
     plan.status()
     barrier(world)
-    total_ms = sum(a.elapsed_time(b) for a, b in ev)
-    total_ms = allreduce_max(total_ms, world)
-    ms_per_step = total_ms / args.steps
-    value = world * m * n / (ms_per_step / 1e3)
+    value, ms_per_step = job_throughput(sum(a.elapsed_time(b) for a, b in ev), args.steps, m, n,
+                                        world)
 
     # roofline of the dominant kernel (largest share of device time)
     peaks, peak_src = load_peaks()

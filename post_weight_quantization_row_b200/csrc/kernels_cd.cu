@@ -40,21 +40,27 @@ __global__ void __launch_bounds__(CD1_WARPS * 32)
   float* sH = cd_smem;                                  // H[tile, tile]
   float* s_h_all = sH + CD_TILE * CD_TILE;              // per-warp gradient of the tile
   uint16_t* s_i_all = (uint16_t*)(s_h_all + CD1_WARPS * CD_TILE);  // per-warp indices
-  // H[tile, tile] into shared memory: each warp copies rows with coalesced
-  // loads, all of a row's loads in flight together
+  // H[tile, tile] into shared memory: warp w copies rows w, w + 16, ...; all
+  // of a warp's loads are issued before the first store so their latencies
+  // overlap (CD_TILE / CD1_WARPS rows x CD_TILE / 32 values per lane)
   {
+    constexpr int RPW = CD_TILE / CD1_WARPS, VPL = CD_TILE / 32;
     const int wid0 = threadIdx.x >> 5, lane0 = threadIdx.x & 31;
-    for (int i = wid0; i < tw; i += CD1_WARPS) {
+    float v[RPW][VPL];
+#pragma unroll
+    for (int rr = 0; rr < RPW; ++rr) {
+      const int i = wid0 + rr * CD1_WARPS;
       const float* src = H + (t0 + i) * n + t0;
-      float v[CD_TILE / 32];
 #pragma unroll
-      for (int q = 0; q < CD_TILE / 32; ++q) {
+      for (int q = 0; q < VPL; ++q) {
         const int j = lane0 + 32 * q;
-        v[q] = (j < tw) ? src[j] : 0.0f;
+        v[rr][q] = (i < tw && j < tw) ? src[j] : 0.0f;
       }
-#pragma unroll
-      for (int q = 0; q < CD_TILE / 32; ++q) sH[i * CD_TILE + lane0 + 32 * q] = v[q];
     }
+#pragma unroll
+    for (int rr = 0; rr < RPW; ++rr)
+#pragma unroll
+      for (int q = 0; q < VPL; ++q) sH[(wid0 + rr * CD1_WARPS) * CD_TILE + lane0 + 32 * q] = v[rr][q];
   }
   __syncthreads();
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;

@@ -77,6 +77,14 @@ __device__ __forceinline__ double clip_count(double v, double lo, double hi, int
   return c;
 }
 
+// 2^x by the hardware approximation (MUFU ex2, relative error ~2^-22;
+// flushes subnormal results to zero, which is harmless for posterior weights)
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Split of a row for the tensor-core GEMM: a per-row power of two e with
 // max|x| * 2^-e < 2^14, then hi = fp16(x 2^-e), lo = fp16(x 2^-e - hi).
 __device__ __forceinline__ int split_exponent(float amax) {
@@ -187,6 +195,7 @@ __global__ void __launch_bounds__(ROW_THREADS)
 // Posterior over levels k = 0..L-1 (weights scale*k + offset) of
 // q(k) ~ exp(-gamma1/2 (scale k + offset - r)^2) [* anchor]; in level units
 // t = (r - offset)/scale, g = gamma1 scale^2, logit_k = -g/2 (k - t)^2.
+template <int LT>
 __global__ void __launch_bounds__(ROW_THREADS)
     k_denoise_scalar(const float* __restrict__ R1, const double* __restrict__ gamma1,
                      const float* __restrict__ scale, const float* __restrict__ offset,
@@ -203,63 +212,71 @@ __global__ void __launch_bounds__(ROW_THREADS)
   const bool anchored = (W != nullptr);
   const double ga = anchored ? fmin(gamma1_0[row] * inv_tau2 * sc2, 1e30) : 0.0;
   const double geff = g + ga;
-  const float decay = (float)exp(-geff);
-  const double Lm1 = (double)(L - 1);
-  double acc = 0.0;
+  const float A2 = (float)(-0.5 * geff * 1.4426950408889634);  // -geff/2 log2(e)
+  const float inv_sc = (float)inv_dsc;
+  const float Lm1 = (float)(L - 1);
+  const float sc2f = (float)sc2;
+  float acc = 0.0f;
   for (int64_t j = threadIdx.x; j < n; j += blockDim.x) {
     const int64_t o = row * n + j;
-    // the level coordinate is formed in fp64 (the fp32 inputs are exact
-    // there) so that its offset from the nearest level, |dt| <= 1/2 inside
-    // the grid, is accurate to fp32 rounding; the 16 logits then only lose
-    // fp32 relative precision of their own size
-    double t = ((double)R1[o] - doff) * inv_dsc;
-    if (anchored) {
-      const double tw = ((double)W[o] - doff) * inv_dsc;
-      t = (g * t + ga * tw) / geff;
+    const float r = R1[o];
+    float ks, dt;  // nearest level and the offset from it, in level units
+    if (!anchored) {
+      ks = fminf(fmaxf(ceilf((r - off) * inv_sc - 0.5f), 0.0f), Lm1);
+      // r - (scale ks + offset) without rounding the level value: an
+      // error-free product and sum (Dekker / Knuth) give it as s + e.  The
+      // explicitly rounded intrinsics keep the compiler from contracting or
+      // reassociating these steps.
+      const float pr = __fmul_rn(sc, ks);
+      const float pe = fmaf(sc, ks, -pr);
+      const float s = __fadd_rn(pr, off);
+      const float bb = __fsub_rn(s, pr);
+      const float se = __fadd_rn(__fsub_rn(pr, __fsub_rn(s, bb)), __fsub_rn(off, bb));
+      dt = __fmul_rn(__fsub_rn(__fsub_rn(r, s), __fadd_rn(pe, se)), inv_sc);
+    } else {
+      // anchored prior: the effective centre mixes r and w (fp64, rare path)
+      const double tt = (g * ((double)r - doff) + ga * ((double)W[o] - doff)) * inv_dsc / geff;
+      const double kd = fmin(fmax(ceil(tt - 0.5), 0.0), (double)(L - 1));
+      ks = (float)kd;
+      dt = (float)(tt - kd);
     }
-    // argmax of -(k - t)^2, lowest k on ties
-    const double ks = fmin(fmax(ceil(t - 0.5), 0.0), Lm1);
-    const double dt = t - ks;  // |dt| <= 1/2 inside the grid
     const int kstar = (int)ks;
-    // q_k / q_k* = exp(-geff/2 ((k - t)^2 - (k* - t)^2)).  On a uniform grid
-    // consecutive ratios differ by the constant factor exp(-geff), so the L
-    // weights follow from three exponentials and a product recurrence
-    // (relative error ~|k - k*| ulp) instead of L exponentials.
-    const float up0 = __expf(-(float)(geff * (0.5 - dt)));  // q_{k*+1}/q_{k*} <= 1
-    const float dn0 = __expf(-(float)(geff * (0.5 + dt)));  // q_{k*-1}/q_{k*} <= 1
-    float S0 = 1.0f, S1 = 0.0f, S2 = 0.0f;
-    {
-      float e = 1.0f, ratio = up0, dk = 0.0f;
-      for (int k = kstar + 1; k < L; ++k) {
-        e *= ratio;
-        ratio *= decay;
-        dk += 1.0f;
+    // q_k / q_k* = 2^(dk (A dk + B)) with dk = k - k*, A = -geff/2 log2(e),
+    // B = -2 A dt: all L levels in one fixed loop (no lane-dependent trip
+    // counts, so warps do not diverge), one hardware 2^x per level
+    const float B2 = -2.0f * A2 * dt;
+    float S0 = 0.0f, S1 = 0.0f, S2 = 0.0f;
+    if (LT > 0) {
+#pragma unroll
+      for (int k = 0; k < (LT > 0 ? LT : 1); ++k) {
+        const float dk = (float)k - ks;
+        const float e = fast_exp2(fmaf(A2, dk, B2) * dk);
         S0 += e;
-        S1 = fmaf(e, dk, S1);
-        S2 = fmaf(e * dk, dk, S2);
+        const float ed = e * dk;
+        S1 += ed;
+        S2 = fmaf(ed, dk, S2);
+      }
+    } else {
+      for (int k = 0; k < L; ++k) {
+        const float dk = (float)k - ks;
+        const float e = fast_exp2(fmaf(A2, dk, B2) * dk);
+        S0 += e;
+        const float ed = e * dk;
+        S1 += ed;
+        S2 = fmaf(ed, dk, S2);
       }
     }
-    {
-      float e = 1.0f, ratio = dn0, dk = 0.0f;
-      for (int k = kstar - 1; k >= 0; --k) {
-        e *= ratio;
-        ratio *= decay;
-        dk -= 1.0f;
-        S0 += e;
-        S1 = fmaf(e, dk, S1);
-        S2 = fmaf(e * dk, dk, S2);
-      }
-    }
-    const float m1 = S1 / S0;
-    const float var = fmaxf(S2 / S0 - m1 * m1, 0.0f);
-    xhat[o] = fmaf(sc, (float)kstar + m1, off);
-    const float v = (float)(sc2 * (double)var);
+    const float inv = __frcp_rn(S0);
+    const float m1 = S1 * inv;
+    const float var = fmaxf(fmaf(S2, inv, -m1 * m1), 0.0f);
+    xhat[o] = fmaf(sc, ks + m1, off);
+    const float v = sc2f * var;
     if (vblock) vblock[o] = v;
     if (idx) idx[o] = (uint16_t)kstar;
-    acc += (double)v;
+    acc += v;
   }
-  acc = block_sum(acc, ds);
-  if (threadIdx.x == 0) vsum[row] = acc;
+  const double tot = block_sum((double)acc, ds);
+  if (threadIdx.x == 0) vsum[row] = tot;
 }
 
 // ------------------------------------------------------- vector denoiser ---
@@ -690,9 +707,12 @@ mpq_status launch_denoise(const mpq_plan_s* p, const float* R1, const double* ga
   if (p->d == 1) {
     {
       ProfScope ps_("k_denoise_scalar", st);
-      k_denoise_scalar<<<rows_grid(m), ROW_THREADS, 0, st>>>(
-          R1, gamma1, scale, offset, p->n, p->K, anchored ? W : nullptr, gamma1_0, inv_tau2, xhat1,
-          vblock, vsum, idx);
+      auto* kern = (p->K == 16) ? k_denoise_scalar<16>
+                   : (p->K == 8) ? k_denoise_scalar<8>
+                   : (p->K == 4) ? k_denoise_scalar<4> : k_denoise_scalar<0>;
+      kern<<<rows_grid(m), ROW_THREADS, 0, st>>>(R1, gamma1, scale, offset, p->n, p->K,
+                                                 anchored ? W : nullptr, gamma1_0, inv_tau2,
+                                                 xhat1, vblock, vsum, idx);
     }
     count_launch();
     return check_launch("k_denoise_scalar");
