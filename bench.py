@@ -51,6 +51,9 @@ def parse():
     ap.add_argument("--cpu-rows", type=int, default=8, help="oracle sample size (rows)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--rows", type=int, default=0,
+                    help="solve only the first ROWS rows (small cases for ncu captures; "
+                         "the line then names the reduced workload)")
     ap.add_argument("--spectrum-cache", default=None,
                     help="npz file: reuse the spectrum a previous run computed on the device")
     return ap.parse_args()
@@ -175,12 +178,13 @@ def kernel_work(name, m, n, r, d, K, L):
         return "hbm", "GB/s", 12.0 * m * n
     if name == "k_linear_rows":          # read/write U' (m x r)
         return "hbm", "GB/s", 8.0 * m * r
-    if name == "k_denoise_vec":          # candidate evaluations (exp-bound)
+    if name in ("k_denoise_vec", "k_denoise_vec_tc"):  # one exponential per (block, codeword)
         return "sfu", "Gexp/s", float(m) * (n // 8) * K
     return None
 
 
-KERNEL_SOURCE = {"gemm": "gemm_tc.cu", "k_cd": "kernels_cd.cu", "k_": "kernels_vamp.cu"}
+KERNEL_SOURCE = {"gemm": "gemm_tc.cu", "k_cd": "kernels_cd.cu", "k_denoise_vec_tc": "denoise_tc.cu",
+                 "k_": "kernels_vamp.cu"}
 
 
 def source_sha(kernel):
@@ -188,7 +192,7 @@ def source_sha(kernel):
     csrc = os.path.join(ROOT, "post_weight_quantization_row_b200", "csrc")
     fname = next(v for k, v in KERNEL_SOURCE.items() if kernel.startswith(k))
     h = hashlib.sha256()
-    for f in (fname, "mpq_internal.cuh"):
+    for f in (fname, "mpq_internal.cuh", "tc_ptx.cuh"):
         h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 
@@ -294,6 +298,8 @@ def run_mpq(args, world, rank, local):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     p = workload(args.config, rank)
+    if args.rows:
+        p.W = np.ascontiguousarray(p.W[:args.rows])
     cfgd = describe(p, args.config)
     m, n = p.m_out, p.n
     cb = p.codebook if p.d == 8 else None

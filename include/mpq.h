@@ -83,6 +83,16 @@ typedef struct {
   double gamma_hi_rel;    /*   [lo, hi] * gamma1_0 (defaults 1e-10, 1e10) */
   double alpha_min;       /* mean divergences are clipped into            */
   double alpha_max;       /*   [alpha_min, alpha_max] (1e-10, 0.99)       */
+  int32_t vec_engine;     /* d = 8 denoiser: 0 (default) tensor cores when the
+                             codebook qualifies, else SIMT; 1 SIMT always;
+                             2 tensor cores (plan creation fails with
+                             MPQ_ERR_UNSUPPORTED when the codebook does not
+                             qualify).  Qualifies: K a multiple of 128, all
+                             coordinates integer multiples of 2^-e (e <= 8)
+                             with |c_i| 2^e <= 127, and |c|^2 < 2^14, so that
+                             fp16 holds them and the distance terms of the
+                             scores are exact in fp32 (lattice codebooks such
+                             as the offset E8 set).  Ignored for d = 1. */
 } mpq_params;
 
 /* Fill `p` with the defaults above for block size d and codebook size K. */

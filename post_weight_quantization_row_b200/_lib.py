@@ -41,7 +41,8 @@ class Params(C.Structure):
     _fields_ = [("d", C.c_int32), ("K", C.c_int32), ("codebook", C.c_void_p),
                 ("beta0", C.c_double), ("damping", C.c_double), ("tau", C.c_double),
                 ("gamma_lo_rel", C.c_double), ("gamma_hi_rel", C.c_double),
-                ("alpha_min", C.c_double), ("alpha_max", C.c_double)]
+                ("alpha_min", C.c_double), ("alpha_max", C.c_double),
+                ("vec_engine", C.c_int32)]
 
 
 class RowStats(C.Structure):

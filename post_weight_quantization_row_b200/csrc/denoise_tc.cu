@@ -1,0 +1,692 @@
+// Tensor-core blockwise denoiser for vector codebooks (d = 8).
+//
+// For every block b of 8 weights the denoiser needs the posterior
+// q_b(c) ~ exp(-g/2 |c - t_b|^2) over all K codewords (the blockwise
+// denoiser of the MPQ page, section "VAMP in rank space"; g = gamma1 s^2 and
+// t = r1 / s in codebook units), its mean, its total variance and its argmax.
+// The brute-force cost is K exponentials per block; the scores are
+// contractions over the 8 coordinates and run on the tensor cores.
+//
+//   pass 1  s(c) = t.c - |c|^2/2 in fp32                     -> argmax c*
+//   pass 2  logit(c) - logit(c*) = g [ (t - c*).(c - c*) - |c - c*|^2/2 ]
+//
+// Pass 2 splits t - c* = q + r with q on the grid 2^-F (exact in fp16) and
+// a small remainder r (|r| <= 2^-(F+1), scaled up on the way in so that its
+// fp16 pair stays clear of subnormals), and computes three accumulators,
+// each one MMA (K = 16) over the codebook operand [c | |c|^2 (fp16 pair), 1, 1]:
+//
+//   Q(c) = q.c - q.c*                 exact (integers in units 2^-(F+e))
+//   X(c) = c*.c - |c|^2/2 - |c*|^2/2  = -|c - c*|^2/2, exact
+//   R(c) = r.c - r.c*                 small; the only rounded one
+//
+// The per-row constants q.c*, |c*|^2/2 and r.c* ride in the spare K columns
+// against the 1s of the codebook operand.  This needs a codebook whose
+// coordinates are multiples of 2^-e with |c_i| 2^e <= 127 (lattice codebooks
+// such as the offset E8 set).  Q + X is then exact and the logit carries
+// rounding only from R, 2^-(F+1) smaller than t - c*; the weights keep fp32
+// accuracy up to large g.  The c* column (weight exactly 1) is kept out of
+// the sums and added back analytically, so the first moment comes out
+// centred on c* without cancellation; an overflowing sum (a near-tie at a
+// huge g) falls back to the point mass on c*.
+//
+// One tile is 128 blocks x 128 codewords.  The block operands are written by
+// the epilogue threads into shared memory in the no-swizzle K-major layout;
+// the codebook operand tiles (32 bytes per codeword) are prepared at plan
+// time in the same layout and streamed by bulk copies with the fp32
+// coordinates through a 6-stage ring.  Pass 1 is two MMAs (N = 128, t as an
+// fp16 hi/lo pair); pass 2 is eight MMAs (two halves of N = 64, three
+// accumulators).  TMEM holds two buffers so that the MMAs of the next tile
+// overlap the exponentials of this one.  The kernel is persistent: one CTA
+// per SM walks the 128-block tiles.  Warps 0-7 are the epilogue (warp w reads
+// TMEM lanes 32 (w % 4) .. +31; warps 0-3 take the first and warps 4-7 the
+// second half of the columns of each MMA), warp 8 owns TMEM and issues the
+// MMAs, warp 9 issues the loads.
+#include <cuda.h>
+#include <cuda_fp16.h>
+
+#include <cmath>
+#include <vector>
+
+#include "mpq_internal.cuh"
+#include "tc_ptx.cuh"
+
+namespace mpq {
+namespace {
+using namespace tcx;
+
+constexpr int DT_M = 128;                  // blocks per tile (MMA M)
+constexpr int DT_N = 128;                  // codewords per tile (pass 1 MMA N)
+constexpr int DT_N2 = 64;                  // pass 2 MMA N (two per tile)
+constexpr int DT_STAGES = 6;
+constexpr int DT_EPI_WARPS = 8;
+constexpr int DT_THREADS = (DT_EPI_WARPS + 2) * 32;
+constexpr int OPER_BYTES = 128 * 32;       // 128 rows x 16 fp16
+constexpr int CF_BYTES = DT_N * 8 * 4;     // fp32 coordinates of one tile
+constexpr int STAGE_BYTES = OPER_BYTES + CF_BYTES;
+constexpr uint32_t DT_TMEM_COLS = 512;     // 2 buffers of 256 columns
+constexpr uint32_t IDESC_P1 = idesc_f16(DT_M, DT_N);
+constexpr uint32_t IDESC_P2 = idesc_f16(DT_M, DT_N2);
+
+// shared-memory map (offsets from the 1024-aligned base)
+constexpr int N_ATILES = 6;
+constexpr int SM_A = 0;                                   // block operand tiles
+constexpr int SM_B = SM_A + N_ATILES * OPER_BYTES;        // stage ring
+constexpr int SM_ROW = SM_B + DT_STAGES * STAGE_BYTES;    // per-row data
+constexpr int SM_PART = SM_ROW + 6 * DT_M * 4;            // 128 x 10 partial sums
+constexpr int SM_BAR = SM_PART + DT_M * 10 * 4;
+constexpr int SM_END = SM_BAR + 16 * 8 + 16;
+// one CTA per SM: ask for more than half of the shared memory so that two
+// CTAs (and two 512-column TMEM allocations) never share an SM
+constexpr int DT_SMEM_BYTES = 120 * 1024;
+static_assert(SM_END + 1024 <= DT_SMEM_BYTES, "denoiser shared memory");
+
+enum { A1_HI = 0, A1_LO = 1, A2_Q = 2, A2_X = 3, A2_RH = 4, A2_RL = 5 };
+
+struct DenoiseTcArgs {
+  const float* R1;        // m x n (blocks of 8 contiguous)
+  const double* gamma1;   // per row
+  const float* scale;
+  const float* offset;
+  const float* W;         // anchor (nullable)
+  const double* gamma1_0;
+  double inv_tau2;
+  int64_t nblocks;        // m * B
+  int64_t B;              // blocks per row
+  int NT;                 // codeword tiles (K / 128)
+  int F, Fmin;            // grid bits of the exact part q of t - c* (finest, coarsest)
+  int rk;                 // r enters the MMA as r 2^(Fb + 1 + rk)
+  const uint8_t* cb_tc;   // NT x OPER_BYTES operand images
+  const float* cb;        // K x 8 fp32
+  float* xhat;
+  float* vblock;
+  uint16_t* idx;
+  int nearest_only;
+  int* status;
+};
+
+// byte offset of the 16-byte chunk h (k = 8h .. 8h+7) of row r inside a
+// 128 x 16 fp16 operand tile: 8 x 16 B core matrices, the two K chunks
+// 128 B apart (LBO), 8-row groups 256 B apart (SBO).  Rows 64..127 start at
+// byte 2048, so either half is itself a 64-row operand.
+__host__ __device__ __forceinline__ int oper_off(int r, int h) {
+  return (r & 7) * 16 + (r >> 3) * 256 + h * 128;
+}
+
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t saddr) {
+  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)(128 >> 4) << 16;   // LBO: next K chunk
+  d |= (uint64_t)(256 >> 4) << 32;   // SBO: next 8-row group
+  d |= (uint64_t)1 << 46;            // descriptor version
+  return d;                          // layout type 0: no swizzle
+}
+
+__device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+        "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]),
+        "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]),
+        "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ void named_sync_epi() {
+  asm volatile("bar.sync 1, %0;" ::"n"(DT_EPI_WARPS * 32) : "memory");
+}
+
+// Bounded wait that also gives up when another role has aborted.
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity,
+                                              volatile int* abort_flag, int* status) {
+  for (uint32_t i = 0; i < (1u << 25); ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 63) == 63 && *abort_flag) return false;
+    if (i > 256) __nanosleep(64);
+  }
+  atomicOr(status, STATUS_TIMEOUT);
+  *abort_flag = 1;
+  return false;
+}
+
+// fp16 pair of x (|x| clamped to 2^14, NaN kept): x ~ hi + lo with ~22
+// significand bits
+__device__ __forceinline__ void split16(double x, __half& hi, __half& lo) {
+  if (fabs(x) > 16384.0) x = copysign(16384.0, x);
+  hi = __double2half(x);
+  lo = __double2half(x - (double)__half2float(hi));
+}
+
+__device__ __forceinline__ void store_row(uint8_t* tile, int r, const __half (&v)[16]) {
+  uint4 c0, c1;
+  __half* p0 = reinterpret_cast<__half*>(&c0);
+  __half* p1 = reinterpret_cast<__half*>(&c1);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    p0[i] = v[i];
+    p1[i] = v[8 + i];
+  }
+  *reinterpret_cast<uint4*>(tile + oper_off(r, 0)) = c0;
+  *reinterpret_cast<uint4*>(tile + oper_off(r, 1)) = c1;
+}
+
+__global__ void __launch_bounds__(DT_THREADS, 1) k_denoise_vec_tc(DenoiseTcArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* At = smem + SM_A;
+  float* sm_g2 = reinterpret_cast<float*>(smem + SM_ROW);
+  float* sm_rs = sm_g2 + DT_M;
+  float* sm_bval = sm_rs + DT_M;
+  int* sm_bidx = reinterpret_cast<int*>(sm_bval + DT_M);
+  float* sm_part = reinterpret_cast<float*>(smem + SM_PART);
+  uint64_t* b_full = reinterpret_cast<uint64_t*>(smem + SM_BAR);
+  uint64_t* b_empty = b_full + DT_STAGES;
+  uint64_t* tm_full = b_empty + DT_STAGES;
+  uint64_t* tm_empty = tm_full + 2;
+  uint64_t* a_full = tm_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(a_full + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t mtiles = (a.nblocks + DT_M - 1) / DT_M;
+  const int passes = a.nearest_only ? 1 : 2;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < DT_STAGES; ++s) {
+      mbar_init(&b_full[s], 1);
+      mbar_init(&b_empty[s], DT_EPI_WARPS);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tm_full[b], 1);
+      mbar_init(&tm_empty[b], DT_EPI_WARPS);
+    }
+    mbar_init(a_full, DT_M);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == DT_EPI_WARPS) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(DT_TMEM_COLS));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  // Counters shared by all roles: `seq` counts codebook tiles (stage ring),
+  // `tu` counts TMEM buffer uses (one per pass-1 tile, two per pass-2 tile).
+  if (warp == DT_EPI_WARPS + 1) {
+    // ------------------------------------------------------------ loader
+    if (lane == 0) {
+      uint32_t seq = 0;
+      bool ok = true;
+      for (int64_t mt = blockIdx.x; mt < mtiles && ok; mt += gridDim.x)
+        for (int pass = 0; pass < passes && ok; ++pass)
+          for (int j = 0; j < a.NT; ++j, ++seq) {
+            const int s = seq % DT_STAGES;
+            const uint32_t use = seq / DT_STAGES;
+            if (seq >= DT_STAGES && !wait_or_abort(&b_empty[s], (use - 1) & 1, abort_flag, a.status)) {
+              ok = false;
+              break;
+            }
+            uint8_t* st = smem + SM_B + s * STAGE_BYTES;
+            mbar_expect_tx(&b_full[s], pass ? STAGE_BYTES : OPER_BYTES);
+            bulk_load_1d(st, a.cb_tc + (size_t)j * OPER_BYTES, OPER_BYTES, &b_full[s]);
+            if (pass) bulk_load_1d(st + OPER_BYTES, a.cb + (size_t)j * DT_N * 8, CF_BYTES, &b_full[s]);
+          }
+      // the copies in flight land before the CTA may exit
+      const uint32_t last = seq;
+      for (uint32_t q = (last > DT_STAGES ? last - DT_STAGES : 0); q < last; ++q) {
+        const int s = q % DT_STAGES;
+        for (uint32_t i = 0; i < (1u << 25) && !mbar_try_wait(&b_full[s], (q / DT_STAGES) & 1); ++i)
+          if (i > 256) __nanosleep(64);
+      }
+    }
+  } else if (warp == DT_EPI_WARPS) {
+    // ------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      uint32_t seq = 0, tu = 0, aphase = 0;
+      bool ok = true;
+      const uint32_t a_base = smem_u32(At);
+      for (int64_t mt = blockIdx.x; mt < mtiles && ok; mt += gridDim.x)
+        for (int pass = 0; pass < passes && ok; ++pass) {
+          if (!wait_or_abort(a_full, aphase & 1, abort_flag, a.status)) {
+            ok = false;
+            break;
+          }
+          ++aphase;
+          tc_fence_after();
+          for (int j = 0; j < a.NT && ok; ++j, ++seq) {
+            const int s = seq % DT_STAGES;
+            if (!wait_or_abort(&b_full[s], (seq / DT_STAGES) & 1, abort_flag, a.status)) {
+              ok = false;
+              break;
+            }
+            const uint32_t bst = smem_u32(smem + SM_B + s * STAGE_BYTES);
+            for (int h = 0; h < pass + 1; ++h, ++tu) {
+              const int buf = tu & 1;
+              if (tu >= 2 && !wait_or_abort(&tm_empty[buf], ((tu >> 1) - 1) & 1, abort_flag, a.status)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              const uint32_t d = tmem + (uint32_t)buf * 256u;
+              if (pass == 0) {
+                const uint64_t bd = kmajor_desc(bst);
+                umma_f16(d, kmajor_desc(a_base + A1_HI * OPER_BYTES), bd, IDESC_P1, 0u);
+                umma_f16(d, kmajor_desc(a_base + A1_LO * OPER_BYTES), bd, IDESC_P1, 1u);
+              } else {
+                // codewords 64h .. 64h+63 of the tile: rows from byte 2048 h
+                const uint64_t bd = kmajor_desc(bst + (uint32_t)h * 2048u);
+                umma_f16(d, kmajor_desc(a_base + A2_Q * OPER_BYTES), bd, IDESC_P2, 0u);
+                umma_f16(d + 64u, kmajor_desc(a_base + A2_X * OPER_BYTES), bd, IDESC_P2, 0u);
+                umma_f16(d + 128u, kmajor_desc(a_base + A2_RH * OPER_BYTES), bd, IDESC_P2, 0u);
+                umma_f16(d + 128u, kmajor_desc(a_base + A2_RL * OPER_BYTES), bd, IDESC_P2, 1u);
+              }
+              umma_commit(&tm_full[buf]);
+            }
+          }
+        }
+      // the MMAs in flight finish before TMEM is released
+      for (uint32_t q = (tu > 2 ? tu - 2 : 0); q < tu; ++q)
+        for (uint32_t i = 0; i < (1u << 25) && !mbar_try_wait(&tm_full[q & 1], (q >> 1) & 1); ++i)
+          if (i > 256) __nanosleep(64);
+    }
+  } else {
+    // ---------------------------------------------------------- epilogue
+    // After a failed wait a warp stops touching TMEM and the pipelines but
+    // keeps walking the tiles, so that every epilogue warp still reaches
+    // every named barrier (the other roles give up at their next wait).
+    const int wg = warp >> 2, qd = warp & 3;
+    const int rl = qd * 32 + lane;  // row of the tile this thread owns
+    const uint32_t t_lane = tmem + ((uint32_t)(qd * 32) << 16);
+    uint32_t seq = 0, tu = 0;
+    bool ok = true;
+    for (int64_t mt = blockIdx.x; mt < mtiles; mt += gridDim.x) {
+      const int64_t blk = mt * DT_M + rl;
+      const bool active = blk < a.nblocks;
+      const int64_t row = active ? blk / a.B : 0;
+      double t64[8];
+      float g = 0.0f;
+      if (wg == 0) {
+        // t = r1 / s (with the anchor: precision-weighted with w / s)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) t64[i] = 0.0;
+        if (active) {
+          const double sc = a.scale[row];
+          const double sc2 = sc * sc;
+          const float4 r0 = *reinterpret_cast<const float4*>(a.R1 + blk * 8);
+          const float4 r1 = *reinterpret_cast<const float4*>(a.R1 + blk * 8 + 4);
+          const float rv[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+          double gg = 1.0, ga = 0.0;
+          if (!a.nearest_only) {
+            gg = a.gamma1[row] * sc2;
+            ga = a.W ? a.gamma1_0[row] * a.inv_tau2 * sc2 : 0.0;
+          }
+          g = (float)fmin(gg + ga, 1e30);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            double ti = (double)rv[i] / sc;
+            if (a.W && !a.nearest_only) ti = (gg * ti + ga * ((double)a.W[blk * 8 + i] / sc)) / (gg + ga);
+            t64[i] = ti;
+          }
+        }
+        // pass-1 operands [t_hi | -1/2 -1/2 0...] and [t_lo | 0...], scaled
+        // by 2^6 (the argmax does not change) so that t_lo stays out of the
+        // fp16 subnormal range
+        __half hi[16], lo[16];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) split16(t64[i] * 64.0, hi[i], lo[i]);
+#pragma unroll
+        for (int i = 8; i < 16; ++i) hi[i] = lo[i] = __float2half(0.0f);
+        hi[8] = hi[9] = __float2half(-32.0f);
+        store_row(At + A1_HI * OPER_BYTES, rl, hi);
+        store_row(At + A1_LO * OPER_BYTES, rl, lo);
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        mbar_arrive(a_full);
+      }
+
+      // ---------------------------------------------- pass 1: argmax
+      float best = -INFINITY;
+      int bidx = 0;
+      for (int j = 0; j < a.NT; ++j, ++seq, ++tu) {
+        const int s = seq % DT_STAGES, buf = tu & 1;
+        if (ok) ok = __all_sync(0xffffffffu, wait_or_abort(&tm_full[buf], (tu >> 1) & 1, abort_flag, a.status));
+        if (!ok) continue;
+        tc_fence_after();
+        uint32_t v0[32], v1[32];
+        const uint32_t ta = t_lane + (uint32_t)buf * 256u + (uint32_t)(wg * 64);
+        tmem_ld32_nowait(ta, v0);
+        tmem_ld32_nowait(ta + 32u, v1);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&tm_empty[buf]);
+          mbar_arrive(&b_empty[s]);
+        }
+        const int base = j * DT_N + wg * 64;
+        float m0 = __uint_as_float(v0[0]), m1 = __uint_as_float(v1[0]);
+#pragma unroll
+        for (int k = 1; k < 32; ++k) {
+          m0 = fmaxf(m0, __uint_as_float(v0[k]));
+          m1 = fmaxf(m1, __uint_as_float(v1[k]));
+        }
+        if (m0 > best) {  // first index of the chunk maximum
+          int kk = 31;
+#pragma unroll
+          for (int k = 31; k >= 0; --k)
+            if (__uint_as_float(v0[k]) == m0) kk = k;
+          best = m0;
+          bidx = base + kk;
+        }
+        if (m1 > best) {
+          int kk = 31;
+#pragma unroll
+          for (int k = 31; k >= 0; --k)
+            if (__uint_as_float(v1[k]) == m1) kk = k;
+          best = m1;
+          bidx = base + 32 + kk;
+        }
+      }
+      // merge the two column halves: larger score, then the smaller index
+      if (wg == 1) {
+        sm_bval[rl] = best;
+        sm_bidx[rl] = bidx;
+      }
+      named_sync_epi();
+      if (wg == 0) {
+        const float ob = sm_bval[rl];
+        const int oi = sm_bidx[rl];
+        if (ob > best || (ob == best && oi < bidx)) {
+          best = ob;
+          bidx = oi;
+        }
+      }
+      if (a.nearest_only) {
+        if (wg == 0 && active && ok) a.idx[blk] = (uint16_t)bidx;
+        continue;
+      }
+
+      // ---------------------------------- pass 2 operands (centred on c*)
+      float cst[8];
+      if (wg == 0) {
+        const float4 c0 = *reinterpret_cast<const float4*>(a.cb + (int64_t)bidx * 8);
+        const float4 c1 = *reinterpret_cast<const float4*>(a.cb + (int64_t)bidx * 8 + 4);
+        cst[0] = c0.x; cst[1] = c0.y; cst[2] = c0.z; cst[3] = c0.w;
+        cst[4] = c1.x; cst[5] = c1.y; cst[6] = c1.z; cst[7] = c1.w;
+        // t - c* = q + r: q on the grid 2^-Fb with |q_i| 2^Fb <= 2047 (exact
+        // fp16), Fb the finest grid up to F that holds this block's largest
+        // coordinate, so |r| <= 2^-(Fb+1) stays ~2^-11 of |t - c*|.  r enters
+        // the MMA as r 2^(Fb+1+rk), |.| <= 2^rk, an fp16 pair whose low half
+        // is subnormal only for tiny r (rk is set at plan time so that
+        // r.c* stays within fp16); the epilogue scales R back.
+        double mx = 0.0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx = fmax(mx, fabs(t64[i] - (double)cst[i]));
+        int Fb = a.F;
+        while (Fb > a.Fmin && ldexp(mx, Fb) > 2047.0) --Fb;
+        const double sF = ldexp(1.0, Fb), isF = ldexp(1.0, -Fb), sR = ldexp(1.0, Fb + 1 + a.rk);
+        double qc = 0.0, rc = 0.0, nn = 0.0;
+        __half q16[16], x16[16], rh[16], rlo[16];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const double tp = t64[i] - (double)cst[i];
+          const double qi = fmin(fmax(rint(tp * sF), -2047.0), 2047.0);
+          const double tq = qi * isF;
+          q16[i] = __double2half(tq);
+          split16((tp - tq) * sR, rh[i], rlo[i]);
+          qc += tq * (double)cst[i];  // exact
+          rc += ((double)__half2float(rh[i]) + (double)__half2float(rlo[i])) * (double)cst[i];  // x sR
+          nn += (double)cst[i] * (double)cst[i];
+          x16[i] = __float2half(cst[i]);
+        }
+#pragma unroll
+        for (int i = 8; i < 16; ++i) q16[i] = x16[i] = rh[i] = rlo[i] = __float2half(0.0f);
+        // constants against the [.. | n_hi n_lo 1 1 ..] columns of the codebook operand
+        split16(-qc, q16[10], q16[11]);
+        x16[8] = x16[9] = __float2half(-0.5f);
+        split16(-0.5 * nn, x16[10], x16[11]);
+        split16(-rc, rh[10], rh[11]);
+        store_row(At + A2_Q * OPER_BYTES, rl, q16);
+        store_row(At + A2_X * OPER_BYTES, rl, x16);
+        store_row(At + A2_RH * OPER_BYTES, rl, rh);
+        store_row(At + A2_RL * OPER_BYTES, rl, rlo);
+        sm_g2[rl] = g * 1.4426950408889634f;  // logits in log2 units
+        sm_rs[rl] = (float)(1.0 / sR);
+        sm_bidx[rl] = bidx;
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        mbar_arrive(a_full);
+      }
+      named_sync_epi();
+      const float g2 = sm_g2[rl], rs = sm_rs[rl];
+      const int cchunk = sm_bidx[rl] >> 5, kst = sm_bidx[rl] & 31;  // c* as (32-chunk, column)
+
+      // ------------------------------------------- pass 2: moments
+      float S0 = 0.0f, S2 = 0.0f, S1[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) S1[i] = 0.0f;
+      for (int j = 0; j < a.NT; ++j, ++seq) {
+        const int s = seq % DT_STAGES;
+        const float4* cf = reinterpret_cast<const float4*>(smem + SM_B + s * STAGE_BYTES + OPER_BYTES);
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h, ++tu) {
+          const int buf = tu & 1;
+          if (ok) ok = __all_sync(0xffffffffu, wait_or_abort(&tm_full[buf], (tu >> 1) & 1, abort_flag, a.status));
+          if (!ok) continue;
+          tc_fence_after();
+          const uint32_t ta = t_lane + (uint32_t)buf * 256u + (uint32_t)(wg * 32);
+          uint32_t Q[32], X[32], R[32];
+          tmem_ld32_nowait(ta, Q);
+          tmem_ld32_nowait(ta + 64u, X);
+          tmem_ld32_nowait(ta + 128u, R);
+          tmem_wait_ld();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tm_empty[buf]);
+          float z[32];
+#pragma unroll
+          for (int k = 0; k < 32; ++k)  // Q + X is exact; R carries the rounding
+            z[k] = g2 * fmaf(__uint_as_float(R[k]), rs, __uint_as_float(Q[k]) + __uint_as_float(X[k]));
+          // the argmax column (weight exactly 1) is left out of the sums and
+          // added back at the end, so that the moments come out centred on c*
+          if (j * 4 + h * 2 + wg == cchunk) {
+#pragma unroll
+            for (int k = 0; k < 32; ++k)
+              if (k == kst) z[k] = -INFINITY;
+          }
+          const float4* cc = cf + (h * 64 + wg * 32) * 2;
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            const float q = ex2_approx(z[k]);
+            S0 += q;
+            S2 = fmaf(q, __uint_as_float(X[k]), S2);  // X = -|c - c*|^2 / 2
+            const float4 ca = cc[2 * k], cb = cc[2 * k + 1];
+            S1[0] = fmaf(q, ca.x, S1[0]);
+            S1[1] = fmaf(q, ca.y, S1[1]);
+            S1[2] = fmaf(q, ca.z, S1[2]);
+            S1[3] = fmaf(q, ca.w, S1[3]);
+            S1[4] = fmaf(q, cb.x, S1[4]);
+            S1[5] = fmaf(q, cb.y, S1[5]);
+            S1[6] = fmaf(q, cb.z, S1[6]);
+            S1[7] = fmaf(q, cb.w, S1[7]);
+          }
+        }
+        if (ok) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&b_empty[s]);
+        }
+      }
+      if (wg == 1) {
+        float* pp = sm_part + rl * 10;
+        pp[0] = S0;
+        pp[1] = S2;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) pp[2 + i] = S1[i];
+      }
+      named_sync_epi();
+      if (wg == 0 && active && ok) {
+        // S0, S1, S2 hold the codewords other than c* (weight 1, X = 0):
+        // E[c - c*] = (S1 - c* S0) / (1 + S0), E|c - c*|^2 = -2 S2 / (1 + S0)
+        const float* pp = sm_part + rl * 10;
+        S0 += pp[0];
+        S2 += pp[1];
+        const float sc = a.scale[row], off = a.offset[row];
+        const float inv = 1.0f / (1.0f + S0);
+        const bool point = !(S0 < INFINITY) && S0 == S0;  // overflow: point mass on c*
+        float mm = 0.0f, xo[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float mc = point ? 0.0f : fmaf(-cst[i], S0, S1[i] + pp[2 + i]) * inv;
+          mm = fmaf(mc, mc, mm);
+          xo[i] = fmaf(sc, cst[i] + mc, off);
+        }
+        *reinterpret_cast<float4*>(a.xhat + blk * 8) = make_float4(xo[0], xo[1], xo[2], xo[3]);
+        *reinterpret_cast<float4*>(a.xhat + blk * 8 + 4) = make_float4(xo[4], xo[5], xo[6], xo[7]);
+        // E|c - c*|^2 - |E c - c*|^2
+        const float var = point ? 0.0f : fmaxf(-2.0f * S2 * inv - mm, 0.0f);
+        a.vblock[blk] = (float)((double)sc * sc * var);
+        if (a.idx) a.idx[blk] = (uint16_t)bidx;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == DT_EPI_WARPS) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(DT_TMEM_COLS));
+  }
+}
+
+}  // namespace
+
+// Plan-time: decide whether the codebook can use the tensor-core denoiser.
+// Returns the grid bits F of the exact part of t - c*, or -1.  Qualifies: K a
+// multiple of 128, every coordinate an integer multiple of 2^-e (e <= 8) with
+// C = max |c_i| 2^e <= 127 and |c|^2 < 2^14.  Then (in units of 2^-(F+e),
+// F = e + f) q.c - q.c* stays below 2^14 C and |c - c*|^2 / 2 below
+// 2^(3+f) C^2, and f (<= 8) is the largest with the sum below 2^22: every
+// partial sum of the MMAs for Q and X is an exact fp32 value.  A block may
+// use any coarser grid down to 2^-(e+1) (the bounds only shrink).
+int vec_tc_grid_bits(const float* cb_host, int K, int* e_out, int* rk_out) {
+  if (K <= 0 || K % DT_N != 0) return -1;
+  for (int e = 0; e <= 8; ++e) {
+    const double u = std::ldexp(1.0, e);
+    bool ok = true;
+    double cmax = 0.0, nmax = 0.0;
+    for (int64_t c = 0; c < K && ok; ++c) {
+      double nn = 0.0;
+      for (int i = 0; i < 8; ++i) {
+        const double v = (double)cb_host[c * 8 + i];
+        const double w = v * u;
+        if (!std::isfinite(w) || w != std::nearbyint(w)) {
+          ok = false;
+          break;
+        }
+        cmax = std::fmax(cmax, std::fabs(w));
+        nn += v * v;
+      }
+      nmax = std::fmax(nmax, nn);
+    }
+    if (!ok) continue;
+    if (cmax > 127.0 || nmax >= 16384.0) return -1;
+    for (int f = 8; f >= 1; --f)
+      if (std::ldexp(cmax, 14) + std::ldexp(cmax * cmax, 3 + f) < std::ldexp(1.0, 22)) {
+        *e_out = e;
+        // r 2^(Fb+1+rk) is at most 2^rk per coordinate: 8 2^rk max|c_i| <= 2^14
+        const double cm = std::fmax(std::ldexp(cmax, -e), 1e-30);
+        *rk_out = (int)std::fmin(9.0, std::fmax(0.0, std::floor(std::log2(2048.0 / cm))));
+        return e + f;
+      }
+    return -1;
+  }
+  return -1;
+}
+
+// Codebook operand images: per tile of 128 codewords, row r holds
+// [c_0 .. c_7 | n_hi n_lo 1 1 0 0 0 0] (|c|^2 = n_hi + n_lo) in fp16 in the
+// no-swizzle K-major layout the kernel's descriptors describe.
+mpq_status build_vec_tc_tables(mpq_plan_s* p, const float* cb_host) {
+  const int NT = p->K / DT_N;
+  std::vector<__half> img((size_t)NT * OPER_BYTES / 2, __float2half(0.0f));
+  for (int c = 0; c < p->K; ++c) {
+    const int j = c / DT_N, r = c % DT_N;
+    __half* t = img.data() + (size_t)j * OPER_BYTES / 2;
+    double nn = 0.0;
+    for (int i = 0; i < 8; ++i) {
+      const float v = cb_host[(size_t)c * 8 + i];
+      t[oper_off(r, 0) / 2 + i] = __float2half(v);
+      nn += (double)v * v;
+    }
+    const __half nh = __double2half(nn);
+    __half* k1 = t + oper_off(r, 1) / 2;
+    k1[0] = nh;
+    k1[1] = __double2half(nn - (double)__half2float(nh));
+    k1[2] = k1[3] = __float2half(1.0f);
+  }
+  MPQ_CUDA(cudaMalloc(&p->cb_tc, img.size() * sizeof(__half)));
+  MPQ_CUDA(cudaMemcpy(p->cb_tc, img.data(), img.size() * sizeof(__half), cudaMemcpyHostToDevice));
+  return MPQ_OK;
+}
+
+mpq_status launch_denoise_vec_tc(const mpq_plan_s* p, const float* R1, const double* gamma1,
+                                 const float* scale, const float* offset, int64_t m,
+                                 const float* W, const double* gamma1_0, double inv_tau2,
+                                 float* xhat1, float* vblock, uint16_t* idx, int nearest_only,
+                                 cudaStream_t st) {
+  static bool attr_set[64] = {};
+  int dev = 0;
+  MPQ_CUDA(cudaGetDevice(&dev));
+  if (dev < 64 && !attr_set[dev]) {
+    MPQ_CUDA(cudaFuncSetAttribute(k_denoise_vec_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  DT_SMEM_BYTES));
+    attr_set[dev] = true;
+  }
+  int sms = 0;
+  MPQ_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  DenoiseTcArgs a{};
+  a.R1 = R1;
+  a.gamma1 = gamma1;
+  a.scale = scale;
+  a.offset = offset;
+  a.W = W;
+  a.gamma1_0 = gamma1_0;
+  a.inv_tau2 = inv_tau2;
+  a.B = p->B;
+  a.nblocks = m * p->B;
+  a.NT = p->K / DT_N;
+  a.F = p->vec_tc_F;
+  a.Fmin = p->vec_tc_Fmin;
+  a.rk = p->vec_tc_rk;
+  a.cb_tc = reinterpret_cast<const uint8_t*>(p->cb_tc);
+  a.cb = p->cb;
+  a.xhat = xhat1;
+  a.vblock = vblock;
+  a.idx = idx;
+  a.nearest_only = nearest_only;
+  a.status = p->status;
+  const int64_t mtiles = cdiv(a.nblocks, DT_M);
+  const unsigned grid = (unsigned)std::min<int64_t>(mtiles, (int64_t)sms);
+  {
+    ProfScope ps_(nearest_only ? "k_denoise_vec_tc(nearest)" : "k_denoise_vec_tc", st);
+    k_denoise_vec_tc<<<grid, DT_THREADS, DT_SMEM_BYTES, st>>>(a);
+  }
+  count_launch();
+  return check_launch("k_denoise_vec_tc");
+}
+
+}  // namespace mpq

@@ -358,13 +358,16 @@ __global__ void __launch_bounds__(VEC_THREADS) k_denoise_vec(VecDenoiseArgs a) {
     return;
   }
   // pass 2: moments centred on the argmax codeword c*.  With dc = c - c*
-  // (exact for lattice codebooks) and tp = t - c*, the logit relative to
-  // the best is g (dc.tp - |dc|^2/2), which keeps fp32 cancellation small.
-  float cs[8], tp[8];
+  // and tp = t - c*, the logit relative to the best is g (dc.tp - |dc|^2/2);
+  // its two terms cancel (both O(1) for the codewords that matter), so it is
+  // formed in fp64 before the fp32 exponential.
+  float cs[8];
+  double tp[8];
+  const double gd = (double)g;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     cs[i] = active ? a.cb[(int64_t)bidx * 8 + i] : 0.0f;
-    tp[i] = (float)(t64[i] - (double)cs[i]);
+    tp[i] = t64[i] - (double)cs[i];
   }
   float S0 = 0.0f, m2 = 0.0f, m1[8];
 #pragma unroll
@@ -380,16 +383,17 @@ __global__ void __launch_bounds__(VEC_THREADS) k_denoise_vec(VecDenoiseArgs a) {
     if (active) {
       for (int c = 0; c < cn; ++c) {
         float dc[8];
-        float dot = 0.0f, nn = 0.0f;
+        double dot = 0.0, nn = 0.0;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          dc[i] = scb[c][i] - cs[i];
-          dot = fmaf(dc[i], tp[i], dot);
-          nn = fmaf(dc[i], dc[i], nn);
+          const double d = (double)scb[c][i] - (double)cs[i];  // exact
+          dc[i] = (float)d;
+          dot = fma(d, tp[i], dot);
+          nn = fma(d, d, nn);
         }
-        const float q = __expf(g * (dot - 0.5f * nn));
+        const float q = __expf((float)(gd * (dot - 0.5 * nn)));
         S0 += q;
-        m2 = fmaf(q, nn, m2);
+        m2 = fmaf(q, (float)nn, m2);
 #pragma unroll
         for (int i = 0; i < 8; ++i) m1[i] = fmaf(q, dc[i], m1[i]);
       }
@@ -671,6 +675,11 @@ mpq_status launch_init(const mpq_plan_s* p, const float* W, int64_t m, int given
   }
   count_launch();
   MPQ_TRY(check_launch("k_init_rms"));
+  const int64_t nb = m * (p->n / 8);
+  if (p->vec_tc) {
+    MPQ_TRY(launch_denoise_vec_tc(p, W, nullptr, scale, offset, m, nullptr, nullptr, 0.0, nullptr,
+                                  nullptr, idx, 1, st));
+  } else {
   VecDenoiseArgs a{};
   a.R1 = W;
   a.scale = scale;
@@ -682,13 +691,13 @@ mpq_status launch_init(const mpq_plan_s* p, const float* W, int64_t m, int given
   a.cb_norm = p->cb_norm;
   a.idx = idx;
   a.nearest_only = 1;
-  const int64_t nb = m * (p->n / 8);
   {
     ProfScope ps_("k_denoise_vec", st);
     k_denoise_vec<<<(unsigned)cdiv(nb, VEC_THREADS), VEC_THREADS, 0, st>>>(a);
   }
   count_launch();
   MPQ_TRY(check_launch("k_denoise_vec(nearest)"));
+  }
   {
     ProfScope ps_("k_gamma0_vec", st);
     k_gamma0_vec<<<rows_grid(m), ROW_THREADS, 0, st>>>(W, p->n, p->cb, scale, offset, idx, gamma1_0);
@@ -718,6 +727,10 @@ mpq_status launch_denoise(const mpq_plan_s* p, const float* R1, const double* ga
     return check_launch("k_denoise_scalar");
   }
   if (vblock == nullptr) return fail(MPQ_ERR_INVALID_ARG, "vector denoiser needs vblock");
+  if (p->vec_tc) {
+    MPQ_TRY(launch_denoise_vec_tc(p, R1, gamma1, scale, offset, m, anchored ? W : nullptr,
+                                  gamma1_0, inv_tau2, xhat1, vblock, idx, 0, st));
+  } else {
   VecDenoiseArgs a{};
   a.R1 = R1;
   a.gamma1 = gamma1;
@@ -742,6 +755,7 @@ mpq_status launch_denoise(const mpq_plan_s* p, const float* R1, const double* ga
   }
   count_launch();
   MPQ_TRY(check_launch("k_denoise_vec"));
+  }
   {
     ProfScope ps_("k_row_sum", st);
     k_row_sum<<<rows_grid(m), ROW_THREADS, 0, st>>>(vblock, p->n / 8, vsum);

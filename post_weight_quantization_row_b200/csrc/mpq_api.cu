@@ -123,6 +123,7 @@ mpq_status validate_params(const mpq_params* q, int64_t n) {
     return fail(MPQ_ERR_INVALID_ARG, "d must be 1 or 8");
   }
   if (n <= 0 || n % q->d != 0) return fail(MPQ_ERR_INVALID_ARG, "n must be a positive multiple of d");
+  if (q->vec_engine < 0 || q->vec_engine > 2) return fail(MPQ_ERR_INVALID_ARG, "vec_engine must be 0, 1 or 2");
   if (!(q->beta0 > 0.0) || !isfinite(q->beta0)) return fail(MPQ_ERR_INVALID_ARG, "beta0 must be > 0");
   if (!(q->damping >= 0.0 && q->damping <= 1.0)) return fail(MPQ_ERR_INVALID_ARG, "damping must be in [0,1]");
   if (!(q->tau > 0.0)) return fail(MPQ_ERR_INVALID_ARG, "tau must be > 0 (INFINITY = uniform prior)");
@@ -416,6 +417,7 @@ void destroy_plan(mpq_plan_s* p) {
   free_workspace(p->ws);
   dfree(p->s64); dfree(p->V64); dfree(p->s32); dfree(p->V32); dfree(p->Vt32); dfree(p->H32);
   dfree(p->Hdiag); dfree(p->cb); dfree(p->cb_norm); dfree(p->qtab); dfree(p->status);
+  if (p->cb_tc) cudaFree(p->cb_tc);
   free_split(p->Vt_s); free_split(p->V_s); free_split(p->H_s);
   delete p;
 }
@@ -435,6 +437,15 @@ mpq_status new_plan(const mpq_params* params, int64_t n, mpq_plan_s** out) {
     if (st == MPQ_OK) {
       cudaError_t e = cudaMemcpy(p->cb, params->codebook, sizeof(float) * p->K * 8, cudaMemcpyHostToDevice);
       if (e != cudaSuccess) st = cuda_fail(e, "codebook copy");
+    }
+    if (st == MPQ_OK && params->vec_engine != 1) {
+      int e = 0;
+      p->vec_tc_F = vec_tc_grid_bits(params->codebook, p->K, &e, &p->vec_tc_rk);
+      p->vec_tc_Fmin = e + 1;
+      p->vec_tc = p->vec_tc_F > 0;
+      if (!p->vec_tc && params->vec_engine == 2)
+        st = fail(MPQ_ERR_UNSUPPORTED, "codebook does not qualify for the tensor-core denoiser");
+      if (st == MPQ_OK && p->vec_tc) st = build_vec_tc_tables(p, params->codebook);
     }
     if (st != MPQ_OK) {
       destroy_plan(p);
@@ -470,6 +481,7 @@ void mpq_params_default(mpq_params* p, int32_t d, int32_t K) {
   p->gamma_hi_rel = 1e10;
   p->alpha_min = 1e-10;
   p->alpha_max = 0.99;
+  p->vec_engine = 0;
 }
 
 mpq_status mpq_plan_create_from_spectrum(const double* s, const double* V, int64_t n, int64_t r,

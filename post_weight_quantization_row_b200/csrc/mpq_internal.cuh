@@ -121,6 +121,11 @@ struct mpq_plan_s {
   float* cb = nullptr;       // K x 8
   float* cb_norm = nullptr;  // K  |c|^2
   float* qtab = nullptr;     // B x K  1/2 c^T H_bb c
+  bool vec_tc = false;       // the denoiser runs on the tensor cores
+  int vec_tc_F = 0;          // grid bits of its exact split of t - c*
+  int vec_tc_Fmin = 0;       //   (finest, coarsest)
+  int vec_tc_rk = 0;         // extra scale bits of its remainder operand
+  void* cb_tc = nullptr;     // (K / 128) x 4 KiB codebook operand images
   // status
   int* status = nullptr;     // device word
   int64_t ws_cap = 0;
@@ -198,6 +203,15 @@ mpq_status gemm_tc(const SplitOperand& A, const CUtensorMap& ta_hi, const CUtens
                    const SplitOperand& B, const CUtensorMap& tb_hi, const CUtensorMap& tb_lo,
                    float* C, int64_t ldc, int64_t M, int64_t N, int64_t K, float b_scale_host,
                    int* status, cudaStream_t st, const char* tag, const GemmOpts& o = GemmOpts());
+
+// tensor-core vector denoiser (denoise_tc.cu)
+int vec_tc_grid_bits(const float* cb_host, int K, int* e_out, int* rk_out);  // -1: not eligible
+mpq_status build_vec_tc_tables(mpq_plan_s* p, const float* cb_host);
+mpq_status launch_denoise_vec_tc(const mpq_plan_s* p, const float* R1, const double* gamma1,
+                                 const float* scale, const float* offset, int64_t m,
+                                 const float* W, const double* gamma1_0, double inv_tau2,
+                                 float* xhat1, float* vblock, uint16_t* idx, int nearest_only,
+                                 cudaStream_t st);
 
 // plan-time builders
 mpq_status build_hessian(mpq_plan_s* p, cudaStream_t st);
