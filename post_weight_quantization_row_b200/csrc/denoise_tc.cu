@@ -4,16 +4,17 @@
 // q_b(c) ~ exp(-g/2 |c - t_b|^2) over all K codewords (the blockwise
 // denoiser of the MPQ page, section "VAMP in rank space"; g = gamma1 s^2 and
 // t = r1 / s in codebook units), its mean, its total variance and its argmax.
-// The brute-force cost is K exponentials per block; the scores are
-// contractions over the 8 coordinates and run on the tensor cores.
+// The brute-force cost is K exponentials per block; everything else runs on
+// the tensor cores:
 //
 //   pass 1  s(c) = t.c - |c|^2/2 in fp32                     -> argmax c*
 //   pass 2  logit(c) - logit(c*) = g [ (t - c*).(c - c*) - |c - c*|^2/2 ]
+//           q(c) = 2^(log2e logit + 8),  S0 = sum q,  S1 = sum q c  (c != c*)
 //
-// Pass 2 splits t - c* = q + r with q on the grid 2^-F (exact in fp16) and
-// a small remainder r (|r| <= 2^-(F+1), scaled up on the way in so that its
-// fp16 pair stays clear of subnormals), and computes three accumulators,
-// each one MMA (K = 16) over the codebook operand [c | |c|^2 (fp16 pair), 1, 1]:
+// Logits.  t - c* = q + r with q on the grid 2^-F (exact in fp16) and a small
+// remainder r (|r| <= 2^-(F+1), scaled up on the way in so that its fp16 pair
+// stays clear of subnormals).  Three accumulators, each one MMA (K = 16) over
+// the codebook operand [c | |c|^2 (fp16 pair), 1, 1]:
 //
 //   Q(c) = q.c - q.c*                 exact (integers in units 2^-(F+e))
 //   X(c) = c*.c - |c|^2/2 - |c*|^2/2  = -|c - c*|^2/2, exact
@@ -23,24 +24,31 @@
 // against the 1s of the codebook operand.  This needs a codebook whose
 // coordinates are multiples of 2^-e with |c_i| 2^e <= 127 (lattice codebooks
 // such as the offset E8 set).  Q + X is then exact and the logit carries
-// rounding only from R, 2^-(F+1) smaller than t - c*; the weights keep fp32
-// accuracy up to large g.  The c* column (weight exactly 1) is kept out of
-// the sums and added back analytically, so the first moment comes out
-// centred on c* without cancellation; an overflowing sum (a near-tie at a
-// huge g) falls back to the point mass on c*.
+// rounding only from R, 2^-(F+1) smaller than t - c*.
 //
-// One tile is 128 blocks x 128 codewords.  The block operands are written by
-// the epilogue threads into shared memory in the no-swizzle K-major layout;
-// the codebook operand tiles (32 bytes per codeword) are prepared at plan
-// time in the same layout and streamed by bulk copies with the fp32
-// coordinates through a 6-stage ring.  Pass 1 is two MMAs (N = 128, t as an
-// fp16 hi/lo pair); pass 2 is eight MMAs (two halves of N = 64, three
-// accumulators).  TMEM holds two buffers so that the MMAs of the next tile
-// overlap the exponentials of this one.  The kernel is persistent: one CTA
-// per SM walks the 128-block tiles.  Warps 0-7 are the epilogue (warp w reads
-// TMEM lanes 32 (w % 4) .. +31; warps 0-3 take the first and warps 4-7 the
-// second half of the columns of each MMA), warp 8 owns TMEM and issues the
-// MMAs, warp 9 issues the loads.
+// Moments.  The weights (c* excluded: its weight 2^8 is added back at the
+// end, which leaves the first moment centred on c* without cancellation) go
+// to shared memory as fp16 hi/lo pairs and one more MMA (N = 16) against the
+// transposed codebook [c_0 .. c_7, 1] accumulates S1 and S0 in TMEM for the
+// whole 128-block tile; only S2 = sum q X (the centred second moment, -1/2
+// |c - c*|^2 per codeword) and the exponential stay on the ALU.  A logit
+// above c*'s by 2^7 (the argmax pass's fp32 scores misjudged a near-tie at
+// an enormous g) would overflow the fp16 weights: the tile falls back to the
+// point mass on c*.
+//
+// Pipeline.  One tile is 128 blocks x 128 codewords.  The block operands are
+// written by the epilogue threads into shared memory in the no-swizzle
+// K-major layout; the codebook operands (8 KiB per 128 codewords: scores
+// and transposed) are prepared at plan time in the same layout and streamed
+// by bulk copies through a 6-stage ring.  Pass 1 is two MMAs (N = 128, t as
+// an fp16 hi/lo pair); pass 2 is, per half of 64 codewords, four score MMAs
+// (N = 64, three accumulators) and eight moment MMAs (N = 16, K = 64 as hi
+// and lo).  TMEM holds two score buffers so that the MMAs of the next half
+// overlap the exponentials of this one, plus the moment accumulator.  The
+// kernel is persistent: one CTA per SM walks the 128-block tiles.  Warps 0-15
+// are the epilogue (warp w reads TMEM lanes 32 (w % 4) .. +31; warpgroup
+// w / 4 takes one quarter of the columns of each MMA), warp 16 owns TMEM and
+// issues the MMAs, warp 17 issues the loads.
 #include <cuda.h>
 #include <cuda_fp16.h>
 
@@ -56,28 +64,39 @@ using namespace tcx;
 
 constexpr int DT_M = 128;                  // blocks per tile (MMA M)
 constexpr int DT_N = 128;                  // codewords per tile (pass 1 MMA N)
-constexpr int DT_N2 = 64;                  // pass 2 MMA N (two per tile)
+constexpr int DT_N2 = 64;                  // pass 2 score MMA N (two halves per tile)
 constexpr int DT_STAGES = 6;
-constexpr int DT_EPI_WARPS = 8;
+constexpr int DT_EPI_WARPS = 16;
+constexpr int DT_WGS = DT_EPI_WARPS / 4;   // column quarters
 constexpr int DT_THREADS = (DT_EPI_WARPS + 2) * 32;
+constexpr int MMA_WARP = DT_EPI_WARPS, LOAD_WARP = DT_EPI_WARPS + 1;
 constexpr int OPER_BYTES = 128 * 32;       // 128 rows x 16 fp16
-constexpr int CF_BYTES = DT_N * 8 * 4;     // fp32 coordinates of one tile
-constexpr int STAGE_BYTES = OPER_BYTES + CF_BYTES;
-constexpr uint32_t DT_TMEM_COLS = 512;     // 2 buffers of 256 columns
+constexpr int CBT_BYTES = 16 * 128 * 2;    // transposed codebook tile: 16 x 128 fp16
+constexpr int STAGE_BYTES = OPER_BYTES + CBT_BYTES;
+constexpr int QW_BYTES = 128 * 64 * 2;     // weights of one half: 128 x 64 fp16
+// TMEM: pass 1 cycles through 4 score buffers of 128 columns; pass 2 through
+// 2 buffers of 192 (Q | X | R, 64 each) and keeps the moments at 384.  The
+// passes reuse the same columns: every pass starts after the epilogue has
+// read all of the previous one.
+constexpr uint32_t DT_TMEM_COLS = 512;
+constexpr int T1_BUFS = 4, T2_BUFS = 2;
+constexpr uint32_t T1_COLS = 128, T2_COLS = 192, TM_MOM = 384;
 constexpr uint32_t IDESC_P1 = idesc_f16(DT_M, DT_N);
 constexpr uint32_t IDESC_P2 = idesc_f16(DT_M, DT_N2);
+constexpr uint32_t IDESC_MOM = idesc_f16(DT_M, 16);
+constexpr float Q_SHIFT = 8.0f;            // weights carry 2^8: c*'s is 256
 
 // shared-memory map (offsets from the 1024-aligned base)
 constexpr int N_ATILES = 6;
 constexpr int SM_A = 0;                                   // block operand tiles
 constexpr int SM_B = SM_A + N_ATILES * OPER_BYTES;        // stage ring
-constexpr int SM_ROW = SM_B + DT_STAGES * STAGE_BYTES;    // per-row data
-constexpr int SM_PART = SM_ROW + 6 * DT_M * 4;            // 128 x 10 partial sums
-constexpr int SM_BAR = SM_PART + DT_M * 10 * 4;
-constexpr int SM_END = SM_BAR + 16 * 8 + 16;
-// one CTA per SM: ask for more than half of the shared memory so that two
-// CTAs (and two 512-column TMEM allocations) never share an SM
-constexpr int DT_SMEM_BYTES = 120 * 1024;
+constexpr int SM_QW = SM_B + DT_STAGES * STAGE_BYTES;     // 2 x (hi | lo) weights
+constexpr int SM_T = SM_QW + 2 * 2 * QW_BYTES;            // t per row (fp64, 128 x 8)
+constexpr int SM_ROW = SM_T + DT_M * 8 * 8;               // per-row data
+constexpr int SM_BAR = SM_ROW + (3 + 2 * DT_WGS + DT_WGS) * DT_M * 4;
+constexpr int N_BARS = 2 * DT_STAGES + 2 * T1_BUFS + 2 * T2_BUFS + 1 + 2 + 2 + 1;
+constexpr int SM_END = SM_BAR + N_BARS * 8 + 16;
+constexpr int DT_SMEM_BYTES = 160 * 1024;  // > half of the SM: one CTA (and TMEM owner) per SM
 static_assert(SM_END + 1024 <= DT_SMEM_BYTES, "denoiser shared memory");
 
 enum { A1_HI = 0, A1_LO = 1, A2_Q = 2, A2_X = 3, A2_RH = 4, A2_RL = 5 };
@@ -95,7 +114,7 @@ struct DenoiseTcArgs {
   int NT;                 // codeword tiles (K / 128)
   int F, Fmin;            // grid bits of the exact part q of t - c* (finest, coarsest)
   int rk;                 // r enters the MMA as r 2^(Fb + 1 + rk)
-  const uint8_t* cb_tc;   // NT x OPER_BYTES operand images
+  const uint8_t* cb_tc;   // NT x STAGE_BYTES operand images
   const float* cb;        // K x 8 fp32
   float* xhat;
   float* vblock;
@@ -104,18 +123,17 @@ struct DenoiseTcArgs {
   int* status;
 };
 
-// byte offset of the 16-byte chunk h (k = 8h .. 8h+7) of row r inside a
-// 128 x 16 fp16 operand tile: 8 x 16 B core matrices, the two K chunks
-// 128 B apart (LBO), 8-row groups 256 B apart (SBO).  Rows 64..127 start at
-// byte 2048, so either half is itself a 64-row operand.
-__host__ __device__ __forceinline__ int oper_off(int r, int h) {
-  return (r & 7) * 16 + (r >> 3) * 256 + h * 128;
+// Byte offset of element (row r, k) of a no-swizzle K-major fp16 tile whose
+// 8-row groups are `sbo` bytes apart: 8 x 16 B core matrices, consecutive K
+// chunks of 8 elements 128 B apart (the descriptor's LBO).
+__host__ __device__ __forceinline__ int kmaj_off(int r, int k, int sbo) {
+  return (r & 7) * 16 + (r >> 3) * sbo + (k >> 3) * 128 + (k & 7) * 2;
 }
 
-__device__ __forceinline__ uint64_t kmajor_desc(uint32_t saddr) {
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t saddr, uint32_t sbo) {
   uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
   d |= (uint64_t)(128 >> 4) << 16;   // LBO: next K chunk
-  d |= (uint64_t)(256 >> 4) << 32;   // SBO: next 8-row group
+  d |= (uint64_t)(sbo >> 4) << 32;   // SBO: next 8-row group
   d |= (uint64_t)1 << 46;            // descriptor version
   return d;                          // layout type 0: no swizzle
 }
@@ -130,6 +148,15 @@ __device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, uint32_t (&v)[3
         "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]),
         "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]),
         "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld16_nowait(uint32_t taddr, uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+        "=r"(v[14]), "=r"(v[15])
       : "r"(taddr));
 }
 __device__ __forceinline__ void tmem_wait_ld() {
@@ -159,6 +186,12 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity,
   return false;
 }
 
+// Warp-uniform bounded wait (every lane polls; all must see the phase).
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          int* status) {
+  return __all_sync(0xffffffffu, wait_or_abort(bar, parity, abort_flag, status));
+}
+
 // fp16 pair of x (|x| clamped to 2^14, NaN kept): x ~ hi + lo with ~22
 // significand bits
 __device__ __forceinline__ void split16(double x, __half& hi, __half& lo) {
@@ -167,6 +200,7 @@ __device__ __forceinline__ void split16(double x, __half& hi, __half& lo) {
   lo = __double2half(x - (double)__half2float(hi));
 }
 
+// one 16-element row of a 128 x 16 block operand tile
 __device__ __forceinline__ void store_row(uint8_t* tile, int r, const __half (&v)[16]) {
   uint4 c0, c1;
   __half* p0 = reinterpret_cast<__half*>(&c0);
@@ -176,25 +210,41 @@ __device__ __forceinline__ void store_row(uint8_t* tile, int r, const __half (&v
     p0[i] = v[i];
     p1[i] = v[8 + i];
   }
-  *reinterpret_cast<uint4*>(tile + oper_off(r, 0)) = c0;
-  *reinterpret_cast<uint4*>(tile + oper_off(r, 1)) = c1;
+  *reinterpret_cast<uint4*>(tile + kmaj_off(r, 0, 256)) = c0;
+  *reinterpret_cast<uint4*>(tile + kmaj_off(r, 8, 256)) = c1;
 }
 
+// (hi, lo) fp16 pairs of two fp32 values: x ~ hi + lo; saturating, so an
+// overflow (caught separately) cannot turn into inf - inf
+__device__ __forceinline__ void split_pair(float a, float b, uint32_t& hi, uint32_t& lo) {
+  asm("cvt.rn.satfinite.f16x2.f32 %0, %2, %1;" : "=r"(hi) : "f"(a), "f"(b));
+  const float2 h = __half22float2(*reinterpret_cast<const __half2*>(&hi));
+  asm("cvt.rn.satfinite.f16x2.f32 %0, %2, %1;" : "=r"(lo) : "f"(a - h.x), "f"(b - h.y));
+}
+
+// 18 warps: five share an SM sub-partition's 16K registers, so at most 96 each
 __global__ void __launch_bounds__(DT_THREADS, 1) k_denoise_vec_tc(DenoiseTcArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* At = smem + SM_A;
+  double* sm_t = reinterpret_cast<double*>(smem + SM_T);        // [128][8]
   float* sm_g2 = reinterpret_cast<float*>(smem + SM_ROW);
   float* sm_rs = sm_g2 + DT_M;
-  float* sm_bval = sm_rs + DT_M;
-  int* sm_bidx = reinterpret_cast<int*>(sm_bval + DT_M);
-  float* sm_part = reinterpret_cast<float*>(smem + SM_PART);
+  float* sm_g = sm_rs + DT_M;
+  float* sm_bval = sm_g + DT_M;                                   // [DT_WGS][128]
+  int* sm_bidx = reinterpret_cast<int*>(sm_bval + DT_WGS * DT_M);  // [DT_WGS][128]
+  float* sm_s2 = reinterpret_cast<float*>(sm_bidx + DT_WGS * DT_M);  // [DT_WGS][128]
   uint64_t* b_full = reinterpret_cast<uint64_t*>(smem + SM_BAR);
   uint64_t* b_empty = b_full + DT_STAGES;
-  uint64_t* tm_full = b_empty + DT_STAGES;
-  uint64_t* tm_empty = tm_full + 2;
-  uint64_t* a_full = tm_empty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(a_full + 1);
+  uint64_t* t1_full = b_empty + DT_STAGES;
+  uint64_t* t1_empty = t1_full + T1_BUFS;
+  uint64_t* t2_full = t1_empty + T1_BUFS;
+  uint64_t* t2_empty = t2_full + T2_BUFS;
+  uint64_t* a_full = t2_empty + T2_BUFS;
+  uint64_t* q_full = a_full + 1;
+  uint64_t* q_free = q_full + 2;
+  uint64_t* mom_done = q_free + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mom_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -204,18 +254,25 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_denoise_vec_tc(DenoiseTcArgs 
   if (threadIdx.x == 0) {
     for (int s = 0; s < DT_STAGES; ++s) {
       mbar_init(&b_full[s], 1);
-      mbar_init(&b_empty[s], DT_EPI_WARPS);
+      mbar_init(&b_empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&tm_full[b], 1);
-      mbar_init(&tm_empty[b], DT_EPI_WARPS);
+    for (int b = 0; b < T1_BUFS; ++b) {
+      mbar_init(&t1_full[b], 1);
+      mbar_init(&t1_empty[b], DT_EPI_WARPS);
+    }
+    for (int b = 0; b < T2_BUFS; ++b) {
+      mbar_init(&t2_full[b], 1);
+      mbar_init(&t2_empty[b], DT_EPI_WARPS);
+      mbar_init(&q_full[b], DT_EPI_WARPS);
+      mbar_init(&q_free[b], 1);
     }
     mbar_init(a_full, DT_M);
+    mbar_init(mom_done, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
-  if (warp == DT_EPI_WARPS) {
+  if (warp == MMA_WARP) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(tmem_slot)),
                  "r"(DT_TMEM_COLS));
@@ -226,9 +283,10 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_denoise_vec_tc(DenoiseTcArgs 
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  // Counters shared by all roles: `seq` counts codebook tiles (stage ring),
-  // `tu` counts TMEM buffer uses (one per pass-1 tile, two per pass-2 tile).
-  if (warp == DT_EPI_WARPS + 1) {
+  // Counters every role keeps in step: `seq` codebook tiles (stage ring),
+  // `tu1` pass-1 tiles (4 TMEM buffers), `hq` pass-2 halves (2 TMEM buffers
+  // and 2 weights buffers), `mt_n` block tiles done (moment phases).
+  if (warp == LOAD_WARP) {
     // ------------------------------------------------------------ loader
     if (lane == 0) {
       uint32_t seq = 0;
@@ -242,10 +300,10 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_denoise_vec_tc(DenoiseTcArgs 
               ok = false;
               break;
             }
-            uint8_t* st = smem + SM_B + s * STAGE_BYTES;
-            mbar_expect_tx(&b_full[s], pass ? STAGE_BYTES : OPER_BYTES);
-            bulk_load_1d(st, a.cb_tc + (size_t)j * OPER_BYTES, OPER_BYTES, &b_full[s]);
-            if (pass) bulk_load_1d(st + OPER_BYTES, a.cb + (size_t)j * DT_N * 8, CF_BYTES, &b_full[s]);
+            const uint32_t bytes = pass ? STAGE_BYTES : OPER_BYTES;
+            mbar_expect_tx(&b_full[s], bytes);
+            bulk_load_1d(smem + SM_B + s * STAGE_BYTES, a.cb_tc + (size_t)j * STAGE_BYTES, bytes,
+                         &b_full[s]);
           }
       // the copies in flight land before the CTA may exit
       const uint32_t last = seq;
@@ -255,54 +313,107 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_denoise_vec_tc(DenoiseTcArgs 
           if (i > 256) __nanosleep(64);
       }
     }
-  } else if (warp == DT_EPI_WARPS) {
+  } else if (warp == MMA_WARP) {
     // ------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      uint32_t seq = 0, tu = 0, aphase = 0;
+      uint32_t seq = 0, tu1 = 0, hq = 0, aphase = 0;
       bool ok = true;
       const uint32_t a_base = smem_u32(At);
-      for (int64_t mt = blockIdx.x; mt < mtiles && ok; mt += gridDim.x)
-        for (int pass = 0; pass < passes && ok; ++pass) {
-          if (!wait_or_abort(a_full, aphase & 1, abort_flag, a.status)) {
-            ok = false;
+      const uint32_t qw_base = smem_u32(smem + SM_QW);
+      for (int64_t mt = blockIdx.x; mt < mtiles && ok; mt += gridDim.x) {
+        // ------------------------------------------ pass 1: scores
+        if (!(ok = wait_or_abort(a_full, aphase++ & 1, abort_flag, a.status))) break;
+        tc_fence_after();
+        for (int j = 0; j < a.NT; ++j, ++seq, ++tu1) {
+          const int s = seq % DT_STAGES, b = tu1 % T1_BUFS;
+          if (!(ok = wait_or_abort(&b_full[s], (seq / DT_STAGES) & 1, abort_flag, a.status))) break;
+          if (tu1 >= T1_BUFS &&
+              !(ok = wait_or_abort(&t1_empty[b], (tu1 / T1_BUFS - 1) & 1, abort_flag, a.status)))
             break;
-          }
-          ++aphase;
           tc_fence_after();
-          for (int j = 0; j < a.NT && ok; ++j, ++seq) {
-            const int s = seq % DT_STAGES;
-            if (!wait_or_abort(&b_full[s], (seq / DT_STAGES) & 1, abort_flag, a.status)) {
-              ok = false;
-              break;
-            }
-            const uint32_t bst = smem_u32(smem + SM_B + s * STAGE_BYTES);
-            for (int h = 0; h < pass + 1; ++h, ++tu) {
-              const int buf = tu & 1;
-              if (tu >= 2 && !wait_or_abort(&tm_empty[buf], ((tu >> 1) - 1) & 1, abort_flag, a.status)) {
-                ok = false;
-                break;
-              }
+          const uint32_t d = tmem + (uint32_t)b * T1_COLS;
+          const uint64_t bd = kmajor_desc(smem_u32(smem + SM_B + s * STAGE_BYTES), 256);
+          umma_f16(d, kmajor_desc(a_base + A1_HI * OPER_BYTES, 256), bd, IDESC_P1, 0u);
+          umma_f16(d, kmajor_desc(a_base + A1_LO * OPER_BYTES, 256), bd, IDESC_P1, 1u);
+          umma_commit(&t1_full[b]);
+          umma_commit(&b_empty[s]);
+        }
+        if (!ok || a.nearest_only) continue;
+        // ---------------------------------- pass 2: scores and moments
+        // A polling scheduler: the score MMAs of a half go out as soon as its
+        // TMEM buffer and codebook stage are ready, the moment MMAs of a half
+        // as soon as its weights are in shared memory, so neither waits on
+        // the other.
+        if (!(ok = wait_or_abort(a_full, aphase++ & 1, abort_flag, a.status))) break;
+        tc_fence_after();
+        const uint32_t total = 2u * (uint32_t)a.NT;
+        uint32_t us = 0, um = 0, idle = 0;
+        bool staged = false;
+        while (um < total) {
+          bool prog = false;
+          if (us < total) {
+            const uint32_t sq = seq + (us >> 1), u = hq + us;
+            const int s = sq % DT_STAGES, b = u % T2_BUFS;
+            if (!staged) staged = mbar_test_wait(&b_full[s], (sq / DT_STAGES) & 1);
+            if (staged && (u < T2_BUFS || mbar_test_wait(&t2_empty[b], (u / T2_BUFS - 1) & 1))) {
               tc_fence_after();
-              const uint32_t d = tmem + (uint32_t)buf * 256u;
-              if (pass == 0) {
-                const uint64_t bd = kmajor_desc(bst);
-                umma_f16(d, kmajor_desc(a_base + A1_HI * OPER_BYTES), bd, IDESC_P1, 0u);
-                umma_f16(d, kmajor_desc(a_base + A1_LO * OPER_BYTES), bd, IDESC_P1, 1u);
-              } else {
-                // codewords 64h .. 64h+63 of the tile: rows from byte 2048 h
-                const uint64_t bd = kmajor_desc(bst + (uint32_t)h * 2048u);
-                umma_f16(d, kmajor_desc(a_base + A2_Q * OPER_BYTES), bd, IDESC_P2, 0u);
-                umma_f16(d + 64u, kmajor_desc(a_base + A2_X * OPER_BYTES), bd, IDESC_P2, 0u);
-                umma_f16(d + 128u, kmajor_desc(a_base + A2_RH * OPER_BYTES), bd, IDESC_P2, 0u);
-                umma_f16(d + 128u, kmajor_desc(a_base + A2_RL * OPER_BYTES), bd, IDESC_P2, 1u);
-              }
-              umma_commit(&tm_full[buf]);
+              // codewords 64h .. 64h+63 of the tile: rows from byte 2048 h
+              const uint32_t d = tmem + (uint32_t)b * T2_COLS;
+              const uint64_t bd = kmajor_desc(smem_u32(smem + SM_B + s * STAGE_BYTES) + (us & 1) * 2048u, 256);
+              umma_f16(d, kmajor_desc(a_base + A2_Q * OPER_BYTES, 256), bd, IDESC_P2, 0u);
+              umma_f16(d + 64u, kmajor_desc(a_base + A2_X * OPER_BYTES, 256), bd, IDESC_P2, 0u);
+              umma_f16(d + 128u, kmajor_desc(a_base + A2_RH * OPER_BYTES, 256), bd, IDESC_P2, 0u);
+              umma_f16(d + 128u, kmajor_desc(a_base + A2_RL * OPER_BYTES, 256), bd, IDESC_P2, 1u);
+              umma_commit(&t2_full[b]);
+              if (++us % 2 == 0) staged = false;
+              prog = true;
             }
+          }
+          if (um < us) {
+            const uint32_t u = hq + um, qb = u % T2_BUFS;
+            if (mbar_test_wait(&q_full[qb], (u / T2_BUFS) & 1)) {
+              tc_fence_after();
+              const int s = (seq + (um >> 1)) % DT_STAGES;
+              const uint32_t wq = qw_base + qb * 2u * QW_BYTES;
+              const uint32_t bt = smem_u32(smem + SM_B + s * STAGE_BYTES + OPER_BYTES) + (um & 1) * 1024u;
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {  // weights (hi, lo) x transposed codebook
+                const uint64_t bd = kmajor_desc(bt + kk * 256u, 2048);
+                umma_f16(tmem + TM_MOM, kmajor_desc(wq + kk * 256u, 1024), bd, IDESC_MOM,
+                         (um == 0 && kk == 0) ? 0u : 1u);
+                umma_f16(tmem + TM_MOM, kmajor_desc(wq + QW_BYTES + kk * 256u, 1024), bd, IDESC_MOM, 1u);
+              }
+              umma_commit(&q_free[qb]);
+              if (um & 1) umma_commit(&b_empty[s]);  // both halves of the stage are done
+              ++um;
+              prog = true;
+            }
+          }
+          if (prog) {
+            idle = 0;
+          } else {
+            if (++idle >= (1u << 25)) {
+              atomicOr(a.status, STATUS_TIMEOUT);
+              *abort_flag = 1;
+            }
+            if ((idle & 63) == 63 && *abort_flag) break;
+            if (idle > 256) __nanosleep(32);
           }
         }
+        if (um < total) {
+          ok = false;
+          break;
+        }
+        umma_commit(mom_done);
+        seq += a.NT;
+        hq += total;
+      }
       // the MMAs in flight finish before TMEM is released
-      for (uint32_t q = (tu > 2 ? tu - 2 : 0); q < tu; ++q)
-        for (uint32_t i = 0; i < (1u << 25) && !mbar_try_wait(&tm_full[q & 1], (q >> 1) & 1); ++i)
+      for (uint32_t q = (tu1 > T1_BUFS ? tu1 - T1_BUFS : 0); q < tu1; ++q)
+        for (uint32_t i = 0; i < (1u << 25) && !mbar_try_wait(&t1_full[q % T1_BUFS], (q / T1_BUFS) & 1); ++i)
+          if (i > 256) __nanosleep(64);
+      for (uint32_t q = (hq > T2_BUFS ? hq - T2_BUFS : 0); q < hq; ++q)
+        for (uint32_t i = 0; i < (1u << 25) && !mbar_try_wait(&q_free[q % T2_BUFS], (q / T2_BUFS) & 1); ++i)
           if (i > 256) __nanosleep(64);
     }
   } else {
@@ -313,16 +424,19 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_denoise_vec_tc(DenoiseTcArgs 
     const int wg = warp >> 2, qd = warp & 3;
     const int rl = qd * 32 + lane;  // row of the tile this thread owns
     const uint32_t t_lane = tmem + ((uint32_t)(qd * 32) << 16);
-    uint32_t seq = 0, tu = 0;
+    uint8_t* qw = smem + SM_QW;
+    const int w_off = kmaj_off(rl, wg * 16, 1024);  // this thread's 16 weights of a half
+    uint32_t tu1 = 0, hq = 0, mt_n = 0;
     bool ok = true;
     for (int64_t mt = blockIdx.x; mt < mtiles; mt += gridDim.x) {
       const int64_t blk = mt * DT_M + rl;
       const bool active = blk < a.nblocks;
       const int64_t row = active ? blk / a.B : 0;
-      double t64[8];
-      float g = 0.0f;
       if (wg == 0) {
-        // t = r1 / s (with the anchor: precision-weighted with w / s)
+        // t = r1 / s (with the anchor: precision-weighted with w / s); kept in
+        // shared memory across pass 1 to spare registers
+        double t64[8];
+        float g = 0.0f;
 #pragma unroll
         for (int i = 0; i < 8; ++i) t64[i] = 0.0;
         if (active) {
@@ -355,6 +469,9 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_denoise_vec_tc(DenoiseTcArgs 
         hi[8] = hi[9] = __float2half(-32.0f);
         store_row(At + A1_HI * OPER_BYTES, rl, hi);
         store_row(At + A1_LO * OPER_BYTES, rl, lo);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) sm_t[rl * 8 + i] = t64[i];
+        sm_g[rl] = g;
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         mbar_arrive(a_full);
       }
@@ -362,58 +479,42 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_denoise_vec_tc(DenoiseTcArgs 
       // ---------------------------------------------- pass 1: argmax
       float best = -INFINITY;
       int bidx = 0;
-      for (int j = 0; j < a.NT; ++j, ++seq, ++tu) {
-        const int s = seq % DT_STAGES, buf = tu & 1;
-        if (ok) ok = __all_sync(0xffffffffu, wait_or_abort(&tm_full[buf], (tu >> 1) & 1, abort_flag, a.status));
+      for (int j = 0; j < a.NT; ++j, ++tu1) {
+        const int buf = tu1 % T1_BUFS;
+        if (ok) ok = warp_wait(&t1_full[buf], (tu1 / T1_BUFS) & 1, abort_flag, a.status);
         if (!ok) continue;
         tc_fence_after();
-        uint32_t v0[32], v1[32];
-        const uint32_t ta = t_lane + (uint32_t)buf * 256u + (uint32_t)(wg * 64);
-        tmem_ld32_nowait(ta, v0);
-        tmem_ld32_nowait(ta + 32u, v1);
+        uint32_t v[32];
+        tmem_ld32_nowait(t_lane + (uint32_t)buf * T1_COLS + (uint32_t)(wg * 32), v);
         tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&tm_empty[buf]);
-          mbar_arrive(&b_empty[s]);
-        }
-        const int base = j * DT_N + wg * 64;
-        float m0 = __uint_as_float(v0[0]), m1 = __uint_as_float(v1[0]);
+        if (lane == 0) mbar_arrive(&t1_empty[buf]);
+        float m0 = __uint_as_float(v[0]);
 #pragma unroll
-        for (int k = 1; k < 32; ++k) {
-          m0 = fmaxf(m0, __uint_as_float(v0[k]));
-          m1 = fmaxf(m1, __uint_as_float(v1[k]));
-        }
+        for (int k = 1; k < 32; ++k) m0 = fmaxf(m0, __uint_as_float(v[k]));
         if (m0 > best) {  // first index of the chunk maximum
           int kk = 31;
 #pragma unroll
           for (int k = 31; k >= 0; --k)
-            if (__uint_as_float(v0[k]) == m0) kk = k;
+            if (__uint_as_float(v[k]) == m0) kk = k;
           best = m0;
-          bidx = base + kk;
-        }
-        if (m1 > best) {
-          int kk = 31;
-#pragma unroll
-          for (int k = 31; k >= 0; --k)
-            if (__uint_as_float(v1[k]) == m1) kk = k;
-          best = m1;
-          bidx = base + 32 + kk;
+          bidx = j * DT_N + wg * 32 + kk;
         }
       }
-      // merge the two column halves: larger score, then the smaller index
-      if (wg == 1) {
-        sm_bval[rl] = best;
-        sm_bidx[rl] = bidx;
-      }
+      // merge the column quarters: larger score, then the smaller index
+      sm_bval[wg * DT_M + rl] = best;
+      sm_bidx[wg * DT_M + rl] = bidx;
       named_sync_epi();
       if (wg == 0) {
-        const float ob = sm_bval[rl];
-        const int oi = sm_bidx[rl];
-        if (ob > best || (ob == best && oi < bidx)) {
-          best = ob;
-          bidx = oi;
+#pragma unroll
+        for (int w = 1; w < DT_WGS; ++w) {
+          const float ob = sm_bval[w * DT_M + rl];
+          const int oi = sm_bidx[w * DT_M + rl];
+          if (ob > best || (ob == best && oi < bidx)) {
+            best = ob;
+            bidx = oi;
+          }
         }
       }
       if (a.nearest_only) {
@@ -422,12 +523,16 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_denoise_vec_tc(DenoiseTcArgs 
       }
 
       // ---------------------------------- pass 2 operands (centred on c*)
-      float cst[8];
       if (wg == 0) {
+        float cst[8];
+        double t64[8];
         const float4 c0 = *reinterpret_cast<const float4*>(a.cb + (int64_t)bidx * 8);
         const float4 c1 = *reinterpret_cast<const float4*>(a.cb + (int64_t)bidx * 8 + 4);
         cst[0] = c0.x; cst[1] = c0.y; cst[2] = c0.z; cst[3] = c0.w;
         cst[4] = c1.x; cst[5] = c1.y; cst[6] = c1.z; cst[7] = c1.w;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) t64[i] = sm_t[rl * 8 + i];
+        const float g = sm_g[rl];
         // t - c* = q + r: q on the grid 2^-Fb with |q_i| 2^Fb <= 2047 (exact
         // fp16), Fb the finest grid up to F that holds this block's largest
         // coordinate, so |r| <= 2^-(Fb+1) stays ~2^-11 of |t - c*|.  r enters
@@ -473,99 +578,113 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_denoise_vec_tc(DenoiseTcArgs 
       }
       named_sync_epi();
       const float g2 = sm_g2[rl], rs = sm_rs[rl];
-      const int cchunk = sm_bidx[rl] >> 5, kst = sm_bidx[rl] & 31;  // c* as (32-chunk, column)
+      const int c16 = sm_bidx[rl] >> 4, kst = sm_bidx[rl] & 15;  // c* as (16-chunk, column)
 
-      // ------------------------------------------- pass 2: moments
-      float S0 = 0.0f, S2 = 0.0f, S1[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) S1[i] = 0.0f;
-      for (int j = 0; j < a.NT; ++j, ++seq) {
-        const int s = seq % DT_STAGES;
-        const float4* cf = reinterpret_cast<const float4*>(smem + SM_B + s * STAGE_BYTES + OPER_BYTES);
+      // ------------------------------------------- pass 2: weights
+      float S2 = 0.0f, zmax = -INFINITY;
+      for (int j = 0; j < a.NT; ++j) {
 #pragma unroll 1
-        for (int h = 0; h < 2; ++h, ++tu) {
-          const int buf = tu & 1;
-          if (ok) ok = __all_sync(0xffffffffu, wait_or_abort(&tm_full[buf], (tu >> 1) & 1, abort_flag, a.status));
+        for (int h = 0; h < 2; ++h, ++hq) {
+          const int buf = hq % T2_BUFS, qb = buf;
+          if (ok) ok = warp_wait(&t2_full[buf], (hq / T2_BUFS) & 1, abort_flag, a.status);
           if (!ok) continue;
           tc_fence_after();
-          const uint32_t ta = t_lane + (uint32_t)buf * 256u + (uint32_t)(wg * 32);
-          uint32_t Q[32], X[32], R[32];
-          tmem_ld32_nowait(ta, Q);
-          tmem_ld32_nowait(ta + 64u, X);
-          tmem_ld32_nowait(ta + 128u, R);
+          const uint32_t ta = t_lane + (uint32_t)buf * T2_COLS + (uint32_t)(wg * 16);
+          uint32_t Q[16], X[16], R[16];
+          tmem_ld16_nowait(ta, Q);
+          tmem_ld16_nowait(ta + 64u, X);
+          tmem_ld16_nowait(ta + 128u, R);
           tmem_wait_ld();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&tm_empty[buf]);
-          float z[32];
+          if (lane == 0) mbar_arrive(&t2_empty[buf]);
+          // c* needs no special case here: X(c*) = 0 exactly, so it adds
+          // nothing to S2, and its weight is zeroed in the moment operand
+          // below.  (Its logit is 0 up to R's rounding, so z(c*) reaches the
+          // overflow mark only at g > ~5e9, where the point mass on c* that
+          // the overflow fallback returns is the answer.)
+          float q[16];
 #pragma unroll
-          for (int k = 0; k < 32; ++k)  // Q + X is exact; R carries the rounding
-            z[k] = g2 * fmaf(__uint_as_float(R[k]), rs, __uint_as_float(Q[k]) + __uint_as_float(X[k]));
-          // the argmax column (weight exactly 1) is left out of the sums and
-          // added back at the end, so that the moments come out centred on c*
-          if (j * 4 + h * 2 + wg == cchunk) {
-#pragma unroll
-            for (int k = 0; k < 32; ++k)
-              if (k == kst) z[k] = -INFINITY;
+          for (int k = 0; k < 16; ++k) {  // Q + X is exact; R carries the rounding
+            const float z = fmaf(g2, fmaf(__uint_as_float(R[k]), rs, __uint_as_float(Q[k]) + __uint_as_float(X[k])),
+                                 Q_SHIFT);
+            zmax = fmaxf(zmax, z);
+            q[k] = ex2_approx(z);
+            S2 = fmaf(q[k], __uint_as_float(X[k]), S2);  // X = -|c - c*|^2 / 2
           }
-          const float4* cc = cf + (h * 64 + wg * 32) * 2;
+          uint32_t hi[8], lo[8];
 #pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            const float q = ex2_approx(z[k]);
-            S0 += q;
-            S2 = fmaf(q, __uint_as_float(X[k]), S2);  // X = -|c - c*|^2 / 2
-            const float4 ca = cc[2 * k], cb = cc[2 * k + 1];
-            S1[0] = fmaf(q, ca.x, S1[0]);
-            S1[1] = fmaf(q, ca.y, S1[1]);
-            S1[2] = fmaf(q, ca.z, S1[2]);
-            S1[3] = fmaf(q, ca.w, S1[3]);
-            S1[4] = fmaf(q, cb.x, S1[4]);
-            S1[5] = fmaf(q, cb.y, S1[5]);
-            S1[6] = fmaf(q, cb.z, S1[6]);
-            S1[7] = fmaf(q, cb.w, S1[7]);
+          for (int p = 0; p < 8; ++p) split_pair(q[2 * p], q[2 * p + 1], hi[p], lo[p]);
+          // the moment MMAs of two halves ago have read this buffer
+          if (hq >= 2) ok = warp_wait(&q_free[qb], ((hq >> 1) - 1) & 1, abort_flag, a.status);
+          if (!ok) continue;
+          uint8_t* wb = qw + qb * 2 * QW_BYTES + w_off;
+          *reinterpret_cast<uint4*>(wb) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+          *reinterpret_cast<uint4*>(wb + 128) = make_uint4(hi[4], hi[5], hi[6], hi[7]);
+          *reinterpret_cast<uint4*>(wb + QW_BYTES) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+          *reinterpret_cast<uint4*>(wb + QW_BYTES + 128) = make_uint4(lo[4], lo[5], lo[6], lo[7]);
+          if (j * 8 + h * 4 + wg == c16) {  // c* is in this chunk: weight 0 (added back at the end)
+            const int o = (kst >> 3) * 128 + (kst & 7) * 2;
+            *reinterpret_cast<uint16_t*>(wb + o) = 0;
+            *reinterpret_cast<uint16_t*>(wb + QW_BYTES + o) = 0;
           }
-        }
-        if (ok) {
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
           __syncwarp();
-          if (lane == 0) mbar_arrive(&b_empty[s]);
+          if (lane == 0) mbar_arrive(&q_full[qb]);
         }
       }
-      if (wg == 1) {
-        float* pp = sm_part + rl * 10;
-        pp[0] = S0;
-        pp[1] = S2;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) pp[2 + i] = S1[i];
-      }
+      sm_s2[wg * DT_M + rl] = S2;
+      sm_bval[wg * DT_M + rl] = zmax;
       named_sync_epi();
-      if (wg == 0 && active && ok) {
-        // S0, S1, S2 hold the codewords other than c* (weight 1, X = 0):
-        // E[c - c*] = (S1 - c* S0) / (1 + S0), E|c - c*|^2 = -2 S2 / (1 + S0)
-        const float* pp = sm_part + rl * 10;
-        S0 += pp[0];
-        S2 += pp[1];
-        const float sc = a.scale[row], off = a.offset[row];
-        const float inv = 1.0f / (1.0f + S0);
-        const bool point = !(S0 < INFINITY) && S0 == S0;  // overflow: point mass on c*
-        float mm = 0.0f, xo[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float mc = point ? 0.0f : fmaf(-cst[i], S0, S1[i] + pp[2 + i]) * inv;
-          mm = fmaf(mc, mc, mm);
-          xo[i] = fmaf(sc, cst[i] + mc, off);
+      if (wg == 0) {
+        // S0 = sum q, S1 = sum q c over c != c* (weights x 2^8) from the
+        // moment accumulator; c* adds 2^8 to S0, 2^8 c* to S1 and 0 to S2:
+        // E[c - c*] = (S1 - c* S0) / (2^8 + S0), E|c - c*|^2 = -2 S2 / (2^8 + S0)
+        if (ok) ok = warp_wait(mom_done, mt_n & 1, abort_flag, a.status);
+        uint32_t mv[16];
+        if (ok) {
+          tc_fence_after();
+          tmem_ld16_nowait(t_lane + TM_MOM, mv);
+          tmem_wait_ld();
+          tc_fence_before();
         }
-        *reinterpret_cast<float4*>(a.xhat + blk * 8) = make_float4(xo[0], xo[1], xo[2], xo[3]);
-        *reinterpret_cast<float4*>(a.xhat + blk * 8 + 4) = make_float4(xo[4], xo[5], xo[6], xo[7]);
-        // E|c - c*|^2 - |E c - c*|^2
-        const float var = point ? 0.0f : fmaxf(-2.0f * S2 * inv - mm, 0.0f);
-        a.vblock[blk] = (float)((double)sc * sc * var);
-        if (a.idx) a.idx[blk] = (uint16_t)bidx;
+        if (active && ok) {
+          const int bi = sm_bidx[rl];
+          const float4 c0 = *reinterpret_cast<const float4*>(a.cb + (int64_t)bi * 8);
+          const float4 c1 = *reinterpret_cast<const float4*>(a.cb + (int64_t)bi * 8 + 4);
+          const float cst[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+          float s2 = 0.0f, zm = -INFINITY;
+#pragma unroll
+          for (int w = 0; w < DT_WGS; ++w) {
+            s2 += sm_s2[w * DT_M + rl];
+            zm = fmaxf(zm, sm_bval[w * DT_M + rl]);
+          }
+          const float S0 = __uint_as_float(mv[8]);
+          const float sc = a.scale[row], off = a.offset[row];
+          const float inv = 1.0f / (256.0f + S0);
+          // a weight past the fp16 range (logit 2^7 above c*'s): point mass
+          const bool point = zm >= 15.99f;
+          float mm = 0.0f, xo[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float mc = point ? 0.0f : fmaf(-cst[i], S0, __uint_as_float(mv[i])) * inv;
+            mm = fmaf(mc, mc, mm);
+            xo[i] = fmaf(sc, cst[i] + mc, off);
+          }
+          *reinterpret_cast<float4*>(a.xhat + blk * 8) = make_float4(xo[0], xo[1], xo[2], xo[3]);
+          *reinterpret_cast<float4*>(a.xhat + blk * 8 + 4) = make_float4(xo[4], xo[5], xo[6], xo[7]);
+          // E|c - c*|^2 - |E c - c*|^2
+          const float var = point ? 0.0f : fmaxf(-2.0f * s2 * inv - mm, 0.0f);
+          a.vblock[blk] = (float)((double)sc * sc * var);
+          if (a.idx) a.idx[blk] = (uint16_t)bi;
+        }
       }
+      ++mt_n;
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == DT_EPI_WARPS) {
+  if (warp == MMA_WARP) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                  "r"(DT_TMEM_COLS));
@@ -617,26 +736,31 @@ int vec_tc_grid_bits(const float* cb_host, int K, int* e_out, int* rk_out) {
   return -1;
 }
 
-// Codebook operand images: per tile of 128 codewords, row r holds
-// [c_0 .. c_7 | n_hi n_lo 1 1 0 0 0 0] (|c|^2 = n_hi + n_lo) in fp16 in the
-// no-swizzle K-major layout the kernel's descriptors describe.
+// Codebook operand images, 8 KiB per tile of 128 codewords, in the no-swizzle
+// K-major layout the kernel's descriptors describe:
+//   scores      128 rows (codewords) x 16: [c_0 .. c_7 | n_hi n_lo 1 1 0 0 0 0],
+//               |c|^2 = n_hi + n_lo  (8-row groups 256 B apart)
+//   moments     16 rows x 128 (codewords): rows 0-7 the coordinates, row 8 ones
+//               (8-row groups 2048 B apart)
 mpq_status build_vec_tc_tables(mpq_plan_s* p, const float* cb_host) {
   const int NT = p->K / DT_N;
-  std::vector<__half> img((size_t)NT * OPER_BYTES / 2, __float2half(0.0f));
+  std::vector<__half> img((size_t)NT * STAGE_BYTES / 2, __float2half(0.0f));
   for (int c = 0; c < p->K; ++c) {
     const int j = c / DT_N, r = c % DT_N;
-    __half* t = img.data() + (size_t)j * OPER_BYTES / 2;
+    __half* sc = img.data() + (size_t)j * STAGE_BYTES / 2;
+    __half* mo = sc + OPER_BYTES / 2;
     double nn = 0.0;
     for (int i = 0; i < 8; ++i) {
       const float v = cb_host[(size_t)c * 8 + i];
-      t[oper_off(r, 0) / 2 + i] = __float2half(v);
+      sc[kmaj_off(r, i, 256) / 2] = __float2half(v);
+      mo[kmaj_off(i, r, 2048) / 2] = __float2half(v);
       nn += (double)v * v;
     }
     const __half nh = __double2half(nn);
-    __half* k1 = t + oper_off(r, 1) / 2;
-    k1[0] = nh;
-    k1[1] = __double2half(nn - (double)__half2float(nh));
-    k1[2] = k1[3] = __float2half(1.0f);
+    sc[kmaj_off(r, 8, 256) / 2] = nh;
+    sc[kmaj_off(r, 9, 256) / 2] = __double2half(nn - (double)__half2float(nh));
+    sc[kmaj_off(r, 10, 256) / 2] = sc[kmaj_off(r, 11, 256) / 2] = __float2half(1.0f);
+    mo[kmaj_off(8, r, 2048) / 2] = __float2half(1.0f);
   }
   MPQ_CUDA(cudaMalloc(&p->cb_tc, img.size() * sizeof(__half)));
   MPQ_CUDA(cudaMemcpy(p->cb_tc, img.data(), img.size() * sizeof(__half), cudaMemcpyHostToDevice));
@@ -658,6 +782,12 @@ mpq_status launch_denoise_vec_tc(const mpq_plan_s* p, const float* R1, const dou
   }
   int sms = 0;
   MPQ_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  cudaFuncAttributes fa{};
+  MPQ_CUDA(cudaFuncGetAttributes(&fa, k_denoise_vec_tc));
+  if (fa.maxThreadsPerBlock < DT_THREADS)
+    return fail(MPQ_ERR_CUDA, "k_denoise_vec_tc: " + std::to_string(fa.numRegs) +
+                                  " registers/thread allow only " +
+                                  std::to_string(fa.maxThreadsPerBlock) + " threads per block");
   DenoiseTcArgs a{};
   a.R1 = R1;
   a.gamma1 = gamma1;
