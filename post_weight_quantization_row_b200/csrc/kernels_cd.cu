@@ -147,22 +147,29 @@ __global__ void __launch_bounds__(CD1_WARPS * 32)
 }
 
 // ------------------------------------------------------------------ d = 8 --
-// Per block step b (all rows together): score(c) = qtab_b(c) - c . g'/1,
+// Per block step b (all rows together): score(c) = qtab_b(c) - c . g',
 // with qtab_b(c) = 1/2 c^T G_b c, g' = (h_b + G_b x_b)/scale; the energy
 // change of codeword c is scale^2 (score(c) - score(c_cur)).
+// A sweep visits the blocks in tiles of CD_TILE columns (16 blocks), like the
+// scalar path: within a tile the gradient lives in a tile-local copy hl that
+// the apply step updates with H[tile, block]; the tile's changes leave as
+// Delta/scale = c_new - c_old in the A operand of the tensor-core update
+// h += (-scale) Delta H[tile, :] over all columns, run once per tile.
 // Kernel A: partial argmin over a chunk of codewords for a tile of rows.
-// Kernel B: combine chunks, accept if strictly better, update idx and h.
-constexpr int CD8_ROWS = 64;    // rows per CTA (8 warps x 8 rows)
-constexpr int CD8_CHUNK = 1024; // codewords per CTA
+// Kernel B: combine chunks, accept if strictly better, update idx, hl, Delta.
+constexpr int CD8_ROWS = 256;   // rows per eval CTA (8 warps x 4 groups of 8 rows)
+constexpr int CD8_CHUNK = 1024; // codewords per eval CTA
+constexpr int CD8_APPLY_WARPS = 16;
 
 __device__ __forceinline__ bool row_active(const int32_t* changes, int64_t row, int sweeps,
                                            int sw) {
   return sw == 0 || changes[row * sweeps + sw - 1] > 0;
 }
 
-// g' for one row at block b; G_b and x_b in weight units.
+// g' for one row at block b from the block's 8 gradient entries hb; G_b and
+// x_b in weight units.
 __device__ __forceinline__ void block_gradient(const float* __restrict__ H, int64_t n,
-                                               const float* __restrict__ hrow,
+                                               const float* __restrict__ hb,
                                                const float* __restrict__ cb, int kcur,
                                                float sc, int64_t b, float* gout) {
   float x[8];
@@ -170,7 +177,7 @@ __device__ __forceinline__ void block_gradient(const float* __restrict__ H, int6
   for (int j = 0; j < 8; ++j) x[j] = sc * cb[(int64_t)kcur * 8 + j];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    float g = hrow[8 * b + i];
+    float g = hb[i];
     const float* Hi = H + (8 * b + i) * n + 8 * b;
 #pragma unroll
     for (int j = 0; j < 8; ++j) g = fmaf(Hi[j], x[j], g);
@@ -178,144 +185,184 @@ __device__ __forceinline__ void block_gradient(const float* __restrict__ H, int6
   }
 }
 
+// the block's current gradient: h itself at the first block of a tile, else
+// the tile-local copy (h at the tile start plus the tile's own updates)
+__device__ __forceinline__ const float* block_h(const float* h, int64_t ldh, const float* hl,
+                                                int64_t row, int64_t b, int64_t t0) {
+  return (8 * b == t0) ? h + row * ldh + 8 * b : hl + row * CD_TILE + (8 * b - t0);
+}
+
 __global__ void __launch_bounds__(256)
-    k_cd_vec_eval(int64_t m, int64_t n, int K, int64_t b, const float* __restrict__ cb,
+    k_cd_vec_eval(int64_t m, int64_t n, int K, int64_t b, int64_t t0, const float* __restrict__ cb,
                   const float* __restrict__ qtab, const float* __restrict__ H,
                   const float* __restrict__ scale, const uint16_t* __restrict__ idx,
-                  const float* __restrict__ h, int64_t ldh, int sweeps, int sw,
-                  const int32_t* __restrict__ changes, float* __restrict__ part_val,
-                  int* __restrict__ part_idx, int nchunks) {
-  __shared__ float scb[CD8_CHUNK][8];
+                  const float* __restrict__ h, int64_t ldh, const float* __restrict__ hl,
+                  int sweeps, int sw, const int32_t* __restrict__ changes,
+                  float* __restrict__ part_val, int* __restrict__ part_idx, int nchunks) {
+  __shared__ float scb[8][CD8_CHUNK];  // transposed: lanes read consecutive codewords
   __shared__ float sq[CD8_CHUNK];
   __shared__ float sg[CD8_ROWS][8];
+  __shared__ int sact[CD8_ROWS / 8];   // row groups with an active row
   const int64_t B = n / 8;
   const int chunk = blockIdx.x;
   const int64_t r0 = (int64_t)blockIdx.y * CD8_ROWS;
   const int c0 = chunk * CD8_CHUNK;
   const int cn = min(CD8_CHUNK, K - c0);
-  for (int e = threadIdx.x; e < cn * 8; e += blockDim.x) scb[e / 8][e % 8] = cb[(int64_t)c0 * 8 + e];
+  for (int e = threadIdx.x; e < cn * 8; e += blockDim.x) scb[e % 8][e / 8] = cb[(int64_t)c0 * 8 + e];
   for (int e = threadIdx.x; e < cn; e += blockDim.x) sq[e] = qtab[b * K + c0 + e];
-  if (threadIdx.x < CD8_ROWS) {
-    const int64_t row = r0 + threadIdx.x;
+  if (threadIdx.x < CD8_ROWS / 8) sact[threadIdx.x] = 0;
+  __syncthreads();
+  for (int rl = threadIdx.x; rl < CD8_ROWS; rl += blockDim.x) {
+    const int64_t row = r0 + rl;
     const bool act = row < m && row_active(changes, row, sweeps, sw);
     if (act) {
       float g[8];
-      block_gradient(H, n, h + row * ldh, cb, idx[row * B + b], scale[row], b, g);
+      block_gradient(H, n, block_h(h, ldh, hl, row, b, t0), cb, idx[row * B + b], scale[row], b, g);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) sg[threadIdx.x][i] = g[i];
+      for (int i = 0; i < 8; ++i) sg[rl][i] = g[i];
+      sact[rl / 8] = 1;
     } else {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) sg[threadIdx.x][i] = 0.0f;
+      for (int i = 0; i < 8; ++i) sg[rl][i] = 0.0f;
     }
   }
   __syncthreads();
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;  // warp w: rows 8w..8w+7
-  float g[8][8];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  // warp w takes row groups w, w + 8, ... of 8 rows; the lanes split the codewords
+  for (int grp = w; grp < CD8_ROWS / 8; grp += 8) {
+    if (!sact[grp]) continue;
+    float g[8][8];
 #pragma unroll
-  for (int rr = 0; rr < 8; ++rr)
+    for (int rr = 0; rr < 8; ++rr)
 #pragma unroll
-    for (int i = 0; i < 8; ++i) g[rr][i] = sg[8 * w + rr][i];
-  float best[8];
-  int bidx[8];
-#pragma unroll
-  for (int rr = 0; rr < 8; ++rr) {
-    best[rr] = INFINITY;
-    bidx[rr] = 0x7fffffff;
-  }
-  for (int c = lane; c < cn; c += 32) {
-    float cv[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) cv[i] = scb[c][i];
-    const float q = sq[c];
+      for (int i = 0; i < 8; ++i) g[rr][i] = sg[8 * grp + rr][i];
+    float best[8];
+    int bidx[8];
 #pragma unroll
     for (int rr = 0; rr < 8; ++rr) {
-      float s = q;
+      best[rr] = INFINITY;
+      bidx[rr] = 0x7fffffff;
+    }
+    for (int c = lane; c < cn; c += 32) {
+      float cv[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) s = fmaf(-cv[i], g[rr][i], s);
-      if (s < best[rr]) {
-        best[rr] = s;
-        bidx[rr] = c0 + c;
+      for (int i = 0; i < 8; ++i) cv[i] = scb[i][c];
+      const float q = sq[c];
+#pragma unroll
+      for (int rr = 0; rr < 8; ++rr) {
+        float s = q;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) s = fmaf(-cv[i], g[rr][i], s);
+        if (s < best[rr]) {
+          best[rr] = s;
+          bidx[rr] = c0 + c;
+        }
       }
     }
-  }
-  // warp argmin per row, lowest index on ties
+    // warp argmin per row, lowest index on ties
 #pragma unroll
-  for (int rr = 0; rr < 8; ++rr) {
-    float v = best[rr];
-    int k = bidx[rr];
+    for (int rr = 0; rr < 8; ++rr) {
+      float v = best[rr];
+      int k = bidx[rr];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float v2 = __shfl_xor_sync(0xffffffffu, v, o);
-      const int k2 = __shfl_xor_sync(0xffffffffu, k, o);
-      if (v2 < v || (v2 == v && k2 < k)) {
-        v = v2;
-        k = k2;
+      for (int o = 16; o > 0; o >>= 1) {
+        const float v2 = __shfl_xor_sync(0xffffffffu, v, o);
+        const int k2 = __shfl_xor_sync(0xffffffffu, k, o);
+        if (v2 < v || (v2 == v && k2 < k)) {
+          v = v2;
+          k = k2;
+        }
       }
-    }
-    const int64_t row = r0 + 8 * w + rr;
-    if (lane == 0 && row < m) {
-      part_val[row * nchunks + chunk] = v;
-      part_idx[row * nchunks + chunk] = k;
+      const int64_t row = r0 + 8 * grp + rr;
+      if (lane == 0 && row < m) {
+        part_val[row * nchunks + chunk] = v;
+        part_idx[row * nchunks + chunk] = k;
+      }
     }
   }
 }
 
-__global__ void __launch_bounds__(256)
-    k_cd_vec_apply(int64_t m, int64_t n, int K, int64_t b, const float* __restrict__ cb,
-                   const float* __restrict__ qtab, const float* __restrict__ H,
-                   const float* __restrict__ scale, uint16_t* __restrict__ idx,
-                   float* __restrict__ h, int64_t ldh, int sweeps, int sw,
-                   int32_t* __restrict__ changes,
+// One warp per row.  At the first block of a tile every row (active or not)
+// clears its Delta row and copies h[tile] into hl.
+__global__ void __launch_bounds__(CD8_APPLY_WARPS * 32)
+    k_cd_vec_apply(int64_t m, int64_t n, int K, int64_t b, int64_t t0, int tw, int tile,
+                   int ntiles, const float* __restrict__ cb, const float* __restrict__ qtab,
+                   const float* __restrict__ H, const float* __restrict__ scale,
+                   uint16_t* __restrict__ idx, const float* __restrict__ h, int64_t ldh,
+                   float* __restrict__ hl, int sweeps, int sw, int32_t* __restrict__ changes,
                    const float* __restrict__ part_val, const int* __restrict__ part_idx,
-                   int nchunks) {
-  __shared__ float sdelta[8];
-  __shared__ int sdo;
-  const int64_t row = blockIdx.x;
+                   int nchunks, __half* __restrict__ dhi, __half* __restrict__ dlo, int64_t lda,
+                   float* __restrict__ d_unscale, int* __restrict__ tile_count) {
+  __shared__ float sHb[CD_TILE][8];  // H[tile, block b]
   const int64_t B = n / 8;
-  if (!row_active(changes, row, sweeps, sw)) {
-    if (threadIdx.x == 0 && b == 0) changes[row * sweeps + sw] = 0;
-    return;
-  }
-  if (threadIdx.x == 0) {
-    if (b == 0) changes[row * sweeps + sw] = 0;
-    float v = INFINITY;
-    int k = 0x7fffffff;
-    for (int c = 0; c < nchunks; ++c) {
-      const float v2 = part_val[row * nchunks + c];
-      const int k2 = part_idx[row * nchunks + c];
-      if (v2 < v || (v2 == v && k2 < k)) {
-        v = v2;
-        k = k2;
-      }
-    }
-    const int kcur = idx[row * B + b];
-    const float sc = scale[row];
-    float g[8];
-    block_gradient(H, n, h + row * ldh, cb, kcur, sc, b, g);
-    float scur = qtab[b * K + kcur];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) scur = fmaf(-cb[(int64_t)kcur * 8 + i], g[i], scur);
-    const bool accept = (v < scur) && k >= 0 && k < K;
-    sdo = accept;
-    if (accept) {
-      idx[row * B + b] = (uint16_t)k;
-      changes[row * sweeps + sw] += 1;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) sdelta[i] = sc * (cb[(int64_t)k * 8 + i] - cb[(int64_t)kcur * 8 + i]);
-    }
-  }
+  const bool first = 8 * b == t0;
+  for (int e = threadIdx.x; e < tw * 8; e += blockDim.x)
+    sHb[e / 8][e % 8] = H[(t0 + e / 8) * n + 8 * b + e % 8];
   __syncthreads();
-  if (!sdo) return;
-  float dl[8];
+  const int lane = threadIdx.x & 31;
+  const int64_t row = (int64_t)blockIdx.x * CD8_APPLY_WARPS + (threadIdx.x >> 5);
+  if (row >= m) return;
+  float* hlr = hl + row * CD_TILE;
+  const float sc = scale[row];
+  if (first) {
+    for (int i = lane; i < CD_TILE; i += 32) {
+      dhi[row * lda + i] = __float2half_rn(0.0f);
+      dlo[row * lda + i] = __float2half_rn(0.0f);
+      hlr[i] = i < tw ? h[row * ldh + t0 + i] : 0.0f;
+    }
+    if (lane == 0) d_unscale[row] = -sc;
+  }
+  if (!row_active(changes, row, sweeps, sw)) return;
+  // combine the chunk minima (lowest index on ties)
+  float v = INFINITY;
+  int k = 0x7fffffff;
+  for (int c = lane; c < nchunks; c += 32) {
+    const float v2 = part_val[row * nchunks + c];
+    const int k2 = part_idx[row * nchunks + c];
+    if (v2 < v || (v2 == v && k2 < k)) {
+      v = v2;
+      k = k2;
+    }
+  }
 #pragma unroll
-  for (int j = 0; j < 8; ++j) dl[j] = sdelta[j];
-  float* hr = h + row * ldh;
-  for (int64_t i = threadIdx.x; i < n; i += blockDim.x) {
-    const float* Hi = H + i * n + 8 * b;
-    float acc = hr[i];
+  for (int o = 16; o > 0; o >>= 1) {
+    const float v2 = __shfl_xor_sync(0xffffffffu, v, o);
+    const int k2 = __shfl_xor_sync(0xffffffffu, k, o);
+    if (v2 < v || (v2 == v && k2 < k)) {
+      v = v2;
+      k = k2;
+    }
+  }
+  __syncwarp();  // hl of the first block is written before it is read
+  const int kcur = idx[row * B + b];
+  float g[8];
+  block_gradient(H, n, hlr + (8 * b - t0), cb, kcur, sc, b, g);
+  float scur = qtab[b * K + kcur];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) acc = fmaf(-Hi[j], dl[j], acc);
-    hr[i] = acc;
+  for (int i = 0; i < 8; ++i) scur = fmaf(-cb[(int64_t)kcur * 8 + i], g[i], scur);
+  const bool accept = (v < scur) && k >= 0 && k < K;
+  if (!accept) return;
+  float dd[8], dl[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    dd[j] = cb[(int64_t)k * 8 + j] - cb[(int64_t)kcur * 8 + j];
+    dl[j] = sc * dd[j];
+  }
+  if (lane == 0) {
+    idx[row * B + b] = (uint16_t)k;
+    changes[row * sweeps + sw] += 1;
+    tile_count[sw * ntiles + tile] = 1;  // gate of the update: some row changed
+  }
+  if (lane < 8) {  // Delta / scale as an fp16 pair (exact for lattice codebooks)
+    const __half hi = __float2half_rn(dd[lane]);
+    dhi[row * lda + 8 * b - t0 + lane] = hi;
+    dlo[row * lda + 8 * b - t0 + lane] = __float2half_rn(dd[lane] - __half2float(hi));
+  }
+  for (int i = lane; i < tw; i += 32) {
+    float acc = hlr[i];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc = fmaf(-sHb[i][j], dl[j], acc);
+    hlr[i] = acc;
   }
 }
 
@@ -365,25 +412,44 @@ mpq_status launch_cd(mpq_plan_s* p, const float* W, int64_t m, const float* scal
   int* part_idx = nullptr;
   MPQ_CUDA(cudaMallocAsync(&part_val, sizeof(float) * m * nchunks, st));
   MPQ_CUDA(cudaMallocAsync(&part_idx, sizeof(int) * m * nchunks, st));
-  const int64_t B = p->n / 8;
+  Workspace& w = p->ws;
+  const int64_t n = p->n;
+  const int nt = (int)cdiv(n, CD_TILE);
+  float* hl = w.Hl;  // m x CD_TILE tile-local gradient
+  MPQ_CUDA(cudaMemsetAsync(w.tile_count, 0, sizeof(int) * sweeps * nt, st));
   mpq_status rc = MPQ_OK;
   for (int sw = 0; sw < sweeps && rc == MPQ_OK; ++sw) {
-    for (int64_t b = 0; b < B; ++b) {
-      dim3 ga((unsigned)nchunks, (unsigned)cdiv(m, CD8_ROWS));
-      {
-        ProfScope ps_("k_cd_vec_eval", st);
-        k_cd_vec_eval<<<ga, 256, 0, st>>>(m, p->n, p->K, b, p->cb, p->qtab, p->H32, scale, idx, h,
-                                          ldh, sweeps, sw, changes, part_val, part_idx, nchunks);
+    for (int j = 0; j < nt && rc == MPQ_OK; ++j) {
+      const int64_t t0 = (int64_t)j * CD_TILE;
+      const int tw = (int)std::min<int64_t>(CD_TILE, n - t0);
+      for (int64_t b = t0 / 8; b < (t0 + tw) / 8; ++b) {
+        dim3 ga((unsigned)nchunks, (unsigned)cdiv(m, CD8_ROWS));
+        {
+          ProfScope ps_("k_cd_vec_eval", st);
+          k_cd_vec_eval<<<ga, 256, 0, st>>>(m, n, p->K, b, t0, p->cb, p->qtab, p->H32, scale, idx,
+                                            h, ldh, hl, sweeps, sw, changes, part_val, part_idx,
+                                            nchunks);
+        }
+        {
+          ProfScope ps_("k_cd_vec_apply", st);
+          k_cd_vec_apply<<<(unsigned)cdiv(m, CD8_APPLY_WARPS), CD8_APPLY_WARPS * 32, 0, st>>>(
+              m, n, p->K, b, t0, tw, j, nt, p->cb, p->qtab, p->H32, scale, idx, h, ldh, hl,
+              sweeps, sw, changes, part_val, part_idx, nchunks, w.As.hi, w.As.lo, w.As.ld,
+              w.As.row_unscale, w.tile_count);
+        }
+        count_launch(2);
+        rc = check_launch("k_cd_vec");
+        if (rc != MPQ_OK) break;
       }
-      {
-        ProfScope ps_("k_cd_vec_apply", st);
-        k_cd_vec_apply<<<(unsigned)m, 256, 0, st>>>(m, p->n, p->K, b, p->cb, p->qtab, p->H32,
-                                                    scale, idx, h, ldh, sweeps, sw, changes,
-                                                    part_val, part_idx, nchunks);
-      }
-      count_launch(2);
-      rc = check_launch("k_cd_vec");
       if (rc != MPQ_OK) break;
+      GemmOpts o;
+      o.b_k0 = t0;
+      o.accumulate = true;
+      o.a_exact = p->vec_tc;  // c_new - c_old is exact in fp16 for lattice codebooks
+      o.gate = w.tile_count + sw * nt + j;
+      o.c_reduce = (h == w.Hg) ? &w.tm_hg : nullptr;
+      rc = gemm_tc(w.As, w.tm_at_hi, w.tm_at_lo, p->H_s, p->tm_h_hi, p->tm_h_lo, h, ldh, m, n, tw,
+                   p->H_s.unscale_host, p->status, st, "gemm_cd_update", o);
     }
   }
   cudaFreeAsync(part_val, st);

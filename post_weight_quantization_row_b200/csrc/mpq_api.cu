@@ -181,6 +181,7 @@ void free_workspace(Workspace& w) {
   free_split(w.As);
   dfree(w.tile_count);
   dfree(w.Hg);
+  dfree(w.Hl);
   dfree(w.scale); dfree(w.offset); dfree(w.gamma1); dfree(w.gamma1_0); dfree(w.gamma2);
   dfree(w.beta); dfree(w.vsum); dfree(w.coef); dfree(w.kappa); dfree(w.clamps); dfree(w.W); dfree(w.w_hat);
   dfree(w.energy); dfree(w.idx_stage);
@@ -193,7 +194,7 @@ constexpr int MAX_SWEEPS = 64;
 int64_t ws_bytes_per_row(const mpq_plan_s* p) {
   return 3 * p->n * 4 + round_up(p->n, 32) * 4 + p->r * 4 +
          4 * round_up(std::max<int64_t>(std::max(p->n, p->r), CD_TILE), 64) + p->B * 2 + 3 * 4 +
-         8 * 8 + 4 + MAX_SWEEPS * 4;
+         8 * 8 + 4 + MAX_SWEEPS * 4 + (p->d == 8 ? CD_TILE * 4 : 0);
 }
 
 // changes buffer rides in the tail of `clamps`: rows x (1 + MAX_SWEEPS) ints
@@ -214,6 +215,7 @@ mpq_status ensure_workspace(mpq_plan_s* p, int64_t rows) {
   chk(dalloc(&w.tile_count, (int64_t)MAX_SWEEPS * cdiv(p->n, CD_TILE)));
   w.ldh = round_up(p->n, 32);
   chk(dalloc(&w.Hg, round_up(std::max<int64_t>(rows, 32), 32) * w.ldh));
+  if (p->d == 8) chk(dalloc(&w.Hl, rows * CD_TILE));
   if (st == MPQ_OK)
     chk(make_tmap_f32_out(&w.tm_hg, w.Hg, std::max<int64_t>(p->n, 32),
                           round_up(std::max<int64_t>(rows, 32), 32), w.ldh));

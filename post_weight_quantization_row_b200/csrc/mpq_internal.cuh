@@ -76,6 +76,7 @@ struct Workspace {
   float* Hg = nullptr;
   int64_t ldh = 0;
   CUtensorMap tm_hg;               // reduce-add target of the CD updates
+  float* Hl = nullptr;             // d = 8 CD: rows x CD_TILE tile-local gradient
   // m x r fp32
   float* P = nullptr;
   // m x B
