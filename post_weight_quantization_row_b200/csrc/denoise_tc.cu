@@ -31,10 +31,10 @@
 // to shared memory as fp16 hi/lo pairs and one more MMA (N = 16) against the
 // transposed codebook [c_0 .. c_7, 1] accumulates S1 and S0 in TMEM for the
 // whole 128-block tile; only S2 = sum q X (the centred second moment, -1/2
-// |c - c*|^2 per codeword) and the exponential stay on the ALU.  A logit
-// above c*'s by 2^7 (the argmax pass's fp32 scores misjudged a near-tie at
-// an enormous g) would overflow the fp16 weights: the tile falls back to the
-// point mass on c*.
+// |c - c*|^2 per codeword) and the exponential stay on the ALU.  A weight
+// more than 2^8 times c*'s (the argmax pass's fp32 scores misjudged a
+// near-tie at an enormous g) would overflow the fp16 weights: that block
+// falls back to the point mass on c*.
 //
 // Pipeline.  One tile is 128 blocks x 128 codewords.  The block operands are
 // written by the epilogue threads into shared memory in the no-swizzle
@@ -662,7 +662,7 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_denoise_vec_tc(DenoiseTcArgs 
           const float S0 = __uint_as_float(mv[8]);
           const float sc = a.scale[row], off = a.offset[row];
           const float inv = 1.0f / (256.0f + S0);
-          // a weight past the fp16 range (logit 2^7 above c*'s): point mass
+          // a weight past the fp16 range (more than 2^8 times c*'s): point mass
           const bool point = zm >= 15.99f;
           float mm = 0.0f, xo[8];
 #pragma unroll
