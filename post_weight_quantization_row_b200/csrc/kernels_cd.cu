@@ -26,7 +26,7 @@ namespace {
 // core update  h += (-scale) Delta H[tile, :]  over all columns, which also
 // reproduces the in-tile updates for the next tile and the next sweep.
 constexpr int CD1_WARPS = 16;
-constexpr int CD1_SMEM = (CD_TILE * CD_TILE + CD1_WARPS * CD_TILE) * 4 + CD1_WARPS * CD_TILE * 2;
+constexpr int CD1_SMEM = (CD_TILE * CD_TILE + CD_TILE + CD1_WARPS * CD_TILE) * 4 + CD1_WARPS * CD_TILE * 2;
 
 __global__ void __launch_bounds__(CD1_WARPS * 32)
     k_cd_tile_decide(int64_t m, int64_t n, int L, int64_t t0, int tw, int tile, int ntiles,
@@ -38,7 +38,8 @@ __global__ void __launch_bounds__(CD1_WARPS * 32)
                      int* __restrict__ tile_count) {
   extern __shared__ float cd_smem[];
   float* sH = cd_smem;                                  // H[tile, tile]
-  float* s_h_all = sH + CD_TILE * CD_TILE;              // per-warp gradient of the tile
+  float* s_rg = sH + CD_TILE * CD_TILE;                 // 1 / H_jj (0 where H_jj <= 0)
+  float* s_h_all = s_rg + CD_TILE;                      // per-warp gradient of the tile
   uint16_t* s_i_all = (uint16_t*)(s_h_all + CD1_WARPS * CD_TILE);  // per-warp indices
   // H[tile, tile] into shared memory: warp w copies rows w, w + 16, ...; all
   // of a warp's loads are issued before the first store so their latencies
@@ -63,6 +64,11 @@ __global__ void __launch_bounds__(CD1_WARPS * 32)
       for (int q = 0; q < VPL; ++q) sH[(wid0 + rr * CD1_WARPS) * CD_TILE + lane0 + 32 * q] = v[rr][q];
   }
   __syncthreads();
+  for (int j = threadIdx.x; j < CD_TILE; j += blockDim.x) {
+    const float gj = sH[j * CD_TILE + j];
+    s_rg[j] = gj > 0.0f ? 1.0f / gj : 0.0f;
+  }
+  __syncthreads();
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int64_t row = (int64_t)blockIdx.x * CD1_WARPS + wid;
   if (row >= m) return;
@@ -72,7 +78,7 @@ __global__ void __launch_bounds__(CD1_WARPS * 32)
     drow_hi[i] = __float2half_rn(0.0f);
     drow_lo[i] = __float2half_rn(0.0f);
   }
-  const float sc = scale[row];
+  const float sc = scale[row], isc = 1.0f / sc;
   if (lane == 0) d_unscale[row] = -sc;
   // a row stops after a sweep without change (its Delta row stays zero)
   if (sw > 0 && changes[row * sweeps + sw - 1] == 0) return;
@@ -99,7 +105,9 @@ __global__ void __launch_bounds__(CD1_WARPS * 32)
       // one (the grid ends when g <= 0), lowest index on ties
       int k0, k1;
       if (g > 0.0f) {
-        const float kcont = (float)kc + hj / (sc * g);
+        // (a reciprocal instead of a division moves kcont by ulps, which
+        // leaves the best integer level among the two candidates)
+        const float kcont = (float)kc + hj * (isc * s_rg[j]);
         k0 = (int)fminf(fmaxf(floorf(kcont), 0.0f), (float)(L - 1));
         k1 = min(k0 + 1, L - 1);
       } else {

@@ -213,6 +213,19 @@ __global__ void __launch_bounds__(ROW_THREADS)
   const double ga = anchored ? fmin(gamma1_0[row] * inv_tau2 * sc2, 1e30) : 0.0;
   const double geff = g + ga;
   const float A2 = (float)(-0.5 * geff * 1.4426950408889634);  // -geff/2 log2(e)
+  // Levels far from the nearest one carry no weight: with |dt| <= 1/2 (or dt
+  // pointing away from the grid at its ends) the log2-weight of level k* + dk
+  // relative to k* is at most A2 (dk^2 - |dk|), so a window of 2hw+1 levels
+  // with |A2| hw (hw+1) >= 64 drops only weights below 2^-64 of the largest
+  // (at most 2^-55 relative in the moments).  hw is uniform over the row's CTA.
+  int hw = L;  // half-width of the window
+  if (-A2 > 0.0f) {
+    const double w = ceil(0.5 * (-1.0 + sqrt(1.0 + 256.0 / (double)(-A2))));
+    hw = (int)fmin(w, (double)L);
+  }
+  // high precision (|A| > 5): the exact exponent form below, over the window
+  const bool precise = -A2 > 5.0f;
+  const int nlev = min(2 * hw + 1, L);
   const float inv_sc = (float)inv_dsc;
   const float Lm1 = (float)(L - 1);
   const float sc2f = (float)sc2;
@@ -220,50 +233,84 @@ __global__ void __launch_bounds__(ROW_THREADS)
   for (int64_t j = threadIdx.x; j < n; j += blockDim.x) {
     const int64_t o = row * n + j;
     const float r = R1[o];
-    float ks, dt;  // nearest level and the offset from it, in level units
+    // nearest level and the offset from it in level units, dt ~ dh + dl
+    // (the pair matters only in the high-precision rows)
+    float ks, dh, dl;
     if (!anchored) {
       ks = fminf(fmaxf(ceilf((r - off) * inv_sc - 0.5f), 0.0f), Lm1);
-      // r - (scale ks + offset) without rounding the level value: an
-      // error-free product and sum (Dekker / Knuth) give it as s + e.  The
-      // explicitly rounded intrinsics keep the compiler from contracting or
+      // r - (scale ks + offset) without rounding the level value: error-free
+      // products and sums (Dekker / Knuth) give it as d0 + lo.  The explicitly
+      // rounded intrinsics keep the compiler from contracting or
       // reassociating these steps.
       const float pr = __fmul_rn(sc, ks);
       const float pe = fmaf(sc, ks, -pr);
       const float s = __fadd_rn(pr, off);
       const float bb = __fsub_rn(s, pr);
       const float se = __fadd_rn(__fsub_rn(pr, __fsub_rn(s, bb)), __fsub_rn(off, bb));
-      dt = __fmul_rn(__fsub_rn(__fsub_rn(r, s), __fadd_rn(pe, se)), inv_sc);
+      const float d0 = __fsub_rn(r, s);
+      if (precise) {
+        const float b2 = __fsub_rn(d0, r);
+        const float de = __fadd_rn(__fsub_rn(r, __fsub_rn(d0, b2)), __fsub_rn(-s, b2));  // r - s = d0 + de
+        const float lo = __fsub_rn(de, __fadd_rn(pe, se));
+        dh = __fmul_rn(__fadd_rn(d0, lo), inv_sc);
+        dl = __fmul_rn(__fadd_rn(fmaf(-dh, sc, d0), lo), inv_sc);
+      } else {
+        dh = __fmul_rn(__fsub_rn(d0, __fadd_rn(pe, se)), inv_sc);
+        dl = 0.0f;
+      }
     } else {
       // anchored prior: the effective centre mixes r and w (fp64, rare path)
       const double tt = (g * ((double)r - doff) + ga * ((double)W[o] - doff)) * inv_dsc / geff;
       const double kd = fmin(fmax(ceil(tt - 0.5), 0.0), (double)(L - 1));
       ks = (float)kd;
-      dt = (float)(tt - kd);
+      const double dtd = tt - kd;
+      dh = (float)dtd;
+      dl = (float)(dtd - (double)dh);
     }
     const int kstar = (int)ks;
-    // q_k / q_k* = 2^(dk (A dk + B)) with dk = k - k*, A = -geff/2 log2(e),
-    // B = -2 A dt: all L levels in one fixed loop (no lane-dependent trip
-    // counts, so warps do not diverge), one hardware 2^x per level
-    const float B2 = -2.0f * A2 * dt;
     float S0 = 0.0f, S1 = 0.0f, S2 = 0.0f;
-    if (LT > 0) {
-#pragma unroll
-      for (int k = 0; k < (LT > 0 ? LT : 1); ++k) {
-        const float dk = (float)k - ks;
-        const float e = fast_exp2(fmaf(A2, dk, B2) * dk);
+    if (precise) {
+      // q_k / q_k* = 2^(A dk (dk - 2 dt)) with dk = k - k* an exact integer and
+      // A = -geff/2 log2(e).  Here geff is large: dk - 2 dt is formed from the
+      // pair (dh, dl) before scaling by A, so the exponent keeps fp32 accuracy
+      // relative to itself (A dk^2 - 2 A dk dt would cancel, and a plain fp32
+      // dt would cost more than 1e-4 of a weight).  min(2hw+1, L) consecutive
+      // levels around k*, shifted to stay on the grid.
+      const int k0 = min(max(kstar - hw, 0), L - nlev);
+#pragma unroll 4
+      for (int i = 0; i < nlev; ++i) {
+        const float dk = (float)(k0 + i) - ks;
+        const float e = fast_exp2((A2 * dk) * fmaf(-2.0f, dl, fmaf(-2.0f, dh, dk)));
         S0 += e;
         const float ed = e * dk;
         S1 += ed;
         S2 = fmaf(ed, dk, S2);
       }
     } else {
-      for (int k = 0; k < L; ++k) {
-        const float dk = (float)k - ks;
-        const float e = fast_exp2(fmaf(A2, dk, B2) * dk);
-        S0 += e;
-        const float ed = e * dk;
-        S1 += ed;
-        S2 = fmaf(ed, dk, S2);
+      // q_k / q_k* = 2^(dk (A dk + B)), B = -2 A dt: with |A| <= 5 the
+      // rounding of B costs under 1e-5 of a weight.  All L levels in one fixed
+      // loop (no lane-dependent trip counts, so warps do not diverge), one
+      // hardware 2^x per level.
+      const float B2 = -2.0f * A2 * dh;
+      if (LT > 0) {
+#pragma unroll
+        for (int k = 0; k < (LT > 0 ? LT : 1); ++k) {
+          const float dk = (float)k - ks;
+          const float e = fast_exp2(fmaf(A2, dk, B2) * dk);
+          S0 += e;
+          const float ed = e * dk;
+          S1 += ed;
+          S2 = fmaf(ed, dk, S2);
+        }
+      } else {
+        for (int k = 0; k < L; ++k) {
+          const float dk = (float)k - ks;
+          const float e = fast_exp2(fmaf(A2, dk, B2) * dk);
+          S0 += e;
+          const float ed = e * dk;
+          S1 += ed;
+          S2 = fmaf(ed, dk, S2);
+        }
       }
     }
     const float inv = __frcp_rn(S0);

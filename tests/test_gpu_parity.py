@@ -107,6 +107,23 @@ def test_stage_denoise_scalar(mpq, tau):
     assert np.array_equal(idx_np(out["idx"])[ok], ref.idx[ok])
 
 
+@pytest.mark.parametrize("g_lo,g_hi", [(100.0, 1e4), (0.05, 0.5)])
+def test_stage_denoise_scalar_precision_extremes(mpq, g_lo, g_hi):
+    # concentrated posteriors (a window of 3 levels) and nearly flat ones (all 8)
+    p = scalar_case()
+    s, V, s_cu, V_cu = spectrum_cuda(p.X)
+    plan = make_plan(mpq, p, s_cu, V_cu)
+    sc, off = oracle_grid_f32(p)
+    R1, g1, _, _, _, _ = injected_state(17, p.W, sc, s, g_lo, g_hi)
+    ref = orc.denoise(R1, g1, codebook_for(p), sc.astype(np.float64), off.astype(np.float64))
+    out = plan.stage_denoise(cu(R1), cu(g1, torch.float64), cu(sc), cu(off))
+    assert_rows_close("xhat1", host(out["xhat"]), ref.xhat)
+    assert_rows_close("vblock", host(out["vblock"]), ref.vblock)
+    assert_scalars_close("vsum", host(out["vsum"]), ref.vsum)
+    ok = ref.gap > LOGIT_TIE
+    assert np.array_equal(idx_np(out["idx"])[ok], ref.idx[ok])
+
+
 def test_stage_denoise_vector(mpq):
     p = vec_case()
     s, V, s_cu, V_cu = spectrum_cuda(p.X)
