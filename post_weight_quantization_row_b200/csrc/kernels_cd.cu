@@ -345,11 +345,17 @@ __global__ void __launch_bounds__(CD8_APPLY_WARPS * 32)
   const int kcur = idx[row * B + b];
   float g[8];
   block_gradient(H, n, hlr + (8 * b - t0), cb, kcur, sc, b, g);
-  float scur = qtab[b * K + kcur];
+  // the candidate's score is recomputed here in the same fp32 arithmetic as
+  // the current codeword's, so that acceptance (strictly lower) does not
+  // depend on how the scan evaluated it
+  if (k < 0 || k >= K || k == kcur) return;
+  float scur = qtab[b * K + kcur], snew = qtab[b * K + k];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) scur = fmaf(-cb[(int64_t)kcur * 8 + i], g[i], scur);
-  const bool accept = (v < scur) && k >= 0 && k < K;
-  if (!accept) return;
+  for (int i = 0; i < 8; ++i) {
+    scur = fmaf(-cb[(int64_t)kcur * 8 + i], g[i], scur);
+    snew = fmaf(-cb[(int64_t)k * 8 + i], g[i], snew);
+  }
+  if (!(snew < scur)) return;
   float dd[8], dl[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
@@ -415,7 +421,10 @@ mpq_status launch_cd(mpq_plan_s* p, const float* W, int64_t m, const float* scal
     }
     return MPQ_OK;
   }
-  const int nchunks = (int)cdiv(p->K, CD8_CHUNK);
+  // candidate scan: tensor cores for lattice codebooks (one partial minimum
+  // per codebook slice), else the SIMT kernel (one per chunk of CD8_CHUNK)
+  const bool tc = p->vec_tc;
+  const int nchunks = tc ? cd_scan_slices(m, p->K) : (int)cdiv(p->K, CD8_CHUNK);
   float* part_val = nullptr;
   int* part_idx = nullptr;
   MPQ_CUDA(cudaMallocAsync(&part_val, sizeof(float) * m * nchunks, st));
@@ -431,8 +440,11 @@ mpq_status launch_cd(mpq_plan_s* p, const float* W, int64_t m, const float* scal
       const int64_t t0 = (int64_t)j * CD_TILE;
       const int tw = (int)std::min<int64_t>(CD_TILE, n - t0);
       for (int64_t b = t0 / 8; b < (t0 + tw) / 8; ++b) {
-        dim3 ga((unsigned)nchunks, (unsigned)cdiv(m, CD8_ROWS));
-        {
+        if (tc) {
+          rc = launch_cd_vec_scan(p, m, b, t0, scale, idx, h, ldh, hl, part_val, part_idx, nchunks, st);
+          if (rc != MPQ_OK) break;
+        } else {
+          dim3 ga((unsigned)nchunks, (unsigned)cdiv(m, CD8_ROWS));
           ProfScope ps_("k_cd_vec_eval", st);
           k_cd_vec_eval<<<ga, 256, 0, st>>>(m, n, p->K, b, t0, p->cb, p->qtab, p->H32, scale, idx,
                                             h, ldh, hl, sweeps, sw, changes, part_val, part_idx,
@@ -445,7 +457,7 @@ mpq_status launch_cd(mpq_plan_s* p, const float* W, int64_t m, const float* scal
               sweeps, sw, changes, part_val, part_idx, nchunks, w.As.hi, w.As.lo, w.As.ld,
               w.As.row_unscale, w.tile_count);
         }
-        count_launch(2);
+        count_launch(tc ? 1 : 2);
         rc = check_launch("k_cd_vec");
         if (rc != MPQ_OK) break;
       }

@@ -9,6 +9,8 @@
 // the NeUQI note, existing pain points section.
 #include <math.h>
 
+#include <type_traits>
+
 #include "mpq_internal.cuh"
 
 namespace mpq {
@@ -229,6 +231,10 @@ __global__ void __launch_bounds__(ROW_THREADS)
   const float inv_sc = (float)inv_dsc;
   const float Lm1 = (float)(L - 1);
   const float sc2f = (float)sc2;
+  // the per-weight loop, instantiated once per precision regime so that the
+  // row-uniform choice costs no branch per weight
+  auto weights = [&](auto prec) -> float {
+  constexpr bool PRECISE = decltype(prec)::value;
   float acc = 0.0f;
   for (int64_t j = threadIdx.x; j < n; j += blockDim.x) {
     const int64_t o = row * n + j;
@@ -248,7 +254,7 @@ __global__ void __launch_bounds__(ROW_THREADS)
       const float bb = __fsub_rn(s, pr);
       const float se = __fadd_rn(__fsub_rn(pr, __fsub_rn(s, bb)), __fsub_rn(off, bb));
       const float d0 = __fsub_rn(r, s);
-      if (precise) {
+      if constexpr (PRECISE) {
         const float b2 = __fsub_rn(d0, r);
         const float de = __fadd_rn(__fsub_rn(r, __fsub_rn(d0, b2)), __fsub_rn(-s, b2));  // r - s = d0 + de
         const float lo = __fsub_rn(de, __fadd_rn(pe, se));
@@ -269,7 +275,7 @@ __global__ void __launch_bounds__(ROW_THREADS)
     }
     const int kstar = (int)ks;
     float S0 = 0.0f, S1 = 0.0f, S2 = 0.0f;
-    if (precise) {
+    if constexpr (PRECISE) {
       // q_k / q_k* = 2^(A dk (dk - 2 dt)) with dk = k - k* an exact integer and
       // A = -geff/2 log2(e).  Here geff is large: dk - 2 dt is formed from the
       // pair (dh, dl) before scaling by A, so the exponent keeps fp32 accuracy
@@ -322,6 +328,9 @@ __global__ void __launch_bounds__(ROW_THREADS)
     if (idx) idx[o] = (uint16_t)kstar;
     acc += v;
   }
+  return acc;
+  };
+  const float acc = precise ? weights(std::true_type{}) : weights(std::false_type{});
   const double tot = block_sum((double)acc, ds);
   if (threadIdx.x == 0) vsum[row] = tot;
 }

@@ -214,6 +214,13 @@ mpq_status launch_denoise_vec_tc(const mpq_plan_s* p, const float* R1, const dou
                                  float* xhat1, float* vblock, uint16_t* idx, int nearest_only,
                                  cudaStream_t st);
 
+// tensor-core candidate scan of the vector CD step (cd_scan_tc.cu)
+int cd_scan_slices(int64_t m, int K);
+mpq_status launch_cd_vec_scan(const mpq_plan_s* p, int64_t m, int64_t b, int64_t t0,
+                              const float* scale, const uint16_t* idx, const float* h,
+                              int64_t ldh, const float* hl, float* part_val, int* part_idx,
+                              int nslices, cudaStream_t st);
+
 // plan-time builders
 mpq_status build_hessian(mpq_plan_s* p, cudaStream_t st);
 mpq_status build_codebook_tables(mpq_plan_s* p, cudaStream_t st);
