@@ -6,11 +6,13 @@
 // (x * 2^-e = hi + lo, hi = fp16(x * 2^-e), lo = fp16(x * 2^-e - hi)), so
 // hi + lo carries ~22 significand bits and the three products recover an
 // fp32-accurate contraction (the dropped lo*lo term is ~2^-22 relative).
-// Both operands are K-major (K contiguous).  Tiles: 128 x 256 x 64, fp16
-// kind::f16 MMAs with the fp32 accumulator in TMEM (256 columns), operands
-// staged by TMA (128-byte swizzle, no multicast) through a 2-stage mbarrier
-// pipeline.  Warp 0 issues TMA, warp 1 owns TMEM and issues the MMAs from one
-// thread, warps 2-5 read the accumulator back (tcgen05.ld) and store C.
+// Both operands are K-major (K contiguous).  Persistent kernel, one CTA per
+// SM walking 128 x 128 x 64 tiles: fp16 kind::f16 MMAs with the fp32
+// accumulator in TMEM (two 128-column accumulators, so that the epilogue of
+// one tile overlaps the MMAs of the next), operands staged by TMA (128-byte
+// swizzle, no multicast) through a 3-stage mbarrier ring that runs across
+// tiles.  Warp 0 issues TMA, warp 1 owns TMEM and issues the MMAs from one
+// thread, warps 2-5 read the accumulators back (tcgen05.ld) and store C.
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <cudaTypedefs.h>
@@ -24,49 +26,69 @@ namespace mpq {
 namespace {
 using namespace tcx;
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 2;
+constexpr int BM = 128, BK = 64;
 constexpr int A_TILE = BM * BK * 2;                 // 16 KiB
-constexpr int B_TILE = BN * BK * 2;                 // 32 KiB
-constexpr int STAGE_BYTES = 2 * A_TILE + 2 * B_TILE;  // 96 KiB
 constexpr int TC_THREADS = 192;
-constexpr uint32_t TMEM_COLS = 256;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /* alignment slack */ + 128;
 
-constexpr uint32_t IDESC = idesc_f16(BM, BN);
+// ------------------------------------------------------- persistent GEMM --
+// The same product with 128 x 128 tiles walked by one CTA per SM: a 3-stage
+// TMA ring runs across tiles, and two TMEM accumulators let the epilogue of
+// one tile overlap the MMAs of the next.  Tiles go in groups of 8 M-tiles
+// (M fastest) so that the A and B panels in flight stay in L2.
+constexpr int PBN = 128, PSTAGES = 3, PGROUP = 8;
+constexpr int P_B_TILE = PBN * BK * 2;                        // 16 KiB
+constexpr int P_STAGE = 2 * A_TILE + 2 * P_B_TILE;            // 64 KiB
+constexpr int P_STG_WARP = 8192;                              // epilogue staging per warp
+constexpr int P_SMEM = PSTAGES * P_STAGE + 4 * P_STG_WARP + 1024 + 256;
+constexpr uint32_t P_TMEM_COLS = 2 * PBN;
+constexpr uint32_t P_IDESC = idesc_f16(BM, PBN);
+
+__device__ __forceinline__ void p_tile(int t, int mtiles, int ntiles, int& m0, int& n0) {
+  const int per_group = PGROUP * ntiles;
+  const int g = t / per_group, w = t % per_group;
+  const int gm = min(PGROUP, mtiles - g * PGROUP);  // M-tiles in this group
+  m0 = (g * PGROUP + w % gm) * BM;
+  n0 = (w / gm) * PBN;
+}
 
 __global__ void __launch_bounds__(TC_THREADS, 1)
-    k_gemm_tc(const __grid_constant__ CUtensorMap ta_hi, const __grid_constant__ CUtensorMap ta_lo,
-              const __grid_constant__ CUtensorMap tb_hi, const __grid_constant__ CUtensorMap tb_lo,
-              float* __restrict__ C, int64_t ldc, int M, int N, int K, int b_k0,
-              const float* __restrict__ row_scale, float b_scale, int accumulate, int a_exact,
-              const int* __restrict__ gate, const __grid_constant__ CUtensorMap tc_out,
-              int use_reduce, int* status) {
-  // a zero gate means there is nothing to add: skip the whole tile
-  if (gate != nullptr && *gate == 0) return;
+    k_gemm_tcp(const __grid_constant__ CUtensorMap ta_hi, const __grid_constant__ CUtensorMap ta_lo,
+               const __grid_constant__ CUtensorMap tb_hi, const __grid_constant__ CUtensorMap tb_lo,
+               float* __restrict__ C, int64_t ldc, int M, int N, int K, int b_k0,
+               const float* __restrict__ row_scale, float b_scale, int accumulate, int a_exact,
+               const int* __restrict__ gate, const __grid_constant__ CUtensorMap tc_out,
+               int use_reduce, int* status) {
+  if (gate != nullptr && *gate == 0) return;  // nothing to add
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint64_t* full = (uint64_t*)(smem + STAGES * STAGE_BYTES);
-  uint64_t* empty = full + STAGES;
-  uint64_t* done = empty + STAGES;
-  uint32_t* tmem_slot = (uint32_t*)(done + 1);
+  uint8_t* stg_all = smem + PSTAGES * P_STAGE;
+  uint64_t* full = (uint64_t*)(stg_all + 4 * P_STG_WARP);
+  uint64_t* empty = full + PSTAGES;
+  uint64_t* tm_full = empty + PSTAGES;
+  uint64_t* tm_empty = tm_full + 2;
+  uint32_t* tmem_slot = (uint32_t*)(tm_empty + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
+  const int mtiles = (M + BM - 1) / BM, ntiles = (N + PBN - 1) / PBN;
+  const int tiles = mtiles * ntiles;
   const int KT = (K + BK - 1) / BK;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < PSTAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(done, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tm_full[b], 1);
+      mbar_init(&tm_empty[b], 4);  // the four epilogue warps
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(tmem_slot)),
-                 "r"(TMEM_COLS));
+                 "r"(P_TMEM_COLS));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   tc_fence_before();
@@ -76,120 +98,153 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 
   if (warp == 0 && lane == 0) {
     // ---------------------------------------------------------- producer
-    for (int kt = 0; kt < KT; ++kt) {
-      const int s = kt % STAGES, it = kt / STAGES;
-      if (kt >= STAGES && !mbar_wait(&empty[s], (it - 1) & 1)) {
-        atomicOr(status, STATUS_TIMEOUT);
-        break;
+    uint32_t it = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+      int m0, n0;
+      p_tile(t, mtiles, ntiles, m0, n0);
+      for (int kt = 0; kt < KT; ++kt, ++it) {
+        const int s = it % PSTAGES;
+        if (it >= PSTAGES && !mbar_wait(&empty[s], (it / PSTAGES - 1) & 1)) {
+          atomicOr(status, STATUS_TIMEOUT);
+          ok = false;
+          break;
+        }
+        uint8_t* base = smem + s * P_STAGE;
+        mbar_expect_tx(&full[s], a_exact ? P_STAGE - A_TILE : P_STAGE);
+        tma_load_2d(&ta_hi, &full[s], base, kt * BK, m0);
+        if (!a_exact) tma_load_2d(&ta_lo, &full[s], base + A_TILE, kt * BK, m0);
+        tma_load_2d(&tb_hi, &full[s], base + 2 * A_TILE, b_k0 + kt * BK, n0);
+        tma_load_2d(&tb_lo, &full[s], base + 2 * A_TILE + P_B_TILE, b_k0 + kt * BK, n0);
       }
-      uint8_t* base = smem + s * STAGE_BYTES;
-      mbar_expect_tx(&full[s], a_exact ? STAGE_BYTES - A_TILE : STAGE_BYTES);
-      tma_load_2d(&ta_hi, &full[s], base, kt * BK, m0);
-      if (!a_exact) tma_load_2d(&ta_lo, &full[s], base + A_TILE, kt * BK, m0);
-      tma_load_2d(&tb_hi, &full[s], base + 2 * A_TILE, b_k0 + kt * BK, n0);
-      tma_load_2d(&tb_lo, &full[s], base + 2 * A_TILE + B_TILE, b_k0 + kt * BK, n0);
     }
+    for (uint32_t q = (it > PSTAGES ? it - PSTAGES : 0); q < it; ++q)  // copies land before exit
+      for (uint32_t i = 0; i < (1u << 25) && !mbar_try_wait(&full[q % PSTAGES], (q / PSTAGES) & 1); ++i)
+        if (i > 256) __nanosleep(64);
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------- MMA issuer
+    uint32_t it = 0, tl = 0;
     bool ok = true;
-    for (int kt = 0; kt < KT && ok; ++kt) {
-      const int s = kt % STAGES, it = kt / STAGES;
-      if (!mbar_wait(&full[s], it & 1)) {
+    for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++tl) {
+      const int buf = tl & 1;
+      if (tl >= 2 && !mbar_wait(&tm_empty[buf], (tl / 2 - 1) & 1)) {
         atomicOr(status, STATUS_TIMEOUT);
         ok = false;
         break;
       }
       tc_fence_after();
-      const uint32_t a_hi = smem_u32(smem + s * STAGE_BYTES);
-      const uint32_t a_lo = a_hi + A_TILE;
-      const uint32_t b_hi = a_hi + 2 * A_TILE;
-      const uint32_t b_lo = b_hi + B_TILE;
+      const uint32_t d = tmem + (uint32_t)buf * PBN;
+      for (int kt = 0; kt < KT; ++kt, ++it) {
+        const int s = it % PSTAGES;
+        if (!mbar_wait(&full[s], (it / PSTAGES) & 1)) {
+          atomicOr(status, STATUS_TIMEOUT);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a_hi = smem_u32(smem + s * P_STAGE);
+        const uint32_t a_lo = a_hi + A_TILE;
+        const uint32_t b_hi = a_hi + 2 * A_TILE;
+        const uint32_t b_lo = b_hi + P_B_TILE;
 #pragma unroll
-      for (int kk = 0; kk < BK / 16; ++kk) {
-        const uint32_t off = kk * 32;  // 16 fp16 along K inside the 128-byte row
-        const uint64_t dah = sw128_desc(a_hi + off), dal = sw128_desc(a_lo + off);
-        const uint64_t dbh = sw128_desc(b_hi + off), dbl = sw128_desc(b_lo + off);
-        umma_f16(tmem, dah, dbh, IDESC, (kt | kk) != 0 ? 1u : 0u);
-        umma_f16(tmem, dah, dbl, IDESC, 1u);
-        if (!a_exact) umma_f16(tmem, dal, dbh, IDESC, 1u);
+        for (int kk = 0; kk < BK / 16; ++kk) {
+          const uint32_t off = kk * 32;
+          const uint64_t dah = sw128_desc(a_hi + off), dal = sw128_desc(a_lo + off);
+          const uint64_t dbh = sw128_desc(b_hi + off), dbl = sw128_desc(b_lo + off);
+          umma_f16(d, dah, dbh, P_IDESC, (kt | kk) != 0 ? 1u : 0u);
+          umma_f16(d, dah, dbl, P_IDESC, 1u);
+          if (!a_exact) umma_f16(d, dal, dbh, P_IDESC, 1u);
+        }
+        umma_commit(&empty[s]);
       }
-      umma_commit(&empty[s]);
+      if (ok) umma_commit(&tm_full[buf]);
     }
-    umma_commit(done);
+    for (uint32_t q = (tl > 2 ? tl - 2 : 0); q < tl; ++q)  // MMAs finish before TMEM is freed
+      for (uint32_t i = 0; i < (1u << 25) && !mbar_try_wait(&tm_full[q & 1], (q / 2) & 1); ++i)
+        if (i > 256) __nanosleep(64);
   } else if (warp >= 2) {
     // --------------------------------------------------------- epilogue
-    // warp-uniform outcome: the TMEM loads below are .sync.aligned
-    const bool ok = __all_sync(0xffffffffu, mbar_wait(done, 0));
-    if (!ok && lane == 0) atomicOr(status, STATUS_TIMEOUT);
-    tc_fence_after();
     const int q = warp & 3;  // TMEM lane quadrant this warp may read
-    const int row = m0 + q * 32 + lane;
-    const float rs = (row < M) ? row_scale[row] * b_scale : 0.0f;
-    if (use_reduce) {
-      // accumulate through the TMA unit: each warp stages its 32 x 32 block in
-      // a 128B-swizzled buffer (two per warp, alternating) and issues a
-      // tensor reduce-add into C; L2 performs the read-modify-write
-      uint8_t* stg0 = smem + (warp - 2) * 8192;
-      int nb = 0;
-      for (int c0 = 0; c0 < BN && ok; c0 += 32) {
-        if (n0 + c0 >= N) break;
+    uint8_t* stg0 = stg_all + (warp - 2) * P_STG_WARP;
+    float* stage = reinterpret_cast<float*>(stg0);
+    uint32_t tl = 0;
+    int nb = 0;  // bulk reduce groups issued by this warp
+    for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++tl) {
+      const int buf = tl & 1;
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&tm_full[buf], (tl / 2) & 1));
+      if (!ok) {
+        if (lane == 0) atomicOr(status, STATUS_TIMEOUT);
+        break;
+      }
+      tc_fence_after();
+      int m0, n0;
+      p_tile(t, mtiles, ntiles, m0, n0);
+      const int row = m0 + q * 32 + lane;
+      const float rs = (row < M) ? row_scale[row] * b_scale : 0.0f;
+      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)buf * PBN;
+      for (int c0 = 0; c0 < PBN; c0 += 32) {
         uint32_t v[32];
-        tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c0, v);
-        uint8_t* stg = stg0 + (nb & 1) * 4096;
-        if (lane == 0 && nb >= 2) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-        __syncwarp();
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          float4 o = make_float4(__uint_as_float(v[4 * k]) * rs, __uint_as_float(v[4 * k + 1]) * rs,
-                                 __uint_as_float(v[4 * k + 2]) * rs, __uint_as_float(v[4 * k + 3]) * rs);
-          *reinterpret_cast<float4*>(stg + lane * 128 + ((k ^ (lane & 7)) * 16)) = o;
+        tmem_ld32(tbase + (uint32_t)c0, v);
+        if (c0 + 32 == PBN) {  // the accumulator is read: hand it back to the MMAs
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tm_empty[buf]);
         }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        __syncwarp();
-        if (lane == 0) tma_reduce_add_2d(&tc_out, stg, n0 + c0, m0 + q * 32);
-        ++nb;
-      }
-      if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-      __syncwarp();
-    } else {
-    // the pipeline buffers are idle now: a 32 x 33 staging tile per warp turns
-    // the lane-per-row TMEM layout into row-contiguous, coalesced accesses
-    float* stage = reinterpret_cast<float*>(smem) + (warp - 2) * (32 * 33);
-    for (int c0 = 0; c0 < BN && ok; c0 += 32) {
-      if (n0 + c0 >= N) break;
-      uint32_t v[32];
-      tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c0, v);
+        if (n0 + c0 >= N) continue;
+        if (use_reduce) {
+          // accumulate through the TMA unit: a 32 x 32 block in a
+          // 128B-swizzled buffer (two per warp, alternating), tensor
+          // reduce-add into C; L2 performs the read-modify-write
+          uint8_t* sb = stg0 + (nb & 1) * 4096;
+          if (lane == 0 && nb >= 2) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+          __syncwarp();
 #pragma unroll
-      for (int j = 0; j < 32; ++j) stage[lane * 33 + j] = __uint_as_float(v[j]) * rs;
-      __syncwarp();
-      const int col = n0 + c0 + lane;
-      const int nrow = min(32, M - (m0 + q * 32));
-      float* cbase = C + (int64_t)(m0 + q * 32) * ldc + col;
-      if (col < N) {
-        if (accumulate) {
-          float prev[32];
-#pragma unroll
-          for (int rr = 0; rr < 32; ++rr)  // all loads in flight before any store
-            prev[rr] = (rr < nrow) ? cbase[(int64_t)rr * ldc] : 0.0f;
-#pragma unroll
-          for (int rr = 0; rr < 32; ++rr)
-            if (rr < nrow) cbase[(int64_t)rr * ldc] = prev[rr] + stage[rr * 33 + lane];
+          for (int k = 0; k < 8; ++k) {
+            float4 o = make_float4(__uint_as_float(v[4 * k]) * rs, __uint_as_float(v[4 * k + 1]) * rs,
+                                   __uint_as_float(v[4 * k + 2]) * rs, __uint_as_float(v[4 * k + 3]) * rs);
+            *reinterpret_cast<float4*>(sb + lane * 128 + ((k ^ (lane & 7)) * 16)) = o;
+          }
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          __syncwarp();
+          if (lane == 0) tma_reduce_add_2d(&tc_out, sb, n0 + c0, m0 + q * 32);
+          ++nb;
         } else {
+          // a 32 x 33 staging tile turns the lane-per-row TMEM layout into
+          // row-contiguous, coalesced accesses
 #pragma unroll
-          for (int rr = 0; rr < 32; ++rr)
-            if (rr < nrow) cbase[(int64_t)rr * ldc] = stage[rr * 33 + lane];
+          for (int j = 0; j < 32; ++j) stage[lane * 33 + j] = __uint_as_float(v[j]) * rs;
+          __syncwarp();
+          const int col = n0 + c0 + lane;
+          const int nrow = min(32, M - (m0 + q * 32));
+          float* cbase = C + (int64_t)(m0 + q * 32) * ldc + col;
+          if (col < N) {
+            if (accumulate) {
+              float prev[32];
+#pragma unroll
+              for (int rr = 0; rr < 32; ++rr)  // all loads in flight before any store
+                prev[rr] = (rr < nrow) ? cbase[(int64_t)rr * ldc] : 0.0f;
+#pragma unroll
+              for (int rr = 0; rr < 32; ++rr)
+                if (rr < nrow) cbase[(int64_t)rr * ldc] = prev[rr] + stage[rr * 33 + lane];
+            } else {
+#pragma unroll
+              for (int rr = 0; rr < 32; ++rr)
+                if (rr < nrow) cbase[(int64_t)rr * ldc] = stage[rr * 33 + lane];
+            }
+          }
+          __syncwarp();
         }
       }
-      __syncwarp();
     }
-    }
+    if (use_reduce && lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
-                 "r"(TMEM_COLS));
+                 "r"(P_TMEM_COLS));
   }
 }
 
@@ -242,6 +297,7 @@ mpq_status get_encoder() {
 }
 
 bool g_smem_attr_set[64] = {};
+int g_sms[64] = {};
 
 }  // namespace
 
@@ -309,16 +365,18 @@ mpq_status gemm_tc(const SplitOperand& A, const CUtensorMap& ta_hi, const CUtens
   int dev = 0;
   MPQ_CUDA(cudaGetDevice(&dev));
   if (dev >= 0 && dev < 64 && !g_smem_attr_set[dev]) {
-    MPQ_CUDA(cudaFuncSetAttribute(k_gemm_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES));
+    MPQ_CUDA(cudaFuncSetAttribute(k_gemm_tcp, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM));
+    MPQ_CUDA(cudaDeviceGetAttribute(&g_sms[dev], cudaDevAttrMultiProcessorCount, dev));
     g_smem_attr_set[dev] = true;
   }
   if (o.c_reduce && !o.accumulate)
     return fail(MPQ_ERR_INVALID_ARG, "gemm_tc: reduce output needs accumulate");
-  dim3 grid((unsigned)cdiv(N, BN), (unsigned)cdiv(M, BM));
+  const int64_t tiles = cdiv(M, BM) * cdiv(N, PBN);
+  const unsigned grid = (unsigned)std::min<int64_t>(tiles, dev < 64 ? g_sms[dev] : 148);
   const CUtensorMap& cmap = o.c_reduce ? *o.c_reduce : tb_hi;  // unused unless reducing
   {
     ProfScope ps_(tag, st);
-    k_gemm_tc<<<grid, TC_THREADS, SMEM_BYTES, st>>>(
+    k_gemm_tcp<<<grid, TC_THREADS, P_SMEM, st>>>(
         ta_hi, ta_lo, tb_hi, tb_lo, C, ldc, (int)M, (int)N, (int)K, (int)o.b_k0, A.row_unscale,
         b_scale_host, o.accumulate ? 1 : 0, o.a_exact ? 1 : 0, o.gate, cmap, o.c_reduce ? 1 : 0,
         status);

@@ -398,12 +398,12 @@ mpq_status finish_plan(mpq_plan_s* p, cudaStream_t st) {
   MPQ_CUDA(cudaMemcpyAsync(&p->Vt_s.unscale_host, p->Vt_s.unscale, sizeof(float), cudaMemcpyDeviceToHost, st));
   MPQ_CUDA(cudaMemcpyAsync(&p->V_s.unscale_host, p->V_s.unscale, sizeof(float), cudaMemcpyDeviceToHost, st));
   MPQ_CUDA(cudaMemcpyAsync(&p->H_s.unscale_host, p->H_s.unscale, sizeof(float), cudaMemcpyDeviceToHost, st));
-  MPQ_TRY(make_tmap_f16(&p->tm_vt_hi, p->Vt_s.hi, p->Vt_s.ld, p->Vt_s.rows_pad, p->Vt_s.ld, 256));
-  MPQ_TRY(make_tmap_f16(&p->tm_vt_lo, p->Vt_s.lo, p->Vt_s.ld, p->Vt_s.rows_pad, p->Vt_s.ld, 256));
-  MPQ_TRY(make_tmap_f16(&p->tm_v_hi, p->V_s.hi, p->V_s.ld, p->V_s.rows_pad, p->V_s.ld, 256));
-  MPQ_TRY(make_tmap_f16(&p->tm_v_lo, p->V_s.lo, p->V_s.ld, p->V_s.rows_pad, p->V_s.ld, 256));
-  MPQ_TRY(make_tmap_f16(&p->tm_h_hi, p->H_s.hi, p->H_s.ld, p->H_s.rows_pad, p->H_s.ld, 256));
-  MPQ_TRY(make_tmap_f16(&p->tm_h_lo, p->H_s.lo, p->H_s.ld, p->H_s.rows_pad, p->H_s.ld, 256));
+  MPQ_TRY(make_tmap_f16(&p->tm_vt_hi, p->Vt_s.hi, p->Vt_s.ld, p->Vt_s.rows_pad, p->Vt_s.ld, 128));
+  MPQ_TRY(make_tmap_f16(&p->tm_vt_lo, p->Vt_s.lo, p->Vt_s.ld, p->Vt_s.rows_pad, p->Vt_s.ld, 128));
+  MPQ_TRY(make_tmap_f16(&p->tm_v_hi, p->V_s.hi, p->V_s.ld, p->V_s.rows_pad, p->V_s.ld, 128));
+  MPQ_TRY(make_tmap_f16(&p->tm_v_lo, p->V_s.lo, p->V_s.ld, p->V_s.rows_pad, p->V_s.ld, 128));
+  MPQ_TRY(make_tmap_f16(&p->tm_h_hi, p->H_s.hi, p->H_s.ld, p->H_s.rows_pad, p->H_s.ld, 128));
+  MPQ_TRY(make_tmap_f16(&p->tm_h_lo, p->H_s.lo, p->H_s.ld, p->H_s.rows_pad, p->H_s.ld, 128));
   if (p->d == 8) {
     MPQ_TRY(dalloc(&p->cb_norm, p->K));
     MPQ_TRY(dalloc(&p->qtab, p->B * (int64_t)p->K));
