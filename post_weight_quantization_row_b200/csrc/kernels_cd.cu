@@ -10,6 +10,8 @@
 // delta = c - x_b, and accepting it updates h <- h - H[:, b] delta.
 #include <math.h>
 
+#include <type_traits>
+
 #include "mpq_internal.cuh"
 
 namespace mpq {
@@ -17,18 +19,29 @@ namespace {
 
 // ------------------------------------------------------------------ d = 1 --
 // A sweep visits the columns in tiles of CD_TILE.  For tile j the decide
-// kernel runs one warp per row on the tile's own gradient (shared memory):
-// the 32 lanes evaluate 32 consecutive columns, which is exact up to the
-// first lane that accepts a change; the warp commits that change, updates
-// the tile-local gradient with the row of H, and resumes right after it --
-// identical to visiting the columns one by one.  The tile's changes leave as
-// Delta/scale (small integers, exact in fp16) in the A operand of a tensor-
-// core update  h += (-scale) Delta H[tile, :]  over all columns, which also
-// reproduces the in-tile updates for the next tile and the next sweep.
+// kernel runs one warp per row; lane l keeps, in registers, the state of the
+// tile's columns l, l + 32, l + 64, l + 96 (gradient, level, and the two
+// per-column constants of the energy change).  The warp takes the tile 32
+// columns at a time: all live lanes evaluate their column, which is exact up
+// to the first lane that accepts a change; the warp commits that change,
+// updates the gradient of the later columns with the row of H, and resumes
+// right after it -- identical to visiting the columns one by one.  The
+// tile's changes leave as Delta/scale (small integers, exact in fp16) in the
+// A operand of a tensor-core update  h += (-scale) Delta H[tile, :]  over all
+// columns, which also reproduces the in-tile updates for the next tile and
+// the next sweep.
 constexpr int CD1_WARPS = 16;
-constexpr int CD1_SMEM = (CD_TILE * CD_TILE + CD_TILE + CD1_WARPS * CD_TILE) * 4 + CD1_WARPS * CD_TILE * 2;
+constexpr int CD1_SLOTS = CD_TILE / 32;
+constexpr int CD1_SMEM = (CD_TILE * CD_TILE + CD_TILE) * 4;
 
-__global__ void __launch_bounds__(CD1_WARPS * 32)
+// 4-byte asynchronous copy global -> shared; src_bytes = 0 fills zero
+__device__ __forceinline__ void cp_async4(float* dst, const float* src, int src_bytes) {
+  const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(d), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+
+__global__ void __launch_bounds__(CD1_WARPS * 32, 2)
     k_cd_tile_decide(int64_t m, int64_t n, int L, int64_t t0, int tw, int tile, int ntiles,
                      const float* __restrict__ scale, const float* __restrict__ H,
                      uint16_t* __restrict__ idx, const float* __restrict__ h, int64_t ldh,
@@ -37,116 +50,115 @@ __global__ void __launch_bounds__(CD1_WARPS * 32)
                      __half* __restrict__ dlo, int64_t lda, float* __restrict__ d_unscale,
                      int* __restrict__ tile_count) {
   extern __shared__ float cd_smem[];
-  float* sH = cd_smem;                                  // H[tile, tile]
-  float* s_rg = sH + CD_TILE * CD_TILE;                 // 1 / H_jj (0 where H_jj <= 0)
-  float* s_h_all = s_rg + CD_TILE;                      // per-warp gradient of the tile
-  uint16_t* s_i_all = (uint16_t*)(s_h_all + CD1_WARPS * CD_TILE);  // per-warp indices
-  // H[tile, tile] into shared memory: warp w copies rows w, w + 16, ...; all
-  // of a warp's loads are issued before the first store so their latencies
-  // overlap (CD_TILE / CD1_WARPS rows x CD_TILE / 32 values per lane)
-  {
-    constexpr int RPW = CD_TILE / CD1_WARPS, VPL = CD_TILE / 32;
-    const int wid0 = threadIdx.x >> 5, lane0 = threadIdx.x & 31;
-    float v[RPW][VPL];
-#pragma unroll
-    for (int rr = 0; rr < RPW; ++rr) {
-      const int i = wid0 + rr * CD1_WARPS;
-      const float* src = H + (t0 + i) * n + t0;
-#pragma unroll
-      for (int q = 0; q < VPL; ++q) {
-        const int j = lane0 + 32 * q;
-        v[rr][q] = (i < tw && j < tw) ? src[j] : 0.0f;
-      }
-    }
-#pragma unroll
-    for (int rr = 0; rr < RPW; ++rr)
-#pragma unroll
-      for (int q = 0; q < VPL; ++q) sH[(wid0 + rr * CD1_WARPS) * CD_TILE + lane0 + 32 * q] = v[rr][q];
+  float* sH = cd_smem;                   // H[tile, tile], zero outside tw x tw
+  float* s_rg = sH + CD_TILE * CD_TILE;  // 1 / H_jj (0 where H_jj <= 0)
+  for (int e = threadIdx.x; e < CD_TILE * CD_TILE; e += blockDim.x) {
+    const int i = e / CD_TILE, j = e % CD_TILE;
+    const bool in = i < tw && j < tw;
+    cp_async4(sH + e, in ? H + (t0 + i) * n + t0 + j : H, in ? 4 : 0);
   }
+  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;\n" ::: "memory");
   __syncthreads();
+  bool pos = true;  // every diagonal entry of the tile positive
   for (int j = threadIdx.x; j < CD_TILE; j += blockDim.x) {
     const float gj = sH[j * CD_TILE + j];
     s_rg[j] = gj > 0.0f ? 1.0f / gj : 0.0f;
+    if (j < tw && !(gj > 0.0f)) pos = false;
   }
-  __syncthreads();
+  pos = __syncthreads_and(pos);
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int64_t row = (int64_t)blockIdx.x * CD1_WARPS + wid;
   if (row >= m) return;
   __half* drow_hi = dhi + row * lda;
   __half* drow_lo = dlo + row * lda;
-  for (int i = lane; i < CD_TILE; i += 32) {
-    drow_hi[i] = __float2half_rn(0.0f);
-    drow_lo[i] = __float2half_rn(0.0f);
-  }
-  const float sc = scale[row], isc = 1.0f / sc;
+  const float sc = scale[row];
   if (lane == 0) d_unscale[row] = -sc;
-  // a row stops after a sweep without change (its Delta row stays zero)
-  if (sw > 0 && changes[row * sweeps + sw - 1] == 0) return;
-  float* sh = s_h_all + wid * CD_TILE;
-  uint16_t* si = s_i_all + wid * CD_TILE;
-  const float* hr = h + row * ldh + t0;
   uint16_t* ir = idx + row * n + t0;
-  for (int i = lane; i < tw; i += 32) {
-    sh[i] = hr[i];
-    si[i] = ir[i];
+  // a row stops after a sweep without change (its Delta row stays zero)
+  if (sw > 0 && changes[row * sweeps + sw - 1] == 0) {
+    for (int i = lane; i < CD_TILE; i += 32) {
+      drow_hi[i] = __float2half_rn(0.0f);
+      drow_lo[i] = __float2half_rn(0.0f);
+    }
+    return;
   }
-  __syncwarp();
-  int ntile = 0;
-  int c = 0;
-  while (c < tw) {
-    const int j = c + lane;
-    bool acc = false;
-    int kb = 0, kc = 0;
-    if (j < tw) {
-      const float hj = sh[j], g = sH[j * CD_TILE + j];
-      kc = si[j];
-      // dE(k) = d (d g/2 - h), d = scale (k - kc), is a convex quadratic in k:
-      // its integer minimiser is one of the two levels around the continuous
-      // one (the grid ends when g <= 0), lowest index on ties
-      int k0, k1;
-      if (g > 0.0f) {
-        // (a reciprocal instead of a division moves kcont by ulps, which
-        // leaves the best integer level among the two candidates)
-        const float kcont = (float)kc + hj * (isc * s_rg[j]);
-        k0 = (int)fminf(fmaxf(floorf(kcont), 0.0f), (float)(L - 1));
-        k1 = min(k0 + 1, L - 1);
-      } else {
-        k0 = 0;
-        k1 = L - 1;
+  // Energy change of level k in index units u = k - kc (dE = u (a u - hs),
+  // hs = scale h, a = scale^2 H_jj / 2): a parabola in k with its vertex at
+  // kcont = kc + hs rq, rq = 1 / (scale^2 H_jj).  The best level is the one
+  // nearest kcont (the lower on an exact half: lowest index on ties), clamped
+  // to the grid; a reciprocal instead of a division moves kcont by ulps,
+  // which changes the choice only between levels whose energies tie to
+  // rounding.  With H_jj <= 0 the candidates are the grid ends.
+  const float s2 = sc * sc, is2 = 1.0f / s2, Lm1 = (float)(L - 1);
+  const float* hr = h + row * ldh + t0;
+  float hs[CD1_SLOTS], kc[CD1_SLOTS], a[CD1_SLOTS], rq[CD1_SLOTS];
+#pragma unroll
+  for (int q = 0; q < CD1_SLOTS; ++q) {
+    const int col = 32 * q + lane;
+    const bool in = col < tw;
+    hs[q] = in ? sc * hr[col] : 0.0f;
+    kc[q] = in ? (float)ir[col] : 0.0f;
+    a[q] = 0.5f * s2 * sH[col * CD_TILE + col];
+    rq[q] = is2 * s_rg[col];
+  }
+  auto sweep_tile = [&](auto all_pos) -> int {
+    constexpr bool POS = decltype(all_pos)::value;
+    int nchg = 0;
+#pragma unroll
+    for (int q = 0; q < CD1_SLOTS; ++q) {
+      if (32 * q >= tw) break;
+      unsigned live = tw - 32 * q >= 32 ? 0xffffffffu : (1u << (tw - 32 * q)) - 1u;
+      while (true) {
+        float kn, e;
+        {
+          const float kcont = fmaf(hs[q], rq[q], kc[q]);
+          kn = fminf(fmaxf(ceilf(kcont - 0.5f), 0.0f), Lm1);
+          const float u = kn - kc[q];
+          e = u * fmaf(a[q], u, -hs[q]);
+        }
+        if (!POS && !(a[q] > 0.0f)) {
+          const float u0 = -kc[q], u1 = Lm1 - kc[q];
+          const float e0 = u0 * fmaf(a[q], u0, -hs[q]), e1 = u1 * fmaf(a[q], u1, -hs[q]);
+          kn = kc[q];
+          e = 0.0f;  // staying put
+          if (e0 < e) {
+            e = e0;
+            kn = 0.0f;
+          }
+          if (e1 < e) {
+            e = e1;
+            kn = Lm1;
+          }
+        }
+        const unsigned mask = __ballot_sync(0xffffffffu, e < 0.0f) & live;
+        if (mask == 0u) break;
+        const int first = __ffs(mask) - 1;
+        const float u = __shfl_sync(0xffffffffu, kn - kc[q], first);
+        if (lane == first) kc[q] = kn;
+        live &= ~((2u << first) - 1u);  // this column and the ones before it are done
+        ++nchg;
+        // gradient of the later columns: hs <- hs - scale^2 H[jj, :] u
+        const float* Hj = sH + (32 * q + first) * CD_TILE + lane;
+        const float s2u = s2 * u;
+#pragma unroll
+        for (int qq = q; qq < CD1_SLOTS; ++qq) hs[qq] = fmaf(-Hj[32 * qq], s2u, hs[qq]);
       }
-      const float d0 = sc * (float)(k0 - kc), d1 = sc * (float)(k1 - kc);
-      const float e0 = d0 * fmaf(0.5f * d0, g, -hj), e1 = d1 * fmaf(0.5f * d1, g, -hj);
-      float best = 0.0f;  // staying put
-      if (e0 < best) {
-        best = e0;
-        kb = k0;
-      }
-      if (e1 < best) {
-        best = e1;
-        kb = k1;
-      }
-      acc = best < 0.0f;
     }
-    const unsigned mask = __ballot_sync(0xffffffffu, acc);
-    if (mask == 0u) {
-      c += 32;
-      continue;
+    return nchg;
+  };
+  const int ntile = pos ? sweep_tile(std::true_type{}) : sweep_tile(std::false_type{});
+  // levels and Delta/scale = k_new - k_old (zero outside the tile's columns)
+#pragma unroll
+  for (int q = 0; q < CD1_SLOTS; ++q) {
+    const int col = 32 * q + lane;
+    float dk = 0.0f;
+    if (col < tw) {
+      const int knew = (int)kc[q];
+      dk = (float)(knew - (int)ir[col]);
+      ir[col] = (uint16_t)knew;
     }
-    const int first = __ffs(mask) - 1;
-    const int jj = c + first;
-    const int knew = __shfl_sync(0xffffffffu, kb, first);
-    const int kold = __shfl_sync(0xffffffffu, kc, first);
-    const float dl = sc * (float)(knew - kold);
-    if (lane == first) {
-      ir[jj] = (uint16_t)knew;
-      si[jj] = (uint16_t)knew;
-      drow_hi[jj] = __float2half_rn((float)(knew - kold));
-    }
-    ++ntile;
-    const float* Hj = sH + jj * CD_TILE;
-    for (int i = lane; i < tw; i += 32) sh[i] = fmaf(-Hj[i], dl, sh[i]);
-    __syncwarp();
-    c = jj + 1;
+    drow_hi[col] = __float2half_rn(dk);
+    drow_lo[col] = __float2half_rn(0.0f);
   }
   if (lane == 0 && ntile > 0) {
     changes[row * sweeps + sw] += ntile;
