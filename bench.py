@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--rows", type=int, default=0,
                     help="solve only the first ROWS rows (small cases for ncu captures; "
                          "the line then names the reduced workload)")
+    ap.add_argument("--cd-panel", type=int, default=0,
+                    help="columns per CD panel (multiple of 128; 0 = automatic)")
     ap.add_argument("--spectrum-cache", default=None,
                     help="npz file: reuse the spectrum a previous run computed on the device")
     return ap.parse_args()
@@ -301,19 +303,21 @@ def run_mpq(args, world, rank, local):
     if args.rows:
         p.W = np.ascontiguousarray(p.W[:args.rows])
     cfgd = describe(p, args.config)
+    cfgd["cd_panel"] = args.cd_panel or "auto"
     m, n = p.m_out, p.n
     cb = p.codebook if p.d == 8 else None
     cache = args.spectrum_cache
     if cache and os.path.exists(cache):
         z = np.load(cache)
         plan = mpq.Plan.from_spectrum(torch.from_numpy(z["s"]).to(dev),
-                                      torch.from_numpy(z["V"]).to(dev), p.d, p.levels, codebook=cb)
+                                      torch.from_numpy(z["V"]).to(dev), p.d, p.levels, codebook=cb,
+                                      cd_panel=args.cd_panel)
         setup_s = None
     else:
         X = torch.from_numpy(p.X).to(dev)
         torch.cuda.synchronize()
         t0 = time.time()
-        plan = mpq.Plan.from_x(X, p.d, p.levels, codebook=cb)
+        plan = mpq.Plan.from_x(X, p.d, p.levels, codebook=cb, cd_panel=args.cd_panel)
         torch.cuda.synchronize()
         setup_s = time.time() - t0
         del X

@@ -93,6 +93,15 @@ typedef struct {
                              fp16 holds them and the distance terms of the
                              scores are exact in fp32 (lattice codebooks such
                              as the offset E8 set).  Ignored for d = 1. */
+  int32_t cd_panel;       /* block CD visits the columns in panels: a change
+                             updates the gradient of its own panel at once and
+                             of all other columns when the panel ends (same
+                             result, less memory traffic).  0 (default):
+                             automatic, the widest multiple of 128 columns
+                             whose slice of the gradient (rows x panel x 4
+                             bytes) fits in 32 MiB, at least 512; else the
+                             panel width in columns, a positive multiple of
+                             128 (a panel as wide as n is one panel). */
 } mpq_params;
 
 /* Fill `p` with the defaults above for block size d and codebook size K. */

@@ -54,7 +54,8 @@ __device__ __forceinline__ void p_tile(int t, int mtiles, int ntiles, int& m0, i
 __global__ void __launch_bounds__(TC_THREADS, 1)
     k_gemm_tcp(const __grid_constant__ CUtensorMap ta_hi, const __grid_constant__ CUtensorMap ta_lo,
                const __grid_constant__ CUtensorMap tb_hi, const __grid_constant__ CUtensorMap tb_lo,
-               float* __restrict__ C, int64_t ldc, int M, int N, int K, int b_k0,
+               float* __restrict__ C, int64_t ldc, int M, int N, int K, int a_k0, int b_k0,
+               int n_off,
                const float* __restrict__ row_scale, float b_scale, int accumulate, int a_exact,
                const int* __restrict__ gate, const __grid_constant__ CUtensorMap tc_out,
                int use_reduce, int* status) {
@@ -112,10 +113,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
         uint8_t* base = smem + s * P_STAGE;
         mbar_expect_tx(&full[s], a_exact ? P_STAGE - A_TILE : P_STAGE);
-        tma_load_2d(&ta_hi, &full[s], base, kt * BK, m0);
-        if (!a_exact) tma_load_2d(&ta_lo, &full[s], base + A_TILE, kt * BK, m0);
-        tma_load_2d(&tb_hi, &full[s], base + 2 * A_TILE, b_k0 + kt * BK, n0);
-        tma_load_2d(&tb_lo, &full[s], base + 2 * A_TILE + P_B_TILE, b_k0 + kt * BK, n0);
+        tma_load_2d(&ta_hi, &full[s], base, a_k0 + kt * BK, m0);
+        if (!a_exact) tma_load_2d(&ta_lo, &full[s], base + A_TILE, a_k0 + kt * BK, m0);
+        tma_load_2d(&tb_hi, &full[s], base + 2 * A_TILE, b_k0 + kt * BK, n_off + n0);
+        tma_load_2d(&tb_lo, &full[s], base + 2 * A_TILE + P_B_TILE, b_k0 + kt * BK, n_off + n0);
       }
     }
     for (uint32_t q = (it > PSTAGES ? it - PSTAGES : 0); q < it; ++q)  // copies land before exit
@@ -206,7 +207,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           }
           asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
           __syncwarp();
-          if (lane == 0) tma_reduce_add_2d(&tc_out, sb, n0 + c0, m0 + q * 32);
+          if (lane == 0) tma_reduce_add_2d(&tc_out, sb, n_off + n0 + c0, m0 + q * 32);
           ++nb;
         } else {
           // a 32 x 33 staging tile turns the lane-per-row TMEM layout into
@@ -216,7 +217,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           __syncwarp();
           const int col = n0 + c0 + lane;
           const int nrow = min(32, M - (m0 + q * 32));
-          float* cbase = C + (int64_t)(m0 + q * 32) * ldc + col;
+          float* cbase = C + (int64_t)(m0 + q * 32) * ldc + n_off + col;
           if (col < N) {
             if (accumulate) {
               float prev[32];
@@ -360,7 +361,8 @@ mpq_status gemm_tc(const SplitOperand& A, const CUtensorMap& ta_hi, const CUtens
                    float* C, int64_t ldc, int64_t M, int64_t N, int64_t K, float b_scale_host,
                    int* status, cudaStream_t st, const char* tag, const GemmOpts& o) {
   if (M <= 0 || N <= 0) return MPQ_OK;
-  if (M > A.rows_pad || N > B.rows_pad || K > A.ld || o.b_k0 + K > B.ld || o.b_k0 % 64)
+  if (M > A.rows_pad || o.n0 < 0 || o.n0 + N > B.rows_pad || o.a_k0 < 0 || o.a_k0 + K > A.ld ||
+      o.b_k0 < 0 || o.b_k0 + K > B.ld || o.a_k0 % 64 || o.b_k0 % 64)
     return fail(MPQ_ERR_INVALID_ARG, "gemm_tc: operand smaller than the problem");
   int dev = 0;
   MPQ_CUDA(cudaGetDevice(&dev));
@@ -377,7 +379,8 @@ mpq_status gemm_tc(const SplitOperand& A, const CUtensorMap& ta_hi, const CUtens
   {
     ProfScope ps_(tag, st);
     k_gemm_tcp<<<grid, TC_THREADS, P_SMEM, st>>>(
-        ta_hi, ta_lo, tb_hi, tb_lo, C, ldc, (int)M, (int)N, (int)K, (int)o.b_k0, A.row_unscale,
+        ta_hi, ta_lo, tb_hi, tb_lo, C, ldc, (int)M, (int)N, (int)K, (int)o.a_k0, (int)o.b_k0,
+        (int)o.n0, A.row_unscale,
         b_scale_host, o.accumulate ? 1 : 0, o.a_exact ? 1 : 0, o.gate, cmap, o.c_reduce ? 1 : 0,
         status);
   }

@@ -42,13 +42,13 @@ __device__ __forceinline__ void cp_async4(float* dst, const float* src, int src_
 }
 
 __global__ void __launch_bounds__(CD1_WARPS * 32, 2)
-    k_cd_tile_decide(int64_t m, int64_t n, int L, int64_t t0, int tw, int tile, int ntiles,
+    k_cd_tile_decide(int64_t m, int64_t n, int L, int64_t t0, int tw,
                      const float* __restrict__ scale, const float* __restrict__ H,
                      uint16_t* __restrict__ idx, const float* __restrict__ h, int64_t ldh,
                      int sweeps, int sw,
                      int32_t* __restrict__ changes, __half* __restrict__ dhi,
                      __half* __restrict__ dlo, int64_t lda, float* __restrict__ d_unscale,
-                     int* __restrict__ tile_count) {
+                     int* __restrict__ tile_flag, int* __restrict__ panel_flag) {
   extern __shared__ float cd_smem[];
   float* sH = cd_smem;                   // H[tile, tile], zero outside tw x tw
   float* s_rg = sH + CD_TILE * CD_TILE;  // 1 / H_jj (0 where H_jj <= 0)
@@ -162,7 +162,8 @@ __global__ void __launch_bounds__(CD1_WARPS * 32, 2)
   }
   if (lane == 0 && ntile > 0) {
     changes[row * sweeps + sw] += ntile;
-    tile_count[sw * ntiles + tile] = 1;  // gate of the update: some row changed
+    *tile_flag = 1;  // gates of the updates: some row changed
+    *panel_flag = 1;
   }
 }
 
@@ -305,14 +306,15 @@ __global__ void __launch_bounds__(256)
 // One warp per row.  At the first block of a tile every row (active or not)
 // clears its Delta row and copies h[tile] into hl.
 __global__ void __launch_bounds__(CD8_APPLY_WARPS * 32)
-    k_cd_vec_apply(int64_t m, int64_t n, int K, int64_t b, int64_t t0, int tw, int tile,
-                   int ntiles, const float* __restrict__ cb, const float* __restrict__ qtab,
+    k_cd_vec_apply(int64_t m, int64_t n, int K, int64_t b, int64_t t0, int tw,
+                   const float* __restrict__ cb, const float* __restrict__ qtab,
                    const float* __restrict__ H, const float* __restrict__ scale,
                    uint16_t* __restrict__ idx, const float* __restrict__ h, int64_t ldh,
                    float* __restrict__ hl, int sweeps, int sw, int32_t* __restrict__ changes,
                    const float* __restrict__ part_val, const int* __restrict__ part_idx,
                    int nchunks, __half* __restrict__ dhi, __half* __restrict__ dlo, int64_t lda,
-                   float* __restrict__ d_unscale, int* __restrict__ tile_count) {
+                   float* __restrict__ d_unscale, int* __restrict__ tile_flag,
+                   int* __restrict__ panel_flag) {
   __shared__ float sHb[CD_TILE][8];  // H[tile, block b]
   const int64_t B = n / 8;
   const bool first = 8 * b == t0;
@@ -377,7 +379,8 @@ __global__ void __launch_bounds__(CD8_APPLY_WARPS * 32)
   if (lane == 0) {
     idx[row * B + b] = (uint16_t)k;
     changes[row * sweeps + sw] += 1;
-    tile_count[sw * ntiles + tile] = 1;  // gate of the update: some row changed
+    *tile_flag = 1;  // gates of the updates: some row changed
+    *panel_flag = 1;
   }
   if (lane < 8) {  // Delta / scale as an fp16 pair (exact for lattice codebooks)
     const __half hi = __float2half_rn(dd[lane]);
@@ -394,6 +397,15 @@ __global__ void __launch_bounds__(CD8_APPLY_WARPS * 32)
 
 }  // namespace
 
+// Width of a CD panel: whole tiles, with the panel's slab of the gradient
+// (m x P fp32) within CD_PANEL_BYTES so that it stays in L2 while the
+// panel's tiles update it; never below CD_PANEL_MIN columns (the K of the
+// GEMM that closes a panel) and never above the padded width.
+int64_t cd_panel_cols(int64_t m, int64_t n) {
+  const int64_t fit = CD_PANEL_BYTES / (4 * std::max<int64_t>(m, 1)) / CD_TILE * CD_TILE;
+  return std::min(std::max<int64_t>(fit, CD_PANEL_MIN), round_up(n, CD_TILE));
+}
+
 mpq_status launch_cd(mpq_plan_s* p, const float* W, int64_t m, const float* scale,
                      const float* offset, uint16_t* idx, float* h, int64_t ldh, int32_t sweeps,
                      int32_t* changes, cudaStream_t st) {
@@ -402,90 +414,106 @@ mpq_status launch_cd(mpq_plan_s* p, const float* W, int64_t m, const float* scal
   if (m <= 0 || sweeps <= 0) return MPQ_OK;
   if (changes == nullptr) return fail(MPQ_ERR_INVALID_ARG, "CD needs a changes buffer");
   MPQ_CUDA(cudaMemsetAsync(changes, 0, sizeof(int32_t) * m * sweeps, st));
-  if (p->d == 1) {
-    Workspace& w = p->ws;
-    const int64_t n = p->n;
-    const int nt = (int)cdiv(n, CD_TILE);
-    MPQ_CUDA(cudaFuncSetAttribute(k_cd_tile_decide, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  CD1_SMEM));
-    MPQ_CUDA(cudaMemsetAsync(w.tile_count, 0, sizeof(int) * sweeps * nt, st));
-    for (int sw = 0; sw < sweeps; ++sw) {
-      for (int j = 0; j < nt; ++j) {
-        const int64_t t0 = (int64_t)j * CD_TILE;
-        const int tw = (int)std::min<int64_t>(CD_TILE, n - t0);
-        {
-          ProfScope ps_("k_cd_tile_decide", st);
-          k_cd_tile_decide<<<(unsigned)cdiv(m, CD1_WARPS), CD1_WARPS * 32, CD1_SMEM, st>>>(
-              m, n, p->K, t0, tw, j, nt, scale, p->H32, idx, h, ldh, sweeps, sw, changes,
-              w.As.hi, w.As.lo, w.As.ld, w.As.row_unscale, w.tile_count);
-        }
-        count_launch();
-        MPQ_TRY(check_launch("k_cd_tile_decide"));
-        GemmOpts o;
-        o.b_k0 = t0;
-        o.accumulate = true;
-        o.a_exact = true;
-        o.gate = w.tile_count + sw * nt + j;
-        o.c_reduce = (h == w.Hg) ? &w.tm_hg : nullptr;
-        MPQ_TRY(gemm_tc(w.As, w.tm_at_hi, w.tm_at_lo, p->H_s, p->tm_h_hi, p->tm_h_lo, h, ldh, m, n,
-                        tw, p->H_s.unscale_host, p->status, st, "gemm_cd_update", o));
-      }
-    }
-    return MPQ_OK;
-  }
-  // candidate scan: tensor cores for lattice codebooks (one partial minimum
-  // per codebook slice), else the SIMT kernel (one per chunk of CD8_CHUNK)
-  const bool tc = p->vec_tc;
-  const int nchunks = tc ? cd_scan_slices(m, p->K) : (int)cdiv(p->K, CD8_CHUNK);
-  float* part_val = nullptr;
-  int* part_idx = nullptr;
-  MPQ_CUDA(cudaMallocAsync(&part_val, sizeof(float) * m * nchunks, st));
-  MPQ_CUDA(cudaMallocAsync(&part_idx, sizeof(int) * m * nchunks, st));
   Workspace& w = p->ws;
   const int64_t n = p->n;
   const int nt = (int)cdiv(n, CD_TILE);
-  float* hl = w.Hl;  // m x CD_TILE tile-local gradient
-  MPQ_CUDA(cudaMemsetAsync(w.tile_count, 0, sizeof(int) * sweeps * nt, st));
+  // Columns are visited in panels of whole tiles whose slab of h (m x P
+  // fp32) stays in L2.  Each tile's changes update the gradient of its own
+  // panel only (all of the panel's columns, so the panel stays exact for the
+  // next sweep too); at the end of a panel one GEMM with K = P brings every
+  // column outside it up to date.  With one panel this is the plain
+  // per-tile update of all columns.
+  const int64_t P = p->params.cd_panel > 0 ? std::min<int64_t>(p->params.cd_panel, round_up(n, CD_TILE))
+                                           : cd_panel_cols(m, n);
+  const int np = (int)cdiv(n, P);
+  int* tile_flags = w.tile_count;                       // sweeps x nt
+  int* panel_flags = w.tile_count + (int64_t)sweeps * nt;  // sweeps x np
+  MPQ_CUDA(cudaMemsetAsync(w.tile_count, 0, sizeof(int) * sweeps * (nt + np), st));
+  const CUtensorMap* c_reduce = (h == w.Hg) ? &w.tm_hg : nullptr;
+  const bool a_exact = p->d == 1 || p->vec_tc;  // c_new - c_old is exact in fp16
+  auto update = [&](int64_t a_k0, int64_t b_k0, int64_t K, int64_t c0, int64_t c1,
+                    const int* gate) -> mpq_status {
+    if (c1 <= c0) return MPQ_OK;
+    GemmOpts o;
+    o.a_k0 = a_k0;
+    o.b_k0 = b_k0;
+    o.n0 = c0;
+    o.accumulate = true;
+    o.a_exact = a_exact;
+    o.gate = gate;
+    o.c_reduce = c_reduce;
+    return gemm_tc(w.As, w.tm_an_hi, w.tm_an_lo, p->H_s, p->tm_h_hi, p->tm_h_lo, h, ldh, m,
+                   c1 - c0, K, p->H_s.unscale_host, p->status, st, "gemm_cd_update", o);
+  };
+  // candidate scan of the vector path: tensor cores for lattice codebooks
+  // (one partial minimum per codebook slice), else the SIMT kernel (one per
+  // chunk of CD8_CHUNK codewords)
+  const bool tc = p->d == 8 && p->vec_tc;
+  const int nchunks = p->d == 1 ? 0 : tc ? cd_scan_slices(m, p->K) : (int)cdiv(p->K, CD8_CHUNK);
+  float* part_val = nullptr;
+  int* part_idx = nullptr;
+  if (p->d == 1) {
+    MPQ_CUDA(cudaFuncSetAttribute(k_cd_tile_decide, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  CD1_SMEM));
+  } else {
+    MPQ_CUDA(cudaMallocAsync(&part_val, sizeof(float) * m * nchunks, st));
+    MPQ_CUDA(cudaMallocAsync(&part_idx, sizeof(int) * m * nchunks, st));
+  }
+  float* hl = w.Hl;  // d = 8: m x CD_TILE tile-local gradient
   mpq_status rc = MPQ_OK;
   for (int sw = 0; sw < sweeps && rc == MPQ_OK; ++sw) {
-    for (int j = 0; j < nt && rc == MPQ_OK; ++j) {
-      const int64_t t0 = (int64_t)j * CD_TILE;
-      const int tw = (int)std::min<int64_t>(CD_TILE, n - t0);
-      for (int64_t b = t0 / 8; b < (t0 + tw) / 8; ++b) {
-        if (tc) {
-          rc = launch_cd_vec_scan(p, m, b, t0, scale, idx, h, ldh, hl, part_val, part_idx, nchunks, st);
-          if (rc != MPQ_OK) break;
+    for (int pi = 0; pi < np && rc == MPQ_OK; ++pi) {
+      const int64_t ps = (int64_t)pi * P, pe = std::min<int64_t>(n, ps + P);
+      int* pflag = panel_flags + (int64_t)sw * np + pi;
+      for (int64_t t0 = ps; t0 < pe && rc == MPQ_OK; t0 += CD_TILE) {
+        const int j = (int)(t0 / CD_TILE);
+        const int tw = (int)std::min<int64_t>(CD_TILE, n - t0);
+        int* tflag = tile_flags + (int64_t)sw * nt + j;
+        // the tile's Delta/scale lands at its place in the panel's A operand
+        __half* dhi = w.As.hi + (t0 - ps);
+        __half* dlo = w.As.lo + (t0 - ps);
+        if (p->d == 1) {
+          ProfScope ps_("k_cd_tile_decide", st);
+          k_cd_tile_decide<<<(unsigned)cdiv(m, CD1_WARPS), CD1_WARPS * 32, CD1_SMEM, st>>>(
+              m, n, p->K, t0, tw, scale, p->H32, idx, h, ldh, sweeps, sw, changes, dhi, dlo,
+              w.As.ld, w.As.row_unscale, tflag, pflag);
+          count_launch();
+          rc = check_launch("k_cd_tile_decide");
         } else {
-          dim3 ga((unsigned)nchunks, (unsigned)cdiv(m, CD8_ROWS));
-          ProfScope ps_("k_cd_vec_eval", st);
-          k_cd_vec_eval<<<ga, 256, 0, st>>>(m, n, p->K, b, t0, p->cb, p->qtab, p->H32, scale, idx,
-                                            h, ldh, hl, sweeps, sw, changes, part_val, part_idx,
-                                            nchunks);
+          for (int64_t b = t0 / 8; b < (t0 + tw) / 8; ++b) {
+            if (tc) {
+              rc = launch_cd_vec_scan(p, m, b, t0, scale, idx, h, ldh, hl, part_val, part_idx,
+                                      nchunks, st);
+              if (rc != MPQ_OK) break;
+            } else {
+              dim3 ga((unsigned)nchunks, (unsigned)cdiv(m, CD8_ROWS));
+              ProfScope ps_("k_cd_vec_eval", st);
+              k_cd_vec_eval<<<ga, 256, 0, st>>>(m, n, p->K, b, t0, p->cb, p->qtab, p->H32, scale,
+                                                idx, h, ldh, hl, sweeps, sw, changes, part_val,
+                                                part_idx, nchunks);
+            }
+            {
+              ProfScope ps_("k_cd_vec_apply", st);
+              k_cd_vec_apply<<<(unsigned)cdiv(m, CD8_APPLY_WARPS), CD8_APPLY_WARPS * 32, 0, st>>>(
+                  m, n, p->K, b, t0, tw, p->cb, p->qtab, p->H32, scale, idx, h, ldh, hl, sweeps,
+                  sw, changes, part_val, part_idx, nchunks, dhi, dlo, w.As.ld, w.As.row_unscale,
+                  tflag, pflag);
+            }
+            count_launch(tc ? 1 : 2);
+            rc = check_launch("k_cd_vec");
+            if (rc != MPQ_OK) break;
+          }
         }
-        {
-          ProfScope ps_("k_cd_vec_apply", st);
-          k_cd_vec_apply<<<(unsigned)cdiv(m, CD8_APPLY_WARPS), CD8_APPLY_WARPS * 32, 0, st>>>(
-              m, n, p->K, b, t0, tw, j, nt, p->cb, p->qtab, p->H32, scale, idx, h, ldh, hl,
-              sweeps, sw, changes, part_val, part_idx, nchunks, w.As.hi, w.As.lo, w.As.ld,
-              w.As.row_unscale, w.tile_count);
-        }
-        count_launch(tc ? 1 : 2);
-        rc = check_launch("k_cd_vec");
         if (rc != MPQ_OK) break;
+        rc = update(t0 - ps, t0, tw, ps, pe, tflag);  // the panel's own columns
       }
-      if (rc != MPQ_OK) break;
-      GemmOpts o;
-      o.b_k0 = t0;
-      o.accumulate = true;
-      o.a_exact = p->vec_tc;  // c_new - c_old is exact in fp16 for lattice codebooks
-      o.gate = w.tile_count + sw * nt + j;
-      o.c_reduce = (h == w.Hg) ? &w.tm_hg : nullptr;
-      rc = gemm_tc(w.As, w.tm_at_hi, w.tm_at_lo, p->H_s, p->tm_h_hi, p->tm_h_lo, h, ldh, m, n, tw,
-                   p->H_s.unscale_host, p->status, st, "gemm_cd_update", o);
+      if (rc != MPQ_OK || np == 1) continue;
+      rc = update(0, ps, pe - ps, 0, ps, pflag);  // columns before the panel
+      if (rc == MPQ_OK) rc = update(0, ps, pe - ps, pe, n, pflag);  // and after it
     }
   }
-  cudaFreeAsync(part_val, st);
-  cudaFreeAsync(part_idx, st);
+  if (part_val) cudaFreeAsync(part_val, st);
+  if (part_idx) cudaFreeAsync(part_idx, st);
   return rc;
 }
 

@@ -124,6 +124,8 @@ mpq_status validate_params(const mpq_params* q, int64_t n) {
   }
   if (n <= 0 || n % q->d != 0) return fail(MPQ_ERR_INVALID_ARG, "n must be a positive multiple of d");
   if (q->vec_engine < 0 || q->vec_engine > 2) return fail(MPQ_ERR_INVALID_ARG, "vec_engine must be 0, 1 or 2");
+  if (q->cd_panel < 0 || q->cd_panel % 128)
+    return fail(MPQ_ERR_INVALID_ARG, "cd_panel must be 0 or a positive multiple of 128");
   if (!(q->beta0 > 0.0) || !isfinite(q->beta0)) return fail(MPQ_ERR_INVALID_ARG, "beta0 must be > 0");
   if (!(q->damping >= 0.0 && q->damping <= 1.0)) return fail(MPQ_ERR_INVALID_ARG, "damping must be in [0,1]");
   if (!(q->tau > 0.0)) return fail(MPQ_ERR_INVALID_ARG, "tau must be > 0 (INFINITY = uniform prior)");
@@ -193,7 +195,7 @@ constexpr int MAX_SWEEPS = 64;
 
 int64_t ws_bytes_per_row(const mpq_plan_s* p) {
   return 3 * p->n * 4 + round_up(p->n, 32) * 4 + p->r * 4 +
-         4 * round_up(std::max<int64_t>(std::max(p->n, p->r), CD_TILE), 64) + p->B * 2 + 3 * 4 +
+         4 * round_up(std::max(p->n, p->r), CD_TILE) + p->B * 2 + 3 * 4 +
          8 * 8 + 4 + MAX_SWEEPS * 4 + (p->d == 8 ? CD_TILE * 4 : 0);
 }
 
@@ -211,8 +213,8 @@ mpq_status ensure_workspace(mpq_plan_s* p, int64_t rows) {
   auto chk = [&](mpq_status s) { if (st == MPQ_OK) st = s; };
   chk(dalloc(&w.R1, mn)); chk(dalloc(&w.X1, mn)); chk(dalloc(&w.R2, mn));
   if (st == MPQ_OK)
-    chk(alloc_split(w.As, rows, std::max<int64_t>(std::max(p->n, p->r), CD_TILE), true));
-  chk(dalloc(&w.tile_count, (int64_t)MAX_SWEEPS * cdiv(p->n, CD_TILE)));
+    chk(alloc_split(w.As, rows, round_up(std::max(p->n, p->r), CD_TILE), true));
+  chk(dalloc(&w.tile_count, (int64_t)MAX_SWEEPS * 2 * cdiv(p->n, CD_TILE)));  // tiles + panels
   w.ldh = round_up(p->n, 32);
   chk(dalloc(&w.Hg, round_up(std::max<int64_t>(rows, 32), 32) * w.ldh));
   if (p->d == 8) chk(dalloc(&w.Hl, rows * CD_TILE));
@@ -227,10 +229,6 @@ mpq_status ensure_workspace(mpq_plan_s* p, int64_t rows) {
     chk(make_tmap_f16(&w.tm_ar_hi, w.As.hi, round_up(p->r, 64), w.As.rows_pad, w.As.ld, 128));
   if (st == MPQ_OK)
     chk(make_tmap_f16(&w.tm_ar_lo, w.As.lo, round_up(p->r, 64), w.As.rows_pad, w.As.ld, 128));
-  if (st == MPQ_OK)
-    chk(make_tmap_f16(&w.tm_at_hi, w.As.hi, CD_TILE, w.As.rows_pad, w.As.ld, 128));
-  if (st == MPQ_OK)
-    chk(make_tmap_f16(&w.tm_at_lo, w.As.lo, CD_TILE, w.As.rows_pad, w.As.ld, 128));
   chk(dalloc(&w.P, rows * p->r)); chk(dalloc(&w.idx, rows * p->B));
   chk(dalloc(&w.scale, rows)); chk(dalloc(&w.offset, rows));
   chk(dalloc(&w.gamma1, rows)); chk(dalloc(&w.gamma1_0, rows)); chk(dalloc(&w.gamma2, rows));
@@ -484,6 +482,7 @@ void mpq_params_default(mpq_params* p, int32_t d, int32_t K) {
   p->alpha_min = 1e-10;
   p->alpha_max = 0.99;
   p->vec_engine = 0;
+  p->cd_panel = 0;
 }
 
 mpq_status mpq_plan_create_from_spectrum(const double* s, const double* V, int64_t n, int64_t r,

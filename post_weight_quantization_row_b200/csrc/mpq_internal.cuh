@@ -70,7 +70,6 @@ struct Workspace {
   SplitOperand As;
   CUtensorMap tm_an_hi, tm_an_lo;  // K = n view
   CUtensorMap tm_ar_hi, tm_ar_lo;  // K = r view
-  CUtensorMap tm_at_hi, tm_at_lo;  // K = CD tile view
   int* tile_count = nullptr;       // CD: changes per (sweep, tile)
   // CD gradient h = H (w - x), rows x ldh (ldh = n rounded up to 32)
   float* Hg = nullptr;
@@ -182,6 +181,9 @@ mpq_status launch_cd(mpq_plan_s* p, const float* W, int64_t m, const float* scal
                      const float* offset, uint16_t* idx, float* h, int64_t ldh, int32_t sweeps,
                      int32_t* changes, cudaStream_t st);
 constexpr int CD_TILE = 128;  // columns per scalar CD tile (multiple of 64)
+constexpr int64_t CD_PANEL_BYTES = 32ll << 20;  // L2-resident slab of the CD gradient
+constexpr int64_t CD_PANEL_MIN = 512;           // narrowest CD panel (columns)
+int64_t cd_panel_cols(int64_t m, int64_t n);
 mpq_status launch_check_finite(const float* x, int64_t count, int* status, cudaStream_t st);
 
 // tensor-core GEMM (gemm_tc.cu): C = diag(A.row_unscale) (A B^T) * b_scale
@@ -191,6 +193,8 @@ mpq_status split_global(const float* src, int64_t rows, int64_t K, SplitOperand*
                         cudaStream_t st);
 struct GemmOpts {
   int64_t b_k0 = 0;         // K offset into B (a multiple of 64)
+  int64_t a_k0 = 0;         // K offset into A (a multiple of 64)
+  int64_t n0 = 0;           // first output column (= first row of B)
   bool accumulate = false;  // C += result instead of C = result
   bool a_exact = false;     // A_lo is zero: skip its load and product
   const int* gate = nullptr;  // device int; 0 -> the launch does nothing
