@@ -432,7 +432,7 @@ mpq_status launch_cd(mpq_plan_s* p, const float* W, int64_t m, const float* scal
   const CUtensorMap* c_reduce = (h == w.Hg) ? &w.tm_hg : nullptr;
   const bool a_exact = p->d == 1 || p->vec_tc;  // c_new - c_old is exact in fp16
   auto update = [&](int64_t a_k0, int64_t b_k0, int64_t K, int64_t c0, int64_t c1,
-                    const int* gate) -> mpq_status {
+                    const int* gate, const char* tag) -> mpq_status {
     if (c1 <= c0) return MPQ_OK;
     GemmOpts o;
     o.a_k0 = a_k0;
@@ -443,7 +443,7 @@ mpq_status launch_cd(mpq_plan_s* p, const float* W, int64_t m, const float* scal
     o.gate = gate;
     o.c_reduce = c_reduce;
     return gemm_tc(w.As, w.tm_an_hi, w.tm_an_lo, p->H_s, p->tm_h_hi, p->tm_h_lo, h, ldh, m,
-                   c1 - c0, K, p->H_s.unscale_host, p->status, st, "gemm_cd_update", o);
+                   c1 - c0, K, p->H_s.unscale_host, p->status, st, tag, o);
   };
   // candidate scan of the vector path: tensor cores for lattice codebooks
   // (one partial minimum per codebook slice), else the SIMT kernel (one per
@@ -462,6 +462,7 @@ mpq_status launch_cd(mpq_plan_s* p, const float* W, int64_t m, const float* scal
   float* hl = w.Hl;  // d = 8: m x CD_TILE tile-local gradient
   mpq_status rc = MPQ_OK;
   for (int sw = 0; sw < sweeps && rc == MPQ_OK; ++sw) {
+    const bool last = sw == sweeps - 1;
     for (int pi = 0; pi < np && rc == MPQ_OK; ++pi) {
       const int64_t ps = (int64_t)pi * P, pe = std::min<int64_t>(n, ps + P);
       int* pflag = panel_flags + (int64_t)sw * np + pi;
@@ -505,11 +506,13 @@ mpq_status launch_cd(mpq_plan_s* p, const float* W, int64_t m, const float* scal
           }
         }
         if (rc != MPQ_OK) break;
-        rc = update(t0 - ps, t0, tw, ps, pe, tflag);  // the panel's own columns
+        // the panel's columns; in the last sweep only the ones still to be
+        // visited (the gradient is not read after it)
+        rc = update(t0 - ps, t0, tw, last ? t0 + tw : ps, pe, tflag, "gemm_cd_update");
       }
       if (rc != MPQ_OK || np == 1) continue;
-      rc = update(0, ps, pe - ps, 0, ps, pflag);  // columns before the panel
-      if (rc == MPQ_OK) rc = update(0, ps, pe - ps, pe, n, pflag);  // and after it
+      if (!last) rc = update(0, ps, pe - ps, 0, ps, pflag, "gemm_cd_panel");  // columns before
+      if (rc == MPQ_OK) rc = update(0, ps, pe - ps, pe, n, pflag, "gemm_cd_panel");  // and after
     }
   }
   if (part_val) cudaFreeAsync(part_val, st);

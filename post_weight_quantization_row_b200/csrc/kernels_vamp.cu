@@ -17,6 +17,7 @@ namespace mpq {
 namespace {
 
 constexpr int ROW_THREADS = 256;
+constexpr int ROW_UNROLL = 4;  // elements per thread whose loads are in flight together
 
 // ------------------------------------------------------------ reductions ---
 template <typename T, typename Op>
@@ -236,9 +237,8 @@ __global__ void __launch_bounds__(ROW_THREADS)
   auto weights = [&](auto prec) -> float {
   constexpr bool PRECISE = decltype(prec)::value;
   float acc = 0.0f;
-  for (int64_t j = threadIdx.x; j < n; j += blockDim.x) {
-    const int64_t o = row * n + j;
-    const float r = R1[o];
+  // one weight: r1 (and w for the anchored prior) already loaded
+  auto element = [&](const int64_t o, const float r, const float wr) {
     // nearest level and the offset from it in level units, dt ~ dh + dl
     // (the pair matters only in the high-precision rows)
     float ks, dh, dl;
@@ -266,7 +266,7 @@ __global__ void __launch_bounds__(ROW_THREADS)
       }
     } else {
       // anchored prior: the effective centre mixes r and w (fp64, rare path)
-      const double tt = (g * ((double)r - doff) + ga * ((double)W[o] - doff)) * inv_dsc / geff;
+      const double tt = (g * ((double)r - doff) + ga * ((double)wr - doff)) * inv_dsc / geff;
       const double kd = fmin(fmax(ceil(tt - 0.5), 0.0), (double)(L - 1));
       ks = (float)kd;
       const double dtd = tt - kd;
@@ -327,6 +327,22 @@ __global__ void __launch_bounds__(ROW_THREADS)
     if (vblock) vblock[o] = v;
     if (idx) idx[o] = (uint16_t)kstar;
     acc += v;
+  };
+  // ROW_UNROLL weights per thread and pass, all loads issued before the
+  // first is used (one load in flight per thread cannot cover HBM latency)
+  for (int64_t j0 = threadIdx.x; j0 < n; j0 += ROW_UNROLL * blockDim.x) {
+    float rv[ROW_UNROLL], wv[ROW_UNROLL];
+#pragma unroll
+    for (int u = 0; u < ROW_UNROLL; ++u) {
+      const int64_t j = j0 + (int64_t)u * blockDim.x;
+      rv[u] = j < n ? R1[row * n + j] : 0.0f;
+      wv[u] = (anchored && j < n) ? W[row * n + j] : 0.0f;
+    }
+#pragma unroll
+    for (int u = 0; u < ROW_UNROLL; ++u) {
+      const int64_t j = j0 + (int64_t)u * blockDim.x;
+      if (j < n) element(row * n + j, rv[u], wv[u]);
+    }
   }
   return acc;
   };
@@ -510,19 +526,41 @@ __global__ void __launch_bounds__(ROW_THREADS)
   __syncthreads();
   const float c = cf;
   float mx = 0.0f;
-  for (int64_t j = threadIdx.x; j < n; j += blockDim.x) {
-    const int64_t o = row * n + j;
-    const float r1 = R1[o];
-    const float r2 = fmaf(c, X1[o] - r1, r1);
-    R2[o] = r2;
-    mx = fmaxf(mx, fabsf(W[o] - r2));
+  for (int64_t j0 = threadIdx.x; j0 < n; j0 += ROW_UNROLL * blockDim.x) {
+    float r1v[ROW_UNROLL], xv[ROW_UNROLL], wv[ROW_UNROLL];
+#pragma unroll
+    for (int u = 0; u < ROW_UNROLL; ++u) {
+      const int64_t j = j0 + (int64_t)u * blockDim.x;
+      const bool in = j < n;
+      r1v[u] = in ? R1[row * n + j] : 0.0f;
+      xv[u] = in ? X1[row * n + j] : 0.0f;
+      wv[u] = in ? W[row * n + j] : 0.0f;
+    }
+#pragma unroll
+    for (int u = 0; u < ROW_UNROLL; ++u) {
+      const int64_t j = j0 + (int64_t)u * blockDim.x;
+      if (j < n) {
+        const float r2 = fmaf(c, xv[u] - r1v[u], r1v[u]);
+        R2[row * n + j] = r2;
+        mx = fmaxf(mx, fabsf(wv[u] - r2));
+      }
+    }
   }
   mx = block_reduce(mx, MaxF(), fs);
   const int ex = split_exponent(mx);
   const float down = ldexpf(1.0f, -ex);
-  for (int64_t j = threadIdx.x; j < ldn; j += blockDim.x) {
-    const float x = (j < n) ? (W[row * n + j] - R2[row * n + j]) * down : 0.0f;
-    split_store(x, ahi, alo, row * lda + j);
+  for (int64_t j0 = threadIdx.x; j0 < ldn; j0 += ROW_UNROLL * blockDim.x) {
+    float xv[ROW_UNROLL];
+#pragma unroll
+    for (int u = 0; u < ROW_UNROLL; ++u) {
+      const int64_t j = j0 + (int64_t)u * blockDim.x;
+      xv[u] = (j < n) ? (W[row * n + j] - R2[row * n + j]) * down : 0.0f;
+    }
+#pragma unroll
+    for (int u = 0; u < ROW_UNROLL; ++u) {
+      const int64_t j = j0 + (int64_t)u * blockDim.x;
+      if (j < ldn) split_store(xv[u], ahi, alo, row * lda + j);
+    }
   }
   if (threadIdx.x == 0) a_unscale[row] = ldexpf(1.0f, ex);
 }
@@ -554,10 +592,8 @@ __global__ void __launch_bounds__(ROW_THREADS)
   double a2s = 0.0, bs = 0.0;
   float mx = 0.0f;
   const float bf = (float)b, g2f = (float)g2;
-  for (int64_t l = threadIdx.x; l < r; l += blockDim.x) {
+  auto element = [&](const int64_t l, const float sl, const float pl) {
     // per element in fp32 (relative error ~1e-7), sums in fp64
-    const float sl = s32[l];
-    const float pl = P[row * r + l];
     const float u = sl * pl;
     const float den = fmaf(bf * sl, sl, g2f);
     const float inv = 1.0f / den;
@@ -568,15 +604,38 @@ __global__ void __launch_bounds__(ROW_THREADS)
     const float q = full_rank ? -f * pl : (1.0f - f) * pl;
     P[row * r + l] = q;
     mx = fmaxf(mx, fabsf(q));
+  };
+  for (int64_t l0 = threadIdx.x; l0 < r; l0 += ROW_UNROLL * blockDim.x) {
+    float sv[ROW_UNROLL], pv[ROW_UNROLL];
+#pragma unroll
+    for (int u = 0; u < ROW_UNROLL; ++u) {
+      const int64_t l = l0 + (int64_t)u * blockDim.x;
+      sv[u] = l < r ? s32[l] : 0.0f;
+      pv[u] = l < r ? P[row * r + l] : 0.0f;
+    }
+#pragma unroll
+    for (int u = 0; u < ROW_UNROLL; ++u) {
+      const int64_t l = l0 + (int64_t)u * blockDim.x;
+      if (l < r) element(l, sv[u], pv[u]);
+    }
   }
   a2s = block_sum(a2s, ds);
   bs = block_sum(bs, ds);
   mx = block_reduce(mx, MaxF(), fs);
   const int ex = split_exponent(mx);
   const float down = ldexpf(1.0f, -ex);
-  for (int64_t l = threadIdx.x; l < ldr; l += blockDim.x) {
-    const float x = (l < r) ? P[row * r + l] * down : 0.0f;
-    split_store(x, ahi, alo, row * lda + l);
+  for (int64_t l0 = threadIdx.x; l0 < ldr; l0 += ROW_UNROLL * blockDim.x) {
+    float xv[ROW_UNROLL];
+#pragma unroll
+    for (int u = 0; u < ROW_UNROLL; ++u) {
+      const int64_t l = l0 + (int64_t)u * blockDim.x;
+      xv[u] = (l < r) ? P[row * r + l] * down : 0.0f;
+    }
+#pragma unroll
+    for (int u = 0; u < ROW_UNROLL; ++u) {
+      const int64_t l = l0 + (int64_t)u * blockDim.x;
+      if (l < ldr) split_store(xv[u], ahi, alo, row * lda + l);
+    }
   }
   if (threadIdx.x == 0) {
     a_unscale[row] = ldexpf(1.0f, ex);
@@ -607,16 +666,30 @@ __global__ void __launch_bounds__(ROW_THREADS)
   const int64_t row = blockIdx.x;
   const float c = (float)coef[row];
   const float k = (float)kappa[row];
-  for (int64_t j = threadIdx.x; j < n; j += blockDim.x) {
-    const int64_t o = row * n + j;
-    const float g = G[o], r2 = R2[o];
-    if (full_rank) {
-      const float w = W[o];
-      R1[o] = fmaf(c, g, fmaf(k, w - r2, w));
-      if (xhat2) xhat2[o] = w + g;
-    } else {
-      R1[o] = fmaf(c, g, r2);
-      if (xhat2) xhat2[o] = r2 + g;
+  for (int64_t j0 = threadIdx.x; j0 < n; j0 += ROW_UNROLL * blockDim.x) {
+    float gv[ROW_UNROLL], r2v[ROW_UNROLL], wv[ROW_UNROLL];
+#pragma unroll
+    for (int u = 0; u < ROW_UNROLL; ++u) {
+      const int64_t j = j0 + (int64_t)u * blockDim.x;
+      const bool in = j < n;
+      gv[u] = in ? G[row * n + j] : 0.0f;
+      r2v[u] = in ? R2[row * n + j] : 0.0f;
+      wv[u] = (in && full_rank) ? W[row * n + j] : 0.0f;
+    }
+#pragma unroll
+    for (int u = 0; u < ROW_UNROLL; ++u) {
+      const int64_t j = j0 + (int64_t)u * blockDim.x;
+      if (j >= n) continue;
+      const int64_t o = row * n + j;
+      const float g = gv[u], r2 = r2v[u];
+      if (full_rank) {
+        const float w = wv[u];
+        R1[o] = fmaf(c, g, fmaf(k, w - r2, w));
+        if (xhat2) xhat2[o] = w + g;
+      } else {
+        R1[o] = fmaf(c, g, r2);
+        if (xhat2) xhat2[o] = r2 + g;
+      }
     }
   }
 }
