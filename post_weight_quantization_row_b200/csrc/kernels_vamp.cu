@@ -198,6 +198,144 @@ __global__ void __launch_bounds__(ROW_THREADS)
 // Posterior over levels k = 0..L-1 (weights scale*k + offset) of
 // q(k) ~ exp(-gamma1/2 (scale k + offset - r)^2) [* anchor]; in level units
 // t = (r - offset)/scale, g = gamma1 scale^2, logit_k = -g/2 (k - t)^2.
+
+// per-row constants (the stage kernel and the fused VAMP row kernel share them)
+struct ScalarDen {
+  float sc, off, inv_sc, Lm1, sc2f, A2;
+  double doff, inv_dsc, g, ga, geff;
+  int L, hw, nlev;
+  bool anchored, precise;
+};
+
+__device__ __forceinline__ ScalarDen scalar_den_row(float sc, float off, double gamma1, int L,
+                                                    bool anchored, double gamma1_0,
+                                                    double inv_tau2) {
+  ScalarDen c;
+  c.sc = sc;
+  c.off = off;
+  const double dsc = sc;
+  c.doff = off;
+  c.inv_dsc = 1.0 / dsc;
+  const double sc2 = dsc * dsc;
+  c.g = fmin(gamma1 * sc2, 1e30);
+  c.anchored = anchored;
+  c.ga = anchored ? fmin(gamma1_0 * inv_tau2 * sc2, 1e30) : 0.0;
+  c.geff = c.g + c.ga;
+  c.A2 = (float)(-0.5 * c.geff * 1.4426950408889634);  // -geff/2 log2(e)
+  c.L = L;
+  // Levels far from the nearest one carry no weight: with |dt| <= 1/2 (or dt
+  // pointing away from the grid at its ends) the log2-weight of level k* + dk
+  // relative to k* is at most A2 (dk^2 - |dk|), so a window of 2hw+1 levels
+  // with |A2| hw (hw+1) >= 64 drops only weights below 2^-64 of the largest
+  // (at most 2^-55 relative in the moments).  hw is uniform over the row.
+  c.hw = L;  // half-width of the window
+  if (-c.A2 > 0.0f) {
+    const double w = ceil(0.5 * (-1.0 + sqrt(1.0 + 256.0 / (double)(-c.A2))));
+    c.hw = (int)fmin(w, (double)L);
+  }
+  // high precision (|A| > 5): the exact exponent form below, over the window
+  c.precise = -c.A2 > 5.0f;
+  c.nlev = min(2 * c.hw + 1, L);
+  c.inv_sc = (float)c.inv_dsc;
+  c.Lm1 = (float)(L - 1);
+  c.sc2f = (float)sc2;
+  return c;
+}
+
+// One weight: cavity r (and w for the anchored prior) -> posterior mean xh,
+// variance (returned) and the most likely level kstar.  Instantiated per
+// precision regime and prior, both uniform over a row.
+template <bool PRECISE, bool ANCH, int LT>
+__device__ __forceinline__ float scalar_den_elem(const ScalarDen& c, const float r, const float wr,
+                                                 float& xh, int& kstar) {
+  const float sc = c.sc, off = c.off, inv_sc = c.inv_sc, A2 = c.A2;
+  // nearest level and the offset from it in level units, dt ~ dh + dl
+  // (the pair matters only in the high-precision rows)
+  float ks, dh, dl;
+  if constexpr (!ANCH) {
+    ks = fminf(fmaxf(ceilf((r - off) * inv_sc - 0.5f), 0.0f), c.Lm1);
+    // r - (scale ks + offset) without rounding the level value: error-free
+    // products and sums (Dekker / Knuth) give it as d0 + lo.  The explicitly
+    // rounded intrinsics keep the compiler from contracting or
+    // reassociating these steps.
+    const float pr = __fmul_rn(sc, ks);
+    const float pe = fmaf(sc, ks, -pr);
+    const float s = __fadd_rn(pr, off);
+    const float bb = __fsub_rn(s, pr);
+    const float se = __fadd_rn(__fsub_rn(pr, __fsub_rn(s, bb)), __fsub_rn(off, bb));
+    const float d0 = __fsub_rn(r, s);
+    if constexpr (PRECISE) {
+      const float b2 = __fsub_rn(d0, r);
+      const float de = __fadd_rn(__fsub_rn(r, __fsub_rn(d0, b2)), __fsub_rn(-s, b2));  // r - s = d0 + de
+      const float lo = __fsub_rn(de, __fadd_rn(pe, se));
+      dh = __fmul_rn(__fadd_rn(d0, lo), inv_sc);
+      dl = __fmul_rn(__fadd_rn(fmaf(-dh, sc, d0), lo), inv_sc);
+    } else {
+      dh = __fmul_rn(__fsub_rn(d0, __fadd_rn(pe, se)), inv_sc);
+      dl = 0.0f;
+    }
+  } else {
+    // anchored prior: the effective centre mixes r and w (fp64, rare path)
+    const double tt = (c.g * ((double)r - c.doff) + c.ga * ((double)wr - c.doff)) * c.inv_dsc / c.geff;
+    const double kd = fmin(fmax(ceil(tt - 0.5), 0.0), (double)(c.L - 1));
+    ks = (float)kd;
+    const double dtd = tt - kd;
+    dh = (float)dtd;
+    dl = (float)(dtd - (double)dh);
+  }
+  kstar = (int)ks;
+  float S0 = 0.0f, S1 = 0.0f, S2 = 0.0f;
+  if constexpr (PRECISE) {
+    // q_k / q_k* = 2^(A dk (dk - 2 dt)) with dk = k - k* an exact integer and
+    // A = -geff/2 log2(e).  Here geff is large: dk - 2 dt is formed from the
+    // pair (dh, dl) before scaling by A, so the exponent keeps fp32 accuracy
+    // relative to itself (A dk^2 - 2 A dk dt would cancel, and a plain fp32
+    // dt would cost more than 1e-4 of a weight).  min(2hw+1, L) consecutive
+    // levels around k*, shifted to stay on the grid.
+    const int k0 = min(max(kstar - c.hw, 0), c.L - c.nlev);
+#pragma unroll 4
+    for (int i = 0; i < c.nlev; ++i) {
+      const float dk = (float)(k0 + i) - ks;
+      const float e = fast_exp2((A2 * dk) * fmaf(-2.0f, dl, fmaf(-2.0f, dh, dk)));
+      S0 += e;
+      const float ed = e * dk;
+      S1 += ed;
+      S2 = fmaf(ed, dk, S2);
+    }
+  } else {
+    // q_k / q_k* = 2^(dk (A dk + B)), B = -2 A dt: with |A| <= 5 the
+    // rounding of B costs under 1e-5 of a weight.  All L levels in one fixed
+    // loop (no lane-dependent trip counts, so warps do not diverge), one
+    // hardware 2^x per level.
+    const float B2 = -2.0f * A2 * dh;
+    if (LT > 0) {
+#pragma unroll
+      for (int k = 0; k < (LT > 0 ? LT : 1); ++k) {
+        const float dk = (float)k - ks;
+        const float e = fast_exp2(fmaf(A2, dk, B2) * dk);
+        S0 += e;
+        const float ed = e * dk;
+        S1 += ed;
+        S2 = fmaf(ed, dk, S2);
+      }
+    } else {
+      for (int k = 0; k < c.L; ++k) {
+        const float dk = (float)k - ks;
+        const float e = fast_exp2(fmaf(A2, dk, B2) * dk);
+        S0 += e;
+        const float ed = e * dk;
+        S1 += ed;
+        S2 = fmaf(ed, dk, S2);
+      }
+    }
+  }
+  const float inv = __frcp_rn(S0);
+  const float m1 = S1 * inv;
+  const float var = fmaxf(fmaf(S2, inv, -m1 * m1), 0.0f);
+  xh = fmaf(sc, ks + m1, off);
+  return c.sc2f * var;
+}
+
 template <int LT>
 __global__ void __launch_bounds__(ROW_THREADS)
     k_denoise_scalar(const float* __restrict__ R1, const double* __restrict__ gamma1,
@@ -208,145 +346,46 @@ __global__ void __launch_bounds__(ROW_THREADS)
                      double* __restrict__ vsum, uint16_t* __restrict__ idx) {
   __shared__ double ds[33];
   const int64_t row = blockIdx.x;
-  const float sc = scale[row], off = offset[row];
-  const double dsc = sc, doff = off, inv_dsc = 1.0 / dsc;
-  const double sc2 = dsc * dsc;
-  const double g = fmin(gamma1[row] * sc2, 1e30);
   const bool anchored = (W != nullptr);
-  const double ga = anchored ? fmin(gamma1_0[row] * inv_tau2 * sc2, 1e30) : 0.0;
-  const double geff = g + ga;
-  const float A2 = (float)(-0.5 * geff * 1.4426950408889634);  // -geff/2 log2(e)
-  // Levels far from the nearest one carry no weight: with |dt| <= 1/2 (or dt
-  // pointing away from the grid at its ends) the log2-weight of level k* + dk
-  // relative to k* is at most A2 (dk^2 - |dk|), so a window of 2hw+1 levels
-  // with |A2| hw (hw+1) >= 64 drops only weights below 2^-64 of the largest
-  // (at most 2^-55 relative in the moments).  hw is uniform over the row's CTA.
-  int hw = L;  // half-width of the window
-  if (-A2 > 0.0f) {
-    const double w = ceil(0.5 * (-1.0 + sqrt(1.0 + 256.0 / (double)(-A2))));
-    hw = (int)fmin(w, (double)L);
-  }
-  // high precision (|A| > 5): the exact exponent form below, over the window
-  const bool precise = -A2 > 5.0f;
-  const int nlev = min(2 * hw + 1, L);
-  const float inv_sc = (float)inv_dsc;
-  const float Lm1 = (float)(L - 1);
-  const float sc2f = (float)sc2;
-  // the per-weight loop, instantiated once per precision regime so that the
-  // row-uniform choice costs no branch per weight
-  auto weights = [&](auto prec) -> float {
-  constexpr bool PRECISE = decltype(prec)::value;
-  float acc = 0.0f;
-  // one weight: r1 (and w for the anchored prior) already loaded
-  auto element = [&](const int64_t o, const float r, const float wr) {
-    // nearest level and the offset from it in level units, dt ~ dh + dl
-    // (the pair matters only in the high-precision rows)
-    float ks, dh, dl;
-    if (!anchored) {
-      ks = fminf(fmaxf(ceilf((r - off) * inv_sc - 0.5f), 0.0f), Lm1);
-      // r - (scale ks + offset) without rounding the level value: error-free
-      // products and sums (Dekker / Knuth) give it as d0 + lo.  The explicitly
-      // rounded intrinsics keep the compiler from contracting or
-      // reassociating these steps.
-      const float pr = __fmul_rn(sc, ks);
-      const float pe = fmaf(sc, ks, -pr);
-      const float s = __fadd_rn(pr, off);
-      const float bb = __fsub_rn(s, pr);
-      const float se = __fadd_rn(__fsub_rn(pr, __fsub_rn(s, bb)), __fsub_rn(off, bb));
-      const float d0 = __fsub_rn(r, s);
-      if constexpr (PRECISE) {
-        const float b2 = __fsub_rn(d0, r);
-        const float de = __fadd_rn(__fsub_rn(r, __fsub_rn(d0, b2)), __fsub_rn(-s, b2));  // r - s = d0 + de
-        const float lo = __fsub_rn(de, __fadd_rn(pe, se));
-        dh = __fmul_rn(__fadd_rn(d0, lo), inv_sc);
-        dl = __fmul_rn(__fadd_rn(fmaf(-dh, sc, d0), lo), inv_sc);
-      } else {
-        dh = __fmul_rn(__fsub_rn(d0, __fadd_rn(pe, se)), inv_sc);
-        dl = 0.0f;
-      }
-    } else {
-      // anchored prior: the effective centre mixes r and w (fp64, rare path)
-      const double tt = (g * ((double)r - doff) + ga * ((double)wr - doff)) * inv_dsc / geff;
-      const double kd = fmin(fmax(ceil(tt - 0.5), 0.0), (double)(L - 1));
-      ks = (float)kd;
-      const double dtd = tt - kd;
-      dh = (float)dtd;
-      dl = (float)(dtd - (double)dh);
-    }
-    const int kstar = (int)ks;
-    float S0 = 0.0f, S1 = 0.0f, S2 = 0.0f;
-    if constexpr (PRECISE) {
-      // q_k / q_k* = 2^(A dk (dk - 2 dt)) with dk = k - k* an exact integer and
-      // A = -geff/2 log2(e).  Here geff is large: dk - 2 dt is formed from the
-      // pair (dh, dl) before scaling by A, so the exponent keeps fp32 accuracy
-      // relative to itself (A dk^2 - 2 A dk dt would cancel, and a plain fp32
-      // dt would cost more than 1e-4 of a weight).  min(2hw+1, L) consecutive
-      // levels around k*, shifted to stay on the grid.
-      const int k0 = min(max(kstar - hw, 0), L - nlev);
-#pragma unroll 4
-      for (int i = 0; i < nlev; ++i) {
-        const float dk = (float)(k0 + i) - ks;
-        const float e = fast_exp2((A2 * dk) * fmaf(-2.0f, dl, fmaf(-2.0f, dh, dk)));
-        S0 += e;
-        const float ed = e * dk;
-        S1 += ed;
-        S2 = fmaf(ed, dk, S2);
-      }
-    } else {
-      // q_k / q_k* = 2^(dk (A dk + B)), B = -2 A dt: with |A| <= 5 the
-      // rounding of B costs under 1e-5 of a weight.  All L levels in one fixed
-      // loop (no lane-dependent trip counts, so warps do not diverge), one
-      // hardware 2^x per level.
-      const float B2 = -2.0f * A2 * dh;
-      if (LT > 0) {
+  const ScalarDen c = scalar_den_row(scale[row], offset[row], gamma1[row], L, anchored,
+                                     anchored ? gamma1_0[row] : 0.0, inv_tau2);
+  // the per-weight loop, instantiated once per precision regime and prior so
+  // that the row-uniform choices cost no branch per weight
+  auto weights = [&](auto prec, auto anch) -> float {
+    constexpr bool PRECISE = decltype(prec)::value;
+    constexpr bool ANCH = decltype(anch)::value;
+    float acc = 0.0f;
+    // ROW_UNROLL weights per thread and pass, all loads issued before the
+    // first is used
+    for (int64_t j0 = threadIdx.x; j0 < n; j0 += ROW_UNROLL * blockDim.x) {
+      float rv[ROW_UNROLL], wv[ROW_UNROLL];
 #pragma unroll
-        for (int k = 0; k < (LT > 0 ? LT : 1); ++k) {
-          const float dk = (float)k - ks;
-          const float e = fast_exp2(fmaf(A2, dk, B2) * dk);
-          S0 += e;
-          const float ed = e * dk;
-          S1 += ed;
-          S2 = fmaf(ed, dk, S2);
-        }
-      } else {
-        for (int k = 0; k < L; ++k) {
-          const float dk = (float)k - ks;
-          const float e = fast_exp2(fmaf(A2, dk, B2) * dk);
-          S0 += e;
-          const float ed = e * dk;
-          S1 += ed;
-          S2 = fmaf(ed, dk, S2);
+      for (int u = 0; u < ROW_UNROLL; ++u) {
+        const int64_t j = j0 + (int64_t)u * blockDim.x;
+        rv[u] = j < n ? R1[row * n + j] : 0.0f;
+        wv[u] = (ANCH && j < n) ? W[row * n + j] : 0.0f;
+      }
+#pragma unroll
+      for (int u = 0; u < ROW_UNROLL; ++u) {
+        const int64_t j = j0 + (int64_t)u * blockDim.x;
+        if (j < n) {
+          const int64_t o = row * n + j;
+          float xh;
+          int ks;
+          const float v = scalar_den_elem<PRECISE, ANCH, LT>(c, rv[u], wv[u], xh, ks);
+          xhat[o] = xh;
+          if (vblock) vblock[o] = v;
+          if (idx) idx[o] = (uint16_t)ks;
+          acc += v;
         }
       }
     }
-    const float inv = __frcp_rn(S0);
-    const float m1 = S1 * inv;
-    const float var = fmaxf(fmaf(S2, inv, -m1 * m1), 0.0f);
-    xhat[o] = fmaf(sc, ks + m1, off);
-    const float v = sc2f * var;
-    if (vblock) vblock[o] = v;
-    if (idx) idx[o] = (uint16_t)kstar;
-    acc += v;
+    return acc;
   };
-  // ROW_UNROLL weights per thread and pass, all loads issued before the
-  // first is used (one load in flight per thread cannot cover HBM latency)
-  for (int64_t j0 = threadIdx.x; j0 < n; j0 += ROW_UNROLL * blockDim.x) {
-    float rv[ROW_UNROLL], wv[ROW_UNROLL];
-#pragma unroll
-    for (int u = 0; u < ROW_UNROLL; ++u) {
-      const int64_t j = j0 + (int64_t)u * blockDim.x;
-      rv[u] = j < n ? R1[row * n + j] : 0.0f;
-      wv[u] = (anchored && j < n) ? W[row * n + j] : 0.0f;
-    }
-#pragma unroll
-    for (int u = 0; u < ROW_UNROLL; ++u) {
-      const int64_t j = j0 + (int64_t)u * blockDim.x;
-      if (j < n) element(row * n + j, rv[u], wv[u]);
-    }
-  }
-  return acc;
-  };
-  const float acc = precise ? weights(std::true_type{}) : weights(std::false_type{});
+  using T_ = std::true_type;
+  using F_ = std::false_type;
+  const float acc = anchored ? (c.precise ? weights(T_{}, T_{}) : weights(F_{}, T_{}))
+                             : (c.precise ? weights(T_{}, F_{}) : weights(F_{}, F_{}));
   const double tot = block_sum((double)acc, ds);
   if (threadIdx.x == 0) vsum[row] = tot;
 }
@@ -498,6 +537,18 @@ __global__ void __launch_bounds__(ROW_THREADS)
 }
 
 // ------------------------------------------------- extrinsic d -> linear ---
+// Row scalars: alpha1 = gamma1 vsum / n and gamma2 = gamma1 (1 - alpha1) /
+// alpha1, both clipped (clips counted); returns 1 / (1 - alpha1).
+__device__ __forceinline__ float d2l_row(double g1, double vsum, int64_t n, double g0, double glo,
+                                         double ghi, double amin, double amax, double* gamma2,
+                                         int32_t* clamps) {
+  int cnt = 0;
+  const double a1 = clip_count(g1 * vsum / (double)n, amin, amax, &cnt);
+  *gamma2 = clip_count(g1 * (1.0 - a1) / a1, glo * g0, ghi * g0, &cnt);
+  if (clamps) *clamps += cnt;
+  return (float)(1.0 / (1.0 - a1));
+}
+
 // alpha1 = gamma1 vsum / n (clipped), gamma2 = gamma1 (1 - alpha1)/alpha1
 // (clipped), r2 = r1 + (xhat1 - r1)/(1 - alpha1)  [= (xhat1 - alpha1 r1)/
 // (1 - alpha1) = (eta1 xhat1 - gamma1 r1)/gamma2].  Also writes the GEMM1
@@ -513,16 +564,9 @@ __global__ void __launch_bounds__(ROW_THREADS)
   __shared__ float cf;
   __shared__ float fs[33];
   const int64_t row = blockIdx.x;
-  if (threadIdx.x == 0) {
-    int cnt = 0;
-    const double g1 = gamma1[row];
-    const double a1 = clip_count(g1 * vsum[row] / (double)n, amin, amax, &cnt);
-    const double g0 = gamma1_0[row];
-    const double g2 = clip_count(g1 * (1.0 - a1) / a1, glo * g0, ghi * g0, &cnt);
-    gamma2[row] = g2;
-    cf = (float)(1.0 / (1.0 - a1));
-    if (clamps) clamps[row] += cnt;
-  }
+  if (threadIdx.x == 0)
+    cf = d2l_row(gamma1[row], vsum[row], n, gamma1_0[row], glo, ghi, amin, amax, gamma2 + row,
+                 clamps ? clamps + row : nullptr);
   __syncthreads();
   const float c = cf;
   float mx = 0.0f;
@@ -692,6 +736,125 @@ __global__ void __launch_bounds__(ROW_THREADS)
       }
     }
   }
+}
+
+// ------------------------------------------------ fused scalar VAMP row ---
+// One row of a scalar (d = 1) VAMP iteration in one pass over HBM: the
+// extrinsic linear -> denoiser step (r1 from the GEMM output G, r2 and w, as
+// in k_extrinsic_l2d; r1 = w in the first iteration), the denoiser
+// (scalar_den_elem), and the extrinsic denoiser -> linear step with the split
+// GEMM operand w - r2 (as in k_extrinsic_d2l).  r1 and x_hat1 of the row stay
+// in shared memory between the two halves; each arithmetic step is the one
+// of the separate kernels, in the same order.  MAP = 1: the marginal MAP
+// after the last iteration (l2d and the denoiser's argmax only).
+constexpr int FUSED_MAX_THREADS = 1024;
+
+template <int LT, int MAP>
+__global__ void __launch_bounds__(FUSED_MAX_THREADS)
+    k_vamp_row_scalar(const float* __restrict__ W, const float* __restrict__ G,
+                      float* __restrict__ R2, int64_t n, int first, int full_rank,
+                      const double* __restrict__ coef, const double* __restrict__ kappa,
+                      const double* __restrict__ gamma1, const float* __restrict__ scale,
+                      const float* __restrict__ offset, int L, int anchored,
+                      const double* __restrict__ gamma1_0, double inv_tau2, double glo,
+                      double ghi, double amin, double amax, __half* __restrict__ ahi,
+                      __half* __restrict__ alo, int64_t lda, int64_t ldn,
+                      float* __restrict__ a_unscale, double* __restrict__ gamma2,
+                      int32_t* __restrict__ clamps, uint16_t* __restrict__ idx) {
+  extern __shared__ float vrow[];  // r1 (then r2) and x_hat1 of the row
+  __shared__ double ds[33];
+  __shared__ float fs[33];
+  __shared__ float cf_s;
+  float* s_r = vrow;
+  float* s_x = vrow + n;
+  const int64_t row = blockIdx.x;
+  const ScalarDen c = scalar_den_row(scale[row], offset[row], gamma1[row], L, anchored != 0,
+                                     anchored ? gamma1_0[row] : 0.0, inv_tau2);
+  const float lc = first ? 0.0f : (float)coef[row];
+  const float lk = first ? 0.0f : (float)kappa[row];
+  auto pass1 = [&](auto prec, auto anch) -> float {
+    constexpr bool PRECISE = decltype(prec)::value;
+    constexpr bool ANCH = decltype(anch)::value;
+    float acc = 0.0f;
+    for (int64_t j0 = threadIdx.x; j0 < n; j0 += ROW_UNROLL * blockDim.x) {
+      float gv[ROW_UNROLL], r2v[ROW_UNROLL], wv[ROW_UNROLL];
+#pragma unroll
+      for (int u = 0; u < ROW_UNROLL; ++u) {
+        const int64_t j = j0 + (int64_t)u * blockDim.x;
+        const bool in = j < n;
+        gv[u] = (in && !first) ? G[row * n + j] : 0.0f;
+        r2v[u] = (in && !first) ? R2[row * n + j] : 0.0f;
+        wv[u] = in ? W[row * n + j] : 0.0f;
+      }
+#pragma unroll
+      for (int u = 0; u < ROW_UNROLL; ++u) {
+        const int64_t j = j0 + (int64_t)u * blockDim.x;
+        if (j >= n) continue;
+        const float w = wv[u];
+        const float r1 = first ? w
+                         : full_rank ? fmaf(lc, gv[u], fmaf(lk, w - r2v[u], w))
+                                     : fmaf(lc, gv[u], r2v[u]);
+        float xh;
+        int ks;
+        const float v = scalar_den_elem<PRECISE, ANCH, LT>(c, r1, w, xh, ks);
+        if (MAP) {
+          idx[row * n + j] = (uint16_t)ks;
+        } else {
+          s_r[j] = r1;
+          s_x[j] = xh;
+          acc += v;
+        }
+      }
+    }
+    return acc;
+  };
+  using T_ = std::true_type;
+  using F_ = std::false_type;
+  const float acc = anchored ? (c.precise ? pass1(T_{}, T_{}) : pass1(F_{}, T_{}))
+                             : (c.precise ? pass1(T_{}, F_{}) : pass1(F_{}, F_{}));
+  if (MAP) return;
+  const double vsum = block_sum((double)acc, ds);  // its barriers also publish s_r, s_x
+  if (threadIdx.x == 0)
+    cf_s = d2l_row(gamma1[row], vsum, n, gamma1_0[row], glo, ghi, amin, amax, gamma2 + row,
+                   clamps ? clamps + row : nullptr);
+  __syncthreads();
+  const float cf = cf_s;
+  float mx = 0.0f;
+  for (int64_t j0 = threadIdx.x; j0 < n; j0 += ROW_UNROLL * blockDim.x) {
+    float wv[ROW_UNROLL];
+#pragma unroll
+    for (int u = 0; u < ROW_UNROLL; ++u) {
+      const int64_t j = j0 + (int64_t)u * blockDim.x;
+      wv[u] = j < n ? W[row * n + j] : 0.0f;
+    }
+#pragma unroll
+    for (int u = 0; u < ROW_UNROLL; ++u) {
+      const int64_t j = j0 + (int64_t)u * blockDim.x;
+      if (j >= n) continue;
+      const float r1 = s_r[j];
+      const float r2 = fmaf(cf, s_x[j] - r1, r1);
+      R2[row * n + j] = r2;
+      s_r[j] = r2;
+      mx = fmaxf(mx, fabsf(wv[u] - r2));
+    }
+  }
+  mx = block_reduce(mx, MaxF(), fs);  // its barriers also publish the new s_r
+  const int ex = split_exponent(mx);
+  const float down = ldexpf(1.0f, -ex);
+  for (int64_t j0 = threadIdx.x; j0 < ldn; j0 += ROW_UNROLL * blockDim.x) {
+    float xv[ROW_UNROLL];
+#pragma unroll
+    for (int u = 0; u < ROW_UNROLL; ++u) {
+      const int64_t j = j0 + (int64_t)u * blockDim.x;
+      xv[u] = (j < n) ? (W[row * n + j] - s_r[j]) * down : 0.0f;
+    }
+#pragma unroll
+    for (int u = 0; u < ROW_UNROLL; ++u) {
+      const int64_t j = j0 + (int64_t)u * blockDim.x;
+      if (j < ldn) split_store(xv[u], ahi, alo, row * lda + j);
+    }
+  }
+  if (threadIdx.x == 0) a_unscale[row] = ldexpf(1.0f, ex);
 }
 
 // --------------------------------------------------- residual / energies ---
@@ -940,6 +1103,54 @@ mpq_status launch_extrinsic_l2d(const mpq_plan_s* p, const float* W, int64_t m, 
   }
   count_launch();
   return check_launch("k_extrinsic_l2d");
+}
+
+// Threads per row of the fused scalar kernel: its shared memory holds two
+// floats per weight; 0 when the row does not fit (the separate kernels run).
+int vamp_row_threads(int64_t n) {
+  const int64_t bytes = 8 * n;
+  if (bytes <= 56 * 1024) return 256;    // 4 CTAs per SM
+  if (bytes <= 112 * 1024) return 512;   // 2 CTAs per SM
+  if (bytes <= 220 * 1024) return 1024;  // 1 CTA per SM
+  return 0;
+}
+
+mpq_status launch_vamp_row_scalar(const mpq_plan_s* p, const float* W, int64_t m, int first,
+                                  int map, const float* G, float* R2, const double* coef,
+                                  const double* kappa, const double* gamma1, const float* scale,
+                                  const float* offset, const double* gamma1_0, SplitOperand* As,
+                                  double* gamma2, int32_t* clamps, uint16_t* idx, cudaStream_t st) {
+  if (m <= 0) return MPQ_OK;
+  const int threads = vamp_row_threads(p->n);
+  if (p->d != 1 || threads == 0) return fail(MPQ_ERR_INVALID_ARG, "fused row kernel: d = 1 rows that fit");
+  const mpq_params& q = p->params;
+  const bool anchored = std::isfinite(q.tau);
+  const double inv_tau2 = anchored ? 1.0 / (q.tau * q.tau) : 0.0;
+  const size_t smem = sizeof(float) * 2 * p->n;
+  using Kern = void (*)(const float*, const float*, float*, int64_t, int, int, const double*,
+                        const double*, const double*, const float*, const float*, int, int,
+                        const double*, double, double, double, double, double, __half*, __half*,
+                        int64_t, int64_t, float*, double*, int32_t*, uint16_t*);
+  Kern kern;
+  if (map)
+    kern = (p->K == 16) ? k_vamp_row_scalar<16, 1>
+           : (p->K == 8) ? k_vamp_row_scalar<8, 1>
+           : (p->K == 4) ? k_vamp_row_scalar<4, 1> : k_vamp_row_scalar<0, 1>;
+  else
+    kern = (p->K == 16) ? k_vamp_row_scalar<16, 0>
+           : (p->K == 8) ? k_vamp_row_scalar<8, 0>
+           : (p->K == 4) ? k_vamp_row_scalar<4, 0> : k_vamp_row_scalar<0, 0>;
+  MPQ_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  {
+    ProfScope ps_(map ? "k_vamp_row_scalar(map)" : "k_vamp_row_scalar", st);
+    kern<<<rows_grid(m), threads, smem, st>>>(
+        W, G, R2, p->n, first, p->r == p->n ? 1 : 0, coef, kappa, gamma1, scale, offset, p->K,
+        anchored ? 1 : 0, gamma1_0, inv_tau2, q.gamma_lo_rel, q.gamma_hi_rel, q.alpha_min,
+        q.alpha_max, As ? As->hi : nullptr, As ? As->lo : nullptr, As ? As->ld : 0,
+        round_up(p->n, 64), As ? As->row_unscale : nullptr, gamma2, clamps, idx);
+  }
+  count_launch();
+  return check_launch("k_vamp_row_scalar");
 }
 
 mpq_status launch_residual_split(const mpq_plan_s* p, const float* W, int64_t m,

@@ -272,24 +272,38 @@ struct SolveIO {
   const mpq_row_stats* stats;
 };
 
+mpq_status run_linear_core(mpq_plan_s* p, int64_t m, double* gamma2, const double* gamma1_0,
+                           double* beta, double* gamma1_out, float* Uprime, double* alpha2,
+                           double* beta_hat, int32_t* clamps, cudaStream_t st);
+
 // linear half-iteration on workspace state (R1 may alias W on the first call)
 mpq_status run_linear(mpq_plan_s* p, const float* W, int64_t m, const float* R1,
                       const double* gamma1, const float* X1, const double* vsum,
                       const double* gamma1_0, double* beta, float* R1_out, double* gamma1_out,
                       float* R2, double* gamma2, float* Uprime, float* xhat2, double* alpha2,
                       double* beta_hat, int32_t* clamps, cudaStream_t st) {
+  MPQ_TRY(launch_extrinsic_d2l(p, W, m, R1, gamma1, X1, vsum, gamma1_0, R2, &p->ws.As, gamma2,
+                               clamps, st));
+  MPQ_TRY(run_linear_core(p, m, gamma2, gamma1_0, beta, gamma1_out, Uprime, alpha2, beta_hat,
+                          clamps, st));
+  return launch_extrinsic_l2d(p, W, m, R2, p->ws.X1, p->ws.coef, p->ws.kappa, R1_out, xhat2, st);
+}
+
+// the linear module on the split operand w - r2 already in As: p' = V^T
+// (w - r2), its row epilogue and M-step, and G = V (D u) into X1
+mpq_status run_linear_core(mpq_plan_s* p, int64_t m, double* gamma2, const double* gamma1_0,
+                           double* beta, double* gamma1_out, float* Uprime, double* alpha2,
+                           double* beta_hat, int32_t* clamps, cudaStream_t st) {
   Workspace& w = p->ws;
   const int64_t n = p->n, r = p->r;
-  MPQ_TRY(launch_extrinsic_d2l(p, W, m, R1, gamma1, X1, vsum, gamma1_0, R2, &w.As, gamma2, clamps, st));
   // p' = V^T (w - r2)
   MPQ_TRY(gemm_tc(w.As, w.tm_an_hi, w.tm_an_lo, p->Vt_s, p->tm_vt_hi, p->tm_vt_lo, w.P, r, m, r, n,
                   p->Vt_s.unscale_host, p->status, st, "gemm_project"));
   MPQ_TRY(launch_linear_rows(p, m, w.P, gamma2, gamma1_0, beta, gamma1_out, w.coef, w.kappa,
                              alpha2, beta_hat, clamps, Uprime, &w.As, st));
   // G into X1: the denoiser output is consumed by now
-  MPQ_TRY(gemm_tc(w.As, w.tm_ar_hi, w.tm_ar_lo, p->V_s, p->tm_v_hi, p->tm_v_lo, w.X1, n, m, n, r,
-                  p->V_s.unscale_host, p->status, st, "gemm_expand"));
-  return launch_extrinsic_l2d(p, W, m, R2, w.X1, w.coef, w.kappa, R1_out, xhat2, st);
+  return gemm_tc(w.As, w.tm_ar_hi, w.tm_ar_lo, p->V_s, p->tm_v_hi, p->tm_v_lo, w.X1, n, m, n, r,
+                 p->V_s.unscale_host, p->status, st, "gemm_expand");
 }
 
 mpq_status run_cd(mpq_plan_s* p, const float* W, int64_t m, const float* scale,
@@ -335,19 +349,36 @@ mpq_status solve_batch(mpq_plan_s* p, const SolveIO& io, int64_t row0, int64_t m
   MPQ_TRY(launch_init(p, W, mb, given, w.scale, w.offset, idx, w.gamma1_0, st));
   MPQ_CUDA(cudaMemcpyAsync(w.gamma1, w.gamma1_0, sizeof(double) * mb, cudaMemcpyDeviceToDevice, st));
   MPQ_TRY(fill_f64(w.beta, mb, p->params.beta0, st));
-  const float* R1 = W;  // cavity r1_0 = w
-  float* vblock = (p->d == 8) ? w.R2 : nullptr;  // R2 is free while the denoiser runs
-  for (int t = 0; t < io.T_vamp; ++t) {
-    MPQ_TRY(launch_denoise(p, R1, w.gamma1, w.scale, w.offset, mb, W, w.gamma1_0, w.X1, vblock,
-                           w.vsum, nullptr, st));
-    MPQ_TRY(run_linear(p, W, mb, R1, w.gamma1, w.X1, w.vsum, w.gamma1_0, w.beta, w.R1, w.gamma1,
-                       w.R2, w.gamma2, nullptr, nullptr, nullptr, nullptr, clamps, st));
-    R1 = w.R1;
+  if (p->d == 1 && vamp_row_threads(n) > 0) {
+    // scalar rows: l2d, denoiser and d2l of an iteration in one fused row
+    // kernel (r1 never leaves the chip), then the linear module
+    for (int t = 0; t < io.T_vamp; ++t) {
+      MPQ_TRY(launch_vamp_row_scalar(p, W, mb, t == 0, 0, w.X1, w.R2, w.coef, w.kappa, w.gamma1,
+                                     w.scale, w.offset, w.gamma1_0, &w.As, w.gamma2, clamps,
+                                     nullptr, st));
+      MPQ_TRY(run_linear_core(p, mb, w.gamma2, w.gamma1_0, w.beta, w.gamma1, nullptr, nullptr,
+                              nullptr, clamps, st));
+    }
+    // marginal MAP: argmax of the denoiser at the last cavity
+    if (io.T_vamp > 0)
+      MPQ_TRY(launch_vamp_row_scalar(p, W, mb, 0, 1, w.X1, w.R2, w.coef, w.kappa, w.gamma1,
+                                     w.scale, w.offset, w.gamma1_0, nullptr, nullptr, nullptr, idx,
+                                     st));
+  } else {
+    const float* R1 = W;  // cavity r1_0 = w
+    float* vblock = (p->d == 8) ? w.R2 : nullptr;  // R2 is free while the denoiser runs
+    for (int t = 0; t < io.T_vamp; ++t) {
+      MPQ_TRY(launch_denoise(p, R1, w.gamma1, w.scale, w.offset, mb, W, w.gamma1_0, w.X1, vblock,
+                             w.vsum, nullptr, st));
+      MPQ_TRY(run_linear(p, W, mb, R1, w.gamma1, w.X1, w.vsum, w.gamma1_0, w.beta, w.R1,
+                         w.gamma1, w.R2, w.gamma2, nullptr, nullptr, nullptr, nullptr, clamps, st));
+      R1 = w.R1;
+    }
+    // marginal MAP: argmax of one more denoiser call
+    if (io.T_vamp > 0)
+      MPQ_TRY(launch_denoise(p, R1, w.gamma1, w.scale, w.offset, mb, W, w.gamma1_0, w.X1, vblock,
+                             w.vsum, idx, st));
   }
-  // marginal MAP: argmax of one more denoiser call
-  if (io.T_vamp > 0)
-    MPQ_TRY(launch_denoise(p, R1, w.gamma1, w.scale, w.offset, mb, W, w.gamma1_0, w.X1, vblock,
-                           w.vsum, idx, st));
   if (io.sweeps > 0) MPQ_TRY(run_cd(p, W, mb, w.scale, w.offset, idx, io.sweeps, changes, st));
   MPQ_TRY(run_energy(p, W, mb, w.scale, w.offset, idx, io.w_hat ? io.w_hat + row0 * n : nullptr,
                      io.energy ? io.energy + row0 : nullptr, st));

@@ -161,6 +161,12 @@ mpq_status launch_linear_rows(const mpq_plan_s* p, int64_t m, const float* P,
                               double* gamma1_out, double* coef, double* kappa, double* alpha2,
                               double* beta_hat, int32_t* clamps, float* Uprime, SplitOperand* As,
                               cudaStream_t st);
+int vamp_row_threads(int64_t n);  // 0: the fused scalar row kernel does not apply
+mpq_status launch_vamp_row_scalar(const mpq_plan_s* p, const float* W, int64_t m, int first,
+                                  int map, const float* G, float* R2, const double* coef,
+                                  const double* kappa, const double* gamma1, const float* scale,
+                                  const float* offset, const double* gamma1_0, SplitOperand* As,
+                                  double* gamma2, int32_t* clamps, uint16_t* idx, cudaStream_t st);
 mpq_status launch_extrinsic_l2d(const mpq_plan_s* p, const float* W, int64_t m, const float* R2,
                                 const float* G, const double* coef, const double* kappa,
                                 float* R1_out, float* xhat2, cudaStream_t st);

@@ -302,6 +302,29 @@ def _solve_compare(mpq, p, T=None, sweeps=None, min_clean=0.5):
     return ref, out
 
 
+@pytest.mark.parametrize("n", [8000, 15000, 30000])
+def test_solve_scalar_wide_rows(mpq, n):
+    # The fused scalar VAMP row kernel keeps 8 bytes per weight of a row in
+    # shared memory: n = 8000 and 15000 take its 512- and 1024-thread shapes,
+    # n = 30000 does not fit and runs the separate kernels.  No CD (rows this
+    # long always meet CD near-ties); every MAP index outside a near-tie of
+    # the oracle's logits must match, energies and terminal precisions too.
+    p = mi.small_problem(606, 3, n, 600, d=1, levels=8, T_vamp=4, cd_sweeps=0)
+    s, V, s_cu, V_cu = spectrum_cuda(p.X)
+    plan = make_plan(mpq, p, s_cu, V_cu)
+    sc, off = oracle_grid_f32(p)
+    cb = codebook_for(p)
+    ref = orc.solve(p.W, cb, s, V, 4, 0, sc.astype(np.float64), off.astype(np.float64))
+    out = plan.solve(cu(p.W), 4, 0, row_scale=cu(sc), row_offset=cu(off), stats=True)
+    got = idx_np(out["idx"])
+    clean = ref.map_gap > LOGIT_TIE_SOLVE
+    assert clean.mean() > 0.95
+    assert np.array_equal(got[clean], ref.idx[clean])
+    e_gpu = host(out["energy"]).astype(np.float64)
+    assert np.all(np.abs(e_gpu - ref.energy) <= ENERGY_TOL * ref.energy)
+    assert_scalars_close("terminal gamma1", host(out["gamma1"]), ref.gamma1, 1e-2)
+
+
 def test_solve_tiny_workload(mpq):
     p = mi.make_problem("tiny")
     _solve_compare(mpq, p, min_clean=1.0)
