@@ -163,7 +163,7 @@ class ClockSampler:
 # fp32-accurate contractions are issued as fp16 tensor-core MMAs on hi/lo
 # splits: 3 passes per product (2 when the A operand is exact in fp16)
 GEMM_PASSES = {"gemm_project": 3, "gemm_expand": 3, "gemm_energy": 3, "gemm_hessian": 3,
-               "gemm_cd_update": 2}
+               "gemm_cd_update": 2, "gemm_cd_panel": 2}
 
 
 def kernel_work(name, m, n, r, d, K, L):
@@ -182,6 +182,12 @@ def kernel_work(name, m, n, r, d, K, L):
         return "hbm", "GB/s", 8.0 * m * r
     if name in ("k_denoise_vec", "k_denoise_vec_tc"):  # one exponential per (block, codeword)
         return "sfu", "Gexp/s", float(m) * (n // 8) * K
+    if name == "k_vamp_row_scalar":      # read g, r2, w; write r2 and the fp16 hi/lo operand
+        return "hbm", "GB/s", 20.0 * m * n
+    if name == "k_vamp_row_scalar(map)":  # read g, r2, w; write the level index
+        return "hbm", "GB/s", 14.0 * m * n
+    if name == "k_cd_tile_decide":       # per 128-column tile: h, idx in; idx, Delta hi/lo out
+        return "hbm", "GB/s", 12.0 * m * 128
     return None
 
 
@@ -375,6 +381,28 @@ def run_mpq(args, world, rank, local):
     name, (cnt, kms) = dom
     roof = None
     wk = kernel_work(name, m, n, r, p.d, p.levels, p.levels)
+    # the whole step against its roofline: every kernel with a fixed
+    # algorithmic work at its own bound (the CD's decide kernels at their
+    # bytes; the gated CD update GEMMs, whose work depends on the changes,
+    # at zero), over the measured step time -- a lower bound on the fraction
+    ideal_ms = 0.0
+    for kname, (kc, _) in prof.items():
+        kw = kernel_work(kname, m, n, r, p.d, p.levels, p.levels)
+        if not kw:
+            continue
+        kb, _, kwork = kw
+        if kb == "tensor":
+            kpeak = peaks["bf16_tflops"] / GEMM_PASSES.get(kname, 1) * 1e12
+        elif kb == "hbm":
+            kpeak = peaks["hbm_gbs"] * 1e9
+        else:
+            kpeak = 148 * 16 * 1.965e9
+        ideal_ms += kwork * kc / kpeak * 1e3
+    ideal_ms /= args.steps
+    solve_roof = {"ideal_ms": ideal_ms, "measured_ms": ms_per_step, "frac": ideal_ms / ms_per_step,
+                  "basis": "sum over kernels of launches x algorithmic work / measured peak "
+                           "(tensor: bf16 burst / fp16 passes; hbm: copy GB/s; sfu: MUFU ex2 rate); "
+                           "CD update GEMMs counted at zero"}
     if wk:
         bound, unit, work = wk
         avg_s = kms / cnt / 1e3
@@ -443,7 +471,8 @@ def run_mpq(args, world, rank, local):
                 "data": "synthetic", "config": dict(cfgd, setup_s=None if setup_s is None else round(setup_s, 3), rank=r,
                                                     parallelism=f"rows sharded over {world} GPU(s)"),
                 "rows_per_s": world * m / (ms_per_step / 1e3),
-                "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk.summary(),
+                "roofline": roof, "solve_roofline": solve_roof, "cpu_baseline": cpu, "e2e": e2e,
+                "clocks": clk.summary(),
                 "gpu_launches": launches, "kernels": kernels}
         print(json.dumps(line), flush=True)
     plan.close()

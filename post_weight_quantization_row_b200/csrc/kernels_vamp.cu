@@ -619,7 +619,7 @@ __global__ void __launch_bounds__(ROW_THREADS)
 //   r < n: (1 - F) p'            -> G = V (D u) = xhat2 - r2
 //   r = n: -F p'                 -> G = xhat2 - w  (V V^T = I), which avoids
 //          forming r2 + V V^T (w - r2) when r2 is far from w.
-__global__ void __launch_bounds__(ROW_THREADS)
+__global__ void __launch_bounds__(1024)
     k_linear_rows(float* __restrict__ P, int64_t n, int64_t r, const float* __restrict__ s32,
                   const double* __restrict__ gamma2, const double* __restrict__ gamma1_0,
                   double* __restrict__ beta, double damping, double glo, double ghi,
@@ -628,10 +628,12 @@ __global__ void __launch_bounds__(ROW_THREADS)
                   double* __restrict__ alpha2_out, double* __restrict__ beta_hat_out,
                   int32_t* __restrict__ clamps, float* __restrict__ Uprime,
                   __half* __restrict__ ahi, __half* __restrict__ alo, int64_t lda, int64_t ldr,
-                  float* __restrict__ a_unscale) {
+                  float* __restrict__ a_unscale, int q_in_smem) {
   __shared__ double ds[33];
   __shared__ float fs[33];
+  extern __shared__ float s_q[];  // the row's GEMM2 operand when it fits
   const int64_t row = blockIdx.x;
+  float* qrow = q_in_smem ? s_q : P + row * r;
   const double b = beta[row], g2 = gamma2[row];
   double a2s = 0.0, bs = 0.0;
   float mx = 0.0f;
@@ -646,7 +648,7 @@ __global__ void __launch_bounds__(ROW_THREADS)
     bs += (double)(f * f * u * u) + (double)(sl * sl * inv);
     if (Uprime) Uprime[row * r + l] = (1.0f - f) * pl;
     const float q = full_rank ? -f * pl : (1.0f - f) * pl;
-    P[row * r + l] = q;
+    qrow[l] = q;
     mx = fmaxf(mx, fabsf(q));
   };
   for (int64_t l0 = threadIdx.x; l0 < r; l0 += ROW_UNROLL * blockDim.x) {
@@ -673,7 +675,7 @@ __global__ void __launch_bounds__(ROW_THREADS)
 #pragma unroll
     for (int u = 0; u < ROW_UNROLL; ++u) {
       const int64_t l = l0 + (int64_t)u * blockDim.x;
-      xv[u] = (l < r) ? P[row * r + l] * down : 0.0f;
+      xv[u] = (l < r) ? qrow[l] * down : 0.0f;
     }
 #pragma unroll
     for (int u = 0; u < ROW_UNROLL; ++u) {
@@ -1081,12 +1083,19 @@ mpq_status launch_linear_rows(const mpq_plan_s* p, int64_t m, const float* P,
   if (m <= 0) return MPQ_OK;
   const mpq_params& q = p->params;
   {
+    // the row's operand stays on chip between its two passes when it fits
+    const size_t qbytes = sizeof(float) * p->r;
+    const bool in_smem = qbytes <= 200 * 1024;
+    const int threads = qbytes <= 48 * 1024 ? ROW_THREADS : 1024;
+    if (in_smem)
+      MPQ_CUDA(cudaFuncSetAttribute(k_linear_rows, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)qbytes));
     ProfScope ps_("k_linear_rows", st);
-    k_linear_rows<<<rows_grid(m), ROW_THREADS, 0, st>>>(
+    k_linear_rows<<<rows_grid(m), in_smem ? threads : ROW_THREADS, in_smem ? qbytes : 0, st>>>(
         const_cast<float*>(P), p->n, p->r, p->s32, gamma2, gamma1_0, beta, q.damping,
         q.gamma_lo_rel, q.gamma_hi_rel, q.alpha_min, q.alpha_max, p->r == p->n ? 1 : 0,
         gamma1_out, coef, kappa, alpha2, beta_hat, clamps, Uprime, As->hi, As->lo, As->ld,
-        round_up(p->r, 64), As->row_unscale);
+        round_up(p->r, 64), As->row_unscale, in_smem ? 1 : 0);
   }
   count_launch();
   return check_launch("k_linear_rows");
