@@ -112,7 +112,7 @@ __global__ void __launch_bounds__(CD1_WARPS * 32, 2)
         float kn, e;
         {
           const float kcont = fmaf(hs[q], rq[q], kc[q]);
-          kn = fminf(fmaxf(ceilf(kcont - 0.5f), 0.0f), Lm1);
+          kn = fminf(fmaxf(ceil_small(kcont - 0.5f), 0.0f), Lm1);
           const float u = kn - kc[q];
           e = u * fmaf(a[q], u, -hs[q]);
         }

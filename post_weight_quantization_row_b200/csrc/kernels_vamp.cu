@@ -202,6 +202,7 @@ __global__ void __launch_bounds__(ROW_THREADS)
 // per-row constants (the stage kernel and the fused VAMP row kernel share them)
 struct ScalarDen {
   float sc, off, inv_sc, Lm1, sc2f, A2;
+  float hwf, kmax0;  // window half-width and last window start, as floats
   double doff, inv_dsc, g, ga, geff;
   int L, hw, nlev;
   bool anchored, precise;
@@ -233,9 +234,11 @@ __device__ __forceinline__ ScalarDen scalar_den_row(float sc, float off, double 
     const double w = ceil(0.5 * (-1.0 + sqrt(1.0 + 256.0 / (double)(-c.A2))));
     c.hw = (int)fmin(w, (double)L);
   }
-  // high precision (|A| > 5): the exact exponent form below, over the window
+  // high precision (|A| > 5): the exact exponent form below
   c.precise = -c.A2 > 5.0f;
   c.nlev = min(2 * c.hw + 1, L);
+  c.hwf = (float)c.hw;
+  c.kmax0 = (float)(L - c.nlev);
   c.inv_sc = (float)c.inv_dsc;
   c.Lm1 = (float)(L - 1);
   c.sc2f = (float)sc2;
@@ -243,17 +246,17 @@ __device__ __forceinline__ ScalarDen scalar_den_row(float sc, float off, double 
 }
 
 // One weight: cavity r (and w for the anchored prior) -> posterior mean xh,
-// variance (returned) and the most likely level kstar.  Instantiated per
-// precision regime and prior, both uniform over a row.
-template <bool PRECISE, bool ANCH, int LT>
+// variance (returned) and the most likely level ks (an integer as a float).
+// Instantiated per precision regime and prior, both uniform over a row.
+template <bool PRECISE, bool ANCH>
 __device__ __forceinline__ float scalar_den_elem(const ScalarDen& c, const float r, const float wr,
-                                                 float& xh, int& kstar) {
+                                                 float& xh, float& ks) {
   const float sc = c.sc, off = c.off, inv_sc = c.inv_sc, A2 = c.A2;
   // nearest level and the offset from it in level units, dt ~ dh + dl
   // (the pair matters only in the high-precision rows)
-  float ks, dh, dl;
+  float dh, dl;
   if constexpr (!ANCH) {
-    ks = fminf(fmaxf(ceilf((r - off) * inv_sc - 0.5f), 0.0f), c.Lm1);
+    ks = fminf(fmaxf(ceil_small((r - off) * inv_sc - 0.5f), 0.0f), c.Lm1);
     // r - (scale ks + offset) without rounding the level value: error-free
     // products and sums (Dekker / Knuth) give it as d0 + lo.  The explicitly
     // rounded intrinsics keep the compiler from contracting or
@@ -283,20 +286,20 @@ __device__ __forceinline__ float scalar_den_elem(const ScalarDen& c, const float
     dh = (float)dtd;
     dl = (float)(dtd - (double)dh);
   }
-  kstar = (int)ks;
+  // min(2hw+1, L) consecutive levels around k*, shifted to stay on the grid;
+  // dk = k - k* counts up from the window start as an exact float
+  float dk = fminf(fmaxf(ks - c.hwf, 0.0f), c.kmax0) - ks;
   float S0 = 0.0f, S1 = 0.0f, S2 = 0.0f;
   if constexpr (PRECISE) {
-    // q_k / q_k* = 2^(A dk (dk - 2 dt)) with dk = k - k* an exact integer and
-    // A = -geff/2 log2(e).  Here geff is large: dk - 2 dt is formed from the
+    // q_k / q_k* = 2^(A dk (dk - 2 dt)) with dk an exact integer and A =
+    // -geff/2 log2(e).  Here geff is large: dk - 2 dt is formed from the
     // pair (dh, dl) before scaling by A, so the exponent keeps fp32 accuracy
     // relative to itself (A dk^2 - 2 A dk dt would cancel, and a plain fp32
-    // dt would cost more than 1e-4 of a weight).  min(2hw+1, L) consecutive
-    // levels around k*, shifted to stay on the grid.
-    const int k0 = min(max(kstar - c.hw, 0), c.L - c.nlev);
+    // dt would cost more than 1e-4 of a weight).
+    const float m2dh = -2.0f * dh, m2dl = -2.0f * dl;  // exact
 #pragma unroll 4
-    for (int i = 0; i < c.nlev; ++i) {
-      const float dk = (float)(k0 + i) - ks;
-      const float e = fast_exp2((A2 * dk) * fmaf(-2.0f, dl, fmaf(-2.0f, dh, dk)));
+    for (int i = 0; i < c.nlev; ++i, dk += 1.0f) {
+      const float e = fast_exp2((A2 * dk) * ((dk + m2dh) + m2dl));
       S0 += e;
       const float ed = e * dk;
       S1 += ed;
@@ -304,39 +307,27 @@ __device__ __forceinline__ float scalar_den_elem(const ScalarDen& c, const float
     }
   } else {
     // q_k / q_k* = 2^(dk (A dk + B)), B = -2 A dt: with |A| <= 5 the
-    // rounding of B costs under 1e-5 of a weight.  All L levels in one fixed
-    // loop (no lane-dependent trip counts, so warps do not diverge), one
-    // hardware 2^x per level.
+    // rounding of B costs under 1e-5 of a weight
     const float B2 = -2.0f * A2 * dh;
-    if (LT > 0) {
-#pragma unroll
-      for (int k = 0; k < (LT > 0 ? LT : 1); ++k) {
-        const float dk = (float)k - ks;
-        const float e = fast_exp2(fmaf(A2, dk, B2) * dk);
-        S0 += e;
-        const float ed = e * dk;
-        S1 += ed;
-        S2 = fmaf(ed, dk, S2);
-      }
-    } else {
-      for (int k = 0; k < c.L; ++k) {
-        const float dk = (float)k - ks;
-        const float e = fast_exp2(fmaf(A2, dk, B2) * dk);
-        S0 += e;
-        const float ed = e * dk;
-        S1 += ed;
-        S2 = fmaf(ed, dk, S2);
-      }
+#pragma unroll 4
+    for (int i = 0; i < c.nlev; ++i, dk += 1.0f) {
+      const float e = fast_exp2(fmaf(A2, dk, B2) * dk);
+      S0 += e;
+      const float ed = e * dk;
+      S1 += ed;
+      S2 = fmaf(ed, dk, S2);
     }
   }
-  const float inv = __frcp_rn(S0);
+  // S0 >= 1 (k* itself has weight 1): the hardware reciprocal (~1 ulp) is
+  // far inside the stage tolerance
+  float inv;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(inv) : "f"(S0));
   const float m1 = S1 * inv;
   const float var = fmaxf(fmaf(S2, inv, -m1 * m1), 0.0f);
   xh = fmaf(sc, ks + m1, off);
   return c.sc2f * var;
 }
 
-template <int LT>
 __global__ void __launch_bounds__(ROW_THREADS)
     k_denoise_scalar(const float* __restrict__ R1, const double* __restrict__ gamma1,
                      const float* __restrict__ scale, const float* __restrict__ offset,
@@ -370,12 +361,11 @@ __global__ void __launch_bounds__(ROW_THREADS)
         const int64_t j = j0 + (int64_t)u * blockDim.x;
         if (j < n) {
           const int64_t o = row * n + j;
-          float xh;
-          int ks;
-          const float v = scalar_den_elem<PRECISE, ANCH, LT>(c, rv[u], wv[u], xh, ks);
+          float xh, ks;
+          const float v = scalar_den_elem<PRECISE, ANCH>(c, rv[u], wv[u], xh, ks);
           xhat[o] = xh;
           if (vblock) vblock[o] = v;
-          if (idx) idx[o] = (uint16_t)ks;
+          if (idx) idx[o] = (uint16_t)(int)ks;
           acc += v;
         }
       }
@@ -751,7 +741,7 @@ __global__ void __launch_bounds__(ROW_THREADS)
 // after the last iteration (l2d and the denoiser's argmax only).
 constexpr int FUSED_MAX_THREADS = 1024;
 
-template <int LT, int MAP>
+template <int MAP>
 __global__ void __launch_bounds__(FUSED_MAX_THREADS)
     k_vamp_row_scalar(const float* __restrict__ W, const float* __restrict__ G,
                       float* __restrict__ R2, int64_t n, int first, int full_rank,
@@ -796,11 +786,10 @@ __global__ void __launch_bounds__(FUSED_MAX_THREADS)
         const float r1 = first ? w
                          : full_rank ? fmaf(lc, gv[u], fmaf(lk, w - r2v[u], w))
                                      : fmaf(lc, gv[u], r2v[u]);
-        float xh;
-        int ks;
-        const float v = scalar_den_elem<PRECISE, ANCH, LT>(c, r1, w, xh, ks);
+        float xh, ks;
+        const float v = scalar_den_elem<PRECISE, ANCH>(c, r1, w, xh, ks);
         if (MAP) {
-          idx[row * n + j] = (uint16_t)ks;
+          idx[row * n + j] = (uint16_t)(int)ks;
         } else {
           s_r[j] = r1;
           s_x[j] = xh;
@@ -1010,10 +999,7 @@ mpq_status launch_denoise(const mpq_plan_s* p, const float* R1, const double* ga
   if (p->d == 1) {
     {
       ProfScope ps_("k_denoise_scalar", st);
-      auto* kern = (p->K == 16) ? k_denoise_scalar<16>
-                   : (p->K == 8) ? k_denoise_scalar<8>
-                   : (p->K == 4) ? k_denoise_scalar<4> : k_denoise_scalar<0>;
-      kern<<<rows_grid(m), ROW_THREADS, 0, st>>>(R1, gamma1, scale, offset, p->n, p->K,
+      k_denoise_scalar<<<rows_grid(m), ROW_THREADS, 0, st>>>(R1, gamma1, scale, offset, p->n, p->K,
                                                  anchored ? W : nullptr, gamma1_0, inv_tau2,
                                                  xhat1, vblock, vsum, idx);
     }
@@ -1140,15 +1126,7 @@ mpq_status launch_vamp_row_scalar(const mpq_plan_s* p, const float* W, int64_t m
                         const double*, const double*, const float*, const float*, int, int,
                         const double*, double, double, double, double, double, __half*, __half*,
                         int64_t, int64_t, float*, double*, int32_t*, uint16_t*);
-  Kern kern;
-  if (map)
-    kern = (p->K == 16) ? k_vamp_row_scalar<16, 1>
-           : (p->K == 8) ? k_vamp_row_scalar<8, 1>
-           : (p->K == 4) ? k_vamp_row_scalar<4, 1> : k_vamp_row_scalar<0, 1>;
-  else
-    kern = (p->K == 16) ? k_vamp_row_scalar<16, 0>
-           : (p->K == 8) ? k_vamp_row_scalar<8, 0>
-           : (p->K == 4) ? k_vamp_row_scalar<4, 0> : k_vamp_row_scalar<0, 0>;
+  const Kern kern = map ? k_vamp_row_scalar<1> : k_vamp_row_scalar<0>;
   MPQ_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   {
     ProfScope ps_(map ? "k_vamp_row_scalar(map)" : "k_vamp_row_scalar", st);

@@ -186,6 +186,14 @@ mpq_status launch_energy_rows(const mpq_plan_s* p, int64_t m, const float* P, fl
 mpq_status launch_cd(mpq_plan_s* p, const float* W, int64_t m, const float* scale,
                      const float* offset, uint16_t* idx, float* h, int64_t ldh, int32_t sweeps,
                      int32_t* changes, cudaStream_t st);
+// ceil(y) for |y| < 2^22 with one directed-rounding add: y + 1.5 2^23 rounded
+// up lands on the integer grid of [2^23, 2^24) (full-rate adds instead of a
+// rounding instruction).  Larger |y| keeps its sign, which is all the callers
+// need: they clamp the result to a grid of at most 65536 levels.
+__device__ __forceinline__ float ceil_small(float y) {
+  return __fsub_rn(__fadd_ru(y, 12582912.0f), 12582912.0f);
+}
+
 constexpr int CD_TILE = 128;  // columns per scalar CD tile (multiple of 64)
 constexpr int64_t CD_PANEL_BYTES = 32ll << 20;  // L2-resident slab of the CD gradient
 constexpr int64_t CD_PANEL_MIN = 512;           // narrowest CD panel (columns)
