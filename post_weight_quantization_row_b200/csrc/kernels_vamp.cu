@@ -619,65 +619,95 @@ __global__ void __launch_bounds__(1024)
                   int32_t* __restrict__ clamps, float* __restrict__ Uprime,
                   __half* __restrict__ ahi, __half* __restrict__ alo, int64_t lda, int64_t ldr,
                   float* __restrict__ a_unscale, int q_in_smem) {
-  __shared__ double ds[33];
-  __shared__ float fs[33];
+  __shared__ double ds_a[32], ds_b[32];
+  __shared__ float fs_m[32];
+  __shared__ double tot_a, tot_b;
+  __shared__ float tot_m;
   extern __shared__ float s_q[];  // the row's GEMM2 operand when it fits
   const int64_t row = blockIdx.x;
+  const int rr = (int)r;
+  const int bs = blockDim.x;
   float* qrow = q_in_smem ? s_q : P + row * r;
+  const float* Pr = P + row * r;
   const double b = beta[row], g2 = gamma2[row];
-  double a2s = 0.0, bs = 0.0;
-  float mx = 0.0f;
+  // per element in fp32 (relative error ~1e-7); per-thread partial sums in
+  // fp32 (a few dozen terms), the block sum in fp64
+  float a2s = 0.0f, bsum = 0.0f, mx = 0.0f;
   const float bf = (float)b, g2f = (float)g2;
-  auto element = [&](const int64_t l, const float sl, const float pl) {
-    // per element in fp32 (relative error ~1e-7), sums in fp64
+  auto element = [&](const int l, const float sl, const float pl) {
     const float u = sl * pl;
-    const float den = fmaf(bf * sl, sl, g2f);
-    const float inv = 1.0f / den;
+    const float den = fmaf(bf * sl, sl, g2f);  // > 0
+    const float inv = __fdividef(1.0f, den);
     const float f = g2f * inv;
-    a2s += (double)f;
-    bs += (double)(f * f * u * u) + (double)(sl * sl * inv);
+    a2s += f;
+    bsum += fmaf(f * f * u, u, sl * sl * inv);
     if (Uprime) Uprime[row * r + l] = (1.0f - f) * pl;
     const float q = full_rank ? -f * pl : (1.0f - f) * pl;
     qrow[l] = q;
     mx = fmaxf(mx, fabsf(q));
   };
-  for (int64_t l0 = threadIdx.x; l0 < r; l0 += ROW_UNROLL * blockDim.x) {
+  // whole batches of ROW_UNROLL elements per thread without bounds checks,
+  // then the tail one element at a time
+  const int full = rr / (ROW_UNROLL * bs) * (ROW_UNROLL * bs);
+  for (int l0 = threadIdx.x; l0 < full; l0 += ROW_UNROLL * bs) {
     float sv[ROW_UNROLL], pv[ROW_UNROLL];
 #pragma unroll
     for (int u = 0; u < ROW_UNROLL; ++u) {
-      const int64_t l = l0 + (int64_t)u * blockDim.x;
-      sv[u] = l < r ? s32[l] : 0.0f;
-      pv[u] = l < r ? P[row * r + l] : 0.0f;
+      sv[u] = s32[l0 + u * bs];
+      pv[u] = Pr[l0 + u * bs];
     }
 #pragma unroll
-    for (int u = 0; u < ROW_UNROLL; ++u) {
-      const int64_t l = l0 + (int64_t)u * blockDim.x;
-      if (l < r) element(l, sv[u], pv[u]);
-    }
+    for (int u = 0; u < ROW_UNROLL; ++u) element(l0 + u * bs, sv[u], pv[u]);
   }
-  a2s = block_sum(a2s, ds);
-  bs = block_sum(bs, ds);
-  mx = block_reduce(mx, MaxF(), fs);
-  const int ex = split_exponent(mx);
+  for (int l = full + threadIdx.x; l < rr; l += bs) element(l, s32[l], Pr[l]);
+  // the three row reductions in one pass: warps, then warp 0
+  {
+    double da = a2s, db = bsum;
+    float m = mx;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      da += __shfl_xor_sync(0xffffffffu, da, o);
+      db += __shfl_xor_sync(0xffffffffu, db, o);
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    }
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = (bs + 31) >> 5;
+    if (lane == 0) {
+      ds_a[wid] = da;
+      ds_b[wid] = db;
+      fs_m[wid] = m;
+    }
+    __syncthreads();
+    if (wid == 0) {
+      da = lane < nw ? ds_a[lane] : 0.0;
+      db = lane < nw ? ds_b[lane] : 0.0;
+      m = lane < nw ? fs_m[lane] : 0.0f;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        da += __shfl_xor_sync(0xffffffffu, da, o);
+        db += __shfl_xor_sync(0xffffffffu, db, o);
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      }
+      if (lane == 0) {
+        tot_a = da;
+        tot_b = db;
+        tot_m = m;
+      }
+    }
+    __syncthreads();
+  }
+  const double a2tot = tot_a, bstot = tot_b;
+  const int ex = split_exponent(tot_m);
   const float down = ldexpf(1.0f, -ex);
-  for (int64_t l0 = threadIdx.x; l0 < ldr; l0 += ROW_UNROLL * blockDim.x) {
-    float xv[ROW_UNROLL];
-#pragma unroll
-    for (int u = 0; u < ROW_UNROLL; ++u) {
-      const int64_t l = l0 + (int64_t)u * blockDim.x;
-      xv[u] = (l < r) ? qrow[l] * down : 0.0f;
-    }
-#pragma unroll
-    for (int u = 0; u < ROW_UNROLL; ++u) {
-      const int64_t l = l0 + (int64_t)u * blockDim.x;
-      if (l < ldr) split_store(xv[u], ahi, alo, row * lda + l);
-    }
-  }
+  __half* ahr = ahi + row * lda;
+  __half* alr = alo + row * lda;
+  const int ldrr = (int)ldr;
+  for (int l = threadIdx.x; l < ldrr; l += bs)
+    split_store(l < rr ? qrow[l] * down : 0.0f, ahr, alr, l);
   if (threadIdx.x == 0) {
     a_unscale[row] = ldexpf(1.0f, ex);
     int cnt = 0;
-    const double alpha2 = (a2s + (double)(n - r)) / (double)n;
-    const double bhat = (double)r / bs;
+    const double alpha2 = (a2tot + (double)(n - r)) / (double)n;
+    const double bhat = (double)r / bstot;
     beta[row] = (1.0 - damping) * b + damping * bhat;
     const double a2 = clip_count(alpha2, amin, amax, &cnt);
     const double g0 = gamma1_0[row];
@@ -757,46 +787,51 @@ __global__ void __launch_bounds__(FUSED_MAX_THREADS)
   __shared__ double ds[33];
   __shared__ float fs[33];
   __shared__ float cf_s;
+  const int nn = (int)n;  // a row fits in shared memory: 32-bit in-row indices
   float* s_r = vrow;
-  float* s_x = vrow + n;
+  float* s_x = vrow + nn;
   const int64_t row = blockIdx.x;
+  const float* Wr = W + row * n;
+  const float* Gr = G + row * n;
+  float* R2r = R2 + row * n;
   const ScalarDen c = scalar_den_row(scale[row], offset[row], gamma1[row], L, anchored != 0,
                                      anchored ? gamma1_0[row] : 0.0, inv_tau2);
   const float lc = first ? 0.0f : (float)coef[row];
   const float lk = first ? 0.0f : (float)kappa[row];
+  const int bs = blockDim.x;
+  // whole batches of ROW_UNROLL weights per thread (loads first, no bounds
+  // checks), then the tail one weight at a time
+  const int full = nn / (ROW_UNROLL * bs) * (ROW_UNROLL * bs);
   auto pass1 = [&](auto prec, auto anch) -> float {
     constexpr bool PRECISE = decltype(prec)::value;
     constexpr bool ANCH = decltype(anch)::value;
     float acc = 0.0f;
-    for (int64_t j0 = threadIdx.x; j0 < n; j0 += ROW_UNROLL * blockDim.x) {
+    auto one = [&](const int j, const float g, const float r2, const float w) {
+      const float r1 = first ? w : full_rank ? fmaf(lc, g, fmaf(lk, w - r2, w)) : fmaf(lc, g, r2);
+      float xh, ks;
+      const float v = scalar_den_elem<PRECISE, ANCH>(c, r1, w, xh, ks);
+      if (MAP) {
+        idx[row * n + j] = (uint16_t)(int)ks;
+      } else {
+        s_r[j] = r1;
+        s_x[j] = xh;
+        acc += v;
+      }
+    };
+    for (int j0 = threadIdx.x; j0 < full; j0 += ROW_UNROLL * bs) {
       float gv[ROW_UNROLL], r2v[ROW_UNROLL], wv[ROW_UNROLL];
 #pragma unroll
       for (int u = 0; u < ROW_UNROLL; ++u) {
-        const int64_t j = j0 + (int64_t)u * blockDim.x;
-        const bool in = j < n;
-        gv[u] = (in && !first) ? G[row * n + j] : 0.0f;
-        r2v[u] = (in && !first) ? R2[row * n + j] : 0.0f;
-        wv[u] = in ? W[row * n + j] : 0.0f;
+        const int j = j0 + u * bs;
+        gv[u] = first ? 0.0f : Gr[j];
+        r2v[u] = first ? 0.0f : R2r[j];
+        wv[u] = Wr[j];
       }
 #pragma unroll
-      for (int u = 0; u < ROW_UNROLL; ++u) {
-        const int64_t j = j0 + (int64_t)u * blockDim.x;
-        if (j >= n) continue;
-        const float w = wv[u];
-        const float r1 = first ? w
-                         : full_rank ? fmaf(lc, gv[u], fmaf(lk, w - r2v[u], w))
-                                     : fmaf(lc, gv[u], r2v[u]);
-        float xh, ks;
-        const float v = scalar_den_elem<PRECISE, ANCH>(c, r1, w, xh, ks);
-        if (MAP) {
-          idx[row * n + j] = (uint16_t)(int)ks;
-        } else {
-          s_r[j] = r1;
-          s_x[j] = xh;
-          acc += v;
-        }
-      }
+      for (int u = 0; u < ROW_UNROLL; ++u) one(j0 + u * bs, gv[u], r2v[u], wv[u]);
     }
+    for (int j = full + threadIdx.x; j < nn; j += bs)
+      one(j, first ? 0.0f : Gr[j], first ? 0.0f : R2r[j], Wr[j]);
     return acc;
   };
   using T_ = std::true_type;
@@ -811,40 +846,36 @@ __global__ void __launch_bounds__(FUSED_MAX_THREADS)
   __syncthreads();
   const float cf = cf_s;
   float mx = 0.0f;
-  for (int64_t j0 = threadIdx.x; j0 < n; j0 += ROW_UNROLL * blockDim.x) {
+  auto two = [&](const int j, const float w) {
+    const float r1 = s_r[j];
+    const float r2 = fmaf(cf, s_x[j] - r1, r1);
+    R2r[j] = r2;
+    s_r[j] = r2;
+    mx = fmaxf(mx, fabsf(w - r2));
+  };
+  for (int j0 = threadIdx.x; j0 < full; j0 += ROW_UNROLL * bs) {
     float wv[ROW_UNROLL];
 #pragma unroll
-    for (int u = 0; u < ROW_UNROLL; ++u) {
-      const int64_t j = j0 + (int64_t)u * blockDim.x;
-      wv[u] = j < n ? W[row * n + j] : 0.0f;
-    }
+    for (int u = 0; u < ROW_UNROLL; ++u) wv[u] = Wr[j0 + u * bs];
 #pragma unroll
-    for (int u = 0; u < ROW_UNROLL; ++u) {
-      const int64_t j = j0 + (int64_t)u * blockDim.x;
-      if (j >= n) continue;
-      const float r1 = s_r[j];
-      const float r2 = fmaf(cf, s_x[j] - r1, r1);
-      R2[row * n + j] = r2;
-      s_r[j] = r2;
-      mx = fmaxf(mx, fabsf(wv[u] - r2));
-    }
+    for (int u = 0; u < ROW_UNROLL; ++u) two(j0 + u * bs, wv[u]);
   }
+  for (int j = full + threadIdx.x; j < nn; j += bs) two(j, Wr[j]);
   mx = block_reduce(mx, MaxF(), fs);  // its barriers also publish the new s_r
   const int ex = split_exponent(mx);
   const float down = ldexpf(1.0f, -ex);
-  for (int64_t j0 = threadIdx.x; j0 < ldn; j0 += ROW_UNROLL * blockDim.x) {
+  __half* ahr = ahi + row * lda;
+  __half* alr = alo + row * lda;
+  const int ldnn = (int)ldn;
+  for (int j0 = threadIdx.x; j0 < full; j0 += ROW_UNROLL * bs) {
     float xv[ROW_UNROLL];
 #pragma unroll
-    for (int u = 0; u < ROW_UNROLL; ++u) {
-      const int64_t j = j0 + (int64_t)u * blockDim.x;
-      xv[u] = (j < n) ? (W[row * n + j] - s_r[j]) * down : 0.0f;
-    }
+    for (int u = 0; u < ROW_UNROLL; ++u) xv[u] = (Wr[j0 + u * bs] - s_r[j0 + u * bs]) * down;
 #pragma unroll
-    for (int u = 0; u < ROW_UNROLL; ++u) {
-      const int64_t j = j0 + (int64_t)u * blockDim.x;
-      if (j < ldn) split_store(xv[u], ahi, alo, row * lda + j);
-    }
+    for (int u = 0; u < ROW_UNROLL; ++u) split_store(xv[u], ahr, alr, j0 + u * bs);
   }
+  for (int j = full + threadIdx.x; j < ldnn; j += bs)
+    split_store(j < nn ? (Wr[j] - s_r[j]) * down : 0.0f, ahr, alr, j);
   if (threadIdx.x == 0) a_unscale[row] = ldexpf(1.0f, ex);
 }
 
