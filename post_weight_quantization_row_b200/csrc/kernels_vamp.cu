@@ -88,6 +88,32 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// Packed fp32 pairs (sm_100 f32x2 arithmetic: two lanes' worth of fp32
+// work per instruction, each half rounded as the scalar operation would be).
+__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
 // Split of a row for the tensor-core GEMM: a per-row power of two e with
 // max|x| * 2^-e < 2^14, then hi = fp16(x 2^-e), lo = fp16(x 2^-e - hi).
 __device__ __forceinline__ int split_exponent(float amax) {
@@ -289,7 +315,14 @@ __device__ __forceinline__ float scalar_den_elem(const ScalarDen& c, const float
   // min(2hw+1, L) consecutive levels around k*, shifted to stay on the grid;
   // dk = k - k* counts up from the window start as an exact float
   float dk = fminf(fmaxf(ks - c.hwf, 0.0f), c.kmax0) - ks;
-  float S0 = 0.0f, S1 = 0.0f, S2 = 0.0f;
+  // Two levels per packed f32x2 instruction (dk, dk + 1); each level's
+  // arithmetic is the scalar form's, the sums run over even and odd levels
+  // separately.  An odd window ends with one scalar level.
+  uint64_t dkp = f2_pack(dk, dk + 1.0f);
+  uint64_t S0p = 0, S1p = 0, S2p = 0;  // (+0, +0)
+  const uint64_t two = f2_pack(2.0f, 2.0f);
+  const int npair = c.nlev >> 1;
+  float e_t = 0.0f, dk_t = dk + (float)(2 * npair);  // the odd level, if any
   if constexpr (PRECISE) {
     // q_k / q_k* = 2^(A dk (dk - 2 dt)) with dk an exact integer and A =
     // -geff/2 log2(e).  Here geff is large: dk - 2 dt is formed from the
@@ -297,27 +330,45 @@ __device__ __forceinline__ float scalar_den_elem(const ScalarDen& c, const float
     // relative to itself (A dk^2 - 2 A dk dt would cancel, and a plain fp32
     // dt would cost more than 1e-4 of a weight).
     const float m2dh = -2.0f * dh, m2dl = -2.0f * dl;  // exact
-#pragma unroll 4
-    for (int i = 0; i < c.nlev; ++i, dk += 1.0f) {
-      const float e = fast_exp2((A2 * dk) * ((dk + m2dh) + m2dl));
-      S0 += e;
-      const float ed = e * dk;
-      S1 += ed;
-      S2 = fmaf(ed, dk, S2);
+    const uint64_t mh = f2_pack(m2dh, m2dh), ml = f2_pack(m2dl, m2dl), a2 = f2_pack(A2, A2);
+#pragma unroll 2
+    for (int i = 0; i < npair; ++i, dkp = f2_add(dkp, two)) {
+      const uint64_t z = f2_mul(f2_mul(a2, dkp), f2_add(f2_add(dkp, mh), ml));
+      float z0, z1;
+      f2_unpack(z, z0, z1);
+      const uint64_t e = f2_pack(fast_exp2(z0), fast_exp2(z1));
+      S0p = f2_add(S0p, e);
+      const uint64_t ed = f2_mul(e, dkp);
+      S1p = f2_add(S1p, ed);
+      S2p = f2_fma(ed, dkp, S2p);
     }
+    if (c.nlev & 1) e_t = fast_exp2((A2 * dk_t) * ((dk_t + m2dh) + m2dl));
   } else {
     // q_k / q_k* = 2^(dk (A dk + B)), B = -2 A dt: with |A| <= 5 the
     // rounding of B costs under 1e-5 of a weight
     const float B2 = -2.0f * A2 * dh;
-#pragma unroll 4
-    for (int i = 0; i < c.nlev; ++i, dk += 1.0f) {
-      const float e = fast_exp2(fmaf(A2, dk, B2) * dk);
-      S0 += e;
-      const float ed = e * dk;
-      S1 += ed;
-      S2 = fmaf(ed, dk, S2);
+    const uint64_t a2 = f2_pack(A2, A2), b2 = f2_pack(B2, B2);
+#pragma unroll 2
+    for (int i = 0; i < npair; ++i, dkp = f2_add(dkp, two)) {
+      const uint64_t z = f2_mul(f2_fma(a2, dkp, b2), dkp);
+      float z0, z1;
+      f2_unpack(z, z0, z1);
+      const uint64_t e = f2_pack(fast_exp2(z0), fast_exp2(z1));
+      S0p = f2_add(S0p, e);
+      const uint64_t ed = f2_mul(e, dkp);
+      S1p = f2_add(S1p, ed);
+      S2p = f2_fma(ed, dkp, S2p);
     }
+    if (c.nlev & 1) e_t = fast_exp2(fmaf(A2, dk_t, B2) * dk_t);
   }
+  float s0a, s0b, s1a, s1b, s2a, s2b;
+  f2_unpack(S0p, s0a, s0b);
+  f2_unpack(S1p, s1a, s1b);
+  f2_unpack(S2p, s2a, s2b);
+  const float ed_t = e_t * dk_t;
+  const float S0 = (s0a + s0b) + e_t;
+  const float S1 = (s1a + s1b) + ed_t;
+  const float S2 = fmaf(ed_t, dk_t, s2a + s2b);
   // S0 >= 1 (k* itself has weight 1): the hardware reciprocal (~1 ulp) is
   // far inside the stage tolerance
   float inv;
