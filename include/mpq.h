@@ -102,6 +102,15 @@ typedef struct {
                              bytes) fits in 32 MiB, at least 512; else the
                              panel width in columns, a positive multiple of
                              128 (a panel as wide as n is one panel). */
+  int32_t solve_graphs;   /* 1 (default): when mpq_solve or mpq_solve_host is
+                             called a second time with the same buffers, sizes
+                             and options (the buffers' contents may change), it
+                             captures its kernel launches into a CUDA graph, and
+                             later such calls replay it, which removes most
+                             inter-launch gaps; 4 calls are remembered per plan.
+                             0: every call launches its kernels directly.  Calls
+                             made while the per-kernel profiler runs always
+                             launch directly. */
 } mpq_params;
 
 /* Fill `p` with the defaults above for block size d and codebook size K. */

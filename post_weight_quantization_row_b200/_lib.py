@@ -42,7 +42,8 @@ class Params(C.Structure):
                 ("beta0", C.c_double), ("damping", C.c_double), ("tau", C.c_double),
                 ("gamma_lo_rel", C.c_double), ("gamma_hi_rel", C.c_double),
                 ("alpha_min", C.c_double), ("alpha_max", C.c_double),
-                ("vec_engine", C.c_int32), ("cd_panel", C.c_int32)]
+                ("vec_engine", C.c_int32), ("cd_panel", C.c_int32),
+                ("solve_graphs", C.c_int32)]
 
 
 class RowStats(C.Structure):

@@ -34,11 +34,39 @@ constexpr int CD1_WARPS = 16;
 constexpr int CD1_SLOTS = CD_TILE / 32;
 constexpr int CD1_SMEM = (CD_TILE * CD_TILE + CD_TILE) * 4;
 
-// 4-byte asynchronous copy global -> shared; src_bytes = 0 fills zero
+// 4- and 16-byte asynchronous copies global -> shared; bytes past src_bytes
+// are filled with zeros
 __device__ __forceinline__ void cp_async4(float* dst, const float* src, int src_bytes) {
   const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(d), "l"(src), "r"(src_bytes)
                : "memory");
+}
+__device__ __forceinline__ void cp_async16(float* dst, const float* src, int src_bytes) {
+  const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(d), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+
+// H[t0.., t0..] (tw x tw) into a zero-padded CD_TILE x CD_TILE shared tile:
+// 16-byte copies when the rows of H are 16-byte aligned (n % 4 == 0; t0 is a
+// multiple of 128), else 4-byte copies
+__device__ __forceinline__ void load_h_tile(float* sH, const float* H, int64_t n, int64_t t0,
+                                            int tw) {
+  if ((n & 3) == 0) {
+    constexpr int CH = CD_TILE / 4;  // 16-byte chunks per row
+    for (int e = threadIdx.x; e < CD_TILE * CH; e += blockDim.x) {
+      const int i = e / CH, j = 4 * (e % CH);
+      const int bytes = i < tw ? 4 * max(0, min(4, tw - j)) : 0;
+      cp_async16(sH + i * CD_TILE + j, bytes ? H + (t0 + i) * n + t0 + j : H, bytes);
+    }
+  } else {
+    for (int e = threadIdx.x; e < CD_TILE * CD_TILE; e += blockDim.x) {
+      const int i = e / CD_TILE, j = e % CD_TILE;
+      const bool in = i < tw && j < tw;
+      cp_async4(sH + e, in ? H + (t0 + i) * n + t0 + j : H, in ? 4 : 0);
+    }
+  }
+  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;\n" ::: "memory");
 }
 
 __global__ void __launch_bounds__(CD1_WARPS * 32, 2)
@@ -52,12 +80,7 @@ __global__ void __launch_bounds__(CD1_WARPS * 32, 2)
   extern __shared__ float cd_smem[];
   float* sH = cd_smem;                   // H[tile, tile], zero outside tw x tw
   float* s_rg = sH + CD_TILE * CD_TILE;  // 1 / H_jj (0 where H_jj <= 0)
-  for (int e = threadIdx.x; e < CD_TILE * CD_TILE; e += blockDim.x) {
-    const int i = e / CD_TILE, j = e % CD_TILE;
-    const bool in = i < tw && j < tw;
-    cp_async4(sH + e, in ? H + (t0 + i) * n + t0 + j : H, in ? 4 : 0);
-  }
-  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;\n" ::: "memory");
+  load_h_tile(sH, H, n, t0, tw);
   __syncthreads();
   bool pos = true;  // every diagonal entry of the tile positive
   for (int j = threadIdx.x; j < CD_TILE; j += blockDim.x) {

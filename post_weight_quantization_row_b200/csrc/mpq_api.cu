@@ -66,6 +66,11 @@ cudaEvent_t pool_event() {
 }
 }  // namespace
 
+bool profiling_on() {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  return g_prof_on;
+}
+
 ProfScope::ProfScope(const char* name, cudaStream_t stream) : st(stream) {
   std::lock_guard<std::mutex> lk(g_prof_mu);
   if (!g_prof_on) return;
@@ -126,6 +131,8 @@ mpq_status validate_params(const mpq_params* q, int64_t n) {
   if (q->vec_engine < 0 || q->vec_engine > 2) return fail(MPQ_ERR_INVALID_ARG, "vec_engine must be 0, 1 or 2");
   if (q->cd_panel < 0 || q->cd_panel % 128)
     return fail(MPQ_ERR_INVALID_ARG, "cd_panel must be 0 or a positive multiple of 128");
+  if (q->solve_graphs != 0 && q->solve_graphs != 1)
+    return fail(MPQ_ERR_INVALID_ARG, "solve_graphs must be 0 or 1");
   if (!(q->beta0 > 0.0) || !isfinite(q->beta0)) return fail(MPQ_ERR_INVALID_ARG, "beta0 must be > 0");
   if (!(q->damping >= 0.0 && q->damping <= 1.0)) return fail(MPQ_ERR_INVALID_ARG, "damping must be in [0,1]");
   if (!(q->tau > 0.0)) return fail(MPQ_ERR_INVALID_ARG, "tau must be > 0 (INFINITY = uniform prior)");
@@ -200,12 +207,16 @@ int64_t ws_bytes_per_row(const mpq_plan_s* p) {
 }
 
 // changes buffer rides in the tail of `clamps`: rows x (1 + MAX_SWEEPS) ints
+void drop_graphs(mpq_plan_s* p);
+
 mpq_status ensure_workspace(mpq_plan_s* p, int64_t rows) {
   if (rows <= p->ws.rows) return MPQ_OK;
   const int64_t need = rows * ws_bytes_per_row(p);
   if (p->ws_cap > 0 && need > p->ws_cap)
     return fail(MPQ_ERR_OOM, "workspace of " + std::to_string(need) + " bytes exceeds the cap");
   MPQ_CUDA(cudaDeviceSynchronize());
+  drop_graphs(p);  // they hold the old workspace's addresses
+  ++p->ws_gen;
   free_workspace(p->ws);
   Workspace& w = p->ws;
   const int64_t mn = rows * p->n;
@@ -402,9 +413,79 @@ mpq_status solve_device(mpq_plan_s* p, const SolveIO& io, cudaStream_t st) {
     rows = std::min(rows, fit);
   }
   MPQ_TRY(ensure_workspace(p, rows));
-  for (int64_t r0 = 0; r0 < io.m; r0 += rows) {
-    MPQ_TRY(solve_batch(p, io, r0, std::min(rows, io.m - r0), st));
+  auto run = [&](cudaStream_t s) -> mpq_status {
+    for (int64_t r0 = 0; r0 < io.m; r0 += rows)
+      MPQ_TRY(solve_batch(p, io, r0, std::min(rows, io.m - r0), s));
+    return MPQ_OK;
+  };
+  if (!p->params.solve_graphs || profiling_on()) return run(st);
+  // the call's identity: buffers, sizes, options and the workspace generation
+  uint64_t key[mpq_plan_s::GRAPH_KEY] = {
+      (uint64_t)(uintptr_t)io.W, (uint64_t)io.m, (uint64_t)(uintptr_t)io.row_scale,
+      (uint64_t)(uintptr_t)io.row_offset, (uint64_t)io.T_vamp, (uint64_t)io.sweeps,
+      (uint64_t)(uintptr_t)io.idx, (uint64_t)(uintptr_t)io.w_hat,
+      (uint64_t)(uintptr_t)io.energy, 0, 0, 0, 0, (uint64_t)rows, p->ws_gen, 1};
+  if (io.stats) {
+    key[9] = (uint64_t)(uintptr_t)io.stats->gamma1;
+    key[10] = (uint64_t)(uintptr_t)io.stats->beta;
+    key[11] = (uint64_t)(uintptr_t)io.stats->clamps;
+    key[12] = (uint64_t)(uintptr_t)io.stats->cd_changes;
   }
+  mpq_plan_s::SolveGraph* seen = nullptr;
+  for (auto& gr : p->graphs) {
+    if (gr.last_use && std::equal(key, key + mpq_plan_s::GRAPH_KEY, gr.key)) {
+      gr.last_use = ++p->graph_clock;
+      if (!gr.exec) {
+        seen = &gr;
+        break;
+      }
+      MPQ_CUDA(cudaGraphLaunch(gr.exec, st));
+      count_launch((int)gr.launches);
+      return MPQ_OK;
+    }
+  }
+  auto lru = [&]() {
+    mpq_plan_s::SolveGraph* s = &p->graphs[0];
+    for (auto& gr : p->graphs)
+      if (gr.last_use < s->last_use) s = &gr;
+    return s;
+  };
+  if (!seen) {
+    // a call seen for the first time runs directly; the second one captures
+    mpq_plan_s::SolveGraph* s = lru();
+    if (s->exec) cudaGraphExecDestroy(s->exec);
+    *s = mpq_plan_s::SolveGraph{};
+    std::copy(key, key + mpq_plan_s::GRAPH_KEY, s->key);
+    s->last_use = ++p->graph_clock;
+    return run(st);
+  }
+  // capture the launches on a private stream (the caller's may be the legacy
+  // default stream, which cannot be captured); anything that fails to
+  // capture runs directly instead
+  if (!p->capture_stream)
+    MPQ_CUDA(cudaStreamCreateWithFlags(&p->capture_stream, cudaStreamNonBlocking));
+  if (cudaStreamBeginCapture(p->capture_stream, cudaStreamCaptureModeThreadLocal) != cudaSuccess) {
+    cudaGetLastError();
+    return run(st);
+  }
+  const int64_t l0 = mpq_kernel_launch_count();
+  const mpq_status rc = run(p->capture_stream);
+  cudaGraph_t graph = nullptr;
+  const cudaError_t ce = cudaStreamEndCapture(p->capture_stream, &graph);
+  const int64_t nl = mpq_kernel_launch_count() - l0;
+  count_launch((int)-nl);  // nothing ran yet
+  cudaGraphExec_t exec = nullptr;
+  const bool ok = rc == MPQ_OK && ce == cudaSuccess && graph &&
+                  cudaGraphInstantiate(&exec, graph, 0) == cudaSuccess;
+  if (graph) cudaGraphDestroy(graph);
+  if (!ok) {
+    cudaGetLastError();
+    return run(st);
+  }
+  seen->exec = exec;
+  seen->launches = nl;
+  MPQ_CUDA(cudaGraphLaunch(exec, st));
+  count_launch((int)nl);
   return MPQ_OK;
 }
 
@@ -442,9 +523,18 @@ mpq_status finish_plan(mpq_plan_s* p, cudaStream_t st) {
   return MPQ_OK;
 }
 
+void drop_graphs(mpq_plan_s* p) {
+  for (auto& gr : p->graphs) {
+    if (gr.exec) cudaGraphExecDestroy(gr.exec);
+    gr = mpq_plan_s::SolveGraph{};
+  }
+}
+
 void destroy_plan(mpq_plan_s* p) {
   if (!p) return;
   DeviceGuard g(p->device);
+  drop_graphs(p);
+  if (p->capture_stream) cudaStreamDestroy(p->capture_stream);
   free_workspace(p->ws);
   dfree(p->s64); dfree(p->V64); dfree(p->s32); dfree(p->V32); dfree(p->Vt32); dfree(p->H32);
   dfree(p->Hdiag); dfree(p->cb); dfree(p->cb_norm); dfree(p->qtab); dfree(p->status);
@@ -514,6 +604,7 @@ void mpq_params_default(mpq_params* p, int32_t d, int32_t K) {
   p->alpha_max = 0.99;
   p->vec_engine = 0;
   p->cd_panel = 0;
+  p->solve_graphs = 1;
 }
 
 mpq_status mpq_plan_create_from_spectrum(const double* s, const double* V, int64_t n, int64_t r,

@@ -130,6 +130,20 @@ struct mpq_plan_s {
   int* status = nullptr;     // device word
   int64_t ws_cap = 0;
   mpq::Workspace ws;
+  uint64_t ws_gen = 0;       // bumped whenever the workspace is reallocated
+  // captured solves: mpq_solve replays the graph of its launches when it is
+  // called again with the same buffers, sizes and options
+  static constexpr int N_GRAPHS = 4;
+  static constexpr int GRAPH_KEY = 16;
+  struct SolveGraph {
+    uint64_t key[GRAPH_KEY] = {};
+    cudaGraphExec_t exec = nullptr;
+    int64_t launches = 0;
+    uint64_t last_use = 0;  // 0: empty slot
+  };
+  SolveGraph graphs[N_GRAPHS];
+  uint64_t graph_clock = 0;
+  cudaStream_t capture_stream = nullptr;
 };
 
 namespace mpq {
