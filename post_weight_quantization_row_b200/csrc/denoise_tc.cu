@@ -80,6 +80,9 @@ constexpr int QW_BYTES = 128 * 64 * 2;     // weights of one half: 128 x 64 fp16
 // read all of the previous one.
 constexpr uint32_t DT_TMEM_COLS = 512;
 constexpr int T1_BUFS = 4, T2_BUFS = 2;
+// weight tiles in shared memory: more than the TMEM score buffers, so that
+// the epilogue can run ahead of the moment MMAs that still read older halves
+constexpr int QW_BUFS = 4;
 constexpr uint32_t T1_COLS = 128, T2_COLS = 192, TM_MOM = 384;
 constexpr uint32_t IDESC_P1 = idesc_f16(DT_M, DT_N);
 constexpr uint32_t IDESC_P2 = idesc_f16(DT_M, DT_N2);
@@ -90,13 +93,13 @@ constexpr float Q_SHIFT = 8.0f;            // weights carry 2^8: c*'s is 256
 constexpr int N_ATILES = 6;
 constexpr int SM_A = 0;                                   // block operand tiles
 constexpr int SM_B = SM_A + N_ATILES * OPER_BYTES;        // stage ring
-constexpr int SM_QW = SM_B + DT_STAGES * STAGE_BYTES;     // 2 x (hi | lo) weights
-constexpr int SM_T = SM_QW + 2 * 2 * QW_BYTES;            // t per row (fp64, 128 x 8)
+constexpr int SM_QW = SM_B + DT_STAGES * STAGE_BYTES;     // QW_BUFS x (hi | lo) weights
+constexpr int SM_T = SM_QW + QW_BUFS * 2 * QW_BYTES;      // t per row (fp64, 128 x 8)
 constexpr int SM_ROW = SM_T + DT_M * 8 * 8;               // per-row data
 constexpr int SM_BAR = SM_ROW + (3 + 2 * DT_WGS + DT_WGS) * DT_M * 4;
-constexpr int N_BARS = 2 * DT_STAGES + 2 * T1_BUFS + 2 * T2_BUFS + 1 + 2 + 2 + 1;
+constexpr int N_BARS = 2 * DT_STAGES + 2 * T1_BUFS + 2 * T2_BUFS + 1 + 2 * QW_BUFS + 1;
 constexpr int SM_END = SM_BAR + N_BARS * 8 + 16;
-constexpr int DT_SMEM_BYTES = 160 * 1024;  // > half of the SM: one CTA (and TMEM owner) per SM
+constexpr int DT_SMEM_BYTES = 220 * 1024;  // > half of the SM: one CTA (and TMEM owner) per SM
 static_assert(SM_END + 1024 <= DT_SMEM_BYTES, "denoiser shared memory");
 
 enum { A1_HI = 0, A1_LO = 1, A2_Q = 2, A2_X = 3, A2_RH = 4, A2_RL = 5 };
@@ -242,8 +245,8 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_denoise_vec_tc(DenoiseTcArgs 
   uint64_t* t2_empty = t2_full + T2_BUFS;
   uint64_t* a_full = t2_empty + T2_BUFS;
   uint64_t* q_full = a_full + 1;
-  uint64_t* q_free = q_full + 2;
-  uint64_t* mom_done = q_free + 2;
+  uint64_t* q_free = q_full + QW_BUFS;
+  uint64_t* mom_done = q_free + QW_BUFS;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mom_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -263,6 +266,8 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_denoise_vec_tc(DenoiseTcArgs 
     for (int b = 0; b < T2_BUFS; ++b) {
       mbar_init(&t2_full[b], 1);
       mbar_init(&t2_empty[b], DT_EPI_WARPS);
+    }
+    for (int b = 0; b < QW_BUFS; ++b) {
       mbar_init(&q_full[b], DT_EPI_WARPS);
       mbar_init(&q_free[b], 1);
     }
@@ -370,8 +375,8 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_denoise_vec_tc(DenoiseTcArgs 
             }
           }
           if (um < us) {
-            const uint32_t u = hq + um, qb = u % T2_BUFS;
-            if (mbar_test_wait(&q_full[qb], (u / T2_BUFS) & 1)) {
+            const uint32_t u = hq + um, qb = u % QW_BUFS;
+            if (mbar_test_wait(&q_full[qb], (u / QW_BUFS) & 1)) {
               tc_fence_after();
               const int s = (seq + (um >> 1)) % DT_STAGES;
               const uint32_t wq = qw_base + qb * 2u * QW_BYTES;
@@ -412,8 +417,8 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_denoise_vec_tc(DenoiseTcArgs 
       for (uint32_t q = (tu1 > T1_BUFS ? tu1 - T1_BUFS : 0); q < tu1; ++q)
         for (uint32_t i = 0; i < (1u << 25) && !mbar_try_wait(&t1_full[q % T1_BUFS], (q / T1_BUFS) & 1); ++i)
           if (i > 256) __nanosleep(64);
-      for (uint32_t q = (hq > T2_BUFS ? hq - T2_BUFS : 0); q < hq; ++q)
-        for (uint32_t i = 0; i < (1u << 25) && !mbar_try_wait(&q_free[q % T2_BUFS], (q / T2_BUFS) & 1); ++i)
+      for (uint32_t q = (hq > QW_BUFS ? hq - QW_BUFS : 0); q < hq; ++q)
+        for (uint32_t i = 0; i < (1u << 25) && !mbar_try_wait(&q_free[q % QW_BUFS], (q / QW_BUFS) & 1); ++i)
           if (i > 256) __nanosleep(64);
     }
   } else {
@@ -585,7 +590,7 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_denoise_vec_tc(DenoiseTcArgs 
       for (int j = 0; j < a.NT; ++j) {
 #pragma unroll 1
         for (int h = 0; h < 2; ++h, ++hq) {
-          const int buf = hq % T2_BUFS, qb = buf;
+          const int buf = hq % T2_BUFS, qb = hq % QW_BUFS;
           if (ok) ok = warp_wait(&t2_full[buf], (hq / T2_BUFS) & 1, abort_flag, a.status);
           if (!ok) continue;
           tc_fence_after();
@@ -615,8 +620,8 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_denoise_vec_tc(DenoiseTcArgs 
           uint32_t hi[8], lo[8];
 #pragma unroll
           for (int p = 0; p < 8; ++p) split_pair(q[2 * p], q[2 * p + 1], hi[p], lo[p]);
-          // the moment MMAs of two halves ago have read this buffer
-          if (hq >= 2) ok = warp_wait(&q_free[qb], ((hq >> 1) - 1) & 1, abort_flag, a.status);
+          // the moment MMAs of this buffer's previous use have read it
+          if (hq >= QW_BUFS) ok = warp_wait(&q_free[qb], (hq / QW_BUFS - 1) & 1, abort_flag, a.status);
           if (!ok) continue;
           uint8_t* wb = qw + qb * 2 * QW_BYTES + w_off;
           *reinterpret_cast<uint4*>(wb) = make_uint4(hi[0], hi[1], hi[2], hi[3]);

@@ -258,6 +258,18 @@ def test_stage_cd_panels(mpq, kind):
     assert (ref.changes[clean, 1] > 0).any()   # a second sweep reads the closed panels
 
 
+def test_stage_cd_low_rank(mpq):
+    # X 150 x 400 has rank r = 150 < n/2 (H singular, most directions free)
+    p = scalar_case(seed=141, m_out=30, n=400, m=150)
+    s, V, s_cu, V_cu = spectrum_cuda(p.X)
+    assert 2 * len(s) < p.n
+    plan = make_plan(mpq, p, s_cu, V_cu)
+    sc, off = oracle_grid_f32(p)
+    st = orc.init(p.W, codebook_for(p), sc.astype(np.float64), off.astype(np.float64))
+    ref = _cd_compare(p, plan, sc, off, st.idx_rtn, s, V, min_clean=0.25)
+    assert ref.changes[:, 0].sum() > 0
+
+
 def test_stage_energy(mpq):
     p = scalar_case()
     s, V, s_cu, V_cu = spectrum_cuda(p.X)
