@@ -191,16 +191,18 @@ def kernel_work(name, m, n, r, d, K, L):
     return None
 
 
-KERNEL_SOURCE = {"gemm": "gemm_tc.cu", "k_cd": "kernels_cd.cu", "k_denoise_vec_tc": "denoise_tc.cu",
-                 "k_": "kernels_vamp.cu"}
+KERNEL_SOURCE = {"gemm": "gemm_tc.cu", "k_cd_vec_scan": "cd_scan_tc.cu", "k_cd": "kernels_cd.cu",
+                 "k_denoise_vec_tc": "denoise_tc.cu", "k_": "kernels_vamp.cu"}
 
 
 def source_sha(kernel):
-    """Hash of the source file that defines `kernel` plus the shared header."""
+    """Hash of the source file that defines `kernel` plus the device PTX
+    helpers it may use (the host-side declarations elsewhere do not change
+    what a capture measured)."""
     csrc = os.path.join(ROOT, "post_weight_quantization_row_b200", "csrc")
     fname = next(v for k, v in KERNEL_SOURCE.items() if kernel.startswith(k))
     h = hashlib.sha256()
-    for f in (fname, "mpq_internal.cuh", "tc_ptx.cuh"):
+    for f in (fname, "tc_ptx.cuh"):
         h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 
