@@ -55,6 +55,7 @@
 #include <cmath>
 #include <vector>
 
+#include "f32x2.cuh"
 #include "mpq_internal.cuh"
 #include "tc_ptx.cuh"
 
@@ -215,14 +216,6 @@ __device__ __forceinline__ void store_row(uint8_t* tile, int r, const __half (&v
   }
   *reinterpret_cast<uint4*>(tile + kmaj_off(r, 0, 256)) = c0;
   *reinterpret_cast<uint4*>(tile + kmaj_off(r, 8, 256)) = c1;
-}
-
-// (hi, lo) fp16 pairs of two fp32 values: x ~ hi + lo; saturating, so an
-// overflow (caught separately) cannot turn into inf - inf
-__device__ __forceinline__ void split_pair(float a, float b, uint32_t& hi, uint32_t& lo) {
-  asm("cvt.rn.satfinite.f16x2.f32 %0, %2, %1;" : "=r"(hi) : "f"(a), "f"(b));
-  const float2 h = __half22float2(*reinterpret_cast<const __half2*>(&hi));
-  asm("cvt.rn.satfinite.f16x2.f32 %0, %2, %1;" : "=r"(lo) : "f"(a - h.x), "f"(b - h.y));
 }
 
 // 18 warps: five share an SM sub-partition's 16K registers, so at most 96 each
@@ -586,7 +579,9 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_denoise_vec_tc(DenoiseTcArgs 
       const int c16 = sm_bidx[rl] >> 4, kst = sm_bidx[rl] & 15;  // c* as (16-chunk, column)
 
       // ------------------------------------------- pass 2: weights
-      float S2 = 0.0f, zmax = -INFINITY;
+      float zmax = -INFINITY;
+      uint64_t S2p = 0;  // (+0, +0): S2 over even and odd codewords
+      const uint64_t rs2 = f2_pack(rs, rs), g22 = f2_pack(g2, g2), sh2 = f2_pack(Q_SHIFT, Q_SHIFT);
       for (int j = 0; j < a.NT; ++j) {
 #pragma unroll 1
         for (int h = 0; h < 2; ++h, ++hq) {
@@ -608,18 +603,28 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_denoise_vec_tc(DenoiseTcArgs 
           // below.  (Its logit is 0 up to R's rounding, so z(c*) reaches the
           // overflow mark only at g > ~5e9, where the point mass on c* that
           // the overflow fallback returns is the answer.)
-          float q[16];
-#pragma unroll
-          for (int k = 0; k < 16; ++k) {  // Q + X is exact; R carries the rounding
-            const float z = fmaf(g2, fmaf(__uint_as_float(R[k]), rs, __uint_as_float(Q[k]) + __uint_as_float(X[k])),
-                                 Q_SHIFT);
-            zmax = fmaxf(zmax, z);
-            q[k] = ex2_approx(z);
-            S2 = fmaf(q[k], __uint_as_float(X[k]), S2);  // X = -|c - c*|^2 / 2
-          }
+          // Two codewords per packed f32x2 instruction, each half rounded as
+          // the scalar form: z = g2 (R rs + (Q + X)) + 8 (Q + X is exact, R
+          // carries the rounding), q = 2^z, S2 += q X (X = -|c - c*|^2 / 2),
+          // and the weight as a saturating fp16 pair hi + lo.
           uint32_t hi[8], lo[8];
 #pragma unroll
-          for (int p = 0; p < 8; ++p) split_pair(q[2 * p], q[2 * p + 1], hi[p], lo[p]);
+          for (int p = 0; p < 8; ++p) {
+            const uint64_t xv = f2_pack(__uint_as_float(X[2 * p]), __uint_as_float(X[2 * p + 1]));
+            const uint64_t qx = f2_add(f2_pack(__uint_as_float(Q[2 * p]), __uint_as_float(Q[2 * p + 1])), xv);
+            const uint64_t rr = f2_pack(__uint_as_float(R[2 * p]), __uint_as_float(R[2 * p + 1]));
+            float z0, z1;
+            f2_unpack(f2_fma(g22, f2_fma(rr, rs2, qx), sh2), z0, z1);
+            zmax = fmaxf(zmax, fmaxf(z0, z1));
+            const float e0 = ex2_approx(z0), e1 = ex2_approx(z1);
+            const uint64_t e = f2_pack(e0, e1);
+            S2p = f2_fma(e, xv, S2p);
+            asm("cvt.rn.satfinite.f16x2.f32 %0, %2, %1;" : "=r"(hi[p]) : "f"(e0), "f"(e1));
+            const float2 h = __half22float2(*reinterpret_cast<const __half2*>(&hi[p]));
+            float d0, d1;
+            f2_unpack(f2_sub(e, f2_pack(h.x, h.y)), d0, d1);
+            asm("cvt.rn.satfinite.f16x2.f32 %0, %2, %1;" : "=r"(lo[p]) : "f"(d0), "f"(d1));
+          }
           // the moment MMAs of this buffer's previous use have read it
           if (hq >= QW_BUFS) ok = warp_wait(&q_free[qb], (hq / QW_BUFS - 1) & 1, abort_flag, a.status);
           if (!ok) continue;
@@ -638,7 +643,11 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_denoise_vec_tc(DenoiseTcArgs 
           if (lane == 0) mbar_arrive(&q_full[qb]);
         }
       }
-      sm_s2[wg * DT_M + rl] = S2;
+      {
+        float s2a, s2b;
+        f2_unpack(S2p, s2a, s2b);
+        sm_s2[wg * DT_M + rl] = s2a + s2b;
+      }
       sm_bval[wg * DT_M + rl] = zmax;
       named_sync_epi();
       if (wg == 0) {
