@@ -23,6 +23,7 @@
 
 #include <cmath>
 
+#include "f32x2.cuh"
 #include "mpq_internal.cuh"
 #include "tc_ptx.cuh"
 
@@ -250,6 +251,7 @@ __global__ void __launch_bounds__(SC_THREADS, 1) k_cd_vec_scan(ScanArgs a) {
     }
     asm volatile("bar.sync 1, %0;" ::"n"(SC_EPI_WARPS * 32) : "memory");
     const float rsc = sm_rsc[rl];
+    const uint64_t rsc2 = f2_pack(rsc, rsc);
     float best = INFINITY;
     int bidx = 0x7fffffff;
     bool ok = true;
@@ -264,20 +266,24 @@ __global__ void __launch_bounds__(SC_THREADS, 1) k_cd_vec_scan(ScanArgs a) {
       __syncwarp();
       if (lane == 0) mbar_arrive(&t_empty[buf]);
       const float4* q4 = reinterpret_cast<const float4*>(smem + SC_B + s * SC_STAGE + SC_OPER) + wg * 8;
+      // score = D rsc + qtab, two codewords per packed f32x2 fma
       float sv[32];
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         const float4 q = q4[c];
-        sv[4 * c + 0] = fmaf(__uint_as_float(v[4 * c + 0]), rsc, q.x);
-        sv[4 * c + 1] = fmaf(__uint_as_float(v[4 * c + 1]), rsc, q.y);
-        sv[4 * c + 2] = fmaf(__uint_as_float(v[4 * c + 2]), rsc, q.z);
-        sv[4 * c + 3] = fmaf(__uint_as_float(v[4 * c + 3]), rsc, q.w);
+        f2_unpack(f2_fma(f2_pack(__uint_as_float(v[4 * c]), __uint_as_float(v[4 * c + 1])), rsc2,
+                         f2_pack(q.x, q.y)),
+                  sv[4 * c], sv[4 * c + 1]);
+        f2_unpack(f2_fma(f2_pack(__uint_as_float(v[4 * c + 2]), __uint_as_float(v[4 * c + 3])), rsc2,
+                         f2_pack(q.z, q.w)),
+                  sv[4 * c + 2], sv[4 * c + 3]);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&b_empty[s]);  // qtab of this stage is read
-      float m0 = sv[0];
+      float m0 = fmin3(sv[0], sv[1], sv[2]);
 #pragma unroll
-      for (int c = 1; c < 32; ++c) m0 = fminf(m0, sv[c]);
+      for (int c = 3; c < 31; c += 2) m0 = fmin3(m0, sv[c], sv[c + 1]);
+      m0 = fminf(m0, sv[31]);
       if (m0 < best) {  // first index of the chunk minimum
         int kk = 31;
 #pragma unroll

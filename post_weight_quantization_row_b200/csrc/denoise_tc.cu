@@ -488,9 +488,10 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_denoise_vec_tc(DenoiseTcArgs 
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&t1_empty[buf]);
-        float m0 = __uint_as_float(v[0]);
+        float m0 = fmax3(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]));
 #pragma unroll
-        for (int k = 1; k < 32; ++k) m0 = fmaxf(m0, __uint_as_float(v[k]));
+        for (int k = 3; k < 31; k += 2) m0 = fmax3(m0, __uint_as_float(v[k]), __uint_as_float(v[k + 1]));
+        m0 = fmaxf(m0, __uint_as_float(v[31]));
         if (m0 > best) {  // first index of the chunk maximum
           int kk = 31;
 #pragma unroll
@@ -615,7 +616,7 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_denoise_vec_tc(DenoiseTcArgs 
             const uint64_t rr = f2_pack(__uint_as_float(R[2 * p]), __uint_as_float(R[2 * p + 1]));
             float z0, z1;
             f2_unpack(f2_fma(g22, f2_fma(rr, rs2, qx), sh2), z0, z1);
-            zmax = fmaxf(zmax, fmaxf(z0, z1));
+            zmax = fmax3(zmax, z0, z1);
             const float e0 = ex2_approx(z0), e1 = ex2_approx(z1);
             const uint64_t e = f2_pack(e0, e1);
             S2p = f2_fma(e, xv, S2p);

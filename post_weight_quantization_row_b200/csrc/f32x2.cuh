@@ -1,5 +1,6 @@
-// Packed fp32 pairs for sm_100 (f32x2 add/mul/fma: two fp32 operations per
-// instruction, each half rounded exactly as the scalar operation).
+// sm_100 fp32 arithmetic helpers: packed pairs (f32x2 add/sub/mul/fma, two
+// fp32 operations per instruction, each half rounded exactly as the scalar
+// operation) and three-input min/max (exact, like two two-input ones).
 #pragma once
 #include <stdint.h>
 
@@ -32,6 +33,17 @@ __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
 __device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
   uint64_t d;
   asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+__device__ __forceinline__ float fmin3(float a, float b, float c) {
+  float d;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
 }
 
