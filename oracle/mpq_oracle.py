@@ -96,18 +96,24 @@ def hessian(s: np.ndarray, V: np.ndarray) -> np.ndarray:
 # codebooks and a2: init
 # ----------------------------------------------------------------------------
 
-def minmax_grid(W: np.ndarray, L: int):
-    """Per-row uniform grid of L levels (reading R2), following the min-max
-    formula of the [NeUQI] note ("Existing pain points"):
+def minmax_grid(W: np.ndarray, L: int, group: int = 0):
+    """Uniform grid of L levels (reading R2), following the min-max formula
+    of the [NeUQI] note ("Existing pain points"):
     s = (max w - min w) / (2^k - 1), z = -round(min w / s).
-    Returns (scale, offset) with level k = scale * k + offset."""
+    Returns (scale, offset) with level k = scale * k + offset: one grid per
+    row (m), or with ``group`` > 0 one grid per group of that many
+    consecutive columns of a row (m x n/group; the pages' group-wise setting,
+    [MPQ-note] experimental setup "group 128")."""
     W = np.asarray(W, np.float64)
-    lo, hi = W.min(axis=1), W.max(axis=1)
+    m, n = W.shape
+    Wg = W.reshape(m, n // group, group) if group else W[:, None, :]
+    lo, hi = Wg.min(axis=2), Wg.max(axis=2)
     scale = (hi - lo) / (L - 1)
     const = ~(hi > lo)
     scale[const] = np.where(hi[const] != 0.0, np.abs(hi[const]), 1.0)
     z = np.clip(np.rint(-lo / scale), 0, L - 1)
-    return scale, -scale * z
+    offset = -scale * z
+    return (scale, offset) if group else (scale[:, 0], offset[:, 0])
 
 
 def rms_scale(W: np.ndarray):
@@ -121,6 +127,19 @@ def rms_scale(W: np.ndarray):
 def row_candidates(codebook: np.ndarray, scale: float, offset: float) -> np.ndarray:
     """All codewords of one row's block codebook C_b, K x d, in weight units."""
     return scale * np.asarray(codebook, np.float64) + offset
+
+
+def block_candidates(codebook: np.ndarray, scale_i, offset_i, B: int) -> np.ndarray:
+    """The codebooks C_b of every block of one row, B x K x d: the same for
+    all blocks with a per-row grid (scalar scale_i), or the grid of each
+    block's group (scale_i of length n/group, B a multiple of it)."""
+    s = np.asarray(scale_i, np.float64)
+    o = np.asarray(offset_i, np.float64)
+    cb = np.asarray(codebook, np.float64)
+    if s.ndim == 0:
+        return np.broadcast_to(s * cb + o, (B,) + cb.shape)
+    per = B // s.size  # blocks per group
+    return np.repeat(s, per)[:, None, None] * cb[None] + np.repeat(o, per)[:, None, None]
 
 
 def scalar_levels(L: int) -> np.ndarray:
@@ -145,26 +164,30 @@ class InitState:
     beta: np.ndarray
 
 
-def init(W: np.ndarray, codebook: np.ndarray, scale=None, offset=None, beta0: float = 1.0) -> InitState:
+def init(W: np.ndarray, codebook: np.ndarray, scale=None, offset=None, beta0: float = 1.0,
+         group: int = 0) -> InitState:
     """[MPQ-note] hyper-parameter section: gamma1_0 = 1 / MSE(w, w_rtn);
-    cavity r1_0 = w (R4); beta_0 = 1.  Scale/offset default to the per-row
-    min-max grid (d = 1) or the RMS lattice scale (d > 1)."""
+    cavity r1_0 = w (R4); beta_0 = 1.  Scale/offset default to the min-max
+    grid (d = 1; per row, or per group of ``group`` columns) or the RMS
+    lattice scale (d > 1)."""
     W = np.asarray(W, np.float64)
     d = codebook.shape[1]
     if scale is None:
         if d == 1:
-            scale, offset = minmax_grid(W, codebook.shape[0])
+            scale, offset = minmax_grid(W, codebook.shape[0], group)
         else:
             scale, offset = rms_scale(W)
     scale = np.asarray(scale, np.float64)
     offset = np.asarray(offset, np.float64)
     m, n = W.shape
-    idx = np.zeros((m, n // d), dtype=np.int64)
+    B = n // d
+    idx = np.zeros((m, B), dtype=np.int64)
     g1 = np.zeros(m)
     for i in range(m):
-        cand = row_candidates(codebook, scale[i], offset[i])
-        idx[i] = nearest_codewords(W[i], cand)
-        w_rtn = cand[idx[i]].reshape(-1)
+        cand = block_candidates(codebook, scale[i], offset[i], B)      # B x K x d
+        blocks = W[i].reshape(B, d)
+        idx[i] = np.argmin(((blocks[:, None, :] - cand) ** 2).sum(axis=2), axis=1)
+        w_rtn = cand[np.arange(B), idx[i]].reshape(-1)
         mse = np.mean((W[i] - w_rtn) ** 2)
         g1[i] = 1.0 / max(mse, 1e-30)
     return InitState(scale, offset, idx, g1, W.copy(), np.full(m, float(beta0)))
@@ -198,19 +221,19 @@ def denoise(R1, gamma1, codebook, scale, offset, W=None, gamma_anchor=None) -> D
     idx = np.zeros((m, B), dtype=np.int64)
     gap = np.zeros((m, B))
     for i in range(m):
-        cand = row_candidates(codebook, scale[i], offset[i])          # K x d
+        cand = block_candidates(codebook, scale[i], offset[i], B)      # B x K x d
         r = R1[i].reshape(B, d)
-        logit = -0.5 * gamma1[i] * ((r[:, None, :] - cand[None, :, :]) ** 2).sum(axis=2)
+        logit = -0.5 * gamma1[i] * ((r[:, None, :] - cand) ** 2).sum(axis=2)
         if gamma_anchor is not None:
             wb = np.asarray(W[i], np.float64).reshape(B, d)
-            logit = logit - 0.5 * gamma_anchor[i] * ((wb[:, None, :] - cand[None, :, :]) ** 2).sum(axis=2)
+            logit = logit - 0.5 * gamma_anchor[i] * ((wb[:, None, :] - cand) ** 2).sum(axis=2)
         top = np.argmax(logit, axis=1)
         mx = logit[np.arange(B), top]
         q = np.exp(logit - mx[:, None])
         q /= q.sum(axis=1, keepdims=True)
         # moments centred on the argmax codeword (no cancellation)
-        cstar = cand[top]                                               # B x d
-        dc = cand[None, :, :] - cstar[:, None, :]                       # B x K x d
+        cstar = cand[np.arange(B), top]                                 # B x d
+        dc = cand - cstar[:, None, :]                                   # B x K x d
         m1 = np.einsum("bk,bkd->bd", q, dc)
         m2 = np.einsum("bk,bk->b", q, (dc * dc).sum(axis=2))
         xhat[i] = (cstar + m1).reshape(-1)
@@ -326,8 +349,9 @@ def decode(idx, codebook, scale, offset):
     m = idx.shape[0]
     out = []
     for i in range(m):
-        cand = row_candidates(codebook, scale[i], offset[i])
-        out.append(cand[idx[i]].reshape(-1))
+        B = idx[i].size
+        cand = block_candidates(codebook, scale[i], offset[i], B)
+        out.append(cand[np.arange(B), idx[i]].reshape(-1))
     return np.asarray(out)
 
 
@@ -351,7 +375,7 @@ def cd(W, idx0, codebook, scale, offset, H, sweeps: int, tie_rel: float = 1e-5) 
     first_tie = np.full(m, -1, dtype=np.int64)
     min_gap = np.full(m, np.inf)
     for i in range(m):
-        cand = row_candidates(codebook, scale[i], offset[i])
+        cand = block_candidates(codebook, scale[i], offset[i], B)      # B x K x d
         x = X[i].copy()
         h = H @ (W[i] - x)
         step = 0
@@ -361,7 +385,7 @@ def cd(W, idx0, codebook, scale, offset, H, sweeps: int, tie_rel: float = 1e-5) 
             for b in range(B):
                 sl = slice(b * d, (b + 1) * d)
                 G = H[sl, sl]
-                delta = cand - x[sl][None, :]
+                delta = cand[b] - x[sl][None, :]
                 dE = -delta @ h[sl] + 0.5 * np.einsum("kd,de,ke->k", delta, G, delta)
                 k = int(np.argmin(dE))
                 E = 0.5 * float((W[i] - x) @ h)
@@ -374,7 +398,7 @@ def cd(W, idx0, codebook, scale, offset, H, sweeps: int, tie_rel: float = 1e-5) 
                 if dE[k] < 0.0:
                     dlt = delta[k]
                     h -= H[:, sl] @ dlt
-                    x[sl] = cand[k]
+                    x[sl] = cand[b, k]
                     idx[i, b] = k
                     nchg += 1
                 step += 1
@@ -423,12 +447,12 @@ class SolveOut:
 
 def solve(W, codebook, s, V, T_vamp: int, cd_sweeps: int, scale=None, offset=None,
           beta0: float = 1.0, damping: float = 0.5, tau: float = math.inf,
-          keep_trace: bool = False) -> SolveOut:
+          keep_trace: bool = False, group: int = 0) -> SolveOut:
     """The MPQ solve of every row ([MPQ-note] flowchart and Overall
     framework): init -> T_vamp x (denoiser -> extrinsic -> linear module ->
     M-step) -> marginal MAP argmax -> exact block CD -> energies."""
     W = np.asarray(W, np.float64)
-    st = init(W, codebook, scale, offset, beta0)
+    st = init(W, codebook, scale, offset, beta0, group)
     g10 = st.gamma1.copy()
     ga = None if not math.isfinite(tau) else g10 / (tau * tau)
     R1, g1, beta = st.R1, st.gamma1.copy(), st.beta.copy()
