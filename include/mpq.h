@@ -102,6 +102,13 @@ typedef struct {
                              bytes) fits in 32 MiB, at least 512; else the
                              panel width in columns, a positive multiple of
                              128 (a panel as wide as n is one panel). */
+  int32_t group_size;     /* d = 1: 0 (default) one min-max grid per row; G > 0
+                             (a multiple of 128 dividing n) one grid per group
+                             of G consecutive columns of a row, the pages'
+                             group-wise setting ("group 128").  Then every
+                             scale/offset array of the API (row_scale,
+                             row_offset, the stage hooks' scale/offset) holds
+                             m x n/G values, row-major.  Must be 0 for d = 8. */
   int32_t solve_graphs;   /* 1 (default): when mpq_solve or mpq_solve_host is
                              called a second time with the same buffers, sizes
                              and options (the buffers' contents may change), it

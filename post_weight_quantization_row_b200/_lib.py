@@ -43,7 +43,7 @@ class Params(C.Structure):
                 ("gamma_lo_rel", C.c_double), ("gamma_hi_rel", C.c_double),
                 ("alpha_min", C.c_double), ("alpha_max", C.c_double),
                 ("vec_engine", C.c_int32), ("cd_panel", C.c_int32),
-                ("solve_graphs", C.c_int32)]
+                ("group_size", C.c_int32), ("solve_graphs", C.c_int32)]
 
 
 class RowStats(C.Structure):
@@ -157,13 +157,19 @@ def make_params(d: int, K: int, codebook=None, **kw) -> tuple:
 class Plan:
     """A solver plan: the spectrum of X and the codebook tables, on one GPU."""
 
-    def __init__(self, handle):
+    def __init__(self, handle, group_size: int = 0):
         self._h = P(handle)
         n, r, d, K = I64(), I64(), I32(), I32()
         check(lib.mpq_plan_info(self._h, C.byref(n), C.byref(r), C.byref(d), C.byref(K)), "info")
         self.n, self.r, self.d, self.K = n.value, r.value, d.value, K.value
         self.B = self.n // self.d
+        self.G = int(group_size)                      # scalar grid group (0: per row)
+        self.ng = self.n // self.G if self.G else 1   # grids per row
         self.device = torch.cuda.current_device()
+
+    def _sshape(self, m):
+        """Shape of a scale/offset array for m rows."""
+        return (m,) if self.ng == 1 else (m, self.ng)
 
     # ------------------------------------------------------------ creation --
     @classmethod
@@ -179,7 +185,7 @@ class Plan:
                                                 C.byref(prm), _stream(), C.byref(h)),
               "mpq_plan_create_from_spectrum")
         del keep
-        return cls(h.value)
+        return cls(h.value, kw.get("group_size", 0))
 
     @classmethod
     def from_x(cls, X: torch.Tensor, d: int, K: int, codebook=None, **kw):
@@ -189,7 +195,7 @@ class Plan:
         check(lib.mpq_plan_create_from_x(_ptr(X, torch.float32, name="X"), m, n, C.byref(prm),
                                          _stream(), C.byref(h)), "mpq_plan_create_from_x")
         del keep
-        return cls(h.value)
+        return cls(h.value, kw.get("group_size", 0))
 
     def close(self):
         if self._h is not None and self._h.value:
@@ -243,8 +249,8 @@ class Plan:
             out["cd_changes"] = torch.zeros(m, max(cd_sweeps, 1), dtype=torch.int32, device=dev)
             st = RowStats(out["gamma1"].data_ptr(), out["beta"].data_ptr(),
                           out["clamps"].data_ptr(), out["cd_changes"].data_ptr())
-        check(lib.mpq_solve(self._h, _ptr(W), m, _ptr(row_scale, torch.float32, (m,), "row_scale"),
-                            _ptr(row_offset, torch.float32, (m,), "row_offset"), T_vamp, cd_sweeps,
+        check(lib.mpq_solve(self._h, _ptr(W), m, _ptr(row_scale, torch.float32, self._sshape(m), "row_scale"),
+                            _ptr(row_offset, torch.float32, self._sshape(m), "row_offset"), T_vamp, cd_sweeps,
                             _ptr(out["idx"], torch.int16, (m, self.B), "idx"),
                             _ptr(out.get("w_hat"), torch.float32, None, "w_hat"),
                             _ptr(out.get("energy"), torch.float32, None, "energy"),
@@ -277,8 +283,8 @@ class Plan:
             scale = scale.clone()
             offset = offset.clone()
         else:
-            scale = torch.empty(m, dtype=torch.float32, device=dev)
-            offset = torch.empty(m, dtype=torch.float32, device=dev)
+            scale = torch.empty(self._sshape(m), dtype=torch.float32, device=dev)
+            offset = torch.empty(self._sshape(m), dtype=torch.float32, device=dev)
         idx = torch.empty(m, self.B, dtype=torch.int16, device=dev)
         g0 = torch.empty(m, dtype=torch.float64, device=dev)
         check(lib.mpq_stage_init(self._h, _ptr(W, torch.float32, (m, self.n), "W"), m, int(given),
@@ -295,8 +301,8 @@ class Plan:
         idx = torch.empty(m, self.B, dtype=torch.int16, device=dev)
         check(lib.mpq_stage_denoise(self._h, _ptr(R1, torch.float32, (m, self.n), "R1"),
                                     _ptr(gamma1, torch.float64, (m,), "gamma1"),
-                                    _ptr(scale, torch.float32, (m,), "scale"),
-                                    _ptr(offset, torch.float32, (m,), "offset"), m,
+                                    _ptr(scale, torch.float32, self._sshape(m), "scale"),
+                                    _ptr(offset, torch.float32, self._sshape(m), "offset"), m,
                                     _ptr(W, torch.float32, None, "W"),
                                     _ptr(gamma1_0, torch.float64, None, "gamma1_0"), _ptr(xhat),
                                     _ptr(vblock), _ptr(vsum), _ptr(idx), _stream()),
@@ -334,8 +340,8 @@ class Plan:
         idx = idx.clone()
         changes = torch.zeros(m, max(sweeps, 1), dtype=torch.int32, device=W.device)
         check(lib.mpq_stage_cd(self._h, _ptr(W, torch.float32, (m, self.n), "W"), m,
-                               _ptr(scale, torch.float32, (m,), "scale"),
-                               _ptr(offset, torch.float32, (m,), "offset"),
+                               _ptr(scale, torch.float32, self._sshape(m), "scale"),
+                               _ptr(offset, torch.float32, self._sshape(m), "offset"),
                                _ptr(idx, torch.int16, (m, self.B), "idx"), sweeps, _ptr(changes),
                                _stream()), "mpq_stage_cd")
         return {"idx": idx, "changes": changes}
@@ -345,8 +351,8 @@ class Plan:
         w_hat = torch.empty(m, self.n, dtype=torch.float32, device=W.device)
         energy = torch.empty(m, dtype=torch.float32, device=W.device)
         check(lib.mpq_stage_energy(self._h, _ptr(W, torch.float32, (m, self.n), "W"), m,
-                                   _ptr(scale, torch.float32, (m,), "scale"),
-                                   _ptr(offset, torch.float32, (m,), "offset"),
+                                   _ptr(scale, torch.float32, self._sshape(m), "scale"),
+                                   _ptr(offset, torch.float32, self._sshape(m), "offset"),
                                    _ptr(idx, torch.int16, (m, self.B), "idx"), _ptr(w_hat),
                                    _ptr(energy), _stream()), "mpq_stage_energy")
         return {"w_hat": w_hat, "energy": energy}
@@ -362,8 +368,8 @@ class Plan:
         if energy is None:
             energy = torch.empty(m, dtype=torch.float32, device=W.device)
         check(lib.mpq_stage_energy_noalloc(self._h, _ptr(W, torch.float32, (m, self.n), "W"), m,
-                                           _ptr(scale, torch.float32, (m,), "scale"),
-                                           _ptr(offset, torch.float32, (m,), "offset"),
+                                           _ptr(scale, torch.float32, self._sshape(m), "scale"),
+                                           _ptr(offset, torch.float32, self._sshape(m), "offset"),
                                            _ptr(idx, torch.int16, (m, self.B), "idx"),
                                            _ptr(w_hat), _ptr(energy), _stream()),
               "mpq_stage_energy_noalloc")

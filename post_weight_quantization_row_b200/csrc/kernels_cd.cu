@@ -71,7 +71,8 @@ __device__ __forceinline__ void load_h_tile(float* sH, const float* H, int64_t n
 
 __global__ void __launch_bounds__(CD1_WARPS * 32, 2)
     k_cd_tile_decide(int64_t m, int64_t n, int L, int64_t t0, int tw,
-                     const float* __restrict__ scale, const float* __restrict__ H,
+                     const float* __restrict__ scale, int ng, int gi,
+                     const float* __restrict__ sref, const float* __restrict__ H,
                      uint16_t* __restrict__ idx, const float* __restrict__ h, int64_t ldh,
                      int sweeps, int sw,
                      int32_t* __restrict__ changes, __half* __restrict__ dhi,
@@ -94,8 +95,13 @@ __global__ void __launch_bounds__(CD1_WARPS * 32, 2)
   if (row >= m) return;
   __half* drow_hi = dhi + row * lda;
   __half* drow_lo = dlo + row * lda;
-  const float sc = scale[row];
-  if (lane == 0) d_unscale[row] = -sc;
+  // the tile's grid: the row's, or its group's (a group holds whole tiles).
+  // With group-wise grids the tiles of a panel have different scales, so
+  // Delta leaves as (k_new - k_old) scale / sref, an fp16 pair, against the
+  // row's reference scale sref; otherwise as the exact level difference.
+  const float sc = scale[row * ng + gi];
+  const float dsc = sref ? sc / sref[row] : 1.0f;
+  if (lane == 0) d_unscale[row] = sref ? -sref[row] : -sc;
   uint16_t* ir = idx + row * n + t0;
   // a row stops after a sweep without change (its Delta row stays zero)
   if (sw > 0 && changes[row * sweeps + sw - 1] == 0) {
@@ -180,8 +186,10 @@ __global__ void __launch_bounds__(CD1_WARPS * 32, 2)
       dk = (float)(knew - (int)ir[col]);
       ir[col] = (uint16_t)knew;
     }
-    drow_hi[col] = __float2half_rn(dk);
-    drow_lo[col] = __float2half_rn(0.0f);
+    const float dv = dk * dsc;  // exact when dsc = 1
+    const __half dh = __float2half_rn(dv);
+    drow_hi[col] = dh;
+    drow_lo[col] = __float2half_rn(dv - __half2float(dh));
   }
   if (lane == 0 && ntile > 0) {
     changes[row * sweeps + sw] += ntile;
@@ -418,7 +426,27 @@ __global__ void __launch_bounds__(CD8_APPLY_WARPS * 32)
   }
 }
 
+// per-row maximum of the group scales (the reference scale of grouped Delta)
+__global__ void k_row_max(const float* __restrict__ scale, int64_t m, int64_t ng,
+                          float* __restrict__ out) {
+  const int64_t row = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (row >= m) return;
+  float mx = scale[row * ng];
+  for (int64_t g = 1; g < ng; ++g) mx = fmaxf(mx, scale[row * ng + g]);
+  out[row] = mx;
+}
+
 }  // namespace
+
+mpq_status launch_row_max(const float* scale, int64_t m, int64_t ng, float* out, cudaStream_t st) {
+  if (m <= 0) return MPQ_OK;
+  {
+    ProfScope ps_("k_row_max", st);
+    k_row_max<<<(unsigned)cdiv(m, 256), 256, 0, st>>>(scale, m, ng, out);
+  }
+  count_launch();
+  return check_launch("k_row_max");
+}
 
 // Width of a CD panel: whole tiles, with the panel's slab of the gradient
 // (m x P fp32) within CD_PANEL_BYTES so that it stays in L2 while the
@@ -453,7 +481,10 @@ mpq_status launch_cd(mpq_plan_s* p, const float* W, int64_t m, const float* scal
   int* panel_flags = w.tile_count + (int64_t)sweeps * nt;  // sweeps x np
   MPQ_CUDA(cudaMemsetAsync(w.tile_count, 0, sizeof(int) * sweeps * (nt + np), st));
   const CUtensorMap* c_reduce = (h == w.Hg) ? &w.tm_hg : nullptr;
-  const bool a_exact = p->d == 1 || p->vec_tc;  // c_new - c_old is exact in fp16
+  // c_new - c_old is exact in fp16 (level differences, lattice coordinates);
+  // with group-wise grids Delta carries the group's scale ratio (an fp16 pair)
+  const bool a_exact = (p->d == 1 && !p->G) || p->vec_tc;
+  if (p->d == 1 && p->G) MPQ_TRY(launch_row_max(scale, m, p->ng, w.sref, st));
   auto update = [&](int64_t a_k0, int64_t b_k0, int64_t K, int64_t c0, int64_t c1,
                     const int* gate, const char* tag) -> mpq_status {
     if (c1 <= c0) return MPQ_OK;
@@ -499,7 +530,8 @@ mpq_status launch_cd(mpq_plan_s* p, const float* W, int64_t m, const float* scal
         if (p->d == 1) {
           ProfScope ps_("k_cd_tile_decide", st);
           k_cd_tile_decide<<<(unsigned)cdiv(m, CD1_WARPS), CD1_WARPS * 32, CD1_SMEM, st>>>(
-              m, n, p->K, t0, tw, scale, p->H32, idx, h, ldh, sweeps, sw, changes, dhi, dlo,
+              m, n, p->K, t0, tw, scale, (int)p->ng, p->G ? (int)(t0 / p->G) : 0,
+              p->G ? w.sref : nullptr, p->H32, idx, h, ldh, sweeps, sw, changes, dhi, dlo,
               w.As.ld, w.As.row_unscale, tflag, pflag);
           count_launch();
           rc = check_launch("k_cd_tile_decide");

@@ -153,6 +153,65 @@ __global__ void __launch_bounds__(ROW_THREADS)
   if (threadIdx.x == 0) gamma1_0[row] = 1.0 / fmax(se / (double)n, 1e-30);
 }
 
+// d = 1 with group-wise grids: one min-max grid per group of G consecutive
+// columns (unless given; scale/offset are m x n/G), nearest level, and
+// gamma1_0 from the whole row.  One warp per group.
+__global__ void __launch_bounds__(ROW_THREADS)
+    k_init_scalar_groups(const float* __restrict__ W, int64_t n, int L, int G, int given,
+                         float* __restrict__ scale, float* __restrict__ offset,
+                         uint16_t* __restrict__ idx, double* __restrict__ gamma1_0, int* status) {
+  __shared__ double ds[33];
+  const int64_t row = blockIdx.x;
+  const int ng = (int)(n / G);
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const float* w = W + row * n;
+  double se = 0.0;
+  bool bad = false;
+  for (int g = wid; g < ng; g += nw) {
+    const float* wg = w + (int64_t)g * G;
+    float s32, o32;
+    if (!given) {
+      float lo = INFINITY, hi = -INFINITY;
+      for (int j = lane; j < G; j += 32) {
+        const float x = wg[j];
+        bad |= !isfinite(x);
+        lo = fminf(lo, x);
+        hi = fmaxf(hi, x);
+      }
+      lo = warp_reduce(lo, MinF());
+      hi = warp_reduce(hi, MaxF());
+      double s = ((double)hi - (double)lo) / (double)(L - 1);
+      if (!(hi > lo)) s = (hi != 0.0f) ? fabs((double)hi) : 1.0;
+      double z = rint(-(double)lo / s);
+      z = fmin(fmax(z, 0.0), (double)(L - 1));
+      s32 = (float)s;
+      o32 = (float)(-s * z);
+      if (lane == 0) {
+        scale[row * ng + g] = s32;
+        offset[row * ng + g] = o32;
+      }
+    } else {
+      s32 = scale[row * ng + g];
+      o32 = offset[row * ng + g];
+    }
+    const double sc = s32, off = o32;
+    for (int j = lane; j < G; j += 32) {
+      const double x = wg[j];
+      const double t = (x - off) / sc;
+      const double k0 = fmin(fmax(floor(t), 0.0), (double)(L - 1));
+      const double k1 = fmin(k0 + 1.0, (double)(L - 1));
+      const double d0 = fabs(sc * k0 + off - x), d1 = fabs(sc * k1 + off - x);
+      const double k = (d1 < d0) ? k1 : k0;
+      idx[row * n + (int64_t)g * G + j] = (uint16_t)k;
+      const double e = x - (sc * k + off);
+      se += e * e;
+    }
+  }
+  if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(status, STATUS_NONFINITE);
+  se = block_sum(se, ds);
+  if (threadIdx.x == 0) gamma1_0[row] = 1.0 / fmax(se / (double)n, 1e-30);
+}
+
 // d = 8: per-row RMS scale (unless given), offset 0.
 __global__ void __launch_bounds__(ROW_THREADS)
     k_init_rms(const float* __restrict__ W, int64_t n, int given, float* __restrict__ scale,
@@ -354,18 +413,30 @@ __device__ __forceinline__ float scalar_den_elem(const ScalarDen& c, const float
   return c.sc2f * var;
 }
 
+// With GROUPED, scale/offset hold one grid per group of G columns and the
+// per-group constants (precision regime included) live in shared memory.
+template <bool GROUPED>
 __global__ void __launch_bounds__(ROW_THREADS)
     k_denoise_scalar(const float* __restrict__ R1, const double* __restrict__ gamma1,
                      const float* __restrict__ scale, const float* __restrict__ offset,
-                     int64_t n, int L, const float* __restrict__ W,
+                     int64_t n, int L, int G, const float* __restrict__ W,
                      const double* __restrict__ gamma1_0, double inv_tau2,
                      float* __restrict__ xhat, float* __restrict__ vblock,
                      double* __restrict__ vsum, uint16_t* __restrict__ idx) {
   __shared__ double ds[33];
+  extern __shared__ __align__(16) uint8_t den_smem[];
+  ScalarDen* s_den = reinterpret_cast<ScalarDen*>(den_smem);  // GROUPED: one per group
   const int64_t row = blockIdx.x;
   const bool anchored = (W != nullptr);
-  const ScalarDen c = scalar_den_row(scale[row], offset[row], gamma1[row], L, anchored,
+  const int ng = GROUPED ? (int)(n / G) : 1;
+  const ScalarDen c = scalar_den_row(scale[row * ng], offset[row * ng], gamma1[row], L, anchored,
                                      anchored ? gamma1_0[row] : 0.0, inv_tau2);
+  if (GROUPED) {
+    for (int g = threadIdx.x; g < ng; g += blockDim.x)
+      s_den[g] = scalar_den_row(scale[row * ng + g], offset[row * ng + g], gamma1[row], L,
+                                anchored, anchored ? gamma1_0[row] : 0.0, inv_tau2);
+    __syncthreads();
+  }
   // the per-weight loop, instantiated once per precision regime and prior so
   // that the row-uniform choices cost no branch per weight
   auto weights = [&](auto prec, auto anch) -> float {
@@ -387,8 +458,14 @@ __global__ void __launch_bounds__(ROW_THREADS)
         const int64_t j = j0 + (int64_t)u * blockDim.x;
         if (j < n) {
           const int64_t o = row * n + j;
-          float xh, ks;
-          const float v = scalar_den_elem<PRECISE, ANCH>(c, rv[u], wv[u], xh, ks);
+          float xh, ks, v;
+          if constexpr (GROUPED) {
+            const ScalarDen& cg = s_den[j / G];  // uniform over a warp (G % 32 == 0)
+            v = cg.precise ? scalar_den_elem<true, ANCH>(cg, rv[u], wv[u], xh, ks)
+                           : scalar_den_elem<false, ANCH>(cg, rv[u], wv[u], xh, ks);
+          } else {
+            v = scalar_den_elem<PRECISE, ANCH>(c, rv[u], wv[u], xh, ks);
+          }
           xhat[o] = xh;
           if (vblock) vblock[o] = v;
           if (idx) idx[o] = (uint16_t)(int)ks;
@@ -400,8 +477,9 @@ __global__ void __launch_bounds__(ROW_THREADS)
   };
   using T_ = std::true_type;
   using F_ = std::false_type;
-  const float acc = anchored ? (c.precise ? weights(T_{}, T_{}) : weights(F_{}, T_{}))
-                             : (c.precise ? weights(T_{}, F_{}) : weights(F_{}, F_{}));
+  const bool pr = !GROUPED && c.precise;  // grouped rows choose the regime per group
+  const float acc = anchored ? (pr ? weights(T_{}, T_{}) : weights(F_{}, T_{}))
+                             : (pr ? weights(T_{}, F_{}) : weights(F_{}, F_{}));
   const double tot = block_sum((double)acc, ds);
   if (threadIdx.x == 0) vsum[row] = tot;
 }
@@ -797,10 +875,10 @@ __global__ void __launch_bounds__(ROW_THREADS)
 // after the last iteration (l2d and the denoiser's argmax only).
 constexpr int FUSED_MAX_THREADS = 1024;
 
-template <int MAP>
+template <int MAP, bool GROUPED>
 __global__ void __launch_bounds__(FUSED_MAX_THREADS)
     k_vamp_row_scalar(const float* __restrict__ W, const float* __restrict__ G,
-                      float* __restrict__ R2, int64_t n, int first, int full_rank,
+                      float* __restrict__ R2, int64_t n, int gsize, int first, int full_rank,
                       const double* __restrict__ coef, const double* __restrict__ kappa,
                       const double* __restrict__ gamma1, const float* __restrict__ scale,
                       const float* __restrict__ offset, int L, int anchored,
@@ -816,12 +894,20 @@ __global__ void __launch_bounds__(FUSED_MAX_THREADS)
   const int nn = (int)n;  // a row fits in shared memory: 32-bit in-row indices
   float* s_r = vrow;
   float* s_x = vrow + nn;
+  ScalarDen* s_den = reinterpret_cast<ScalarDen*>(vrow + 2 * nn);  // GROUPED: one per group
   const int64_t row = blockIdx.x;
   const float* Wr = W + row * n;
   const float* Gr = G + row * n;
   float* R2r = R2 + row * n;
-  const ScalarDen c = scalar_den_row(scale[row], offset[row], gamma1[row], L, anchored != 0,
-                                     anchored ? gamma1_0[row] : 0.0, inv_tau2);
+  const int ng = GROUPED ? nn / gsize : 1;
+  const ScalarDen c = scalar_den_row(scale[row * ng], offset[row * ng], gamma1[row], L,
+                                     anchored != 0, anchored ? gamma1_0[row] : 0.0, inv_tau2);
+  if (GROUPED) {
+    for (int g = threadIdx.x; g < ng; g += blockDim.x)
+      s_den[g] = scalar_den_row(scale[row * ng + g], offset[row * ng + g], gamma1[row], L,
+                                anchored != 0, anchored ? gamma1_0[row] : 0.0, inv_tau2);
+    __syncthreads();
+  }
   const float lc = first ? 0.0f : (float)coef[row];
   const float lk = first ? 0.0f : (float)kappa[row];
   const int bs = blockDim.x;
@@ -834,8 +920,14 @@ __global__ void __launch_bounds__(FUSED_MAX_THREADS)
     float acc = 0.0f;
     auto one = [&](const int j, const float g, const float r2, const float w) {
       const float r1 = first ? w : full_rank ? fmaf(lc, g, fmaf(lk, w - r2, w)) : fmaf(lc, g, r2);
-      float xh, ks;
-      const float v = scalar_den_elem<PRECISE, ANCH>(c, r1, w, xh, ks);
+      float xh, ks, v;
+      if constexpr (GROUPED) {
+        const ScalarDen& cg = s_den[j / gsize];  // uniform over a warp (gsize % 32 == 0)
+        v = cg.precise ? scalar_den_elem<true, ANCH>(cg, r1, w, xh, ks)
+                       : scalar_den_elem<false, ANCH>(cg, r1, w, xh, ks);
+      } else {
+        v = scalar_den_elem<PRECISE, ANCH>(c, r1, w, xh, ks);
+      }
       if (MAP) {
         idx[row * n + j] = (uint16_t)(int)ks;
       } else {
@@ -862,8 +954,9 @@ __global__ void __launch_bounds__(FUSED_MAX_THREADS)
   };
   using T_ = std::true_type;
   using F_ = std::false_type;
-  const float acc = anchored ? (c.precise ? pass1(T_{}, T_{}) : pass1(F_{}, T_{}))
-                             : (c.precise ? pass1(T_{}, F_{}) : pass1(F_{}, F_{}));
+  const bool pr = !GROUPED && c.precise;  // grouped rows choose the regime per group
+  const float acc = anchored ? (pr ? pass1(T_{}, T_{}) : pass1(F_{}, T_{}))
+                             : (pr ? pass1(T_{}, F_{}) : pass1(F_{}, F_{}));
   if (MAP) return;
   const double vsum = block_sum((double)acc, ds);  // its barriers also publish s_r, s_x
   if (threadIdx.x == 0)
@@ -907,14 +1000,16 @@ __global__ void __launch_bounds__(FUSED_MAX_THREADS)
 
 // --------------------------------------------------- residual / energies ---
 __global__ void __launch_bounds__(ROW_THREADS)
-    k_residual(const float* __restrict__ W, int64_t n, int d, const float* __restrict__ cb,
+    k_residual(const float* __restrict__ W, int64_t n, int d, int G, const float* __restrict__ cb,
                const float* __restrict__ scale, const float* __restrict__ offset,
                const uint16_t* __restrict__ idx, float* __restrict__ E,
                float* __restrict__ w_hat) {
   const int64_t row = blockIdx.x;
-  const float sc = scale[row], off = offset[row];
+  const int64_t ng = G ? n / G : 1;  // grids per row (G = 0: one)
   const int64_t B = n / d;
   for (int64_t j = threadIdx.x; j < n; j += blockDim.x) {
+    const int64_t gi = row * ng + (G ? j / G : 0);
+    const float sc = scale[gi], off = offset[gi];
     const int k = idx[row * B + j / d];  // in range: sanitised on entry
     const float c = (d == 1) ? (float)k : cb[(int64_t)k * d + (j % d)];
     const float wh = fmaf(sc, c, off);
@@ -925,17 +1020,20 @@ __global__ void __launch_bounds__(ROW_THREADS)
 
 // residual w - w_hat split for the tensor cores (K = n view), w_hat optional
 __global__ void __launch_bounds__(ROW_THREADS)
-    k_residual_split(const float* __restrict__ W, int64_t n, int d, const float* __restrict__ cb,
-                     const float* __restrict__ scale, const float* __restrict__ offset,
-                     const uint16_t* __restrict__ idx, float* __restrict__ w_hat,
-                     __half* __restrict__ ahi, __half* __restrict__ alo, int64_t lda, int64_t ldn,
+    k_residual_split(const float* __restrict__ W, int64_t n, int d, int G,
+                     const float* __restrict__ cb, const float* __restrict__ scale,
+                     const float* __restrict__ offset, const uint16_t* __restrict__ idx,
+                     float* __restrict__ w_hat, __half* __restrict__ ahi,
+                     __half* __restrict__ alo, int64_t lda, int64_t ldn,
                      float* __restrict__ a_unscale) {
   __shared__ float fs[33];
   const int64_t row = blockIdx.x;
-  const float sc = scale[row], off = offset[row];
+  const int64_t ng = G ? n / G : 1;  // grids per row (G = 0: one)
   const int64_t B = n / d;
   float mx = 0.0f;
   for (int64_t j = threadIdx.x; j < n; j += blockDim.x) {
+    const int64_t gi = row * ng + (G ? j / G : 0);
+    const float sc = scale[gi], off = offset[gi];
     const int k = idx[row * B + j / d];
     const float c = (d == 1) ? (float)k : cb[(int64_t)k * d + (j % d)];
     const float wh = fmaf(sc, c, off);
@@ -948,9 +1046,10 @@ __global__ void __launch_bounds__(ROW_THREADS)
   for (int64_t j = threadIdx.x; j < ldn; j += blockDim.x) {
     float x = 0.0f;
     if (j < n) {
+      const int64_t gi = row * ng + (G ? j / G : 0);
       const int k = idx[row * B + j / d];
       const float c = (d == 1) ? (float)k : cb[(int64_t)k * d + (j % d)];
-      x = (W[row * n + j] - fmaf(sc, c, off)) * down;
+      x = (W[row * n + j] - fmaf(scale[gi], c, offset[gi])) * down;
     }
     split_store(x, ahi, alo, row * lda + j);
   }
@@ -1003,8 +1102,13 @@ mpq_status launch_init(const mpq_plan_s* p, const float* W, int64_t m, int given
   if (p->d == 1) {
     {
       ProfScope ps_("k_init_scalar", st);
-      k_init_scalar<<<rows_grid(m), ROW_THREADS, 0, st>>>(W, p->n, p->K, given, scale, offset, idx,
-                                                          gamma1_0, p->status);
+      if (p->G)
+        k_init_scalar_groups<<<rows_grid(m), ROW_THREADS, 0, st>>>(W, p->n, p->K, p->G, given,
+                                                                   scale, offset, idx, gamma1_0,
+                                                                   p->status);
+      else
+        k_init_scalar<<<rows_grid(m), ROW_THREADS, 0, st>>>(W, p->n, p->K, given, scale, offset,
+                                                            idx, gamma1_0, p->status);
     }
     count_launch();
     return check_launch("k_init_scalar");
@@ -1056,9 +1160,18 @@ mpq_status launch_denoise(const mpq_plan_s* p, const float* R1, const double* ga
   if (p->d == 1) {
     {
       ProfScope ps_("k_denoise_scalar", st);
-      k_denoise_scalar<<<rows_grid(m), ROW_THREADS, 0, st>>>(R1, gamma1, scale, offset, p->n, p->K,
-                                                 anchored ? W : nullptr, gamma1_0, inv_tau2,
-                                                 xhat1, vblock, vsum, idx);
+      if (p->G) {
+        const size_t smem = sizeof(ScalarDen) * (size_t)(p->n / p->G);
+        MPQ_CUDA(cudaFuncSetAttribute(k_denoise_scalar<true>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+        k_denoise_scalar<true><<<rows_grid(m), ROW_THREADS, smem, st>>>(
+            R1, gamma1, scale, offset, p->n, p->K, p->G, anchored ? W : nullptr, gamma1_0,
+            inv_tau2, xhat1, vblock, vsum, idx);
+      } else {
+        k_denoise_scalar<false><<<rows_grid(m), ROW_THREADS, 0, st>>>(
+            R1, gamma1, scale, offset, p->n, p->K, 0, anchored ? W : nullptr, gamma1_0, inv_tau2,
+            xhat1, vblock, vsum, idx);
+      }
     }
     count_launch();
     return check_launch("k_denoise_scalar");
@@ -1159,8 +1272,9 @@ mpq_status launch_extrinsic_l2d(const mpq_plan_s* p, const float* W, int64_t m, 
 
 // Threads per row of the fused scalar kernel: its shared memory holds two
 // floats per weight; 0 when the row does not fit (the separate kernels run).
-int vamp_row_threads(int64_t n) {
-  const int64_t bytes = 8 * n;
+// (plus the per-group denoiser constants with group-wise grids)
+int vamp_row_threads(int64_t n, int G) {
+  const int64_t bytes = 8 * n + (G ? (n / G) * (int64_t)sizeof(ScalarDen) : 0);
   if (bytes <= 56 * 1024) return 256;    // 4 CTAs per SM
   if (bytes <= 112 * 1024) return 512;   // 2 CTAs per SM
   if (bytes <= 220 * 1024) return 1024;  // 1 CTA per SM
@@ -1173,22 +1287,24 @@ mpq_status launch_vamp_row_scalar(const mpq_plan_s* p, const float* W, int64_t m
                                   const float* offset, const double* gamma1_0, SplitOperand* As,
                                   double* gamma2, int32_t* clamps, uint16_t* idx, cudaStream_t st) {
   if (m <= 0) return MPQ_OK;
-  const int threads = vamp_row_threads(p->n);
+  const int threads = vamp_row_threads(p->n, p->G);
   if (p->d != 1 || threads == 0) return fail(MPQ_ERR_INVALID_ARG, "fused row kernel: d = 1 rows that fit");
   const mpq_params& q = p->params;
   const bool anchored = std::isfinite(q.tau);
   const double inv_tau2 = anchored ? 1.0 / (q.tau * q.tau) : 0.0;
-  const size_t smem = sizeof(float) * 2 * p->n;
-  using Kern = void (*)(const float*, const float*, float*, int64_t, int, int, const double*,
+  const size_t smem =
+      sizeof(float) * 2 * p->n + (p->G ? sizeof(ScalarDen) * (size_t)(p->n / p->G) : 0);
+  using Kern = void (*)(const float*, const float*, float*, int64_t, int, int, int, const double*,
                         const double*, const double*, const float*, const float*, int, int,
                         const double*, double, double, double, double, double, __half*, __half*,
                         int64_t, int64_t, float*, double*, int32_t*, uint16_t*);
-  const Kern kern = map ? k_vamp_row_scalar<1> : k_vamp_row_scalar<0>;
+  const Kern kern = p->G ? (map ? k_vamp_row_scalar<1, true> : k_vamp_row_scalar<0, true>)
+                         : (map ? k_vamp_row_scalar<1, false> : k_vamp_row_scalar<0, false>);
   MPQ_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   {
     ProfScope ps_(map ? "k_vamp_row_scalar(map)" : "k_vamp_row_scalar", st);
     kern<<<rows_grid(m), threads, smem, st>>>(
-        W, G, R2, p->n, first, p->r == p->n ? 1 : 0, coef, kappa, gamma1, scale, offset, p->K,
+        W, G, R2, p->n, p->G, first, p->r == p->n ? 1 : 0, coef, kappa, gamma1, scale, offset, p->K,
         anchored ? 1 : 0, gamma1_0, inv_tau2, q.gamma_lo_rel, q.gamma_hi_rel, q.alpha_min,
         q.alpha_max, As ? As->hi : nullptr, As ? As->lo : nullptr, As ? As->ld : 0,
         round_up(p->n, 64), As ? As->row_unscale : nullptr, gamma2, clamps, idx);
@@ -1203,7 +1319,7 @@ mpq_status launch_residual_split(const mpq_plan_s* p, const float* W, int64_t m,
   if (m <= 0) return MPQ_OK;
   {
     ProfScope ps_("k_residual_split", st);
-    k_residual_split<<<rows_grid(m), ROW_THREADS, 0, st>>>(W, p->n, p->d, p->cb, scale, offset,
+    k_residual_split<<<rows_grid(m), ROW_THREADS, 0, st>>>(W, p->n, p->d, p->G, p->cb, scale, offset,
                                                            idx, w_hat, As->hi, As->lo, As->ld,
                                                            round_up(p->n, 64), As->row_unscale);
   }
@@ -1217,7 +1333,7 @@ mpq_status launch_residual(const mpq_plan_s* p, const float* W, int64_t m, const
   if (m <= 0) return MPQ_OK;
   {
     ProfScope ps_("k_residual", st);
-    k_residual<<<rows_grid(m), ROW_THREADS, 0, st>>>(W, p->n, p->d, p->cb, scale, offset, idx, E,
+    k_residual<<<rows_grid(m), ROW_THREADS, 0, st>>>(W, p->n, p->d, p->G, p->cb, scale, offset, idx, E,
                                                      w_hat);
   }
   count_launch();

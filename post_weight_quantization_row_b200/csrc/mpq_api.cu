@@ -133,6 +133,10 @@ mpq_status validate_params(const mpq_params* q, int64_t n) {
     return fail(MPQ_ERR_INVALID_ARG, "cd_panel must be 0 or a positive multiple of 128");
   if (q->solve_graphs != 0 && q->solve_graphs != 1)
     return fail(MPQ_ERR_INVALID_ARG, "solve_graphs must be 0 or 1");
+  if (q->group_size < 0 || (q->group_size > 0 && (q->d != 1 || q->group_size % 128 ||
+                                                   n % q->group_size)))
+    return fail(MPQ_ERR_INVALID_ARG,
+                "group_size must be 0, or for d = 1 a multiple of 128 that divides n");
   if (!(q->beta0 > 0.0) || !isfinite(q->beta0)) return fail(MPQ_ERR_INVALID_ARG, "beta0 must be > 0");
   if (!(q->damping >= 0.0 && q->damping <= 1.0)) return fail(MPQ_ERR_INVALID_ARG, "damping must be in [0,1]");
   if (!(q->tau > 0.0)) return fail(MPQ_ERR_INVALID_ARG, "tau must be > 0 (INFINITY = uniform prior)");
@@ -191,7 +195,7 @@ void free_workspace(Workspace& w) {
   dfree(w.tile_count);
   dfree(w.Hg);
   dfree(w.Hl);
-  dfree(w.scale); dfree(w.offset); dfree(w.gamma1); dfree(w.gamma1_0); dfree(w.gamma2);
+  dfree(w.scale); dfree(w.offset); dfree(w.sref); dfree(w.gamma1); dfree(w.gamma1_0); dfree(w.gamma2);
   dfree(w.beta); dfree(w.vsum); dfree(w.coef); dfree(w.kappa); dfree(w.clamps); dfree(w.W); dfree(w.w_hat);
   dfree(w.energy); dfree(w.idx_stage);
   w.rows = 0;
@@ -203,7 +207,7 @@ constexpr int MAX_SWEEPS = 64;
 int64_t ws_bytes_per_row(const mpq_plan_s* p) {
   return 3 * p->n * 4 + round_up(p->n, 32) * 4 + p->r * 4 +
          4 * round_up(std::max(p->n, p->r), CD_TILE) + p->B * 2 + 3 * 4 +
-         8 * 8 + 4 + MAX_SWEEPS * 4 + (p->d == 8 ? CD_TILE * 4 : 0);
+         8 * 8 + 4 + MAX_SWEEPS * 4 + (p->d == 8 ? CD_TILE * 4 : 0) + 8 * (p->ng - 1) + 4;
 }
 
 // changes buffer rides in the tail of `clamps`: rows x (1 + MAX_SWEEPS) ints
@@ -241,7 +245,8 @@ mpq_status ensure_workspace(mpq_plan_s* p, int64_t rows) {
   if (st == MPQ_OK)
     chk(make_tmap_f16(&w.tm_ar_lo, w.As.lo, round_up(p->r, 64), w.As.rows_pad, w.As.ld, 128));
   chk(dalloc(&w.P, rows * p->r)); chk(dalloc(&w.idx, rows * p->B));
-  chk(dalloc(&w.scale, rows)); chk(dalloc(&w.offset, rows));
+  chk(dalloc(&w.scale, rows * p->ng)); chk(dalloc(&w.offset, rows * p->ng));
+  chk(dalloc(&w.sref, rows));
   chk(dalloc(&w.gamma1, rows)); chk(dalloc(&w.gamma1_0, rows)); chk(dalloc(&w.gamma2, rows));
   chk(dalloc(&w.beta, rows)); chk(dalloc(&w.vsum, rows)); chk(dalloc(&w.coef, rows));
   chk(dalloc(&w.kappa, rows));
@@ -350,8 +355,11 @@ mpq_status solve_batch(mpq_plan_s* p, const SolveIO& io, int64_t row0, int64_t m
   uint16_t* idx = io.idx + row0 * B;
   const int given = io.row_scale != nullptr;
   if (given) {
-    MPQ_CUDA(cudaMemcpyAsync(w.scale, io.row_scale + row0, sizeof(float) * mb, cudaMemcpyDeviceToDevice, st));
-    MPQ_CUDA(cudaMemcpyAsync(w.offset, io.row_offset + row0, sizeof(float) * mb, cudaMemcpyDeviceToDevice, st));
+    const int64_t ng = p->ng;
+    MPQ_CUDA(cudaMemcpyAsync(w.scale, io.row_scale + row0 * ng, sizeof(float) * mb * ng,
+                             cudaMemcpyDeviceToDevice, st));
+    MPQ_CUDA(cudaMemcpyAsync(w.offset, io.row_offset + row0 * ng, sizeof(float) * mb * ng,
+                             cudaMemcpyDeviceToDevice, st));
   }
   int32_t* clamps = w.clamps;
   int32_t* changes = w.clamps + w.rows;  // rows x MAX_SWEEPS
@@ -360,7 +368,7 @@ mpq_status solve_batch(mpq_plan_s* p, const SolveIO& io, int64_t row0, int64_t m
   MPQ_TRY(launch_init(p, W, mb, given, w.scale, w.offset, idx, w.gamma1_0, st));
   MPQ_CUDA(cudaMemcpyAsync(w.gamma1, w.gamma1_0, sizeof(double) * mb, cudaMemcpyDeviceToDevice, st));
   MPQ_TRY(fill_f64(w.beta, mb, p->params.beta0, st));
-  if (p->d == 1 && vamp_row_threads(n) > 0) {
+  if (p->d == 1 && vamp_row_threads(n, p->G) > 0) {
     // scalar rows: l2d, denoiser and d2l of an iteration in one fused row
     // kernel (r1 never leaves the chip), then the linear module
     for (int t = 0; t < io.T_vamp; ++t) {
@@ -553,6 +561,8 @@ mpq_status new_plan(const mpq_params* params, int64_t n, mpq_plan_s** out) {
   p->d = params->d;
   p->K = params->K;
   p->B = n / params->d;
+  p->G = params->group_size;
+  p->ng = p->G ? n / p->G : 1;
   if (p->d == 8) {
     mpq_status st = dalloc(&p->cb, (int64_t)p->K * 8);
     if (st == MPQ_OK) {
@@ -604,6 +614,7 @@ void mpq_params_default(mpq_params* p, int32_t d, int32_t K) {
   p->alpha_max = 0.99;
   p->vec_engine = 0;
   p->cd_panel = 0;
+  p->group_size = 0;
   p->solve_graphs = 1;
 }
 

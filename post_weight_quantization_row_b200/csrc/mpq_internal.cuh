@@ -76,6 +76,7 @@ struct Workspace {
   int64_t ldh = 0;
   CUtensorMap tm_hg;               // reduce-add target of the CD updates
   float* Hl = nullptr;             // d = 8 CD: rows x CD_TILE tile-local gradient
+  float* sref = nullptr;           // grouped CD: per-row reference scale of Delta
   // m x r fp32
   float* P = nullptr;
   // m x B
@@ -105,6 +106,8 @@ struct mpq_plan_s {
   int64_t n = 0, r = 0;
   int32_t d = 1, K = 2;
   int64_t B = 0;
+  int G = 0;        // scalar grid group size (columns); 0: one grid per row
+  int64_t ng = 1;   // grids per row
   mpq_params params{};
   // spectrum
   double* s64 = nullptr;   // r
@@ -175,7 +178,7 @@ mpq_status launch_linear_rows(const mpq_plan_s* p, int64_t m, const float* P,
                               double* gamma1_out, double* coef, double* kappa, double* alpha2,
                               double* beta_hat, int32_t* clamps, float* Uprime, SplitOperand* As,
                               cudaStream_t st);
-int vamp_row_threads(int64_t n);  // 0: the fused scalar row kernel does not apply
+int vamp_row_threads(int64_t n, int G);  // 0: the fused scalar row kernel does not apply
 mpq_status launch_vamp_row_scalar(const mpq_plan_s* p, const float* W, int64_t m, int first,
                                   int map, const float* G, float* R2, const double* coef,
                                   const double* kappa, const double* gamma1, const float* scale,
@@ -212,6 +215,7 @@ constexpr int CD_TILE = 128;  // columns per scalar CD tile (multiple of 64)
 constexpr int64_t CD_PANEL_BYTES = 32ll << 20;  // L2-resident slab of the CD gradient
 constexpr int64_t CD_PANEL_MIN = 512;           // narrowest CD panel (columns)
 int64_t cd_panel_cols(int64_t m, int64_t n);
+mpq_status launch_row_max(const float* scale, int64_t m, int64_t ng, float* out, cudaStream_t st);
 mpq_status launch_check_finite(const float* x, int64_t count, int* status, cudaStream_t st);
 
 // tensor-core GEMM (gemm_tc.cu): C = diag(A.row_unscale) (A B^T) * b_scale

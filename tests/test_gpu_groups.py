@@ -1,0 +1,121 @@
+"""Group-wise scalar grids (mpq_params.group_size = 128: one min-max grid per
+group of 128 consecutive columns of a row, the MPQ note's experimental
+setting) against the oracle on identical inputs: init exactly, the denoiser
+at the stage bar in every precision regime, CD indices exactly outside ties
+(with several panels, so that Delta carries the group scales through the
+panel GEMM), and the whole solve."""
+import numpy as np
+import pytest
+import torch
+
+import mpq_inputs as mi
+from oracle import mpq_oracle as orc
+from tests.helpers import (ENERGY_TOL, assert_rows_close, assert_scalars_close, cu, host, idx_np,
+                           injected_state, spectrum_cuda)
+
+pytestmark = pytest.mark.gpu
+
+G = 128
+LOGIT_TIE = 1e-3
+
+
+@pytest.fixture(scope="module")
+def mpq():
+    import post_weight_quantization_row_b200 as m
+    return m
+
+
+def case(seed, m_out=20, n=640, m=900, L=8):
+    return mi.small_problem(seed, m_out, n, m, d=1, levels=L, T_vamp=4, cd_sweeps=3)
+
+
+def plan_for(mpq, p, **kw):
+    _, _, s_cu, V_cu = spectrum_cuda(p.X)
+    return mpq.Plan.from_spectrum(s_cu, V_cu, 1, p.levels, group_size=G, **kw)
+
+
+def grid_f32(p):
+    sc, off = orc.minmax_grid(p.W, p.levels, G)
+    return sc.astype(np.float32), off.astype(np.float32)
+
+
+def test_init_grouped_grid(mpq):
+    p = case(801)
+    plan = plan_for(mpq, p)
+    out = plan.stage_init(cu(p.W))
+    sc, off = grid_f32(p)
+    assert host(out["scale"]).shape == (p.m_out, p.n // G)
+    assert np.array_equal(host(out["scale"]), sc)
+    assert np.array_equal(host(out["offset"]), off)
+    cb = orc.scalar_levels(p.levels)
+    st = orc.init(p.W, cb, sc.astype(np.float64), off.astype(np.float64))
+    t = (p.W - np.repeat(off, G, axis=1)) / np.repeat(sc, G, axis=1)
+    tie = np.abs(t - np.floor(t) - 0.5) < 1e-5
+    assert np.array_equal(idx_np(out["idx"])[~tie], st.idx_rtn[~tie])
+    assert_scalars_close("gamma1_0", host(out["gamma1_0"]), st.gamma1, 1e-5)
+
+
+@pytest.mark.parametrize("g_lo,g_hi", [(1.0, 40.0), (0.05, 0.5), (100.0, 1e4)])
+def test_denoise_grouped(mpq, g_lo, g_hi):
+    p = case(802)
+    plan = plan_for(mpq, p)
+    sc, off = grid_f32(p)
+    s, _ = orc.spectrum(p.X)
+    # the precision is per row; the groups' scales make gamma1 s^2 (and with
+    # it the precision regime) differ from group to group
+    R1, g1, _, _, _, _ = injected_state(11, p.W, sc.mean(axis=1), s, g_lo, g_hi)
+    ref = orc.denoise(R1, g1, orc.scalar_levels(p.levels), sc.astype(np.float64),
+                      off.astype(np.float64))
+    out = plan.stage_denoise(cu(R1), cu(g1, torch.float64), cu(sc), cu(off))
+    assert_rows_close("xhat1", host(out["xhat"]), ref.xhat)
+    assert_rows_close("vblock", host(out["vblock"]), ref.vblock)
+    assert_scalars_close("vsum", host(out["vsum"]), ref.vsum)
+    ok = ref.gap > LOGIT_TIE
+    assert np.array_equal(idx_np(out["idx"])[ok], ref.idx[ok])
+
+
+def test_cd_grouped_several_panels(mpq):
+    p = case(803, m_out=24, n=512, m=700)
+    plan = plan_for(mpq, p, cd_panel=256)
+    sc, off = grid_f32(p)
+    cb = orc.scalar_levels(p.levels)
+    s, V = orc.spectrum(p.X)
+    st = orc.init(p.W, cb, sc.astype(np.float64), off.astype(np.float64))
+    ref = orc.cd(p.W, st.idx_rtn, cb, sc.astype(np.float64), off.astype(np.float64),
+                 orc.hessian(s, V), 3)
+    out = plan.stage_cd(cu(p.W), cu(sc), cu(off),
+                        cu(st.idx_rtn.astype(np.uint16).view(np.int16), torch.int16), 3)
+    got = idx_np(out["idx"])
+    clean = ref.first_tie < 0
+    assert clean.mean() >= 0.25
+    assert np.array_equal(got[clean], ref.idx[clean])
+    assert np.array_equal(host(out["changes"])[clean], ref.changes[clean])
+    assert (ref.changes[clean, 1] > 0).any()
+    e_gpu = orc.energy(p.W, orc.decode(got, cb, sc.astype(np.float64), off.astype(np.float64)), s, V)
+    e_ref = orc.energy(p.W, ref.x, s, V)
+    assert np.all(np.abs(e_gpu - e_ref) <= ENERGY_TOL * e_ref)
+
+
+def test_solve_grouped(mpq):
+    p = case(804, m_out=24, n=384, m=600)
+    plan = plan_for(mpq, p)
+    sc, off = grid_f32(p)
+    cb = orc.scalar_levels(p.levels)
+    s, V = orc.spectrum(p.X)
+    ref = orc.solve(p.W, cb, s, V, p.T_vamp, p.cd_sweeps, sc.astype(np.float64),
+                    off.astype(np.float64))
+    out = plan.solve(cu(p.W), p.T_vamp, p.cd_sweeps, row_scale=cu(sc), row_offset=cu(off),
+                     stats=True)
+    got = idx_np(out["idx"])
+    e_gpu = host(out["energy"]).astype(np.float64)
+    clean = np.all(ref.map_gap > 1e-4, axis=1) & (ref.cd.first_tie < 0)
+    assert clean.mean() >= 0.25
+    assert np.array_equal(got[clean], ref.idx[clean])
+    assert np.all(np.abs(e_gpu[clean] - ref.energy[clean]) <= ENERGY_TOL * ref.energy[clean])
+    assert abs(e_gpu.sum() - ref.energy.sum()) <= ENERGY_TOL * ref.energy.sum()
+    # the library's own grid (no row_scale given) is the same grid
+    own = plan.solve(cu(p.W), p.T_vamp, p.cd_sweeps)
+    assert abs(host(own["energy"]).astype(np.float64).sum() - e_gpu.sum()) <= ENERGY_TOL * e_gpu.sum()
+    # and group-wise grids fit the rows better than one grid per row
+    per_row = orc.solve(p.W, cb, s, V, p.T_vamp, p.cd_sweeps)
+    assert e_gpu.sum() < per_row.energy.sum()
