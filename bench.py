@@ -56,6 +56,9 @@ def parse():
                          "the line then names the reduced workload)")
     ap.add_argument("--cd-panel", type=int, default=0,
                     help="columns per CD panel (multiple of 128; 0 = automatic)")
+    ap.add_argument("--group-size", type=int, default=0,
+                    help="scalar workloads: one min-max grid per group of this many columns "
+                         "(0 = one per row)")
     ap.add_argument("--spectrum-cache", default=None,
                     help="npz file: reuse the spectrum a previous run computed on the device")
     return ap.parse_args()
@@ -246,10 +249,11 @@ def workload(cfg, rank=0):
     return p
 
 
-def describe(p, cfg):
+def describe(p, cfg, group=0):
     bits = {8: 3, 16: 4}.get(p.levels, None) if p.d == 1 else 2
+    grid = f"group-{group}" if group else "per-row"
     return {"workload": f"{cfg}: W {p.m_out}x{p.n}, X {p.X.shape[0]}x{p.n}, "
-                        + (f"{bits}-bit per-row min-max grid" if p.d == 1 else
+                        + (f"{bits}-bit {grid} min-max grid" if p.d == 1 else
                            f"offset-E8 d=8 K={p.levels}, RHT")
                         + f", T_vamp={p.T_vamp}, CD sweeps<={p.cd_sweeps}",
             "m_out": p.m_out, "n": p.n, "m_calib": int(p.X.shape[0]), "d": p.d,
@@ -257,7 +261,7 @@ def describe(p, cfg):
             "seeds": p.seeds, "l2": "flushed between timed steps (512 MiB write)"}
 
 
-def oracle_sample(p, rows, steps=1):
+def oracle_sample(p, rows, steps=1, group=0):
     """Time the float64 oracle on `rows` rows of the layer (spectrum excluded)."""
     from oracle import mpq_oracle as orc
     t0 = time.time()
@@ -268,7 +272,7 @@ def oracle_sample(p, rows, steps=1):
     for k in range(steps):
         sel = slice((k * rows) % p.m_out, (k * rows) % p.m_out + rows)
         t0 = time.perf_counter()
-        orc.solve(p.W[sel], cb, s, V, p.T_vamp, p.cd_sweeps)
+        orc.solve(p.W[sel], cb, s, V, p.T_vamp, p.cd_sweeps, group=group)
         times.append(time.perf_counter() - t0)
     return times, t_spec
 
@@ -280,12 +284,12 @@ def run_reference(args, world, rank):
         return
     p = workload(args.config)
     rows = max(1, args.cpu_rows // 2)
-    times, t_spec = oracle_sample(p, rows, args.warmup + args.steps)
+    times, t_spec = oracle_sample(p, rows, args.warmup + args.steps, args.group_size)
     timed = times[args.warmup:]
     sec = sum(timed) / len(timed)
     value = rows * p.n / sec
     cores = len(os.sched_getaffinity(0))
-    cfgd = describe(p, args.config)
+    cfgd = describe(p, args.config, args.group_size)
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
@@ -310,7 +314,7 @@ def run_mpq(args, world, rank, local):
     p = workload(args.config, rank)
     if args.rows:
         p.W = np.ascontiguousarray(p.W[:args.rows])
-    cfgd = describe(p, args.config)
+    cfgd = describe(p, args.config, args.group_size)
     cfgd["cd_panel"] = args.cd_panel or "auto"
     m, n = p.m_out, p.n
     cb = p.codebook if p.d == 8 else None
@@ -319,13 +323,14 @@ def run_mpq(args, world, rank, local):
         z = np.load(cache)
         plan = mpq.Plan.from_spectrum(torch.from_numpy(z["s"]).to(dev),
                                       torch.from_numpy(z["V"]).to(dev), p.d, p.levels, codebook=cb,
-                                      cd_panel=args.cd_panel)
+                                      cd_panel=args.cd_panel, group_size=args.group_size)
         setup_s = None
     else:
         X = torch.from_numpy(p.X).to(dev)
         torch.cuda.synchronize()
         t0 = time.time()
-        plan = mpq.Plan.from_x(X, p.d, p.levels, codebook=cb, cd_panel=args.cd_panel)
+        plan = mpq.Plan.from_x(X, p.d, p.levels, codebook=cb, cd_panel=args.cd_panel,
+                               group_size=args.group_size)
         torch.cuda.synchronize()
         setup_s = time.time() - t0
         del X
@@ -460,7 +465,7 @@ def run_mpq(args, world, rank, local):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        times, t_spec = oracle_sample(p, args.cpu_rows)
+        times, t_spec = oracle_sample(p, args.cpu_rows, 1, args.group_size)
         cpu = {"value": args.cpu_rows * n / times[0], "unit": UNIT,
                "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
                "sample": f"rows 0..{args.cpu_rows - 1} of the layer (independent problems), "
