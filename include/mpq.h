@@ -118,6 +118,13 @@ typedef struct {
                              0: every call launches its kernels directly.  Calls
                              made while the per-kernel profiler runs always
                              launch directly. */
+  double cd_skip_precision;  /* adaptive CD: 0 (default) every row runs CD; > 0:
+                             in mpq_solve / mpq_solve_host, rows whose terminal
+                             VAMP precision gamma1 s^2 exceeds this (s the row's
+                             scale, its largest group scale with group-wise
+                             grids) skip CD and keep the marginal MAP; their
+                             cd_changes are 0.  The stage hook mpq_stage_cd
+                             always runs CD. */
 } mpq_params;
 
 /* Fill `p` with the defaults above for block size d and codebook size K. */

@@ -445,12 +445,24 @@ class SolveOut:
     trace: list = field(default_factory=list)
 
 
+def terminal_precision(gamma1, scale):
+    """Terminal VAMP precision in grid units, gamma1 s^2, with s the row's
+    scale (its largest group scale with group-wise grids)."""
+    s = np.asarray(scale, np.float64)
+    s = s if s.ndim == 1 else s.max(axis=1)
+    return np.asarray(gamma1, np.float64) * s * s
+
+
 def solve(W, codebook, s, V, T_vamp: int, cd_sweeps: int, scale=None, offset=None,
           beta0: float = 1.0, damping: float = 0.5, tau: float = math.inf,
-          keep_trace: bool = False, group: int = 0) -> SolveOut:
+          keep_trace: bool = False, group: int = 0, cd_skip_precision: float = 0.0) -> SolveOut:
     """The MPQ solve of every row ([MPQ-note] flowchart and Overall
     framework): init -> T_vamp x (denoiser -> extrinsic -> linear module ->
-    M-step) -> marginal MAP argmax -> exact block CD -> energies."""
+    M-step) -> marginal MAP argmax -> exact block CD -> energies.
+    With ``cd_skip_precision`` > 0, rows whose terminal precision (see
+    terminal_precision) exceeds it keep the marginal MAP and run no CD: the
+    [MPQ-note] diagnostics report terminal precisions near 1e5 at 3-bit
+    scalar with CD changing almost no block (reading R13)."""
     W = np.asarray(W, np.float64)
     st = init(W, codebook, scale, offset, beta0, group)
     g10 = st.gamma1.copy()
@@ -473,6 +485,13 @@ def solve(W, codebook, s, V, T_vamp: int, cd_sweeps: int, scale=None, offset=Non
         H = hessian(s, V)
         cdo = cd(W, idx_map, codebook, st.scale, st.offset, H, cd_sweeps)
         idx = cdo.idx
+        if cd_skip_precision > 0:
+            skip = terminal_precision(g1, st.scale) > cd_skip_precision
+            idx = np.where(skip[:, None], idx_map, cdo.idx)
+            cdo.idx = idx
+            cdo.changes[skip] = 0
+            cdo.first_tie[skip] = -1
+            cdo.x = decode(idx, codebook, st.scale, st.offset)
     w_hat = decode(idx, codebook, st.scale, st.offset)
     E = energy(W, w_hat, s, V)
     return SolveOut(idx, w_hat, E, idx_map, dn.gap, g1, beta, clamps, cdo, trace)

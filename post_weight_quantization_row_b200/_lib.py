@@ -43,7 +43,8 @@ class Params(C.Structure):
                 ("gamma_lo_rel", C.c_double), ("gamma_hi_rel", C.c_double),
                 ("alpha_min", C.c_double), ("alpha_max", C.c_double),
                 ("vec_engine", C.c_int32), ("cd_panel", C.c_int32),
-                ("group_size", C.c_int32), ("solve_graphs", C.c_int32)]
+                ("group_size", C.c_int32), ("solve_graphs", C.c_int32),
+                ("cd_skip_precision", C.c_double)]
 
 
 class RowStats(C.Structure):

@@ -77,7 +77,8 @@ __global__ void __launch_bounds__(CD1_WARPS * 32, 2)
                      int sweeps, int sw,
                      int32_t* __restrict__ changes, __half* __restrict__ dhi,
                      __half* __restrict__ dlo, int64_t lda, float* __restrict__ d_unscale,
-                     int* __restrict__ tile_flag, int* __restrict__ panel_flag) {
+                     int* __restrict__ tile_flag, int* __restrict__ panel_flag,
+                     const int32_t* __restrict__ skip) {
   extern __shared__ float cd_smem[];
   float* sH = cd_smem;                   // H[tile, tile], zero outside tw x tw
   float* s_rg = sH + CD_TILE * CD_TILE;  // 1 / H_jj (0 where H_jj <= 0)
@@ -103,8 +104,9 @@ __global__ void __launch_bounds__(CD1_WARPS * 32, 2)
   const float dsc = sref ? sc / sref[row] : 1.0f;
   if (lane == 0) d_unscale[row] = sref ? -sref[row] : -sc;
   uint16_t* ir = idx + row * n + t0;
-  // a row stops after a sweep without change (its Delta row stays zero)
-  if (sw > 0 && changes[row * sweeps + sw - 1] == 0) {
+  // a row stops after a sweep without change, and a skipped row never starts
+  // (its Delta row stays zero)
+  if ((sw > 0 && changes[row * sweeps + sw - 1] == 0) || (skip && skip[row])) {
     for (int i = lane; i < CD_TILE; i += 32) {
       drow_hi[i] = __float2half_rn(0.0f);
       drow_lo[i] = __float2half_rn(0.0f);
@@ -213,9 +215,9 @@ constexpr int CD8_ROWS = 256;   // rows per eval CTA (8 warps x 4 groups of 8 ro
 constexpr int CD8_CHUNK = 1024; // codewords per eval CTA
 constexpr int CD8_APPLY_WARPS = 16;
 
-__device__ __forceinline__ bool row_active(const int32_t* changes, int64_t row, int sweeps,
-                                           int sw) {
-  return sw == 0 || changes[row * sweeps + sw - 1] > 0;
+__device__ __forceinline__ bool row_active(const int32_t* changes, const int32_t* skip,
+                                           int64_t row, int sweeps, int sw) {
+  return (sw == 0 || changes[row * sweeps + sw - 1] > 0) && !(skip && skip[row]);
 }
 
 // g' for one row at block b from the block's 8 gradient entries hb; G_b and
@@ -250,7 +252,8 @@ __global__ void __launch_bounds__(256)
                   const float* __restrict__ scale, const uint16_t* __restrict__ idx,
                   const float* __restrict__ h, int64_t ldh, const float* __restrict__ hl,
                   int sweeps, int sw, const int32_t* __restrict__ changes,
-                  float* __restrict__ part_val, int* __restrict__ part_idx, int nchunks) {
+                  const int32_t* __restrict__ skip, float* __restrict__ part_val,
+                  int* __restrict__ part_idx, int nchunks) {
   __shared__ float scb[8][CD8_CHUNK];  // transposed: lanes read consecutive codewords
   __shared__ float sq[CD8_CHUNK];
   __shared__ float sg[CD8_ROWS][8];
@@ -266,7 +269,7 @@ __global__ void __launch_bounds__(256)
   __syncthreads();
   for (int rl = threadIdx.x; rl < CD8_ROWS; rl += blockDim.x) {
     const int64_t row = r0 + rl;
-    const bool act = row < m && row_active(changes, row, sweeps, sw);
+    const bool act = row < m && row_active(changes, skip, row, sweeps, sw);
     if (act) {
       float g[8];
       block_gradient(H, n, block_h(h, ldh, hl, row, b, t0), cb, idx[row * B + b], scale[row], b, g);
@@ -345,7 +348,7 @@ __global__ void __launch_bounds__(CD8_APPLY_WARPS * 32)
                    const float* __restrict__ part_val, const int* __restrict__ part_idx,
                    int nchunks, __half* __restrict__ dhi, __half* __restrict__ dlo, int64_t lda,
                    float* __restrict__ d_unscale, int* __restrict__ tile_flag,
-                   int* __restrict__ panel_flag) {
+                   int* __restrict__ panel_flag, const int32_t* __restrict__ skip) {
   __shared__ float sHb[CD_TILE][8];  // H[tile, block b]
   const int64_t B = n / 8;
   const bool first = 8 * b == t0;
@@ -365,7 +368,7 @@ __global__ void __launch_bounds__(CD8_APPLY_WARPS * 32)
     }
     if (lane == 0) d_unscale[row] = -sc;
   }
-  if (!row_active(changes, row, sweeps, sw)) return;
+  if (!row_active(changes, skip, row, sweeps, sw)) return;
   // combine the chunk minima (lowest index on ties)
   float v = INFINITY;
   int k = 0x7fffffff;
@@ -436,7 +439,30 @@ __global__ void k_row_max(const float* __restrict__ scale, int64_t m, int64_t ng
   out[row] = mx;
 }
 
+// Adaptive CD: rows whose terminal precision gamma1 s^2 (s the row's scale,
+// its largest group scale with group-wise grids) exceeds the threshold skip
+// CD and keep the marginal MAP.
+__global__ void k_cd_skip(const double* __restrict__ gamma1, const float* __restrict__ scale,
+                          int64_t m, int64_t ng, double threshold, int32_t* __restrict__ skip) {
+  const int64_t row = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (row >= m) return;
+  float s = scale[row * ng];
+  for (int64_t g = 1; g < ng; ++g) s = fmaxf(s, scale[row * ng + g]);
+  skip[row] = gamma1[row] * (double)s * (double)s > threshold ? 1 : 0;
+}
+
 }  // namespace
+
+mpq_status launch_cd_skip(const double* gamma1, const float* scale, int64_t m, int64_t ng,
+                          double threshold, int32_t* skip, cudaStream_t st) {
+  if (m <= 0) return MPQ_OK;
+  {
+    ProfScope ps_("k_cd_skip", st);
+    k_cd_skip<<<(unsigned)cdiv(m, 256), 256, 0, st>>>(gamma1, scale, m, ng, threshold, skip);
+  }
+  count_launch();
+  return check_launch("k_cd_skip");
+}
 
 mpq_status launch_row_max(const float* scale, int64_t m, int64_t ng, float* out, cudaStream_t st) {
   if (m <= 0) return MPQ_OK;
@@ -459,7 +485,7 @@ int64_t cd_panel_cols(int64_t m, int64_t n) {
 
 mpq_status launch_cd(mpq_plan_s* p, const float* W, int64_t m, const float* scale,
                      const float* offset, uint16_t* idx, float* h, int64_t ldh, int32_t sweeps,
-                     int32_t* changes, cudaStream_t st) {
+                     int32_t* changes, cudaStream_t st, const int32_t* skip) {
   (void)W;
   (void)offset;
   if (m <= 0 || sweeps <= 0) return MPQ_OK;
@@ -532,7 +558,7 @@ mpq_status launch_cd(mpq_plan_s* p, const float* W, int64_t m, const float* scal
           k_cd_tile_decide<<<(unsigned)cdiv(m, CD1_WARPS), CD1_WARPS * 32, CD1_SMEM, st>>>(
               m, n, p->K, t0, tw, scale, (int)p->ng, p->G ? (int)(t0 / p->G) : 0,
               p->G ? w.sref : nullptr, p->H32, idx, h, ldh, sweeps, sw, changes, dhi, dlo,
-              w.As.ld, w.As.row_unscale, tflag, pflag);
+              w.As.ld, w.As.row_unscale, tflag, pflag, skip);
           count_launch();
           rc = check_launch("k_cd_tile_decide");
         } else {
@@ -545,15 +571,15 @@ mpq_status launch_cd(mpq_plan_s* p, const float* W, int64_t m, const float* scal
               dim3 ga((unsigned)nchunks, (unsigned)cdiv(m, CD8_ROWS));
               ProfScope ps_("k_cd_vec_eval", st);
               k_cd_vec_eval<<<ga, 256, 0, st>>>(m, n, p->K, b, t0, p->cb, p->qtab, p->H32, scale,
-                                                idx, h, ldh, hl, sweeps, sw, changes, part_val,
-                                                part_idx, nchunks);
+                                                idx, h, ldh, hl, sweeps, sw, changes, skip,
+                                                part_val, part_idx, nchunks);
             }
             {
               ProfScope ps_("k_cd_vec_apply", st);
               k_cd_vec_apply<<<(unsigned)cdiv(m, CD8_APPLY_WARPS), CD8_APPLY_WARPS * 32, 0, st>>>(
                   m, n, p->K, b, t0, tw, p->cb, p->qtab, p->H32, scale, idx, h, ldh, hl, sweeps,
                   sw, changes, part_val, part_idx, nchunks, dhi, dlo, w.As.ld, w.As.row_unscale,
-                  tflag, pflag);
+                  tflag, pflag, skip);
             }
             count_launch(tc ? 1 : 2);
             rc = check_launch("k_cd_vec");

@@ -133,6 +133,8 @@ mpq_status validate_params(const mpq_params* q, int64_t n) {
     return fail(MPQ_ERR_INVALID_ARG, "cd_panel must be 0 or a positive multiple of 128");
   if (q->solve_graphs != 0 && q->solve_graphs != 1)
     return fail(MPQ_ERR_INVALID_ARG, "solve_graphs must be 0 or 1");
+  if (!(q->cd_skip_precision >= 0.0))
+    return fail(MPQ_ERR_INVALID_ARG, "cd_skip_precision must be >= 0 (0: never skip)");
   if (q->group_size < 0 || (q->group_size > 0 && (q->d != 1 || q->group_size % 128 ||
                                                    n % q->group_size)))
     return fail(MPQ_ERR_INVALID_ARG,
@@ -195,7 +197,7 @@ void free_workspace(Workspace& w) {
   dfree(w.tile_count);
   dfree(w.Hg);
   dfree(w.Hl);
-  dfree(w.scale); dfree(w.offset); dfree(w.sref); dfree(w.gamma1); dfree(w.gamma1_0); dfree(w.gamma2);
+  dfree(w.scale); dfree(w.offset); dfree(w.sref); dfree(w.cd_skip); dfree(w.gamma1); dfree(w.gamma1_0); dfree(w.gamma2);
   dfree(w.beta); dfree(w.vsum); dfree(w.coef); dfree(w.kappa); dfree(w.clamps); dfree(w.W); dfree(w.w_hat);
   dfree(w.energy); dfree(w.idx_stage);
   w.rows = 0;
@@ -207,7 +209,7 @@ constexpr int MAX_SWEEPS = 64;
 int64_t ws_bytes_per_row(const mpq_plan_s* p) {
   return 3 * p->n * 4 + round_up(p->n, 32) * 4 + p->r * 4 +
          4 * round_up(std::max(p->n, p->r), CD_TILE) + p->B * 2 + 3 * 4 +
-         8 * 8 + 4 + MAX_SWEEPS * 4 + (p->d == 8 ? CD_TILE * 4 : 0) + 8 * (p->ng - 1) + 4;
+         8 * 8 + 4 + MAX_SWEEPS * 4 + (p->d == 8 ? CD_TILE * 4 : 0) + 8 * (p->ng - 1) + 8;
 }
 
 // changes buffer rides in the tail of `clamps`: rows x (1 + MAX_SWEEPS) ints
@@ -247,6 +249,7 @@ mpq_status ensure_workspace(mpq_plan_s* p, int64_t rows) {
   chk(dalloc(&w.P, rows * p->r)); chk(dalloc(&w.idx, rows * p->B));
   chk(dalloc(&w.scale, rows * p->ng)); chk(dalloc(&w.offset, rows * p->ng));
   chk(dalloc(&w.sref, rows));
+  chk(dalloc(&w.cd_skip, rows));
   chk(dalloc(&w.gamma1, rows)); chk(dalloc(&w.gamma1_0, rows)); chk(dalloc(&w.gamma2, rows));
   chk(dalloc(&w.beta, rows)); chk(dalloc(&w.vsum, rows)); chk(dalloc(&w.coef, rows));
   chk(dalloc(&w.kappa, rows));
@@ -324,14 +327,20 @@ mpq_status run_linear_core(mpq_plan_s* p, int64_t m, double* gamma2, const doubl
 
 mpq_status run_cd(mpq_plan_s* p, const float* W, int64_t m, const float* scale,
                   const float* offset, uint16_t* idx, int sweeps, int32_t* changes,
-                  cudaStream_t st) {
+                  cudaStream_t st, const double* gamma1 = nullptr) {
   Workspace& w = p->ws;
   const int64_t n = p->n;
   MPQ_TRY(launch_residual_split(p, W, m, scale, offset, idx, &w.As, nullptr, st));
   // h = H (w - x), in its own padded buffer (the CD updates reduce into it)
   MPQ_TRY(gemm_tc(w.As, w.tm_an_hi, w.tm_an_lo, p->H_s, p->tm_h_hi, p->tm_h_lo, w.Hg, w.ldh, m, n,
                   n, p->H_s.unscale_host, p->status, st, "gemm_hessian"));
-  return launch_cd(p, W, m, scale, offset, idx, w.Hg, w.ldh, sweeps, changes, st);
+  // adaptive CD (solve only: it needs the terminal precision)
+  const int32_t* skip = nullptr;
+  if (gamma1 && p->params.cd_skip_precision > 0.0) {
+    MPQ_TRY(launch_cd_skip(gamma1, scale, m, p->ng, p->params.cd_skip_precision, w.cd_skip, st));
+    skip = w.cd_skip;
+  }
+  return launch_cd(p, W, m, scale, offset, idx, w.Hg, w.ldh, sweeps, changes, st, skip);
 }
 
 mpq_status run_energy(mpq_plan_s* p, const float* W, int64_t m, const float* scale,
@@ -398,7 +407,8 @@ mpq_status solve_batch(mpq_plan_s* p, const SolveIO& io, int64_t row0, int64_t m
       MPQ_TRY(launch_denoise(p, R1, w.gamma1, w.scale, w.offset, mb, W, w.gamma1_0, w.X1, vblock,
                              w.vsum, idx, st));
   }
-  if (io.sweeps > 0) MPQ_TRY(run_cd(p, W, mb, w.scale, w.offset, idx, io.sweeps, changes, st));
+  if (io.sweeps > 0)
+    MPQ_TRY(run_cd(p, W, mb, w.scale, w.offset, idx, io.sweeps, changes, st, w.gamma1));
   MPQ_TRY(run_energy(p, W, mb, w.scale, w.offset, idx, io.w_hat ? io.w_hat + row0 * n : nullptr,
                      io.energy ? io.energy + row0 : nullptr, st));
   if (io.stats) {
@@ -616,6 +626,7 @@ void mpq_params_default(mpq_params* p, int32_t d, int32_t K) {
   p->cd_panel = 0;
   p->group_size = 0;
   p->solve_graphs = 1;
+  p->cd_skip_precision = 0.0;
 }
 
 mpq_status mpq_plan_create_from_spectrum(const double* s, const double* V, int64_t n, int64_t r,

@@ -77,6 +77,7 @@ struct Workspace {
   CUtensorMap tm_hg;               // reduce-add target of the CD updates
   float* Hl = nullptr;             // d = 8 CD: rows x CD_TILE tile-local gradient
   float* sref = nullptr;           // grouped CD: per-row reference scale of Delta
+  int32_t* cd_skip = nullptr;      // adaptive CD: rows that keep the marginal MAP
   // m x r fp32
   float* P = nullptr;
   // m x B
@@ -200,9 +201,12 @@ mpq_status launch_sanitize_idx(const mpq_plan_s* p, uint16_t* idx, int64_t count
 mpq_status launch_energy_rows(const mpq_plan_s* p, int64_t m, const float* P, float* energy,
                               cudaStream_t st);
 // CD sweeps; h (m x ldh) holds H (w - x) on entry and is updated in place
+// (rows with skip[row] != 0 run no CD; skip may be null)
 mpq_status launch_cd(mpq_plan_s* p, const float* W, int64_t m, const float* scale,
                      const float* offset, uint16_t* idx, float* h, int64_t ldh, int32_t sweeps,
-                     int32_t* changes, cudaStream_t st);
+                     int32_t* changes, cudaStream_t st, const int32_t* skip = nullptr);
+mpq_status launch_cd_skip(const double* gamma1, const float* scale, int64_t m, int64_t ng,
+                          double threshold, int32_t* skip, cudaStream_t st);
 // ceil(y) for |y| < 2^22 with one directed-rounding add: y + 1.5 2^23 rounded
 // up lands on the integer grid of [2^23, 2^24) (full-rate adds instead of a
 // rounding instruction).  Larger |y| keeps its sign, which is all the callers

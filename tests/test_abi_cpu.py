@@ -40,13 +40,14 @@ def test_params_default(mpq):
     assert math.isinf(p.tau) and p.gamma_lo_rel == 1e-10 and p.gamma_hi_rel == 1e10
     assert p.alpha_min == 1e-10 and p.alpha_max == 0.99
     assert p.vec_engine == 0 and p.cd_panel == 0 and p.solve_graphs == 1 and p.group_size == 0
+    assert p.cd_skip_precision == 0.0
 
 
 @pytest.mark.parametrize("field,value", [("d", 3), ("K", 1), ("damping", 1.5), ("beta0", -1.0),
                                          ("tau", 0.0), ("alpha_max", 1.0), ("vec_engine", 3),
                                          ("cd_panel", 100), ("cd_panel", -128),
                                          ("solve_graphs", 2), ("group_size", 100),
-                                         ("group_size", -128)])
+                                         ("group_size", -128), ("cd_skip_precision", -1.0)])
 def test_bad_params_rejected_without_a_device(mpq, field, value):
     p = mpq.Params()
     mpq.lib.mpq_params_default(C.byref(p), 1, 8)

@@ -119,3 +119,40 @@ def test_solve_grouped(mpq):
     # and group-wise grids fit the rows better than one grid per row
     per_row = orc.solve(p.W, cb, s, V, p.T_vamp, p.cd_sweeps)
     assert e_gpu.sum() < per_row.energy.sum()
+
+
+# ------------------------------------------------------------- adaptive CD ---
+
+@pytest.mark.parametrize("group", [0, G])
+def test_adaptive_cd_rows_follow_their_terminal_precision(mpq, group):
+    # rows whose terminal precision gamma1 s^2 exceeds the threshold keep the
+    # marginal MAP (as a solve without CD), the others run the full CD (as a
+    # solve without the threshold); the device decides from its own terminal
+    # gamma1, the oracle's decisions agree away from the threshold
+    p = case(805, m_out=32, n=384, m=600)
+    _, _, s_cu, V_cu = spectrum_cuda(p.X)
+    plans = {k: mpq.Plan.from_spectrum(s_cu, V_cu, 1, p.levels, group_size=group, **kw)
+             for k, kw in (("full", {}), ("skip", {"cd_skip_precision": 1.0}))}
+    W = cu(p.W)
+    full = plans["full"].solve(W, p.T_vamp, p.cd_sweeps, stats=True)
+    none = plans["full"].solve(W, p.T_vamp, 0, stats=True)
+    sc = host(plans["full"].stage_init(W)["scale"]).astype(np.float64)
+    smax = sc if sc.ndim == 1 else sc.max(axis=1)
+    prec = host(full["gamma1"]) * smax * smax
+    thr = float(np.median(prec))
+    pl = mpq.Plan.from_spectrum(s_cu, V_cu, 1, p.levels, group_size=group, cd_skip_precision=thr)
+    mix = pl.solve(W, p.T_vamp, p.cd_sweeps, stats=True)
+    skip = prec > thr
+    assert 0 < skip.sum() < p.m_out
+    got, g_full, g_none = idx_np(mix["idx"]), idx_np(full["idx"]), idx_np(none["idx"])
+    assert np.array_equal(got[skip], g_none[skip])
+    assert np.array_equal(got[~skip], g_full[~skip])
+    assert np.all(host(mix["cd_changes"])[skip] == 0)
+    # the oracle's decisions on the same threshold, away from it
+    cb = orc.scalar_levels(p.levels)
+    s, V = orc.spectrum(p.X)
+    ref = orc.solve(p.W, cb, s, V, p.T_vamp, p.cd_sweeps, group=group, cd_skip_precision=thr)
+    st = orc.init(p.W, cb, group=group)
+    prec_ref = orc.terminal_precision(ref.gamma1, st.scale)
+    far = np.abs(prec_ref / thr - 1.0) > 0.05
+    assert np.array_equal((prec_ref > thr)[far], skip[far])

@@ -107,3 +107,30 @@ def test_grouped_solve_runs_and_beats_round_to_nearest():
     # the grouped grid fits the row better than one grid for the whole row
     per_row = orc.solve(p.W, cb, s, V, 4, 3)
     assert out.energy.sum() < per_row.energy.sum()
+
+
+# ----------------------------------------------------------------------------
+# adaptive CD: rows above a terminal precision keep the marginal MAP
+# ----------------------------------------------------------------------------
+
+def test_cd_skip_precision_extremes():
+    p = mi.make_problem("tiny")
+    cb = orc.scalar_levels(p.levels)
+    s, V = orc.spectrum(p.X)
+    full = orc.solve(p.W, cb, s, V, 4, 3)
+    prec = orc.terminal_precision(full.gamma1, orc.init(p.W, cb).scale)
+    # a threshold above every row's precision changes nothing
+    hi = orc.solve(p.W, cb, s, V, 4, 3, cd_skip_precision=2 * prec.max())
+    assert np.array_equal(hi.idx, full.idx) and np.array_equal(hi.energy, full.energy)
+    # below every row's precision: no CD at all, the marginal MAP is the answer
+    lo = orc.solve(p.W, cb, s, V, 4, 3, cd_skip_precision=0.5 * prec.min())
+    none = orc.solve(p.W, cb, s, V, 4, 0)
+    assert np.array_equal(lo.idx, none.idx) and np.array_equal(lo.energy, none.energy)
+    assert np.all(lo.cd.changes == 0)
+    # in between: each row follows its own precision
+    mid = float(np.median(prec))
+    mix = orc.solve(p.W, cb, s, V, 4, 3, cd_skip_precision=mid)
+    skip = prec > mid
+    assert 0 < skip.sum() < p.m_out
+    assert np.array_equal(mix.idx[skip], none.idx[skip])
+    assert np.array_equal(mix.idx[~skip], full.idx[~skip])
