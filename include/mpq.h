@@ -17,7 +17,11 @@
  *                        G_b = T_b^T T_b;
  *   [Hyper-parameters]   (loss / training strategy section) T_vamp = 16,
  *                        rho_damp = 0.5, tau, S_CD = 3 with early stop,
- *                        gamma1_0 = 1/MSE(w, w_rtn), E8 d = 8, M_b = 2^16.
+ *                        gamma1_0 = 1/MSE(w, w_rtn), E8 d = 8, M_b = 2^16;
+ *   [Main experiments]   (key experimental data) calibration on 128 C4
+ *                        sequences of length 2048.
+ * [ai.info findings] is the ai.info page on the same paper, its list of
+ * findings (random Hadamard transforms and E_lin).
  * The min-max scalar grid follows the NeUQI note ("Near-Optimal Uniform
  * Quantization Parameter Initialization for Low-Bit LLMs"), existing pain
  * points section: s = (max - min)/(2^k - 1), z = -round(min/s).
@@ -55,6 +59,7 @@ extern "C" {
 #endif
 
 typedef struct mpq_plan_s* mpq_plan_t;
+typedef struct mpq_gram_s* mpq_gram_t;
 typedef void* mpq_stream_t; /* cudaStream_t */
 
 typedef enum {
@@ -149,6 +154,42 @@ MPQ_API mpq_status mpq_plan_create_from_spectrum(const double* s, const double* 
  * space r = rank(X)).  Synchronises `stream`.  MPQ_ERR_RANK if X == 0. */
 MPQ_API mpq_status mpq_plan_create_from_x(const float* X, int64_t m, int64_t n, const mpq_params* params,
                                   mpq_stream_t stream, mpq_plan_t* plan);
+
+/* ------------------------------------------------ streamed calibration --- */
+/* Calibration at scale ([Main experiments]: 128 sequences x 2048 tokens, so
+ * m = 262144 activation rows) does not fit one X matrix: stream it.  A gram
+ * handle owns G = sum_c X_c^T X_c (n x n, fp64, device); each chunk X_c
+ * (rows x n fp32, device, row-major) adds its products in fp64.  The plan
+ * built from it has the spectrum of X = [X_1; X_2; ...] through the right
+ * Gram (Jacobi eigenpairs of G, s = sqrt(lambda), V = eigenvectors) and the
+ * same rank cut as mpq_plan_create_from_x with m = the total row count.
+ *   create:     n in [1, 131072]; G = 0.  Synchronises `stream`.
+ *   accumulate: rows >= 0 (0 is a no-op); X is read, never kept; the call
+ *               synchronises `stream` before returning (it frees a fp64
+ *               rows x n staging copy).  Chunks may differ in row count.
+ *   info:       HOST outputs (either may be NULL): n and the rows so far.
+ *   get:        copy G out (device, n x n doubles, row-major).
+ *   create_from_gram: MPQ_ERR_RANK with no rows or G == 0; the gram stays
+ *               owned by the caller and may keep accumulating.
+ *   destroy:    NULL is a no-op. */
+MPQ_API mpq_status mpq_gram_create(int64_t n, mpq_stream_t stream, mpq_gram_t* gram);
+MPQ_API mpq_status mpq_gram_accumulate(mpq_gram_t gram, const float* X, int64_t rows, mpq_stream_t stream);
+MPQ_API mpq_status mpq_gram_info(mpq_gram_t gram, int64_t* n, int64_t* rows);
+MPQ_API mpq_status mpq_gram_get(mpq_gram_t gram, double* G, mpq_stream_t stream);
+MPQ_API mpq_status mpq_gram_destroy(mpq_gram_t gram);
+MPQ_API mpq_status mpq_plan_create_from_gram(mpq_gram_t gram, const mpq_params* params,
+                                             mpq_stream_t stream, mpq_plan_t* plan);
+
+/* Random Hadamard rotation, in place, on the device (incoherence
+ * preprocessing; [ai.info findings]: the rotation leaves E_lin unchanged, as
+ * E_lin sees the Hessian only through its eigenvalues).  Every row x of X
+ * (rows x n fp32, row-major, device) becomes x Q^T, Q = H_n diag(signs) /
+ * sqrt(n) with H_n the Sylvester-Hadamard matrix; apply it to both W and X
+ * and the objective ||(W - W_hat) X^T||^2 is unchanged.  signs: n floats,
+ * each +1 or -1 (device).  n a power of two in [1, MPQ_RHT_MAX_N].
+ * Asynchronous on `stream`. */
+#define MPQ_RHT_MAX_N 32768
+MPQ_API mpq_status mpq_rht(float* X, int64_t rows, int64_t n, const float* signs, mpq_stream_t stream);
 
 /* Release every device buffer the plan owns.  NULL is a no-op. */
 MPQ_API mpq_status mpq_plan_destroy(mpq_plan_t plan);

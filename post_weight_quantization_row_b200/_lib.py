@@ -69,6 +69,13 @@ _sig("mpq_params_default", None, C.POINTER(Params), I32, I32)
 _sig("mpq_plan_create_from_spectrum", ST, P, P, I64, I64, C.POINTER(Params), P, C.POINTER(P))
 _sig("mpq_plan_create_from_x", ST, P, I64, I64, C.POINTER(Params), P, C.POINTER(P))
 _sig("mpq_plan_destroy", ST, P)
+_sig("mpq_gram_create", ST, I64, P, C.POINTER(P))
+_sig("mpq_gram_accumulate", ST, P, P, I64, P)
+_sig("mpq_gram_info", ST, P, C.POINTER(I64), C.POINTER(I64))
+_sig("mpq_gram_get", ST, P, P, P)
+_sig("mpq_gram_destroy", ST, P)
+_sig("mpq_plan_create_from_gram", ST, P, C.POINTER(Params), P, C.POINTER(P))
+_sig("mpq_rht", ST, P, I64, I64, P, P)
 _sig("mpq_plan_info", ST, P, C.POINTER(I64), C.POINTER(I64), C.POINTER(I32), C.POINTER(I32))
 _sig("mpq_plan_get_spectrum", ST, P, P, P, P)
 _sig("mpq_plan_status", ST, P, P)
@@ -88,7 +95,9 @@ _sig("mpq_last_error", C.c_char_p)
 _sig("mpq_kernel_launch_count", I64)
 
 EXPORTED = ["mpq_params_default", "mpq_plan_create_from_spectrum", "mpq_plan_create_from_x",
-            "mpq_plan_destroy", "mpq_plan_info", "mpq_plan_get_spectrum", "mpq_plan_status",
+            "mpq_plan_destroy", "mpq_gram_create", "mpq_gram_accumulate", "mpq_gram_info",
+            "mpq_gram_get", "mpq_gram_destroy", "mpq_plan_create_from_gram", "mpq_rht",
+            "mpq_plan_info", "mpq_plan_get_spectrum", "mpq_plan_status",
             "mpq_plan_workspace_bytes", "mpq_plan_set_workspace_cap", "mpq_solve",
             "mpq_solve_host", "mpq_stage_init", "mpq_stage_denoise", "mpq_stage_linear",
             "mpq_stage_cd", "mpq_stage_energy", "mpq_stage_energy_noalloc",
@@ -155,6 +164,55 @@ def make_params(d: int, K: int, codebook=None, **kw) -> tuple:
     return p, keep
 
 
+class Gram:
+    """Streamed calibration: G = sum over chunks of X_c^T X_c (n x n, fp64, on
+    the device); Plan.from_gram takes the spectrum from it."""
+
+    def __init__(self, n: int):
+        self._h = P()
+        check(lib.mpq_gram_create(int(n), _stream(), C.byref(self._h)), "mpq_gram_create")
+        self.n = int(n)
+
+    def accumulate(self, X: torch.Tensor):
+        if X.dim() != 2 or X.shape[1] != self.n:
+            raise ValueError(f"X must be rows x {self.n}")
+        check(lib.mpq_gram_accumulate(self._h, _ptr(X, torch.float32, name="X"), X.shape[0],
+                                      _stream()), "mpq_gram_accumulate")
+        return self
+
+    @property
+    def rows(self) -> int:
+        n, r = I64(), I64()
+        check(lib.mpq_gram_info(self._h, C.byref(n), C.byref(r)), "mpq_gram_info")
+        return r.value
+
+    def matrix(self) -> torch.Tensor:
+        G = torch.empty((self.n, self.n), dtype=torch.float64, device="cuda")
+        check(lib.mpq_gram_get(self._h, _ptr(G), _stream()), "mpq_gram_get")
+        return G
+
+    def close(self):
+        if self._h is not None and self._h.value:
+            lib.mpq_gram_destroy(self._h)
+        self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def rht(X: torch.Tensor, signs: torch.Tensor) -> torch.Tensor:
+    """In place: every row x of X becomes (x .* signs) H_n / sqrt(n)."""
+    if X.dim() != 2:
+        raise ValueError("X must be 2-D")
+    rows, n = X.shape
+    check(lib.mpq_rht(_ptr(X, torch.float32, name="X"), rows, n,
+                      _ptr(signs, torch.float32, (n,), name="signs"), _stream()), "mpq_rht")
+    return X
+
+
 class Plan:
     """A solver plan: the spectrum of X and the codebook tables, on one GPU."""
 
@@ -195,6 +253,15 @@ class Plan:
         h = P()
         check(lib.mpq_plan_create_from_x(_ptr(X, torch.float32, name="X"), m, n, C.byref(prm),
                                          _stream(), C.byref(h)), "mpq_plan_create_from_x")
+        del keep
+        return cls(h.value, kw.get("group_size", 0))
+
+    @classmethod
+    def from_gram(cls, gram: "Gram", d: int, K: int, codebook=None, **kw):
+        prm, keep = make_params(d, K, codebook, **kw)
+        h = P()
+        check(lib.mpq_plan_create_from_gram(gram._h, C.byref(prm), _stream(), C.byref(h)),
+              "mpq_plan_create_from_gram")
         del keep
         return cls(h.value, kw.get("group_size", 0))
 

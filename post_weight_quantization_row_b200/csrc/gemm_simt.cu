@@ -21,7 +21,7 @@ struct GemmCfg {
 template <typename T, int BM, int BN, int BK>
 __global__ void __launch_bounds__(256)
     k_gemm_nt(const T* __restrict__ A, int64_t lda, const T* __restrict__ B, int64_t ldb,
-              T* __restrict__ C, int64_t ldc, int64_t M, int64_t N, int64_t K) {
+              T* __restrict__ C, int64_t ldc, int64_t M, int64_t N, int64_t K, bool accumulate) {
   using Cfg = GemmCfg<T, BM, BN, BK>;
   constexpr int TM = Cfg::TM, TN = Cfg::TN, EA = Cfg::EA, EB = Cfg::EB;
   __shared__ __align__(16) T As[2][BK][BM + Cfg::PAD];
@@ -98,7 +98,7 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
     for (int j = 0; j < TN; ++j) {
       const int64_t gc = bn + (j / 4) * (BN / Cfg::SPLIT_N) + tx * 4 + (j % 4);
-      if (gc < N) C[gr * ldc + gc] = acc[i][j];
+      if (gc < N) C[gr * ldc + gc] = accumulate ? C[gr * ldc + gc] + acc[i][j] : acc[i][j];
     }
   }
 }
@@ -114,21 +114,23 @@ mpq_status gemm_nt_f32(const float* A, int64_t lda, const float* B, int64_t ldb,
   if (grid.y > 65535) return fail(MPQ_ERR_INVALID_ARG, "gemm: too many row tiles");
   {
     ProfScope ps_(tag, st);
-    k_gemm_nt<float, BM, BN, BK><<<grid, 256, 0, st>>>(A, lda, B, ldb, C, ldc, M, N, K);
+    k_gemm_nt<float, BM, BN, BK><<<grid, 256, 0, st>>>(A, lda, B, ldb, C, ldc, M, N, K, false);
   }
   count_launch();
   return check_launch("k_gemm_nt<f32>");
 }
 
 mpq_status gemm_nt_f64(const double* A, int64_t lda, const double* B, int64_t ldb, double* C,
-                       int64_t ldc, int64_t M, int64_t N, int64_t K, cudaStream_t st) {
+                       int64_t ldc, int64_t M, int64_t N, int64_t K, cudaStream_t st,
+                       bool accumulate) {
   if (M <= 0 || N <= 0) return MPQ_OK;
   constexpr int BM = 64, BN = 64, BK = 16;
   dim3 grid((unsigned)cdiv(N, BN), (unsigned)cdiv(M, BM));
   if (grid.y > 65535) return fail(MPQ_ERR_INVALID_ARG, "gemm: too many row tiles");
   {
     ProfScope ps_("k_gemm_nt_f64", st);
-    k_gemm_nt<double, BM, BN, BK><<<grid, 256, 0, st>>>(A, lda, B, ldb, C, ldc, M, N, K);
+    k_gemm_nt<double, BM, BN, BK><<<grid, 256, 0, st>>>(A, lda, B, ldb, C, ldc, M, N, K,
+                                                         accumulate);
   }
   count_launch();
   return check_launch("k_gemm_nt<f64>");

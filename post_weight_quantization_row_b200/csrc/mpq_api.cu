@@ -683,6 +683,94 @@ mpq_status mpq_plan_create_from_x(const float* X, int64_t m, int64_t n, const mp
   return MPQ_OK;
 }
 
+// ------------------------------------------------ streamed calibration ---
+struct mpq_gram_s {
+  int device = 0;
+  int64_t n = 0;
+  int64_t rows = 0;
+  double* G = nullptr;  // n x n, fp64, device
+};
+
+mpq_status mpq_gram_create(int64_t n, mpq_stream_t stream, mpq_gram_t* gram) {
+  if (!gram) return fail(MPQ_ERR_INVALID_ARG, "gram out-pointer is NULL");
+  *gram = nullptr;
+  if (n < 1 || n > (int64_t)1 << 17) return fail(MPQ_ERR_INVALID_ARG, "gram: n must be in [1, 131072]");
+  cudaStream_t st = (cudaStream_t)stream;
+  mpq_gram_s* g = new mpq_gram_s();
+  g->n = n;
+  mpq_status rc = MPQ_OK;
+  cudaError_t e = cudaGetDevice(&g->device);
+  if (e == cudaSuccess) e = cudaMalloc((void**)&g->G, sizeof(double) * n * n);
+  if (e == cudaSuccess) e = cudaMemsetAsync(g->G, 0, sizeof(double) * n * n, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) rc = cuda_fail(e, "gram allocation");
+  if (rc != MPQ_OK) {
+    mpq_gram_destroy(g);
+    return rc;
+  }
+  *gram = g;
+  return MPQ_OK;
+}
+
+mpq_status mpq_gram_accumulate(mpq_gram_t g, const float* X, int64_t rows, mpq_stream_t stream) {
+  if (!g) return fail(MPQ_ERR_INVALID_ARG, "gram is NULL");
+  if (rows < 0 || (rows > 0 && !X)) return fail(MPQ_ERR_INVALID_ARG, "X must be a device rows x n matrix");
+  DeviceGuard dg(g->device);
+  MPQ_TRY(gram_accumulate(g->G, g->n, X, rows, (cudaStream_t)stream));
+  g->rows += rows;
+  return MPQ_OK;
+}
+
+mpq_status mpq_gram_info(mpq_gram_t g, int64_t* n, int64_t* rows) {
+  if (!g) return fail(MPQ_ERR_INVALID_ARG, "gram is NULL");
+  if (n) *n = g->n;
+  if (rows) *rows = g->rows;
+  return MPQ_OK;
+}
+
+mpq_status mpq_gram_get(mpq_gram_t g, double* G, mpq_stream_t stream) {
+  if (!g || !G) return fail(MPQ_ERR_INVALID_ARG, "gram and G must be non-NULL");
+  DeviceGuard dg(g->device);
+  MPQ_CUDA(cudaMemcpyAsync(G, g->G, sizeof(double) * g->n * g->n, cudaMemcpyDeviceToDevice,
+                           (cudaStream_t)stream));
+  return MPQ_OK;
+}
+
+mpq_status mpq_gram_destroy(mpq_gram_t g) {
+  if (!g) return MPQ_OK;
+  if (g->G) cudaFree(g->G);
+  delete g;
+  return MPQ_OK;
+}
+
+mpq_status mpq_plan_create_from_gram(mpq_gram_t g, const mpq_params* params, mpq_stream_t stream,
+                                     mpq_plan_t* plan) {
+  if (!plan) return fail(MPQ_ERR_INVALID_ARG, "plan out-pointer is NULL");
+  *plan = nullptr;
+  if (!g) return fail(MPQ_ERR_INVALID_ARG, "gram is NULL");
+  if (g->rows < 1) return fail(MPQ_ERR_RANK, "gram holds no calibration rows");
+  DeviceGuard dg(g->device);
+  cudaStream_t st = (cudaStream_t)stream;
+  mpq_plan_s* p = nullptr;
+  MPQ_TRY(new_plan(params, g->n, &p));
+  mpq_status rc = setup_spectrum_from_gram(p, g->G, g->rows, st);
+  if (rc == MPQ_OK) rc = finish_plan(p, st);
+  if (rc != MPQ_OK) {
+    destroy_plan(p);
+    return rc;
+  }
+  *plan = p;
+  return MPQ_OK;
+}
+
+mpq_status mpq_rht(float* X, int64_t rows, int64_t n, const float* signs, mpq_stream_t stream) {
+  if (n < 1 || n > MPQ_RHT_MAX_N || (n & (n - 1)))
+    return fail(MPQ_ERR_INVALID_ARG, "rht: n must be a power of two in [1, 32768]");
+  if (rows < 0 || (rows > 0 && (!X || !signs)))
+    return fail(MPQ_ERR_INVALID_ARG, "rht: X (rows x n) and signs (n) must be device buffers");
+  return launch_rht(X, rows, n, signs, (cudaStream_t)stream);
+}
+
 mpq_status mpq_plan_destroy(mpq_plan_t plan) {
   destroy_plan(plan);
   return MPQ_OK;

@@ -158,9 +158,11 @@ namespace mpq {
 mpq_status gemm_nt_f32(const float* A, int64_t lda, const float* B, int64_t ldb, float* C,
                        int64_t ldc, int64_t M, int64_t N, int64_t K, cudaStream_t st,
                        const char* tag = "gemm_f32");
-// Same with fp64 operands and accumulation (setup).
+// Same with fp64 operands and accumulation (setup); `accumulate` adds the
+// product to C instead of overwriting it.
 mpq_status gemm_nt_f64(const double* A, int64_t lda, const double* B, int64_t ldb, double* C,
-                       int64_t ldc, int64_t M, int64_t N, int64_t K, cudaStream_t st);
+                       int64_t ldc, int64_t M, int64_t N, int64_t K, cudaStream_t st,
+                       bool accumulate = false);
 
 mpq_status launch_init(const mpq_plan_s* p, const float* W, int64_t m, int given, float* scale,
                        float* offset, uint16_t* idx, double* gamma1_0, cudaStream_t st);
@@ -266,6 +268,13 @@ mpq_status build_hessian(mpq_plan_s* p, cudaStream_t st);
 mpq_status build_codebook_tables(mpq_plan_s* p, cudaStream_t st);
 mpq_status setup_spectrum_from_x(mpq_plan_s* p, const float* X, int64_t m, int64_t n,
                                  cudaStream_t st);
+// Spectrum from an accumulated Gram G = X^T X (n x n fp64, device, n = p->n)
+// of m calibration rows: Jacobi eigenpairs, the same rank cut as from X.
+mpq_status setup_spectrum_from_gram(mpq_plan_s* p, const double* G, int64_t m, cudaStream_t st);
+// G (n x n fp64) += X^T X for X (rows x n fp32, device), fp64 products.
+mpq_status gram_accumulate(double* G, int64_t n, const float* X, int64_t rows, cudaStream_t st);
+// In place: every row x of X (rows x n) becomes (x .* signs) H_n / sqrt(n).
+mpq_status launch_rht(float* X, int64_t rows, int64_t n, const float* signs, cudaStream_t st);
 
 inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 

@@ -289,29 +289,13 @@ mpq_status jacobi_eig(const double* G, int64_t N0, double* lam, double* E, cudaS
   return check_launch("jacobi sort");
 }
 
-}  // namespace
-
-mpq_status setup_spectrum_from_x(mpq_plan_s* p, const float* X, int64_t m, int64_t n,
-                                 cudaStream_t st) {
-  const bool right = n <= m;  // Gram X^T X (n x n); else X X^T (m x m)
-  const int64_t N0 = right ? n : m;
-  DevBuf<double> Xd, G, lam, E;
-  MPQ_TRY(Xd.alloc(m * n));
-  MPQ_TRY(G.alloc(N0 * N0));
-  MPQ_TRY(lam.alloc(N0));
-  MPQ_TRY(E.alloc(N0 * N0));
-  {
-    ProfScope ps_("k_x_to_f64", st);
-    k_x_to_f64<<<g1(m * n), 256, 0, st>>>(X, m, n, right ? 1 : 0, Xd.p);
-  }
-  count_launch();
-  MPQ_TRY(check_launch("k_x_to_f64"));
-  if (right) MPQ_TRY(gemm_nt_f64(Xd.p, m, Xd.p, m, G.p, n, n, n, m, st));   // (X^T)(X^T)^T
-  else MPQ_TRY(gemm_nt_f64(Xd.p, n, Xd.p, n, G.p, m, m, m, n, st));          // X X^T
-  MPQ_TRY(jacobi_eig(G.p, N0, lam.p, E.p, st));
-  // rank cut on the host from the sorted eigenvalues (N0 values)
+// Rank cut on the host from the N0 sorted eigenvalues lam (device):
+// r = #{lambda > lambda_max * max(m, n) * 2^-52}; allocates the plan's s64
+// (r) and V64 (n x r) and fills s = sqrt(lambda[:r]).
+mpq_status cut_and_alloc(mpq_plan_s* p, const double* lam, int64_t N0, int64_t m, int64_t n,
+                         cudaStream_t st) {
   std::vector<double> hl(N0);
-  MPQ_CUDA(cudaMemcpyAsync(hl.data(), lam.p, sizeof(double) * N0, cudaMemcpyDeviceToHost, st));
+  MPQ_CUDA(cudaMemcpyAsync(hl.data(), lam, sizeof(double) * N0, cudaMemcpyDeviceToHost, st));
   MPQ_CUDA(cudaStreamSynchronize(st));
   const double tol = (N0 > 0 ? hl[0] : 0.0) * (double)std::max(m, n) * ldexp(1.0, -52);
   int64_t r = 0;
@@ -326,17 +310,70 @@ mpq_status setup_spectrum_from_x(mpq_plan_s* p, const float* X, int64_t m, int64
   }
   {
     ProfScope ps_("k_sqrt_first", st);
-    k_sqrt_first<<<(unsigned)cdiv(r, 256), 256, 0, st>>>(lam.p, r, p->s64);
+    k_sqrt_first<<<(unsigned)cdiv(r, 256), 256, 0, st>>>(lam, r, p->s64);
   }
   count_launch();
-  if (right) {
-    {
-      ProfScope ps_("k_take_cols", st);
-      k_take_cols<<<(unsigned)cdiv(N0 * r, 256), 256, 0, st>>>(E.p, N0, r, p->V64);
-    }
-    count_launch();
-    return check_launch("setup gather");
+  return check_launch("k_sqrt_first");
+}
+
+}  // namespace
+
+mpq_status setup_spectrum_from_gram(mpq_plan_s* p, const double* G, int64_t m, cudaStream_t st) {
+  const int64_t n = p->n;
+  DevBuf<double> lam, E;
+  MPQ_TRY(lam.alloc(n));
+  MPQ_TRY(E.alloc(n * n));
+  MPQ_TRY(jacobi_eig(G, n, lam.p, E.p, st));
+  MPQ_TRY(cut_and_alloc(p, lam.p, n, m, n, st));
+  {
+    ProfScope ps_("k_take_cols", st);
+    k_take_cols<<<(unsigned)cdiv(n * p->r, 256), 256, 0, st>>>(E.p, n, p->r, p->V64);
   }
+  count_launch();
+  MPQ_TRY(check_launch("setup gather"));
+  MPQ_CUDA(cudaStreamSynchronize(st));
+  return MPQ_OK;
+}
+
+mpq_status gram_accumulate(double* G, int64_t n, const float* X, int64_t rows, cudaStream_t st) {
+  if (rows == 0) return MPQ_OK;
+  DevBuf<double> Xt;
+  MPQ_TRY(Xt.alloc(rows * n));
+  {
+    ProfScope ps_("k_x_to_f64", st);
+    k_x_to_f64<<<g1(rows * n), 256, 0, st>>>(X, rows, n, 1, Xt.p);
+  }
+  count_launch();
+  MPQ_TRY(check_launch("k_x_to_f64"));
+  MPQ_TRY(gemm_nt_f64(Xt.p, rows, Xt.p, rows, G, n, n, n, rows, st, /*accumulate=*/true));
+  MPQ_CUDA(cudaStreamSynchronize(st));  // Xt is released on return
+  return MPQ_OK;
+}
+
+mpq_status setup_spectrum_from_x(mpq_plan_s* p, const float* X, int64_t m, int64_t n,
+                                 cudaStream_t st) {
+  const bool right = n <= m;  // Gram X^T X (n x n); else X X^T (m x m)
+  const int64_t N0 = right ? n : m;
+  DevBuf<double> Xd, G, lam, E;
+  MPQ_TRY(G.alloc(N0 * N0));
+  if (right) {
+    MPQ_CUDA(cudaMemsetAsync(G.p, 0, sizeof(double) * N0 * N0, st));
+    MPQ_TRY(gram_accumulate(G.p, n, X, m, st));
+    return setup_spectrum_from_gram(p, G.p, m, st);
+  }
+  MPQ_TRY(Xd.alloc(m * n));
+  MPQ_TRY(lam.alloc(N0));
+  MPQ_TRY(E.alloc(N0 * N0));
+  {
+    ProfScope ps_("k_x_to_f64", st);
+    k_x_to_f64<<<g1(m * n), 256, 0, st>>>(X, m, n, 0, Xd.p);
+  }
+  count_launch();
+  MPQ_TRY(check_launch("k_x_to_f64"));
+  MPQ_TRY(gemm_nt_f64(Xd.p, n, Xd.p, n, G.p, m, m, m, n, st));  // X X^T
+  MPQ_TRY(jacobi_eig(G.p, N0, lam.p, E.p, st));
+  MPQ_TRY(cut_and_alloc(p, lam.p, N0, m, n, st));
+  const int64_t r = p->r;
   // V = X^T U diag(1/s): (n x r) = Xt (n x m) * Ut (r x m)^T
   DevBuf<double> Xt, Ut;
   MPQ_TRY(Xt.alloc(n * m));
@@ -360,6 +397,55 @@ mpq_status setup_spectrum_from_x(mpq_plan_s* p, const float* X, int64_t m, int64
   MPQ_TRY(check_launch("k_div_cols"));
   MPQ_CUDA(cudaStreamSynchronize(st));
   return MPQ_OK;
+}
+
+// ------------------------------------------- random Hadamard rotation ---
+// Incoherence preprocessing (the ai.info page on MPQ, findings: a random
+// Hadamard rotation leaves E_lin unchanged because E_lin sees the Hessian
+// only through its eigenvalues).  Every row x of X becomes x Q^T with
+// Q = H_n diag(signs) / sqrt(n), H_n the Sylvester-Hadamard matrix
+// (H_1 = [1], H_2k = [[H_k, H_k], [H_k, -H_k]]; symmetric), so that
+// x Q^T = (x .* signs) H_n / sqrt(n).  One CTA per row (grid-stride): the row
+// sits in shared memory and takes log2(n) butterfly stages; pair i of the
+// stage with half-width h is (lo, lo + h), lo = 2h floor(i / h) + i mod h.
+namespace {
+
+__global__ void __launch_bounds__(512)
+    k_rht(float* __restrict__ X, int64_t rows, int n, const float* __restrict__ signs,
+          float inv_sqrt_n) {
+  extern __shared__ float sx[];
+  for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
+    float* x = X + row * n;
+    for (int j = threadIdx.x; j < n; j += blockDim.x) sx[j] = x[j] * signs[j];
+    __syncthreads();
+    for (int h = 1; h < n; h <<= 1) {
+      for (int i = threadIdx.x; i < n / 2; i += blockDim.x) {
+        const int lo = ((i & ~(h - 1)) << 1) | (i & (h - 1));
+        const float a = sx[lo], b = sx[lo + h];
+        sx[lo] = a + b;
+        sx[lo + h] = a - b;
+      }
+      __syncthreads();
+    }
+    for (int j = threadIdx.x; j < n; j += blockDim.x) x[j] = sx[j] * inv_sqrt_n;
+    __syncthreads();
+  }
+}
+
+}  // namespace
+
+mpq_status launch_rht(float* X, int64_t rows, int64_t n, const float* signs, cudaStream_t st) {
+  if (rows == 0) return MPQ_OK;
+  const int threads = (int)std::min<int64_t>(512, std::max<int64_t>(32, n / 2));
+  const size_t smem = sizeof(float) * (size_t)n;
+  MPQ_CUDA(cudaFuncSetAttribute(k_rht, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  const unsigned grid = (unsigned)std::min<int64_t>(rows, 148 * 8);
+  {
+    ProfScope ps_("k_rht", st);
+    k_rht<<<grid, threads, smem, st>>>(X, rows, (int)n, signs, (float)(1.0 / sqrt((double)n)));
+  }
+  count_launch();
+  return check_launch("k_rht");
 }
 
 }  // namespace mpq

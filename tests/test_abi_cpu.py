@@ -72,3 +72,24 @@ def test_codebook_required_for_vector_plans(mpq):
     st = mpq.lib.mpq_plan_create_from_spectrum(C.c_void_p(16), C.c_void_p(16), 64, 8, C.byref(p),
                                                None, C.byref(h))
     assert st == 1
+
+
+def test_streamed_gram_and_rht_reject_bad_arguments_without_a_device(mpq):
+    lib, h = mpq.lib, C.c_void_p()
+    dummy = C.c_void_p(16)
+    assert lib.mpq_gram_create(0, None, C.byref(h)) == 1 and h.value is None
+    assert lib.mpq_gram_create(1 << 18, None, C.byref(h)) == 1
+    assert lib.mpq_gram_create(64, None, None) == 1
+    assert lib.mpq_gram_accumulate(None, dummy, 4, None) == 1
+    assert lib.mpq_gram_info(None, None, None) == 1
+    assert lib.mpq_gram_get(None, dummy, None) == 1
+    assert lib.mpq_gram_destroy(None) == 0
+    p = mpq.Params()
+    lib.mpq_params_default(C.byref(p), 1, 8)
+    assert lib.mpq_plan_create_from_gram(None, C.byref(p), None, C.byref(h)) == 1
+    assert h.value is None
+    # n not a power of two, above the shared-memory limit, negative rows, NULL X
+    for rows, n, x in [(4, 3, dummy), (4, 65536, dummy), (4, 0, dummy), (-1, 64, dummy),
+                       (4, 64, None)]:
+        assert lib.mpq_rht(x, rows, n, dummy, None) == 1, (rows, n)
+    assert "power of two" in lib.mpq_last_error().decode() or "device" in lib.mpq_last_error().decode()

@@ -1,0 +1,220 @@
+"""Calibration-scale setup on the device: the streamed Gram (chunks of X
+accumulated into G = X^T X in fp64, then the spectrum from G) and the random
+Hadamard rotation.
+
+Pins that do not come from the CUDA path: G against X^T X computed by numpy
+in fp64; the spectrum against the oracle's SVD of the stacked chunks
+(through the sign-free H = V diag(s^2) V^T); the rotation against the dense
+Sylvester-Hadamard matrix of scipy.linalg.hadamard and, for n too large for
+a dense matrix, against the Kronecker identity H_ab = H_a (x) H_b and the
+involution (x H / sqrt(n)) H / sqrt(n) = x.  A solve on the Gram plan meets
+the oracle's solve on the oracle's spectrum under the same bars as the other
+whole-solve tests."""
+import math
+
+import numpy as np
+import pytest
+import scipy.linalg
+import torch
+
+import mpq_inputs as mi
+from oracle import mpq_oracle as orc
+from tests.helpers import codebook_for, cu, host, idx_np, oracle_grid_f32
+
+pytestmark = pytest.mark.gpu
+
+ENERGY_TOL = 1e-3
+LOGIT_TIE = 1e-3
+
+
+@pytest.fixture(scope="module")
+def mpq():
+    import post_weight_quantization_row_b200 as m
+    return m
+
+
+def heavy_x(seed, m, n):
+    g = np.random.default_rng(seed)
+    return mi.heavy_tailed_x(g, g, m, n).astype(np.float32)
+
+
+def gram_of(mpq, X, cuts):
+    """Gram handle fed X in the row chunks between consecutive cuts."""
+    gram = mpq.Gram(X.shape[1])
+    for a, b in zip(cuts[:-1], cuts[1:]):
+        gram.accumulate(cu(X[a:b]))
+    return gram
+
+
+def assert_same_spectrum(sg, Vg, s, V):
+    assert sg.size == s.size
+    assert np.allclose(sg, s, rtol=1e-9)
+    Hg = (Vg * sg ** 2) @ Vg.T
+    H = (V * s ** 2) @ V.T
+    assert np.abs(Hg - H).max() <= 1e-9 * np.abs(H).max()
+    assert np.allclose(Vg.T @ Vg, np.eye(sg.size), atol=1e-9)
+
+
+# ------------------------------------------------------------ streamed Gram ---
+
+@pytest.mark.parametrize("m,n,cuts", [
+    (600, 200, [0, 1, 257, 257, 600]),      # a one-row chunk and an empty chunk
+    (150, 200, [0, 64, 150]),               # fewer rows than columns: rank 150
+    (1000, 64, [0, 300, 600, 1000]),
+])
+def test_gram_accumulates_x_transpose_x(mpq, m, n, cuts):
+    X = heavy_x(m + 7 * n, m, n)
+    gram = gram_of(mpq, X, cuts)
+    assert gram.rows == m
+    G = host(gram.matrix())
+    Xd = X.astype(np.float64)
+    G_ref = Xd.T @ Xd
+    assert np.abs(G - G_ref).max() <= 1e-12 * np.abs(G_ref).max()
+    assert np.abs(G - G.T).max() <= 1e-14 * np.abs(G_ref).max()
+    plan = mpq.Plan.from_gram(gram, 1, 8)
+    s, V = orc.spectrum(X)
+    sg, Vg = (host(t) for t in plan.spectrum())
+    assert_same_spectrum(sg, Vg, s, V)
+    if m < n:
+        assert plan.r == m
+
+
+def test_gram_at_calibration_scale(mpq):
+    # 128 sequences x 2048 tokens = 262144 activation rows, streamed in eight
+    # chunks generated on the device (heavy-tailed: a few columns scaled up)
+    n, chunk, chunks = 512, 32768, 8
+    gen = torch.Generator(device="cuda").manual_seed(2026)
+    col = torch.ones(n, device="cuda")
+    col[torch.randperm(n, generator=gen, device="cuda")[:8]] = 20.0
+    gram = mpq.Gram(n)
+    G_ref = torch.zeros((n, n), dtype=torch.float64, device="cuda")
+    for _ in range(chunks):
+        Xc = torch.randn((chunk, n), generator=gen, device="cuda") * col
+        gram.accumulate(Xc)
+        Xd = Xc.double()
+        G_ref += Xd.T @ Xd
+    assert gram.rows == chunk * chunks
+    G = gram.matrix()
+    assert (G - G_ref).abs().max().item() <= 1e-12 * G_ref.abs().max().item()
+    plan = mpq.Plan.from_gram(gram, 1, 8)
+    assert plan.r == n
+    lam_ref = torch.linalg.eigvalsh(G_ref).flip(0).cpu().numpy()
+    s = host(plan.spectrum()[0])
+    assert np.abs(s ** 2 - lam_ref).max() <= 1e-10 * lam_ref[0]
+
+
+def test_gram_plan_equals_from_x_plan(mpq):
+    X = heavy_x(31, 500, 128)
+    a = mpq.Plan.from_gram(gram_of(mpq, X, [0, 100, 500]), 1, 8)
+    b = mpq.Plan.from_x(cu(X), 1, 8)
+    sa, Va = (host(t) for t in a.spectrum())
+    sb, Vb = (host(t) for t in b.spectrum())
+    assert_same_spectrum(sa, Va, sb, Vb)
+
+
+def test_gram_without_rows_is_a_rank_error(mpq):
+    gram = mpq.Gram(64)
+    with pytest.raises(mpq.MPQError) as e:
+        mpq.Plan.from_gram(gram, 1, 8)
+    assert e.value.status == 5
+    gram.accumulate(cu(np.zeros((10, 64), np.float32)))
+    with pytest.raises(mpq.MPQError) as e:
+        mpq.Plan.from_gram(gram, 1, 8)
+    assert e.value.status == 5
+    with pytest.raises(ValueError):
+        gram.accumulate(cu(np.zeros((10, 32), np.float32)))
+
+
+@pytest.mark.parametrize("d", [1, 8])
+def test_solve_on_gram_plan_matches_oracle(mpq, d):
+    if d == 1:
+        p = mi.small_problem(101, 37, 200, 300, d=1, levels=8, T_vamp=4, cd_sweeps=3)
+        sc, off = oracle_grid_f32(p)
+    else:
+        cb = mi.e8_codebook_cached()[:2048]
+        p = mi.small_problem(202, 21, 160, 320, d=8, levels=2048, T_vamp=4, cd_sweeps=3,
+                             codebook=cb)
+        sc = orc.rms_scale(p.W)[0].astype(np.float32)
+        off = np.zeros_like(sc)
+    X = p.X.astype(np.float32)
+    plan = mpq.Plan.from_gram(gram_of(mpq, X, [0, 77, X.shape[0]]), p.d, p.levels,
+                              codebook=p.codebook if d == 8 else None)
+    s, V = orc.spectrum(X)
+    cbk = codebook_for(p)
+    ref = orc.solve(p.W, cbk, s, V, p.T_vamp, p.cd_sweeps, sc.astype(np.float64),
+                    off.astype(np.float64))
+    out = plan.solve(cu(p.W), p.T_vamp, p.cd_sweeps, row_scale=cu(sc), row_offset=cu(off),
+                     stats=True)
+    clean = np.all(ref.map_gap > LOGIT_TIE, axis=1) & (ref.cd.first_tie < 0)
+    assert clean.mean() >= 0.25
+    assert np.array_equal(idx_np(out["idx"])[clean], ref.idx[clean])
+    e = host(out["energy"]).astype(np.float64)
+    assert np.all(np.abs(e[clean] - ref.energy[clean]) <= ENERGY_TOL * ref.energy[clean])
+    assert abs(e.sum() - ref.energy.sum()) <= 1e-2 * ref.energy.sum()
+
+
+# ------------------------------------------------- random Hadamard rotation ---
+
+def signs_of(seed, n):
+    return np.where(np.random.default_rng(seed).random(n) < 0.5, -1.0, 1.0).astype(np.float32)
+
+
+@pytest.mark.parametrize("rows,n", [(5, 1), (7, 2), (37, 64), (2000, 64), (9, 1024), (3, 4096)])
+def test_rht_matches_dense_hadamard(mpq, rows, n):
+    # 2000 rows: more rows than CTAs, so CTAs walk several rows
+    g = np.random.default_rng(rows * 7 + n)
+    X = g.standard_normal((rows, n)).astype(np.float32)
+    sg = signs_of(n, n)
+    Xt = cu(X.copy())
+    mpq.rht(Xt, cu(sg))
+    Q_T = (sg[:, None].astype(np.float64) * scipy.linalg.hadamard(n)) / math.sqrt(n)
+    ref = X.astype(np.float64) @ Q_T
+    got = host(Xt).astype(np.float64)
+    err = np.linalg.norm(got - ref, axis=1) / np.linalg.norm(ref, axis=1)
+    assert err.max() <= 4e-7 * max(1, math.log2(n))
+
+
+@pytest.mark.parametrize("n", [16384, 32768])
+def test_rht_large_rows_kronecker_and_involution(mpq, n):
+    rows = 4
+    g = np.random.default_rng(n)
+    X = g.standard_normal((rows, n)).astype(np.float32)
+    sg = signs_of(n + 1, n)
+    Xt = cu(X.copy())
+    mpq.rht(Xt, cu(sg))
+    # H_n = H_a (x) H_b: a row reshaped a x b maps to H_a Z H_b (both symmetric)
+    a, b = 8, n // 8
+    Ha, Hb = scipy.linalg.hadamard(a), scipy.linalg.hadamard(b)
+    Z = (X.astype(np.float64) * sg).reshape(rows, a, b)
+    ref = np.einsum("ij,rjk,kl->ril", Ha, Z, Hb).reshape(rows, n) / math.sqrt(n)
+    got = host(Xt).astype(np.float64)
+    err = np.linalg.norm(got - ref, axis=1) / np.linalg.norm(ref, axis=1)
+    assert err.max() <= 4e-7 * math.log2(n)
+    # with all signs +1 the rotation is its own inverse
+    ones = cu(np.ones(n, np.float32))
+    Y = cu(X.copy())
+    mpq.rht(mpq.rht(Y, ones), ones)
+    back = host(Y).astype(np.float64)
+    assert np.abs(back - X).max() <= 1e-5 * np.abs(X).max()
+
+
+def test_rht_preserves_the_objective(mpq):
+    # rotating W and X by the same Q leaves ||(W - W_hat) X^T|| unchanged for
+    # any W_hat rotated alongside: the Gram of the rotated X is Q G Q^T
+    n, m = 256, 512
+    X = heavy_x(44, m, n)
+    sg = signs_of(45, n)
+    Xr = cu(X.copy())
+    mpq.rht(Xr, cu(sg))
+    G = X.astype(np.float64).T @ X.astype(np.float64)
+    Gr = host(Xr).astype(np.float64)
+    Gr = Gr.T @ Gr
+    ev, evr = np.linalg.eigvalsh(G), np.linalg.eigvalsh(Gr)
+    assert np.abs(ev - evr).max() <= 1e-5 * ev.max()
+
+
+def test_rht_rejects_bad_sizes(mpq):
+    for n in (3, 96):
+        with pytest.raises(mpq.MPQError):
+            mpq.rht(cu(np.zeros((2, n), np.float32)), cu(np.ones(n, np.float32)))
+    mpq.rht(cu(np.zeros((0, 64), np.float32)), cu(np.ones(64, np.float32)))   # no rows: no-op
