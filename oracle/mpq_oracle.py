@@ -35,6 +35,10 @@ Readings where the pages are silent (each also listed in the design doc):
   R9  CD: blocks in order, argmin over all codewords (lowest index on ties),
       accept iff the energy change is strictly negative; stop after a sweep
       that changes nothing.
+  R16 greedy baseline (LDLQ / GPTQ): blocks in order, each committed to its
+      nearest codeword in the Euclidean metric (lowest index on ties), the
+      error passed on through the factor of (H + lambda I)^-1 with
+      lambda = damp * mean(diag H); damp defaults to 0.01.
 """
 from __future__ import annotations
 
@@ -410,6 +414,61 @@ def cd(W, idx0, codebook, scale, offset, H, sweeps: int, tie_rel: float = 1e-5) 
 
 
 # ----------------------------------------------------------------------------
+# greedy baseline: LDLQ / GPTQ
+# ----------------------------------------------------------------------------
+
+@dataclass
+class GreedyOut:
+    idx: np.ndarray          # m x B
+    gap: np.ndarray          # m x B: top-two distance gap of each decision / scale^2
+
+
+def damped_hessian(H, damp: float):
+    """H + lambda I, lambda = damp * mean(diag H) (reading R16)."""
+    H = np.asarray(H, np.float64)
+    lam = damp * float(np.trace(H)) / H.shape[0]
+    return H + lam * np.eye(H.shape[0])
+
+
+def ldlq(W, codebook, scale, offset, H, damp: float = 0.01) -> GreedyOut:
+    """The greedy hard-decision solver MPQ is measured against ([MPQ-note]
+    motivation: GPTQ and LDLQ visit the blocks in order, commit each one to a
+    single codeword at once and pass its hard error on to the blocks not yet
+    quantised; ablation table: "LDLQ baseline" = T_vamp 0, CD 0, and
+    "LDLQ + CD3").  Error feedback in the GPTQ form: with U the upper
+    Cholesky factor of (H + lambda I)^-1 = U^T U, committing column j to q_j
+    moves every later column k by -(v_j - q_j) U[j, k] / U[j, j], which puts
+    the not-yet-quantised weights at their least-squares optimum given the
+    committed ones.  A block is committed to the codeword nearest (Euclidean)
+    its current values, then its columns feed back one after another."""
+    W = np.asarray(W, np.float64)
+    m, n = W.shape
+    d = codebook.shape[1]
+    B = n // d
+    U = np.linalg.cholesky(np.linalg.inv(damped_hessian(H, damp))).T
+    idx = np.zeros((m, B), dtype=np.int64)
+    gap = np.full((m, B), np.inf)
+    for i in range(m):
+        cand = block_candidates(codebook, scale[i], offset[i], B)      # B x K x d
+        si = np.atleast_1d(np.asarray(scale[i], np.float64))
+        sc = np.repeat(si, B // si.size)                              # scale of each block
+        v = W[i].copy()
+        for b in range(B):
+            sl = slice(b * d, (b + 1) * d)
+            dist = ((v[sl][None, :] - cand[b]) ** 2).sum(axis=1)
+            k = int(np.argmin(dist))
+            if dist.size > 1:
+                two = np.partition(dist, 1)[:2]
+                gap[i, b] = (two[1] - two[0]) / (sc[b] * sc[b])
+            q = cand[b, k]
+            for t, j in enumerate(range(b * d, (b + 1) * d)):
+                err = (v[j] - q[t]) / U[j, j]
+                v[j + 1:] -= err * U[j, j + 1:]
+            idx[i, b] = k
+    return GreedyOut(idx, gap)
+
+
+# ----------------------------------------------------------------------------
 # a10: energies
 # ----------------------------------------------------------------------------
 
@@ -455,14 +514,18 @@ def terminal_precision(gamma1, scale):
 
 def solve(W, codebook, s, V, T_vamp: int, cd_sweeps: int, scale=None, offset=None,
           beta0: float = 1.0, damping: float = 0.5, tau: float = math.inf,
-          keep_trace: bool = False, group: int = 0, cd_skip_precision: float = 0.0) -> SolveOut:
+          keep_trace: bool = False, group: int = 0, cd_skip_precision: float = 0.0,
+          greedy_damp: Optional[float] = None) -> SolveOut:
     """The MPQ solve of every row ([MPQ-note] flowchart and Overall
     framework): init -> T_vamp x (denoiser -> extrinsic -> linear module ->
     M-step) -> marginal MAP argmax -> exact block CD -> energies.
     With ``cd_skip_precision`` > 0, rows whose terminal precision (see
     terminal_precision) exceeds it keep the marginal MAP and run no CD: the
     [MPQ-note] diagnostics report terminal precisions near 1e5 at 3-bit
-    scalar with CD changing almost no block (reading R13)."""
+    scalar with CD changing almost no block (reading R13).
+    With T_vamp = 0 and ``greedy_damp`` given, the hard init that CD refines
+    is the greedy baseline ldlq(..., damp=greedy_damp) instead of
+    round-to-nearest (the ablation's LDLQ and LDLQ + CD rows)."""
     W = np.asarray(W, np.float64)
     st = init(W, codebook, scale, offset, beta0, group)
     g10 = st.gamma1.copy()
@@ -477,8 +540,12 @@ def solve(W, codebook, s, V, T_vamp: int, cd_sweeps: int, scale=None, offset=Non
             trace.append((dn, lo))
         R1, g1, beta = lo.R1, lo.gamma1, lo.beta
         clamps += lo.clamps
-    dn = denoise(R1, g1, codebook, st.scale, st.offset, W, ga)
-    idx_map = dn.idx
+    if T_vamp == 0 and greedy_damp is not None:
+        gr = ldlq(W, codebook, st.scale, st.offset, hessian(s, V), greedy_damp)
+        idx_map, map_gap = gr.idx, gr.gap
+    else:
+        dn = denoise(R1, g1, codebook, st.scale, st.offset, W, ga)
+        idx_map, map_gap = dn.idx, dn.gap
     cdo = None
     idx = idx_map
     if cd_sweeps > 0:
@@ -494,12 +561,35 @@ def solve(W, codebook, s, V, T_vamp: int, cd_sweeps: int, scale=None, offset=Non
             cdo.x = decode(idx, codebook, st.scale, st.offset)
     w_hat = decode(idx, codebook, st.scale, st.offset)
     E = energy(W, w_hat, s, V)
-    return SolveOut(idx, w_hat, E, idx_map, dn.gap, g1, beta, clamps, cdo, trace)
+    return SolveOut(idx, w_hat, E, idx_map, map_gap, g1, beta, clamps, cdo, trace)
 
 
 # ----------------------------------------------------------------------------
 # brute force helpers for pins
 # ----------------------------------------------------------------------------
+
+def greedy_conditional(w, codebook, scale, offset, Ht):
+    """The greedy baseline by its definition, for pins on short rows: block b
+    takes the codeword nearest the b-part of the least-squares optimum of the
+    blocks >= b given the committed blocks < b (minimising e^T Ht e over the
+    free part of the error e = w - x), solved afresh for every block."""
+    w = np.asarray(w, np.float64)
+    n = w.size
+    d = codebook.shape[1]
+    B = n // d
+    cand = block_candidates(codebook, scale, offset, B)
+    x = np.zeros(n)
+    idx = np.zeros(B, dtype=np.int64)
+    for b in range(B):
+        c0 = b * d
+        e_fixed = w[:c0] - x[:c0]
+        e_free = -np.linalg.solve(Ht[c0:, c0:], Ht[c0:, :c0] @ e_fixed) if c0 else np.zeros(n)
+        target = w[c0:c0 + d] - e_free[:d]
+        k = int(np.argmin(((target[None, :] - cand[b]) ** 2).sum(axis=1)))
+        idx[b] = k
+        x[c0:c0 + d] = cand[b, k]
+    return idx
+
 
 def exhaustive_min_energy(w, codebook, scale, offset, H):
     """Exact minimum of 1/2 (w-x)^T H (w-x) over every assignment of a short
