@@ -59,6 +59,9 @@ def parse():
     ap.add_argument("--group-size", type=int, default=0,
                     help="scalar workloads: one min-max grid per group of this many columns "
                          "(0 = one per row)")
+    ap.add_argument("--greedy", action="store_true",
+                    help="scalar workloads: the greedy baseline (LDLQ init, T_vamp = 0) with the "
+                         "same CD sweeps instead of MPQ")
     ap.add_argument("--spectrum-cache", default=None,
                     help="npz file: reuse the spectrum a previous run computed on the device")
     return ap.parse_args()
@@ -191,10 +194,13 @@ def kernel_work(name, m, n, r, d, K, L):
         return "hbm", "GB/s", 14.0 * m * n
     if name == "k_cd_tile_decide":       # per 128-column tile: h, idx in; idx, Delta hi/lo out
         return "hbm", "GB/s", 12.0 * m * 128
+    if name == "k_ldlq_tile":            # per 128-column tile: W_work in; idx, E hi/lo out
+        return "hbm", "GB/s", 10.0 * m * 128
     return None
 
 
 KERNEL_SOURCE = {"gemm": "gemm_tc.cu", "k_cd_vec_scan": "cd_scan_tc.cu", "k_cd": "kernels_cd.cu",
+                 "k_ldlq": "greedy.cu",
                  "k_denoise_vec_tc": "denoise_tc.cu", "k_": "kernels_vamp.cu"}
 
 
@@ -261,7 +267,7 @@ def describe(p, cfg, group=0):
             "seeds": p.seeds, "l2": "flushed between timed steps (512 MiB write)"}
 
 
-def oracle_sample(p, rows, steps=1, group=0):
+def oracle_sample(p, rows, steps=1, group=0, greedy_damp=None):
     """Time the float64 oracle on `rows` rows of the layer (spectrum excluded)."""
     from oracle import mpq_oracle as orc
     t0 = time.time()
@@ -272,7 +278,7 @@ def oracle_sample(p, rows, steps=1, group=0):
     for k in range(steps):
         sel = slice((k * rows) % p.m_out, (k * rows) % p.m_out + rows)
         t0 = time.perf_counter()
-        orc.solve(p.W[sel], cb, s, V, p.T_vamp, p.cd_sweeps, group=group)
+        orc.solve(p.W[sel], cb, s, V, p.T_vamp, p.cd_sweeps, group=group, greedy_damp=greedy_damp)
         times.append(time.perf_counter() - t0)
     return times, t_spec
 
@@ -314,7 +320,16 @@ def run_mpq(args, world, rank, local):
     p = workload(args.config, rank)
     if args.rows:
         p.W = np.ascontiguousarray(p.W[:args.rows])
+    greedy = {}
+    if args.greedy:
+        if p.d != 1:
+            raise SystemExit("--greedy: the greedy baseline is built for scalar grids")
+        p.T_vamp = 0
+        greedy = {"greedy_init": 1}
     cfgd = describe(p, args.config, args.group_size)
+    if args.greedy:
+        cfgd["workload"] += " (greedy baseline: LDLQ init, damp 0.01, then the same CD)"
+        cfgd["init"] = "LDLQ"
     cfgd["cd_panel"] = args.cd_panel or "auto"
     m, n = p.m_out, p.n
     cb = p.codebook if p.d == 8 else None
@@ -323,14 +338,14 @@ def run_mpq(args, world, rank, local):
         z = np.load(cache)
         plan = mpq.Plan.from_spectrum(torch.from_numpy(z["s"]).to(dev),
                                       torch.from_numpy(z["V"]).to(dev), p.d, p.levels, codebook=cb,
-                                      cd_panel=args.cd_panel, group_size=args.group_size)
+                                      cd_panel=args.cd_panel, group_size=args.group_size, **greedy)
         setup_s = None
     else:
         X = torch.from_numpy(p.X).to(dev)
         torch.cuda.synchronize()
         t0 = time.time()
         plan = mpq.Plan.from_x(X, p.d, p.levels, codebook=cb, cd_panel=args.cd_panel,
-                               group_size=args.group_size)
+                               group_size=args.group_size, **greedy)
         torch.cuda.synchronize()
         setup_s = time.time() - t0
         del X
@@ -370,6 +385,7 @@ def run_mpq(args, world, rank, local):
             ev[i][1].record(stream)
         torch.cuda.synchronize()
     launches = mpq.kernel_launch_count() - launches0
+    objective = float(out["energy"].double().mean().item())
     barrier(world)
     mpq.profile_start()
     for i in range(args.steps):
@@ -465,7 +481,8 @@ def run_mpq(args, world, rank, local):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        times, t_spec = oracle_sample(p, args.cpu_rows, 1, args.group_size)
+        times, t_spec = oracle_sample(p, args.cpu_rows, 1, args.group_size,
+                                      0.01 if args.greedy else None)
         cpu = {"value": args.cpu_rows * n / times[0], "unit": UNIT,
                "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
                "sample": f"rows 0..{args.cpu_rows - 1} of the layer (independent problems), "
@@ -478,6 +495,8 @@ def run_mpq(args, world, rank, local):
                 "data": "synthetic", "config": dict(cfgd, setup_s=None if setup_s is None else round(setup_s, 3), rank=r,
                                                     parallelism=f"rows sharded over {world} GPU(s)"),
                 "rows_per_s": world * m / (ms_per_step / 1e3),
+                "objective": {"mean_energy": objective, "what": "mean over rows of "
+                              "1/2 |X (w - w_hat)|^2 after the timed solves"},
                 "roofline": roof, "solve_roofline": solve_roof, "cpu_baseline": cpu, "e2e": e2e,
                 "clocks": clk.summary(),
                 "gpu_launches": launches, "kernels": kernels}

@@ -19,7 +19,11 @@
  *                        rho_damp = 0.5, tau, S_CD = 3 with early stop,
  *                        gamma1_0 = 1/MSE(w, w_rtn), E8 d = 8, M_b = 2^16;
  *   [Main experiments]   (key experimental data) calibration on 128 C4
- *                        sequences of length 2048.
+ *                        sequences of length 2048;
+ *   [Motivation]         (research background) GPTQ, LDLQ and block CD as
+ *                        hard-decision solvers;
+ *   [Ablation]           (ablation table) T_vamp / CD-sweep settings,
+ *                        including the LDLQ and LDLQ + CD3 rows.
  * [ai.info findings] is the ai.info page on the same paper, its list of
  * findings (random Hadamard transforms and E_lin).
  * The min-max scalar grid follows the NeUQI note ("Near-Optimal Uniform
@@ -130,6 +134,21 @@ typedef struct {
                              grids) skip CD and keep the marginal MAP; their
                              cd_changes are 0.  The stage hook mpq_stage_cd
                              always runs CD. */
+  int32_t greedy_init;    /* the greedy baseline ([Motivation]: GPTQ / LDLQ
+                             commit each block to one codeword and pass its
+                             error on; [Ablation] rows "LDLQ" and "LDLQ +
+                             CD3").  0 (default): a solve with T_vamp = 0
+                             starts CD from round-to-nearest.  1: it starts
+                             from LDLQ instead -- columns in order, each
+                             rounded to its nearest level and its error fed
+                             to the later columns through the Cholesky
+                             factor of (H + lambda I)^-1, built at plan
+                             creation (fp64 on the device; n x n fp32 and fp16
+                             copies kept).  d = 1 only (MPQ_ERR_UNSUPPORTED
+                             for d = 8).  T_vamp > 0 is unaffected. */
+  double greedy_damp;     /* lambda = greedy_damp * mean(diag H), default 0.01;
+                             0 needs a full-rank H (else plan creation fails
+                             with MPQ_ERR_RANK). */
 } mpq_params;
 
 /* Fill `p` with the defaults above for block size d and codebook size K. */

@@ -44,7 +44,9 @@ class Params(C.Structure):
                 ("alpha_min", C.c_double), ("alpha_max", C.c_double),
                 ("vec_engine", C.c_int32), ("cd_panel", C.c_int32),
                 ("group_size", C.c_int32), ("solve_graphs", C.c_int32),
-                ("cd_skip_precision", C.c_double)]
+                ("cd_skip_precision", C.c_double),
+                ("greedy_init", C.c_int32),
+                ("greedy_damp", C.c_double)]
 
 
 class RowStats(C.Structure):

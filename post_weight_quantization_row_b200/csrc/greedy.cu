@@ -1,0 +1,354 @@
+// Greedy baseline: LDLQ / GPTQ on scalar grids (d = 1), batched over rows.
+//
+// Source: "MPQ: A Message-Passing View of Post-Training Quantization"
+// (papernotes.org note): the motivation (GPTQ and LDLQ commit each block to
+// one codeword at once and pass its hard error on to the blocks not yet
+// quantised) and the ablation table (LDLQ baseline: T_vamp = 0 and no CD;
+// LDLQ + CD3: the same init refined by three CD sweeps).
+//
+// Error feedback in the GPTQ form: with (H + lambda I)^-1 = L L^T (L the
+// lower Cholesky factor) and B = L diag(L)^-1 (unit lower), committing
+// column j to its nearest level q_j moves every later column k of the row by
+// -(v_j - q_j) B[k, j]; the uncommitted weights are then at their
+// least-squares optimum given the committed ones.  lambda = damp * mean(diag H).
+//
+// Setup, fp64: (H + lambda I)^-1 from the spectrum, V diag(1/(s^2 + lambda))
+// V^T, plus (I - V V^T)/lambda when r < n; then its Cholesky factor by a
+// blocked right-looking algorithm: per panel of 32 columns one warp factors
+// the diagonal block in shared memory, one kernel solves the rows below it
+// against it, and the fp64 SIMT GEMM updates the trailing matrix.
+//
+// Solve: the columns go in tiles of 128 inside L2-resident panels, as in the
+// last CD sweep.  One warp per row walks a tile column by column in registers
+// (the lane's 4 columns of the working row, the tile's block of B^T in shared
+// memory); the tile's errors leave, divided by the row's scale, as the fp16
+// hi/lo A operand of the tensor-core update W_work[:, ahead] -= E B[ahead, tile]^T.
+#include <math.h>
+
+#include <vector>
+
+#include "mpq_internal.cuh"
+
+namespace mpq {
+namespace {
+
+constexpr int CH_NB = 32;     // Cholesky panel width
+constexpr int CH_ROWS = 128;  // rows of the panel per CTA
+constexpr int LQ_WARPS = 16;  // rows per tile CTA
+constexpr int LQ_SLOTS = CD_TILE / 32;
+constexpr int LQ_SMEM = CD_TILE * CD_TILE * 4;
+
+unsigned grid_for(int64_t count) {
+  return (unsigned)std::min<int64_t>(cdiv(count, 256), 148 * 16);
+}
+
+// out = V diag(c), c_l = 1/(s_l^2 + lambda) - (full ? 0 : 1/lambda)
+__global__ void k_hinv_cols(const double* __restrict__ V, const double* __restrict__ s, int64_t n,
+                            int64_t r, double lam, int full, double* __restrict__ out) {
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n * r;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const double s2 = s[e % r] * s[e % r];
+    const double c = 1.0 / (s2 + lam) - (full ? 0.0 : 1.0 / lam);
+    out[e] = V[e] * c;
+  }
+}
+
+__global__ void k_add_diag(double* __restrict__ A, int64_t n, double v) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) A[i * n + i] += v;
+}
+
+// Diagonal block of the panel [k0, k0 + kb) of the blocked Cholesky, in
+// place: one warp, lane i owning row i (zeros written above the diagonal).
+// A pivot that is not positive sets *bad and continues with 1.
+__global__ void __launch_bounds__(32)
+    k_chol_diag(double* __restrict__ A, int64_t n, int64_t k0, int kb, int* __restrict__ bad) {
+  __shared__ double L11[CH_NB][CH_NB + 1];
+  const int t = threadIdx.x;
+  for (int e = t; e < CH_NB * CH_NB; e += 32) {
+    const int i = e / CH_NB, j = e % CH_NB;
+    L11[i][j] = (i < kb && j <= i) ? A[(k0 + i) * n + k0 + j] : (i == j ? 1.0 : 0.0);
+  }
+  __syncwarp();
+  for (int c = 0; c < kb; ++c) {
+    double d = L11[c][c];
+    if (!(d > 0.0)) {
+      if (t == c) *bad = 1;
+      d = 1.0;
+    }
+    const double sd = sqrt(d);
+    __syncwarp();
+    if (t == c) L11[c][c] = sd;
+    if (t > c && t < kb) L11[t][c] /= sd;
+    __syncwarp();
+    if (t > c && t < kb)
+      for (int j = c + 1; j <= t; ++j) L11[t][j] -= L11[t][c] * L11[j][c];
+    __syncwarp();
+  }
+  if (t < kb)
+    for (int j = 0; j < kb; ++j) A[(k0 + t) * n + k0 + j] = j <= t ? L11[t][j] : 0.0;
+}
+
+// Rows below the factored diagonal block: every thread takes one row and
+// solves x L11^T = A[row, panel] by forward substitution, in place.
+__global__ void __launch_bounds__(CH_ROWS)
+    k_chol_panel(double* __restrict__ A, int64_t n, int64_t k0, int kb) {
+  __shared__ double L11[CH_NB][CH_NB + 1];
+  const int t = threadIdx.x;
+  for (int e = t; e < CH_NB * CH_NB; e += blockDim.x) {
+    const int i = e / CH_NB, j = e % CH_NB;
+    L11[i][j] = (i < kb && j <= i) ? A[(k0 + i) * n + k0 + j] : (i == j ? 1.0 : 0.0);
+  }
+  __syncthreads();
+  const int64_t row = k0 + kb + (int64_t)blockIdx.x * CH_ROWS + t;
+  if (row >= n) return;
+  double* Ar = A + row * n + k0;
+  double x[CH_NB];
+#pragma unroll
+  for (int j = 0; j < CH_NB; ++j) {
+    x[j] = 0.0;
+    if (j < kb) {
+      double v = Ar[j];
+#pragma unroll
+      for (int q = 0; q < j; ++q) v -= x[q] * L11[j][q];
+      x[j] = v / L11[j][j];
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < CH_NB; ++j)
+    if (j < kb) Ar[j] = x[j];
+}
+
+// out (M x kb, contiguous) = -A[r0.., c0 .. c0 + kb)
+__global__ void k_neg_panel(const double* __restrict__ A, int64_t n, int64_t r0, int64_t c0,
+                            int64_t M, int kb, double* __restrict__ out) {
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < M * kb;
+       e += (int64_t)gridDim.x * blockDim.x)
+    out[e] = -A[(r0 + e / kb) * n + c0 + e % kb];
+}
+
+// B = L diag(L)^-1 (fp32, n x n, zero above the diagonal) and, per tile of
+// CD_TILE columns, the tile's diagonal block of B^T (unit upper):
+// Ud[tile][j][c] = B[c][j] for columns j, c of the tile.
+__global__ void k_ldlq_factors(const double* __restrict__ Lf, int64_t n, float* __restrict__ Bl,
+                               float* __restrict__ Ud) {
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n * n;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t c = e / n, j = e % n;
+    const float v = j < c ? (float)(Lf[e] / Lf[j * n + j]) : (j == c ? 1.0f : 0.0f);
+    Bl[e] = v;
+    if (c / CD_TILE == j / CD_TILE)
+      Ud[(j / CD_TILE) * CD_TILE * CD_TILE + (j % CD_TILE) * CD_TILE + c % CD_TILE] = v;
+  }
+}
+
+// One tile [t0, t0 + tw) of the greedy pass for a warp per row.  Lane l holds
+// columns l, l + 32, l + 64, l + 96 of the working row v (W plus the feedback
+// of every earlier tile).  Column j: its owner rounds v_j to the nearest level
+// (the lower on an exact half, clamped to the grid), the error e = v_j - q_j
+// goes to all lanes, and every later column moves by -e B[c, j] (row j of the
+// tile's unit upper block: 1 on the diagonal, zeros before it, so the owner's
+// own value just becomes q_j).  The errors leave as e / aref in the A operand
+// (aref = the row's scale, or its largest group scale), with -aref as the
+// operand's row factor.
+__global__ void __launch_bounds__(LQ_WARPS * 32, 2)
+    k_ldlq_tile(int64_t m, int64_t n, int L, int64_t t0, int tw, const float* __restrict__ scale,
+                const float* __restrict__ offset, int ng, int gi, const float* __restrict__ sref,
+                const float* __restrict__ Ud_tile, const float* __restrict__ Wk, int64_t ldw,
+                uint16_t* __restrict__ idx, __half* __restrict__ dhi, __half* __restrict__ dlo,
+                int64_t lda, float* __restrict__ d_unscale) {
+  extern __shared__ float lq_smem[];
+  {
+    const float4* src = reinterpret_cast<const float4*>(Ud_tile);
+    float4* dst = reinterpret_cast<float4*>(lq_smem);
+    for (int e = threadIdx.x; e < CD_TILE * CD_TILE / 4; e += blockDim.x) dst[e] = src[e];
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int64_t row = (int64_t)blockIdx.x * LQ_WARPS + wid;
+  if (row >= m) return;
+  const float sc = scale[row * ng + gi], off = offset[row * ng + gi];
+  const float aref = sref ? sref[row] : sc;
+  const float inv_a = 1.0f / aref;
+  if (lane == 0) d_unscale[row] = -aref;
+  const float* wr = Wk + row * ldw + t0;
+  const float Lm1 = (float)(L - 1);
+  float v[LQ_SLOTS], a[LQ_SLOTS];
+  int k[LQ_SLOTS];
+#pragma unroll
+  for (int q = 0; q < LQ_SLOTS; ++q) {
+    const int col = 32 * q + lane;
+    v[q] = col < tw ? wr[col] : 0.0f;
+    a[q] = 0.0f;
+    k[q] = 0;
+  }
+#pragma unroll
+  for (int q = 0; q < LQ_SLOTS; ++q) {
+    if (32 * q >= tw) break;
+    const int cnt = min(32, tw - 32 * q);
+    for (int jj = 0; jj < cnt; ++jj) {
+      float e = 0.0f;
+      if (lane == jj) {
+        const float t = (v[q] - off) / sc;
+        const float kk = fminf(fmaxf(ceil_small(t - 0.5f), 0.0f), Lm1);
+        k[q] = (int)kk;
+        e = v[q] - fmaf(sc, kk, off);
+        a[q] = e * inv_a;
+      }
+      e = __shfl_sync(0xffffffffu, e, jj);
+      const float* Uj = lq_smem + (32 * q + jj) * CD_TILE + lane;
+#pragma unroll
+      for (int qq = q; qq < LQ_SLOTS; ++qq) v[qq] = fmaf(-e, Uj[32 * qq], v[qq]);
+    }
+  }
+  uint16_t* ir = idx + row * n + t0;
+  __half* drow_hi = dhi + row * lda;
+  __half* drow_lo = dlo + row * lda;
+#pragma unroll
+  for (int q = 0; q < LQ_SLOTS; ++q) {
+    const int col = 32 * q + lane;
+    if (col < tw) ir[col] = (uint16_t)k[q];
+    const __half h = __float2half_rn(a[q]);
+    drow_hi[col] = h;
+    drow_lo[col] = __float2half_rn(a[q] - __half2float(h));
+  }
+}
+
+}  // namespace
+
+mpq_status ldlq_factor(const mpq_plan_s* p, double damp, float* Bl, float* Ud, cudaStream_t st) {
+  const int64_t n = p->n, r = p->r;
+  std::vector<double> hs(r);
+  MPQ_CUDA(cudaMemcpyAsync(hs.data(), p->s64, sizeof(double) * r, cudaMemcpyDeviceToHost, st));
+  MPQ_CUDA(cudaStreamSynchronize(st));
+  double tr = 0.0;  // trace(H) = sum s^2 (V has orthonormal columns)
+  for (double v : hs) tr += v * v;
+  const double lam = damp * tr / (double)n;
+  if (!(lam > 0.0) && r < n)
+    return fail(MPQ_ERR_RANK, "greedy baseline: H is singular (rank < n); set greedy_damp > 0");
+  const bool full = r == n;
+  double *Vc = nullptr, *A = nullptr, *neg = nullptr;
+  int* bad = nullptr;
+  mpq_status rc = MPQ_OK;
+  auto cuda_ok = [&](cudaError_t e, const char* what) {
+    if (rc == MPQ_OK && e != cudaSuccess) rc = cuda_fail(e, what);
+    return rc == MPQ_OK;
+  };
+  cuda_ok(cudaMallocAsync(&Vc, sizeof(double) * n * r, st), "ldlq alloc");
+  cuda_ok(cudaMallocAsync(&A, sizeof(double) * n * n, st), "ldlq alloc");
+  cuda_ok(cudaMallocAsync(&neg, sizeof(double) * n * CH_NB, st), "ldlq alloc");
+  cuda_ok(cudaMallocAsync(&bad, sizeof(int), st), "ldlq alloc");
+  if (rc == MPQ_OK) cuda_ok(cudaMemsetAsync(bad, 0, sizeof(int), st), "ldlq memset");
+  if (rc == MPQ_OK) {
+    {
+      ProfScope ps_("k_hinv_cols", st);
+      k_hinv_cols<<<grid_for(n * r), 256, 0, st>>>(p->V64, p->s64, n, r, lam, full ? 1 : 0, Vc);
+    }
+    count_launch();
+    rc = check_launch("k_hinv_cols");
+  }
+  if (rc == MPQ_OK) rc = gemm_nt_f64(Vc, r, p->V64, r, A, n, n, n, r, st);  // V diag(c) V^T
+  if (rc == MPQ_OK && !full) {
+    {
+      ProfScope ps_("k_add_diag", st);
+      k_add_diag<<<(unsigned)cdiv(n, 256), 256, 0, st>>>(A, n, 1.0 / lam);
+    }
+    count_launch();
+    rc = check_launch("k_add_diag");
+  }
+  for (int64_t k0 = 0; k0 < n && rc == MPQ_OK; k0 += CH_NB) {
+    const int kb = (int)std::min<int64_t>(CH_NB, n - k0);
+    {
+      ProfScope ps_("k_chol_diag", st);
+      k_chol_diag<<<1, 32, 0, st>>>(A, n, k0, kb, bad);
+    }
+    count_launch();
+    rc = check_launch("k_chol_diag");
+    const int64_t r0 = k0 + kb, M = n - r0;
+    if (rc != MPQ_OK || M <= 0) continue;
+    {
+      ProfScope ps_("k_chol_panel", st);
+      k_chol_panel<<<(unsigned)cdiv(M, CH_ROWS), CH_ROWS, 0, st>>>(A, n, k0, kb);
+    }
+    count_launch();
+    rc = check_launch("k_chol_panel");
+    if (rc != MPQ_OK) continue;
+    {
+      ProfScope ps_("k_neg_panel", st);
+      k_neg_panel<<<grid_for(M * kb), 256, 0, st>>>(A, n, r0, k0, M, kb, neg);
+    }
+    count_launch();
+    rc = check_launch("k_neg_panel");
+    // A22 += (-L21) L21^T
+    if (rc == MPQ_OK)
+      rc = gemm_nt_f64(neg, kb, A + r0 * n + k0, n, A + r0 * n + r0, n, M, M, kb, st, true);
+  }
+  if (rc == MPQ_OK) {
+    {
+      ProfScope ps_("k_ldlq_factors", st);
+      k_ldlq_factors<<<grid_for(n * n), 256, 0, st>>>(A, n, Bl, Ud);
+    }
+    count_launch();
+    rc = check_launch("k_ldlq_factors");
+  }
+  int hbad = 0;
+  if (rc == MPQ_OK) cuda_ok(cudaMemcpyAsync(&hbad, bad, sizeof(int), cudaMemcpyDeviceToHost, st), "ldlq flag");
+  if (rc == MPQ_OK) cuda_ok(cudaStreamSynchronize(st), "ldlq sync");
+  if (Vc) cudaFreeAsync(Vc, st);
+  if (A) cudaFreeAsync(A, st);
+  if (neg) cudaFreeAsync(neg, st);
+  if (bad) cudaFreeAsync(bad, st);
+  if (rc == MPQ_OK && hbad)
+    return fail(MPQ_ERR_RANK, "greedy baseline: (H + lambda I)^-1 is not positive definite in fp64");
+  return rc;
+}
+
+mpq_status launch_ldlq(mpq_plan_s* p, const float* W, int64_t m, const float* scale,
+                       const float* offset, uint16_t* idx, cudaStream_t st) {
+  if (m <= 0) return MPQ_OK;
+  if (!p->ldlq_diag) return fail(MPQ_ERR_INVALID_ARG, "the plan was created without greedy_init");
+  Workspace& w = p->ws;
+  const int64_t n = p->n;
+  // working rows W_work = W, in the CD gradient buffer (free until CD starts)
+  MPQ_CUDA(cudaMemcpy2DAsync(w.Hg, sizeof(float) * w.ldh, W, sizeof(float) * n, sizeof(float) * n,
+                             m, cudaMemcpyDeviceToDevice, st));
+  if (p->G) MPQ_TRY(launch_row_max(scale, m, p->ng, w.sref, st));
+  const int64_t P = p->params.cd_panel > 0 ? std::min<int64_t>(p->params.cd_panel, round_up(n, CD_TILE))
+                                           : cd_panel_cols(m, n);
+  const int np = (int)cdiv(n, P);
+  MPQ_CUDA(cudaFuncSetAttribute(k_ldlq_tile, cudaFuncAttributeMaxDynamicSharedMemorySize, LQ_SMEM));
+  auto update = [&](int64_t a_k0, int64_t b_k0, int64_t K, int64_t c0, int64_t c1,
+                    const char* tag) -> mpq_status {
+    if (c1 <= c0) return MPQ_OK;
+    GemmOpts o;
+    o.a_k0 = a_k0;
+    o.b_k0 = b_k0;
+    o.n0 = c0;
+    o.accumulate = true;
+    o.c_reduce = &w.tm_hg;
+    return gemm_tc(w.As, w.tm_an_hi, w.tm_an_lo, p->Lq_s, p->tm_lq_hi, p->tm_lq_lo, w.Hg, w.ldh, m,
+                   c1 - c0, K, p->Lq_s.unscale_host, p->status, st, tag, o);
+  };
+  for (int pi = 0; pi < np; ++pi) {
+    const int64_t ps = (int64_t)pi * P, pe = std::min<int64_t>(n, ps + P);
+    for (int64_t t0 = ps; t0 < pe; t0 += CD_TILE) {
+      const int tw = (int)std::min<int64_t>(CD_TILE, n - t0);
+      {
+        ProfScope ps_("k_ldlq_tile", st);
+        k_ldlq_tile<<<(unsigned)cdiv(m, LQ_WARPS), LQ_WARPS * 32, LQ_SMEM, st>>>(
+            m, n, p->K, t0, tw, scale, offset, (int)p->ng, p->G ? (int)(t0 / p->G) : 0,
+            p->G ? w.sref : nullptr, p->ldlq_diag + (t0 / CD_TILE) * CD_TILE * CD_TILE, w.Hg,
+            w.ldh, idx, w.As.hi + (t0 - ps), w.As.lo + (t0 - ps), w.As.ld, w.As.row_unscale);
+      }
+      count_launch();
+      MPQ_TRY(check_launch("k_ldlq_tile"));
+      // later columns of the panel
+      MPQ_TRY(update(t0 - ps, t0, tw, t0 + tw, pe, "gemm_ldlq_update"));
+    }
+    // every column after the panel
+    if (np > 1) MPQ_TRY(update(0, ps, pe - ps, pe, n, "gemm_ldlq_panel"));
+  }
+  return MPQ_OK;
+}
+
+}  // namespace mpq

@@ -8,6 +8,7 @@
 
 #include <algorithm>
 #include <atomic>
+#include <cmath>
 #include <map>
 #include <mutex>
 #include <string>
@@ -135,6 +136,12 @@ mpq_status validate_params(const mpq_params* q, int64_t n) {
     return fail(MPQ_ERR_INVALID_ARG, "solve_graphs must be 0 or 1");
   if (!(q->cd_skip_precision >= 0.0))
     return fail(MPQ_ERR_INVALID_ARG, "cd_skip_precision must be >= 0 (0: never skip)");
+  if (q->greedy_init != 0 && q->greedy_init != 1)
+    return fail(MPQ_ERR_INVALID_ARG, "greedy_init must be 0 or 1");
+  if (!(q->greedy_damp >= 0.0) || !std::isfinite(q->greedy_damp))
+    return fail(MPQ_ERR_INVALID_ARG, "greedy_damp must be finite and >= 0");
+  if (q->greedy_init && q->d != 1)
+    return fail(MPQ_ERR_UNSUPPORTED, "the greedy baseline is built for scalar grids (d = 1)");
   if (q->group_size < 0 || (q->group_size > 0 && (q->d != 1 || q->group_size % 128 ||
                                                    n % q->group_size)))
     return fail(MPQ_ERR_INVALID_ARG,
@@ -407,6 +414,9 @@ mpq_status solve_batch(mpq_plan_s* p, const SolveIO& io, int64_t row0, int64_t m
       MPQ_TRY(launch_denoise(p, R1, w.gamma1, w.scale, w.offset, mb, W, w.gamma1_0, w.X1, vblock,
                              w.vsum, idx, st));
   }
+  // the greedy baseline replaces round-to-nearest as the hard init
+  if (io.T_vamp == 0 && p->params.greedy_init)
+    MPQ_TRY(launch_ldlq(p, W, mb, w.scale, w.offset, idx, st));
   if (io.sweeps > 0)
     MPQ_TRY(run_cd(p, W, mb, w.scale, w.offset, idx, io.sweeps, changes, st, w.gamma1));
   MPQ_TRY(run_energy(p, W, mb, w.scale, w.offset, idx, io.w_hat ? io.w_hat + row0 * n : nullptr,
@@ -532,6 +542,26 @@ mpq_status finish_plan(mpq_plan_s* p, cudaStream_t st) {
   MPQ_TRY(make_tmap_f16(&p->tm_v_lo, p->V_s.lo, p->V_s.ld, p->V_s.rows_pad, p->V_s.ld, 128));
   MPQ_TRY(make_tmap_f16(&p->tm_h_hi, p->H_s.hi, p->H_s.ld, p->H_s.rows_pad, p->H_s.ld, 128));
   MPQ_TRY(make_tmap_f16(&p->tm_h_lo, p->H_s.lo, p->H_s.ld, p->H_s.rows_pad, p->H_s.ld, 128));
+  if (p->params.greedy_init) {
+    const int64_t nt = cdiv(n, CD_TILE);
+    MPQ_TRY(dalloc(&p->ldlq_diag, nt * CD_TILE * CD_TILE));
+    MPQ_CUDA(cudaMemsetAsync(p->ldlq_diag, 0, sizeof(float) * nt * CD_TILE * CD_TILE, st));
+    float* Bl = nullptr;
+    MPQ_TRY(dalloc(&Bl, n * n));
+    mpq_status rc = ldlq_factor(p, p->params.greedy_damp, Bl, p->ldlq_diag, st);
+    if (rc == MPQ_OK) rc = alloc_split(p->Lq_s, n, n, false);
+    if (rc == MPQ_OK) rc = split_global(Bl, n, n, &p->Lq_s, st);
+    if (rc == MPQ_OK) {
+      cudaError_t e = cudaMemcpyAsync(&p->Lq_s.unscale_host, p->Lq_s.unscale, sizeof(float),
+                                      cudaMemcpyDeviceToHost, st);
+      if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+      if (e != cudaSuccess) rc = cuda_fail(e, "greedy factor");
+    }
+    dfree(Bl);
+    MPQ_TRY(rc);
+    MPQ_TRY(make_tmap_f16(&p->tm_lq_hi, p->Lq_s.hi, p->Lq_s.ld, p->Lq_s.rows_pad, p->Lq_s.ld, 128));
+    MPQ_TRY(make_tmap_f16(&p->tm_lq_lo, p->Lq_s.lo, p->Lq_s.ld, p->Lq_s.rows_pad, p->Lq_s.ld, 128));
+  }
   if (p->d == 8) {
     MPQ_TRY(dalloc(&p->cb_norm, p->K));
     MPQ_TRY(dalloc(&p->qtab, p->B * (int64_t)p->K));
@@ -557,7 +587,8 @@ void destroy_plan(mpq_plan_s* p) {
   dfree(p->s64); dfree(p->V64); dfree(p->s32); dfree(p->V32); dfree(p->Vt32); dfree(p->H32);
   dfree(p->Hdiag); dfree(p->cb); dfree(p->cb_norm); dfree(p->qtab); dfree(p->status);
   if (p->cb_tc) cudaFree(p->cb_tc);
-  free_split(p->Vt_s); free_split(p->V_s); free_split(p->H_s);
+  free_split(p->Vt_s); free_split(p->V_s); free_split(p->H_s); free_split(p->Lq_s);
+  dfree(p->ldlq_diag);
   delete p;
 }
 
@@ -627,6 +658,8 @@ void mpq_params_default(mpq_params* p, int32_t d, int32_t K) {
   p->group_size = 0;
   p->solve_graphs = 1;
   p->cd_skip_precision = 0.0;
+  p->greedy_init = 0;
+  p->greedy_damp = 0.01;
 }
 
 mpq_status mpq_plan_create_from_spectrum(const double* s, const double* V, int64_t n, int64_t r,

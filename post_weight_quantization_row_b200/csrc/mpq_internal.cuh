@@ -121,6 +121,10 @@ struct mpq_plan_s {
   // B operands of the tensor-core GEMMs
   mpq::SplitOperand Vt_s, V_s, H_s;
   CUtensorMap tm_vt_hi, tm_vt_lo, tm_v_hi, tm_v_lo, tm_h_hi, tm_h_lo;
+  // greedy baseline (LDLQ), built when params.greedy_init is set (d = 1)
+  float* ldlq_diag = nullptr;  // per tile of CD_TILE columns: its diagonal block of B^T
+  mpq::SplitOperand Lq_s;      // B = L diag(L)^-1 (n x n), (H + lambda I)^-1 = L L^T
+  CUtensorMap tm_lq_hi, tm_lq_lo;
   // vector codebook (d = 8)
   float* cb = nullptr;       // K x 8
   float* cb_norm = nullptr;  // K  |c|^2
@@ -222,6 +226,13 @@ constexpr int64_t CD_PANEL_BYTES = 32ll << 20;  // L2-resident slab of the CD gr
 constexpr int64_t CD_PANEL_MIN = 512;           // narrowest CD panel (columns)
 int64_t cd_panel_cols(int64_t m, int64_t n);
 mpq_status launch_row_max(const float* scale, int64_t m, int64_t ng, float* out, cudaStream_t st);
+
+// greedy baseline (greedy.cu): the factors of (H + lambda I)^-1, lambda =
+// damp * mean(diag H), into Bl (n x n fp32) and Ud (tiles x CD_TILE^2 fp32,
+// zeroed by the caller); and the LDLQ pass of m rows into idx
+mpq_status ldlq_factor(const mpq_plan_s* p, double damp, float* Bl, float* Ud, cudaStream_t st);
+mpq_status launch_ldlq(mpq_plan_s* p, const float* W, int64_t m, const float* scale,
+                       const float* offset, uint16_t* idx, cudaStream_t st);
 mpq_status launch_check_finite(const float* x, int64_t count, int* status, cudaStream_t st);
 
 // tensor-core GEMM (gemm_tc.cu): C = diag(A.row_unscale) (A B^T) * b_scale

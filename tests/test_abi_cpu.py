@@ -41,13 +41,16 @@ def test_params_default(mpq):
     assert p.alpha_min == 1e-10 and p.alpha_max == 0.99
     assert p.vec_engine == 0 and p.cd_panel == 0 and p.solve_graphs == 1 and p.group_size == 0
     assert p.cd_skip_precision == 0.0
+    assert p.greedy_init == 0 and p.greedy_damp == 0.01
 
 
 @pytest.mark.parametrize("field,value", [("d", 3), ("K", 1), ("damping", 1.5), ("beta0", -1.0),
                                          ("tau", 0.0), ("alpha_max", 1.0), ("vec_engine", 3),
                                          ("cd_panel", 100), ("cd_panel", -128),
                                          ("solve_graphs", 2), ("group_size", 100),
-                                         ("group_size", -128), ("cd_skip_precision", -1.0)])
+                                         ("group_size", -128), ("cd_skip_precision", -1.0),
+                                         ("greedy_init", 2), ("greedy_damp", -0.5),
+                                         ("greedy_damp", math.inf)])
 def test_bad_params_rejected_without_a_device(mpq, field, value):
     p = mpq.Params()
     mpq.lib.mpq_params_default(C.byref(p), 1, 8)

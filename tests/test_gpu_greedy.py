@@ -1,0 +1,111 @@
+"""Parity of the greedy baseline (LDLQ on scalar grids, the T_vamp = 0 init
+of plans created with greedy_init = 1) with the float64 oracle.
+
+Cases span several 128-column tiles with a ragged tail, one panel and
+several panels (cd_panel = 128), group-wise grids, and a rank-deficient X
+(damped factor).  Bars: every decision before a row's first near-tie of the
+oracle (top-two distance gap below 1e-3 grid units^2) is exact, rows without
+one match index for index, and their energies are within 1e-3; after CD the
+whole-solve rules of the other parity tests apply."""
+import numpy as np
+import pytest
+
+import mpq_inputs as mi
+from oracle import mpq_oracle as orc
+from tests.helpers import codebook_for, cu, host, idx_np, oracle_grid_f32, spectrum_cuda
+
+pytestmark = pytest.mark.gpu
+
+TIE = 1e-3
+ENERGY_TOL = 1e-3
+
+
+@pytest.fixture(scope="module")
+def mpq():
+    import post_weight_quantization_row_b200 as m
+    return m
+
+
+def grid(p, group):
+    if group:
+        sc, off = orc.minmax_grid(p.W, p.levels, group)
+        return sc.astype(np.float32), off.astype(np.float32)
+    return oracle_grid_f32(p)
+
+
+def check_greedy(mpq, p, group=0, damp=0.01, cd_panel=0, sweeps=0, min_clean=0.5):
+    s, V, s_cu, V_cu = spectrum_cuda(p.X)
+    plan = mpq.Plan.from_spectrum(s_cu, V_cu, 1, p.levels, greedy_init=1, greedy_damp=damp,
+                                  cd_panel=cd_panel, group_size=group)
+    sc, off = grid(p, group)
+    cb = codebook_for(p)
+    sc64, off64 = sc.astype(np.float64), off.astype(np.float64)
+    g = orc.ldlq(p.W, cb, sc64, off64, orc.hessian(s, V), damp)
+    out = plan.solve(cu(p.W), 0, sweeps, row_scale=cu(sc), row_offset=cu(off), stats=True)
+    got = idx_np(out["idx"])
+    e = host(out["energy"]).astype(np.float64)
+    if sweeps == 0:
+        near = g.gap < TIE
+        clean = ~near.any(axis=1)
+        assert clean.mean() >= min_clean, f"only {clean.mean():.2f} of rows free of near-ties"
+        for i in range(p.m_out):
+            first = int(np.argmax(near[i])) if near[i].any() else p.n
+            assert np.array_equal(got[i, :first], g.idx[i, :first]), (i, first)
+        E = orc.energy(p.W, orc.decode(g.idx, cb, sc64, off64), s, V)
+        assert np.all(np.abs(e[clean] - E[clean]) <= ENERGY_TOL * E[clean])
+        return g, out
+    ref = orc.solve(p.W, cb, s, V, 0, sweeps, sc64, off64, greedy_damp=damp, group=group)
+    clean = np.all(ref.map_gap > TIE, axis=1) & (ref.cd.first_tie < 0)
+    assert clean.mean() >= min_clean, f"only {clean.mean():.2f} of rows free of near-ties"
+    assert np.array_equal(got[clean], ref.idx[clean])
+    assert np.all(np.abs(e[clean] - ref.energy[clean]) <= ENERGY_TOL * ref.energy[clean])
+    assert abs(e.sum() - ref.energy.sum()) <= 1e-2 * ref.energy.sum()
+    return ref, out
+
+
+@pytest.mark.parametrize("cd_panel", [0, 128])
+def test_greedy_ragged_tiles(mpq, cd_panel):
+    # n = 300: tiles of 128, 128 and 44; cd_panel = 128 makes every tile a panel
+    p = mi.small_problem(701, 37, 300, 500, d=1, levels=8, T_vamp=0, cd_sweeps=0)
+    check_greedy(mpq, p, cd_panel=cd_panel)
+
+
+def test_greedy_4bit_many_rows(mpq):
+    # 300 rows: more than one CTA of rows per tile
+    p = mi.small_problem(702, 300, 256, 400, d=1, levels=16, T_vamp=0, cd_sweeps=0)
+    check_greedy(mpq, p, min_clean=0.4)
+
+
+def test_greedy_group_grids(mpq):
+    p = mi.small_problem(703, 21, 384, 600, d=1, levels=8, T_vamp=0, cd_sweeps=0)
+    check_greedy(mpq, p, group=128)
+
+
+def test_greedy_rank_deficient_x(mpq):
+    # m_calib < n: H is singular, the damped factor still exists
+    p = mi.small_problem(704, 19, 256, 120, d=1, levels=8, T_vamp=0, cd_sweeps=0)
+    check_greedy(mpq, p, damp=0.05)
+
+
+def test_greedy_then_cd(mpq):
+    p = mi.small_problem(705, 37, 300, 500, d=1, levels=8, T_vamp=0, cd_sweeps=3)
+    check_greedy(mpq, p, sweeps=3, min_clean=0.25)
+
+
+def test_greedy_undamped_singular_h_is_rejected(mpq):
+    p = mi.small_problem(706, 3, 128, 60, d=1, levels=8)
+    _, _, s_cu, V_cu = spectrum_cuda(p.X)
+    with pytest.raises(mpq.MPQError) as e:
+        mpq.Plan.from_spectrum(s_cu, V_cu, 1, p.levels, greedy_init=1, greedy_damp=0.0)
+    assert e.value.status == 5
+
+
+def test_greedy_does_not_touch_vamp_solves(mpq):
+    # T_vamp > 0 ignores greedy_init: same result as a plan without it
+    p = mi.small_problem(707, 9, 256, 400, d=1, levels=8, T_vamp=3, cd_sweeps=2)
+    _, _, s_cu, V_cu = spectrum_cuda(p.X)
+    a = mpq.Plan.from_spectrum(s_cu, V_cu, 1, p.levels, greedy_init=1)
+    b = mpq.Plan.from_spectrum(s_cu, V_cu, 1, p.levels)
+    oa = a.solve(cu(p.W), 3, 2)
+    ob = b.solve(cu(p.W), 3, 2)
+    assert np.array_equal(idx_np(oa["idx"]), idx_np(ob["idx"]))
