@@ -60,8 +60,8 @@ def parse():
                     help="scalar workloads: one min-max grid per group of this many columns "
                          "(0 = one per row)")
     ap.add_argument("--greedy", action="store_true",
-                    help="scalar workloads: the greedy baseline (LDLQ init, T_vamp = 0) with the "
-                         "same CD sweeps instead of MPQ")
+                    help="the greedy baseline (LDLQ init, T_vamp = 0) with the same CD sweeps "
+                         "instead of MPQ")
     ap.add_argument("--spectrum-cache", default=None,
                     help="npz file: reuse the spectrum a previous run computed on the device")
     return ap.parse_args()
@@ -322,8 +322,6 @@ def run_mpq(args, world, rank, local):
         p.W = np.ascontiguousarray(p.W[:args.rows])
     greedy = {}
     if args.greedy:
-        if p.d != 1:
-            raise SystemExit("--greedy: the greedy baseline is built for scalar grids")
         p.T_vamp = 0
         greedy = {"greedy_init": 1}
     cfgd = describe(p, args.config, args.group_size)

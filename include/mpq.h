@@ -139,13 +139,14 @@ typedef struct {
                              error on; [Ablation] rows "LDLQ" and "LDLQ +
                              CD3").  0 (default): a solve with T_vamp = 0
                              starts CD from round-to-nearest.  1: it starts
-                             from LDLQ instead -- columns in order, each
-                             rounded to its nearest level and its error fed
-                             to the later columns through the Cholesky
-                             factor of (H + lambda I)^-1, built at plan
-                             creation (fp64 on the device; n x n fp32 and fp16
-                             copies kept).  d = 1 only (MPQ_ERR_UNSUPPORTED
-                             for d = 8).  T_vamp > 0 is unaffected. */
+                             from LDLQ instead -- blocks in order, each
+                             committed to its nearest level (d = 1) or
+                             nearest codeword in the Euclidean metric
+                             (d = 8), its error fed to the later columns
+                             through the Cholesky factor of
+                             (H + lambda I)^-1, built at plan creation (fp64
+                             on the device; n x n fp32 and fp16 copies kept).
+                             T_vamp > 0 is unaffected. */
   double greedy_damp;     /* lambda = greedy_damp * mean(diag H), default 0.01;
                              0 needs a full-rank H (else plan creation fails
                              with MPQ_ERR_RANK). */

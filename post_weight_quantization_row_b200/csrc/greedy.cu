@@ -1,4 +1,5 @@
-// Greedy baseline: LDLQ / GPTQ on scalar grids (d = 1), batched over rows.
+// Greedy baseline: LDLQ / GPTQ, batched over rows (scalar grids and d = 8
+// codebooks).
 //
 // Source: "MPQ: A Message-Passing View of Post-Training Quantization"
 // (papernotes.org note): the motivation (GPTQ and LDLQ commit each block to
@@ -214,6 +215,141 @@ __global__ void __launch_bounds__(LQ_WARPS * 32, 2)
   }
 }
 
+// ---------------------------------------------------------------- d = 8 --
+// Block b of a tile: the codeword nearest (Euclidean, in codebook units) the
+// block's current working values, t = v_b / scale: argmin_c 1/2 |c|^2 - c.t
+// (lowest index on ties).  Kernel A scans one chunk of LQ8_CHUNK codewords
+// for LQ8_ROWS rows (a thread per row, the chunk in shared memory, read by
+// broadcast); kernel B (a warp per row) combines the chunk minima, commits
+// the codeword, and feeds the block's 8 errors, one column after another, to
+// the later columns of the tile through the block's 8 rows of B^T.
+constexpr int LQ8_CHUNK = 256;  // small chunks: >= 256 CTAs per scan at K = 65536
+constexpr int LQ8_ROWS = 256;
+constexpr int LQ8_APPLY_WARPS = 16;
+
+__global__ void __launch_bounds__(LQ8_ROWS)
+    k_ldlq8_eval(int64_t m, int K, int64_t b, const float* __restrict__ cb,
+                 const float* __restrict__ cb_norm, const float* __restrict__ scale,
+                 const float* __restrict__ Wk, int64_t ldw, float* __restrict__ part_val,
+                 int* __restrict__ part_idx, int nchunks) {
+  __shared__ float4 s_cb[LQ8_CHUNK * 2];  // codeword c: s_cb[2c], s_cb[2c + 1]
+  __shared__ float s_half_norm[LQ8_CHUNK];
+  const int chunk = blockIdx.x;
+  const int c0 = chunk * LQ8_CHUNK;
+  const int cnt = min(LQ8_CHUNK, K - c0);
+  for (int e = threadIdx.x; e < cnt * 8; e += blockDim.x)
+    reinterpret_cast<float*>(s_cb)[e] = cb[(int64_t)c0 * 8 + e];
+  for (int e = threadIdx.x; e < cnt; e += blockDim.x) s_half_norm[e] = 0.5f * cb_norm[c0 + e];
+  __syncthreads();
+  const int64_t row = (int64_t)blockIdx.y * LQ8_ROWS + threadIdx.x;
+  if (row >= m) return;
+  const float inv = 1.0f / scale[row];
+  float t[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) t[j] = Wk[row * ldw + 8 * b + j] * inv;
+  float best = INFINITY;
+  int bi = 0;
+  for (int c = 0; c < cnt; ++c) {
+    const float4 a = s_cb[2 * c], b4 = s_cb[2 * c + 1];
+    float sc = s_half_norm[c];
+    sc = fmaf(-a.x, t[0], sc);
+    sc = fmaf(-a.y, t[1], sc);
+    sc = fmaf(-a.z, t[2], sc);
+    sc = fmaf(-a.w, t[3], sc);
+    sc = fmaf(-b4.x, t[4], sc);
+    sc = fmaf(-b4.y, t[5], sc);
+    sc = fmaf(-b4.z, t[6], sc);
+    sc = fmaf(-b4.w, t[7], sc);
+    if (sc < best) {
+      best = sc;
+      bi = c;
+    }
+  }
+  part_val[row * nchunks + chunk] = best;
+  part_idx[row * nchunks + chunk] = c0 + bi;
+}
+
+__global__ void __launch_bounds__(LQ8_APPLY_WARPS * 32)
+    k_ldlq8_apply(int64_t m, int64_t n, int K, int64_t b, int64_t t0, int tw,
+                  const float* __restrict__ cb, const float* __restrict__ scale,
+                  const float* __restrict__ Ud_tile, float* __restrict__ Wk, int64_t ldw,
+                  uint16_t* __restrict__ idx, const float* __restrict__ part_val,
+                  const int* __restrict__ part_idx, int nchunks, __half* __restrict__ dhi,
+                  __half* __restrict__ dlo, int64_t lda, float* __restrict__ d_unscale) {
+  __shared__ float s_u[8][CD_TILE];  // the block's rows of the tile's unit upper block
+  const int jl0 = (int)(8 * b - t0);  // tile-local first column of the block
+  for (int e = threadIdx.x; e < 8 * CD_TILE; e += blockDim.x)
+    s_u[e / CD_TILE][e % CD_TILE] = Ud_tile[(int64_t)(jl0 + e / CD_TILE) * CD_TILE + e % CD_TILE];
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int64_t row = (int64_t)blockIdx.x * LQ8_APPLY_WARPS + (threadIdx.x >> 5);
+  if (row >= m) return;
+  const float sc = scale[row];
+  const float inv = 1.0f / sc;
+  __half* drow_hi = dhi + row * lda;
+  __half* drow_lo = dlo + row * lda;
+  if (jl0 == 0) {  // first block of the tile: clear the operand row (zeros past tw)
+    for (int i = lane; i < CD_TILE; i += 32) {
+      drow_hi[i] = __float2half_rn(0.0f);
+      drow_lo[i] = __float2half_rn(0.0f);
+    }
+    if (lane == 0) d_unscale[row] = -sc;
+  }
+  float v = INFINITY;
+  int k = 0x7fffffff;
+  for (int c = lane; c < nchunks; c += 32) {
+    const float v2 = part_val[row * nchunks + c];
+    const int k2 = part_idx[row * nchunks + c];
+    if (v2 < v || (v2 == v && k2 < k)) {
+      v = v2;
+      k = k2;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float v2 = __shfl_xor_sync(0xffffffffu, v, o);
+    const int k2 = __shfl_xor_sync(0xffffffffu, k, o);
+    if (v2 < v || (v2 == v && k2 < k)) {
+      v = v2;
+      k = k2;
+    }
+  }
+  k = min(max(k, 0), K - 1);
+  // working values of the tile's columns from this block on
+  float* wr = Wk + row * ldw + t0;
+  float w[LQ_SLOTS];
+#pragma unroll
+  for (int q = 0; q < LQ_SLOTS; ++q) {
+    const int col = 32 * q + lane;
+    w[q] = (col >= jl0 && col < tw) ? wr[col] : 0.0f;
+  }
+  // the block's columns, one after another: error e_j = v_j - scale c_j
+#pragma unroll
+  for (int jj = 0; jj < 8; ++jj) {
+    const int j = jl0 + jj;
+    const int owner = j & 31, slot = j >> 5;
+    float vj = 0.0f;
+#pragma unroll
+    for (int q = 0; q < LQ_SLOTS; ++q)
+      if (q == slot) vj = w[q];
+    const float e = __shfl_sync(0xffffffffu, vj, owner) - sc * cb[(int64_t)k * 8 + jj];
+#pragma unroll
+    for (int q = 0; q < LQ_SLOTS; ++q) w[q] = fmaf(-e, s_u[jj][32 * q + lane], w[q]);
+    if (lane == jj) {
+      const float a = e * inv;
+      const __half h = __float2half_rn(a);
+      drow_hi[j] = h;
+      drow_lo[j] = __float2half_rn(a - __half2float(h));
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < LQ_SLOTS; ++q) {
+    const int col = 32 * q + lane;
+    if (col >= jl0 + 8 && col < tw) wr[col] = w[q];
+  }
+  if (lane == 0) idx[row * (n / 8) + b] = (uint16_t)k;
+}
+
 }  // namespace
 
 mpq_status ldlq_factor(const mpq_plan_s* p, double damp, float* Bl, float* Ud, cudaStream_t st) {
@@ -317,6 +453,16 @@ mpq_status launch_ldlq(mpq_plan_s* p, const float* W, int64_t m, const float* sc
                                            : cd_panel_cols(m, n);
   const int np = (int)cdiv(n, P);
   MPQ_CUDA(cudaFuncSetAttribute(k_ldlq_tile, cudaFuncAttributeMaxDynamicSharedMemorySize, LQ_SMEM));
+  // d = 8: per-row chunk minima of the nearest-codeword scan
+  const int nchunks = p->d == 8 ? (int)cdiv(p->K, LQ8_CHUNK) : 0;
+  float* part_val = nullptr;
+  int* part_idx = nullptr;
+  if (p->d == 8) {
+    if (!p->cb_norm) return fail(MPQ_ERR_INVALID_ARG, "the plan has no codebook tables");
+    MPQ_CUDA(cudaMallocAsync(&part_val, sizeof(float) * m * nchunks, st));
+    MPQ_CUDA(cudaMallocAsync(&part_idx, sizeof(int) * m * nchunks, st));
+  }
+  mpq_status rc = MPQ_OK;
   auto update = [&](int64_t a_k0, int64_t b_k0, int64_t K, int64_t c0, int64_t c1,
                     const char* tag) -> mpq_status {
     if (c1 <= c0) return MPQ_OK;
@@ -329,26 +475,49 @@ mpq_status launch_ldlq(mpq_plan_s* p, const float* W, int64_t m, const float* sc
     return gemm_tc(w.As, w.tm_an_hi, w.tm_an_lo, p->Lq_s, p->tm_lq_hi, p->tm_lq_lo, w.Hg, w.ldh, m,
                    c1 - c0, K, p->Lq_s.unscale_host, p->status, st, tag, o);
   };
-  for (int pi = 0; pi < np; ++pi) {
+  for (int pi = 0; pi < np && rc == MPQ_OK; ++pi) {
     const int64_t ps = (int64_t)pi * P, pe = std::min<int64_t>(n, ps + P);
-    for (int64_t t0 = ps; t0 < pe; t0 += CD_TILE) {
+    for (int64_t t0 = ps; t0 < pe && rc == MPQ_OK; t0 += CD_TILE) {
       const int tw = (int)std::min<int64_t>(CD_TILE, n - t0);
-      {
-        ProfScope ps_("k_ldlq_tile", st);
-        k_ldlq_tile<<<(unsigned)cdiv(m, LQ_WARPS), LQ_WARPS * 32, LQ_SMEM, st>>>(
-            m, n, p->K, t0, tw, scale, offset, (int)p->ng, p->G ? (int)(t0 / p->G) : 0,
-            p->G ? w.sref : nullptr, p->ldlq_diag + (t0 / CD_TILE) * CD_TILE * CD_TILE, w.Hg,
-            w.ldh, idx, w.As.hi + (t0 - ps), w.As.lo + (t0 - ps), w.As.ld, w.As.row_unscale);
+      const float* Ud = p->ldlq_diag + (t0 / CD_TILE) * CD_TILE * CD_TILE;
+      __half* dhi = w.As.hi + (t0 - ps);
+      __half* dlo = w.As.lo + (t0 - ps);
+      if (p->d == 1) {
+        {
+          ProfScope ps_("k_ldlq_tile", st);
+          k_ldlq_tile<<<(unsigned)cdiv(m, LQ_WARPS), LQ_WARPS * 32, LQ_SMEM, st>>>(
+              m, n, p->K, t0, tw, scale, offset, (int)p->ng, p->G ? (int)(t0 / p->G) : 0,
+              p->G ? w.sref : nullptr, Ud, w.Hg, w.ldh, idx, dhi, dlo, w.As.ld, w.As.row_unscale);
+        }
+        count_launch();
+        rc = check_launch("k_ldlq_tile");
+      } else {
+        for (int64_t b = t0 / 8; b < (t0 + tw) / 8 && rc == MPQ_OK; ++b) {
+          {
+            ProfScope ps_("k_ldlq8_eval", st);
+            dim3 ge((unsigned)nchunks, (unsigned)cdiv(m, LQ8_ROWS));
+            k_ldlq8_eval<<<ge, LQ8_ROWS, 0, st>>>(m, p->K, b, p->cb, p->cb_norm, scale, w.Hg,
+                                                  w.ldh, part_val, part_idx, nchunks);
+          }
+          {
+            ProfScope ps_("k_ldlq8_apply", st);
+            k_ldlq8_apply<<<(unsigned)cdiv(m, LQ8_APPLY_WARPS), LQ8_APPLY_WARPS * 32, 0, st>>>(
+                m, n, p->K, b, t0, tw, p->cb, scale, Ud, w.Hg, w.ldh, idx, part_val, part_idx,
+                nchunks, dhi, dlo, w.As.ld, w.As.row_unscale);
+          }
+          count_launch(2);
+          rc = check_launch("k_ldlq8");
+        }
       }
-      count_launch();
-      MPQ_TRY(check_launch("k_ldlq_tile"));
       // later columns of the panel
-      MPQ_TRY(update(t0 - ps, t0, tw, t0 + tw, pe, "gemm_ldlq_update"));
+      if (rc == MPQ_OK) rc = update(t0 - ps, t0, tw, t0 + tw, pe, "gemm_ldlq_update");
     }
     // every column after the panel
-    if (np > 1) MPQ_TRY(update(0, ps, pe - ps, pe, n, "gemm_ldlq_panel"));
+    if (rc == MPQ_OK && np > 1) rc = update(0, ps, pe - ps, pe, n, "gemm_ldlq_panel");
   }
-  return MPQ_OK;
+  if (part_val) cudaFreeAsync(part_val, st);
+  if (part_idx) cudaFreeAsync(part_idx, st);
+  return rc;
 }
 
 }  // namespace mpq

@@ -140,8 +140,6 @@ mpq_status validate_params(const mpq_params* q, int64_t n) {
     return fail(MPQ_ERR_INVALID_ARG, "greedy_init must be 0 or 1");
   if (!(q->greedy_damp >= 0.0) || !std::isfinite(q->greedy_damp))
     return fail(MPQ_ERR_INVALID_ARG, "greedy_damp must be finite and >= 0");
-  if (q->greedy_init && q->d != 1)
-    return fail(MPQ_ERR_UNSUPPORTED, "the greedy baseline is built for scalar grids (d = 1)");
   if (q->group_size < 0 || (q->group_size > 0 && (q->d != 1 || q->group_size % 128 ||
                                                    n % q->group_size)))
     return fail(MPQ_ERR_INVALID_ARG,

@@ -1,10 +1,10 @@
-"""Parity of the greedy baseline (LDLQ on scalar grids, the T_vamp = 0 init
-of plans created with greedy_init = 1) with the float64 oracle.
+"""Parity of the greedy baseline (LDLQ on scalar grids and E8 codebooks, the
+T_vamp = 0 init of plans created with greedy_init = 1) with the float64 oracle.
 
 Cases span several 128-column tiles with a ragged tail, one panel and
 several panels (cd_panel = 128), group-wise grids, and a rank-deficient X
 (damped factor).  Bars: every decision before a row's first near-tie of the
-oracle (top-two distance gap below 1e-3 grid units^2) is exact, rows without
+oracle (top-two distance gap below 1e-3 in units of scale^2) is exact, rows without
 one match index for index, and their energies are within 1e-3; after CD the
 whole-solve rules of the other parity tests apply."""
 import numpy as np
@@ -27,6 +27,9 @@ def mpq():
 
 
 def grid(p, group):
+    if p.d == 8:
+        sc = orc.rms_scale(p.W)[0].astype(np.float32)
+        return sc, np.zeros_like(sc)
     if group:
         sc, off = orc.minmax_grid(p.W, p.levels, group)
         return sc.astype(np.float32), off.astype(np.float32)
@@ -35,8 +38,9 @@ def grid(p, group):
 
 def check_greedy(mpq, p, group=0, damp=0.01, cd_panel=0, sweeps=0, min_clean=0.5):
     s, V, s_cu, V_cu = spectrum_cuda(p.X)
-    plan = mpq.Plan.from_spectrum(s_cu, V_cu, 1, p.levels, greedy_init=1, greedy_damp=damp,
-                                  cd_panel=cd_panel, group_size=group)
+    plan = mpq.Plan.from_spectrum(s_cu, V_cu, p.d, p.levels, codebook=p.codebook,
+                                  greedy_init=1, greedy_damp=damp, cd_panel=cd_panel,
+                                  group_size=group)
     sc, off = grid(p, group)
     cb = codebook_for(p)
     sc64, off64 = sc.astype(np.float64), off.astype(np.float64)
@@ -49,7 +53,7 @@ def check_greedy(mpq, p, group=0, damp=0.01, cd_panel=0, sweeps=0, min_clean=0.5
         clean = ~near.any(axis=1)
         assert clean.mean() >= min_clean, f"only {clean.mean():.2f} of rows free of near-ties"
         for i in range(p.m_out):
-            first = int(np.argmax(near[i])) if near[i].any() else p.n
+            first = int(np.argmax(near[i])) if near[i].any() else near.shape[1]
             assert np.array_equal(got[i, :first], g.idx[i, :first]), (i, first)
         E = orc.energy(p.W, orc.decode(g.idx, cb, sc64, off64), s, V)
         assert np.all(np.abs(e[clean] - E[clean]) <= ENERGY_TOL * E[clean])
@@ -109,3 +113,47 @@ def test_greedy_does_not_touch_vamp_solves(mpq):
     oa = a.solve(cu(p.W), 3, 2)
     ob = b.solve(cu(p.W), 3, 2)
     assert np.array_equal(idx_np(oa["idx"]), idx_np(ob["idx"]))
+
+
+def e8_problem(seed, m_out, n, m, K=2048, sweeps=0):
+    cb = mi.e8_codebook_cached()[:K]
+    return mi.small_problem(seed, m_out, n, m, d=8, levels=K, T_vamp=0, cd_sweeps=sweeps,
+                            codebook=cb)
+
+
+@pytest.mark.parametrize("cd_panel", [0, 128])
+def test_greedy_e8_ragged_tiles(mpq, cd_panel):
+    # n = 200: a tile of 16 blocks and one of 9; K = 2048 spans two scan chunks
+    check_greedy(mpq, e8_problem(711, 21, 200, 400), cd_panel=cd_panel)
+
+
+def test_greedy_e8_many_rows_full_codebook(mpq):
+    # 300 rows (two row groups of the scan), K = 65536 (64 chunks)
+    check_greedy(mpq, e8_problem(712, 300, 128, 300, K=65536), min_clean=0.3)
+
+
+def test_greedy_e8_then_cd(mpq):
+    check_greedy(mpq, e8_problem(713, 23, 160, 320, sweeps=3), sweeps=3, min_clean=0.25)
+
+
+def test_greedy_full_size_l1b_sampled_rows(mpq):
+    # the bench's l1b layer (2048 x 2048, 3-bit), every row on the device in one
+    # solve, a seeded sample of rows against the oracle's greedy pass
+    p = mi.make_problem("l1b")
+    X = cu(p.X)
+    plan = mpq.Plan.from_x(X, 1, p.levels, greedy_init=1)
+    del X
+    s, V = orc.spectrum(p.X)
+    assert s.size == plan.r
+    sc, off = oracle_grid_f32(p)
+    out = plan.solve(cu(p.W), 0, 0, row_scale=cu(sc), row_offset=cu(off))
+    got = idx_np(out["idx"])
+    rows = np.sort(np.random.default_rng(4).choice(p.m_out, 4, replace=False))
+    cb = codebook_for(p)
+    g = orc.ldlq(p.W[rows], cb, sc[rows].astype(np.float64), off[rows].astype(np.float64),
+                 orc.hessian(s, V), 0.01)
+    near = g.gap < TIE
+    for k, i in enumerate(rows):
+        first = int(np.argmax(near[k])) if near[k].any() else near.shape[1]
+        assert first >= 256, (i, first)   # a long exact prefix on every sampled row
+        assert np.array_equal(got[i, :first], g.idx[k, :first]), (i, first)
