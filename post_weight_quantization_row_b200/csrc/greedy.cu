@@ -219,54 +219,94 @@ __global__ void __launch_bounds__(LQ_WARPS * 32, 2)
 // Block b of a tile: the codeword nearest (Euclidean, in codebook units) the
 // block's current working values, t = v_b / scale: argmin_c 1/2 |c|^2 - c.t
 // (lowest index on ties).  Kernel A scans one chunk of LQ8_CHUNK codewords
-// for LQ8_ROWS rows (a thread per row, the chunk in shared memory, read by
-// broadcast); kernel B (a warp per row) combines the chunk minima, commits
-// the codeword, and feeds the block's 8 errors, one column after another, to
-// the later columns of the tile through the block's 8 rows of B^T.
-constexpr int LQ8_CHUNK = 256;  // small chunks: >= 256 CTAs per scan at K = 65536
+// for LQ8_ROWS rows: the chunk sits transposed in shared memory, each warp
+// takes groups of 8 rows with the lanes splitting the codewords, so every
+// codeword read from shared memory serves 8 rows (8 independent FMA chains).
+// Kernel B (a warp per row) combines the chunk minima, commits the codeword,
+// and feeds the block's 8 errors, one column after another, to the later
+// columns of the tile through the block's 8 rows of B^T.
+constexpr int LQ8_CHUNK = 1024;
 constexpr int LQ8_ROWS = 256;
 constexpr int LQ8_APPLY_WARPS = 16;
 
-__global__ void __launch_bounds__(LQ8_ROWS)
+__global__ void __launch_bounds__(256)
     k_ldlq8_eval(int64_t m, int K, int64_t b, const float* __restrict__ cb,
                  const float* __restrict__ cb_norm, const float* __restrict__ scale,
                  const float* __restrict__ Wk, int64_t ldw, float* __restrict__ part_val,
                  int* __restrict__ part_idx, int nchunks) {
-  __shared__ float4 s_cb[LQ8_CHUNK * 2];  // codeword c: s_cb[2c], s_cb[2c + 1]
-  __shared__ float s_half_norm[LQ8_CHUNK];
+  __shared__ float scb[8][LQ8_CHUNK];  // transposed: lanes read consecutive codewords
+  __shared__ float sq[LQ8_CHUNK];      // 1/2 |c|^2
+  __shared__ float st[LQ8_ROWS][8];    // the rows' targets t
   const int chunk = blockIdx.x;
+  const int64_t r0 = (int64_t)blockIdx.y * LQ8_ROWS;
   const int c0 = chunk * LQ8_CHUNK;
-  const int cnt = min(LQ8_CHUNK, K - c0);
-  for (int e = threadIdx.x; e < cnt * 8; e += blockDim.x)
-    reinterpret_cast<float*>(s_cb)[e] = cb[(int64_t)c0 * 8 + e];
-  for (int e = threadIdx.x; e < cnt; e += blockDim.x) s_half_norm[e] = 0.5f * cb_norm[c0 + e];
-  __syncthreads();
-  const int64_t row = (int64_t)blockIdx.y * LQ8_ROWS + threadIdx.x;
-  if (row >= m) return;
-  const float inv = 1.0f / scale[row];
-  float t[8];
+  const int cn = min(LQ8_CHUNK, K - c0);
+  for (int e = threadIdx.x; e < cn * 8; e += blockDim.x) scb[e % 8][e / 8] = cb[(int64_t)c0 * 8 + e];
+  for (int e = threadIdx.x; e < cn; e += blockDim.x) sq[e] = 0.5f * cb_norm[c0 + e];
+  for (int rl = threadIdx.x; rl < LQ8_ROWS; rl += blockDim.x) {
+    const int64_t row = r0 + rl;
+    if (row < m) {
+      const float inv = 1.0f / scale[row];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) t[j] = Wk[row * ldw + 8 * b + j] * inv;
-  float best = INFINITY;
-  int bi = 0;
-  for (int c = 0; c < cnt; ++c) {
-    const float4 a = s_cb[2 * c], b4 = s_cb[2 * c + 1];
-    float sc = s_half_norm[c];
-    sc = fmaf(-a.x, t[0], sc);
-    sc = fmaf(-a.y, t[1], sc);
-    sc = fmaf(-a.z, t[2], sc);
-    sc = fmaf(-a.w, t[3], sc);
-    sc = fmaf(-b4.x, t[4], sc);
-    sc = fmaf(-b4.y, t[5], sc);
-    sc = fmaf(-b4.z, t[6], sc);
-    sc = fmaf(-b4.w, t[7], sc);
-    if (sc < best) {
-      best = sc;
-      bi = c;
+      for (int i = 0; i < 8; ++i) st[rl][i] = Wk[row * ldw + 8 * b + i] * inv;
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) st[rl][i] = 0.0f;
     }
   }
-  part_val[row * nchunks + chunk] = best;
-  part_idx[row * nchunks + chunk] = c0 + bi;
+  __syncthreads();
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  for (int grp = w; grp < LQ8_ROWS / 8; grp += blockDim.x / 32) {
+    if (r0 + 8 * grp >= m) break;
+    float g[8][8];
+#pragma unroll
+    for (int rr = 0; rr < 8; ++rr)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) g[rr][i] = st[8 * grp + rr][i];
+    float best[8];
+    int bidx[8];
+#pragma unroll
+    for (int rr = 0; rr < 8; ++rr) {
+      best[rr] = INFINITY;
+      bidx[rr] = 0x7fffffff;
+    }
+    for (int c = lane; c < cn; c += 32) {
+      float cv[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) cv[i] = scb[i][c];
+      const float q = sq[c];
+#pragma unroll
+      for (int rr = 0; rr < 8; ++rr) {
+        float sc = q;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) sc = fmaf(-cv[i], g[rr][i], sc);
+        if (sc < best[rr]) {
+          best[rr] = sc;
+          bidx[rr] = c0 + c;
+        }
+      }
+    }
+    // warp minimum per row, lowest index on ties
+#pragma unroll
+    for (int rr = 0; rr < 8; ++rr) {
+      float v = best[rr];
+      int k = bidx[rr];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float v2 = __shfl_xor_sync(0xffffffffu, v, o);
+        const int k2 = __shfl_xor_sync(0xffffffffu, k, o);
+        if (v2 < v || (v2 == v && k2 < k)) {
+          v = v2;
+          k = k2;
+        }
+      }
+      const int64_t row = r0 + 8 * grp + rr;
+      if (lane == 0 && row < m) {
+        part_val[row * nchunks + chunk] = v;
+        part_idx[row * nchunks + chunk] = k;
+      }
+    }
+  }
 }
 
 __global__ void __launch_bounds__(LQ8_APPLY_WARPS * 32)
