@@ -289,13 +289,19 @@ def run_reference(args, world, rank):
     if rank != 0:
         return
     p = workload(args.config)
+    if args.greedy:
+        p.T_vamp = 0
     rows = max(1, args.cpu_rows // 2)
-    times, t_spec = oracle_sample(p, rows, args.warmup + args.steps, args.group_size)
+    times, t_spec = oracle_sample(p, rows, args.warmup + args.steps, args.group_size,
+                                  0.01 if args.greedy else None)
     timed = times[args.warmup:]
     sec = sum(timed) / len(timed)
     value = rows * p.n / sec
     cores = len(os.sched_getaffinity(0))
     cfgd = describe(p, args.config, args.group_size)
+    if args.greedy:
+        cfgd["workload"] += " (greedy baseline: LDLQ init, damp 0.01, then the same CD)"
+        cfgd["init"] = "LDLQ"
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",

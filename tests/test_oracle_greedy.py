@@ -82,3 +82,21 @@ def test_solve_with_greedy_init():
     # without greedy_damp, T_vamp = 0 stays round-to-nearest
     rtn = orc.solve(W, cb, s, V, 0, 0, sc, off)
     assert np.array_equal(rtn.idx, orc.init(W, cb, sc, off).idx_rtn)
+
+
+def test_input_recipe_rotation_is_the_sylvester_hadamard():
+    # the e8 / e8t8 inputs rotate W and X by Q = H_n diag(signs) / sqrt(n);
+    # the generator's fast transform must equal the dense Sylvester matrix and
+    # leave the objective's Gram spectrum unchanged
+    import math
+    import scipy.linalg
+    g = np.random.default_rng(21)
+    for n in (1, 2, 8, 64, 256):
+        a = g.standard_normal((5, n))
+        signs = np.where(g.random(n) < 0.5, -1.0, 1.0)
+        dense = a @ (signs[:, None] * scipy.linalg.hadamard(n)) / math.sqrt(n)
+        assert np.allclose(mi.random_hadamard_apply(a, signs), dense, rtol=1e-12, atol=1e-12)
+    X = g.standard_normal((40, 64))
+    signs = np.where(g.random(64) < 0.5, -1.0, 1.0)
+    Xr = mi.random_hadamard_apply(X, signs)
+    assert np.allclose(np.linalg.svd(X, compute_uv=False), np.linalg.svd(Xr, compute_uv=False))
