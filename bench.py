@@ -449,7 +449,9 @@ def run_mpq(args, world, rank, local):
                          f"(MEASURED_PEAKS.json) / {passes} fp16 MMA passes per fp32-accurate product",
                }.get(bound, f"{peak_src} MEASURED_PEAKS.json")
         roof = {"bound": bound, "kernel": name, "achieved": achieved, "peak": peak, "unit": unit,
-                "frac": achieved / peak, "traffic": recorded_traffic(name, args.config),
+                "frac": achieved / peak,
+                "traffic": recorded_traffic(name, args.config if not args.rows
+                                            else f"{args.config}:rows{args.rows}"),
                 "peak_source": src, "work_per_launch": work, "launches": cnt,
                 "avg_launch_ms": kms / cnt}
         if bound == "tensor":
