@@ -96,3 +96,29 @@ def test_streamed_gram_and_rht_reject_bad_arguments_without_a_device(mpq):
                        (4, 64, None)]:
         assert lib.mpq_rht(x, rows, n, dummy, None) == 1, (rows, n)
     assert "power of two" in lib.mpq_last_error().decode() or "device" in lib.mpq_last_error().decode()
+
+
+@pytest.mark.parametrize("c_name,py_name", [("mpq_params", "Params"), ("mpq_row_stats", "RowStats")])
+def test_struct_layout_matches_the_c_header(mpq, tmp_path, c_name, py_name):
+    # the ctypes mirrors of the ABI structs must have the C compiler's size and
+    # field offsets, or every call would read shifted fields
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    cls = getattr(mpq, py_name)
+    fields = [f[0] for f in cls._fields_]
+    src = ['#include <stdio.h>', '#include <stddef.h>', '#include "mpq.h"', "int main(void) {",
+           f'  printf("%zu\\n", sizeof({c_name}));']
+    src += [f'  printf("%zu\\n", offsetof({c_name}, {f}));' for f in fields]
+    src += ["  return 0;", "}"]
+    c_file = tmp_path / "layout.c"
+    c_file.write_text("\n".join(src) + "\n")
+    exe = tmp_path / "layout"
+    subprocess.run([cc, "-std=c99", "-I", os.path.join(ROOT, "include"), str(c_file), "-o", str(exe)],
+                   check=True)
+    out = [int(x) for x in subprocess.run([str(exe)], check=True, capture_output=True,
+                                          text=True).stdout.split()]
+    assert out[0] == C.sizeof(cls)
+    assert out[1:] == [getattr(cls, f).offset for f in fields]
