@@ -122,3 +122,14 @@ def test_struct_layout_matches_the_c_header(mpq, tmp_path, c_name, py_name):
                                           text=True).stdout.split()]
     assert out[0] == C.sizeof(cls)
     assert out[1:] == [getattr(cls, f).offset for f in fields]
+
+
+def test_binding_argument_counts_match_the_header(mpq):
+    # every ctypes signature takes as many arguments as its C declaration
+    txt = open(os.path.join(ROOT, "include", "mpq.h")).read()
+    decls = re.findall(r"^MPQ_API\s+[\w\s\*]+?\b(mpq_\w+)\s*\(([^;]*?)\)\s*;", txt, flags=re.M | re.S)
+    assert len(decls) == len(declared_symbols())
+    for name, params in decls:
+        params = " ".join(params.split())
+        n_c = 0 if params in ("", "void") else params.count(",") + 1
+        assert len(getattr(mpq.lib, name).argtypes) == n_c, name
