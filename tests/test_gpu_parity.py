@@ -284,18 +284,19 @@ def test_stage_energy(mpq):
 
 # ------------------------------------------------------------ whole solve ---
 
-def _solve_compare(mpq, p, T=None, sweeps=None, min_clean=0.5):
+def _solve_compare(mpq, p, T=None, sweeps=None, min_clean=0.5, tau=math.inf):
     T = p.T_vamp if T is None else T
     sweeps = p.cd_sweeps if sweeps is None else sweeps
     s, V, s_cu, V_cu = spectrum_cuda(p.X)
-    plan = make_plan(mpq, p, s_cu, V_cu)
+    plan = make_plan(mpq, p, s_cu, V_cu, tau=tau)
     if p.d == 1:
         sc, off = oracle_grid_f32(p)
     else:
         sc = orc.rms_scale(p.W)[0].astype(np.float32)
         off = np.zeros_like(sc)
     cb = codebook_for(p)
-    ref = orc.solve(p.W, cb, s, V, T, sweeps, sc.astype(np.float64), off.astype(np.float64))
+    ref = orc.solve(p.W, cb, s, V, T, sweeps, sc.astype(np.float64), off.astype(np.float64),
+                    tau=tau)
     out = plan.solve(cu(p.W), T, sweeps, row_scale=cu(sc), row_offset=cu(off), stats=True)
     got = idx_np(out["idx"])
     e_gpu = host(out["energy"]).astype(np.float64)
@@ -356,6 +357,18 @@ def test_solve_tiny12_rows_never_beat_exhaustive(mpq):
 
 def test_solve_scalar_small(mpq):
     _solve_compare(mpq, scalar_case())
+
+
+@pytest.mark.parametrize("seed,n,L,tau", [(101, 200, 8, 0.2), (102, 256, 16, 0.7)])
+def test_solve_scalar_anchored_prior(mpq, seed, n, L, tau):
+    # finite tau: the fused row kernel's anchored denoiser in a whole solve
+    p = mi.small_problem(seed, 37, n, 300 if n == 200 else 400, d=1, levels=L, T_vamp=4,
+                         cd_sweeps=3)
+    _solve_compare(mpq, p, tau=tau)
+
+
+def test_solve_vector_anchored_prior(mpq):
+    _solve_compare(mpq, vec_case(), tau=0.3)
 
 
 def test_solve_scalar_rank_deficient(mpq):
