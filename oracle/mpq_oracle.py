@@ -16,7 +16,7 @@ Sources (cited by page title and section):
               Initialization for Low-Bit LLMs" note, section "Existing pain
               points" (现有痛点): the min-max scale / zero-point formula.
 
-Readings where the pages are silent (each also listed in the design doc):
+Readings where the pages are silent (the CUDA library takes the same ones):
   R1  rank cut: keep Gram eigenvalues lambda_l > lambda_max * max(m, n) * 2^-52
       (the NumPy matrix_rank convention applied to the Gram matrix).
   R2  scalar grid: per-row min-max, s=(max-min)/(L-1), z=clip(rint(-min/s)),

@@ -631,6 +631,13 @@ mpq_status new_plan(const mpq_params* params, int64_t n, mpq_plan_s** out) {
     if (!(p)) return ::mpq::fail(MPQ_ERR_INVALID_ARG, "plan is NULL");     \
   } while (0)
 
+// row counts index the grid's x dimension (one CTA or warp group per row)
+#define ROWS_CHECK(m)                                                      \
+  do {                                                                     \
+    if ((m) > ::mpq::MAX_ROWS)                                             \
+      return ::mpq::fail(MPQ_ERR_INVALID_ARG, "row count above 2^31 - 1"); \
+  } while (0)
+
 }  // namespace
 }  // namespace mpq
 
@@ -861,7 +868,7 @@ mpq_status mpq_solve(mpq_plan_t p, const float* W, int64_t m_out, const float* r
     return fail(MPQ_ERR_INVALID_ARG, "row_scale and row_offset go together");
   if (T_vamp < 0) return fail(MPQ_ERR_INVALID_ARG, "T_vamp must be >= 0");
   if (cd_sweeps < 0 || cd_sweeps > MAX_SWEEPS) return fail(MPQ_ERR_INVALID_ARG, "cd_sweeps must be in [0, 64]");
-  if (m_out > 2147483647LL) return fail(MPQ_ERR_INVALID_ARG, "m_out too large");
+  ROWS_CHECK(m_out);
   DeviceGuard g(p->device);
   SolveIO io{W, m_out, row_scale, row_offset, T_vamp, cd_sweeps, idx, w_hat, energy, stats};
   return solve_device(p, io, (cudaStream_t)stream);
@@ -873,6 +880,7 @@ mpq_status mpq_solve_host(mpq_plan_t p, const float* W_host, int64_t m_out, int3
   PLAN_CHECK(p);
   if (m_out < 0) return fail(MPQ_ERR_INVALID_ARG, "m_out must be >= 0");
   if (m_out == 0) return MPQ_OK;
+  ROWS_CHECK(m_out);
   if (!W_host || !idx_host) return fail(MPQ_ERR_INVALID_ARG, "W and idx are required");
   if (T_vamp < 0 || cd_sweeps < 0 || cd_sweeps > MAX_SWEEPS)
     return fail(MPQ_ERR_INVALID_ARG, "bad T_vamp / cd_sweeps");
@@ -901,6 +909,7 @@ mpq_status mpq_stage_init(mpq_plan_t p, const float* W, int64_t m, int32_t given
   PLAN_CHECK(p);
   if (m < 0 || (m > 0 && (!W || !scale || !offset || !idx_rtn || !gamma1_0)))
     return fail(MPQ_ERR_INVALID_ARG, "init: missing buffer");
+  ROWS_CHECK(m);
   DeviceGuard g(p->device);
   return launch_init(p, W, m, given ? 1 : 0, scale, offset, idx_rtn, gamma1_0, (cudaStream_t)stream);
 }
@@ -912,6 +921,7 @@ mpq_status mpq_stage_denoise(mpq_plan_t p, const float* R1, const double* gamma1
   PLAN_CHECK(p);
   if (m < 0 || (m > 0 && (!R1 || !gamma1 || !scale || !offset || !xhat1 || !vsum)))
     return fail(MPQ_ERR_INVALID_ARG, "denoise: missing buffer");
+  ROWS_CHECK(m);
   if (isfinite(p->params.tau) && m > 0 && (!W || !gamma1_0))
     return fail(MPQ_ERR_INVALID_ARG, "denoise: an anchored plan needs W and gamma1_0");
   DeviceGuard g(p->device);
@@ -933,6 +943,7 @@ mpq_status mpq_stage_linear(mpq_plan_t p, const float* W, int64_t m, const float
   if (m < 0 || (m > 0 && (!W || !R1 || !gamma1 || !xhat1 || !vsum || !gamma1_0 || !beta ||
                           !R1_out || !gamma1_out)))
     return fail(MPQ_ERR_INVALID_ARG, "linear: missing buffer");
+  ROWS_CHECK(m);
   if (m == 0) return MPQ_OK;
   DeviceGuard g(p->device);
   MPQ_TRY(ensure_workspace(p, m));
@@ -950,6 +961,7 @@ mpq_status mpq_stage_cd(mpq_plan_t p, const float* W, int64_t m, const float* sc
   PLAN_CHECK(p);
   if (m < 0 || (m > 0 && (!W || !scale || !offset || !idx)))
     return fail(MPQ_ERR_INVALID_ARG, "cd: missing buffer");
+  ROWS_CHECK(m);
   if (sweeps < 0 || sweeps > MAX_SWEEPS) return fail(MPQ_ERR_INVALID_ARG, "sweeps must be in [0, 64]");
   if (m == 0 || sweeps == 0) return MPQ_OK;
   DeviceGuard g(p->device);
@@ -965,6 +977,7 @@ mpq_status mpq_stage_energy(mpq_plan_t p, const float* W, int64_t m, const float
   PLAN_CHECK(p);
   if (m < 0 || (m > 0 && (!W || !scale || !offset || !idx || !energy)))
     return fail(MPQ_ERR_INVALID_ARG, "energy: missing buffer");
+  ROWS_CHECK(m);
   if (m == 0) return MPQ_OK;
   DeviceGuard g(p->device);
   MPQ_TRY(ensure_workspace(p, m));

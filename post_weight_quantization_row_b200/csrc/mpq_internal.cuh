@@ -58,6 +58,10 @@ struct SplitOperand {
 
 inline int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
 
+// Largest row count an entry point accepts: rows map to the grid's x
+// dimension, whose limit is 2^31 - 1.
+constexpr int64_t MAX_ROWS = 2147483647LL;
+
 // --------------------------------------------------------------- workspace --
 struct Workspace {
   int64_t rows = 0;       // rows the buffers are sized for

@@ -55,6 +55,13 @@ extern "C" mpq_status mpq_stage_energy_noalloc(mpq_plan_t p, const float* W, int
   if (m < 0 || (m > 0 && (!W || !scale || !offset || !idx || !energy)))
     return fail(MPQ_ERR_INVALID_ARG, "energy_noalloc: missing buffer");
   if (m == 0) return MPQ_OK;
+  // m * per_row > the array size already means refusal; checking it by
+  // division first keeps the byte counts below from wrapping for huge m
+  const uint64_t per_row = 4ull * (uint64_t)p->n + 4ull * (uint64_t)p->r + 2ull * (uint64_t)p->B;
+  if (m > MAX_ROWS || (uint64_t)m > NOALLOC_SCRATCH_BYTES / per_row)
+    return fail(MPQ_ERR_INVALID_ARG,
+                "energy_noalloc: m * (4n + 4r + 2B) bytes exceeds the static scratch of " +
+                    std::to_string(NOALLOC_SCRATCH_BYTES) + " bytes; split the rows");
   const size_t e_bytes = align256((size_t)m * p->n * sizeof(float));
   const size_t p_bytes = align256((size_t)m * p->r * sizeof(float));
   const size_t i_bytes = align256((size_t)m * p->B * sizeof(uint16_t));

@@ -65,3 +65,43 @@ def test_noalloc_refuses_calls_larger_than_its_array(setup):
         plan.stage_energy_noalloc(W, sc, torch.zeros_like(sc), idx)
     assert e.value.status == 1
     assert mpq.kernel_launch_count() == before
+
+
+def test_noalloc_energy_allocates_nothing(setup):
+    """On a fresh plan whose workspace cap (1 byte) makes any workspace
+    allocation fail, the entry point still runs, and the device's free
+    memory and torch's allocated bytes are the same before and after two
+    calls (a first call runs before the measurement: loading the library's
+    kernels on first use may reserve device memory once per process)."""
+    mpq, p, _, st = setup
+    s, V = orc.spectrum(p.X)
+    plan = mpq.Plan.from_spectrum(torch.from_numpy(s).cuda(), torch.from_numpy(V).cuda(), 1,
+                                  p.levels)
+    plan.set_workspace_cap(1)
+    W, sc, off, idx = _args(p, st, 40, 3)
+    w_hat = torch.empty(40, plan.n, dtype=torch.float32, device="cuda")
+    energy = torch.empty(40, dtype=torch.float32, device="cuda")
+    plan.stage_energy_noalloc(W, sc, off, idx, w_hat, energy)
+    plan.status()
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    torch0 = torch.cuda.memory_allocated()
+    for _ in range(2):
+        plan.stage_energy_noalloc(W, sc, off, idx, w_hat, energy)
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0
+    assert torch.cuda.memory_allocated() == torch0
+    plan.status()
+    # the workspace-backed entry point on the same plan needs workspace and
+    # is refused by the cap, so the calls above never created any
+    with pytest.raises(mpq.MPQError) as e:
+        plan.stage_energy(W, sc, off, idx)
+    assert e.value.status == 3
+    e_ref = orc.energy(p.W[:40], orc.decode(idx.cpu().numpy().view(np.uint16).astype(np.int64),
+                                             orc.scalar_levels(p.levels),
+                                             sc.cpu().numpy().astype(np.float64),
+                                             off.cpu().numpy().astype(np.float64)), s, V)
+    got = energy.double().cpu().numpy()
+    assert np.all(np.abs(got - e_ref) <= 1e-4 * e_ref)
+    plan.close()
