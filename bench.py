@@ -62,6 +62,9 @@ def parse():
     ap.add_argument("--greedy", action="store_true",
                     help="the greedy baseline (LDLQ init, T_vamp = 0) with the same CD sweeps "
                          "instead of MPQ")
+    ap.add_argument("--tau", type=float, default=0.2,
+                    help="prior anchor scale in codebook units (the pages' default 0.2; "
+                         "inf = the unanchored form)")
     ap.add_argument("--spectrum-cache", default=None,
                     help="npz file: reuse the spectrum a previous run computed on the device")
     return ap.parse_args()
@@ -184,8 +187,8 @@ def kernel_work(name, m, n, r, d, K, L):
         return "hbm", "GB/s", 20.0 * m * n
     if name == "k_extrinsic_l2d":        # read r2, D; write r1
         return "hbm", "GB/s", 12.0 * m * n
-    if name == "k_linear_rows":          # read/write U' (m x r)
-        return "hbm", "GB/s", 8.0 * m * r
+    if name == "k_linear_finish":        # per row: the column tiles' two M-step sums
+        return "hbm", "GB/s", 8.0 * m * ((r + 127) // 128)
     if name in ("k_denoise_vec", "k_denoise_vec_tc"):  # one exponential per (block, codeword)
         return "sfu", "Gexp/s", float(m) * (n // 8) * K
     if name == "k_vamp_row_scalar":      # read g, r2, w; write r2 and the fp16 hi/lo operand
@@ -255,19 +258,21 @@ def workload(cfg, rank=0):
     return p
 
 
-def describe(p, cfg, group=0):
+def describe(p, cfg, group=0, tau=0.2):
     bits = {8: 3, 16: 4}.get(p.levels, None) if p.d == 1 else 2
     grid = f"group-{group}" if group else "per-row"
+    anchor = f"tau={tau:g}" if math.isfinite(tau) else "unanchored (tau=inf)"
     return {"workload": f"{cfg}: W {p.m_out}x{p.n}, X {p.X.shape[0]}x{p.n}, "
                         + (f"{bits}-bit {grid} min-max grid" if p.d == 1 else
                            f"offset-E8 d=8 K={p.levels}, RHT")
-                        + f", T_vamp={p.T_vamp}, CD sweeps<={p.cd_sweeps}",
+                        + f", T_vamp={p.T_vamp}, rho_damp=0.5, {anchor}, CD sweeps<={p.cd_sweeps}",
             "m_out": p.m_out, "n": p.n, "m_calib": int(p.X.shape[0]), "d": p.d,
             "levels_or_K": p.levels, "T_vamp": p.T_vamp, "cd_sweeps": p.cd_sweeps,
+            "tau": tau if math.isfinite(tau) else "inf",
             "seeds": p.seeds, "l2": "flushed between timed steps (512 MiB write)"}
 
 
-def oracle_sample(p, rows, steps=1, group=0, greedy_damp=None):
+def oracle_sample(p, rows, steps=1, group=0, greedy_damp=None, tau=0.2):
     """Time the float64 oracle on `rows` rows of the layer (spectrum excluded)."""
     from oracle import mpq_oracle as orc
     t0 = time.time()
@@ -278,7 +283,8 @@ def oracle_sample(p, rows, steps=1, group=0, greedy_damp=None):
     for k in range(steps):
         sel = slice((k * rows) % p.m_out, (k * rows) % p.m_out + rows)
         t0 = time.perf_counter()
-        orc.solve(p.W[sel], cb, s, V, p.T_vamp, p.cd_sweeps, group=group, greedy_damp=greedy_damp)
+        orc.solve(p.W[sel], cb, s, V, p.T_vamp, p.cd_sweeps, group=group, greedy_damp=greedy_damp,
+                  tau=tau)
         times.append(time.perf_counter() - t0)
     return times, t_spec
 
@@ -293,12 +299,12 @@ def run_reference(args, world, rank):
         p.T_vamp = 0
     rows = max(1, args.cpu_rows // 2)
     times, t_spec = oracle_sample(p, rows, args.warmup + args.steps, args.group_size,
-                                  0.01 if args.greedy else None)
+                                  0.01 if args.greedy else None, args.tau)
     timed = times[args.warmup:]
     sec = sum(timed) / len(timed)
     value = rows * p.n / sec
     cores = len(os.sched_getaffinity(0))
-    cfgd = describe(p, args.config, args.group_size)
+    cfgd = describe(p, args.config, args.group_size, args.tau)
     if args.greedy:
         cfgd["workload"] += " (greedy baseline: LDLQ init, damp 0.01, then the same CD)"
         cfgd["init"] = "LDLQ"
@@ -330,11 +336,10 @@ def run_mpq(args, world, rank, local):
     if args.greedy:
         p.T_vamp = 0
         greedy = {"greedy_init": 1}
-    cfgd = describe(p, args.config, args.group_size)
+    cfgd = describe(p, args.config, args.group_size, args.tau)
     if args.greedy:
         cfgd["workload"] += " (greedy baseline: LDLQ init, damp 0.01, then the same CD)"
         cfgd["init"] = "LDLQ"
-    cfgd["cd_panel"] = args.cd_panel or "auto"
     m, n = p.m_out, p.n
     cb = p.codebook if p.d == 8 else None
     cache = args.spectrum_cache
@@ -342,14 +347,15 @@ def run_mpq(args, world, rank, local):
         z = np.load(cache)
         plan = mpq.Plan.from_spectrum(torch.from_numpy(z["s"]).to(dev),
                                       torch.from_numpy(z["V"]).to(dev), p.d, p.levels, codebook=cb,
-                                      cd_panel=args.cd_panel, group_size=args.group_size, **greedy)
+                                      cd_panel=args.cd_panel, group_size=args.group_size,
+                                      tau=args.tau, **greedy)
         setup_s = None
     else:
         X = torch.from_numpy(p.X).to(dev)
         torch.cuda.synchronize()
         t0 = time.time()
         plan = mpq.Plan.from_x(X, p.d, p.levels, codebook=cb, cd_panel=args.cd_panel,
-                               group_size=args.group_size, **greedy)
+                               group_size=args.group_size, tau=args.tau, **greedy)
         torch.cuda.synchronize()
         setup_s = time.time() - t0
         del X
@@ -488,7 +494,7 @@ def run_mpq(args, world, rank, local):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         times, t_spec = oracle_sample(p, args.cpu_rows, 1, args.group_size,
-                                      0.01 if args.greedy else None)
+                                      0.01 if args.greedy else None, args.tau)
         cpu = {"value": args.cpu_rows * n / times[0], "unit": UNIT,
                "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
                "sample": f"rows 0..{args.cpu_rows - 1} of the layer (independent problems), "
@@ -498,8 +504,10 @@ def run_mpq(args, world, rank, local):
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-                "data": "synthetic", "config": dict(cfgd, setup_s=None if setup_s is None else round(setup_s, 3), rank=r,
-                                                    parallelism=f"rows sharded over {world} GPU(s)"),
+                "data": "synthetic", "config": cfgd,
+                "run": {"setup_s": None if setup_s is None else round(setup_s, 3), "rank": r,
+                        "cd_panel": args.cd_panel or "auto",
+                        "parallelism": f"rows sharded over {world} GPU(s)"},
                 "rows_per_s": world * m / (ms_per_step / 1e3),
                 "objective": {"mean_energy": objective, "what": "mean over rows of "
                               "1/2 |X (w - w_hat)|^2 after the timed solves"},

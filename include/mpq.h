@@ -86,8 +86,15 @@ typedef struct {
                              mapped per row by scale * k + offset) */
   double beta0;           /* initial inverse temperature, default 1 */
   double damping;         /* rho_damp: beta <- (1-rho) beta + rho beta_hat, default 0.5 */
-  double tau;             /* prior anchor scale; INFINITY (default) = uniform rho_b.
-                             Finite tau: rho_b(c) = exp(-(gamma1_0/tau^2)/2 |c - w_b|^2) */
+  double tau;             /* prior anchor scale ([Hyper-parameters]: tau = 0.2,
+                             the default; [Key design 1]: the denoiser works "under
+                             the prior anchor").  The anchor pins each block to its
+                             own weights w_b with a width of tau codebook units
+                             (grid steps for d = 1, lattice units for d = 8):
+                             rho_b(c) = exp(-|c - w_b|^2 / (2 tau^2 scale^2)) with c
+                             in weight units and scale the row's (or group's)
+                             scale.  INFINITY = uniform rho_b, the unanchored
+                             limit of the pages' analysis. */
   double gamma_lo_rel;    /* extrinsic precisions are clipped into        */
   double gamma_hi_rel;    /*   [lo, hi] * gamma1_0 (defaults 1e-10, 1e10) */
   double alpha_min;       /* mean divergences are clipped into            */
@@ -269,9 +276,15 @@ MPQ_API mpq_status mpq_solve_host(mpq_plan_t plan, const float* W_host, int64_t 
                           float* energy_host, mpq_stream_t stream);
 
 /* -------------------------------------------------- stage entry points --- */
-/* Each runs exactly the kernels that mpq_solve runs for one stage, on state
- * the caller injects, so that every stage can be compared on identical
- * inputs.  B = n/d.  Per-row scalars are fp64, vectors fp32. */
+/* Each runs one stage on state the caller injects, so that every stage can
+ * be compared on identical inputs.  B = n/d.  Per-row scalars are fp64,
+ * vectors fp32.  The init, CD and energy hooks, the linear hook and (for
+ * d = 8, and for d = 1 rows too wide for the fused kernel) the denoiser hook
+ * run the kernels mpq_solve runs.  mpq_solve runs the denoiser and the
+ * extrinsic updates of d = 1 rows that fit in shared memory in one fused row
+ * kernel; mpq_stage_denoise and mpq_stage_linear run the separate kernels
+ * for them (same arithmetic, shared device functions), and
+ * mpq_stage_vamp_scalar runs the fused kernel itself. */
 
 /* Init ([Hyper-parameters]): if `given` == 0, compute scale/offset (built-in
  * rule) into scale/offset; else read them.  idx_rtn: m x B nearest codeword
@@ -281,7 +294,8 @@ MPQ_API mpq_status mpq_stage_init(mpq_plan_t plan, const float* W, int64_t m, in
 
 /* Denoiser ([Key design 1]): for every block the posterior over the row's
  * codewords scale*c + offset.  Inputs R1 (m x n), gamma1 (m), scale/offset
- * (m); for a finite-tau plan also W (m x n) and gamma1_0 (m), else NULL.
+ * (m); for a finite-tau plan also W (m x n), the anchor's centre, else NULL.
+ * (gamma1_0 is not read by the denoiser and may be NULL.)
  * Outputs xhat1 (m x n posterior means), vblock (m x B traces of the
  * posterior covariances, may be NULL), vsum (m, fp64 sums of vblock),
  * idx (m x B argmax, lowest index on ties, may be NULL). */
@@ -302,6 +316,33 @@ MPQ_API mpq_status mpq_stage_linear(mpq_plan_t plan, const float* W, int64_t m, 
                             double* gamma1_out, float* R2, double* gamma2, float* Uprime,
                             float* xhat2, double* alpha2, double* beta_hat, int32_t* clamps,
                             mpq_stream_t stream);
+
+/* One VAMP iteration of scalar (d = 1) rows as mpq_solve runs it, on an
+ * injected cavity ([Key design 1] denoiser and extrinsic updates, [Key
+ * design 2] M-step).  mpq_solve runs these rows through one fused row kernel
+ * per iteration, which forms the cavity r1 from the linear module's output
+ * (extrinsic update linear -> denoiser), runs the denoiser and the extrinsic
+ * update denoiser -> linear; this hook runs that same kernel:
+ *   1. fused pass on the cavity (R1, gamma1): denoiser, then r2 and gamma2;
+ *   2. the linear module and beta M-step (as mpq_stage_linear): beta is read
+ *      and overwritten with the damped update, gamma1_out receives gamma1';
+ *   3. if idx_map: the fused MAP pass on the next cavity r1' (argmax);
+ *   4. if R1_out, R2_next or gamma2_next: the next fused pass, which forms
+ *      r1' (written to R1_out) and runs the denoiser and the d2l step on it
+ *      (r2' to R2_next, gamma2' to gamma2_next).
+ *   W, R1: m x n; scale/offset: as mpq_stage_denoise; gamma1, gamma1_0, beta:
+ *   m doubles.  Outputs R2, R1_out, R2_next (m x n floats), gamma2,
+ *   gamma2_next (m doubles), idx_map (m x n) may each be NULL; clamps (m
+ *   ints, added to) may be NULL.  A finite-tau plan anchors the denoiser at W.
+ * MPQ_ERR_UNSUPPORTED unless d = 1 and a row fits the fused kernel's shared
+ * memory (8 bytes per weight; the same rows mpq_solve runs fused). */
+MPQ_API mpq_status mpq_stage_vamp_scalar(mpq_plan_t plan, const float* W, int64_t m,
+                                         const float* scale, const float* offset, const float* R1,
+                                         const double* gamma1, const double* gamma1_0,
+                                         double* beta, float* R2, double* gamma2, float* R1_out,
+                                         double* gamma1_out, uint16_t* idx_map, float* R2_next,
+                                         double* gamma2_next, int32_t* clamps,
+                                         mpq_stream_t stream);
 
 /* Exact block CD ([Key design 3]) from the codewords in idx (m x B, read
  * and overwritten): h = H (w - x), then at most `sweeps` sweeps over the

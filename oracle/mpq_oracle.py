@@ -22,8 +22,11 @@ Readings where the pages are silent (the CUDA library takes the same ones):
   R2  scalar grid: per-row min-max, s=(max-min)/(L-1), z=clip(rint(-min/s)),
       level k = s*(k - z); a constant row uses s = |w| (or 1 for zero).
   R3  lattice scale: codeword c maps to RMS(w) * c.
-  R4  initial cavity r1 = w; beta0 = 1; tau = inf means uniform rho_b.
-      Finite tau adds the anchor log rho_b(c) = -(gamma1_0/tau^2)/2 |c-w_b|^2.
+  R4  initial cavity r1 = w; beta0 = 1.  The prior anchor pins each block
+      to its own weights with a width of tau codebook units (grid steps of a
+      scalar grid, lattice units of a vector codebook):
+      log rho_b(c) = -|c - w_b|^2 / (2 tau^2 scale_b^2) in weight units.
+      tau = 0.2 is the pages' default; tau = inf means uniform rho_b.
   R5  extrinsic updates use the divergence form (identical to the pages'
       eta form when nothing is clipped): mean divergences alpha are clipped
       into [1e-10, 0.99] before the extrinsic mean is formed, and the
@@ -52,6 +55,7 @@ GAMMA_LO_REL = 1e-10
 GAMMA_HI_REL = 1e10
 ALPHA_MIN = 1e-10
 ALPHA_MAX = 0.99
+TAU = 0.2   # anchor scale, [MPQ-note] hyper-parameter section (reading R4)
 
 
 # ----------------------------------------------------------------------------
@@ -210,12 +214,21 @@ class DenoiseOut:
     gap: np.ndarray      # m x B top-two logit gap (for tie exemptions)
 
 
-def denoise(R1, gamma1, codebook, scale, offset, W=None, gamma_anchor=None) -> DenoiseOut:
+def block_scales(scale_i, B: int) -> np.ndarray:
+    """The scale of each of a row's B blocks (its group's with group-wise
+    grids)."""
+    s = np.atleast_1d(np.asarray(scale_i, np.float64))
+    return np.repeat(s, B // s.size)
+
+
+def denoise(R1, gamma1, codebook, scale, offset, W=None, tau: float = math.inf) -> DenoiseOut:
     """[MPQ-note] Key design 1: for every block b and codeword c,
     q_b(c) proportional to rho_b(c) exp(-gamma1/2 |c - r1_b|^2); returns the
     posterior mean, the trace of the posterior covariance and the argmax.
-    With ``gamma_anchor`` (finite tau, reading R4) the prior is
-    rho_b(c) = exp(-gamma_anchor/2 |c - w_b|^2), else uniform."""
+    With a finite ``tau`` the prior anchors the block to its weights w_b
+    ("the prior anchor", ibid.; reading R4):
+    rho_b(c) = exp(-|c - w_b|^2 / (2 tau^2 scale_b^2)), a width of tau
+    codebook units; tau = inf gives the uniform prior."""
     R1 = np.asarray(R1, np.float64)
     m, n = R1.shape
     d = codebook.shape[1]
@@ -228,9 +241,10 @@ def denoise(R1, gamma1, codebook, scale, offset, W=None, gamma_anchor=None) -> D
         cand = block_candidates(codebook, scale[i], offset[i], B)      # B x K x d
         r = R1[i].reshape(B, d)
         logit = -0.5 * gamma1[i] * ((r[:, None, :] - cand) ** 2).sum(axis=2)
-        if gamma_anchor is not None:
+        if math.isfinite(tau):
             wb = np.asarray(W[i], np.float64).reshape(B, d)
-            logit = logit - 0.5 * gamma_anchor[i] * ((wb[:, None, :] - cand) ** 2).sum(axis=2)
+            ga = 1.0 / (tau * tau * block_scales(scale[i], B) ** 2)    # B anchor precisions
+            logit = logit - 0.5 * ga[:, None] * ((wb[:, None, :] - cand) ** 2).sum(axis=2)
         top = np.argmax(logit, axis=1)
         mx = logit[np.arange(B), top]
         q = np.exp(logit - mx[:, None])
@@ -346,6 +360,7 @@ class CDOut:
     sweeps_run: np.ndarray   # m
     first_tie: np.ndarray    # m: global step index of the first near-tie (or -1)
     min_gap_rel: np.ndarray  # m: smallest top-two gap / |E| seen
+    step_gap: np.ndarray     # m x (sweeps*B): top-two gap / |E| of each step (inf: not run)
 
 
 def decode(idx, codebook, scale, offset):
@@ -378,6 +393,7 @@ def cd(W, idx0, codebook, scale, offset, H, sweeps: int, tie_rel: float = 1e-5) 
     sweeps_run = np.zeros(m, dtype=np.int64)
     first_tie = np.full(m, -1, dtype=np.int64)
     min_gap = np.full(m, np.inf)
+    step_gap = np.full((m, sweeps * B), np.inf)
     for i in range(m):
         cand = block_candidates(codebook, scale[i], offset[i], B)      # B x K x d
         x = X[i].copy()
@@ -396,6 +412,7 @@ def cd(W, idx0, codebook, scale, offset, H, sweeps: int, tie_rel: float = 1e-5) 
                 if dE.size > 1:
                     two = np.partition(dE, 1)[:2]
                     g = (two[1] - two[0]) / max(abs(E), 1e-300)
+                    step_gap[i, step] = g
                     min_gap[i] = min(min_gap[i], g)
                     if g < tie_rel and first_tie[i] < 0:
                         first_tie[i] = step
@@ -410,7 +427,7 @@ def cd(W, idx0, codebook, scale, offset, H, sweeps: int, tie_rel: float = 1e-5) 
             if nchg == 0:
                 break
         X[i] = x
-    return CDOut(idx, X, changes, sweeps_run, first_tie, min_gap)
+    return CDOut(idx, X, changes, sweeps_run, first_tie, min_gap, step_gap)
 
 
 # ----------------------------------------------------------------------------
@@ -513,12 +530,14 @@ def terminal_precision(gamma1, scale):
 
 
 def solve(W, codebook, s, V, T_vamp: int, cd_sweeps: int, scale=None, offset=None,
-          beta0: float = 1.0, damping: float = 0.5, tau: float = math.inf,
+          beta0: float = 1.0, damping: float = 0.5, tau: float = TAU,
           keep_trace: bool = False, group: int = 0, cd_skip_precision: float = 0.0,
           greedy_damp: Optional[float] = None) -> SolveOut:
     """The MPQ solve of every row ([MPQ-note] flowchart and Overall
     framework): init -> T_vamp x (denoiser -> extrinsic -> linear module ->
-    M-step) -> marginal MAP argmax -> exact block CD -> energies.
+    M-step) -> marginal MAP argmax -> exact block CD -> energies, with the
+    denoiser's prior anchored at ``tau`` codebook units (default 0.2, the
+    [MPQ-note] hyper-parameter section; tau = inf is the unanchored form).
     With ``cd_skip_precision`` > 0, rows whose terminal precision (see
     terminal_precision) exceeds it keep the marginal MAP and run no CD: the
     [MPQ-note] diagnostics report terminal precisions near 1e5 at 3-bit
@@ -529,12 +548,11 @@ def solve(W, codebook, s, V, T_vamp: int, cd_sweeps: int, scale=None, offset=Non
     W = np.asarray(W, np.float64)
     st = init(W, codebook, scale, offset, beta0, group)
     g10 = st.gamma1.copy()
-    ga = None if not math.isfinite(tau) else g10 / (tau * tau)
     R1, g1, beta = st.R1, st.gamma1.copy(), st.beta.copy()
     clamps = np.zeros(W.shape[0], dtype=np.int64)
     trace = []
     for _ in range(T_vamp):
-        dn = denoise(R1, g1, codebook, st.scale, st.offset, W, ga)
+        dn = denoise(R1, g1, codebook, st.scale, st.offset, W, tau)
         lo = linear_step(W, R1, g1, dn.xhat, dn.vsum, beta, s, V, g10, damping)
         if keep_trace:
             trace.append((dn, lo))
@@ -544,7 +562,7 @@ def solve(W, codebook, s, V, T_vamp: int, cd_sweeps: int, scale=None, offset=Non
         gr = ldlq(W, codebook, st.scale, st.offset, hessian(s, V), greedy_damp)
         idx_map, map_gap = gr.idx, gr.gap
     else:
-        dn = denoise(R1, g1, codebook, st.scale, st.offset, W, ga)
+        dn = denoise(R1, g1, codebook, st.scale, st.offset, W, tau)
         idx_map, map_gap = dn.idx, dn.gap
     cdo = None
     idx = idx_map

@@ -88,6 +88,7 @@ _sig("mpq_solve_host", ST, P, P, I64, I32, I32, P, P, P, P)
 _sig("mpq_stage_init", ST, P, P, I64, I32, P, P, P, P, P)
 _sig("mpq_stage_denoise", ST, P, P, P, P, P, I64, P, P, P, P, P, P, P)
 _sig("mpq_stage_linear", ST, P, P, I64, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P)
+_sig("mpq_stage_vamp_scalar", ST, P, P, I64, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P)
 _sig("mpq_stage_cd", ST, P, P, I64, P, P, P, I32, P, P)
 _sig("mpq_stage_energy", ST, P, P, I64, P, P, P, P, P, P)
 _sig("mpq_stage_energy_noalloc", ST, P, P, I64, P, P, P, P, P, P)
@@ -102,6 +103,7 @@ EXPORTED = ["mpq_params_default", "mpq_plan_create_from_spectrum", "mpq_plan_cre
             "mpq_plan_info", "mpq_plan_get_spectrum", "mpq_plan_status",
             "mpq_plan_workspace_bytes", "mpq_plan_set_workspace_cap", "mpq_solve",
             "mpq_solve_host", "mpq_stage_init", "mpq_stage_denoise", "mpq_stage_linear",
+            "mpq_stage_vamp_scalar",
             "mpq_stage_cd", "mpq_stage_energy", "mpq_stage_energy_noalloc",
             "mpq_profile_start", "mpq_profile_stop",
             "mpq_last_error", "mpq_kernel_launch_count"]
@@ -402,6 +404,33 @@ class Plan:
                                    _ptr(o["gamma2"]), _ptr(o["Uprime"]), _ptr(o["xhat2"]),
                                    _ptr(o["alpha2"]), _ptr(o["beta_hat"]), _ptr(o["clamps"]),
                                    _stream()), "mpq_stage_linear")
+        o["beta"] = beta
+        return o
+
+    def stage_vamp_scalar(self, W, scale, offset, R1, gamma1, gamma1_0, beta, next_pass=True,
+                          map_pass=True):
+        """mpq_stage_vamp_scalar: one iteration of the fused scalar row kernel
+        and the linear module on an injected cavity (R1, gamma1)."""
+        m = W.shape[0]
+        dev = W.device
+        beta = beta.clone()
+        f32 = lambda *sh: torch.empty(*sh, dtype=torch.float32, device=dev)
+        f64 = lambda *sh: torch.empty(*sh, dtype=torch.float64, device=dev)
+        o = {"R2": f32(m, self.n), "gamma2": f64(m), "gamma1": f64(m),
+             "clamps": torch.zeros(m, dtype=torch.int32, device=dev)}
+        if map_pass:
+            o["idx"] = torch.empty(m, self.n, dtype=torch.int16, device=dev)
+        if next_pass:
+            o.update({"R1": f32(m, self.n), "R2_next": f32(m, self.n), "gamma2_next": f64(m)})
+        check(lib.mpq_stage_vamp_scalar(
+            self._h, _ptr(W, torch.float32, (m, self.n), "W"), m,
+            _ptr(scale, torch.float32, self._sshape(m), "scale"),
+            _ptr(offset, torch.float32, self._sshape(m), "offset"),
+            _ptr(R1, torch.float32, (m, self.n), "R1"), _ptr(gamma1, torch.float64, (m,), "gamma1"),
+            _ptr(gamma1_0, torch.float64, (m,), "gamma1_0"), _ptr(beta), _ptr(o["R2"]),
+            _ptr(o["gamma2"]), _ptr(o.get("R1")), _ptr(o["gamma1"]), _ptr(o.get("idx")),
+            _ptr(o.get("R2_next")), _ptr(o.get("gamma2_next")), _ptr(o["clamps"]), _stream()),
+            "mpq_stage_vamp_scalar")
         o["beta"] = beta
         return o
 

@@ -29,8 +29,12 @@
 // Moments.  The weights (c* excluded: its weight 2^8 is added back at the
 // end, which leaves the first moment centred on c* without cancellation) go
 // to shared memory as fp16 hi/lo pairs and one more MMA (N = 16) against the
-// transposed codebook [c_0 .. c_7, 1] accumulates S1 and S0 in TMEM for the
-// whole 128-block tile; only S2 = sum q X (the centred second moment, -1/2
+// transposed codebook [c_0 .. c_7, 1] accumulates S1 and S0 in TMEM over a
+// chunk of MOM_CHUNK codebook tiles (two accumulators take turns); the
+// epilogue adds the chunks' partial sums in fp32, so that no accumulator
+// sums more than a chunk's worth of MMAs (a broad posterior over the whole
+// 65536-word codebook would otherwise lose ~1e-4 to accumulation in one
+// fp32 register); only S2 = sum q X (the centred second moment, -1/2
 // |c - c*|^2 per codeword) and the exponential stay on the ALU.  A weight
 // more than 2^8 times c*'s (the argmax pass's fp32 scores misjudged a
 // near-tie at an enormous g) would overflow the fp16 weights: that block
@@ -84,7 +88,8 @@ constexpr int T1_BUFS = 4, T2_BUFS = 2;
 // weight tiles in shared memory: more than the TMEM score buffers, so that
 // the epilogue can run ahead of the moment MMAs that still read older halves
 constexpr int QW_BUFS = 4;
-constexpr uint32_t T1_COLS = 128, T2_COLS = 192, TM_MOM = 384;
+constexpr uint32_t T1_COLS = 128, T2_COLS = 192, TM_MOM = 384;  // moments: 2 x 16 columns
+constexpr int MOM_CHUNK = 16;              // codebook tiles per moment accumulator
 constexpr uint32_t IDESC_P1 = idesc_f16(DT_M, DT_N);
 constexpr uint32_t IDESC_P2 = idesc_f16(DT_M, DT_N2);
 constexpr uint32_t IDESC_MOM = idesc_f16(DT_M, 16);
@@ -98,7 +103,7 @@ constexpr int SM_QW = SM_B + DT_STAGES * STAGE_BYTES;     // QW_BUFS x (hi | lo)
 constexpr int SM_T = SM_QW + QW_BUFS * 2 * QW_BYTES;      // t per row (fp64, 128 x 8)
 constexpr int SM_ROW = SM_T + DT_M * 8 * 8;               // per-row data
 constexpr int SM_BAR = SM_ROW + (3 + 2 * DT_WGS + DT_WGS) * DT_M * 4;
-constexpr int N_BARS = 2 * DT_STAGES + 2 * T1_BUFS + 2 * T2_BUFS + 1 + 2 * QW_BUFS + 1;
+constexpr int N_BARS = 2 * DT_STAGES + 2 * T1_BUFS + 2 * T2_BUFS + 1 + 2 * QW_BUFS + 4;
 constexpr int SM_END = SM_BAR + N_BARS * 8 + 16;
 constexpr int DT_SMEM_BYTES = 220 * 1024;  // > half of the SM: one CTA (and TMEM owner) per SM
 static_assert(SM_END + 1024 <= DT_SMEM_BYTES, "denoiser shared memory");
@@ -239,8 +244,9 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_denoise_vec_tc(DenoiseTcArgs 
   uint64_t* a_full = t2_empty + T2_BUFS;
   uint64_t* q_full = a_full + 1;
   uint64_t* q_free = q_full + QW_BUFS;
-  uint64_t* mom_done = q_free + QW_BUFS;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mom_done + 1);
+  uint64_t* mom_full = q_free + QW_BUFS;  // [2]: a chunk's moment MMAs are done
+  uint64_t* mom_free = mom_full + 2;      // [2]: the epilogue has read that accumulator
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mom_free + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -265,7 +271,10 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_denoise_vec_tc(DenoiseTcArgs 
       mbar_init(&q_free[b], 1);
     }
     mbar_init(a_full, DT_M);
-    mbar_init(mom_done, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&mom_full[b], 1);
+      mbar_init(&mom_free[b], 4);  // the four warps of warpgroup 0
+    }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -314,8 +323,9 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_denoise_vec_tc(DenoiseTcArgs 
   } else if (warp == MMA_WARP) {
     // ------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      uint32_t seq = 0, tu1 = 0, hq = 0, aphase = 0;
+      uint32_t seq = 0, tu1 = 0, hq = 0, aphase = 0, cbase = 0;
       bool ok = true;
+      const uint32_t nch = (uint32_t)((a.NT + MOM_CHUNK - 1) / MOM_CHUNK);  // chunks per tile
       const uint32_t a_base = smem_u32(At);
       const uint32_t qw_base = smem_u32(smem + SM_QW);
       for (int64_t mt = blockIdx.x; mt < mtiles && ok; mt += gridDim.x) {
@@ -369,20 +379,31 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_denoise_vec_tc(DenoiseTcArgs 
           }
           if (um < us) {
             const uint32_t u = hq + um, qb = u % QW_BUFS;
-            if (mbar_test_wait(&q_full[qb], (u / QW_BUFS) & 1)) {
+            // the chunk of codebook tiles this half belongs to, and its
+            // moment accumulator (two take turns; a chunk's first MMA waits
+            // until the epilogue has read that accumulator's previous chunk)
+            const uint32_t jt = um >> 1, c = cbase + jt / MOM_CHUNK, mb = c & 1;
+            const bool cfirst = (um & 1) == 0 && jt % MOM_CHUNK == 0;
+            const bool clast = (um & 1) == 1 &&
+                               (jt % MOM_CHUNK == MOM_CHUNK - 1 || jt == (uint32_t)a.NT - 1);
+            bool ready = mbar_test_wait(&q_full[qb], (u / QW_BUFS) & 1);
+            if (ready && cfirst && c >= 2) ready = mbar_test_wait(&mom_free[mb], ((c >> 1) - 1) & 1);
+            if (ready) {
               tc_fence_after();
               const int s = (seq + (um >> 1)) % DT_STAGES;
               const uint32_t wq = qw_base + qb * 2u * QW_BYTES;
               const uint32_t bt = smem_u32(smem + SM_B + s * STAGE_BYTES + OPER_BYTES) + (um & 1) * 1024u;
+              const uint32_t dm = tmem + TM_MOM + 16u * mb;
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk) {  // weights (hi, lo) x transposed codebook
                 const uint64_t bd = kmajor_desc(bt + kk * 256u, 2048);
-                umma_f16(tmem + TM_MOM, kmajor_desc(wq + kk * 256u, 1024), bd, IDESC_MOM,
-                         (um == 0 && kk == 0) ? 0u : 1u);
-                umma_f16(tmem + TM_MOM, kmajor_desc(wq + QW_BYTES + kk * 256u, 1024), bd, IDESC_MOM, 1u);
+                umma_f16(dm, kmajor_desc(wq + kk * 256u, 1024), bd, IDESC_MOM,
+                         (cfirst && kk == 0) ? 0u : 1u);
+                umma_f16(dm, kmajor_desc(wq + QW_BYTES + kk * 256u, 1024), bd, IDESC_MOM, 1u);
               }
               umma_commit(&q_free[qb]);
               if (um & 1) umma_commit(&b_empty[s]);  // both halves of the stage are done
+              if (clast) umma_commit(&mom_full[mb]);
               ++um;
               prog = true;
             }
@@ -402,9 +423,9 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_denoise_vec_tc(DenoiseTcArgs 
           ok = false;
           break;
         }
-        umma_commit(mom_done);
         seq += a.NT;
         hq += total;
+        cbase += nch;
       }
       // the MMAs in flight finish before TMEM is released
       for (uint32_t q = (tu1 > T1_BUFS ? tu1 - T1_BUFS : 0); q < tu1; ++q)
@@ -426,6 +447,25 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_denoise_vec_tc(DenoiseTcArgs 
     const int w_off = kmaj_off(rl, wg * 16, 1024);  // this thread's 16 weights of a half
     uint32_t tu1 = 0, hq = 0, mt_n = 0;
     bool ok = true;
+    const uint32_t nch = (uint32_t)((a.NT + MOM_CHUNK - 1) / MOM_CHUNK);  // chunks per tile
+    // warpgroup 0: the moment chunks' running sums of its row (S1 x 8, S0),
+    // in the shared slot of t, which pass 2 no longer reads once its
+    // operands are built
+    float* msum = reinterpret_cast<float*>(sm_t) + rl * 16;
+    auto read_chunk = [&](uint32_t cl) {
+      const uint32_t c = mt_n * nch + cl, mb = c & 1;
+      if (ok) ok = warp_wait(&mom_full[mb], (c >> 1) & 1, abort_flag, a.status);
+      if (!ok) return;
+      tc_fence_after();
+      uint32_t mv[16];
+      tmem_ld16_nowait(t_lane + TM_MOM + 16u * mb, mv);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&mom_free[mb]);
+#pragma unroll
+      for (int i = 0; i < 9; ++i) msum[i] = (cl == 0 ? 0.0f : msum[i]) + __uint_as_float(mv[i]);
+    };
     for (int64_t mt = blockIdx.x; mt < mtiles; mt += gridDim.x) {
       const int64_t blk = mt * DT_M + rl;
       const bool active = blk < a.nblocks;
@@ -446,7 +486,7 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_denoise_vec_tc(DenoiseTcArgs 
           double gg = 1.0, ga = 0.0;
           if (!a.nearest_only) {
             gg = a.gamma1[row] * sc2;
-            ga = a.W ? a.gamma1_0[row] * a.inv_tau2 * sc2 : 0.0;
+            ga = a.W ? a.inv_tau2 : 0.0;  // anchor: tau codebook units wide
           }
           g = (float)fmin(gg + ga, 1e30);
 #pragma unroll
@@ -583,7 +623,11 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_denoise_vec_tc(DenoiseTcArgs 
       float zmax = -INFINITY;
       uint64_t S2p = 0;  // (+0, +0): S2 over even and odd codewords
       const uint64_t rs2 = f2_pack(rs, rs), g22 = f2_pack(g2, g2), sh2 = f2_pack(Q_SHIFT, Q_SHIFT);
+      uint32_t rd = 0;  // moment chunks read (warpgroup 0)
       for (int j = 0; j < a.NT; ++j) {
+        // a chunk is read one codebook tile into the next chunk, by when its
+        // moment MMAs have long been issued
+        if (wg == 0 && j > MOM_CHUNK && (j - 1) % MOM_CHUNK == 0) read_chunk(rd++);
 #pragma unroll 1
         for (int h = 0; h < 2; ++h, ++hq) {
           const int buf = hq % T2_BUFS, qb = hq % QW_BUFS;
@@ -655,14 +699,10 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_denoise_vec_tc(DenoiseTcArgs 
         // S0 = sum q, S1 = sum q c over c != c* (weights x 2^8) from the
         // moment accumulator; c* adds 2^8 to S0, 2^8 c* to S1 and 0 to S2:
         // E[c - c*] = (S1 - c* S0) / (2^8 + S0), E|c - c*|^2 = -2 S2 / (2^8 + S0)
-        if (ok) ok = warp_wait(mom_done, mt_n & 1, abort_flag, a.status);
-        uint32_t mv[16];
-        if (ok) {
-          tc_fence_after();
-          tmem_ld16_nowait(t_lane + TM_MOM, mv);
-          tmem_wait_ld();
-          tc_fence_before();
-        }
+        for (; rd < nch; ++rd) read_chunk(rd);
+        float mv[9];
+#pragma unroll
+        for (int i = 0; i < 9; ++i) mv[i] = msum[i];
         if (active && ok) {
           const int bi = sm_bidx[rl];
           const float4 c0 = *reinterpret_cast<const float4*>(a.cb + (int64_t)bi * 8);
@@ -674,7 +714,7 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_denoise_vec_tc(DenoiseTcArgs 
             s2 += sm_s2[w * DT_M + rl];
             zm = fmaxf(zm, sm_bval[w * DT_M + rl]);
           }
-          const float S0 = __uint_as_float(mv[8]);
+          const float S0 = mv[8];
           const float sc = a.scale[row], off = a.offset[row];
           const float inv = 1.0f / (256.0f + S0);
           // a weight past the fp16 range (more than 2^8 times c*'s): point mass
@@ -682,7 +722,7 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_denoise_vec_tc(DenoiseTcArgs 
           float mm = 0.0f, xo[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            const float mc = point ? 0.0f : fmaf(-cst[i], S0, __uint_as_float(mv[i])) * inv;
+            const float mc = point ? 0.0f : fmaf(-cst[i], S0, mv[i]) * inv;
             mm = fmaf(mc, mc, mm);
             xo[i] = fmaf(sc, cst[i] + mc, off);
           }

@@ -51,6 +51,8 @@ __device__ __forceinline__ void p_tile(int t, int mtiles, int ntiles, int& m0, i
   n0 = (w / gm) * PBN;
 }
 
+// LIN = 1: the linear module's epilogue (LinEpi) instead of storing C.
+template <int LIN>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     k_gemm_tcp(const __grid_constant__ CUtensorMap ta_hi, const __grid_constant__ CUtensorMap ta_lo,
                const __grid_constant__ CUtensorMap tb_hi, const __grid_constant__ CUtensorMap tb_lo,
@@ -58,7 +60,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                int n_off,
                const float* __restrict__ row_scale, float b_scale, int accumulate, int a_exact,
                const int* __restrict__ gate, const __grid_constant__ CUtensorMap tc_out,
-               int use_reduce, int* status) {
+               int use_reduce, int* status, const __grid_constant__ LinEpi le) {
   if (gate != nullptr && *gate == 0) return;  // nothing to add
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -183,6 +185,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       const int row = m0 + q * 32 + lane;
       const float rs = (row < M) ? row_scale[row] * b_scale : 0.0f;
       const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)buf * PBN;
+      // linear epilogue: this row's beta and gamma2, its M-step sums over the
+      // tile's columns, and the operand scale b_scale 2^-e_bound (the row's
+      // own 2^e_row cancels: p' = acc 2^e_row b_scale)
+      float lb = 0.0f, lg2 = 0.0f, a2s = 0.0f, bsum = 0.0f;
+      const float qk = LIN ? b_scale * ldexpf(1.0f, -le.e_bound) : 0.0f;
+      if (LIN && row < M) {
+        lb = (float)le.beta[row];
+        lg2 = (float)le.gamma2[row];
+      }
       for (int c0 = 0; c0 < PBN; c0 += 32) {
         uint32_t v[32];
         tmem_ld32(tbase + (uint32_t)c0, v);
@@ -192,6 +203,48 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           if (lane == 0) mbar_arrive(&tm_empty[buf]);
         }
         if (n0 + c0 >= N) continue;
+        if constexpr (LIN) {
+          // per element as the M-step states it, in fp32; columns past N are
+          // written as zero (the operand's K padding)
+          if (row < M) {
+            uint32_t hv[16], lv[16];
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+              float qs[2];
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                const int col = n0 + c0 + j + e;
+                const float acc = __uint_as_float(v[j + e]);
+                qs[e] = 0.0f;
+                if (col < N) {
+                  const float sl = __ldg(le.s32 + col);
+                  const float pl = acc * rs;
+                  const float u = sl * pl;
+                  const float den = fmaf(lb * sl, sl, lg2);  // > 0
+                  const float inv = __fdividef(1.0f, den);
+                  const float f = lg2 * inv;
+                  a2s += f;
+                  bsum += fmaf(f * f * u, u, sl * sl * inv);
+                  qs[e] = (le.full_rank ? -f : 1.0f - f) * acc * qk;
+                  if (le.Uprime) le.Uprime[(int64_t)row * N + col] = (1.0f - f) * pl;
+                }
+              }
+              const __half2 h = __floats2half2_rn(qs[0], qs[1]);
+              const float2 hf = __half22float2(h);
+              const __half2 l = __floats2half2_rn(qs[0] - hf.x, qs[1] - hf.y);
+              hv[j / 2] = *reinterpret_cast<const uint32_t*>(&h);
+              lv[j / 2] = *reinterpret_cast<const uint32_t*>(&l);
+            }
+            uint4* qh = reinterpret_cast<uint4*>(le.q_hi + (int64_t)row * le.ldq + n0 + c0);
+            uint4* ql = reinterpret_cast<uint4*>(le.q_lo + (int64_t)row * le.ldq + n0 + c0);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              qh[k] = make_uint4(hv[4 * k], hv[4 * k + 1], hv[4 * k + 2], hv[4 * k + 3]);
+              ql[k] = make_uint4(lv[4 * k], lv[4 * k + 1], lv[4 * k + 2], lv[4 * k + 3]);
+            }
+          }
+          continue;
+        }
         if (use_reduce) {
           // accumulate through the TMA unit: a 32 x 32 block in a
           // 128B-swizzled buffer (two per warp, alternating), tensor
@@ -236,6 +289,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           __syncwarp();
         }
       }
+      if (LIN && row < M) le.part[(int64_t)row * le.ntiles + n0 / PBN] = make_float2(a2s, bsum);
     }
     if (use_reduce && lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
     __syncwarp();
@@ -367,22 +421,28 @@ mpq_status gemm_tc(const SplitOperand& A, const CUtensorMap& ta_hi, const CUtens
   int dev = 0;
   MPQ_CUDA(cudaGetDevice(&dev));
   if (dev >= 0 && dev < 64 && !g_smem_attr_set[dev]) {
-    MPQ_CUDA(cudaFuncSetAttribute(k_gemm_tcp, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM));
+    MPQ_CUDA(cudaFuncSetAttribute(k_gemm_tcp<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM));
+    MPQ_CUDA(cudaFuncSetAttribute(k_gemm_tcp<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM));
     MPQ_CUDA(cudaDeviceGetAttribute(&g_sms[dev], cudaDevAttrMultiProcessorCount, dev));
     g_smem_attr_set[dev] = true;
   }
   if (o.c_reduce && !o.accumulate)
     return fail(MPQ_ERR_INVALID_ARG, "gemm_tc: reduce output needs accumulate");
+  if (o.lin && (o.c_reduce || o.accumulate || o.n0 != 0 || o.lin->ldq < round_up(N, PBN) ||
+                o.lin->ntiles != cdiv(N, PBN) || (o.lin->ldq % 8) != 0))
+    return fail(MPQ_ERR_INVALID_ARG, "gemm_tc: linear epilogue needs a plain product over all N");
   const int64_t tiles = cdiv(M, BM) * cdiv(N, PBN);
   const unsigned grid = (unsigned)std::min<int64_t>(tiles, dev < 64 ? g_sms[dev] : 148);
   const CUtensorMap& cmap = o.c_reduce ? *o.c_reduce : tb_hi;  // unused unless reducing
   {
     ProfScope ps_(tag, st);
-    k_gemm_tcp<<<grid, TC_THREADS, P_SMEM, st>>>(
+    const LinEpi le = o.lin ? *o.lin : LinEpi{};
+    auto kern = o.lin ? k_gemm_tcp<1> : k_gemm_tcp<0>;
+    kern<<<grid, TC_THREADS, P_SMEM, st>>>(
         ta_hi, ta_lo, tb_hi, tb_lo, C, ldc, (int)M, (int)N, (int)K, (int)o.a_k0, (int)o.b_k0,
         (int)o.n0, A.row_unscale,
         b_scale_host, o.accumulate ? 1 : 0, o.a_exact ? 1 : 0, o.gate, cmap, o.c_reduce ? 1 : 0,
-        status);
+        status, le);
   }
   count_launch();
   return check_launch("k_gemm_tc");

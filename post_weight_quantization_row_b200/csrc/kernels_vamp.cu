@@ -268,9 +268,10 @@ struct ScalarDen {
   bool anchored, precise;
 };
 
+// The prior anchor (reading of the pages' "anchor scale" tau) has a width of
+// tau grid steps: its precision in level units is 1/tau^2 for every row.
 __device__ __forceinline__ ScalarDen scalar_den_row(float sc, float off, double gamma1, int L,
-                                                    bool anchored, double gamma1_0,
-                                                    double inv_tau2) {
+                                                    bool anchored, double inv_tau2) {
   ScalarDen c;
   c.sc = sc;
   c.off = off;
@@ -280,7 +281,7 @@ __device__ __forceinline__ ScalarDen scalar_den_row(float sc, float off, double 
   const double sc2 = dsc * dsc;
   c.g = fmin(gamma1 * sc2, 1e30);
   c.anchored = anchored;
-  c.ga = anchored ? fmin(gamma1_0 * inv_tau2 * sc2, 1e30) : 0.0;
+  c.ga = anchored ? fmin(inv_tau2, 1e30) : 0.0;
   c.geff = c.g + c.ga;
   c.A2 = (float)(-0.5 * c.geff * 1.4426950408889634);  // -geff/2 log2(e)
   c.L = L;
@@ -430,11 +431,11 @@ __global__ void __launch_bounds__(ROW_THREADS)
   const bool anchored = (W != nullptr);
   const int ng = GROUPED ? (int)(n / G) : 1;
   const ScalarDen c = scalar_den_row(scale[row * ng], offset[row * ng], gamma1[row], L, anchored,
-                                     anchored ? gamma1_0[row] : 0.0, inv_tau2);
+                                     inv_tau2);
   if (GROUPED) {
     for (int g = threadIdx.x; g < ng; g += blockDim.x)
       s_den[g] = scalar_den_row(scale[row * ng + g], offset[row * ng + g], gamma1[row], L,
-                                anchored, anchored ? gamma1_0[row] : 0.0, inv_tau2);
+                                anchored, inv_tau2);
     __syncthreads();
   }
   // the per-weight loop, instantiated once per precision regime and prior so
@@ -524,7 +525,7 @@ __global__ void __launch_bounds__(VEC_THREADS) k_denoise_vec(VecDenoiseArgs a) {
     double gg = 1.0, ga = 0.0;
     if (!a.nearest_only) {
       gg = a.gamma1[row] * sc2;
-      ga = a.W ? a.gamma1_0[row] * a.inv_tau2 * sc2 : 0.0;
+      ga = a.W ? a.inv_tau2 : 0.0;  // anchor: tau codebook units wide
     }
     g = (float)fmin(gg + ga, 1e30);
 #pragma unroll
@@ -703,125 +704,48 @@ __global__ void __launch_bounds__(ROW_THREADS)
   if (threadIdx.x == 0) a_unscale[row] = ldexpf(1.0f, ex);
 }
 
-// -------------------------------------- linear module epilogue + M-step ---
-// P holds p' = V^T (w - r2) (m x r).  u = s p', F = gamma2/(beta s^2 +
-// gamma2), D u = (1 - F) p', alpha2 = [sum F + n - r]/n,
-// 1/beta_hat = (1/r) sum[F^2 u^2 + s^2/(beta s^2 + gamma2)],
-// beta <- (1-rho) beta + rho beta_hat, gamma1' = gamma2 (1-alpha2)/alpha2
-// (clipped), coef = 1/(1 - alpha2), kappa = alpha2/(1 - alpha2).
-// GEMM2 operand (written into P, then split for the tensor cores, K = r):
-//   r < n: (1 - F) p'            -> G = V (D u) = xhat2 - r2
-//   r = n: -F p'                 -> G = xhat2 - w  (V V^T = I), which avoids
-//          forming r2 + V V^T (w - r2) when r2 is far from w.
-__global__ void __launch_bounds__(1024)
-    k_linear_rows(float* __restrict__ P, int64_t n, int64_t r, const float* __restrict__ s32,
-                  const double* __restrict__ gamma2, const double* __restrict__ gamma1_0,
-                  double* __restrict__ beta, double damping, double glo, double ghi,
-                  double amin, double amax, int full_rank, double* __restrict__ gamma1_out,
-                  double* __restrict__ coef, double* __restrict__ kappa,
-                  double* __restrict__ alpha2_out, double* __restrict__ beta_hat_out,
-                  int32_t* __restrict__ clamps, float* __restrict__ Uprime,
-                  __half* __restrict__ ahi, __half* __restrict__ alo, int64_t lda, int64_t ldr,
-                  float* __restrict__ a_unscale, int q_in_smem) {
-  __shared__ double ds_a[32], ds_b[32];
-  __shared__ float fs_m[32];
-  __shared__ double tot_a, tot_b;
-  __shared__ float tot_m;
-  extern __shared__ float s_q[];  // the row's GEMM2 operand when it fits
-  const int64_t row = blockIdx.x;
-  const int rr = (int)r;
-  const int bs = blockDim.x;
-  float* qrow = q_in_smem ? s_q : P + row * r;
-  const float* Pr = P + row * r;
+// ------------------------------------------------------ M-step finisher ---
+// The projection GEMM's linear epilogue left, per row and column tile of
+// 128 rank components, sum F and sum F^2 u^2 + s^2/(beta s^2 + gamma2) with
+// u = s p', F = gamma2/(beta s^2 + gamma2) (the MPQ note's key design 2:
+// 1/beta_hat = (1/r) sum_l [(gamma2/(beta s_l^2 + gamma2))^2 u_l^2 +
+// s_l^2/(beta s_l^2 + gamma2)]).  One thread per row adds the tiles in order
+// in fp64, then: alpha2 = [sum F + n - r]/n (reading R6), beta_hat, beta <-
+// (1 - rho) beta + rho beta_hat (R7), gamma1' = gamma2 (1 - alpha2)/alpha2
+// and the l2d coefficients 1/(1 - alpha2), alpha2/(1 - alpha2), each clipped
+// (R5), and the second GEMM's row scale 2^(e_row + e_bound).
+__global__ void __launch_bounds__(128)
+    k_linear_finish(const float2* __restrict__ part, int ntiles, int64_t m, int64_t n, int64_t r,
+                    int e_bound, const float* __restrict__ a_unscale,
+                    float* __restrict__ q_unscale, const double* __restrict__ gamma2,
+                    const double* __restrict__ gamma1_0, double* __restrict__ beta,
+                    double damping, double glo, double ghi, double amin, double amax,
+                    double* __restrict__ gamma1_out, double* __restrict__ coef,
+                    double* __restrict__ kappa, double* __restrict__ alpha2_out,
+                    double* __restrict__ beta_hat_out, int32_t* __restrict__ clamps) {
+  const int64_t row = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (row >= m) return;
+  const float2* pr = part + row * ntiles;
+  double a2tot = 0.0, bstot = 0.0;
+  for (int t = 0; t < ntiles; ++t) {
+    const float2 v = pr[t];
+    a2tot += (double)v.x;
+    bstot += (double)v.y;
+  }
+  q_unscale[row] = ldexpf(a_unscale[row], e_bound);
+  int cnt = 0;
   const double b = beta[row], g2 = gamma2[row];
-  // per element in fp32 (relative error ~1e-7); per-thread partial sums in
-  // fp32 (a few dozen terms), the block sum in fp64
-  float a2s = 0.0f, bsum = 0.0f, mx = 0.0f;
-  const float bf = (float)b, g2f = (float)g2;
-  auto element = [&](const int l, const float sl, const float pl) {
-    const float u = sl * pl;
-    const float den = fmaf(bf * sl, sl, g2f);  // > 0
-    const float inv = __fdividef(1.0f, den);
-    const float f = g2f * inv;
-    a2s += f;
-    bsum += fmaf(f * f * u, u, sl * sl * inv);
-    if (Uprime) Uprime[row * r + l] = (1.0f - f) * pl;
-    const float q = full_rank ? -f * pl : (1.0f - f) * pl;
-    qrow[l] = q;
-    mx = fmaxf(mx, fabsf(q));
-  };
-  // whole batches of ROW_UNROLL elements per thread without bounds checks,
-  // then the tail one element at a time
-  const int full = rr / (ROW_UNROLL * bs) * (ROW_UNROLL * bs);
-  for (int l0 = threadIdx.x; l0 < full; l0 += ROW_UNROLL * bs) {
-    float sv[ROW_UNROLL], pv[ROW_UNROLL];
-#pragma unroll
-    for (int u = 0; u < ROW_UNROLL; ++u) {
-      sv[u] = s32[l0 + u * bs];
-      pv[u] = Pr[l0 + u * bs];
-    }
-#pragma unroll
-    for (int u = 0; u < ROW_UNROLL; ++u) element(l0 + u * bs, sv[u], pv[u]);
-  }
-  for (int l = full + threadIdx.x; l < rr; l += bs) element(l, s32[l], Pr[l]);
-  // the three row reductions in one pass: warps, then warp 0
-  {
-    double da = a2s, db = bsum;
-    float m = mx;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      da += __shfl_xor_sync(0xffffffffu, da, o);
-      db += __shfl_xor_sync(0xffffffffu, db, o);
-      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    }
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = (bs + 31) >> 5;
-    if (lane == 0) {
-      ds_a[wid] = da;
-      ds_b[wid] = db;
-      fs_m[wid] = m;
-    }
-    __syncthreads();
-    if (wid == 0) {
-      da = lane < nw ? ds_a[lane] : 0.0;
-      db = lane < nw ? ds_b[lane] : 0.0;
-      m = lane < nw ? fs_m[lane] : 0.0f;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        da += __shfl_xor_sync(0xffffffffu, da, o);
-        db += __shfl_xor_sync(0xffffffffu, db, o);
-        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-      }
-      if (lane == 0) {
-        tot_a = da;
-        tot_b = db;
-        tot_m = m;
-      }
-    }
-    __syncthreads();
-  }
-  const double a2tot = tot_a, bstot = tot_b;
-  const int ex = split_exponent(tot_m);
-  const float down = ldexpf(1.0f, -ex);
-  __half* ahr = ahi + row * lda;
-  __half* alr = alo + row * lda;
-  const int ldrr = (int)ldr;
-  for (int l = threadIdx.x; l < ldrr; l += bs)
-    split_store(l < rr ? qrow[l] * down : 0.0f, ahr, alr, l);
-  if (threadIdx.x == 0) {
-    a_unscale[row] = ldexpf(1.0f, ex);
-    int cnt = 0;
-    const double alpha2 = (a2tot + (double)(n - r)) / (double)n;
-    const double bhat = (double)r / bstot;
-    beta[row] = (1.0 - damping) * b + damping * bhat;
-    const double a2 = clip_count(alpha2, amin, amax, &cnt);
-    const double g0 = gamma1_0[row];
-    gamma1_out[row] = clip_count(g2 * (1.0 - a2) / a2, glo * g0, ghi * g0, &cnt);
-    coef[row] = 1.0 / (1.0 - a2);
-    kappa[row] = a2 / (1.0 - a2);
-    if (alpha2_out) alpha2_out[row] = alpha2;
-    if (beta_hat_out) beta_hat_out[row] = bhat;
-    if (clamps) clamps[row] += cnt;
-  }
+  const double alpha2 = (a2tot + (double)(n - r)) / (double)n;
+  const double bhat = (double)r / bstot;
+  beta[row] = (1.0 - damping) * b + damping * bhat;
+  const double a2 = clip_count(alpha2, amin, amax, &cnt);
+  const double g0 = gamma1_0[row];
+  gamma1_out[row] = clip_count(g2 * (1.0 - a2) / a2, glo * g0, ghi * g0, &cnt);
+  coef[row] = 1.0 / (1.0 - a2);
+  kappa[row] = a2 / (1.0 - a2);
+  if (alpha2_out) alpha2_out[row] = alpha2;
+  if (beta_hat_out) beta_hat_out[row] = bhat;
+  if (clamps) clamps[row] += cnt;
 }
 
 // ------------------------------------------------- extrinsic linear -> d ---
@@ -873,6 +797,9 @@ __global__ void __launch_bounds__(ROW_THREADS)
 // in shared memory between the two halves; each arithmetic step is the one
 // of the separate kernels, in the same order.  MAP = 1: the marginal MAP
 // after the last iteration (l2d and the denoiser's argmax only).
+// first: 0 = r1 from the l2d step; 1 = r1 = w (the solve's first iteration);
+// 2 = r1 read from G (an injected cavity, for the per-stage hook).  R1o, if
+// not NULL, receives the r1 the kernel forms.
 constexpr int FUSED_MAX_THREADS = 1024;
 
 template <int MAP, bool GROUPED>
@@ -886,7 +813,8 @@ __global__ void __launch_bounds__(FUSED_MAX_THREADS)
                       double ghi, double amin, double amax, __half* __restrict__ ahi,
                       __half* __restrict__ alo, int64_t lda, int64_t ldn,
                       float* __restrict__ a_unscale, double* __restrict__ gamma2,
-                      int32_t* __restrict__ clamps, uint16_t* __restrict__ idx) {
+                      int32_t* __restrict__ clamps, uint16_t* __restrict__ idx,
+                      float* __restrict__ R1o) {
   extern __shared__ float vrow[];  // r1 (then r2) and x_hat1 of the row
   __shared__ double ds[33];
   __shared__ float fs[33];
@@ -901,15 +829,17 @@ __global__ void __launch_bounds__(FUSED_MAX_THREADS)
   float* R2r = R2 + row * n;
   const int ng = GROUPED ? nn / gsize : 1;
   const ScalarDen c = scalar_den_row(scale[row * ng], offset[row * ng], gamma1[row], L,
-                                     anchored != 0, anchored ? gamma1_0[row] : 0.0, inv_tau2);
+                                     anchored != 0, inv_tau2);
   if (GROUPED) {
     for (int g = threadIdx.x; g < ng; g += blockDim.x)
       s_den[g] = scalar_den_row(scale[row * ng + g], offset[row * ng + g], gamma1[row], L,
-                                anchored != 0, anchored ? gamma1_0[row] : 0.0, inv_tau2);
+                                anchored != 0, inv_tau2);
     __syncthreads();
   }
   const float lc = first ? 0.0f : (float)coef[row];
   const float lk = first ? 0.0f : (float)kappa[row];
+  const bool injected = first == 2;
+  float* R1or = R1o ? R1o + row * n : nullptr;
   const int bs = blockDim.x;
   // whole batches of ROW_UNROLL weights per thread (loads first, no bounds
   // checks), then the tail one weight at a time
@@ -919,7 +849,11 @@ __global__ void __launch_bounds__(FUSED_MAX_THREADS)
     constexpr bool ANCH = decltype(anch)::value;
     float acc = 0.0f;
     auto one = [&](const int j, const float g, const float r2, const float w) {
-      const float r1 = first ? w : full_rank ? fmaf(lc, g, fmaf(lk, w - r2, w)) : fmaf(lc, g, r2);
+      const float r1 = injected ? g
+                       : first  ? w
+                       : full_rank ? fmaf(lc, g, fmaf(lk, w - r2, w))
+                                   : fmaf(lc, g, r2);
+      if (R1or) R1or[j] = r1;
       float xh, ks, v;
       if constexpr (GROUPED) {
         const ScalarDen& cg = s_den[j / gsize];  // uniform over a warp (gsize % 32 == 0)
@@ -941,7 +875,7 @@ __global__ void __launch_bounds__(FUSED_MAX_THREADS)
 #pragma unroll
       for (int u = 0; u < ROW_UNROLL; ++u) {
         const int j = j0 + u * bs;
-        gv[u] = first ? 0.0f : Gr[j];
+        gv[u] = (first == 1) ? 0.0f : Gr[j];
         r2v[u] = first ? 0.0f : R2r[j];
         wv[u] = Wr[j];
       }
@@ -949,7 +883,7 @@ __global__ void __launch_bounds__(FUSED_MAX_THREADS)
       for (int u = 0; u < ROW_UNROLL; ++u) one(j0 + u * bs, gv[u], r2v[u], wv[u]);
     }
     for (int j = full + threadIdx.x; j < nn; j += bs)
-      one(j, first ? 0.0f : Gr[j], first ? 0.0f : R2r[j], Wr[j]);
+      one(j, (first == 1) ? 0.0f : Gr[j], first ? 0.0f : R2r[j], Wr[j]);
     return acc;
   };
   using T_ = std::true_type;
@@ -1231,30 +1165,22 @@ mpq_status launch_extrinsic_d2l(const mpq_plan_s* p, const float* W, int64_t m, 
   return check_launch("k_extrinsic_d2l");
 }
 
-mpq_status launch_linear_rows(const mpq_plan_s* p, int64_t m, const float* P,
-                              const double* gamma2, const double* gamma1_0, double* beta,
-                              double* gamma1_out, double* coef, double* kappa, double* alpha2,
-                              double* beta_hat, int32_t* clamps, float* Uprime, SplitOperand* As,
-                              cudaStream_t st) {
+mpq_status launch_linear_finish(const mpq_plan_s* p, int64_t m, const float2* part, int ntiles,
+                                int e_bound, const float* a_unscale, float* q_unscale,
+                                const double* gamma2, const double* gamma1_0, double* beta,
+                                double* gamma1_out, double* coef, double* kappa, double* alpha2,
+                                double* beta_hat, int32_t* clamps, cudaStream_t st) {
   if (m <= 0) return MPQ_OK;
   const mpq_params& q = p->params;
   {
-    // the row's operand stays on chip between its two passes when it fits
-    const size_t qbytes = sizeof(float) * p->r;
-    const bool in_smem = qbytes <= 200 * 1024;
-    const int threads = qbytes <= 48 * 1024 ? ROW_THREADS : 1024;
-    if (in_smem)
-      MPQ_CUDA(cudaFuncSetAttribute(k_linear_rows, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)qbytes));
-    ProfScope ps_("k_linear_rows", st);
-    k_linear_rows<<<rows_grid(m), in_smem ? threads : ROW_THREADS, in_smem ? qbytes : 0, st>>>(
-        const_cast<float*>(P), p->n, p->r, p->s32, gamma2, gamma1_0, beta, q.damping,
-        q.gamma_lo_rel, q.gamma_hi_rel, q.alpha_min, q.alpha_max, p->r == p->n ? 1 : 0,
-        gamma1_out, coef, kappa, alpha2, beta_hat, clamps, Uprime, As->hi, As->lo, As->ld,
-        round_up(p->r, 64), As->row_unscale, in_smem ? 1 : 0);
+    ProfScope ps_("k_linear_finish", st);
+    k_linear_finish<<<(unsigned)cdiv(m, 128), 128, 0, st>>>(
+        part, ntiles, m, p->n, p->r, e_bound, a_unscale, q_unscale, gamma2, gamma1_0, beta,
+        q.damping, q.gamma_lo_rel, q.gamma_hi_rel, q.alpha_min, q.alpha_max, gamma1_out, coef,
+        kappa, alpha2, beta_hat, clamps);
   }
   count_launch();
-  return check_launch("k_linear_rows");
+  return check_launch("k_linear_finish");
 }
 
 mpq_status launch_extrinsic_l2d(const mpq_plan_s* p, const float* W, int64_t m, const float* R2,
@@ -1285,7 +1211,8 @@ mpq_status launch_vamp_row_scalar(const mpq_plan_s* p, const float* W, int64_t m
                                   int map, const float* G, float* R2, const double* coef,
                                   const double* kappa, const double* gamma1, const float* scale,
                                   const float* offset, const double* gamma1_0, SplitOperand* As,
-                                  double* gamma2, int32_t* clamps, uint16_t* idx, cudaStream_t st) {
+                                  double* gamma2, int32_t* clamps, uint16_t* idx, cudaStream_t st,
+                                  float* R1o) {
   if (m <= 0) return MPQ_OK;
   const int threads = vamp_row_threads(p->n, p->G);
   if (p->d != 1 || threads == 0) return fail(MPQ_ERR_INVALID_ARG, "fused row kernel: d = 1 rows that fit");
@@ -1297,7 +1224,7 @@ mpq_status launch_vamp_row_scalar(const mpq_plan_s* p, const float* W, int64_t m
   using Kern = void (*)(const float*, const float*, float*, int64_t, int, int, int, const double*,
                         const double*, const double*, const float*, const float*, int, int,
                         const double*, double, double, double, double, double, __half*, __half*,
-                        int64_t, int64_t, float*, double*, int32_t*, uint16_t*);
+                        int64_t, int64_t, float*, double*, int32_t*, uint16_t*, float*);
   const Kern kern = p->G ? (map ? k_vamp_row_scalar<1, true> : k_vamp_row_scalar<0, true>)
                          : (map ? k_vamp_row_scalar<1, false> : k_vamp_row_scalar<0, false>);
   MPQ_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
@@ -1307,7 +1234,7 @@ mpq_status launch_vamp_row_scalar(const mpq_plan_s* p, const float* W, int64_t m
         W, G, R2, p->n, p->G, first, p->r == p->n ? 1 : 0, coef, kappa, gamma1, scale, offset, p->K,
         anchored ? 1 : 0, gamma1_0, inv_tau2, q.gamma_lo_rel, q.gamma_hi_rel, q.alpha_min,
         q.alpha_max, As ? As->hi : nullptr, As ? As->lo : nullptr, As ? As->ld : 0,
-        round_up(p->n, 64), As ? As->row_unscale : nullptr, gamma2, clamps, idx);
+        round_up(p->n, 64), As ? As->row_unscale : nullptr, gamma2, clamps, idx, R1o);
   }
   count_launch();
   return check_launch("k_vamp_row_scalar");

@@ -199,6 +199,8 @@ mpq_status alloc_split(SplitOperand& s, int64_t rows, int64_t K, bool per_row) {
 void free_workspace(Workspace& w) {
   dfree(w.R1); dfree(w.X1); dfree(w.R2); dfree(w.P); dfree(w.idx);
   free_split(w.As);
+  free_split(w.Aq);
+  dfree(w.lin_part);
   dfree(w.tile_count);
   dfree(w.Hg);
   dfree(w.Hl);
@@ -213,7 +215,8 @@ constexpr int MAX_SWEEPS = 64;
 
 int64_t ws_bytes_per_row(const mpq_plan_s* p) {
   return 3 * p->n * 4 + round_up(p->n, 32) * 4 + p->r * 4 +
-         4 * round_up(std::max(p->n, p->r), CD_TILE) + p->B * 2 + 3 * 4 +
+         4 * round_up(std::max(p->n, p->r), CD_TILE) + 4 * round_up(p->r, CD_TILE) +
+         8 * cdiv(p->r, CD_TILE) + p->B * 2 + 3 * 4 +
          8 * 8 + 4 + MAX_SWEEPS * 4 + (p->d == 8 ? CD_TILE * 4 : 0) + 8 * (p->ng - 1) + 8;
 }
 
@@ -236,6 +239,8 @@ mpq_status ensure_workspace(mpq_plan_s* p, int64_t rows) {
   chk(dalloc(&w.R1, mn)); chk(dalloc(&w.X1, mn)); chk(dalloc(&w.R2, mn));
   if (st == MPQ_OK)
     chk(alloc_split(w.As, rows, round_up(std::max(p->n, p->r), CD_TILE), true));
+  if (st == MPQ_OK) chk(alloc_split(w.Aq, rows, round_up(p->r, CD_TILE), true));
+  chk(dalloc(&w.lin_part, rows * cdiv(p->r, CD_TILE)));
   chk(dalloc(&w.tile_count, (int64_t)MAX_SWEEPS * 2 * cdiv(p->n, CD_TILE)));  // tiles + panels
   w.ldh = round_up(p->n, 32);
   chk(dalloc(&w.Hg, round_up(std::max<int64_t>(rows, 32), 32) * w.ldh));
@@ -251,6 +256,10 @@ mpq_status ensure_workspace(mpq_plan_s* p, int64_t rows) {
     chk(make_tmap_f16(&w.tm_ar_hi, w.As.hi, round_up(p->r, 64), w.As.rows_pad, w.As.ld, 128));
   if (st == MPQ_OK)
     chk(make_tmap_f16(&w.tm_ar_lo, w.As.lo, round_up(p->r, 64), w.As.rows_pad, w.As.ld, 128));
+  if (st == MPQ_OK)
+    chk(make_tmap_f16(&w.tm_aq_hi, w.Aq.hi, round_up(p->r, 64), w.Aq.rows_pad, w.Aq.ld, 128));
+  if (st == MPQ_OK)
+    chk(make_tmap_f16(&w.tm_aq_lo, w.Aq.lo, round_up(p->r, 64), w.Aq.rows_pad, w.Aq.ld, 128));
   chk(dalloc(&w.P, rows * p->r)); chk(dalloc(&w.idx, rows * p->B));
   chk(dalloc(&w.scale, rows * p->ng)); chk(dalloc(&w.offset, rows * p->ng));
   chk(dalloc(&w.sref, rows));
@@ -313,20 +322,44 @@ mpq_status run_linear(mpq_plan_s* p, const float* W, int64_t m, const float* R1,
   return launch_extrinsic_l2d(p, W, m, R2, p->ws.X1, p->ws.coef, p->ws.kappa, R1_out, xhat2, st);
 }
 
+// 2^e >= 2 sqrt(n): the linear epilogue's bound on |p'| over max|w - r2|
+// (one bit of headroom over sqrt(n))
+int linear_e_bound(int64_t n) {
+  int e = 0;
+  while ((double)(1ll << e) * (double)(1ll << e) < (double)n) ++e;
+  return e + 1;
+}
+
 // the linear module on the split operand w - r2 already in As: p' = V^T
-// (w - r2), its row epilogue and M-step, and G = V (D u) into X1
+// (w - r2) with its epilogue (the diagonal scaling D, the M-step's trace
+// sums, the second GEMM's operand D u), the M-step finisher, and G = V (D u)
+// into X1
 mpq_status run_linear_core(mpq_plan_s* p, int64_t m, double* gamma2, const double* gamma1_0,
                            double* beta, double* gamma1_out, float* Uprime, double* alpha2,
                            double* beta_hat, int32_t* clamps, cudaStream_t st) {
   Workspace& w = p->ws;
   const int64_t n = p->n, r = p->r;
-  // p' = V^T (w - r2)
+  LinEpi le;
+  le.s32 = p->s32;
+  le.beta = beta;
+  le.gamma2 = gamma2;
+  le.full_rank = (r == n) ? 1 : 0;
+  le.e_bound = linear_e_bound(n);
+  le.q_hi = w.Aq.hi;
+  le.q_lo = w.Aq.lo;
+  le.ldq = w.Aq.ld;
+  le.part = w.lin_part;
+  le.ntiles = (int)cdiv(r, CD_TILE);
+  le.Uprime = Uprime;
+  GemmOpts o;
+  o.lin = &le;
   MPQ_TRY(gemm_tc(w.As, w.tm_an_hi, w.tm_an_lo, p->Vt_s, p->tm_vt_hi, p->tm_vt_lo, w.P, r, m, r, n,
-                  p->Vt_s.unscale_host, p->status, st, "gemm_project"));
-  MPQ_TRY(launch_linear_rows(p, m, w.P, gamma2, gamma1_0, beta, gamma1_out, w.coef, w.kappa,
-                             alpha2, beta_hat, clamps, Uprime, &w.As, st));
+                  p->Vt_s.unscale_host, p->status, st, "gemm_project", o));
+  MPQ_TRY(launch_linear_finish(p, m, w.lin_part, le.ntiles, le.e_bound, w.As.row_unscale,
+                               w.Aq.row_unscale, gamma2, gamma1_0, beta, gamma1_out, w.coef,
+                               w.kappa, alpha2, beta_hat, clamps, st));
   // G into X1: the denoiser output is consumed by now
-  return gemm_tc(w.As, w.tm_ar_hi, w.tm_ar_lo, p->V_s, p->tm_v_hi, p->tm_v_lo, w.X1, n, m, n, r,
+  return gemm_tc(w.Aq, w.tm_aq_hi, w.tm_aq_lo, p->V_s, p->tm_v_hi, p->tm_v_lo, w.X1, n, m, n, r,
                  p->V_s.unscale_host, p->status, st, "gemm_expand");
 }
 
@@ -653,7 +686,7 @@ void mpq_params_default(mpq_params* p, int32_t d, int32_t K) {
   p->codebook = nullptr;
   p->beta0 = 1.0;
   p->damping = 0.5;
-  p->tau = INFINITY;
+  p->tau = 0.2;
   p->gamma_lo_rel = 1e-10;
   p->gamma_hi_rel = 1e10;
   p->alpha_min = 1e-10;
@@ -922,8 +955,8 @@ mpq_status mpq_stage_denoise(mpq_plan_t p, const float* R1, const double* gamma1
   if (m < 0 || (m > 0 && (!R1 || !gamma1 || !scale || !offset || !xhat1 || !vsum)))
     return fail(MPQ_ERR_INVALID_ARG, "denoise: missing buffer");
   ROWS_CHECK(m);
-  if (isfinite(p->params.tau) && m > 0 && (!W || !gamma1_0))
-    return fail(MPQ_ERR_INVALID_ARG, "denoise: an anchored plan needs W and gamma1_0");
+  if (isfinite(p->params.tau) && m > 0 && !W)
+    return fail(MPQ_ERR_INVALID_ARG, "denoise: an anchored plan needs W");
   DeviceGuard g(p->device);
   cudaStream_t st = (cudaStream_t)stream;
   if (p->d == 8 && vblock == nullptr) {
@@ -953,6 +986,49 @@ mpq_status mpq_stage_linear(mpq_plan_t p, const float* W, int64_t m, const float
   if (!gamma2) gamma2 = w.gamma2;
   return run_linear(p, W, m, R1, gamma1, xhat1, vsum, gamma1_0, beta, R1_out, gamma1_out, R2,
                     gamma2, Uprime, xhat2, alpha2, beta_hat, clamps, st);
+}
+
+mpq_status mpq_stage_vamp_scalar(mpq_plan_t p, const float* W, int64_t m, const float* scale,
+                                 const float* offset, const float* R1, const double* gamma1,
+                                 const double* gamma1_0, double* beta, float* R2, double* gamma2,
+                                 float* R1_out, double* gamma1_out, uint16_t* idx_map,
+                                 float* R2_next, double* gamma2_next, int32_t* clamps,
+                                 mpq_stream_t stream) {
+  PLAN_CHECK(p);
+  if (m < 0 || (m > 0 && (!W || !scale || !offset || !R1 || !gamma1 || !gamma1_0 || !beta ||
+                          !gamma1_out)))
+    return fail(MPQ_ERR_INVALID_ARG, "vamp_scalar: missing buffer");
+  ROWS_CHECK(m);
+  if (p->d != 1 || vamp_row_threads(p->n, p->G) == 0)
+    return fail(MPQ_ERR_UNSUPPORTED,
+                "vamp_scalar: the fused row kernel runs d = 1 rows that fit its shared memory");
+  if (m == 0) return MPQ_OK;
+  DeviceGuard g(p->device);
+  MPQ_TRY(ensure_workspace(p, m));
+  Workspace& w = p->ws;
+  cudaStream_t st = (cudaStream_t)stream;
+  // the order of one iteration of mpq_solve: fused denoiser + d2l on the
+  // injected cavity, the linear module, then the next fused pass (l2d,
+  // denoiser, d2l); the MAP pass reads the same G and r2 before that pass
+  // overwrites r2
+  MPQ_TRY(launch_vamp_row_scalar(p, W, m, 2, 0, R1, w.R2, w.coef, w.kappa, gamma1, scale, offset,
+                                 gamma1_0, &w.As, w.gamma2, clamps, nullptr, st));
+  if (R2) MPQ_CUDA(cudaMemcpyAsync(R2, w.R2, sizeof(float) * m * p->n, cudaMemcpyDeviceToDevice, st));
+  if (gamma2) MPQ_CUDA(cudaMemcpyAsync(gamma2, w.gamma2, sizeof(double) * m, cudaMemcpyDeviceToDevice, st));
+  MPQ_TRY(run_linear_core(p, m, w.gamma2, gamma1_0, beta, gamma1_out, nullptr, nullptr, nullptr,
+                          clamps, st));
+  if (idx_map)
+    MPQ_TRY(launch_vamp_row_scalar(p, W, m, 0, 1, w.X1, w.R2, w.coef, w.kappa, gamma1_out, scale,
+                                   offset, gamma1_0, nullptr, nullptr, nullptr, idx_map, st));
+  if (R1_out || R2_next || gamma2_next) {
+    MPQ_TRY(launch_vamp_row_scalar(p, W, m, 0, 0, w.X1, w.R2, w.coef, w.kappa, gamma1_out, scale,
+                                   offset, gamma1_0, &w.As, w.gamma2, clamps, nullptr, st, R1_out));
+    if (R2_next)
+      MPQ_CUDA(cudaMemcpyAsync(R2_next, w.R2, sizeof(float) * m * p->n, cudaMemcpyDeviceToDevice, st));
+    if (gamma2_next)
+      MPQ_CUDA(cudaMemcpyAsync(gamma2_next, w.gamma2, sizeof(double) * m, cudaMemcpyDeviceToDevice, st));
+  }
+  return MPQ_OK;
 }
 
 mpq_status mpq_stage_cd(mpq_plan_t p, const float* W, int64_t m, const float* scale,

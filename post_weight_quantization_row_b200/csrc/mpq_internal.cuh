@@ -74,6 +74,12 @@ struct Workspace {
   SplitOperand As;
   CUtensorMap tm_an_hi, tm_an_lo;  // K = n view
   CUtensorMap tm_ar_hi, tm_ar_lo;  // K = r view
+  // A operand of the linear module's second GEMM (D u, K = r), written by
+  // the first GEMM's epilogue (a buffer of its own: other tiles of that GEMM
+  // still read As), and the epilogue's per-(row, column tile) M-step sums
+  SplitOperand Aq;
+  CUtensorMap tm_aq_hi, tm_aq_lo;
+  float2* lin_part = nullptr;      // rows x cdiv(r, 128)
   int* tile_count = nullptr;       // CD: changes per (sweep, tile)
   // CD gradient h = H (w - x), rows x ldh (ldh = n rounded up to 32)
   float* Hg = nullptr;
@@ -184,17 +190,21 @@ mpq_status launch_extrinsic_d2l(const mpq_plan_s* p, const float* W, int64_t m, 
                                 const double* gamma1_0, float* R2, SplitOperand* As,
                                 double* gamma2, int32_t* clamps, cudaStream_t st);
 // reads p' from P, writes the GEMM2 A operand (split, K = r)
-mpq_status launch_linear_rows(const mpq_plan_s* p, int64_t m, const float* P,
-                              const double* gamma2, const double* gamma1_0, double* beta,
-                              double* gamma1_out, double* coef, double* kappa, double* alpha2,
-                              double* beta_hat, int32_t* clamps, float* Uprime, SplitOperand* As,
-                              cudaStream_t st);
+// M-step finisher after the projection GEMM's linear epilogue: per row, the
+// column tiles' sums in a fixed order, then alpha2, beta_hat, the damped
+// beta, gamma1', the l2d coefficients and the second GEMM's row scale.
+mpq_status launch_linear_finish(const mpq_plan_s* p, int64_t m, const float2* part, int ntiles,
+                                int e_bound, const float* a_unscale, float* q_unscale,
+                                const double* gamma2, const double* gamma1_0, double* beta,
+                                double* gamma1_out, double* coef, double* kappa, double* alpha2,
+                                double* beta_hat, int32_t* clamps, cudaStream_t st);
 int vamp_row_threads(int64_t n, int G);  // 0: the fused scalar row kernel does not apply
 mpq_status launch_vamp_row_scalar(const mpq_plan_s* p, const float* W, int64_t m, int first,
                                   int map, const float* G, float* R2, const double* coef,
                                   const double* kappa, const double* gamma1, const float* scale,
                                   const float* offset, const double* gamma1_0, SplitOperand* As,
-                                  double* gamma2, int32_t* clamps, uint16_t* idx, cudaStream_t st);
+                                  double* gamma2, int32_t* clamps, uint16_t* idx, cudaStream_t st,
+                                  float* R1o = nullptr);
 mpq_status launch_extrinsic_l2d(const mpq_plan_s* p, const float* W, int64_t m, const float* R2,
                                 const float* G, const double* coef, const double* kappa,
                                 float* R1_out, float* xhat2, cudaStream_t st);
@@ -244,6 +254,29 @@ mpq_status make_tmap_f16(CUtensorMap* tm, const void* base, int64_t inner, int64
                          int64_t ld_elems, int box_rows);
 mpq_status split_global(const float* src, int64_t rows, int64_t K, SplitOperand* dst,
                         cudaStream_t st);
+// The linear module's epilogue of the projection GEMM (p' = V^T (w - r2),
+// one output element per (row, rank component l)): with F = gamma2 / (beta
+// s_l^2 + gamma2) and u = s_l p', it accumulates per row and column tile
+// sum F and sum F^2 u^2 + s_l^2 / (beta s_l^2 + gamma2) (the M-step's two
+// traces), and writes the second GEMM's operand q = -F p' (full rank) or
+// (1 - F) p' = D u as a fp16 hi/lo pair scaled by 2^-(e_row + e_bound):
+// |p'| <= |w - r2|_2 <= sqrt(n) max|w - r2| (V has orthonormal columns), so
+// with 2^e_bound >= sqrt(n) the scaled pair stays below 2^14 without a row
+// reduction first.
+struct LinEpi {
+  const float* s32 = nullptr;      // r singular values
+  const double* beta = nullptr;    // per row (before the M-step)
+  const double* gamma2 = nullptr;  // per row
+  int full_rank = 0;
+  int e_bound = 0;
+  __half* q_hi = nullptr;
+  __half* q_lo = nullptr;
+  int64_t ldq = 0;
+  float2* part = nullptr;          // rows x ntiles
+  int ntiles = 0;
+  float* Uprime = nullptr;         // optional: (1 - F) p' (rows x r, fp32)
+};
+
 struct GemmOpts {
   int64_t b_k0 = 0;         // K offset into B (a multiple of 64)
   int64_t a_k0 = 0;         // K offset into A (a multiple of 64)
@@ -254,6 +287,8 @@ struct GemmOpts {
   // accumulate through TMA reduce-add into the fp32 matrix this map
   // describes (box 32 x 32, 128B swizzle) instead of a read-modify-write
   const CUtensorMap* c_reduce = nullptr;
+  // the linear module's epilogue instead of storing C (C is not written)
+  const LinEpi* lin = nullptr;
 };
 mpq_status make_tmap_f32_out(CUtensorMap* tm, const float* base, int64_t cols, int64_t rows,
                              int64_t ld_elems);

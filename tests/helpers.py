@@ -37,6 +37,39 @@ def assert_rows_close(name, gpu, ref, tol=VEC_TOL, rows=None):
     return worst
 
 
+ELEM_FLOOR = 4.0 * 2.0 ** -22   # fp32 absolute rounding of a row, with headroom
+
+
+def assert_elems_close(name, gpu, ref, tol=VEC_TOL, rows=None):
+    """Element-wise companion of assert_rows_close: every element within
+    tol * |ref| + 4 * 2^-22 * |ref row|_2.  The floor is what fp32 (and the
+    22-significand-bit tensor-core contractions) can promise an element that
+    is small next to its row: its absolute error carries the rounding of the
+    row's larger terms, ~2^-22 times the row norm (e.g. a posterior mean
+    formed as scale * level + offset near zero, or a GEMM output summing n
+    terms).  It is about 1/100 of what the per-row l2 bound lets a single
+    element be off, so one bad element cannot hide behind larger ones."""
+    gpu = np.asarray(gpu, np.float64).reshape(ref.shape[0], -1)
+    ref = np.asarray(ref, np.float64).reshape(ref.shape[0], -1)
+    if rows is not None:
+        gpu, ref = gpu[rows], ref[rows]
+    norm = np.linalg.norm(ref, axis=1, keepdims=True)
+    bound = tol * np.abs(ref) + ELEM_FLOOR * norm
+    excess = np.abs(gpu - ref) / np.maximum(bound, 1e-300)
+    worst = float(excess.max()) if excess.size else 0.0
+    if worst > 1.0:
+        i, j = np.unravel_index(np.argmax(excess), excess.shape)
+        raise AssertionError(f"{name}: element ({i}, {j}) {gpu[i, j]:.9g} vs {ref[i, j]:.9g} "
+                             f"(row l2 {norm[i, 0]:.3g}) exceeds its bound by {worst:.2f}x")
+    return worst
+
+
+def assert_vec_close(name, gpu, ref, tol=VEC_TOL, rows=None):
+    """Per-row relative l2 and the element-wise bound."""
+    assert_rows_close(name, gpu, ref, tol, rows)
+    return assert_elems_close(name, gpu, ref, tol, rows)
+
+
 def assert_scalars_close(name, gpu, ref, tol=SCAL_TOL, rows=None):
     gpu = np.asarray(gpu, np.float64)
     ref = np.asarray(ref, np.float64)

@@ -37,7 +37,7 @@ def test_params_default(mpq):
     p = mpq.Params()
     mpq.lib.mpq_params_default(C.byref(p), 1, 8)
     assert p.d == 1 and p.K == 8 and p.beta0 == 1.0 and p.damping == 0.5
-    assert math.isinf(p.tau) and p.gamma_lo_rel == 1e-10 and p.gamma_hi_rel == 1e10
+    assert p.tau == 0.2 and p.gamma_lo_rel == 1e-10 and p.gamma_hi_rel == 1e10
     assert p.alpha_min == 1e-10 and p.alpha_max == 0.99
     assert p.vec_engine == 0 and p.cd_panel == 0 and p.solve_graphs == 1 and p.group_size == 0
     assert p.cd_skip_precision == 0.0

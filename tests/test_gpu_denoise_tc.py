@@ -17,7 +17,7 @@ import torch
 
 import mpq_inputs as mi
 from oracle import mpq_oracle as orc
-from tests.helpers import (assert_rows_close, assert_scalars_close, codebook_for, cu, host,
+from tests.helpers import (assert_vec_close, assert_rows_close, assert_scalars_close, codebook_for, cu, host,
                            idx_np, injected_state, spectrum_cuda)
 
 pytestmark = pytest.mark.gpu
@@ -38,10 +38,10 @@ def e8_case(seed, m_out, n, K, m=None):
                             codebook=cb)
 
 
-def plan_for(mpq, p, engine, **kw):
+def plan_for(mpq, p, engine, tau=math.inf, **kw):
     _, _, s_cu, V_cu = spectrum_cuda(p.X)
     return mpq.Plan.from_spectrum(s_cu, V_cu, 8, p.levels, codebook=p.codebook,
-                                  vec_engine=ENGINES[engine], **kw)
+                                  vec_engine=ENGINES[engine], tau=tau, **kw)
 
 
 def kernels_of(mpq, fn):
@@ -51,18 +51,19 @@ def kernels_of(mpq, fn):
     return out, mpq.profile_stop()
 
 
-def check_denoise(mpq, p, plan, R1, g1, engine, ga=None, g0=None, tau_W=None):
+def check_denoise(mpq, p, plan, R1, g1, engine, tau=math.inf):
+    """Stage parity of the vector denoiser; the plan's anchor must be tau."""
     sc = orc.rms_scale(p.W)[0].astype(np.float32)
     off = np.zeros_like(sc)
+    anchored = math.isfinite(tau)
     ref = orc.denoise(R1, g1, codebook_for(p), sc.astype(np.float64), off.astype(np.float64),
-                      tau_W, ga)
+                      p.W, tau)
     out, kern = kernels_of(mpq, lambda: plan.stage_denoise(
-        cu(R1), cu(g1, torch.float64), cu(sc), cu(off),
-        cu(tau_W) if ga is not None else None, cu(g0, torch.float64) if ga is not None else None))
+        cu(R1), cu(g1, torch.float64), cu(sc), cu(off), cu(p.W) if anchored else None))
     want = "k_denoise_vec_tc" if engine == "tensor" else "k_denoise_vec"
     assert want in kern, kern
-    assert_rows_close("xhat1", host(out["xhat"]), ref.xhat)
-    assert_rows_close("vblock", host(out["vblock"]), ref.vblock)
+    assert_vec_close("xhat1", host(out["xhat"]), ref.xhat)
+    assert_vec_close("vblock", host(out["vblock"]), ref.vblock)
     assert_scalars_close("vsum", host(out["vsum"]), ref.vsum)
     ok = ref.gap > LOGIT_TIE
     assert ok.mean() > 0.9
@@ -83,14 +84,14 @@ def test_denoise_e8_ragged_tiles(mpq, engine, g_lo, g_hi):
 
 
 @pytest.mark.parametrize("engine", ["tensor", "simt"])
-def test_denoise_e8_anchored_prior(mpq, engine):
+@pytest.mark.parametrize("tau", [0.2, 0.7])
+def test_denoise_e8_anchored_prior(mpq, engine, tau):
     p = e8_case(203, 13, 96, 1024)
-    tau = 0.3
     plan = plan_for(mpq, p, engine, tau=tau)
     sc = orc.rms_scale(p.W)[0].astype(np.float32)
     s, _ = orc.spectrum(p.X)
-    R1, g1, _, _, _, g0 = injected_state(9, p.W, sc, s)
-    check_denoise(mpq, p, plan, R1, g1, engine, ga=g0 / tau ** 2, g0=g0, tau_W=p.W)
+    R1, g1, _, _, _, _ = injected_state(9, p.W, sc, s)
+    check_denoise(mpq, p, plan, R1, g1, engine, tau=tau)
 
 
 def test_denoise_e8_persistent_tiles(mpq):
@@ -150,7 +151,7 @@ def test_auto_engine_picks_tensor_cores_for_lattice_codebooks(mpq):
     p = e8_case(207, 5, 64, 256)
     plan = plan_for(mpq, p, "tensor")
     _, _, s_cu, V_cu = spectrum_cuda(p.X)
-    auto = mpq.Plan.from_spectrum(s_cu, V_cu, 8, p.levels, codebook=p.codebook)
+    auto = mpq.Plan.from_spectrum(s_cu, V_cu, 8, p.levels, codebook=p.codebook, tau=math.inf)
     sc = orc.rms_scale(p.W)[0].astype(np.float32)
     args = (cu(p.W), cu(np.full(p.m_out, 5.0) / sc.astype(np.float64) ** 2, torch.float64),
             cu(sc), cu(np.zeros_like(sc)))
@@ -173,7 +174,7 @@ def test_codebooks_that_do_not_qualify(mpq, codebook):
         mpq.Plan.from_spectrum(s_cu, V_cu, 8, p.levels, codebook=cb, vec_engine=2)
     assert e.value.status == 7   # MPQ_ERR_UNSUPPORTED
     # the default engine falls back to the SIMT kernel and matches the oracle
-    plan = mpq.Plan.from_spectrum(s_cu, V_cu, 8, p.levels, codebook=cb)
+    plan = mpq.Plan.from_spectrum(s_cu, V_cu, 8, p.levels, codebook=cb, tau=math.inf)
     sc = orc.rms_scale(p.W)[0].astype(np.float32)
     s, _ = orc.spectrum(p.X)
     R1, g1, _, _, _, _ = injected_state(12, p.W, sc, s)
@@ -181,12 +182,13 @@ def test_codebooks_that_do_not_qualify(mpq, codebook):
 
 
 @pytest.mark.parametrize("engine", ["tensor", "simt"])
-def test_vector_solve_both_engines(mpq, engine):
+@pytest.mark.parametrize("tau", [math.inf, orc.TAU])
+def test_vector_solve_both_engines(mpq, engine, tau):
     p = e8_case(209, 23, 160, 2048, m=320)
-    plan = plan_for(mpq, p, engine)
+    plan = plan_for(mpq, p, engine, tau=tau)
     out = plan.solve(cu(p.W), p.T_vamp, p.cd_sweeps, stats=True)
     s, V = orc.spectrum(p.X)
-    ref = orc.solve(p.W, codebook_for(p), s, V, p.T_vamp, p.cd_sweeps)
+    ref = orc.solve(p.W, codebook_for(p), s, V, p.T_vamp, p.cd_sweeps, tau=tau)
     e_gpu = host(out["energy"]).astype(np.float64)
     rel = np.abs(e_gpu - ref.energy) / ref.energy
     clean = np.all(ref.map_gap > 1e-4, axis=1) & (ref.cd.first_tie < 0)
@@ -194,3 +196,21 @@ def test_vector_solve_both_engines(mpq, engine):
     assert np.array_equal(idx_np(out["idx"])[clean], ref.idx[clean])
     assert rel[clean].max() <= 1e-3
     assert rel.max() <= 5e-2 and np.mean((e_gpu - ref.energy) / ref.energy) <= 1e-2
+
+
+@pytest.mark.parametrize("g_lo,g_hi,tau", [(0.3, 3.0, math.inf), (3.0, 30.0, math.inf),
+                                           (30.0, 300.0, math.inf), (300.0, 3000.0, math.inf),
+                                           (3.0, 30.0, orc.TAU)])
+def test_denoise_full_e8_codebook_on_e8t8_rows(mpq, g_lo, g_hi, tau):
+    # the whole 65536-codeword offset-E8 codebook (every shell up to norm^2
+    # 11.5, all 512 codebook stages of the kernel's ring) on two rows of the
+    # 2-bit workload (1024 blocks, 8 tiles of 128), precisions gamma1 s^2
+    # from 0.3 to 3000; the denoiser reads no spectrum, so the plan takes a
+    # small synthetic one
+    p = mi.make_problem("e8t8", rows=[11, 12], with_x=False)
+    s, V = mi.orthonormal_spectrum(31, p.n, 64)
+    plan = mpq.Plan.from_spectrum(cu(s, torch.float64), cu(V, torch.float64), 8, p.levels,
+                                  codebook=p.codebook, tau=tau)
+    sc = orc.rms_scale(p.W)[0].astype(np.float32)
+    R1, g1, _, _, _, _ = injected_state(13, p.W, sc, s, g_lo, g_hi)
+    check_denoise(mpq, p, plan, R1, g1, "tensor", tau=tau)

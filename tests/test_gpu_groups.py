@@ -4,13 +4,15 @@ setting) against the oracle on identical inputs: init exactly, the denoiser
 at the stage bar in every precision regime, CD indices exactly outside ties
 (with several panels, so that Delta carries the group scales through the
 panel GEMM), and the whole solve."""
+import math
+
 import numpy as np
 import pytest
 import torch
 
 import mpq_inputs as mi
 from oracle import mpq_oracle as orc
-from tests.helpers import (ENERGY_TOL, assert_rows_close, assert_scalars_close, cu, host, idx_np,
+from tests.helpers import (assert_vec_close, ENERGY_TOL, assert_rows_close, assert_scalars_close, cu, host, idx_np,
                            injected_state, spectrum_cuda)
 
 pytestmark = pytest.mark.gpu
@@ -55,20 +57,24 @@ def test_init_grouped_grid(mpq):
     assert_scalars_close("gamma1_0", host(out["gamma1_0"]), st.gamma1, 1e-5)
 
 
-@pytest.mark.parametrize("g_lo,g_hi", [(1.0, 40.0), (0.05, 0.5), (100.0, 1e4)])
-def test_denoise_grouped(mpq, g_lo, g_hi):
+@pytest.mark.parametrize("g_lo,g_hi,tau", [(1.0, 40.0, math.inf), (0.05, 0.5, math.inf),
+                                           (100.0, 1e4, math.inf), (1.0, 40.0, 0.2),
+                                           (0.05, 0.5, 0.2)])
+def test_denoise_grouped(mpq, g_lo, g_hi, tau):
+    # with the anchor, each group's anchor is tau steps of its own grid
     p = case(802)
-    plan = plan_for(mpq, p)
+    plan = plan_for(mpq, p, tau=tau)
     sc, off = grid_f32(p)
     s, _ = orc.spectrum(p.X)
     # the precision is per row; the groups' scales make gamma1 s^2 (and with
     # it the precision regime) differ from group to group
     R1, g1, _, _, _, _ = injected_state(11, p.W, sc.mean(axis=1), s, g_lo, g_hi)
     ref = orc.denoise(R1, g1, orc.scalar_levels(p.levels), sc.astype(np.float64),
-                      off.astype(np.float64))
-    out = plan.stage_denoise(cu(R1), cu(g1, torch.float64), cu(sc), cu(off))
-    assert_rows_close("xhat1", host(out["xhat"]), ref.xhat)
-    assert_rows_close("vblock", host(out["vblock"]), ref.vblock)
+                      off.astype(np.float64), p.W, tau)
+    out = plan.stage_denoise(cu(R1), cu(g1, torch.float64), cu(sc), cu(off),
+                             cu(p.W) if math.isfinite(tau) else None)
+    assert_vec_close("xhat1", host(out["xhat"]), ref.xhat)
+    assert_vec_close("vblock", host(out["vblock"]), ref.vblock)
     assert_scalars_close("vsum", host(out["vsum"]), ref.vsum)
     ok = ref.gap > LOGIT_TIE
     assert np.array_equal(idx_np(out["idx"])[ok], ref.idx[ok])

@@ -142,16 +142,50 @@ def test_denoiser_scalar_vs_50_digit_brute_force():
 
 
 def test_denoiser_anchor_vs_brute_force():
+    # anchor of tau codebook units: precision 1/(tau scale)^2 in weight units
     g = np.random.default_rng(6)
     cb = orc.scalar_levels(4)
     R1 = g.normal(0, 1, size=(1, 5))
     W = g.normal(0, 1, size=(1, 5))
-    out = orc.denoise(R1, np.array([2.0]), cb, np.array([0.8]), np.array([-1.2]), W, np.array([5.0]))
+    tau = 0.2
+    out = orc.denoise(R1, np.array([2.0]), cb, np.array([0.8]), np.array([-1.2]), W, tau)
     cand = orc.row_candidates(cb, 0.8, -1.2)
     for j in range(5):
-        mean, var = _mp_posterior([R1[0, j]], 2.0, cand, [W[0, j]], 5.0)
+        mean, var = _mp_posterior([R1[0, j]], 2.0, cand, [W[0, j]], 1.0 / (tau * 0.8) ** 2)
         assert abs(out.xhat[0, j] - mean[0]) < 1e-12
         assert abs(out.vblock[0, j] - var) < 1e-12
+
+
+def test_denoiser_anchor_per_group_scale_vs_brute_force():
+    # group-wise grids: each block's anchor is tau steps of its own group's grid
+    g = np.random.default_rng(16)
+    cb = orc.scalar_levels(8)
+    R1 = g.normal(0, 1, size=(1, 8))
+    W = g.normal(0, 1, size=(1, 8))
+    sc = np.array([[0.3, 0.5]])
+    off = np.array([[-1.0, -1.5]])
+    tau = 0.7
+    out = orc.denoise(R1, np.array([3.0]), cb, sc, off, W, tau)
+    for j in range(8):
+        k = j // 4
+        cand = orc.row_candidates(cb, sc[0, k], off[0, k])
+        mean, var = _mp_posterior([R1[0, j]], 3.0, cand, [W[0, j]], 1.0 / (tau * sc[0, k]) ** 2)
+        assert abs(out.xhat[0, j] - mean[0]) < 1e-12
+        assert abs(out.vblock[0, j] - var) < 1e-12
+
+
+@pytest.mark.parametrize("tau", [1.5, 3.0])
+def test_anchor_width_is_tau_grid_steps(tau):
+    # an uninformative cavity (gamma1 -> 0) leaves the anchor alone: on a fine
+    # grid around w it is a discrete Gaussian whose variance is (tau s)^2 to
+    # within exp(-2 pi^2 tau^2) (Poisson summation), and whose mean is w
+    cb = orc.scalar_levels(256)
+    s = 0.01
+    W = np.array([[0.0137, -0.0421]])
+    out = orc.denoise(np.zeros((1, 2)), np.array([1e-300]), cb, np.array([s]), np.array([-1.28]),
+                      W, tau)
+    assert np.allclose(out.vblock[0] / (tau * s) ** 2, 1.0, rtol=1e-7, atol=0)
+    assert np.allclose(out.xhat[0], W[0], rtol=0, atol=1e-9 * s)
 
 
 def test_denoiser_vector_small_codebook_vs_brute_force():

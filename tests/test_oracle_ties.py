@@ -69,8 +69,9 @@ def test_denoise_gap_is_the_top_two_logit_difference(d, anchor):
         sc, off = orc.rms_scale(W)
     R1 = W + 0.3 * sc[:, None] * g.standard_normal((m, n))
     gamma1 = g.uniform(2.0, 30.0, m) / (sc * sc)
-    ga = gamma1 * 0.3 if anchor else None
-    dn = orc.denoise(R1, gamma1, cb, sc, off, W, ga)
+    tau = 0.7 if anchor else math.inf
+    ga = 1.0 / (tau * sc) ** 2 if anchor else None
+    dn = orc.denoise(R1, gamma1, cb, sc, off, W, tau)
     want = _brute_gaps(R1, gamma1, cb, sc, off, W, ga)
     scale = 1.0 + np.abs(want).max()
     assert np.allclose(dn.gap, want, rtol=0, atol=1e-10 * scale)
@@ -107,7 +108,7 @@ def _brute_cd(w, idx0, cb, scale, offset, X, sweeps, tie_rel):
     idx = np.array(idx0, dtype=np.int64)
     x = cand[np.arange(B), idx].reshape(-1).copy()
     first_tie, min_gap, step = -1, math.inf, 0
-    changes = []
+    changes, gaps = [], []
     for _ in range(sweeps):
         nchg = 0
         for b in range(B):
@@ -121,6 +122,7 @@ def _brute_cd(w, idx0, cb, scale, offset, X, sweeps, tie_rel):
             k = int(np.argmin(Ec))
             two = np.sort(Ec)[:2]
             gap = (two[1] - two[0]) / abs(E)
+            gaps.append(gap)
             min_gap = min(min_gap, gap)
             if gap < tie_rel and first_tie < 0:
                 first_tie = step
@@ -132,7 +134,7 @@ def _brute_cd(w, idx0, cb, scale, offset, X, sweeps, tie_rel):
         changes.append(nchg)
         if nchg == 0:
             break
-    return idx, first_tie, min_gap, changes
+    return idx, first_tie, min_gap, changes, np.asarray(gaps)
 
 
 @pytest.mark.parametrize("d", [1, 8])
@@ -155,13 +157,16 @@ def test_cd_first_tie_and_min_gap_match_whole_objective_brute_force(d):
     for tie_rel in (1e-5, 1e-3, 1e-2, 1e-1):
         out = orc.cd(W, idx0, cb, sc, off, H, 3, tie_rel=tie_rel)
         for i in range(m):
-            idx, ft, mg, chg = _brute_cd(np.asarray(W[i], np.float64), idx0[i], cb, sc[i], off[i],
-                                         X64, 3, tie_rel)
+            idx, ft, mg, chg, gaps = _brute_cd(np.asarray(W[i], np.float64), idx0[i], cb, sc[i],
+                                               off[i], X64, 3, tie_rel)
             assert np.array_equal(out.idx[i], idx), (tie_rel, i)
             assert list(out.changes[i, :len(chg)]) == chg
             assert out.first_tie[i] == ft, (tie_rel, i, out.first_tie[i], ft)
             # the gap is relative to the energy before the step, to ~1e-9
             assert math.isclose(out.min_gap_rel[i], mg, rel_tol=1e-7, abs_tol=1e-12), (i, mg)
+            # every step's gap, and no gap recorded for steps not taken
+            assert np.allclose(out.step_gap[i, :gaps.size], gaps, rtol=1e-7, atol=1e-12)
+            assert np.all(np.isinf(out.step_gap[i, gaps.size:]))
             seen_tie |= ft >= 0
     assert seen_tie  # the larger thresholds make the first-tie branch live
 
@@ -185,7 +190,7 @@ def test_cd_planted_exact_tie_is_the_first_tie():
     assert out.min_gap_rel[0] < 1e-12
     assert np.array_equal(out.idx, idx0) and out.changes[0, 0] == 0
     # an exact tie with the current codeword is not a move
-    _, ft, mg, chg = _brute_cd(w[0], idx0[0], cb, 1.0, 0.0, X, 3, 1e-5)
+    _, ft, mg, chg, _ = _brute_cd(w[0], idx0[0], cb, 1.0, 0.0, X, 3, 1e-5)
     assert ft == 5 and chg == [0]
 
 
