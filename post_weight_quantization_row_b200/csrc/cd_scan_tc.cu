@@ -12,6 +12,11 @@
 // (M = 128 rows, N = 128 codewords, K = 16) per tile into TMEM; the epilogue
 // forms score = qtab + 2^-k D in fp32 and keeps the first minimum.
 //
+// The same scan serves the greedy baseline (LDLQ with E8 rounding): the
+// codeword nearest a block's working values v_b is the argmin of
+// 1/2 |c|^2 - c.t with t = v_b / scale, i.e. score(c) with qtab replaced by
+// 1/2 |c|^2 and g' by t.
+//
 // Grid: (slices of the codebook) x (tiles of 128 rows); every CTA writes the
 // minimum of its slice per row, and the apply step combines the slices.
 // Warps 0-15 read TMEM (warp w: lanes 32 (w % 4) .. +31, columns 32 (w / 4)
@@ -56,7 +61,9 @@ struct ScanArgs {
   int64_t b, t0;          // block, first column of its CD tile
   const uint8_t* cb_tc;   // NT x 8 KiB operand images (the first 4 KiB: scores)
   const float* cb;        // K x 8
-  const float* qtab;      // B x K
+  const float* qtab_row;  // K: the score table of this scan (qtab_b, or 1/2 |c|^2)
+  const float* Wk;        // greedy mode: working rows (t = Wk[row, block] / scale), else NULL
+  int64_t ldw;
   const float* H;         // n x n fp32
   const float* scale;
   const uint16_t* idx;
@@ -161,7 +168,7 @@ __global__ void __launch_bounds__(SC_THREADS, 1) k_cd_vec_scan(ScanArgs a) {
         uint8_t* st = smem + SC_B + s * SC_STAGE;
         mbar_expect_tx(&b_full[s], SC_STAGE);
         bulk_load_1d(st, a.cb_tc + (size_t)(j0 + t) * SC_IMG_STRIDE, SC_OPER, &b_full[s]);
-        bulk_load_1d(st + SC_OPER, a.qtab + a.b * a.K + (int64_t)(j0 + t) * SC_N, SC_QT, &b_full[s]);
+        bulk_load_1d(st + SC_OPER, a.qtab_row + (int64_t)(j0 + t) * SC_N, SC_QT, &b_full[s]);
       }
       for (int q = (t > SC_STAGES ? t - SC_STAGES : 0); q < t; ++q)  // copies land before exit
         for (uint32_t i = 0; i < (1u << 25) && !mbar_try_wait(&b_full[q % SC_STAGES], (q / SC_STAGES) & 1); ++i)
@@ -198,7 +205,11 @@ __global__ void __launch_bounds__(SC_THREADS, 1) k_cd_vec_scan(ScanArgs a) {
     if (wg == 0) {
       // g' = (h_b + G_b x_b) / scale; A = -2^k g' as an fp16 pair
       float g[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-      if (active) {
+      if (active && a.Wk) {  // greedy: the block's working values in codebook units
+        const float inv = 1.0f / a.scale[row];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) g[i] = a.Wk[row * a.ldw + 8 * a.b + i] * inv;
+      } else if (active) {
         const float sc = a.scale[row];
         const int kcur = a.idx[row * (a.n / 8) + a.b];
         const float* hb = (8 * a.b == a.t0) ? a.h + row * a.ldh + 8 * a.b
@@ -346,7 +357,7 @@ mpq_status launch_cd_vec_scan(const mpq_plan_s* p, int64_t m, int64_t b, int64_t
   a.t0 = t0;
   a.cb_tc = reinterpret_cast<const uint8_t*>(p->cb_tc);
   a.cb = p->cb;
-  a.qtab = p->qtab;
+  a.qtab_row = p->qtab + b * p->K;
   a.H = p->H32;
   a.scale = scale;
   a.idx = idx;
@@ -364,6 +375,43 @@ mpq_status launch_cd_vec_scan(const mpq_plan_s* p, int64_t m, int64_t b, int64_t
   }
   count_launch();
   return check_launch("k_cd_vec_scan");
+}
+
+mpq_status launch_ldlq_vec_scan(const mpq_plan_s* p, int64_t m, int64_t b, const float* scale,
+                                const float* Wk, int64_t ldw, float* part_val, int* part_idx,
+                                int nslices, cudaStream_t st) {
+  static bool attr_set[64] = {};
+  int dev = 0;
+  MPQ_CUDA(cudaGetDevice(&dev));
+  if (dev < 64 && !attr_set[dev]) {
+    MPQ_CUDA(cudaFuncSetAttribute(k_cd_vec_scan, cudaFuncAttributeMaxDynamicSharedMemorySize, SC_SMEM));
+    attr_set[dev] = true;
+  }
+  if (!p->cb_hnorm) return fail(MPQ_ERR_INVALID_ARG, "the plan has no half-norm table");
+  ScanArgs a{};
+  a.m = m;
+  a.n = p->n;
+  a.K = p->K;
+  a.NT = p->K / SC_N;
+  a.b = b;
+  a.t0 = 8 * b;
+  a.cb_tc = reinterpret_cast<const uint8_t*>(p->cb_tc);
+  a.cb = p->cb;
+  a.qtab_row = p->cb_hnorm;
+  a.Wk = Wk;
+  a.ldw = ldw;
+  a.scale = scale;
+  a.part_val = part_val;
+  a.part_idx = part_idx;
+  a.nslices = nslices;
+  a.status = p->status;
+  dim3 grid((unsigned)nslices, (unsigned)cdiv(m, SC_M));
+  {
+    ProfScope ps_("k_ldlq8_scan", st);
+    k_cd_vec_scan<<<grid, SC_THREADS, SC_SMEM, st>>>(a);
+  }
+  count_launch();
+  return check_launch("k_ldlq8_scan");
 }
 
 }  // namespace mpq

@@ -31,24 +31,61 @@ constexpr int A_TILE = BM * BK * 2;                 // 16 KiB
 constexpr int TC_THREADS = 192;
 
 // ------------------------------------------------------- persistent GEMM --
-// The same product with 128 x 128 tiles walked by one CTA per SM: a 3-stage
-// TMA ring runs across tiles, and two TMEM accumulators let the epilogue of
-// one tile overlap the MMAs of the next.  Tiles go in groups of 8 M-tiles
-// (M fastest) so that the A and B panels in flight stay in L2.
-constexpr int PBN = 128, PSTAGES = 3, PGROUP = 8;
-constexpr int P_B_TILE = PBN * BK * 2;                        // 16 KiB
-constexpr int P_STAGE = 2 * A_TILE + 2 * P_B_TILE;            // 64 KiB
+// One CTA per SM walks the output tiles: a 2-stage TMA ring runs across
+// tiles, and two TMEM accumulators let the epilogue of one tile overlap the
+// MMAs of the next.  Tiles are 128 x 256 (the three MMAs of a k-step then
+// read 96 B of shared memory per cycle of tensor work, against 128 B, the
+// whole shared-memory bandwidth, at 128 x 128) for as many full waves of
+// the grid as the product holds; the 128 x 256 tiles left over for a last,
+// partial wave run as two 128 x 128 tiles each, and an odd 128-column strip
+// at the right edge as 128 x 128 tiles too.  Wide tiles go in groups of 8
+// M-tiles (M fastest) so that the A and B panels in flight stay in L2.
+constexpr int PBN = 128, WBN = 256, PSTAGES = 2, PGROUP = 8;
+constexpr int P_B_TILE = PBN * BK * 2;                        // 16 KiB per 128 rows of B
+constexpr int P_STAGE = 2 * A_TILE + 2 * 2 * P_B_TILE;        // 96 KiB
 constexpr int P_STG_WARP = 8192;                              // epilogue staging per warp
 constexpr int P_SMEM = PSTAGES * P_STAGE + 4 * P_STG_WARP + 1024 + 256;
-constexpr uint32_t P_TMEM_COLS = 2 * PBN;
-constexpr uint32_t P_IDESC = idesc_f16(BM, PBN);
+constexpr uint32_t P_TMEM_COLS = 2 * WBN;
+constexpr uint32_t P_IDESC_W = idesc_f16(BM, WBN), P_IDESC_N = idesc_f16(BM, PBN);
 
-__device__ __forceinline__ void p_tile(int t, int mtiles, int ntiles, int& m0, int& n0) {
-  const int per_group = PGROUP * ntiles;
+// The walk over tiles for a grid of G CTAs: T2 wide tiles in all, the first
+// tmain (whole waves) as such, the rest split in halves, then the strip.
+struct TileWalk {
+  int mtiles, np2, tmain, nsplit, total;
+};
+__device__ __forceinline__ TileWalk tile_walk(int M, int N, int G) {
+  TileWalk tw;
+  tw.mtiles = (M + BM - 1) / BM;
+  const int n128 = (N + PBN - 1) / PBN;
+  tw.np2 = n128 / 2;
+  const int t2 = tw.mtiles * tw.np2;
+  tw.tmain = t2 / G * G;
+  tw.nsplit = 2 * (t2 - tw.tmain);
+  tw.total = tw.tmain + tw.nsplit + tw.mtiles * (n128 % 2);
+  return tw;
+}
+__device__ __forceinline__ void wide_tile(int t, int mtiles, int np2, int& m0, int& n0) {
+  const int per_group = PGROUP * np2;
   const int g = t / per_group, w = t % per_group;
   const int gm = min(PGROUP, mtiles - g * PGROUP);  // M-tiles in this group
   m0 = (g * PGROUP + w % gm) * BM;
-  n0 = (w / gm) * PBN;
+  n0 = (w / gm) * WBN;
+}
+// tile t of the walk: its origin and width (256 or 128 columns)
+__device__ __forceinline__ void p_tile(const TileWalk& tw, int t, int& m0, int& n0, int& wn) {
+  if (t < tw.tmain) {
+    wide_tile(t, tw.mtiles, tw.np2, m0, n0);
+    wn = WBN;
+  } else if (t < tw.tmain + tw.nsplit) {
+    const int s = t - tw.tmain;
+    wide_tile(tw.tmain + s / 2, tw.mtiles, tw.np2, m0, n0);
+    n0 += (s & 1) * PBN;
+    wn = PBN;
+  } else {
+    m0 = (t - tw.tmain - tw.nsplit) * BM;
+    n0 = tw.np2 * WBN;
+    wn = PBN;
+  }
 }
 
 // LIN = 1: the linear module's epilogue (LinEpi) instead of storing C.
@@ -72,8 +109,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   uint32_t* tmem_slot = (uint32_t*)(tm_empty + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int mtiles = (M + BM - 1) / BM, ntiles = (N + PBN - 1) / PBN;
-  const int tiles = mtiles * ntiles;
+  const TileWalk walk = tile_walk(M, N, gridDim.x);
+  const int tiles = walk.total;
   const int KT = (K + BK - 1) / BK;
 
   if (threadIdx.x == 0) {
@@ -104,8 +141,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     uint32_t it = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-      int m0, n0;
-      p_tile(t, mtiles, ntiles, m0, n0);
+      int m0, n0, wn;
+      p_tile(walk, t, m0, n0, wn);
+      const int nb = wn / PBN;  // 128-row boxes of B
       for (int kt = 0; kt < KT; ++kt, ++it) {
         const int s = it % PSTAGES;
         if (it >= PSTAGES && !mbar_wait(&empty[s], (it / PSTAGES - 1) & 1)) {
@@ -114,11 +152,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           break;
         }
         uint8_t* base = smem + s * P_STAGE;
-        mbar_expect_tx(&full[s], a_exact ? P_STAGE - A_TILE : P_STAGE);
+        mbar_expect_tx(&full[s], (a_exact ? A_TILE : 2 * A_TILE) + 2 * nb * P_B_TILE);
         tma_load_2d(&ta_hi, &full[s], base, a_k0 + kt * BK, m0);
         if (!a_exact) tma_load_2d(&ta_lo, &full[s], base + A_TILE, a_k0 + kt * BK, m0);
-        tma_load_2d(&tb_hi, &full[s], base + 2 * A_TILE, b_k0 + kt * BK, n_off + n0);
-        tma_load_2d(&tb_lo, &full[s], base + 2 * A_TILE + P_B_TILE, b_k0 + kt * BK, n_off + n0);
+        for (int b = 0; b < nb; ++b) {
+          tma_load_2d(&tb_hi, &full[s], base + 2 * A_TILE + b * P_B_TILE, b_k0 + kt * BK,
+                      n_off + n0 + b * PBN);
+          tma_load_2d(&tb_lo, &full[s], base + 2 * A_TILE + (2 + b) * P_B_TILE, b_k0 + kt * BK,
+                      n_off + n0 + b * PBN);
+        }
       }
     }
     for (uint32_t q = (it > PSTAGES ? it - PSTAGES : 0); q < it; ++q)  // copies land before exit
@@ -130,13 +172,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     bool ok = true;
     for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++tl) {
       const int buf = tl & 1;
+      int m0, n0, wn;
+      p_tile(walk, t, m0, n0, wn);
+      const uint32_t idesc = wn == WBN ? P_IDESC_W : P_IDESC_N;
       if (tl >= 2 && !mbar_wait(&tm_empty[buf], (tl / 2 - 1) & 1)) {
         atomicOr(status, STATUS_TIMEOUT);
         ok = false;
         break;
       }
       tc_fence_after();
-      const uint32_t d = tmem + (uint32_t)buf * PBN;
+      const uint32_t d = tmem + (uint32_t)buf * WBN;
       for (int kt = 0; kt < KT; ++kt, ++it) {
         const int s = it % PSTAGES;
         if (!mbar_wait(&full[s], (it / PSTAGES) & 1)) {
@@ -147,16 +192,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         tc_fence_after();
         const uint32_t a_hi = smem_u32(smem + s * P_STAGE);
         const uint32_t a_lo = a_hi + A_TILE;
-        const uint32_t b_hi = a_hi + 2 * A_TILE;
-        const uint32_t b_lo = b_hi + P_B_TILE;
+        const uint32_t b_hi = a_hi + 2 * A_TILE;     // wn rows: one or two 128-row boxes
+        const uint32_t b_lo = b_hi + 2 * P_B_TILE;
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk) {
           const uint32_t off = kk * 32;
           const uint64_t dah = sw128_desc(a_hi + off), dal = sw128_desc(a_lo + off);
           const uint64_t dbh = sw128_desc(b_hi + off), dbl = sw128_desc(b_lo + off);
-          umma_f16(d, dah, dbh, P_IDESC, (kt | kk) != 0 ? 1u : 0u);
-          umma_f16(d, dah, dbl, P_IDESC, 1u);
-          if (!a_exact) umma_f16(d, dal, dbh, P_IDESC, 1u);
+          umma_f16(d, dah, dbh, idesc, (kt | kk) != 0 ? 1u : 0u);
+          umma_f16(d, dah, dbl, idesc, 1u);
+          if (!a_exact) umma_f16(d, dal, dbh, idesc, 1u);
         }
         umma_commit(&empty[s]);
       }
@@ -180,11 +225,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         break;
       }
       tc_fence_after();
-      int m0, n0;
-      p_tile(t, mtiles, ntiles, m0, n0);
+      int m0, n0, wn;
+      p_tile(walk, t, m0, n0, wn);
       const int row = m0 + q * 32 + lane;
       const float rs = (row < M) ? row_scale[row] * b_scale : 0.0f;
-      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)buf * PBN;
+      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)buf * WBN;
       // linear epilogue: this row's beta and gamma2, its M-step sums over the
       // tile's columns, and the operand scale b_scale 2^-e_bound (the row's
       // own 2^e_row cancels: p' = acc 2^e_row b_scale)
@@ -194,15 +239,23 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         lb = (float)le.beta[row];
         lg2 = (float)le.gamma2[row];
       }
-      for (int c0 = 0; c0 < PBN; c0 += 32) {
+      for (int c0 = 0; c0 < wn; c0 += 32) {
         uint32_t v[32];
         tmem_ld32(tbase + (uint32_t)c0, v);
-        if (c0 + 32 == PBN) {  // the accumulator is read: hand it back to the MMAs
+        if (c0 + 32 == wn) {  // the accumulator is read: hand it back to the MMAs
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&tm_empty[buf]);
         }
-        if (n0 + c0 >= N) continue;
+        if (LIN && (c0 & (PBN - 1)) == 0) {  // a 128-column group starts: fresh sums
+          a2s = 0.0f;
+          bsum = 0.0f;
+        }
+        if (n0 + c0 >= N) {
+          if (LIN && (c0 & (PBN - 1)) == PBN - 32 && row < M && n0 + c0 - (PBN - 32) < N)
+            le.part[(int64_t)((n0 + c0) / PBN) * M + row] = make_float2(a2s, bsum);
+          continue;
+        }
         if constexpr (LIN) {
           // per element as the M-step states it, in fp32; columns past N are
           // written as zero (the operand's K padding)
@@ -242,6 +295,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
               qh[k] = make_uint4(hv[4 * k], hv[4 * k + 1], hv[4 * k + 2], hv[4 * k + 3]);
               ql[k] = make_uint4(lv[4 * k], lv[4 * k + 1], lv[4 * k + 2], lv[4 * k + 3]);
             }
+            if ((c0 & (PBN - 1)) == PBN - 32)  // the group's last chunk: its M-step sums
+              le.part[(int64_t)((n0 + c0) / PBN) * M + row] = make_float2(a2s, bsum);
           }
           continue;
         }
@@ -289,7 +344,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           __syncwarp();
         }
       }
-      if (LIN && row < M) le.part[(int64_t)row * le.ntiles + n0 / PBN] = make_float2(a2s, bsum);
     }
     if (use_reduce && lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
     __syncwarp();

@@ -493,8 +493,10 @@ mpq_status launch_ldlq(mpq_plan_s* p, const float* W, int64_t m, const float* sc
                                            : cd_panel_cols(m, n);
   const int np = (int)cdiv(n, P);
   MPQ_CUDA(cudaFuncSetAttribute(k_ldlq_tile, cudaFuncAttributeMaxDynamicSharedMemorySize, LQ_SMEM));
-  // d = 8: per-row chunk minima of the nearest-codeword scan
-  const int nchunks = p->d == 8 ? (int)cdiv(p->K, LQ8_CHUNK) : 0;
+  // d = 8: per-row minima of the nearest-codeword scan over slices of the
+  // codebook (tensor cores for lattice codebooks, else SIMT chunks)
+  const bool tc = p->d == 8 && p->vec_tc;
+  const int nchunks = p->d != 8 ? 0 : tc ? cd_scan_slices(m, p->K) : (int)cdiv(p->K, LQ8_CHUNK);
   float* part_val = nullptr;
   int* part_idx = nullptr;
   if (p->d == 8) {
@@ -533,7 +535,10 @@ mpq_status launch_ldlq(mpq_plan_s* p, const float* W, int64_t m, const float* sc
         rc = check_launch("k_ldlq_tile");
       } else {
         for (int64_t b = t0 / 8; b < (t0 + tw) / 8 && rc == MPQ_OK; ++b) {
-          {
+          if (tc) {
+            rc = launch_ldlq_vec_scan(p, m, b, scale, w.Hg, w.ldh, part_val, part_idx, nchunks, st);
+            if (rc != MPQ_OK) break;
+          } else {
             ProfScope ps_("k_ldlq8_eval", st);
             dim3 ge((unsigned)nchunks, (unsigned)cdiv(m, LQ8_ROWS));
             k_ldlq8_eval<<<ge, LQ8_ROWS, 0, st>>>(m, p->K, b, p->cb, p->cb_norm, scale, w.Hg,
@@ -545,7 +550,7 @@ mpq_status launch_ldlq(mpq_plan_s* p, const float* W, int64_t m, const float* sc
                 m, n, p->K, b, t0, tw, p->cb, scale, Ud, w.Hg, w.ldh, idx, part_val, part_idx,
                 nchunks, dhi, dlo, w.As.ld, w.As.row_unscale);
           }
-          count_launch(2);
+          count_launch(tc ? 1 : 2);
           rc = check_launch("k_ldlq8");
         }
       }

@@ -725,10 +725,9 @@ __global__ void __launch_bounds__(128)
                     double* __restrict__ beta_hat_out, int32_t* __restrict__ clamps) {
   const int64_t row = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (row >= m) return;
-  const float2* pr = part + row * ntiles;
   double a2tot = 0.0, bstot = 0.0;
   for (int t = 0; t < ntiles; ++t) {
-    const float2 v = pr[t];
+    const float2 v = part[(int64_t)t * m + row];  // tile-major: coalesced over rows
     a2tot += (double)v.x;
     bstot += (double)v.y;
   }
@@ -1031,7 +1030,8 @@ inline unsigned rows_grid(int64_t m) { return (unsigned)m; }
 // =============================================================== launchers ==
 
 mpq_status launch_init(const mpq_plan_s* p, const float* W, int64_t m, int given, float* scale,
-                       float* offset, uint16_t* idx, double* gamma1_0, cudaStream_t st) {
+                       float* offset, uint16_t* idx, double* gamma1_0, cudaStream_t st,
+                       bool rtn) {
   if (m <= 0) return MPQ_OK;
   if (p->d == 1) {
     {
@@ -1053,6 +1053,7 @@ mpq_status launch_init(const mpq_plan_s* p, const float* W, int64_t m, int given
   }
   count_launch();
   MPQ_TRY(check_launch("k_init_rms"));
+  if (!rtn) return MPQ_OK;  // the scale alone (idx and gamma1_0 are not needed)
   const int64_t nb = m * (p->n / 8);
   if (p->vec_tc) {
     MPQ_TRY(launch_denoise_vec_tc(p, W, nullptr, scale, offset, m, nullptr, nullptr, 0.0, nullptr,

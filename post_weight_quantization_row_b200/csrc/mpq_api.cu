@@ -411,8 +411,14 @@ mpq_status solve_batch(mpq_plan_s* p, const SolveIO& io, int64_t row0, int64_t m
   int32_t* clamps = w.clamps;
   int32_t* changes = w.clamps + w.rows;  // rows x MAX_SWEEPS
   MPQ_CUDA(cudaMemsetAsync(clamps, 0, sizeof(int32_t) * mb, st));
-  // init: scale/offset, round-to-nearest (into idx), gamma1_0
-  MPQ_TRY(launch_init(p, W, mb, given, w.scale, w.offset, idx, w.gamma1_0, st));
+  // init: scale/offset, round-to-nearest (into idx), gamma1_0.  A greedy
+  // vector solve overwrites idx with the greedy pass and reads gamma1_0 only
+  // for adaptive CD or the row statistics: without those it skips the
+  // round-to-nearest pass
+  const bool rtn = !(io.T_vamp == 0 && p->params.greedy_init && p->d == 8 &&
+                     !(p->params.cd_skip_precision > 0.0) && io.stats == nullptr);
+  MPQ_TRY(launch_init(p, W, mb, given, w.scale, w.offset, idx, w.gamma1_0, st, rtn));
+  if (!rtn) MPQ_TRY(fill_f64(w.gamma1_0, mb, 0.0, st));
   MPQ_CUDA(cudaMemcpyAsync(w.gamma1, w.gamma1_0, sizeof(double) * mb, cudaMemcpyDeviceToDevice, st));
   MPQ_TRY(fill_f64(w.beta, mb, p->params.beta0, st));
   if (p->d == 1 && vamp_row_threads(n, p->G) > 0) {
@@ -595,6 +601,7 @@ mpq_status finish_plan(mpq_plan_s* p, cudaStream_t st) {
   }
   if (p->d == 8) {
     MPQ_TRY(dalloc(&p->cb_norm, p->K));
+    MPQ_TRY(dalloc(&p->cb_hnorm, p->K));
     MPQ_TRY(dalloc(&p->qtab, p->B * (int64_t)p->K));
     MPQ_TRY(build_codebook_tables(p, st));
   }
@@ -616,7 +623,7 @@ void destroy_plan(mpq_plan_s* p) {
   if (p->capture_stream) cudaStreamDestroy(p->capture_stream);
   free_workspace(p->ws);
   dfree(p->s64); dfree(p->V64); dfree(p->s32); dfree(p->V32); dfree(p->Vt32); dfree(p->H32);
-  dfree(p->Hdiag); dfree(p->cb); dfree(p->cb_norm); dfree(p->qtab); dfree(p->status);
+  dfree(p->Hdiag); dfree(p->cb); dfree(p->cb_norm); dfree(p->cb_hnorm); dfree(p->qtab); dfree(p->status);
   if (p->cb_tc) cudaFree(p->cb_tc);
   free_split(p->Vt_s); free_split(p->V_s); free_split(p->H_s); free_split(p->Lq_s);
   dfree(p->ldlq_diag);

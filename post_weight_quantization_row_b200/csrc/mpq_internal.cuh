@@ -79,7 +79,7 @@ struct Workspace {
   // still read As), and the epilogue's per-(row, column tile) M-step sums
   SplitOperand Aq;
   CUtensorMap tm_aq_hi, tm_aq_lo;
-  float2* lin_part = nullptr;      // rows x cdiv(r, 128)
+  float2* lin_part = nullptr;      // cdiv(r, 128) x rows
   int* tile_count = nullptr;       // CD: changes per (sweep, tile)
   // CD gradient h = H (w - x), rows x ldh (ldh = n rounded up to 32)
   float* Hg = nullptr;
@@ -138,6 +138,7 @@ struct mpq_plan_s {
   // vector codebook (d = 8)
   float* cb = nullptr;       // K x 8
   float* cb_norm = nullptr;  // K  |c|^2
+  float* cb_hnorm = nullptr; // K  1/2 |c|^2 (the greedy scan's score table)
   float* qtab = nullptr;     // B x K  1/2 c^T H_bb c
   bool vec_tc = false;       // the denoiser runs on the tensor cores
   int vec_tc_F = 0;          // grid bits of its exact split of t - c*
@@ -179,7 +180,8 @@ mpq_status gemm_nt_f64(const double* A, int64_t lda, const double* B, int64_t ld
                        bool accumulate = false);
 
 mpq_status launch_init(const mpq_plan_s* p, const float* W, int64_t m, int given, float* scale,
-                       float* offset, uint16_t* idx, double* gamma1_0, cudaStream_t st);
+                       float* offset, uint16_t* idx, double* gamma1_0, cudaStream_t st,
+                       bool rtn = true);
 mpq_status launch_denoise(const mpq_plan_s* p, const float* R1, const double* gamma1,
                           const float* scale, const float* offset, int64_t m, const float* W,
                           const double* gamma1_0, float* xhat1, float* vblock, double* vsum,
@@ -272,7 +274,7 @@ struct LinEpi {
   __half* q_hi = nullptr;
   __half* q_lo = nullptr;
   int64_t ldq = 0;
-  float2* part = nullptr;          // rows x ntiles
+  float2* part = nullptr;          // ntiles x rows (column tile major)
   int ntiles = 0;
   float* Uprime = nullptr;         // optional: (1 - F) p' (rows x r, fp32)
 };
@@ -308,6 +310,11 @@ mpq_status launch_denoise_vec_tc(const mpq_plan_s* p, const float* R1, const dou
 
 // tensor-core candidate scan of the vector CD step (cd_scan_tc.cu)
 int cd_scan_slices(int64_t m, int K);
+// the greedy baseline's nearest-codeword scan on the tensor cores (block b,
+// t = Wk[row, 8b..8b+7] / scale), partial minima as the CD scan's
+mpq_status launch_ldlq_vec_scan(const mpq_plan_s* p, int64_t m, int64_t b, const float* scale,
+                                const float* Wk, int64_t ldw, float* part_val, int* part_idx,
+                                int nslices, cudaStream_t st);
 mpq_status launch_cd_vec_scan(const mpq_plan_s* p, int64_t m, int64_t b, int64_t t0,
                               const float* scale, const uint16_t* idx, const float* h,
                               int64_t ldh, const float* hl, float* part_val, int* part_idx,

@@ -122,6 +122,12 @@ mpq_status build_hessian(mpq_plan_s* p, cudaStream_t st) {
   return MPQ_OK;
 }
 
+// 1/2 |c|^2, exact in fp32 (the greedy scan's score table)
+__global__ void k_half_norms(const float* __restrict__ nrm, int K, float* __restrict__ out) {
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c < K) out[c] = 0.5f * nrm[c];
+}
+
 mpq_status build_codebook_tables(mpq_plan_s* p, cudaStream_t st) {
   if (p->d != 8) return MPQ_OK;
   {
@@ -130,6 +136,12 @@ mpq_status build_codebook_tables(mpq_plan_s* p, cudaStream_t st) {
   }
   count_launch();
   MPQ_TRY(check_launch("k_codebook_norms"));
+  {
+    ProfScope ps_("k_half_norms", st);
+    k_half_norms<<<(unsigned)cdiv(p->K, 256), 256, 0, st>>>(p->cb_norm, p->K, p->cb_hnorm);
+  }
+  count_launch();
+  MPQ_TRY(check_launch("k_half_norms"));
   dim3 g((unsigned)cdiv(p->K, 256), (unsigned)p->B);
   {
     ProfScope ps_("k_block_quad", st);

@@ -122,6 +122,180 @@ __global__ void k_offdiag(const double* __restrict__ A, int64_t N, double* __res
   }
 }
 
+// ----------------------------------------------------- blocked Jacobi --
+// The same cyclic Jacobi method on blocks (Golub & Van Loan, section 8.5,
+// block Jacobi): the columns form blocks of BJ_B, block pairs follow the
+// round-robin ordering above, and in every round each pair's 2BJ_B x 2BJ_B
+// diagonal submatrix gets one cyclic sweep of 2x2 rotations (k_bj_inner, in
+// shared memory), whose product Q_I is then applied to the whole matrix at
+// once: A <- Q^T A Q tile by tile (k_bj_apply_a, tiles of rows of pair I and
+// columns of pair J: Q_I^T A_IJ Q_J) and V <- V Q (k_bj_apply_v).  A round
+// thus moves A and V through memory once instead of once per 2x2 round.
+constexpr int BJ_B = 32, BJ_P = 2 * BJ_B;  // block and pair width
+constexpr int BJ_LD = BJ_P + 1;            // padded shared-memory rows
+constexpr int BJ_TILE = BJ_P * BJ_LD;      // doubles per shared tile
+
+__device__ __forceinline__ void bj_pair_index(int64_t nb, int64_t k, int64_t pi, int* gi) {
+  int64_t p, q;
+  rr_pair(nb, k, pi, &p, &q);
+  for (int t = 0; t < BJ_P; ++t) gi[t] = (int)(t < BJ_B ? p * BJ_B + t : q * BJ_B + t - BJ_B);
+}
+
+// One sweep of the 2x2 cyclic Jacobi on the pair's submatrix; Q (64 x 64,
+// row-major) is the product of its rotations.
+__global__ void __launch_bounds__(256)
+    k_bj_inner(const double* __restrict__ A, int64_t N, int64_t nb, int64_t k,
+               double* __restrict__ Qout) {
+  extern __shared__ double bj_in[];
+  double(*S)[BJ_LD] = reinterpret_cast<double(*)[BJ_LD]>(bj_in);
+  double(*Q)[BJ_LD] = reinterpret_cast<double(*)[BJ_LD]>(bj_in + BJ_P * BJ_LD);
+  __shared__ double cs[BJ_B][2];
+  __shared__ int pr[BJ_B][2];
+  __shared__ int gi[BJ_P];
+  const int t = threadIdx.x;
+  if (t == 0) bj_pair_index(nb, k, blockIdx.x, gi);
+  __syncthreads();
+  for (int e = t; e < BJ_P * BJ_P; e += blockDim.x) {
+    const int i = e / BJ_P, j = e % BJ_P;
+    S[i][j] = A[(int64_t)gi[i] * N + gi[j]];
+    Q[i][j] = (i == j) ? 1.0 : 0.0;
+  }
+  __syncthreads();
+  for (int kk = 0; kk < BJ_P - 1; ++kk) {
+    if (t < BJ_B) {
+      int64_t pp, qq;
+      rr_pair(BJ_P, kk, t, &pp, &qq);
+      const double app = S[pp][pp], aqq = S[qq][qq], apq = S[pp][qq];
+      double c = 1.0, sn = 0.0;
+      if (apq != 0.0 && fabs(apq) > 1e-300) {
+        const double tau = (aqq - app) / (2.0 * apq);
+        const double tt = (tau >= 0.0) ? 1.0 / (tau + sqrt(1.0 + tau * tau))
+                                       : -1.0 / (-tau + sqrt(1.0 + tau * tau));
+        c = 1.0 / sqrt(1.0 + tt * tt);
+        sn = tt * c;
+      }
+      cs[t][0] = c;
+      cs[t][1] = sn;
+      pr[t][0] = (int)pp;
+      pr[t][1] = (int)qq;
+    }
+    __syncthreads();
+    for (int e = t; e < BJ_B * BJ_P; e += blockDim.x) {  // rows: J^T S
+      const int r = e / BJ_P, j = e % BJ_P;
+      const int pp = pr[r][0], qq = pr[r][1];
+      const double c = cs[r][0], sn = cs[r][1];
+      const double sp = S[pp][j], sq = S[qq][j];
+      S[pp][j] = c * sp - sn * sq;
+      S[qq][j] = sn * sp + c * sq;
+    }
+    __syncthreads();
+    for (int e = t; e < BJ_B * BJ_P; e += blockDim.x) {  // columns: (J^T S) J, and Q J
+      const int r = e / BJ_P, i = e % BJ_P;
+      const int pp = pr[r][0], qq = pr[r][1];
+      const double c = cs[r][0], sn = cs[r][1];
+      const double sp = S[i][pp], sq = S[i][qq];
+      S[i][pp] = c * sp - sn * sq;
+      S[i][qq] = sn * sp + c * sq;
+      const double qp = Q[i][pp], qv = Q[i][qq];
+      Q[i][pp] = c * qp - sn * qv;
+      Q[i][qq] = sn * qp + c * qv;
+    }
+    __syncthreads();
+    if (t < BJ_B) S[pr[t][0]][pr[t][1]] = S[pr[t][1]][pr[t][0]] = 0.0;  // annihilated
+    __syncthreads();
+  }
+  double* qo = Qout + (int64_t)blockIdx.x * BJ_P * BJ_P;
+  for (int e = t; e < BJ_P * BJ_P; e += blockDim.x) qo[e] = Q[e / BJ_P][e % BJ_P];
+}
+
+// 64 x 64 x 64 products in shared memory: each of 256 threads owns a 4 x 4
+// block of the result
+__device__ __forceinline__ void bj_mm(const double (*X)[BJ_LD], bool xt, const double (*Y)[BJ_LD],
+                                      double (*Z)[BJ_LD]) {
+  const int ti = (threadIdx.x / 16) * 4, tj = (threadIdx.x % 16) * 4;
+  double acc[4][4] = {};
+  for (int kk = 0; kk < BJ_P; ++kk) {
+    double xv[4], yv[4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a) xv[a] = xt ? X[kk][ti + a] : X[ti + a][kk];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) yv[b] = Y[kk][tj + b];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) acc[a][b] = fma(xv[a], yv[b], acc[a][b]);
+  }
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) Z[ti + a][tj + b] = acc[a][b];
+}
+
+constexpr int BJ_APPLY_SMEM = 4 * BJ_TILE * (int)sizeof(double);
+
+// A[rows of pair I, cols of pair J] <- Q_I^T A_IJ Q_J (the tiles partition A)
+__global__ void __launch_bounds__(256)
+    k_bj_apply_a(double* __restrict__ A, int64_t N, int64_t nb, int64_t k,
+                 const double* __restrict__ Qall) {
+  extern __shared__ double bj_sm[];
+  double(*T)[BJ_LD] = reinterpret_cast<double(*)[BJ_LD]>(bj_sm);
+  double(*QI)[BJ_LD] = reinterpret_cast<double(*)[BJ_LD]>(bj_sm + BJ_TILE);
+  double(*QJ)[BJ_LD] = reinterpret_cast<double(*)[BJ_LD]>(bj_sm + 2 * BJ_TILE);
+  double(*U)[BJ_LD] = reinterpret_cast<double(*)[BJ_LD]>(bj_sm + 3 * BJ_TILE);
+  __shared__ int gI[BJ_P], gJ[BJ_P];
+  const int t = threadIdx.x;
+  if (t == 0) {
+    bj_pair_index(nb, k, blockIdx.y, gI);
+    bj_pair_index(nb, k, blockIdx.x, gJ);
+  }
+  __syncthreads();
+  const double* qi = Qall + (int64_t)blockIdx.y * BJ_P * BJ_P;
+  const double* qj = Qall + (int64_t)blockIdx.x * BJ_P * BJ_P;
+  for (int e = t; e < BJ_P * BJ_P; e += blockDim.x) {
+    const int i = e / BJ_P, j = e % BJ_P;
+    T[i][j] = A[(int64_t)gI[i] * N + gJ[j]];
+    QI[i][j] = qi[e];
+    QJ[i][j] = qj[e];
+  }
+  __syncthreads();
+  bj_mm(QI, true, T, U);   // U = Q_I^T T
+  __syncthreads();
+  bj_mm(U, false, QJ, T);  // T = U Q_J
+  __syncthreads();
+  for (int e = t; e < BJ_P * BJ_P; e += blockDim.x) {
+    const int i = e / BJ_P, j = e % BJ_P;
+    A[(int64_t)gI[i] * N + gJ[j]] = T[i][j];
+  }
+}
+
+// V[rows r0 .. r0+63, cols of pair J] <- V[.., pair J] Q_J
+__global__ void __launch_bounds__(256)
+    k_bj_apply_v(double* __restrict__ V, int64_t N, int64_t nb, int64_t k,
+                 const double* __restrict__ Qall) {
+  extern __shared__ double bj_sm[];
+  double(*T)[BJ_LD] = reinterpret_cast<double(*)[BJ_LD]>(bj_sm);
+  double(*QJ)[BJ_LD] = reinterpret_cast<double(*)[BJ_LD]>(bj_sm + BJ_TILE);
+  double(*U)[BJ_LD] = reinterpret_cast<double(*)[BJ_LD]>(bj_sm + 2 * BJ_TILE);
+  __shared__ int gJ[BJ_P];
+  const int t = threadIdx.x;
+  const int64_t r0 = (int64_t)blockIdx.y * BJ_P;
+  if (t == 0) bj_pair_index(nb, k, blockIdx.x, gJ);
+  __syncthreads();
+  const double* qj = Qall + (int64_t)blockIdx.x * BJ_P * BJ_P;
+  for (int e = t; e < BJ_P * BJ_P; e += blockDim.x) {
+    const int i = e / BJ_P, j = e % BJ_P;
+    T[i][j] = V[(r0 + i) * N + gJ[j]];
+    QJ[i][j] = qj[e];
+  }
+  __syncthreads();
+  bj_mm(T, false, QJ, U);
+  __syncthreads();
+  for (int e = t; e < BJ_P * BJ_P; e += blockDim.x) {
+    const int i = e / BJ_P, j = e % BJ_P;
+    V[(r0 + i) * N + gJ[j]] = U[i][j];
+  }
+}
+
 __global__ void k_eye(double* V, int64_t N) {
   for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < N * N;
        e += (int64_t)gridDim.x * blockDim.x)
@@ -220,7 +394,11 @@ struct DevBuf {
 
 // Symmetric eigendecomposition of the N0 x N0 matrix G (device, fp64):
 // descending eigenvalues lam (N0) and eigenvectors E (N0 x N0, columns).
+mpq_status jacobi_eig_blocked(const double* G, int64_t N0, double* lam, double* E,
+                              cudaStream_t st);
+
 mpq_status jacobi_eig(const double* G, int64_t N0, double* lam, double* E, cudaStream_t st) {
+  if (N0 >= 256) return jacobi_eig_blocked(G, N0, lam, E, st);
   const int64_t N = N0 + (N0 & 1);  // even; the pad row/col is zero
   DevBuf<double> A, V, cs, red;
   DevBuf<int> rank;
@@ -275,6 +453,86 @@ mpq_status jacobi_eig(const double* G, int64_t N0, double* lam, double* E, cudaS
       dg += h[2 * b + 1];
     }
     converged = !(off > 1e-28 * dg) || dg == 0.0;
+  }
+  if (!converged) return fail(MPQ_ERR_TIMEOUT, "Jacobi eigensolver did not converge in 40 sweeps");
+  {
+    ProfScope ps_("k_rank", st);
+    k_rank<<<(unsigned)cdiv(N0, 256), 256, 0, st>>>(A.p, N, N0, rank.p);
+  }
+  {
+    ProfScope ps_("k_gather_sorted", st);
+    k_gather_sorted<<<(unsigned)cdiv(N0 * N0, 256), 256, 0, st>>>(A.p, V.p, N, N0, rank.p, lam, E);
+  }
+  count_launch(2);
+  return check_launch("jacobi sort");
+}
+
+// Blocked cyclic Jacobi (k_bj_*): N0 padded with zero rows and columns to a
+// multiple of the pair width (a zero row never rotates, so the padding stays
+// decoupled and the first N0 diagonal entries are G's eigenvalues).
+mpq_status jacobi_eig_blocked(const double* G, int64_t N0, double* lam, double* E,
+                              cudaStream_t st) {
+  const int64_t N = round_up(N0, BJ_P);
+  const int64_t nb = N / BJ_B, npairs = nb / 2;
+  DevBuf<double> A, V, Q, red;
+  DevBuf<int> rank;
+  MPQ_TRY(A.alloc(N * N));
+  MPQ_TRY(V.alloc(N * N));
+  MPQ_TRY(Q.alloc(npairs * BJ_P * BJ_P));
+  const int red_blocks = 256;
+  MPQ_TRY(red.alloc(2 * red_blocks));
+  MPQ_TRY(rank.alloc(N0));
+  MPQ_CUDA(cudaFuncSetAttribute(k_bj_inner, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                2 * BJ_TILE * (int)sizeof(double)));
+  MPQ_CUDA(cudaFuncSetAttribute(k_bj_apply_a, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                BJ_APPLY_SMEM));
+  MPQ_CUDA(cudaFuncSetAttribute(k_bj_apply_v, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                3 * BJ_TILE * (int)sizeof(double)));
+  {
+    ProfScope ps_("k_pad", st);
+    k_pad<<<g1(N * N), 256, 0, st>>>(G, N0, N, A.p);
+  }
+  {
+    ProfScope ps_("k_eye", st);
+    k_eye<<<g1(N * N), 256, 0, st>>>(V.p, N);
+  }
+  count_launch(2);
+  MPQ_TRY(check_launch("jacobi init"));
+  std::vector<double> h(2 * red_blocks);
+  bool converged = false;
+  for (int sweep = 0; sweep < JACOBI_MAX_SWEEPS && !converged; ++sweep) {
+    {
+      ProfScope ps_("k_offdiag", st);
+      k_offdiag<<<red_blocks, 256, 0, st>>>(A.p, N, red.p);
+    }
+    count_launch();
+    MPQ_CUDA(cudaMemcpyAsync(h.data(), red.p, sizeof(double) * 2 * red_blocks, cudaMemcpyDeviceToHost, st));
+    MPQ_CUDA(cudaStreamSynchronize(st));
+    double off = 0.0, dg = 0.0;
+    for (int b = 0; b < red_blocks; ++b) {
+      off += h[2 * b];
+      dg += h[2 * b + 1];
+    }
+    converged = !(off > 1e-28 * dg) || dg == 0.0;
+    if (converged) break;
+    for (int64_t k = 0; k < nb - 1; ++k) {
+      {
+        ProfScope ps_("k_bj_inner", st);
+        k_bj_inner<<<(unsigned)npairs, 256, 2 * BJ_TILE * sizeof(double), st>>>(A.p, N, nb, k, Q.p);
+      }
+      {
+        ProfScope ps_("k_bj_apply_a", st);
+        k_bj_apply_a<<<dim3((unsigned)npairs, (unsigned)npairs), 256, BJ_APPLY_SMEM, st>>>(
+            A.p, N, nb, k, Q.p);
+      }
+      {
+        ProfScope ps_("k_bj_apply_v", st);
+        k_bj_apply_v<<<dim3((unsigned)npairs, (unsigned)(N / BJ_P)), 256,
+                       3 * BJ_TILE * sizeof(double), st>>>(V.p, N, nb, k, Q.p);
+      }
+      count_launch(3);
+    }
+    MPQ_TRY(check_launch("blocked jacobi sweep"));
   }
   if (!converged) return fail(MPQ_ERR_TIMEOUT, "Jacobi eigensolver did not converge in 40 sweeps");
   {

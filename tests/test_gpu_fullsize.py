@@ -18,13 +18,24 @@ its own spectrum from X.
    within 1e-5 |E|, the stated exemption).  Every decision before it is held
    bit-exact; only the rest of that row's sweep is exempt.
 
-3. The whole solve: every marginal-MAP index whose oracle logit gap exceeds
-   1e-4 matches; rows whose final indices match the oracle's hold the final
-   energy to 1e-3; rows whose trajectories parted at a near-tie end in other
-   local minima of the same objective, within 10% each (a sanity bound), and
+3. The whole solve.  Unanchored (tau = inf), VAMP carries a rounding-level
+   perturbation of w through 16 iterations unchanged (1e-7 stays 1e-7 in the
+   oracle), so every marginal-MAP index whose oracle cavity lies more than
+   1e-3 codebook units from a decision boundary must match; rows whose final
+   indices match the oracle's hold the final energy to 1e-3; rows that parted
+   must have met a near-tie.  With the default anchor (tau = 0.2) the last
+   iterations are not contracting on these layers (the oracle turns a 1e-7
+   perturbation of w into a 5e-3 change of the cavity by iteration 15), so
+   fp32 and fp64 trajectories part legitimately and only the statistics are
+   compared.  In both, rows that parted end in other local minima of the same
+   objective, within 10% each unanchored and 25% anchored (sanity bounds),
    the sample mean of the signed relative energy difference stays within 1%
-   (no bias).  At these sizes nearly every row meets a CD near-tie
-   somewhere in its 3 sweeps, hence the sweep-by-sweep check of item 2."""
+   (no bias), and the device's mean energy is at most 1% above the
+   oracle's.  At these
+   sizes nearly every row meets a CD near-tie somewhere in its 3 sweeps,
+   hence the sweep-by-sweep check of item 2."""
+import math
+
 import numpy as np
 import pytest
 import torch
@@ -38,16 +49,18 @@ pytestmark = pytest.mark.gpu
 
 ENERGY_TOL = 1e-3
 EXEMPT_ROW_TOL = 1e-1   # a sanity bound on rows whose trajectories parted at a near-tie
+ANCHORED_ROW_TOL = 2.5e-1  # and on rows whose anchored VAMP trajectories parted
 EXEMPT_MEAN_TOL = 1e-2
 CD_TIE = 1e-5
 # marginal MAP near-ties in codebook units (reading of the exemption for the
 # argmax after T_vamp fp32 iterations): the oracle's logit gap over the
-# effective precision g = gamma1 s^2 + 1/tau^2 is half the difference of the
-# two nearest squared distances to the effective cavity, i.e. the cavity's
-# distance to the decision boundary in grid steps for a scalar grid
-MAP_TIE_CB = 1e-2
+# precision gamma1 s^2 is half the difference of the two nearest squared
+# distances to the cavity, i.e. the cavity's distance to the decision
+# boundary in grid steps for a scalar grid
+MAP_TIE_CB = 1e-3
 _CACHE = {}
 _REF = {}
+_PLANS = {}
 
 
 def _plan_and_spectrum(name):
@@ -81,18 +94,33 @@ def _grid32(p, rows):
     return sc.astype(np.float32), off.astype(np.float32)
 
 
-def _oracle_solve(name, k):
+def _oracle_solve(name, k, tau=orc.TAU):
     """The oracle's solve of k sampled rows on the fp32 grid (cached: the CD
     test starts from its marginal MAP)."""
-    key = (name, k)
+    key = (name, k, tau)
     if key not in _REF:
         p, _, s, V = _plan_and_spectrum(name)
         rows = _sample(p, k)
         sc, off = _grid32(p, rows)
         ref = orc.solve(p.W[rows], codebook_for(p), s, V, p.T_vamp, p.cd_sweeps,
-                        sc.astype(np.float64), off.astype(np.float64))
+                        sc.astype(np.float64), off.astype(np.float64), tau=tau)
         _REF[key] = (rows, sc, off, ref)
     return _REF[key]
+
+
+def _plan_tau(name, tau):
+    """A plan with another anchor, on the spectrum the default plan computed
+    from X (no second eigensolve)."""
+    import post_weight_quantization_row_b200 as mpq
+    p, plan, _, _ = _plan_and_spectrum(name)
+    if tau == orc.TAU:
+        return plan
+    if (name, tau) not in _PLANS:
+        s_cu, V_cu = plan.spectrum()
+        _PLANS[(name, tau)] = mpq.Plan.from_spectrum(s_cu, V_cu, p.d, p.levels,
+                                                     codebook=p.codebook if p.d == 8 else None,
+                                                     tau=tau)
+    return _PLANS[(name, tau)]
 
 
 # ---------------------------------------------------------- linear module ---
@@ -191,34 +219,38 @@ def test_fullsize_cd_identical_init_e8t8():
 
 # --------------------------------------------------------------- the solve ---
 
-def _solve(name, k):
-    p, plan, s, V = _plan_and_spectrum(name)
-    rows, sc, off, ref = _oracle_solve(name, k)
+def _solve(name, k, tau=orc.TAU, min_sure=0.99):
+    p, _, s, V = _plan_and_spectrum(name)
+    plan = _plan_tau(name, tau)
+    rows, sc, off, ref = _oracle_solve(name, k, tau)
     cb = codebook_for(p)
     W = cu(p.W)
     out = plan.solve(W, p.T_vamp, p.cd_sweeps, stats=True)
-    mp = plan.solve(W, p.T_vamp, 0)
     # the device's own grid is the fp32 grid the oracle was given
     st = plan.stage_init(W)
     assert np.array_equal(host(st["scale"])[rows], sc)
     assert np.array_equal(host(st["offset"])[rows], off)
-    # marginal MAP: every index outside the oracle's near-ties
-    got_map = idx_np(mp["idx"])[rows]
-    g_eff = ref.gamma1 * sc.astype(np.float64) ** 2 + 1.0 / orc.TAU ** 2
-    sure = ref.map_gap / g_eff[:, None] > MAP_TIE_CB
-    assert sure.mean() > 0.97, sure.mean()
-    bad = np.flatnonzero((got_map != ref.idx_map) & sure)
-    assert bad.size == 0, (bad[:10], (ref.map_gap / g_eff[:, None]).ravel()[bad[:10]])
-    # final indices and energies
     got = idx_np(out["idx"])[rows]
     e_gpu = host(out["energy"]).astype(np.float64)[rows]
     rel = (e_gpu - ref.energy) / ref.energy
     same = np.all(got == ref.idx, axis=1)
-    assert np.all(np.abs(rel[same]) <= ENERGY_TOL)
-    # rows that parted must have met a near-tie of the oracle
-    tied = np.any(~sure, axis=1) | (ref.cd.first_tie >= 0)
-    assert np.all(tied[~same]), rows[~same & ~tied]
-    assert np.all(np.abs(rel) <= EXEMPT_ROW_TOL), (rows, e_gpu, ref.energy)
+    if not np.isfinite(tau):
+        # marginal MAP: every index outside the oracle's near-ties
+        mp = plan.solve(W, p.T_vamp, 0)
+        got_map = idx_np(mp["idx"])[rows]
+        gap = ref.map_gap / (ref.gamma1 * sc.astype(np.float64) ** 2)[:, None]
+        sure = gap > MAP_TIE_CB
+        assert sure.mean() > min_sure, sure.mean()
+        bad = np.flatnonzero((got_map != ref.idx_map) & sure)
+        assert bad.size == 0, (bad[:10], gap.ravel()[bad[:10]])
+        # final indices and energies; rows that parted met a near-tie
+        assert np.all(np.abs(rel[same]) <= ENERGY_TOL)
+        tied = np.any(~sure, axis=1) | (ref.cd.first_tie >= 0)
+        assert np.all(tied[~same]), rows[~same & ~tied]
+    row_tol = EXEMPT_ROW_TOL if not np.isfinite(tau) else ANCHORED_ROW_TOL
+    assert np.all(np.abs(rel) <= row_tol), (rows, e_gpu, ref.energy)
+    # on the sample, the device is not worse than the oracle on average
+    assert e_gpu.mean() <= (1.0 + EXEMPT_MEAN_TOL) * ref.energy.mean()
     assert abs(np.mean(rel)) <= EXEMPT_MEAN_TOL, np.mean(rel)
     # the outputs agree with each other on the device
     wh = host(out["w_hat"])[rows]
@@ -236,23 +268,27 @@ def _solve(name, k):
     return same.mean()
 
 
-def test_fullsize_solve_l1b():
-    _solve("l1b", 32)
+@pytest.mark.parametrize("tau", [math.inf, orc.TAU])
+def test_fullsize_solve_l1b(tau):
+    _solve("l1b", 32, tau)
 
 
-def test_fullsize_solve_q4096():
-    _solve("q4096", 32)
+@pytest.mark.parametrize("tau", [math.inf, orc.TAU])
+def test_fullsize_solve_q4096(tau):
+    _solve("q4096", 32, tau)
 
 
-def test_fullsize_solve_down_rank_space():
-    _solve("down", 8)
+@pytest.mark.parametrize("tau", [math.inf, orc.TAU])
+def test_fullsize_solve_down_rank_space(tau):
+    _solve("down", 8, tau)
     assert _CACHE["down"][1].r == 4096 and _CACHE["down"][1].n == 14336
 
 
 def test_fullsize_solve_e8t8_lattice():
-    _solve("e8t8", 2)
+    _solve("e8t8", 2, math.inf, min_sure=0.95)
 
 
 def test_fullsize_solve_e8_lattice_t16():
-    # the 2-bit E8 configuration at T_vamp = 16 (its own spectrum: same X)
+    # the 2-bit E8 configuration at T_vamp = 16 and the default anchor (its
+    # plan shares the e8t8 plan: same X)
     _solve("e8", 2)
