@@ -7,11 +7,11 @@
 // hi + lo carries ~22 significand bits and the three products recover an
 // fp32-accurate contraction (the dropped lo*lo term is ~2^-22 relative).
 // Both operands are K-major (K contiguous).  Persistent kernel, one CTA per
-// SM walking 128 x 128 x 64 tiles: fp16 kind::f16 MMAs with the fp32
-// accumulator in TMEM (two 128-column accumulators, so that the epilogue of
-// one tile overlaps the MMAs of the next), operands staged by TMA (128-byte
-// swizzle, no multicast) through a 3-stage mbarrier ring that runs across
-// tiles.  Warp 0 issues TMA, warp 1 owns TMEM and issues the MMAs from one
+// SM walking 128 x 256 (or 128 x 128) tiles in K steps of 32: fp16 kind::f16
+// MMAs with the fp32 accumulator in TMEM (two 256-column accumulators, so
+// that the epilogue of one tile overlaps the MMAs of the next), operands
+// staged by TMA (64-byte swizzle, no multicast) through a 4-stage mbarrier
+// ring that runs across tiles.  Warp 0 issues TMA, warp 1 owns TMEM and issues the MMAs from one
 // thread, warps 2-5 read the accumulators back (tcgen05.ld) and store C.
 #include <cuda.h>
 #include <cuda_fp16.h>
@@ -26,23 +26,24 @@ namespace mpq {
 namespace {
 using namespace tcx;
 
-constexpr int BM = 128, BK = 64;
-constexpr int A_TILE = BM * BK * 2;                 // 16 KiB
+constexpr int BM = 128, BK = 32;
+constexpr int A_TILE = BM * BK * 2;                 // 8 KiB
 constexpr int TC_THREADS = 192;
 
 // ------------------------------------------------------- persistent GEMM --
-// One CTA per SM walks the output tiles: a 2-stage TMA ring runs across
-// tiles, and two TMEM accumulators let the epilogue of one tile overlap the
-// MMAs of the next.  Tiles are 128 x 256 (the three MMAs of a k-step then
+// One CTA per SM walks the output tiles: a 4-stage TMA ring of K = 32 slices
+// (48 KiB per stage, so that three stages of loads are in flight while the
+// MMAs read the fourth) runs across tiles, and two TMEM accumulators let the
+// epilogue of one tile overlap the MMAs of the next.  Tiles are 128 x 256 (the three MMAs of a k-step then
 // read 96 B of shared memory per cycle of tensor work, against 128 B, the
 // whole shared-memory bandwidth, at 128 x 128) for as many full waves of
 // the grid as the product holds; the 128 x 256 tiles left over for a last,
 // partial wave run as two 128 x 128 tiles each, and an odd 128-column strip
 // at the right edge as 128 x 128 tiles too.  Wide tiles go in groups of 8
 // M-tiles (M fastest) so that the A and B panels in flight stay in L2.
-constexpr int PBN = 128, WBN = 256, PSTAGES = 2, PGROUP = 8;
-constexpr int P_B_TILE = PBN * BK * 2;                        // 16 KiB per 128 rows of B
-constexpr int P_STAGE = 2 * A_TILE + 2 * 2 * P_B_TILE;        // 96 KiB
+constexpr int PBN = 128, WBN = 256, PSTAGES = 4, PGROUP = 8;
+constexpr int P_B_TILE = PBN * BK * 2;                        // 8 KiB per 128 rows of B
+constexpr int P_STAGE = 2 * A_TILE + 2 * 2 * P_B_TILE;        // 48 KiB
 constexpr int P_STG_WARP = 8192;                              // epilogue staging per warp
 constexpr int P_SMEM = PSTAGES * P_STAGE + 4 * P_STG_WARP + 1024 + 256;
 constexpr uint32_t P_TMEM_COLS = 2 * WBN;
@@ -197,8 +198,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk) {
           const uint32_t off = kk * 32;
-          const uint64_t dah = sw128_desc(a_hi + off), dal = sw128_desc(a_lo + off);
-          const uint64_t dbh = sw128_desc(b_hi + off), dbl = sw128_desc(b_lo + off);
+          const uint64_t dah = sw64_desc(a_hi + off), dal = sw64_desc(a_lo + off);
+          const uint64_t dbh = sw64_desc(b_hi + off), dbl = sw64_desc(b_lo + off);
           umma_f16(d, dah, dbh, idesc, (kt | kk) != 0 ? 1u : 0u);
           umma_f16(d, dah, dbl, idesc, 1u);
           if (!a_exact) umma_f16(d, dal, dbh, idesc, 1u);
@@ -420,7 +421,7 @@ mpq_status make_tmap_f16(CUtensorMap* tm, const void* base, int64_t inner, int64
   cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
   cuuint32_t es[2] = {1, 1};
   CUresult r = g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims,
-                        strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS)
     return fail(MPQ_ERR_CUDA, "cuTensorMapEncodeTiled failed with code " + std::to_string((int)r));

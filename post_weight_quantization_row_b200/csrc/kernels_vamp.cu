@@ -709,12 +709,12 @@ __global__ void __launch_bounds__(ROW_THREADS)
 // 128 rank components, sum F and sum F^2 u^2 + s^2/(beta s^2 + gamma2) with
 // u = s p', F = gamma2/(beta s^2 + gamma2) (the MPQ note's key design 2:
 // 1/beta_hat = (1/r) sum_l [(gamma2/(beta s_l^2 + gamma2))^2 u_l^2 +
-// s_l^2/(beta s_l^2 + gamma2)]).  One thread per row adds the tiles in order
-// in fp64, then: alpha2 = [sum F + n - r]/n (reading R6), beta_hat, beta <-
+// s_l^2/(beta s_l^2 + gamma2)]).  One warp per row adds the tiles in fp64 in
+// a fixed order, then: alpha2 = [sum F + n - r]/n (reading R6), beta_hat, beta <-
 // (1 - rho) beta + rho beta_hat (R7), gamma1' = gamma2 (1 - alpha2)/alpha2
 // and the l2d coefficients 1/(1 - alpha2), alpha2/(1 - alpha2), each clipped
 // (R5), and the second GEMM's row scale 2^(e_row + e_bound).
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(256)
     k_linear_finish(const float2* __restrict__ part, int ntiles, int64_t m, int64_t n, int64_t r,
                     int e_bound, const float* __restrict__ a_unscale,
                     float* __restrict__ q_unscale, const double* __restrict__ gamma2,
@@ -723,14 +723,24 @@ __global__ void __launch_bounds__(128)
                     double* __restrict__ gamma1_out, double* __restrict__ coef,
                     double* __restrict__ kappa, double* __restrict__ alpha2_out,
                     double* __restrict__ beta_hat_out, int32_t* __restrict__ clamps) {
-  const int64_t row = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  // one warp per row: lane l adds the column groups l, l + 32, ... in fp64,
+  // then a butterfly over the lanes (a fixed order: the sums are
+  // deterministic); lane 0 finishes the row
+  const int lane = threadIdx.x & 31;
+  const int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (row >= m) return;
   double a2tot = 0.0, bstot = 0.0;
-  for (int t = 0; t < ntiles; ++t) {
-    const float2 v = part[(int64_t)t * m + row];  // tile-major: coalesced over rows
+  for (int t = lane; t < ntiles; t += 32) {
+    const float2 v = part[(int64_t)t * m + row];
     a2tot += (double)v.x;
     bstot += (double)v.y;
   }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    a2tot += __shfl_xor_sync(0xffffffffu, a2tot, o);
+    bstot += __shfl_xor_sync(0xffffffffu, bstot, o);
+  }
+  if (lane != 0) return;
   q_unscale[row] = ldexpf(a_unscale[row], e_bound);
   int cnt = 0;
   const double b = beta[row], g2 = gamma2[row];
@@ -1175,7 +1185,7 @@ mpq_status launch_linear_finish(const mpq_plan_s* p, int64_t m, const float2* pa
   const mpq_params& q = p->params;
   {
     ProfScope ps_("k_linear_finish", st);
-    k_linear_finish<<<(unsigned)cdiv(m, 128), 128, 0, st>>>(
+    k_linear_finish<<<(unsigned)cdiv(m * 32, 256), 256, 0, st>>>(
         part, ntiles, m, p->n, p->r, e_bound, a_unscale, q_unscale, gamma2, gamma1_0, beta,
         q.damping, q.gamma_lo_rel, q.gamma_hi_rel, q.alpha_min, q.alpha_max, gamma1_out, coef,
         kappa, alpha2, beta_hat, clamps);

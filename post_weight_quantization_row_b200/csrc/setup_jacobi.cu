@@ -132,8 +132,10 @@ __global__ void k_offdiag(const double* __restrict__ A, int64_t N, double* __res
 // columns of pair J: Q_I^T A_IJ Q_J) and V <- V Q (k_bj_apply_v).  A round
 // thus moves A and V through memory once instead of once per 2x2 round.
 constexpr int BJ_B = 32, BJ_P = 2 * BJ_B;  // block and pair width
-constexpr int BJ_LD = BJ_P + 1;            // padded shared-memory rows
+constexpr int BJ_LD = BJ_P + 2;            // padded rows of the product tiles (16-byte aligned)
 constexpr int BJ_TILE = BJ_P * BJ_LD;      // doubles per shared tile
+constexpr int BJ_LDI = BJ_P + 1;           // rows of the rotation tiles: odd, so that a column
+                                           // read by 32 lanes touches every bank pair once
 
 __device__ __forceinline__ void bj_pair_index(int64_t nb, int64_t k, int64_t pi, int* gi) {
   int64_t p, q;
@@ -147,8 +149,8 @@ __global__ void __launch_bounds__(256)
     k_bj_inner(const double* __restrict__ A, int64_t N, int64_t nb, int64_t k,
                double* __restrict__ Qout) {
   extern __shared__ double bj_in[];
-  double(*S)[BJ_LD] = reinterpret_cast<double(*)[BJ_LD]>(bj_in);
-  double(*Q)[BJ_LD] = reinterpret_cast<double(*)[BJ_LD]>(bj_in + BJ_P * BJ_LD);
+  double(*S)[BJ_LDI] = reinterpret_cast<double(*)[BJ_LDI]>(bj_in);
+  double(*Q)[BJ_LDI] = reinterpret_cast<double(*)[BJ_LDI]>(bj_in + BJ_P * BJ_LDI);
   __shared__ double cs[BJ_B][2];
   __shared__ int pr[BJ_B][2];
   __shared__ int gi[BJ_P];
@@ -208,36 +210,50 @@ __global__ void __launch_bounds__(256)
   for (int e = t; e < BJ_P * BJ_P; e += blockDim.x) qo[e] = Q[e / BJ_P][e % BJ_P];
 }
 
-// 64 x 64 x 64 products in shared memory: each of 256 threads owns a 4 x 4
-// block of the result
-__device__ __forceinline__ void bj_mm(const double (*X)[BJ_LD], bool xt, const double (*Y)[BJ_LD],
-                                      double (*Z)[BJ_LD]) {
-  const int ti = (threadIdx.x / 16) * 4, tj = (threadIdx.x % 16) * 4;
-  double acc[4][4] = {};
+// 64 x 64 x 64 products in shared memory, Z = Xt^T Y (Xt holds X transposed,
+// so that both operands are read along rows): each of 128 threads owns an
+// 8 x 4 block of Z and reads 8 + 4 values per k as 16-byte loads (6 loads per
+// 32 FMAs).  With tout the block is stored transposed.
+constexpr int BJ_THREADS = 128;
+__device__ __forceinline__ void bj_mm(const double (*Xt)[BJ_LD], const double (*Y)[BJ_LD],
+                                      double (*Z)[BJ_LD], bool tout) {
+  const int ti = (threadIdx.x / 16) * 8, tj = (threadIdx.x % 16) * 4;
+  double acc[8][4] = {};
   for (int kk = 0; kk < BJ_P; ++kk) {
-    double xv[4], yv[4];
+    double xv[8], yv[4];
 #pragma unroll
-    for (int a = 0; a < 4; ++a) xv[a] = xt ? X[kk][ti + a] : X[ti + a][kk];
+    for (int a = 0; a < 8; a += 2) {
+      const double2 v = *reinterpret_cast<const double2*>(&Xt[kk][ti + a]);
+      xv[a] = v.x;
+      xv[a + 1] = v.y;
+    }
 #pragma unroll
-    for (int b = 0; b < 4; ++b) yv[b] = Y[kk][tj + b];
+    for (int b = 0; b < 4; b += 2) {
+      const double2 v = *reinterpret_cast<const double2*>(&Y[kk][tj + b]);
+      yv[b] = v.x;
+      yv[b + 1] = v.y;
+    }
 #pragma unroll
-    for (int a = 0; a < 4; ++a)
+    for (int a = 0; a < 8; ++a)
 #pragma unroll
       for (int b = 0; b < 4; ++b) acc[a][b] = fma(xv[a], yv[b], acc[a][b]);
   }
 #pragma unroll
-  for (int a = 0; a < 4; ++a)
+  for (int a = 0; a < 8; ++a)
 #pragma unroll
-    for (int b = 0; b < 4; ++b) Z[ti + a][tj + b] = acc[a][b];
+    for (int b = 0; b < 4; ++b) {
+      if (tout) Z[tj + b][ti + a] = acc[a][b];
+      else Z[ti + a][tj + b] = acc[a][b];
+    }
 }
 
 constexpr int BJ_APPLY_SMEM = 4 * BJ_TILE * (int)sizeof(double);
 
 // A[rows of pair I, cols of pair J] <- Q_I^T A_IJ Q_J (the tiles partition A)
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(BJ_THREADS)
     k_bj_apply_a(double* __restrict__ A, int64_t N, int64_t nb, int64_t k,
                  const double* __restrict__ Qall) {
-  extern __shared__ double bj_sm[];
+  extern __shared__ __align__(16) double bj_sm[];
   double(*T)[BJ_LD] = reinterpret_cast<double(*)[BJ_LD]>(bj_sm);
   double(*QI)[BJ_LD] = reinterpret_cast<double(*)[BJ_LD]>(bj_sm + BJ_TILE);
   double(*QJ)[BJ_LD] = reinterpret_cast<double(*)[BJ_LD]>(bj_sm + 2 * BJ_TILE);
@@ -258,9 +274,9 @@ __global__ void __launch_bounds__(256)
     QJ[i][j] = qj[e];
   }
   __syncthreads();
-  bj_mm(QI, true, T, U);   // U = Q_I^T T
+  bj_mm(QI, T, U, true);   // U^T with U = Q_I^T T
   __syncthreads();
-  bj_mm(U, false, QJ, T);  // T = U Q_J
+  bj_mm(U, QJ, T, false);  // T = U Q_J
   __syncthreads();
   for (int e = t; e < BJ_P * BJ_P; e += blockDim.x) {
     const int i = e / BJ_P, j = e % BJ_P;
@@ -269,11 +285,11 @@ __global__ void __launch_bounds__(256)
 }
 
 // V[rows r0 .. r0+63, cols of pair J] <- V[.., pair J] Q_J
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(BJ_THREADS)
     k_bj_apply_v(double* __restrict__ V, int64_t N, int64_t nb, int64_t k,
                  const double* __restrict__ Qall) {
-  extern __shared__ double bj_sm[];
-  double(*T)[BJ_LD] = reinterpret_cast<double(*)[BJ_LD]>(bj_sm);
+  extern __shared__ __align__(16) double bj_sm[];
+  double(*Tt)[BJ_LD] = reinterpret_cast<double(*)[BJ_LD]>(bj_sm);
   double(*QJ)[BJ_LD] = reinterpret_cast<double(*)[BJ_LD]>(bj_sm + BJ_TILE);
   double(*U)[BJ_LD] = reinterpret_cast<double(*)[BJ_LD]>(bj_sm + 2 * BJ_TILE);
   __shared__ int gJ[BJ_P];
@@ -284,11 +300,11 @@ __global__ void __launch_bounds__(256)
   const double* qj = Qall + (int64_t)blockIdx.x * BJ_P * BJ_P;
   for (int e = t; e < BJ_P * BJ_P; e += blockDim.x) {
     const int i = e / BJ_P, j = e % BJ_P;
-    T[i][j] = V[(r0 + i) * N + gJ[j]];
+    Tt[j][i] = V[(r0 + i) * N + gJ[j]];  // the tile, transposed
     QJ[i][j] = qj[e];
   }
   __syncthreads();
-  bj_mm(T, false, QJ, U);
+  bj_mm(Tt, QJ, U, false);  // U = T Q_J
   __syncthreads();
   for (int e = t; e < BJ_P * BJ_P; e += blockDim.x) {
     const int i = e / BJ_P, j = e % BJ_P;
@@ -522,12 +538,12 @@ mpq_status jacobi_eig_blocked(const double* G, int64_t N0, double* lam, double* 
       }
       {
         ProfScope ps_("k_bj_apply_a", st);
-        k_bj_apply_a<<<dim3((unsigned)npairs, (unsigned)npairs), 256, BJ_APPLY_SMEM, st>>>(
+        k_bj_apply_a<<<dim3((unsigned)npairs, (unsigned)npairs), BJ_THREADS, BJ_APPLY_SMEM, st>>>(
             A.p, N, nb, k, Q.p);
       }
       {
         ProfScope ps_("k_bj_apply_v", st);
-        k_bj_apply_v<<<dim3((unsigned)npairs, (unsigned)(N / BJ_P)), 256,
+        k_bj_apply_v<<<dim3((unsigned)npairs, (unsigned)(N / BJ_P)), BJ_THREADS,
                        3 * BJ_TILE * sizeof(double), st>>>(V.p, N, nb, k, Q.p);
       }
       count_launch(3);

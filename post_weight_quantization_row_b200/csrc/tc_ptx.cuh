@@ -96,6 +96,19 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
   return d;
 }
 
+// K-major tile with 64-byte rows (32 fp16) and 64-byte swizzle, as TMA writes
+// it with CU_TENSOR_MAP_SWIZZLE_64B: 8-row groups 512 B apart (SBO), layout
+// type 4 (SWIZZLE_64B), version 1; the second 16-element K step of a row
+// starts 32 B further.
+__device__ __forceinline__ uint64_t sw64_desc(uint32_t saddr) {
+  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1 << 16;
+  d |= (uint64_t)(512 >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)4 << 61;
+  return d;
+}
+
 __device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
                                          uint32_t idesc, uint32_t accum) {
   asm volatile(
