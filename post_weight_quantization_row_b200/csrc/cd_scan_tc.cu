@@ -21,7 +21,7 @@
 // minimum of its slice per row, and the apply step combines the slices.
 // Warps 0-15 read TMEM (warp w: lanes 32 (w % 4) .. +31, columns 32 (w / 4)
 // .. +31 of each tile), warp 16 owns TMEM and issues the MMAs, warp 17 issues
-// the bulk copies of the codebook operand and the qtab row through a 6-stage
+// the bulk copies of the codebook operand and the qtab row through a 20-stage
 // ring; TMEM holds 4 score buffers.  All waits are bounded.
 #include <cuda.h>
 #include <cuda_fp16.h>
@@ -36,7 +36,10 @@ namespace mpq {
 namespace {
 using namespace tcx;
 
-constexpr int SC_M = 128, SC_N = 128, SC_STAGES = 6, SC_BUFS = 4;
+// The ring runs 20 codebook tiles (4.5 KiB each) ahead of the MMAs: an
+// epilogue pass over a tile takes a few hundred cycles, so fewer stages would
+// leave the scan waiting on the latency of the copies from L2.
+constexpr int SC_M = 128, SC_N = 128, SC_STAGES = 20, SC_BUFS = 4;
 constexpr int SC_EPI_WARPS = 16, SC_WGS = 4;
 constexpr int SC_THREADS = (SC_EPI_WARPS + 2) * 32;
 constexpr int SC_MMA_WARP = SC_EPI_WARPS, SC_LOAD_WARP = SC_EPI_WARPS + 1;

@@ -6,18 +6,30 @@
 // (x * 2^-e = hi + lo, hi = fp16(x * 2^-e), lo = fp16(x * 2^-e - hi)), so
 // hi + lo carries ~22 significand bits and the three products recover an
 // fp32-accurate contraction (the dropped lo*lo term is ~2^-22 relative).
-// Both operands are K-major (K contiguous).  Persistent kernel, one CTA per
-// SM walking 128 x 256 (or 128 x 128) tiles in K steps of 32: fp16 kind::f16
-// MMAs with the fp32 accumulator in TMEM (two 256-column accumulators, so
-// that the epilogue of one tile overlaps the MMAs of the next), operands
-// staged by TMA (64-byte swizzle, no multicast) through a 4-stage mbarrier
-// ring that runs across tiles.  Warp 0 issues TMA, warp 1 owns TMEM and issues the MMAs from one
-// thread, warps 2-5 read the accumulators back (tcgen05.ld) and store C.
+// Both operands are K-major (K contiguous).  Persistent kernel in two forms:
+//  - CTA pairs (M > 128, K >= 512): a cluster of two CTAs on two SMs computes each
+//    256 x 256 tile with tcgen05.mma.cta_group::2.  Each CTA stages 128 rows
+//    of A and its half (128 rows) of the tile's B; the MMAs, issued by the
+//    even CTA, read both CTAs' shared memory and leave each CTA's 128 x 256
+//    accumulator in its own TMEM.  K steps of 64 with 128-byte swizzle
+//    through a 3-stage ring of 64 KiB.  Per MAC an SM moves 2/3 of the
+//    operand bytes of a single-CTA 128 x 256 tile, in half as many
+//    128-byte requests as 64-byte rows take.
+//  - single CTAs (M <= 128, K < 512, or no pair fits): 128 x 256 tiles, K
+//    steps of 32 with 64-byte swizzle through a 4-stage ring of 48 KiB.
+// fp16 kind::f16 MMAs with the fp32 accumulator in TMEM (two 256-column
+// accumulators, so that the epilogue of one tile overlaps the MMAs of the
+// next); operands staged by TMA (no multicast) through an mbarrier ring that
+// runs across tiles.  Warp 0 issues TMA, warp 1 owns TMEM and issues the MMAs
+// from one thread, warps 2-5 read the accumulators back (tcgen05.ld) and
+// store C.
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <cudaTypedefs.h>
 
+#include <map>
 #include <mutex>
+#include <tuple>
 
 #include "mpq_internal.cuh"
 #include "tc_ptx.cuh"
@@ -26,37 +38,55 @@ namespace mpq {
 namespace {
 using namespace tcx;
 
-constexpr int BM = 128, BK = 32;
-constexpr int A_TILE = BM * BK * 2;                 // 8 KiB
 constexpr int TC_THREADS = 192;
 
-// ------------------------------------------------------- persistent GEMM --
-// One CTA per SM walks the output tiles: a 4-stage TMA ring of K = 32 slices
-// (48 KiB per stage, so that three stages of loads are in flight while the
-// MMAs read the fourth) runs across tiles, and two TMEM accumulators let the
-// epilogue of one tile overlap the MMAs of the next.  Tiles are 128 x 256 (the three MMAs of a k-step then
-// read 96 B of shared memory per cycle of tensor work, against 128 B, the
-// whole shared-memory bandwidth, at 128 x 128) for as many full waves of
-// the grid as the product holds; the 128 x 256 tiles left over for a last,
-// partial wave run as two 128 x 128 tiles each, and an odd 128-column strip
-// at the right edge as 128 x 128 tiles too.  Wide tiles go in groups of 8
-// M-tiles (M fastest) so that the A and B panels in flight stay in L2.
-constexpr int PBN = 128, WBN = 256, PSTAGES = 4, PGROUP = 8;
-constexpr int P_B_TILE = PBN * BK * 2;                        // 8 KiB per 128 rows of B
-constexpr int P_STAGE = 2 * A_TILE + 2 * 2 * P_B_TILE;        // 48 KiB
-constexpr int P_STG_WARP = 8192;                              // epilogue staging per warp
-constexpr int P_SMEM = PSTAGES * P_STAGE + 4 * P_STG_WARP + 1024 + 256;
+// Tiles are 128 (single) or 256 (pair) rows by 256 columns (the three MMAs of
+// a k-step then read 96 B of shared memory per cycle of tensor work, against
+// 128 B, the whole shared-memory bandwidth, at 128 x 128) for as many full
+// waves of the grid as the product holds; the 256-column tiles left over for
+// a last, partial wave run as two 128-column tiles each, and an odd
+// 128-column strip at the right edge as 128-column tiles too.  Wide tiles go
+// in groups of 8 M-tiles (M fastest) so that the A and B panels in flight
+// stay in L2.
+constexpr int PBN = 128, WBN = 256, PGROUP = 8;
+constexpr int P_STG_WARP = 8192;  // epilogue staging per warp
 constexpr uint32_t P_TMEM_COLS = 2 * WBN;
-constexpr uint32_t P_IDESC_W = idesc_f16(BM, WBN), P_IDESC_N = idesc_f16(BM, PBN);
 
-// The walk over tiles for a grid of G CTAs: T2 wide tiles in all, the first
-// tmain (whole waves) as such, the rest split in halves, then the strip.
+template <bool PAIR>
+struct TcCfg;
+template <>
+struct TcCfg<false> {
+  static constexpr int BK = 32, STAGES = 4, TM = 128;
+  static constexpr int B_BOX = 128;                 // rows of B per TMA box
+  static constexpr int B_HALF = 256 * BK * 2;       // one split half of up to 256 rows of B
+  static constexpr uint32_t IDESC_W = idesc_f16(128, WBN), IDESC_N = idesc_f16(128, PBN);
+  __device__ static uint64_t desc(uint32_t a) { return sw64_desc(a); }
+};
+template <>
+struct TcCfg<true> {
+  static constexpr int BK = 64, STAGES = 3, TM = 256;
+  static constexpr int B_BOX = 64;
+  static constexpr int B_HALF = 128 * BK * 2;       // this CTA's half of the tile's B
+  static constexpr uint32_t IDESC_W = idesc_f16(256, WBN), IDESC_N = idesc_f16(256, PBN);
+  __device__ static uint64_t desc(uint32_t a) { return sw128_desc(a); }
+};
+template <bool PAIR>
+struct TcLayout {
+  static constexpr int A_TILE = 128 * TcCfg<PAIR>::BK * 2;  // 128 rows of one split half
+  static constexpr int STAGE = 2 * A_TILE + 2 * TcCfg<PAIR>::B_HALF;
+  static constexpr int SMEM = TcCfg<PAIR>::STAGES * STAGE + 4 * P_STG_WARP + 1024 + 256;
+};
+static_assert(TcLayout<true>::SMEM <= 232448, "pair GEMM shared memory");
+
+// The walk over tiles for G workers (CTAs or CTA pairs) and tiles TM rows
+// high: T2 wide tiles in all, the first tmain (whole waves) as such, the rest
+// split in halves, then the strip.
 struct TileWalk {
   int mtiles, np2, tmain, nsplit, total;
 };
-__device__ __forceinline__ TileWalk tile_walk(int M, int N, int G) {
+__device__ __forceinline__ TileWalk tile_walk(int M, int N, int G, int TM) {
   TileWalk tw;
-  tw.mtiles = (M + BM - 1) / BM;
+  tw.mtiles = (M + TM - 1) / TM;
   const int n128 = (N + PBN - 1) / PBN;
   tw.np2 = n128 / 2;
   const int t2 = tw.mtiles * tw.np2;
@@ -65,32 +95,34 @@ __device__ __forceinline__ TileWalk tile_walk(int M, int N, int G) {
   tw.total = tw.tmain + tw.nsplit + tw.mtiles * (n128 % 2);
   return tw;
 }
-__device__ __forceinline__ void wide_tile(int t, int mtiles, int np2, int& m0, int& n0) {
+__device__ __forceinline__ void wide_tile(int t, int mtiles, int np2, int TM, int& m0, int& n0) {
   const int per_group = PGROUP * np2;
   const int g = t / per_group, w = t % per_group;
   const int gm = min(PGROUP, mtiles - g * PGROUP);  // M-tiles in this group
-  m0 = (g * PGROUP + w % gm) * BM;
+  m0 = (g * PGROUP + w % gm) * TM;
   n0 = (w / gm) * WBN;
 }
 // tile t of the walk: its origin and width (256 or 128 columns)
-__device__ __forceinline__ void p_tile(const TileWalk& tw, int t, int& m0, int& n0, int& wn) {
+__device__ __forceinline__ void p_tile(const TileWalk& tw, int t, int TM, int& m0, int& n0,
+                                       int& wn) {
   if (t < tw.tmain) {
-    wide_tile(t, tw.mtiles, tw.np2, m0, n0);
+    wide_tile(t, tw.mtiles, tw.np2, TM, m0, n0);
     wn = WBN;
   } else if (t < tw.tmain + tw.nsplit) {
     const int s = t - tw.tmain;
-    wide_tile(tw.tmain + s / 2, tw.mtiles, tw.np2, m0, n0);
+    wide_tile(tw.tmain + s / 2, tw.mtiles, tw.np2, TM, m0, n0);
     n0 += (s & 1) * PBN;
     wn = PBN;
   } else {
-    m0 = (t - tw.tmain - tw.nsplit) * BM;
+    m0 = (t - tw.tmain - tw.nsplit) * TM;
     n0 = tw.np2 * WBN;
     wn = PBN;
   }
 }
 
 // LIN = 1: the linear module's epilogue (LinEpi) instead of storing C.
-template <int LIN>
+// PAIR: launched in clusters of two CTAs (see the head of the file).
+template <int LIN, bool PAIR>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     k_gemm_tcp(const __grid_constant__ CUtensorMap ta_hi, const __grid_constant__ CUtensorMap ta_lo,
                const __grid_constant__ CUtensorMap tb_hi, const __grid_constant__ CUtensorMap tb_lo,
@@ -99,84 +131,127 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                const float* __restrict__ row_scale, float b_scale, int accumulate, int a_exact,
                const int* __restrict__ gate, const __grid_constant__ CUtensorMap tc_out,
                int use_reduce, int* status, const __grid_constant__ LinEpi le) {
+  using Cfg = TcCfg<PAIR>;
+  using Lay = TcLayout<PAIR>;
+  constexpr int BK = Cfg::BK, NST = Cfg::STAGES, TM = Cfg::TM;
+  constexpr int A_TILE = Lay::A_TILE, STAGE = Lay::STAGE;
+  // (a gate read by both CTAs of a pair: they leave together, before any
+  // cluster-wide step)
   if (gate != nullptr && *gate == 0) return;  // nothing to add
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t* stg_all = smem + PSTAGES * P_STAGE;
+  uint8_t* stg_all = smem + NST * STAGE;
   uint64_t* full = (uint64_t*)(stg_all + 4 * P_STG_WARP);
-  uint64_t* empty = full + PSTAGES;
-  uint64_t* tm_full = empty + PSTAGES;
+  uint64_t* empty = full + NST;
+  uint64_t* tm_full = empty + NST;
   uint64_t* tm_empty = tm_full + 2;
   uint32_t* tmem_slot = (uint32_t*)(tm_empty + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const TileWalk walk = tile_walk(M, N, gridDim.x);
+  // rank 0 of a pair issues the MMAs and owns the pair's full / TMEM-empty
+  // barriers; both ranks own their empty and TMEM-full barriers
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const int worker = PAIR ? (int)cluster_id_x() : (int)blockIdx.x;
+  const int nworkers = PAIR ? (int)(gridDim.x / 2) : (int)gridDim.x;
+  const TileWalk walk = tile_walk(M, N, nworkers, TM);
   const int tiles = walk.total;
   const int KT = (K + BK - 1) / BK;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < PSTAGES; ++s) {
+    for (int s = 0; s < NST; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tm_full[b], 1);
-      mbar_init(&tm_empty[b], 4);  // the four epilogue warps
+      mbar_init(&tm_empty[b], PAIR ? 8 : 4);  // the epilogue warps (of both CTAs)
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
   if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(tmem_slot)),
-                 "r"(P_TMEM_COLS));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    if constexpr (PAIR) {
+      asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       smem_u32(tmem_slot)),
+                   "r"(P_TMEM_COLS));
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+    } else {
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       smem_u32(tmem_slot)),
+                   "r"(P_TMEM_COLS));
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync();  // both CTAs' barriers exist before any remote use
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // shared::cluster addresses of rank 0's barriers (the own ones on rank 0)
+  const uint32_t full_r0 = PAIR ? map_to_rank(smem_u32(full), 0) : smem_u32(full);
+  const uint32_t tm_empty_r0 = PAIR ? map_to_rank(smem_u32(tm_empty), 0) : smem_u32(tm_empty);
 
   if (warp == 0 && lane == 0) {
     // ---------------------------------------------------------- producer
     uint32_t it = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+    for (int t = worker; t < tiles && ok; t += nworkers) {
       int m0, n0, wn;
-      p_tile(walk, t, m0, n0, wn);
-      const int nb = wn / PBN;  // 128-row boxes of B
+      p_tile(walk, t, TM, m0, n0, wn);
+      const int am0 = m0 + (int)rank * 128;              // this CTA's 128 rows of A
+      const int brows = PAIR ? wn / 2 : wn;               // and its rows of B
+      const int bn0 = n_off + n0 + (int)rank * brows;
+      const int nbox = brows / Cfg::B_BOX;
+      const uint32_t bytes = (uint32_t)((a_exact ? 1 : 2) * A_TILE + 2 * brows * BK * 2);
       for (int kt = 0; kt < KT; ++kt, ++it) {
-        const int s = it % PSTAGES;
-        if (it >= PSTAGES && !mbar_wait(&empty[s], (it / PSTAGES - 1) & 1)) {
+        const int s = it % NST;
+        if (it >= NST && !mbar_wait(&empty[s], (it / NST - 1) & 1)) {
           atomicOr(status, STATUS_TIMEOUT);
           ok = false;
           break;
         }
-        uint8_t* base = smem + s * P_STAGE;
-        mbar_expect_tx(&full[s], (a_exact ? A_TILE : 2 * A_TILE) + 2 * nb * P_B_TILE);
-        tma_load_2d(&ta_hi, &full[s], base, a_k0 + kt * BK, m0);
-        if (!a_exact) tma_load_2d(&ta_lo, &full[s], base + A_TILE, a_k0 + kt * BK, m0);
-        for (int b = 0; b < nb; ++b) {
-          tma_load_2d(&tb_hi, &full[s], base + 2 * A_TILE + b * P_B_TILE, b_k0 + kt * BK,
-                      n_off + n0 + b * PBN);
-          tma_load_2d(&tb_lo, &full[s], base + 2 * A_TILE + (2 + b) * P_B_TILE, b_k0 + kt * BK,
-                      n_off + n0 + b * PBN);
+        uint8_t* base = smem + s * STAGE;
+        const int kc_a = a_k0 + kt * BK, kc_b = b_k0 + kt * BK;
+        if constexpr (PAIR) {
+          // rank 0's full barrier counts both CTAs' bytes; rank 1's copies
+          // complete on it from the peer
+          const uint32_t fb = full_r0 + 8u * (uint32_t)s;
+          if (rank == 0) mbar_expect_tx(&full[s], 2 * bytes);
+          tma_load_2d_cg2(&ta_hi, fb, base, kc_a, am0);
+          if (!a_exact) tma_load_2d_cg2(&ta_lo, fb, base + A_TILE, kc_a, am0);
+          for (int b = 0; b < nbox; ++b) {
+            uint8_t* bb = base + 2 * A_TILE + b * Cfg::B_BOX * BK * 2;
+            tma_load_2d_cg2(&tb_hi, fb, bb, kc_b, bn0 + b * Cfg::B_BOX);
+            tma_load_2d_cg2(&tb_lo, fb, bb + Cfg::B_HALF, kc_b, bn0 + b * Cfg::B_BOX);
+          }
+        } else {
+          mbar_expect_tx(&full[s], bytes);
+          tma_load_2d(&ta_hi, &full[s], base, kc_a, am0);
+          if (!a_exact) tma_load_2d(&ta_lo, &full[s], base + A_TILE, kc_a, am0);
+          for (int b = 0; b < nbox; ++b) {
+            uint8_t* bb = base + 2 * A_TILE + b * Cfg::B_BOX * BK * 2;
+            tma_load_2d(&tb_hi, &full[s], bb, kc_b, bn0 + b * Cfg::B_BOX);
+            tma_load_2d(&tb_lo, &full[s], bb + Cfg::B_HALF, kc_b, bn0 + b * Cfg::B_BOX);
+          }
         }
       }
     }
-    for (uint32_t q = (it > PSTAGES ? it - PSTAGES : 0); q < it; ++q)  // copies land before exit
-      for (uint32_t i = 0; i < (1u << 25) && !mbar_try_wait(&full[q % PSTAGES], (q / PSTAGES) & 1); ++i)
-        if (i > 256) __nanosleep(64);
-  } else if (warp == 1 && lane == 0) {
+    // copies land before exit (rank 0's full barriers count both CTAs' copies;
+    // rank 1 waits for rank 0 at the closing cluster barrier)
+    if (rank == 0)
+      for (uint32_t q = (it > (uint32_t)NST ? it - NST : 0); q < it; ++q)
+        for (uint32_t i = 0; i < (1u << 25) && !mbar_try_wait(&full[q % NST], (q / NST) & 1); ++i)
+          if (i > 256) __nanosleep(64);
+  } else if (warp == 1 && lane == 0 && rank == 0) {
     // ------------------------------------------------------- MMA issuer
     uint32_t it = 0, tl = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++tl) {
+    for (int t = worker; t < tiles && ok; t += nworkers, ++tl) {
       const int buf = tl & 1;
       int m0, n0, wn;
-      p_tile(walk, t, m0, n0, wn);
-      const uint32_t idesc = wn == WBN ? P_IDESC_W : P_IDESC_N;
-      if (tl >= 2 && !mbar_wait(&tm_empty[buf], (tl / 2 - 1) & 1)) {
+      p_tile(walk, t, TM, m0, n0, wn);
+      const uint32_t idesc = wn == WBN ? Cfg::IDESC_W : Cfg::IDESC_N;
+      if (tl >= 2 && !mbar_wait_cl(&tm_empty[buf], (tl / 2 - 1) & 1)) {
         atomicOr(status, STATUS_TIMEOUT);
         ok = false;
         break;
@@ -184,29 +259,48 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       tc_fence_after();
       const uint32_t d = tmem + (uint32_t)buf * WBN;
       for (int kt = 0; kt < KT; ++kt, ++it) {
-        const int s = it % PSTAGES;
-        if (!mbar_wait(&full[s], (it / PSTAGES) & 1)) {
+        const int s = it % NST;
+        if (!mbar_wait_cl(&full[s], (it / NST) & 1)) {
           atomicOr(status, STATUS_TIMEOUT);
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t a_hi = smem_u32(smem + s * P_STAGE);
+        const uint32_t a_hi = smem_u32(smem + s * STAGE);
         const uint32_t a_lo = a_hi + A_TILE;
-        const uint32_t b_hi = a_hi + 2 * A_TILE;     // wn rows: one or two 128-row boxes
-        const uint32_t b_lo = b_hi + 2 * P_B_TILE;
+        const uint32_t b_hi = a_hi + 2 * A_TILE;  // this CTA's rows of B (the peer's at the same offset)
+        const uint32_t b_lo = b_hi + Cfg::B_HALF;
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk) {
-          const uint32_t off = kk * 32;
-          const uint64_t dah = sw64_desc(a_hi + off), dal = sw64_desc(a_lo + off);
-          const uint64_t dbh = sw64_desc(b_hi + off), dbl = sw64_desc(b_lo + off);
-          umma_f16(d, dah, dbh, idesc, (kt | kk) != 0 ? 1u : 0u);
-          umma_f16(d, dah, dbl, idesc, 1u);
-          if (!a_exact) umma_f16(d, dal, dbh, idesc, 1u);
+          const uint32_t off = kk * 32;  // 16 fp16 along a swizzled row
+          const uint64_t dah = Cfg::desc(a_hi + off), dal = Cfg::desc(a_lo + off);
+          const uint64_t dbh = Cfg::desc(b_hi + off), dbl = Cfg::desc(b_lo + off);
+          const uint32_t acc0 = (kt | kk) != 0 ? 1u : 0u;
+          if constexpr (PAIR) {
+            umma_f16_cg2(d, dah, dbh, idesc, acc0);
+            umma_f16_cg2(d, dah, dbl, idesc, 1u);
+            if (!a_exact) umma_f16_cg2(d, dal, dbh, idesc, 1u);
+          } else {
+            umma_f16(d, dah, dbh, idesc, acc0);
+            umma_f16(d, dah, dbl, idesc, 1u);
+            if (!a_exact) umma_f16(d, dal, dbh, idesc, 1u);
+          }
         }
-        umma_commit(&empty[s]);
+        if constexpr (PAIR) {
+          umma_commit_cg2(smem_u32(&empty[s]));                 // this CTA's stage
+          umma_commit_cg2(map_to_rank(smem_u32(&empty[s]), 1));  // and the peer's
+        } else {
+          umma_commit(&empty[s]);
+        }
       }
-      if (ok) umma_commit(&tm_full[buf]);
+      if (ok) {
+        if constexpr (PAIR) {
+          umma_commit_cg2(smem_u32(&tm_full[buf]));
+          umma_commit_cg2(map_to_rank(smem_u32(&tm_full[buf]), 1));
+        } else {
+          umma_commit(&tm_full[buf]);
+        }
+      }
     }
     for (uint32_t q = (tl > 2 ? tl - 2 : 0); q < tl; ++q)  // MMAs finish before TMEM is freed
       for (uint32_t i = 0; i < (1u << 25) && !mbar_try_wait(&tm_full[q & 1], (q / 2) & 1); ++i)
@@ -218,16 +312,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     float* stage = reinterpret_cast<float*>(stg0);
     uint32_t tl = 0;
     int nb = 0;  // bulk reduce groups issued by this warp
-    for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++tl) {
+    for (int t = worker; t < tiles; t += nworkers, ++tl) {
       const int buf = tl & 1;
-      const bool ok = __all_sync(0xffffffffu, mbar_wait(&tm_full[buf], (tl / 2) & 1));
+      const bool ok = __all_sync(0xffffffffu, mbar_wait_cl(&tm_full[buf], (tl / 2) & 1));
       if (!ok) {
         if (lane == 0) atomicOr(status, STATUS_TIMEOUT);
         break;
       }
       tc_fence_after();
       int m0, n0, wn;
-      p_tile(walk, t, m0, n0, wn);
+      p_tile(walk, t, TM, m0, n0, wn);
+      m0 += (int)rank * 128;  // this CTA's rows of the tile
       const int row = m0 + q * 32 + lane;
       const float rs = (row < M) ? row_scale[row] * b_scale : 0.0f;
       const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)buf * WBN;
@@ -246,7 +341,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if (c0 + 32 == wn) {  // the accumulator is read: hand it back to the MMAs
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&tm_empty[buf]);
+          if (lane == 0) {
+            if constexpr (PAIR) mbar_arrive_cl(tm_empty_r0 + 8u * (uint32_t)buf);
+            else mbar_arrive(&tm_empty[buf]);
+          }
         }
         if (LIN && (c0 & (PBN - 1)) == 0) {  // a 128-column group starts: fresh sums
           a2s = 0.0f;
@@ -351,10 +449,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync();  // no peer still reads this CTA's memory or barriers
   if (warp == 1) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
-                 "r"(P_TMEM_COLS));
+    if constexpr (PAIR)
+      asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                   "r"(P_TMEM_COLS));
+    else
+      asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                   "r"(P_TMEM_COLS));
   }
 }
 
@@ -408,24 +511,58 @@ mpq_status get_encoder() {
 
 bool g_smem_attr_set[64] = {};
 int g_sms[64] = {};
+int g_pairs[64] = {};
 
 }  // namespace
 
-mpq_status make_tmap_f16(CUtensorMap* tm, const void* base, int64_t inner, int64_t rows,
-                         int64_t ld_elems, int box_rows) {
+namespace {
+// K-major fp16 operand map: boxes of box_k x box_rows with the swizzle of the
+// kernel that reads them (32 x rows with 64-byte, 64 x rows with 128-byte)
+mpq_status encode_f16(CUtensorMap* tm, const void* base, int64_t inner, int64_t rows,
+                      int64_t ld_elems, int box_k, int box_rows) {
   MPQ_TRY(get_encoder());
   if (((uintptr_t)base & 15) || (ld_elems * 2) % 16 || inner % 64 || rows < box_rows)
     return fail(MPQ_ERR_INVALID_ARG, "tensor map: misaligned operand");
   cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)(ld_elems * 2)};
-  cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+  cuuint32_t box[2] = {(cuuint32_t)box_k, (cuuint32_t)box_rows};
   cuuint32_t es[2] = {1, 1};
+  const CUtensorMapSwizzle sw = box_k == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   CUresult r = g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims,
-                        strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                        strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS)
     return fail(MPQ_ERR_CUDA, "cuTensorMapEncodeTiled failed with code " + std::to_string((int)r));
   return MPQ_OK;
+}
+
+// Maps of the pair kernel, encoded on first use over the operand's whole
+// padded width (its zero K padding included) and kept: an encoding depends
+// only on the key, so a key met again (memory reused with the same shape)
+// maps the same bytes.
+using PairKey = std::tuple<const void*, int64_t, int64_t, int>;
+std::map<PairKey, CUtensorMap> g_pair_maps;
+std::mutex g_pair_mu;
+
+mpq_status pair_map(const void* base, int64_t rows_pad, int64_t ld, int box_rows,
+                    CUtensorMap* out) {
+  std::lock_guard<std::mutex> lk(g_pair_mu);
+  const PairKey key{base, rows_pad, ld, box_rows};
+  auto f = g_pair_maps.find(key);
+  if (f != g_pair_maps.end()) {
+    *out = f->second;
+    return MPQ_OK;
+  }
+  if (g_pair_maps.size() > 4096) g_pair_maps.clear();
+  MPQ_TRY(encode_f16(out, base, ld, rows_pad, ld, 64, box_rows));
+  g_pair_maps.emplace(key, *out);
+  return MPQ_OK;
+}
+}  // namespace
+
+mpq_status make_tmap_f16(CUtensorMap* tm, const void* base, int64_t inner, int64_t rows,
+                         int64_t ld_elems, int box_rows) {
+  return encode_f16(tm, base, inner, rows, ld_elems, TcCfg<false>::BK, box_rows);
 }
 
 mpq_status make_tmap_f32_out(CUtensorMap* tm, const float* base, int64_t cols, int64_t rows,
@@ -475,10 +612,35 @@ mpq_status gemm_tc(const SplitOperand& A, const CUtensorMap& ta_hi, const CUtens
     return fail(MPQ_ERR_INVALID_ARG, "gemm_tc: operand smaller than the problem");
   int dev = 0;
   MPQ_CUDA(cudaGetDevice(&dev));
-  if (dev >= 0 && dev < 64 && !g_smem_attr_set[dev]) {
-    MPQ_CUDA(cudaFuncSetAttribute(k_gemm_tcp<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM));
-    MPQ_CUDA(cudaFuncSetAttribute(k_gemm_tcp<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM));
+  if (dev < 0 || dev >= 64) return fail(MPQ_ERR_CUDA, "gemm_tc: device index out of range");
+  if (!g_smem_attr_set[dev]) {
+    MPQ_CUDA(cudaFuncSetAttribute(k_gemm_tcp<0, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  TcLayout<false>::SMEM));
+    MPQ_CUDA(cudaFuncSetAttribute(k_gemm_tcp<1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  TcLayout<false>::SMEM));
+    MPQ_CUDA(cudaFuncSetAttribute(k_gemm_tcp<0, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  TcLayout<true>::SMEM));
+    MPQ_CUDA(cudaFuncSetAttribute(k_gemm_tcp<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  TcLayout<true>::SMEM));
     MPQ_CUDA(cudaDeviceGetAttribute(&g_sms[dev], cudaDevAttrMultiProcessorCount, dev));
+    // CTA pairs that can be resident at once (0: no pair fits, single CTAs only)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (unsigned)g_sms[dev]);
+    cfg.blockDim = dim3(TC_THREADS);
+    cfg.dynamicSmemBytes = TcLayout<true>::SMEM;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 2;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    int nc = 0;
+    if (cudaOccupancyMaxActiveClusters(&nc, k_gemm_tcp<0, true>, &cfg) != cudaSuccess) {
+      (void)cudaGetLastError();
+      nc = 0;
+    }
+    g_pairs[dev] = nc;
     g_smem_attr_set[dev] = true;
   }
   if (o.c_reduce && !o.accumulate)
@@ -486,18 +648,45 @@ mpq_status gemm_tc(const SplitOperand& A, const CUtensorMap& ta_hi, const CUtens
   if (o.lin && (o.c_reduce || o.accumulate || o.n0 != 0 || o.lin->ldq < round_up(N, PBN) ||
                 o.lin->ntiles != cdiv(N, PBN) || (o.lin->ldq % 8) != 0))
     return fail(MPQ_ERR_INVALID_ARG, "gemm_tc: linear epilogue needs a plain product over all N");
-  const int64_t tiles = cdiv(M, BM) * cdiv(N, PBN);
-  const unsigned grid = (unsigned)std::min<int64_t>(tiles, dev < 64 ? g_sms[dev] : 148);
   const CUtensorMap& cmap = o.c_reduce ? *o.c_reduce : tb_hi;  // unused unless reducing
-  {
-    ProfScope ps_(tag, st);
-    const LinEpi le = o.lin ? *o.lin : LinEpi{};
-    auto kern = o.lin ? k_gemm_tcp<1> : k_gemm_tcp<0>;
-    kern<<<grid, TC_THREADS, P_SMEM, st>>>(
+  const LinEpi le = o.lin ? *o.lin : LinEpi{};
+  // CTA pairs for the long contractions; a short K (the CD updates, K = 128)
+  // is better served by the single-CTA ring, whose four 48 KiB stages hold a
+  // whole tile's K while the pair's three 64 KiB stages hold one and a half
+  const bool pair = M > 128 && K >= 512 && g_pairs[dev] > 0;
+  ProfScope ps_(tag, st);
+  if (pair) {
+    CUtensorMap pa_hi, pa_lo, pb_hi, pb_lo;
+    MPQ_TRY(pair_map(A.hi, A.rows_pad, A.ld, 128, &pa_hi));
+    MPQ_TRY(pair_map(A.lo, A.rows_pad, A.ld, 128, &pa_lo));
+    MPQ_TRY(pair_map(B.hi, B.rows_pad, B.ld, TcCfg<true>::B_BOX, &pb_hi));
+    MPQ_TRY(pair_map(B.lo, B.rows_pad, B.ld, TcCfg<true>::B_BOX, &pb_lo));
+    const int64_t tiles = cdiv(M, 256) * cdiv(N, PBN);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (unsigned)std::min<int64_t>(tiles, g_pairs[dev]));
+    cfg.blockDim = dim3(TC_THREADS);
+    cfg.dynamicSmemBytes = TcLayout<true>::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 2;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    MPQ_CUDA(cudaLaunchKernelEx(&cfg, o.lin ? k_gemm_tcp<1, true> : k_gemm_tcp<0, true>, pa_hi,
+                                pa_lo, pb_hi, pb_lo, C, ldc, (int)M, (int)N, (int)K, (int)o.a_k0,
+                                (int)o.b_k0, (int)o.n0, (const float*)A.row_unscale, b_scale_host,
+                                o.accumulate ? 1 : 0, o.a_exact ? 1 : 0, o.gate, cmap,
+                                o.c_reduce ? 1 : 0, status, le));
+  } else {
+    const int64_t tiles = cdiv(M, 128) * cdiv(N, PBN);
+    const unsigned grid = (unsigned)std::min<int64_t>(tiles, g_sms[dev]);
+    auto kern = o.lin ? k_gemm_tcp<1, false> : k_gemm_tcp<0, false>;
+    kern<<<grid, TC_THREADS, TcLayout<false>::SMEM, st>>>(
         ta_hi, ta_lo, tb_hi, tb_lo, C, ldc, (int)M, (int)N, (int)K, (int)o.a_k0, (int)o.b_k0,
-        (int)o.n0, A.row_unscale,
-        b_scale_host, o.accumulate ? 1 : 0, o.a_exact ? 1 : 0, o.gate, cmap, o.c_reduce ? 1 : 0,
-        status, le);
+        (int)o.n0, A.row_unscale, b_scale_host, o.accumulate ? 1 : 0, o.a_exact ? 1 : 0, o.gate,
+        cmap, o.c_reduce ? 1 : 0, status, le);
   }
   count_launch();
   return check_launch("k_gemm_tc");

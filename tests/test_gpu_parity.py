@@ -169,7 +169,9 @@ def test_stage_linear(mpq, m_calib):
 
 @pytest.mark.parametrize("m_out,n,m_calib", [(300, 520, 700), (130, 300, 257)])
 def test_stage_linear_multitile(mpq, m_out, n, m_calib):
-    """Several 128 x 256 x 64 tensor-core tiles with ragged M, N and K edges."""
+    """Several tensor-core tiles with ragged M, N and K edges.  At 300 and 130
+    rows the GEMMs run on CTA pairs (256-row tiles; the second pair tile of
+    300 rows is 44 rows deep, and at 130 rows the odd CTA holds 2 rows)."""
     p = mi.small_problem(313, m_out, n, m_calib, d=1, levels=8)
     s, V, s_cu, V_cu = spectrum_cuda(p.X)
     plan = make_plan(mpq, p, s_cu, V_cu)
@@ -299,15 +301,16 @@ def test_stage_cd_vector(mpq):
     assert ref.changes[:, 0].sum() > 0
 
 
-@pytest.mark.parametrize("kind", ["scalar", "e8_tensor", "gaussian_simt"])
+@pytest.mark.parametrize("kind", ["scalar", "scalar_300_rows", "e8_tensor", "gaussian_simt"])
 def test_stage_cd_panels(mpq, kind):
     # cd_panel = 256 over n = 600: panels of 256, 256 and 88 columns, the
     # last one ragged (tiles 128, 128 | 128, 128 | 88); every change reaches
     # the other panels' columns through the GEMM that closes its panel.
     # Long rows meet more near-ties (1800 steps), hence the lower bar on
-    # the share of tie-free rows.
-    if kind == "scalar":
-        p = scalar_case(seed=131, m_out=48, n=600, m=900)
+    # the share of tie-free rows.  300 rows: the gradient GEMM (K = n) runs
+    # on CTA pairs (256-row tiles, the second one 44 rows deep).
+    if kind.startswith("scalar"):
+        p = scalar_case(seed=131, m_out=300 if kind.endswith("rows") else 48, n=600, m=900)
         off_rms = False
     else:
         cb = (mi.e8_codebook_cached()[:512] if kind == "e8_tensor"
