@@ -67,7 +67,38 @@ def parse():
                          "inf = the unanchored form)")
     ap.add_argument("--spectrum-cache", default=None,
                     help="npz file: reuse the spectrum a previous run computed on the device")
+    ap.add_argument("--gram-rows", type=int, default=262144,
+                    help="also time the streamed fp64 Gram accumulation of this many calibration "
+                         "rows (chunks of 16384 through mpq_gram_accumulate; 0 = skip)")
     return ap.parse_args()
+
+
+def gram_timing(n, rows, dev):
+    """Seconds (CUDA events) to accumulate X^T X over `rows` synthetic rows
+    of width n in chunks of 16384 through the streamed Gram handle; two
+    device-resident chunks take turns, so the time is the accumulation's."""
+    import torch
+    import post_weight_quantization_row_b200 as mpq
+    chunk = min(16384, rows)
+    g = torch.Generator(device=dev)
+    g.manual_seed(20261299)
+    xs = [torch.randn(chunk, n, generator=g, device=dev, dtype=torch.float32) for _ in range(2)]
+    gram = mpq.Gram(n)
+    gram.accumulate(xs[0])  # warm-up (first use of the kernels)
+    torch.cuda.synchronize()
+    gram.close()
+    gram = mpq.Gram(n)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    done = 0
+    while done < rows:
+        k = min(chunk, rows - done)
+        gram.accumulate(xs[(done // chunk) % 2][:k])
+        done += k
+    e1.record()
+    torch.cuda.synchronize()
+    gram.close()
+    return e0.elapsed_time(e1) / 1e3
 
 
 # ------------------------------------------------------------------ dist ---
@@ -363,6 +394,12 @@ def run_mpq(args, world, rank, local):
             s_, V_ = plan.spectrum()
             np.savez(cache, s=s_.cpu().numpy(), V=V_.cpu().numpy())
     r = plan.r
+    gram_run = None
+    if args.gram_rows > 0 and rank == 0:
+        gs = gram_timing(n, args.gram_rows, dev)
+        gram_run = {"rows": args.gram_rows, "n": n, "s": round(gs, 3),
+                    "fp64_tflops": round(2.0 * args.gram_rows * n * n / gs / 1e12, 2),
+                    "what": "streamed X^T X in fp64 (mpq_gram_accumulate, 16384-row chunks)"}
     W = torch.from_numpy(p.W).to(dev)
     out = {"idx": torch.empty(m, plan.B, dtype=torch.int16, device=dev),
            "w_hat": torch.empty(m, n, dtype=torch.float32, device=dev),
@@ -505,7 +542,8 @@ def run_mpq(args, world, rank, local):
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
                 "data": "synthetic", "config": cfgd,
-                "run": {"setup_s": None if setup_s is None else round(setup_s, 3), "rank": r,
+                "run": {"setup_s": None if setup_s is None else round(setup_s, 3),
+                        "gram": gram_run, "rank": r,
                         "cd_panel": args.cd_panel or "auto",
                         "parallelism": f"rows sharded over {world} GPU(s)"},
                 "rows_per_s": world * m / (ms_per_step / 1e3),

@@ -106,10 +106,11 @@ __device__ __forceinline__ void sc_ld32(uint32_t taddr, uint32_t (&v)[32]) {
 // bounded wait that gives up when another role has aborted
 __device__ __forceinline__ bool sc_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                         int* status) {
-  for (uint32_t i = 0; i < (1u << 25); ++i) {
+  for (uint32_t i = 0; i < WAIT_SPIN; ++i)
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 63) == 63 && *abort_flag) return false;
-    if (i > 256) __nanosleep(64);
+  for (uint32_t i = 0; i < WAIT_TRIES; ++i) {
+    if (mbar_try_wait_sleep(bar, parity, WAIT_SLICE_NS)) return true;
+    if (*abort_flag) return false;
   }
   atomicOr(status, STATUS_TIMEOUT);
   *abort_flag = 1;

@@ -128,7 +128,8 @@ struct DenoiseTcArgs {
   float* xhat;
   float* vblock;
   uint16_t* idx;
-  int nearest_only;
+  int mode;  // 0: both passes; 1: nearest codeword to r1 / s (pass 1, no prior); 2: the
+             // posterior's argmax only (pass 1 on the cavity / anchor mean): the marginal MAP
   int* status;
 };
 
@@ -185,10 +186,11 @@ __device__ __forceinline__ void named_sync_epi() {
 // Bounded wait that also gives up when another role has aborted.
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity,
                                               volatile int* abort_flag, int* status) {
-  for (uint32_t i = 0; i < (1u << 25); ++i) {
+  for (uint32_t i = 0; i < WAIT_SPIN; ++i)
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 63) == 63 && *abort_flag) return false;
-    if (i > 256) __nanosleep(64);
+  for (uint32_t i = 0; i < WAIT_TRIES; ++i) {
+    if (mbar_try_wait_sleep(bar, parity, WAIT_SLICE_NS)) return true;
+    if (*abort_flag) return false;
   }
   atomicOr(status, STATUS_TIMEOUT);
   *abort_flag = 1;
@@ -251,7 +253,7 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_denoise_vec_tc(DenoiseTcArgs 
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t mtiles = (a.nblocks + DT_M - 1) / DT_M;
-  const int passes = a.nearest_only ? 1 : 2;
+  const int passes = a.mode ? 1 : 2;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < DT_STAGES; ++s) {
@@ -264,10 +266,10 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_denoise_vec_tc(DenoiseTcArgs 
     }
     for (int b = 0; b < T2_BUFS; ++b) {
       mbar_init(&t2_full[b], 1);
-      mbar_init(&t2_empty[b], DT_EPI_WARPS);
+      mbar_init(&t2_empty[b], DT_EPI_WARPS / 2);  // the group of eight warps that owns it
     }
     for (int b = 0; b < QW_BUFS; ++b) {
-      mbar_init(&q_full[b], DT_EPI_WARPS);
+      mbar_init(&q_full[b], DT_EPI_WARPS / 2);
       mbar_init(&q_free[b], 1);
     }
     mbar_init(a_full, DT_M);
@@ -346,7 +348,7 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_denoise_vec_tc(DenoiseTcArgs 
           umma_commit(&t1_full[b]);
           umma_commit(&b_empty[s]);
         }
-        if (!ok || a.nearest_only) continue;
+        if (!ok || a.mode) continue;
         // ---------------------------------- pass 2: scores and moments
         // A polling scheduler: the score MMAs of a half go out as soon as its
         // TMEM buffer and codebook stage are ready, the moment MMAs of a half
@@ -416,7 +418,7 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_denoise_vec_tc(DenoiseTcArgs 
               *abort_flag = 1;
             }
             if ((idle & 63) == 63 && *abort_flag) break;
-            if (idle > 256) __nanosleep(32);
+            if (idle > 8) __nanosleep(32);
           }
         }
         if (um < total) {
@@ -444,7 +446,8 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_denoise_vec_tc(DenoiseTcArgs 
     const int rl = qd * 32 + lane;  // row of the tile this thread owns
     const uint32_t t_lane = tmem + ((uint32_t)(qd * 32) << 16);
     uint8_t* qw = smem + SM_QW;
-    const int w_off = kmaj_off(rl, wg * 16, 1024);  // this thread's 16 weights of a half
+    const int grp = wg >> 1, sub = wg & 1;  // pass 2: halves hq % 2 == grp, codewords 32 sub ..
+    const int w_off = kmaj_off(rl, sub * 32, 1024);  // this thread's 32 weights of a half
     uint32_t tu1 = 0, hq = 0, mt_n = 0;
     bool ok = true;
     const uint32_t nch = (uint32_t)((a.NT + MOM_CHUNK - 1) / MOM_CHUNK);  // chunks per tile
@@ -484,7 +487,7 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_denoise_vec_tc(DenoiseTcArgs 
           const float4 r1 = *reinterpret_cast<const float4*>(a.R1 + blk * 8 + 4);
           const float rv[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
           double gg = 1.0, ga = 0.0;
-          if (!a.nearest_only) {
+          if (a.mode != 1) {
             gg = a.gamma1[row] * sc2;
             ga = a.W ? a.inv_tau2 : 0.0;  // anchor: tau codebook units wide
           }
@@ -492,7 +495,7 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_denoise_vec_tc(DenoiseTcArgs 
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             double ti = (double)rv[i] / sc;
-            if (a.W && !a.nearest_only) ti = (gg * ti + ga * ((double)a.W[blk * 8 + i] / sc)) / (gg + ga);
+            if (a.W && a.mode != 1) ti = (gg * ti + ga * ((double)a.W[blk * 8 + i] / sc)) / (gg + ga);
             t64[i] = ti;
           }
         }
@@ -556,7 +559,7 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_denoise_vec_tc(DenoiseTcArgs 
           }
         }
       }
-      if (a.nearest_only) {
+      if (a.mode) {
         if (wg == 0 && active && ok) a.idx[blk] = (uint16_t)bidx;
         continue;
       }
@@ -624,25 +627,37 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_denoise_vec_tc(DenoiseTcArgs 
       uint64_t S2p = 0;  // (+0, +0): S2 over even and odd codewords
       const uint64_t rs2 = f2_pack(rs, rs), g22 = f2_pack(g2, g2), sh2 = f2_pack(Q_SHIFT, Q_SHIFT);
       uint32_t rd = 0;  // moment chunks read (warpgroup 0)
+      // The two halves of every codebook tile go to the two groups of eight
+      // warps (group g takes the halves with hq % 2 == g, so TMEM score
+      // buffer g and weights buffers g, g + 2): while one group turns its
+      // half's scores into weights the other waits for its MMAs or stores,
+      // so the exponentials of one overlap the latencies of the other.  A
+      // warp covers 32 of its half's 64 codewords, 16 at a time.
       for (int j = 0; j < a.NT; ++j) {
         // a chunk is read one codebook tile into the next chunk, by when its
         // moment MMAs have long been issued
         if (wg == 0 && j > MOM_CHUNK && (j - 1) % MOM_CHUNK == 0) read_chunk(rd++);
+        const uint32_t u = hq + 2u * (uint32_t)j + (uint32_t)grp;  // this group's half of tile j
+        const int buf = (int)(u % T2_BUFS), qb = (int)(u % QW_BUFS);
+        if (ok) ok = warp_wait(&t2_full[buf], (u / T2_BUFS) & 1, abort_flag, a.status);
+        // the moment MMAs of the weights buffer's previous use have read it
+        if (ok && u >= QW_BUFS) ok = warp_wait(&q_free[qb], (u / QW_BUFS - 1) & 1, abort_flag, a.status);
+        if (!ok) continue;
+        tc_fence_after();
+        uint8_t* wb = qw + qb * 2 * QW_BYTES + w_off;
 #pragma unroll 1
-        for (int h = 0; h < 2; ++h, ++hq) {
-          const int buf = hq % T2_BUFS, qb = hq % QW_BUFS;
-          if (ok) ok = warp_wait(&t2_full[buf], (hq / T2_BUFS) & 1, abort_flag, a.status);
-          if (!ok) continue;
-          tc_fence_after();
-          const uint32_t ta = t_lane + (uint32_t)buf * T2_COLS + (uint32_t)(wg * 16);
+        for (int k = 0; k < 2; ++k) {
+          const uint32_t ta = t_lane + (uint32_t)buf * T2_COLS + (uint32_t)(sub * 32 + k * 16);
           uint32_t Q[16], X[16], R[16];
           tmem_ld16_nowait(ta, Q);
           tmem_ld16_nowait(ta + 64u, X);
           tmem_ld16_nowait(ta + 128u, R);
           tmem_wait_ld();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&t2_empty[buf]);
+          if (k == 1) {  // the half's scores are read: hand the buffer back
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&t2_empty[buf]);
+          }
           // c* needs no special case here: X(c*) = 0 exactly, so it adds
           // nothing to S2, and its weight is zeroed in the moment operand
           // below.  (Its logit is 0 up to R's rounding, so z(c*) reaches the
@@ -670,24 +685,22 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_denoise_vec_tc(DenoiseTcArgs 
             f2_unpack(f2_sub(e, f2_pack(h.x, h.y)), d0, d1);
             asm("cvt.rn.satfinite.f16x2.f32 %0, %2, %1;" : "=r"(lo[p]) : "f"(d0), "f"(d1));
           }
-          // the moment MMAs of this buffer's previous use have read it
-          if (hq >= QW_BUFS) ok = warp_wait(&q_free[qb], (hq / QW_BUFS - 1) & 1, abort_flag, a.status);
-          if (!ok) continue;
-          uint8_t* wb = qw + qb * 2 * QW_BYTES + w_off;
-          *reinterpret_cast<uint4*>(wb) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-          *reinterpret_cast<uint4*>(wb + 128) = make_uint4(hi[4], hi[5], hi[6], hi[7]);
-          *reinterpret_cast<uint4*>(wb + QW_BYTES) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-          *reinterpret_cast<uint4*>(wb + QW_BYTES + 128) = make_uint4(lo[4], lo[5], lo[6], lo[7]);
-          if (j * 8 + h * 4 + wg == c16) {  // c* is in this chunk: weight 0 (added back at the end)
+          uint8_t* wk = wb + k * 256;  // codewords 16k .. 16k + 15 of this warp's 32
+          *reinterpret_cast<uint4*>(wk) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+          *reinterpret_cast<uint4*>(wk + 128) = make_uint4(hi[4], hi[5], hi[6], hi[7]);
+          *reinterpret_cast<uint4*>(wk + QW_BYTES) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+          *reinterpret_cast<uint4*>(wk + QW_BYTES + 128) = make_uint4(lo[4], lo[5], lo[6], lo[7]);
+          if (j * 8 + grp * 4 + sub * 2 + k == c16) {  // c*: weight 0 (added back at the end)
             const int o = (kst >> 3) * 128 + (kst & 7) * 2;
-            *reinterpret_cast<uint16_t*>(wb + o) = 0;
-            *reinterpret_cast<uint16_t*>(wb + QW_BYTES + o) = 0;
+            *reinterpret_cast<uint16_t*>(wk + o) = 0;
+            *reinterpret_cast<uint16_t*>(wk + QW_BYTES + o) = 0;
           }
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&q_full[qb]);
         }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&q_full[qb]);
       }
+      hq += 2u * (uint32_t)a.NT;
       {
         float s2a, s2b;
         f2_unpack(S2p, s2a, s2b);
@@ -825,7 +838,7 @@ mpq_status build_vec_tc_tables(mpq_plan_s* p, const float* cb_host) {
 mpq_status launch_denoise_vec_tc(const mpq_plan_s* p, const float* R1, const double* gamma1,
                                  const float* scale, const float* offset, int64_t m,
                                  const float* W, const double* gamma1_0, double inv_tau2,
-                                 float* xhat1, float* vblock, uint16_t* idx, int nearest_only,
+                                 float* xhat1, float* vblock, uint16_t* idx, int mode,
                                  cudaStream_t st) {
   static bool attr_set[64] = {};
   int dev = 0;
@@ -862,12 +875,13 @@ mpq_status launch_denoise_vec_tc(const mpq_plan_s* p, const float* R1, const dou
   a.xhat = xhat1;
   a.vblock = vblock;
   a.idx = idx;
-  a.nearest_only = nearest_only;
+  a.mode = mode;
   a.status = p->status;
   const int64_t mtiles = cdiv(a.nblocks, DT_M);
   const unsigned grid = (unsigned)std::min<int64_t>(mtiles, (int64_t)sms);
   {
-    ProfScope ps_(nearest_only ? "k_denoise_vec_tc(nearest)" : "k_denoise_vec_tc", st);
+    ProfScope ps_(mode == 1 ? "k_denoise_vec_tc(nearest)" : mode == 2 ? "k_denoise_vec_tc(map)" : "k_denoise_vec_tc",
+                  st);
     k_denoise_vec_tc<<<grid, DT_THREADS, DT_SMEM_BYTES, st>>>(a);
   }
   count_launch();

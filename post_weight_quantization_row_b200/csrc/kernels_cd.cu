@@ -30,9 +30,19 @@ namespace {
 // A operand of a tensor-core update  h += (-scale) Delta H[tile, :]  over all
 // columns, which also reproduces the in-tile updates for the next tile and
 // the next sweep.
-constexpr int CD1_WARPS = 16;
+//
+// Tiles go in groups of CD1_GROUP.  The gradient in memory is brought up to
+// date once per group (one GEMM with K = the group's width over the panel);
+// within a group, tile k starts from that gradient and first applies the
+// changes of the group's tiles before it to its own columns, in registers,
+// from their Delta rows and the blocks H[earlier tile, this tile] staged in
+// shared memory.
+constexpr int CD1_WARPS = 32;  // at most; the launch takes as many as spread the rows evenly
 constexpr int CD1_SLOTS = CD_TILE / 32;
-constexpr int CD1_SMEM = (CD_TILE * CD_TILE + CD_TILE) * 4;
+constexpr int CD1_GROUP = 3;   // (1 + earlier tiles) H blocks of 64 KiB fit in shared memory
+constexpr int CD1_BLOCK = CD_TILE * CD_TILE * 4;
+constexpr int CD1_SMEM = CD1_BLOCK + CD_TILE * 4;
+constexpr int CD1_SMEM_MAX = CD1_SMEM + (CD1_GROUP - 1) * CD1_BLOCK;
 
 // 4- and 16-byte asynchronous copies global -> shared; bytes past src_bytes
 // are filled with zeros
@@ -47,30 +57,33 @@ __device__ __forceinline__ void cp_async16(float* dst, const float* src, int src
                : "memory");
 }
 
-// H[t0.., t0..] (tw x tw) into a zero-padded CD_TILE x CD_TILE shared tile:
-// 16-byte copies when the rows of H are 16-byte aligned (n % 4 == 0; t0 is a
-// multiple of 128), else 4-byte copies
-__device__ __forceinline__ void load_h_tile(float* sH, const float* H, int64_t n, int64_t t0,
-                                            int tw) {
+// H[r0 .. r0+rw, c0 .. c0+cw] into a zero-padded CD_TILE x CD_TILE shared
+// block: 16-byte copies when the rows of H are 16-byte aligned (n % 4 == 0;
+// r0 and c0 are multiples of 128), else 4-byte copies.  The copies are
+// committed, not waited for.
+__device__ __forceinline__ void load_h_block(float* sH, const float* H, int64_t n, int64_t r0,
+                                             int rw, int64_t c0, int cw) {
   if ((n & 3) == 0) {
     constexpr int CH = CD_TILE / 4;  // 16-byte chunks per row
     for (int e = threadIdx.x; e < CD_TILE * CH; e += blockDim.x) {
       const int i = e / CH, j = 4 * (e % CH);
-      const int bytes = i < tw ? 4 * max(0, min(4, tw - j)) : 0;
-      cp_async16(sH + i * CD_TILE + j, bytes ? H + (t0 + i) * n + t0 + j : H, bytes);
+      const int bytes = i < rw ? 4 * max(0, min(4, cw - j)) : 0;
+      cp_async16(sH + i * CD_TILE + j, bytes ? H + (r0 + i) * n + c0 + j : H, bytes);
     }
   } else {
     for (int e = threadIdx.x; e < CD_TILE * CD_TILE; e += blockDim.x) {
       const int i = e / CD_TILE, j = e % CD_TILE;
-      const bool in = i < tw && j < tw;
-      cp_async4(sH + e, in ? H + (t0 + i) * n + t0 + j : H, in ? 4 : 0);
+      const bool in = i < rw && j < cw;
+      cp_async4(sH + e, in ? H + (r0 + i) * n + c0 + j : H, in ? 4 : 0);
     }
   }
-  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;\n" ::: "memory");
+  asm volatile("cp.async.commit_group;\n" ::: "memory");
 }
 
-__global__ void __launch_bounds__(CD1_WARPS * 32, 2)
-    k_cd_tile_decide(int64_t m, int64_t n, int L, int64_t t0, int tw,
+// gk: this tile's place in its group (the gk tiles before it, full width,
+// end at t0; their Delta rows end where this tile's begins)
+__global__ void __launch_bounds__(CD1_WARPS * 32, 1)
+    k_cd_tile_decide(int64_t m, int64_t n, int L, int64_t t0, int tw, int gk,
                      const float* __restrict__ scale, int ng, int gi,
                      const float* __restrict__ sref, const float* __restrict__ H,
                      uint16_t* __restrict__ idx, const float* __restrict__ h, int64_t ldh,
@@ -82,7 +95,12 @@ __global__ void __launch_bounds__(CD1_WARPS * 32, 2)
   extern __shared__ float cd_smem[];
   float* sH = cd_smem;                   // H[tile, tile], zero outside tw x tw
   float* s_rg = sH + CD_TILE * CD_TILE;  // 1 / H_jj (0 where H_jj <= 0)
-  load_h_tile(sH, H, n, t0, tw);
+  float* sHp = s_rg + CD_TILE;           // gk blocks H[earlier tile p, tile]
+  load_h_block(sH, H, n, t0, tw, t0, tw);
+  for (int p = 0; p < gk; ++p)
+    load_h_block(sHp + p * CD_TILE * CD_TILE, H, n, t0 - (int64_t)(gk - p) * CD_TILE, CD_TILE, t0,
+                 tw);
+  asm volatile("cp.async.wait_group 0;\n" ::: "memory");
   __syncthreads();
   bool pos = true;  // every diagonal entry of the tile positive
   for (int j = threadIdx.x; j < CD_TILE; j += blockDim.x) {
@@ -92,7 +110,7 @@ __global__ void __launch_bounds__(CD1_WARPS * 32, 2)
   }
   pos = __syncthreads_and(pos);
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  const int64_t row = (int64_t)blockIdx.x * CD1_WARPS + wid;
+  const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + wid;
   if (row >= m) return;
   __half* drow_hi = dhi + row * lda;
   __half* drow_lo = dlo + row * lda;
@@ -131,6 +149,30 @@ __global__ void __launch_bounds__(CD1_WARPS * 32, 2)
     kc[q] = in ? (float)ir[col] : 0.0f;
     a[q] = 0.5f * s2 * sH[col * CD_TILE + col];
     rq[q] = is2 * s_rg[col];
+  }
+  // the changes of the group's earlier tiles: h += du sum_j Delta_j H[j, .]
+  // (Delta_j = hi + lo as the update GEMM reads it, du = -scale, or -sref
+  // with group-wise grids), scaled like hs
+  if (gk > 0) {
+    const float f0 = sc * (sref ? -sref[row] : -sc);
+    for (int p = 0; p < gk; ++p) {
+      const __half* ph = drow_hi - (int64_t)(gk - p) * CD_TILE;
+      const __half* pl = drow_lo - (int64_t)(gk - p) * CD_TILE;
+      const float* Hp = sHp + p * CD_TILE * CD_TILE + lane;
+#pragma unroll
+      for (int q = 0; q < CD1_SLOTS; ++q) {
+        const float av = __half2float(ph[32 * q + lane]) + __half2float(pl[32 * q + lane]);
+        unsigned mk = __ballot_sync(0xffffffffu, av != 0.0f);
+        while (mk) {
+          const int l = __ffs(mk) - 1;
+          mk &= mk - 1u;
+          const float f = f0 * __shfl_sync(0xffffffffu, av, l);
+          const float* Hj = Hp + (32 * q + l) * CD_TILE;
+#pragma unroll
+          for (int qq = 0; qq < CD1_SLOTS; ++qq) hs[qq] = fmaf(Hj[32 * qq], f, hs[qq]);
+        }
+      }
+    }
   }
   auto sweep_tile = [&](auto all_pos) -> int {
     constexpr bool POS = decltype(all_pos)::value;
@@ -532,21 +574,35 @@ mpq_status launch_cd(mpq_plan_s* p, const float* W, int64_t m, const float* scal
   const int nchunks = p->d == 1 ? 0 : tc ? cd_scan_slices(m, p->K) : (int)cdiv(p->K, CD8_CHUNK);
   float* part_val = nullptr;
   int* part_idx = nullptr;
+  int dev = 0, sms = 148;
   if (p->d == 1) {
     MPQ_CUDA(cudaFuncSetAttribute(k_cd_tile_decide, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  CD1_SMEM));
+                                  CD1_SMEM_MAX));
+    MPQ_CUDA(cudaGetDevice(&dev));
+    MPQ_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
   } else {
     MPQ_CUDA(cudaMallocAsync(&part_val, sizeof(float) * m * nchunks, st));
     MPQ_CUDA(cudaMallocAsync(&part_idx, sizeof(int) * m * nchunks, st));
   }
   float* hl = w.Hl;  // d = 8: m x CD_TILE tile-local gradient
   mpq_status rc = MPQ_OK;
+  // Within a panel the tiles go in groups.  d = 1 (CD1_GROUP tiles): each
+  // tile applies the group's earlier changes to its own columns itself, and
+  // one GEMM with K = the group's width brings the panel's gradient up to
+  // date after the group.  d = 8 (CD_GROUP tiles): a tile's changes update
+  // the gradient of its own group's columns at once (the next tile reads
+  // them), and one GEMM after the group brings the rest of the panel up to
+  // date.  Either way a per-tile update moves at most m x (group width) of
+  // the gradient through L2 instead of the panel's slab.
+  const int64_t GW = (int64_t)(p->d == 1 ? CD1_GROUP : CD_GROUP) * CD_TILE;
   for (int sw = 0; sw < sweeps && rc == MPQ_OK; ++sw) {
     const bool last = sw == sweeps - 1;
     for (int pi = 0; pi < np && rc == MPQ_OK; ++pi) {
       const int64_t ps = (int64_t)pi * P, pe = std::min<int64_t>(n, ps + P);
       int* pflag = panel_flags + (int64_t)sw * np + pi;
-      for (int64_t t0 = ps; t0 < pe && rc == MPQ_OK; t0 += CD_TILE) {
+      for (int64_t g0 = ps; g0 < pe && rc == MPQ_OK; g0 += GW) {
+      const int64_t g1 = std::min<int64_t>(pe, g0 + GW);
+      for (int64_t t0 = g0; t0 < g1 && rc == MPQ_OK; t0 += CD_TILE) {
         const int j = (int)(t0 / CD_TILE);
         const int tw = (int)std::min<int64_t>(CD_TILE, n - t0);
         int* tflag = tile_flags + (int64_t)sw * nt + j;
@@ -554,9 +610,15 @@ mpq_status launch_cd(mpq_plan_s* p, const float* W, int64_t m, const float* scal
         __half* dhi = w.As.hi + (t0 - ps);
         __half* dlo = w.As.lo + (t0 - ps);
         if (p->d == 1) {
+          // rows per CTA such that one wave holds all rows with the fewest on
+          // the busiest SM: two CTAs fit an SM with one H block, one with more
+          const int gk = (int)((t0 - g0) / CD_TILE);
+          const int per_sm = gk == 0 ? 2 : 1;
+          const int warps = (int)std::min<int64_t>(
+              CD1_WARPS / per_sm, std::max<int64_t>(4, cdiv(m, (int64_t)per_sm * sms)));
           ProfScope ps_("k_cd_tile_decide", st);
-          k_cd_tile_decide<<<(unsigned)cdiv(m, CD1_WARPS), CD1_WARPS * 32, CD1_SMEM, st>>>(
-              m, n, p->K, t0, tw, scale, (int)p->ng, p->G ? (int)(t0 / p->G) : 0,
+          k_cd_tile_decide<<<(unsigned)cdiv(m, warps), warps * 32, CD1_SMEM + gk * CD1_BLOCK, st>>>(
+              m, n, p->K, t0, tw, gk, scale, (int)p->ng, p->G ? (int)(t0 / p->G) : 0,
               p->G ? w.sref : nullptr, p->H32, idx, h, ldh, sweeps, sw, changes, dhi, dlo,
               w.As.ld, w.As.row_unscale, tflag, pflag, skip);
           count_launch();
@@ -587,9 +649,22 @@ mpq_status launch_cd(mpq_plan_s* p, const float* W, int64_t m, const float* scal
           }
         }
         if (rc != MPQ_OK) break;
-        // the panel's columns; in the last sweep only the ones still to be
-        // visited (the gradient is not read after it)
-        rc = update(t0 - ps, t0, tw, last ? t0 + tw : ps, pe, tflag, "gemm_cd_update");
+        // d = 8: the group's columns; in the last sweep only the ones still
+        // to be visited (the gradient is not read after it)
+        if (p->d != 1) rc = update(t0 - ps, t0, tw, last ? t0 + tw : g0, g1, tflag, "gemm_cd_update");
+      }
+      // the group's changes reach the rest of the panel (d = 1: the whole
+      // panel, the group's own columns too), gated on any change in the panel
+      // so far, which covers this group's; in the last sweep only the columns
+      // after the group
+      if (rc == MPQ_OK && p->d == 1 && !last) {
+        rc = update(g0 - ps, g0, g1 - g0, ps, pe, pflag, "gemm_cd_group");
+      } else {
+        if (rc == MPQ_OK && !last && g0 > ps)
+          rc = update(g0 - ps, g0, g1 - g0, ps, g0, pflag, "gemm_cd_group");
+        if (rc == MPQ_OK && g1 < pe)
+          rc = update(g0 - ps, g0, g1 - g0, g1, pe, pflag, "gemm_cd_group");
+      }
       }
       if (rc != MPQ_OK || np == 1) continue;
       if (!last) rc = update(0, ps, pe - ps, 0, ps, pflag, "gemm_cd_panel");  // columns before

@@ -97,6 +97,23 @@ __device__ __forceinline__ int split_exponent(float amax) {
   return (amax > 0.0f) ? ex - 14 : 0;
 }
 
+// the same split for four adjacent elements (o a multiple of 4), two packed
+// conversions and one 8-byte store per half
+__device__ __forceinline__ void split_store4(const float (&x)[4], __half* __restrict__ hi,
+                                             __half* __restrict__ lo, int64_t o) {
+  const __half2 h0 = __floats2half2_rn(x[0], x[1]), h1 = __floats2half2_rn(x[2], x[3]);
+  const float2 f0 = __half22float2(h0), f1 = __half22float2(h1);
+  const __half2 l0 = __floats2half2_rn(x[0] - f0.x, x[1] - f0.y);
+  const __half2 l1 = __floats2half2_rn(x[2] - f1.x, x[3] - f1.y);
+  uint2 hv, lv;
+  hv.x = *reinterpret_cast<const uint32_t*>(&h0);
+  hv.y = *reinterpret_cast<const uint32_t*>(&h1);
+  lv.x = *reinterpret_cast<const uint32_t*>(&l0);
+  lv.y = *reinterpret_cast<const uint32_t*>(&l1);
+  *reinterpret_cast<uint2*>(hi + o) = hv;
+  *reinterpret_cast<uint2*>(lo + o) = lv;
+}
+
 __device__ __forceinline__ void split_store(float xs, __half* __restrict__ hi,
                                             __half* __restrict__ lo, int64_t o) {
   const __half h = __float2half_rn(xs);
@@ -264,6 +281,7 @@ struct ScalarDen {
   float sc, off, inv_sc, Lm1, sc2f, A2;
   float hwf, kmax0;  // window half-width and last window start, as floats
   double doff, inv_dsc, g, ga, geff;
+  double cr, cw, coff;  // anchored centre in level units: cr r + cw w - coff
   int L, hw, nlev;
   bool anchored, precise;
 };
@@ -283,6 +301,11 @@ __device__ __forceinline__ ScalarDen scalar_den_row(float sc, float off, double 
   c.anchored = anchored;
   c.ga = anchored ? fmin(inv_tau2, 1e30) : 0.0;
   c.geff = c.g + c.ga;
+  // (g (r - off) + ga (w - off)) / (scale geff), with the division and the
+  // offset folded into row constants ((g + ga) / geff = 1)
+  c.cr = c.g * c.inv_dsc / c.geff;
+  c.cw = c.ga * c.inv_dsc / c.geff;
+  c.coff = c.doff * c.inv_dsc;
   c.A2 = (float)(-0.5 * c.geff * 1.4426950408889634);  // -geff/2 log2(e)
   c.L = L;
   // Levels far from the nearest one carry no weight: with |dt| <= 1/2 (or dt
@@ -340,7 +363,7 @@ __device__ __forceinline__ float scalar_den_elem(const ScalarDen& c, const float
     }
   } else {
     // anchored prior: the effective centre mixes r and w (fp64, rare path)
-    const double tt = (c.g * ((double)r - c.doff) + c.ga * ((double)wr - c.doff)) * c.inv_dsc / c.geff;
+    const double tt = fma(c.cr, (double)r, fma(c.cw, (double)wr, -c.coff));
     const double kd = fmin(fmax(ceil(tt - 0.5), 0.0), (double)(c.L - 1));
     ks = (float)kd;
     const double dtd = tt - kd;
@@ -824,14 +847,16 @@ __global__ void __launch_bounds__(FUSED_MAX_THREADS)
                       float* __restrict__ a_unscale, double* __restrict__ gamma2,
                       int32_t* __restrict__ clamps, uint16_t* __restrict__ idx,
                       float* __restrict__ R1o) {
-  extern __shared__ float vrow[];  // r1 (then r2) and x_hat1 of the row
+  extern __shared__ __align__(16) float vrow[];  // the row: r1 (then r2), x_hat1 (then w - r2), w
   __shared__ double ds[33];
   __shared__ float fs[33];
   __shared__ float cf_s;
   const int nn = (int)n;  // a row fits in shared memory: 32-bit in-row indices
+  const int np4 = (nn + 3) & ~3;
   float* s_r = vrow;
-  float* s_x = vrow + nn;
-  ScalarDen* s_den = reinterpret_cast<ScalarDen*>(vrow + 2 * nn);  // GROUPED: one per group
+  float* s_x = vrow + np4;
+  float* s_w = vrow + 2 * np4;
+  ScalarDen* s_den = reinterpret_cast<ScalarDen*>(vrow + 3 * np4);  // GROUPED: one per group
   const int64_t row = blockIdx.x;
   const float* Wr = W + row * n;
   const float* Gr = G + row * n;
@@ -850,18 +875,22 @@ __global__ void __launch_bounds__(FUSED_MAX_THREADS)
   const bool injected = first == 2;
   float* R1or = R1o ? R1o + row * n : nullptr;
   const int bs = blockDim.x;
-  // whole batches of ROW_UNROLL weights per thread (loads first, no bounds
-  // checks), then the tail one weight at a time
-  const int full = nn / (ROW_UNROLL * bs) * (ROW_UNROLL * bs);
+  // Rows of a multiple of 4 weights move as float4 (rows start 16-byte
+  // aligned then): each thread takes VQ groups of 4 consecutive weights, their
+  // loads in flight together.  Other rows go one weight at a time.
+  constexpr int VQ = 1;  // more spills registers at the 64 a 1024-thread launch allows
+  const bool vec = (nn & 3) == 0;
+  const int nq = nn >> 2;
   auto pass1 = [&](auto prec, auto anch) -> float {
     constexpr bool PRECISE = decltype(prec)::value;
     constexpr bool ANCH = decltype(anch)::value;
     float acc = 0.0f;
-    auto one = [&](const int j, const float g, const float r2, const float w) {
-      const float r1 = injected ? g
-                       : first  ? w
-                       : full_rank ? fmaf(lc, g, fmaf(lk, w - r2, w))
-                                   : fmaf(lc, g, r2);
+    // weight j: r1 from the l2d step, then the denoiser; x_hat1 returned
+    auto one = [&](const int j, const float g, const float r2, const float w, float& r1) -> float {
+      r1 = injected ? g
+           : first  ? w
+           : full_rank ? fmaf(lc, g, fmaf(lk, w - r2, w))
+                       : fmaf(lc, g, r2);
       if (R1or) R1or[j] = r1;
       float xh, ks, v;
       if constexpr (GROUPED) {
@@ -871,28 +900,53 @@ __global__ void __launch_bounds__(FUSED_MAX_THREADS)
       } else {
         v = scalar_den_elem<PRECISE, ANCH>(c, r1, w, xh, ks);
       }
-      if (MAP) {
-        idx[row * n + j] = (uint16_t)(int)ks;
-      } else {
-        s_r[j] = r1;
-        s_x[j] = xh;
-        acc += v;
-      }
+      if (MAP) idx[row * n + j] = (uint16_t)(int)ks;
+      acc += v;
+      return xh;
     };
-    for (int j0 = threadIdx.x; j0 < full; j0 += ROW_UNROLL * bs) {
-      float gv[ROW_UNROLL], r2v[ROW_UNROLL], wv[ROW_UNROLL];
+    if (vec) {
+      const float4* G4 = reinterpret_cast<const float4*>(Gr);
+      const float4* R4 = reinterpret_cast<const float4*>(R2r);
+      const float4* W4 = reinterpret_cast<const float4*>(Wr);
+      for (int q0 = threadIdx.x; q0 < nq; q0 += VQ * bs) {
+        float4 gv[VQ], rv[VQ], wv[VQ];
 #pragma unroll
-      for (int u = 0; u < ROW_UNROLL; ++u) {
-        const int j = j0 + u * bs;
-        gv[u] = (first == 1) ? 0.0f : Gr[j];
-        r2v[u] = first ? 0.0f : R2r[j];
-        wv[u] = Wr[j];
+        for (int u = 0; u < VQ; ++u) {
+          const int q = q0 + u * bs;
+          const bool in = q < nq;
+          const float4 z = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+          gv[u] = (in && first != 1) ? G4[q] : z;
+          rv[u] = (in && !first) ? R4[q] : z;
+          wv[u] = in ? W4[q] : z;
+        }
+#pragma unroll
+        for (int u = 0; u < VQ; ++u) {
+          const int q = q0 + u * bs;
+          if (q >= nq) continue;
+          float4 r1, xh;
+          xh.x = one(4 * q, gv[u].x, rv[u].x, wv[u].x, r1.x);
+          xh.y = one(4 * q + 1, gv[u].y, rv[u].y, wv[u].y, r1.y);
+          xh.z = one(4 * q + 2, gv[u].z, rv[u].z, wv[u].z, r1.z);
+          xh.w = one(4 * q + 3, gv[u].w, rv[u].w, wv[u].w, r1.w);
+          if (!MAP) {
+            reinterpret_cast<float4*>(s_r)[q] = r1;
+            reinterpret_cast<float4*>(s_x)[q] = xh;
+            reinterpret_cast<float4*>(s_w)[q] = wv[u];
+          }
+        }
       }
-#pragma unroll
-      for (int u = 0; u < ROW_UNROLL; ++u) one(j0 + u * bs, gv[u], r2v[u], wv[u]);
+    } else {
+      for (int j = threadIdx.x; j < nn; j += bs) {
+        const float w = Wr[j];
+        float r1;
+        const float xh = one(j, (first == 1) ? 0.0f : Gr[j], first ? 0.0f : R2r[j], w, r1);
+        if (!MAP) {
+          s_r[j] = r1;
+          s_x[j] = xh;
+          s_w[j] = w;
+        }
+      }
     }
-    for (int j = full + threadIdx.x; j < nn; j += bs)
-      one(j, (first == 1) ? 0.0f : Gr[j], first ? 0.0f : R2r[j], Wr[j]);
     return acc;
   };
   using T_ = std::true_type;
@@ -901,43 +955,64 @@ __global__ void __launch_bounds__(FUSED_MAX_THREADS)
   const float acc = anchored ? (pr ? pass1(T_{}, T_{}) : pass1(F_{}, T_{}))
                              : (pr ? pass1(T_{}, F_{}) : pass1(F_{}, F_{}));
   if (MAP) return;
-  const double vsum = block_sum((double)acc, ds);  // its barriers also publish s_r, s_x
+  const double vsum = block_sum((double)acc, ds);  // its barriers also publish the row
   if (threadIdx.x == 0)
     cf_s = d2l_row(gamma1[row], vsum, n, gamma1_0[row], glo, ghi, amin, amax, gamma2 + row,
                    clamps ? clamps + row : nullptr);
   __syncthreads();
   const float cf = cf_s;
+  // r2 = r1 + cf (x_hat1 - r1) out, and w - r2 kept (in s_x) for the split
   float mx = 0.0f;
-  auto two = [&](const int j, const float w) {
-    const float r1 = s_r[j];
-    const float r2 = fmaf(cf, s_x[j] - r1, r1);
-    R2r[j] = r2;
-    s_r[j] = r2;
-    mx = fmaxf(mx, fabsf(w - r2));
-  };
-  for (int j0 = threadIdx.x; j0 < full; j0 += ROW_UNROLL * bs) {
-    float wv[ROW_UNROLL];
-#pragma unroll
-    for (int u = 0; u < ROW_UNROLL; ++u) wv[u] = Wr[j0 + u * bs];
-#pragma unroll
-    for (int u = 0; u < ROW_UNROLL; ++u) two(j0 + u * bs, wv[u]);
+  if (vec) {
+    for (int q = threadIdx.x; q < nq; q += bs) {
+      const float4 r1 = reinterpret_cast<const float4*>(s_r)[q];
+      const float4 xh = reinterpret_cast<const float4*>(s_x)[q];
+      const float4 w = reinterpret_cast<const float4*>(s_w)[q];
+      float4 r2, d;
+      r2.x = fmaf(cf, xh.x - r1.x, r1.x);
+      r2.y = fmaf(cf, xh.y - r1.y, r1.y);
+      r2.z = fmaf(cf, xh.z - r1.z, r1.z);
+      r2.w = fmaf(cf, xh.w - r1.w, r1.w);
+      reinterpret_cast<float4*>(R2r)[q] = r2;
+      d.x = w.x - r2.x;
+      d.y = w.y - r2.y;
+      d.z = w.z - r2.z;
+      d.w = w.w - r2.w;
+      reinterpret_cast<float4*>(s_x)[q] = d;
+      mx = fmaxf(mx, fmaxf(fmaxf(fabsf(d.x), fabsf(d.y)), fmaxf(fabsf(d.z), fabsf(d.w))));
+    }
+  } else {
+    for (int j = threadIdx.x; j < nn; j += bs) {
+      const float r1 = s_r[j];
+      const float r2 = fmaf(cf, s_x[j] - r1, r1);
+      R2r[j] = r2;
+      const float d = s_w[j] - r2;
+      s_x[j] = d;
+      mx = fmaxf(mx, fabsf(d));
+    }
   }
-  for (int j = full + threadIdx.x; j < nn; j += bs) two(j, Wr[j]);
-  mx = block_reduce(mx, MaxF(), fs);  // its barriers also publish the new s_r
+  mx = block_reduce(mx, MaxF(), fs);  // its barriers also publish w - r2
   const int ex = split_exponent(mx);
   const float down = ldexpf(1.0f, -ex);
   __half* ahr = ahi + row * lda;
   __half* alr = alo + row * lda;
-  const int ldnn = (int)ldn;
-  for (int j0 = threadIdx.x; j0 < full; j0 += ROW_UNROLL * bs) {
-    float xv[ROW_UNROLL];
+  const int ldnn = (int)ldn;  // a multiple of 64 (and lda even): whole quads, 8-byte aligned
+  for (int q = threadIdx.x; q < ldnn / 4; q += bs) {
+    const int j = 4 * q;
+    float x[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    if (vec && j < nn) {
+      const float4 d = reinterpret_cast<const float4*>(s_x)[q];
+      x[0] = d.x * down;
+      x[1] = d.y * down;
+      x[2] = d.z * down;
+      x[3] = d.w * down;
+    } else if (!vec) {
 #pragma unroll
-    for (int u = 0; u < ROW_UNROLL; ++u) xv[u] = (Wr[j0 + u * bs] - s_r[j0 + u * bs]) * down;
-#pragma unroll
-    for (int u = 0; u < ROW_UNROLL; ++u) split_store(xv[u], ahr, alr, j0 + u * bs);
+      for (int e = 0; e < 4; ++e)
+        if (j + e < nn) x[e] = s_x[j + e] * down;
+    }
+    split_store4(x, ahr, alr, j);
   }
-  for (int j = full + threadIdx.x; j < ldnn; j += bs)
-    split_store(j < nn ? (Wr[j] - s_r[j]) * down : 0.0f, ahr, alr, j);
   if (threadIdx.x == 0) a_unscale[row] = ldexpf(1.0f, ex);
 }
 
@@ -1098,7 +1173,7 @@ mpq_status launch_init(const mpq_plan_s* p, const float* W, int64_t m, int given
 mpq_status launch_denoise(const mpq_plan_s* p, const float* R1, const double* gamma1,
                           const float* scale, const float* offset, int64_t m, const float* W,
                           const double* gamma1_0, float* xhat1, float* vblock, double* vsum,
-                          uint16_t* idx, cudaStream_t st) {
+                          uint16_t* idx, cudaStream_t st, bool map_only) {
   if (m <= 0) return MPQ_OK;
   const bool anchored = std::isfinite(p->params.tau);
   const double inv_tau2 = anchored ? 1.0 / (p->params.tau * p->params.tau) : 0.0;
@@ -1124,7 +1199,9 @@ mpq_status launch_denoise(const mpq_plan_s* p, const float* R1, const double* ga
   if (vblock == nullptr) return fail(MPQ_ERR_INVALID_ARG, "vector denoiser needs vblock");
   if (p->vec_tc) {
     MPQ_TRY(launch_denoise_vec_tc(p, R1, gamma1, scale, offset, m, anchored ? W : nullptr,
-                                  gamma1_0, inv_tau2, xhat1, vblock, idx, 0, st));
+                                  gamma1_0, inv_tau2, xhat1, vblock, idx,
+                                  map_only && idx ? 2 : 0, st));
+    if (map_only && idx) return MPQ_OK;  // no x_hat, no variance sums
   } else {
   VecDenoiseArgs a{};
   a.R1 = R1;
@@ -1210,8 +1287,12 @@ mpq_status launch_extrinsic_l2d(const mpq_plan_s* p, const float* W, int64_t m, 
 // Threads per row of the fused scalar kernel: its shared memory holds two
 // floats per weight; 0 when the row does not fit (the separate kernels run).
 // (plus the per-group denoiser constants with group-wise grids)
+int64_t vamp_row_smem(int64_t n, int G) {
+  return 12 * ((n + 3) / 4 * 4) + (G ? (n / G) * (int64_t)sizeof(ScalarDen) : 0);
+}
+
 int vamp_row_threads(int64_t n, int G) {
-  const int64_t bytes = 8 * n + (G ? (n / G) * (int64_t)sizeof(ScalarDen) : 0);
+  const int64_t bytes = vamp_row_smem(n, G);
   if (bytes <= 56 * 1024) return 256;    // 4 CTAs per SM
   if (bytes <= 112 * 1024) return 512;   // 2 CTAs per SM
   if (bytes <= 220 * 1024) return 1024;  // 1 CTA per SM
@@ -1230,8 +1311,7 @@ mpq_status launch_vamp_row_scalar(const mpq_plan_s* p, const float* W, int64_t m
   const mpq_params& q = p->params;
   const bool anchored = std::isfinite(q.tau);
   const double inv_tau2 = anchored ? 1.0 / (q.tau * q.tau) : 0.0;
-  const size_t smem =
-      sizeof(float) * 2 * p->n + (p->G ? sizeof(ScalarDen) * (size_t)(p->n / p->G) : 0);
+  const size_t smem = (size_t)vamp_row_smem(p->n, p->G);
   using Kern = void (*)(const float*, const float*, float*, int64_t, int, int, int, const double*,
                         const double*, const double*, const float*, const float*, int, int,
                         const double*, double, double, double, double, double, __half*, __half*,

@@ -446,10 +446,10 @@ mpq_status solve_batch(mpq_plan_s* p, const SolveIO& io, int64_t row0, int64_t m
                          w.gamma1, w.R2, w.gamma2, nullptr, nullptr, nullptr, nullptr, clamps, st));
       R1 = w.R1;
     }
-    // marginal MAP: argmax of one more denoiser call
+    // marginal MAP: argmax of one more denoiser call (only the index is used)
     if (io.T_vamp > 0)
       MPQ_TRY(launch_denoise(p, R1, w.gamma1, w.scale, w.offset, mb, W, w.gamma1_0, w.X1, vblock,
-                             w.vsum, idx, st));
+                             w.vsum, idx, st, /*map_only=*/true));
   }
   // the greedy baseline replaces round-to-nearest as the hard init
   if (io.T_vamp == 0 && p->params.greedy_init)

@@ -185,7 +185,9 @@ mpq_status launch_init(const mpq_plan_s* p, const float* W, int64_t m, int given
 mpq_status launch_denoise(const mpq_plan_s* p, const float* R1, const double* gamma1,
                           const float* scale, const float* offset, int64_t m, const float* W,
                           const double* gamma1_0, float* xhat1, float* vblock, double* vsum,
-                          uint16_t* idx, cudaStream_t st);
+                          uint16_t* idx, cudaStream_t st, bool map_only = false);
+// (map_only: only idx, the posterior's argmax, is wanted; the tensor-core
+// vector denoiser then skips its second pass and writes nothing else)
 // writes r2 and the A operand w - r2 (split, K = n)
 mpq_status launch_extrinsic_d2l(const mpq_plan_s* p, const float* W, int64_t m, const float* R1,
                                 const double* gamma1, const float* xhat1, const double* vsum,
@@ -238,6 +240,7 @@ __device__ __forceinline__ float ceil_small(float y) {
 }
 
 constexpr int CD_TILE = 128;  // columns per scalar CD tile (multiple of 64)
+constexpr int CD_GROUP = 4;   // CD tiles per group of eager gradient updates
 constexpr int64_t CD_PANEL_BYTES = 32ll << 20;  // L2-resident slab of the CD gradient
 constexpr int64_t CD_PANEL_MIN = 512;           // narrowest CD panel (columns)
 int64_t cd_panel_cols(int64_t m, int64_t n);
@@ -305,8 +308,8 @@ mpq_status build_vec_tc_tables(mpq_plan_s* p, const float* cb_host);
 mpq_status launch_denoise_vec_tc(const mpq_plan_s* p, const float* R1, const double* gamma1,
                                  const float* scale, const float* offset, int64_t m,
                                  const float* W, const double* gamma1_0, double inv_tau2,
-                                 float* xhat1, float* vblock, uint16_t* idx, int nearest_only,
-                                 cudaStream_t st);
+                                 float* xhat1, float* vblock, uint16_t* idx, int mode,
+                                 cudaStream_t st);  // mode: 0 full, 1 nearest, 2 MAP index only
 
 // tensor-core candidate scan of the vector CD step (cd_scan_tc.cu)
 int cd_scan_slices(int64_t m, int K);

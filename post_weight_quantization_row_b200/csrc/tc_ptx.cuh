@@ -48,12 +48,42 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait (>= about a second of polling); false on timeout.
+// Test of a phase that suspends the thread until the phase completes or
+// about `ns` nanoseconds pass: a waiting warp issues nothing meanwhile, so
+// it takes no issue slots from the warps that compute.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_try_wait_sleep_cl(uint64_t* bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+
+// Waits are bounded: WAIT_SPIN plain tests (a short wait resumes fastest
+// that way), then WAIT_TRIES suspended tests of up to WAIT_SLICE_NS each
+// (about two seconds in all); false on timeout.
+constexpr uint32_t WAIT_SPIN = 64, WAIT_SLICE_NS = 20000, WAIT_TRIES = 100000;
+
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  for (uint32_t i = 0; i < (1u << 25); ++i) {
+  for (uint32_t i = 0; i < WAIT_SPIN; ++i)
     if (mbar_try_wait(bar, parity)) return true;
-    if (i > 256) __nanosleep(64);
-  }
+  for (uint32_t i = 0; i < WAIT_TRIES; ++i)
+    if (mbar_try_wait_sleep(bar, parity, WAIT_SLICE_NS)) return true;
   return false;
 }
 
@@ -200,18 +230,10 @@ __device__ __forceinline__ void mbar_arrive_cl(uint32_t cl_addr) {
 // Bounded wait with cluster-scope acquire (arrivals and copies from the peer
 // CTA); false on timeout.
 __device__ __forceinline__ bool mbar_wait_cl(uint64_t* bar, uint32_t parity) {
-  for (uint32_t i = 0; i < (1u << 25); ++i) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    if (ok) return true;
-    if (i > 256) __nanosleep(64);
-  }
+  for (uint32_t i = 0; i < WAIT_SPIN; ++i)
+    if (mbar_try_wait_sleep_cl(bar, parity, 0)) return true;
+  for (uint32_t i = 0; i < WAIT_TRIES; ++i)
+    if (mbar_try_wait_sleep_cl(bar, parity, WAIT_SLICE_NS)) return true;
   return false;
 }
 // Tiled TMA load into this CTA's shared memory whose completion is signalled

@@ -301,7 +301,8 @@ def test_stage_cd_vector(mpq):
     assert ref.changes[:, 0].sum() > 0
 
 
-@pytest.mark.parametrize("kind", ["scalar", "scalar_300_rows", "e8_tensor", "gaussian_simt"])
+@pytest.mark.parametrize("kind", ["scalar", "scalar_300_rows", "scalar_one_panel", "e8_tensor",
+                                  "gaussian_simt"])
 def test_stage_cd_panels(mpq, kind):
     # cd_panel = 256 over n = 600: panels of 256, 256 and 88 columns, the
     # last one ragged (tiles 128, 128 | 128, 128 | 88); every change reaches
@@ -317,8 +318,11 @@ def test_stage_cd_panels(mpq, kind):
               else np.random.default_rng(13).standard_normal((256, 8)).astype(np.float32))
         p = mi.small_problem(132, 40, 600, 900, d=8, levels=cb.shape[0], codebook=cb)
         off_rms = True
+    # one_panel: a single panel of 640 columns whose tiles go in groups of
+    # four: the first group's changes reach columns 512..599 through the
+    # group GEMM (K = 512), the second's reach columns 0..511 (K = 88)
     s, V, s_cu, V_cu = spectrum_cuda(p.X)
-    plan = make_plan(mpq, p, s_cu, V_cu, cd_panel=256)
+    plan = make_plan(mpq, p, s_cu, V_cu, cd_panel=0 if kind.endswith("panel") else 256)
     if off_rms:
         sc = orc.rms_scale(p.W)[0].astype(np.float32)
         off = np.zeros_like(sc)
