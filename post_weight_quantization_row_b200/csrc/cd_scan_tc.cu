@@ -295,10 +295,14 @@ __global__ void __launch_bounds__(SC_THREADS, 1) k_cd_vec_scan(ScanArgs a) {
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&b_empty[s]);  // qtab of this stage is read
-      float m0 = fmin3(sv[0], sv[1], sv[2]);
+      // minimum of the 32 scores as a tree of three-input minima (depth 4)
+      float t1[11];
 #pragma unroll
-      for (int c = 3; c < 31; c += 2) m0 = fmin3(m0, sv[c], sv[c + 1]);
-      m0 = fminf(m0, sv[31]);
+      for (int c = 0; c < 10; ++c) t1[c] = fmin3(sv[3 * c], sv[3 * c + 1], sv[3 * c + 2]);
+      t1[10] = fminf(sv[30], sv[31]);
+      const float m0 = fminf(fmin3(fmin3(t1[0], t1[1], t1[2]), fmin3(t1[3], t1[4], t1[5]),
+                                   fmin3(t1[6], t1[7], t1[8])),
+                             fminf(t1[9], t1[10]));
       if (m0 < best) {  // first index of the chunk minimum
         int kk = 31;
 #pragma unroll

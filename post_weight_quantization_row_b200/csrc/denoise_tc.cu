@@ -531,10 +531,15 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_denoise_vec_tc(DenoiseTcArgs 
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&t1_empty[buf]);
-        float m0 = fmax3(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]));
+        // maximum of the 32 scores as a tree of three-input maxima (depth 4)
+        float t1[11];
 #pragma unroll
-        for (int k = 3; k < 31; k += 2) m0 = fmax3(m0, __uint_as_float(v[k]), __uint_as_float(v[k + 1]));
-        m0 = fmaxf(m0, __uint_as_float(v[31]));
+        for (int k = 0; k < 10; ++k)
+          t1[k] = fmax3(__uint_as_float(v[3 * k]), __uint_as_float(v[3 * k + 1]), __uint_as_float(v[3 * k + 2]));
+        t1[10] = fmaxf(__uint_as_float(v[30]), __uint_as_float(v[31]));
+        const float m0 = fmaxf(fmax3(fmax3(t1[0], t1[1], t1[2]), fmax3(t1[3], t1[4], t1[5]),
+                                     fmax3(t1[6], t1[7], t1[8])),
+                               fmaxf(t1[9], t1[10]));
         if (m0 > best) {  // first index of the chunk maximum
           int kk = 31;
 #pragma unroll

@@ -100,6 +100,17 @@ __global__ void __launch_bounds__(CD1_WARPS * 32, 1)
   for (int p = 0; p < gk; ++p)
     load_h_block(sHp + p * CD_TILE * CD_TILE, H, n, t0 - (int64_t)(gk - p) * CD_TILE, CD_TILE, t0,
                  tw);
+  // the row's gradient and levels in the tile travel while the H blocks do
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + wid;
+  float h_in[CD1_SLOTS], k_in[CD1_SLOTS];
+#pragma unroll
+  for (int q = 0; q < CD1_SLOTS; ++q) {
+    const int col = 32 * q + lane;
+    const bool in = row < m && col < tw;
+    h_in[q] = in ? h[row * ldh + t0 + col] : 0.0f;
+    k_in[q] = in ? (float)idx[row * n + t0 + col] : 0.0f;
+  }
   asm volatile("cp.async.wait_group 0;\n" ::: "memory");
   __syncthreads();
   bool pos = true;  // every diagonal entry of the tile positive
@@ -109,8 +120,6 @@ __global__ void __launch_bounds__(CD1_WARPS * 32, 1)
     if (j < tw && !(gj > 0.0f)) pos = false;
   }
   pos = __syncthreads_and(pos);
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + wid;
   if (row >= m) return;
   __half* drow_hi = dhi + row * lda;
   __half* drow_lo = dlo + row * lda;
@@ -139,14 +148,12 @@ __global__ void __launch_bounds__(CD1_WARPS * 32, 1)
   // which changes the choice only between levels whose energies tie to
   // rounding.  With H_jj <= 0 the candidates are the grid ends.
   const float s2 = sc * sc, is2 = 1.0f / s2, Lm1 = (float)(L - 1);
-  const float* hr = h + row * ldh + t0;
   float hs[CD1_SLOTS], kc[CD1_SLOTS], a[CD1_SLOTS], rq[CD1_SLOTS];
 #pragma unroll
   for (int q = 0; q < CD1_SLOTS; ++q) {
     const int col = 32 * q + lane;
-    const bool in = col < tw;
-    hs[q] = in ? sc * hr[col] : 0.0f;
-    kc[q] = in ? (float)ir[col] : 0.0f;
+    hs[q] = sc * h_in[q];
+    kc[q] = k_in[q];
     a[q] = 0.5f * s2 * sH[col * CD_TILE + col];
     rq[q] = is2 * s_rg[col];
   }
@@ -227,7 +234,7 @@ __global__ void __launch_bounds__(CD1_WARPS * 32, 1)
     float dk = 0.0f;
     if (col < tw) {
       const int knew = (int)kc[q];
-      dk = (float)(knew - (int)ir[col]);
+      dk = (float)(knew - (int)k_in[q]);
       ir[col] = (uint16_t)knew;
     }
     const float dv = dk * dsc;  // exact when dsc = 1
@@ -610,12 +617,11 @@ mpq_status launch_cd(mpq_plan_s* p, const float* W, int64_t m, const float* scal
         __half* dhi = w.As.hi + (t0 - ps);
         __half* dlo = w.As.lo + (t0 - ps);
         if (p->d == 1) {
-          // rows per CTA such that one wave holds all rows with the fewest on
-          // the busiest SM: two CTAs fit an SM with one H block, one with more
+          // one CTA per SM, with rows per CTA such that one wave holds all
+          // rows with the fewest on the busiest SM (every CTA stages the same
+          // H blocks from L2, so fewer CTAs move fewer bytes)
           const int gk = (int)((t0 - g0) / CD_TILE);
-          const int per_sm = gk == 0 ? 2 : 1;
-          const int warps = (int)std::min<int64_t>(
-              CD1_WARPS / per_sm, std::max<int64_t>(4, cdiv(m, (int64_t)per_sm * sms)));
+          const int warps = (int)std::min<int64_t>(CD1_WARPS, std::max<int64_t>(4, cdiv(m, sms)));
           ProfScope ps_("k_cd_tile_decide", st);
           k_cd_tile_decide<<<(unsigned)cdiv(m, warps), warps * 32, CD1_SMEM + gk * CD1_BLOCK, st>>>(
               m, n, p->K, t0, tw, gk, scale, (int)p->ng, p->G ? (int)(t0 / p->G) : 0,
