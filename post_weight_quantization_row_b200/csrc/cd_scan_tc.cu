@@ -9,7 +9,7 @@
 // tensor cores: A = -2^k g' as an fp16 hi/lo pair (k per row, so that the low
 // half stays clear of subnormals) against the plan's codebook operand
 // [c | |c|^2 pair, 1, 1] (the extra columns meet zeros), two MMAs
-// (M = 128 rows, N = 128 codewords, K = 16) per tile into TMEM; the epilogue
+// (M = 128 rows, N = 256 codewords, K = 16) per tile into TMEM; the epilogue
 // forms score = qtab + 2^-k D in fp32 and keeps the first minimum.
 //
 // The same scan serves the greedy baseline (LDLQ with E8 rounding): the
@@ -19,10 +19,10 @@
 //
 // Grid: (slices of the codebook) x (tiles of 128 rows); every CTA writes the
 // minimum of its slice per row, and the apply step combines the slices.
-// Warps 0-15 read TMEM (warp w: lanes 32 (w % 4) .. +31, columns 32 (w / 4)
-// .. +31 of each tile), warp 16 owns TMEM and issues the MMAs, warp 17 issues
-// the bulk copies of the codebook operand and the qtab row through a 20-stage
-// ring; TMEM holds 4 score buffers.  All waits are bounded.
+// Warps 0-15 read TMEM (warp w: lanes 32 (w % 4) .. +31, columns 64 (w / 4)
+// .. +63 of each 256-codeword tile), warp 16 owns TMEM and issues the MMAs,
+// warp 17 issues the bulk copies of the codebook operand and the qtab row
+// through a 10-stage ring; TMEM holds 2 score buffers.  All waits are bounded.
 #include <cuda.h>
 #include <cuda_fp16.h>
 
@@ -36,16 +36,18 @@ namespace mpq {
 namespace {
 using namespace tcx;
 
-// The ring runs 20 codebook tiles (4.5 KiB each) ahead of the MMAs: an
-// epilogue pass over a tile takes a few hundred cycles, so fewer stages would
-// leave the scan waiting on the latency of the copies from L2.
-constexpr int SC_M = 128, SC_N = 128, SC_STAGES = 20, SC_BUFS = 4;
+// A scan tile is 256 codewords (two of the plan's 128-codeword operand
+// images, copied side by side): one MMA pair of N = 256 per tile, so that the
+// fixed cost of issuing an MMA and of each pipeline handshake is spread over
+// twice the codewords (two TMEM buffers of 256 columns).  The ring holds 10
+// tiles of 9 KiB.
+constexpr int SC_M = 128, SC_N = 256, SC_TN = SC_N / 128, SC_STAGES = 10, SC_BUFS = 2;
 constexpr int SC_EPI_WARPS = 16, SC_WGS = 4;
 constexpr int SC_THREADS = (SC_EPI_WARPS + 2) * 32;
 constexpr int SC_MMA_WARP = SC_EPI_WARPS, SC_LOAD_WARP = SC_EPI_WARPS + 1;
 constexpr int SC_OPER = 128 * 32;           // 128 rows x 16 fp16
 constexpr int SC_QT = SC_N * 4;             // qtab of one tile (fp32)
-constexpr int SC_STAGE = SC_OPER + SC_QT;
+constexpr int SC_STAGE = SC_TN * SC_OPER + SC_QT;
 constexpr int SC_IMG_STRIDE = 8192;         // bytes per tile in the plan's operand images
 constexpr uint32_t SC_TMEM_COLS = 512;
 constexpr uint32_t SC_IDESC = idesc_f16(SC_M, SC_N);
@@ -60,7 +62,7 @@ static_assert(SC_END + 1024 <= SC_SMEM, "scan shared memory");
 
 struct ScanArgs {
   int64_t m, n;
-  int K, NT;              // codewords, tiles of 128
+  int K, NT;              // codewords, scan tiles of SC_N (the last one may be partial)
   int64_t b, t0;          // block, first column of its CD tile
   const uint8_t* cb_tc;   // NT x 8 KiB operand images (the first 4 KiB: scores)
   const float* cb;        // K x 8
@@ -170,9 +172,15 @@ __global__ void __launch_bounds__(SC_THREADS, 1) k_cd_vec_scan(ScanArgs a) {
         if (t >= SC_STAGES && !sc_wait(&b_empty[s], (t / SC_STAGES - 1) & 1, abort_flag, a.status))
           break;
         uint8_t* st = smem + SC_B + s * SC_STAGE;
-        mbar_expect_tx(&b_full[s], SC_STAGE);
-        bulk_load_1d(st, a.cb_tc + (size_t)(j0 + t) * SC_IMG_STRIDE, SC_OPER, &b_full[s]);
-        bulk_load_1d(st + SC_OPER, a.qtab_row + (int64_t)(j0 + t) * SC_N, SC_QT, &b_full[s]);
+        // the tile's 128-codeword images present (a partial last tile has
+        // fewer; the MMA's columns past them are never read back)
+        const int nimg = min(SC_TN, (a.K - (j0 + t) * SC_N) / 128);
+        mbar_expect_tx(&b_full[s], (uint32_t)(nimg * (SC_OPER + 128 * 4)));
+        for (int i = 0; i < nimg; ++i)
+          bulk_load_1d(st + i * SC_OPER, a.cb_tc + (size_t)((j0 + t) * SC_TN + i) * SC_IMG_STRIDE,
+                       SC_OPER, &b_full[s]);
+        bulk_load_1d(st + SC_TN * SC_OPER, a.qtab_row + (int64_t)(j0 + t) * SC_N,
+                     (uint32_t)(nimg * 128 * 4), &b_full[s]);
       }
       for (int q = (t > SC_STAGES ? t - SC_STAGES : 0); q < t; ++q)  // copies land before exit
         for (uint32_t i = 0; i < (1u << 25) && !mbar_try_wait(&b_full[q % SC_STAGES], (q / SC_STAGES) & 1); ++i)
@@ -275,42 +283,56 @@ __global__ void __launch_bounds__(SC_THREADS, 1) k_cd_vec_scan(ScanArgs a) {
       if (ok) ok = __all_sync(0xffffffffu, sc_wait(&t_full[buf], (t / SC_BUFS) & 1, abort_flag, a.status));
       if (!ok) continue;
       tc_fence_after();
-      uint32_t v[32];
-      sc_ld32(tmem + ((uint32_t)(qd * 32) << 16) + (uint32_t)buf * SC_N + (uint32_t)(wg * 32), v);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&t_empty[buf]);
-      const float4* q4 = reinterpret_cast<const float4*>(smem + SC_B + s * SC_STAGE + SC_OPER) + wg * 8;
-      // score = D rsc + qtab, two codewords per packed f32x2 fma
-      float sv[32];
+      const int nvalid = min(SC_N, a.K - (j0 + t) * SC_N);  // codewords in this tile
+#pragma unroll 1
+      for (int hh = 0; hh < 2; ++hh) {  // this warp's 64 columns, 32 at a time
+        const int cbase = wg * 64 + hh * 32;
+        uint32_t v[32];
+        sc_ld32(tmem + ((uint32_t)(qd * 32) << 16) + (uint32_t)buf * SC_N + (uint32_t)cbase, v);
+        if (hh == 1) {  // the tile's scores are read: hand the buffer back
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&t_empty[buf]);
+        }
+        const float4* q4 = reinterpret_cast<const float4*>(smem + SC_B + s * SC_STAGE + SC_TN * SC_OPER) +
+                           cbase / 4;
+        // score = D rsc + qtab, two codewords per packed f32x2 fma; columns
+        // past the codebook's end (a partial last tile) score +inf
+        float sv[32];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const float4 q = q4[c];
-        f2_unpack(f2_fma(f2_pack(__uint_as_float(v[4 * c]), __uint_as_float(v[4 * c + 1])), rsc2,
-                         f2_pack(q.x, q.y)),
-                  sv[4 * c], sv[4 * c + 1]);
-        f2_unpack(f2_fma(f2_pack(__uint_as_float(v[4 * c + 2]), __uint_as_float(v[4 * c + 3])), rsc2,
-                         f2_pack(q.z, q.w)),
-                  sv[4 * c + 2], sv[4 * c + 3]);
+        for (int c = 0; c < 8; ++c) {
+          const float4 q = q4[c];
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(v[4 * c]), __uint_as_float(v[4 * c + 1])), rsc2,
+                           f2_pack(q.x, q.y)),
+                    sv[4 * c], sv[4 * c + 1]);
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(v[4 * c + 2]), __uint_as_float(v[4 * c + 3])), rsc2,
+                           f2_pack(q.z, q.w)),
+                    sv[4 * c + 2], sv[4 * c + 3]);
+        }
+        if (cbase + 32 > nvalid) {
+#pragma unroll
+          for (int c = 0; c < 32; ++c)
+            if (cbase + c >= nvalid) sv[c] = INFINITY;
+        }
+        // minimum of the 32 scores as a tree of three-input minima (depth 4)
+        float t1[11];
+#pragma unroll
+        for (int c = 0; c < 10; ++c) t1[c] = fmin3(sv[3 * c], sv[3 * c + 1], sv[3 * c + 2]);
+        t1[10] = fminf(sv[30], sv[31]);
+        const float m0 = fminf(fmin3(fmin3(t1[0], t1[1], t1[2]), fmin3(t1[3], t1[4], t1[5]),
+                                     fmin3(t1[6], t1[7], t1[8])),
+                               fminf(t1[9], t1[10]));
+        if (m0 < best) {  // first index of the chunk minimum
+          int kk = 31;
+#pragma unroll
+          for (int c = 31; c >= 0; --c)
+            if (sv[c] == m0) kk = c;
+          best = m0;
+          bidx = (j0 + t) * SC_N + cbase + kk;
+        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&b_empty[s]);  // qtab of this stage is read
-      // minimum of the 32 scores as a tree of three-input minima (depth 4)
-      float t1[11];
-#pragma unroll
-      for (int c = 0; c < 10; ++c) t1[c] = fmin3(sv[3 * c], sv[3 * c + 1], sv[3 * c + 2]);
-      t1[10] = fminf(sv[30], sv[31]);
-      const float m0 = fminf(fmin3(fmin3(t1[0], t1[1], t1[2]), fmin3(t1[3], t1[4], t1[5]),
-                                   fmin3(t1[6], t1[7], t1[8])),
-                             fminf(t1[9], t1[10]));
-      if (m0 < best) {  // first index of the chunk minimum
-        int kk = 31;
-#pragma unroll
-        for (int c = 31; c >= 0; --c)
-          if (sv[c] == m0) kk = c;
-        best = m0;
-        bidx = (j0 + t) * SC_N + wg * 32 + kk;
-      }
     }
     sm_bval[wg * SC_M + rl] = best;
     sm_bidx[wg * SC_M + rl] = bidx;
@@ -342,7 +364,7 @@ __global__ void __launch_bounds__(SC_THREADS, 1) k_cd_vec_scan(ScanArgs a) {
 
 int cd_scan_slices(int64_t m, int K) {
   const int64_t mtiles = cdiv(m, SC_M);
-  return (int)std::max<int64_t>(1, std::min<int64_t>(K / SC_N, 148 / std::max<int64_t>(mtiles, 1)));
+  return (int)std::max<int64_t>(1, std::min<int64_t>((K + SC_N - 1) / SC_N, 148 / std::max<int64_t>(mtiles, 1)));
 }
 
 mpq_status launch_cd_vec_scan(const mpq_plan_s* p, int64_t m, int64_t b, int64_t t0,
@@ -360,7 +382,7 @@ mpq_status launch_cd_vec_scan(const mpq_plan_s* p, int64_t m, int64_t b, int64_t
   a.m = m;
   a.n = p->n;
   a.K = p->K;
-  a.NT = p->K / SC_N;
+  a.NT = (p->K + SC_N - 1) / SC_N;
   a.b = b;
   a.t0 = t0;
   a.cb_tc = reinterpret_cast<const uint8_t*>(p->cb_tc);
@@ -400,7 +422,7 @@ mpq_status launch_ldlq_vec_scan(const mpq_plan_s* p, int64_t m, int64_t b, const
   a.m = m;
   a.n = p->n;
   a.K = p->K;
-  a.NT = p->K / SC_N;
+  a.NT = (p->K + SC_N - 1) / SC_N;
   a.b = b;
   a.t0 = 8 * b;
   a.cb_tc = reinterpret_cast<const uint8_t*>(p->cb_tc);

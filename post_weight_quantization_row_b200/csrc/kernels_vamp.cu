@@ -282,6 +282,7 @@ struct ScalarDen {
   float hwf, kmax0;  // window half-width and last window start, as floats
   double doff, inv_dsc, g, ga, geff;
   double cr, cw, coff;  // anchored centre in level units: cr r + cw w - coff
+  float crh, crl, cwh, cwl, cofh, cofl;  // the same as fp32 pairs (hi + lo)
   int L, hw, nlev;
   bool anchored, precise;
 };
@@ -306,6 +307,12 @@ __device__ __forceinline__ ScalarDen scalar_den_row(float sc, float off, double 
   c.cr = c.g * c.inv_dsc / c.geff;
   c.cw = c.ga * c.inv_dsc / c.geff;
   c.coff = c.doff * c.inv_dsc;
+  c.crh = (float)c.cr;
+  c.crl = (float)(c.cr - (double)c.crh);
+  c.cwh = (float)c.cw;
+  c.cwl = (float)(c.cw - (double)c.cwh);
+  c.cofh = (float)c.coff;
+  c.cofl = (float)(c.coff - (double)c.cofh);
   c.A2 = (float)(-0.5 * c.geff * 1.4426950408889634);  // -geff/2 log2(e)
   c.L = L;
   // Levels far from the nearest one carry no weight: with |dt| <= 1/2 (or dt
@@ -332,7 +339,11 @@ __device__ __forceinline__ ScalarDen scalar_den_row(float sc, float off, double 
 // One weight: cavity r (and w for the anchored prior) -> posterior mean xh,
 // variance (returned) and the most likely level ks (an integer as a float).
 // Instantiated per precision regime and prior, both uniform over a row.
-template <bool PRECISE, bool ANCH>
+// PAIR_CENTRE (anchored rows): form the centre as an fp32 pair instead of in
+// fp64; the nearest level ks is then decided from the pair's rounded sum, so
+// it may differ from the exact rounding by one level at an exact half, which
+// only moves the window's centre (use it where ks is not an output).
+template <bool PRECISE, bool ANCH, bool PAIR_CENTRE = false>
 __device__ __forceinline__ float scalar_den_elem(const ScalarDen& c, const float r, const float wr,
                                                  float& xh, float& ks) {
   const float sc = c.sc, off = c.off, inv_sc = c.inv_sc, A2 = c.A2;
@@ -361,8 +372,26 @@ __device__ __forceinline__ float scalar_den_elem(const ScalarDen& c, const float
       dh = __fmul_rn(__fsub_rn(d0, __fadd_rn(pe, se)), inv_sc);
       dl = 0.0f;
     }
+  } else if constexpr (PAIR_CENTRE) {
+    // anchored prior, centre cr r + cw w - coff as an fp32 pair: error-free
+    // products (TwoProduct by fma) and sums (TwoSum), the small terms of the
+    // constants' low halves added in plain fp32; the explicitly rounded
+    // intrinsics keep the compiler from contracting or reassociating
+    const float ph = __fmul_rn(c.crh, r), pe = fmaf(c.crh, r, -ph);
+    const float qh = __fmul_rn(c.cwh, wr), qe = fmaf(c.cwh, wr, -qh);
+    const float s1 = __fadd_rn(ph, qh), b1 = __fsub_rn(s1, ph);
+    const float e1 = __fadd_rn(__fsub_rn(ph, __fsub_rn(s1, b1)), __fsub_rn(qh, b1));
+    const float s2 = __fsub_rn(s1, c.cofh), b2 = __fsub_rn(s2, s1);
+    const float e2 = __fadd_rn(__fsub_rn(s1, __fsub_rn(s2, b2)), __fsub_rn(-c.cofh, b2));
+    const float lo = __fadd_rn(__fadd_rn(__fadd_rn(pe, qe), __fadd_rn(e1, e2)),
+                               __fsub_rn(fmaf(c.crl, r, __fmul_rn(c.cwl, wr)), c.cofl));
+    ks = fminf(fmaxf(ceil_small(__fadd_rn(s2, lo) - 0.5f), 0.0f), c.Lm1);
+    const float d0 = __fsub_rn(s2, ks);  // exact: s2 lies within a level or so of ks
+    dh = __fadd_rn(d0, lo);
+    const float bd = __fsub_rn(dh, d0);
+    dl = __fadd_rn(__fsub_rn(d0, __fsub_rn(dh, bd)), __fsub_rn(lo, bd));
   } else {
-    // anchored prior: the effective centre mixes r and w (fp64, rare path)
+    // anchored prior: the effective centre mixes r and w (fp64)
     const double tt = fma(c.cr, (double)r, fma(c.cw, (double)wr, -c.coff));
     const double kd = fmin(fmax(ceil(tt - 0.5), 0.0), (double)(c.L - 1));
     ks = (float)kd;
@@ -895,10 +924,10 @@ __global__ void __launch_bounds__(FUSED_MAX_THREADS)
       float xh, ks, v;
       if constexpr (GROUPED) {
         const ScalarDen& cg = s_den[j / gsize];  // uniform over a warp (gsize % 32 == 0)
-        v = cg.precise ? scalar_den_elem<true, ANCH>(cg, r1, w, xh, ks)
-                       : scalar_den_elem<false, ANCH>(cg, r1, w, xh, ks);
+        v = cg.precise ? scalar_den_elem<true, ANCH, !MAP>(cg, r1, w, xh, ks)
+                       : scalar_den_elem<false, ANCH, !MAP>(cg, r1, w, xh, ks);
       } else {
-        v = scalar_den_elem<PRECISE, ANCH>(c, r1, w, xh, ks);
+        v = scalar_den_elem<PRECISE, ANCH, !MAP>(c, r1, w, xh, ks);
       }
       if (MAP) idx[row * n + j] = (uint16_t)(int)ks;
       acc += v;

@@ -288,9 +288,10 @@ def test_stage_cd_scalar(mpq):
     assert ref.changes[:, 0].sum() > 0
 
 
-def test_stage_cd_vector(mpq):
-    cb = mi.e8_codebook_cached()[:512]
-    p = mi.small_problem(404, 12, 80, 200, d=8, levels=512, codebook=cb)
+@pytest.mark.parametrize("K", [512, 384])  # 384: the scan's last 256-codeword tile is half full
+def test_stage_cd_vector(mpq, K):
+    cb = mi.e8_codebook_cached()[:K]
+    p = mi.small_problem(404, 12, 80, 200, d=8, levels=K, codebook=cb)
     s, V, s_cu, V_cu = spectrum_cuda(p.X)
     plan = make_plan(mpq, p, s_cu, V_cu)
     rho, _ = orc.rms_scale(p.W)
