@@ -48,7 +48,9 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="mpq", choices=["mpq", "reference"])
     ap.add_argument("--config", default="q4096")
-    ap.add_argument("--cpu-rows", type=int, default=8, help="oracle sample size (rows)")
+    ap.add_argument("--cpu-rows", type=int, default=0,
+                    help="oracle sample size in rows (0: 8 for scalar grids, 1 for the 65536-word "
+                         "E8 codebook, whose oracle denoiser enumerates every codeword per block)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--rows", type=int, default=0,
@@ -558,6 +560,9 @@ def run_mpq(args, world, rank, local):
 
 def main():
     args = parse()
+    if args.cpu_rows <= 0:
+        import mpq_inputs as mi
+        args.cpu_rows = 1 if mi.WORKLOADS[args.config][4] == 8 else 8
     world, rank, local = dist_init(args.gpus)
     try:
         if args.impl == "reference":

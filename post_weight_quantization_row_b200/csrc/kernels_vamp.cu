@@ -766,24 +766,16 @@ __global__ void __launch_bounds__(ROW_THREADS)
 // (1 - rho) beta + rho beta_hat (R7), gamma1' = gamma2 (1 - alpha2)/alpha2
 // and the l2d coefficients 1/(1 - alpha2), alpha2/(1 - alpha2), each clipped
 // (R5), and the second GEMM's row scale 2^(e_row + e_bound).
-__global__ void __launch_bounds__(256)
-    k_linear_finish(const float2* __restrict__ part, int ntiles, int64_t m, int64_t n, int64_t r,
-                    int e_bound, const float* __restrict__ a_unscale,
-                    float* __restrict__ q_unscale, const double* __restrict__ gamma2,
-                    const double* __restrict__ gamma1_0, double* __restrict__ beta,
-                    double damping, double glo, double ghi, double amin, double amax,
-                    double* __restrict__ gamma1_out, double* __restrict__ coef,
-                    double* __restrict__ kappa, double* __restrict__ alpha2_out,
-                    double* __restrict__ beta_hat_out, int32_t* __restrict__ clamps) {
-  // one warp per row: lane l adds the column groups l, l + 32, ... in fp64,
-  // then a butterfly over the lanes (a fixed order: the sums are
-  // deterministic); lane 0 finishes the row
-  const int lane = threadIdx.x & 31;
-  const int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  if (row >= m) return;
+// The M-step's per-row finish (one warp per row): lane l adds the column
+// groups l, l + 32, ... in fp64, then a butterfly over the lanes (a fixed
+// order: the sums are deterministic); lane 0 forms alpha2, beta_hat, the
+// damped beta, gamma1' and the l2d coefficients.  Shared by the finisher
+// kernel and the fused row kernel that runs it in its prologue.
+
+__device__ __forceinline__ void linear_finish_row(const LinFinish& f, int64_t row, int lane) {
   double a2tot = 0.0, bstot = 0.0;
-  for (int t = lane; t < ntiles; t += 32) {
-    const float2 v = part[(int64_t)t * m + row];
+  for (int t = lane; t < f.ntiles; t += 32) {
+    const float2 v = f.part[(int64_t)t * f.m + row];
     a2tot += (double)v.x;
     bstot += (double)v.y;
   }
@@ -793,20 +785,27 @@ __global__ void __launch_bounds__(256)
     bstot += __shfl_xor_sync(0xffffffffu, bstot, o);
   }
   if (lane != 0) return;
-  q_unscale[row] = ldexpf(a_unscale[row], e_bound);
+  if (f.q_unscale) f.q_unscale[row] = ldexpf(f.a_unscale[row], f.e_bound);
   int cnt = 0;
-  const double b = beta[row], g2 = gamma2[row];
-  const double alpha2 = (a2tot + (double)(n - r)) / (double)n;
-  const double bhat = (double)r / bstot;
-  beta[row] = (1.0 - damping) * b + damping * bhat;
-  const double a2 = clip_count(alpha2, amin, amax, &cnt);
-  const double g0 = gamma1_0[row];
-  gamma1_out[row] = clip_count(g2 * (1.0 - a2) / a2, glo * g0, ghi * g0, &cnt);
-  coef[row] = 1.0 / (1.0 - a2);
-  kappa[row] = a2 / (1.0 - a2);
-  if (alpha2_out) alpha2_out[row] = alpha2;
-  if (beta_hat_out) beta_hat_out[row] = bhat;
-  if (clamps) clamps[row] += cnt;
+  const double b = f.beta[row], g2 = f.gamma2[row];
+  const double alpha2 = (a2tot + (double)(f.n - f.r)) / (double)f.n;
+  const double bhat = (double)f.r / bstot;
+  f.beta[row] = (1.0 - f.damping) * b + f.damping * bhat;
+  const double a2 = clip_count(alpha2, f.amin, f.amax, &cnt);
+  const double g0 = f.gamma1_0[row];
+  f.gamma1_out[row] = clip_count(g2 * (1.0 - a2) / a2, f.glo * g0, f.ghi * g0, &cnt);
+  f.coef[row] = 1.0 / (1.0 - a2);
+  f.kappa[row] = a2 / (1.0 - a2);
+  if (f.alpha2_out) f.alpha2_out[row] = alpha2;
+  if (f.beta_hat_out) f.beta_hat_out[row] = bhat;
+  if (f.clamps) f.clamps[row] += cnt;
+}
+
+__global__ void __launch_bounds__(256) k_linear_finish(const __grid_constant__ LinFinish f) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (row >= f.m) return;
+  linear_finish_row(f, row, lane);
 }
 
 // ------------------------------------------------- extrinsic linear -> d ---
@@ -867,15 +866,15 @@ template <int MAP, bool GROUPED>
 __global__ void __launch_bounds__(FUSED_MAX_THREADS)
     k_vamp_row_scalar(const float* __restrict__ W, const float* __restrict__ G,
                       float* __restrict__ R2, int64_t n, int gsize, int first, int full_rank,
-                      const double* __restrict__ coef, const double* __restrict__ kappa,
-                      const double* __restrict__ gamma1, const float* __restrict__ scale,
+                      const double* coef, const double* kappa,
+                      const double* gamma1, const float* __restrict__ scale,
                       const float* __restrict__ offset, int L, int anchored,
                       const double* __restrict__ gamma1_0, double inv_tau2, double glo,
                       double ghi, double amin, double amax, __half* __restrict__ ahi,
                       __half* __restrict__ alo, int64_t lda, int64_t ldn,
-                      float* __restrict__ a_unscale, double* __restrict__ gamma2,
-                      int32_t* __restrict__ clamps, uint16_t* __restrict__ idx,
-                      float* __restrict__ R1o) {
+                      float* __restrict__ a_unscale, double* gamma2,
+                      int32_t* clamps, uint16_t* __restrict__ idx,
+                      float* __restrict__ R1o, const __grid_constant__ LinFinish fin, int has_fin) {
   extern __shared__ __align__(16) float vrow[];  // the row: r1 (then r2), x_hat1 (then w - r2), w
   __shared__ double ds[33];
   __shared__ float fs[33];
@@ -890,17 +889,25 @@ __global__ void __launch_bounds__(FUSED_MAX_THREADS)
   const float* Wr = W + row * n;
   const float* Gr = G + row * n;
   float* R2r = R2 + row * n;
+  // gamma1, coef and kappa may be written by this kernel's own prologue (the
+  // previous linear step's M-step finish for this row): no __restrict__ on
+  // them, and the reads go through L2 (ld.global.cg) after the barrier
+  if (has_fin) {
+    if (threadIdx.x < 32) linear_finish_row(fin, row, threadIdx.x);
+    __syncthreads();
+  }
+  const double g1row = __ldcg(gamma1 + row);
   const int ng = GROUPED ? nn / gsize : 1;
-  const ScalarDen c = scalar_den_row(scale[row * ng], offset[row * ng], gamma1[row], L,
+  const ScalarDen c = scalar_den_row(scale[row * ng], offset[row * ng], g1row, L,
                                      anchored != 0, inv_tau2);
   if (GROUPED) {
     for (int g = threadIdx.x; g < ng; g += blockDim.x)
-      s_den[g] = scalar_den_row(scale[row * ng + g], offset[row * ng + g], gamma1[row], L,
+      s_den[g] = scalar_den_row(scale[row * ng + g], offset[row * ng + g], g1row, L,
                                 anchored != 0, inv_tau2);
     __syncthreads();
   }
-  const float lc = first ? 0.0f : (float)coef[row];
-  const float lk = first ? 0.0f : (float)kappa[row];
+  const float lc = first ? 0.0f : (float)__ldcg(coef + row);
+  const float lk = first ? 0.0f : (float)__ldcg(kappa + row);
   const bool injected = first == 2;
   float* R1or = R1o ? R1o + row * n : nullptr;
   const int bs = blockDim.x;
@@ -986,7 +993,7 @@ __global__ void __launch_bounds__(FUSED_MAX_THREADS)
   if (MAP) return;
   const double vsum = block_sum((double)acc, ds);  // its barriers also publish the row
   if (threadIdx.x == 0)
-    cf_s = d2l_row(gamma1[row], vsum, n, gamma1_0[row], glo, ghi, amin, amax, gamma2 + row,
+    cf_s = d2l_row(g1row, vsum, n, gamma1_0[row], glo, ghi, amin, amax, gamma2 + row,
                    clamps ? clamps + row : nullptr);
   __syncthreads();
   const float cf = cf_s;
@@ -1282,19 +1289,50 @@ mpq_status launch_extrinsic_d2l(const mpq_plan_s* p, const float* W, int64_t m, 
   return check_launch("k_extrinsic_d2l");
 }
 
+LinFinish make_lin_finish(const mpq_plan_s* p, int64_t m, const float2* part, int ntiles,
+                          int e_bound, const float* a_unscale, float* q_unscale,
+                          const double* gamma2, const double* gamma1_0, double* beta,
+                          double* gamma1_out, double* coef, double* kappa, double* alpha2,
+                          double* beta_hat, int32_t* clamps) {
+  const mpq_params& q = p->params;
+  LinFinish f;
+  f.part = part;
+  f.ntiles = ntiles;
+  f.e_bound = e_bound;
+  f.m = m;
+  f.n = p->n;
+  f.r = p->r;
+  f.a_unscale = a_unscale;
+  f.q_unscale = q_unscale;
+  f.gamma2 = gamma2;
+  f.gamma1_0 = gamma1_0;
+  f.beta = beta;
+  f.damping = q.damping;
+  f.glo = q.gamma_lo_rel;
+  f.ghi = q.gamma_hi_rel;
+  f.amin = q.alpha_min;
+  f.amax = q.alpha_max;
+  f.gamma1_out = gamma1_out;
+  f.coef = coef;
+  f.kappa = kappa;
+  f.alpha2_out = alpha2;
+  f.beta_hat_out = beta_hat;
+  f.clamps = clamps;
+  return f;
+}
+
 mpq_status launch_linear_finish(const mpq_plan_s* p, int64_t m, const float2* part, int ntiles,
                                 int e_bound, const float* a_unscale, float* q_unscale,
                                 const double* gamma2, const double* gamma1_0, double* beta,
                                 double* gamma1_out, double* coef, double* kappa, double* alpha2,
                                 double* beta_hat, int32_t* clamps, cudaStream_t st) {
   if (m <= 0) return MPQ_OK;
-  const mpq_params& q = p->params;
+  const LinFinish f = make_lin_finish(p, m, part, ntiles, e_bound, a_unscale, q_unscale, gamma2,
+                                      gamma1_0, beta, gamma1_out, coef, kappa, alpha2, beta_hat,
+                                      clamps);
   {
     ProfScope ps_("k_linear_finish", st);
-    k_linear_finish<<<(unsigned)cdiv(m * 32, 256), 256, 0, st>>>(
-        part, ntiles, m, p->n, p->r, e_bound, a_unscale, q_unscale, gamma2, gamma1_0, beta,
-        q.damping, q.gamma_lo_rel, q.gamma_hi_rel, q.alpha_min, q.alpha_max, gamma1_out, coef,
-        kappa, alpha2, beta_hat, clamps);
+    k_linear_finish<<<(unsigned)cdiv(m * 32, 256), 256, 0, st>>>(f);
   }
   count_launch();
   return check_launch("k_linear_finish");
@@ -1333,7 +1371,7 @@ mpq_status launch_vamp_row_scalar(const mpq_plan_s* p, const float* W, int64_t m
                                   const double* kappa, const double* gamma1, const float* scale,
                                   const float* offset, const double* gamma1_0, SplitOperand* As,
                                   double* gamma2, int32_t* clamps, uint16_t* idx, cudaStream_t st,
-                                  float* R1o) {
+                                  float* R1o, const LinFinish* fin) {
   if (m <= 0) return MPQ_OK;
   const int threads = vamp_row_threads(p->n, p->G);
   if (p->d != 1 || threads == 0) return fail(MPQ_ERR_INVALID_ARG, "fused row kernel: d = 1 rows that fit");
@@ -1344,7 +1382,8 @@ mpq_status launch_vamp_row_scalar(const mpq_plan_s* p, const float* W, int64_t m
   using Kern = void (*)(const float*, const float*, float*, int64_t, int, int, int, const double*,
                         const double*, const double*, const float*, const float*, int, int,
                         const double*, double, double, double, double, double, __half*, __half*,
-                        int64_t, int64_t, float*, double*, int32_t*, uint16_t*, float*);
+                        int64_t, int64_t, float*, double*, int32_t*, uint16_t*, float*,
+                        const LinFinish, int);
   const Kern kern = p->G ? (map ? k_vamp_row_scalar<1, true> : k_vamp_row_scalar<0, true>)
                          : (map ? k_vamp_row_scalar<1, false> : k_vamp_row_scalar<0, false>);
   MPQ_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
@@ -1354,7 +1393,7 @@ mpq_status launch_vamp_row_scalar(const mpq_plan_s* p, const float* W, int64_t m
         W, G, R2, p->n, p->G, first, p->r == p->n ? 1 : 0, coef, kappa, gamma1, scale, offset, p->K,
         anchored ? 1 : 0, gamma1_0, inv_tau2, q.gamma_lo_rel, q.gamma_hi_rel, q.alpha_min,
         q.alpha_max, As ? As->hi : nullptr, As ? As->lo : nullptr, As ? As->ld : 0,
-        round_up(p->n, 64), As ? As->row_unscale : nullptr, gamma2, clamps, idx, R1o);
+        round_up(p->n, 64), As ? As->row_unscale : nullptr, gamma2, clamps, idx, R1o, fin ? *fin : LinFinish{}, fin ? 1 : 0);
   }
   count_launch();
   return check_launch("k_vamp_row_scalar");

@@ -307,7 +307,8 @@ struct SolveIO {
 
 mpq_status run_linear_core(mpq_plan_s* p, int64_t m, double* gamma2, const double* gamma1_0,
                            double* beta, double* gamma1_out, float* Uprime, double* alpha2,
-                           double* beta_hat, int32_t* clamps, cudaStream_t st);
+                           double* beta_hat, int32_t* clamps, cudaStream_t st,
+                           LinFinish* defer_finish = nullptr);
 
 // linear half-iteration on workspace state (R1 may alias W on the first call)
 mpq_status run_linear(mpq_plan_s* p, const float* W, int64_t m, const float* R1,
@@ -334,9 +335,13 @@ int linear_e_bound(int64_t n) {
 // (w - r2) with its epilogue (the diagonal scaling D, the M-step's trace
 // sums, the second GEMM's operand D u), the M-step finisher, and G = V (D u)
 // into X1
+// defer_finish: the M-step finish is left to the caller's next fused row
+// kernel (its arguments returned here), and the second GEMM takes its row
+// scale as the first operand's times 2^e_bound (what the finish would write)
 mpq_status run_linear_core(mpq_plan_s* p, int64_t m, double* gamma2, const double* gamma1_0,
                            double* beta, double* gamma1_out, float* Uprime, double* alpha2,
-                           double* beta_hat, int32_t* clamps, cudaStream_t st) {
+                           double* beta_hat, int32_t* clamps, cudaStream_t st,
+                           LinFinish* defer_finish) {
   Workspace& w = p->ws;
   const int64_t n = p->n, r = p->r;
   LinEpi le;
@@ -355,6 +360,15 @@ mpq_status run_linear_core(mpq_plan_s* p, int64_t m, double* gamma2, const doubl
   o.lin = &le;
   MPQ_TRY(gemm_tc(w.As, w.tm_an_hi, w.tm_an_lo, p->Vt_s, p->tm_vt_hi, p->tm_vt_lo, w.P, r, m, r, n,
                   p->Vt_s.unscale_host, p->status, st, "gemm_project", o));
+  if (defer_finish) {
+    *defer_finish = make_lin_finish(p, m, w.lin_part, le.ntiles, le.e_bound, w.As.row_unscale,
+                                    nullptr, gamma2, gamma1_0, beta, gamma1_out, w.coef, w.kappa,
+                                    alpha2, beta_hat, clamps);
+    SplitOperand aq = w.Aq;
+    aq.row_unscale = w.As.row_unscale;  // times 2^e_bound, folded into b_scale (exact)
+    return gemm_tc(aq, w.tm_aq_hi, w.tm_aq_lo, p->V_s, p->tm_v_hi, p->tm_v_lo, w.X1, n, m, n, r,
+                   ldexpf(p->V_s.unscale_host, le.e_bound), p->status, st, "gemm_expand");
+  }
   MPQ_TRY(launch_linear_finish(p, m, w.lin_part, le.ntiles, le.e_bound, w.As.row_unscale,
                                w.Aq.row_unscale, gamma2, gamma1_0, beta, gamma1_out, w.coef,
                                w.kappa, alpha2, beta_hat, clamps, st));
@@ -424,18 +438,20 @@ mpq_status solve_batch(mpq_plan_s* p, const SolveIO& io, int64_t row0, int64_t m
   if (p->d == 1 && vamp_row_threads(n, p->G) > 0) {
     // scalar rows: l2d, denoiser and d2l of an iteration in one fused row
     // kernel (r1 never leaves the chip), then the linear module
+    // (each linear step's M-step finish runs in the next row kernel's prologue)
+    LinFinish fin{};
     for (int t = 0; t < io.T_vamp; ++t) {
       MPQ_TRY(launch_vamp_row_scalar(p, W, mb, t == 0, 0, w.X1, w.R2, w.coef, w.kappa, w.gamma1,
                                      w.scale, w.offset, w.gamma1_0, &w.As, w.gamma2, clamps,
-                                     nullptr, st));
+                                     nullptr, st, nullptr, t > 0 ? &fin : nullptr));
       MPQ_TRY(run_linear_core(p, mb, w.gamma2, w.gamma1_0, w.beta, w.gamma1, nullptr, nullptr,
-                              nullptr, clamps, st));
+                              nullptr, clamps, st, &fin));
     }
     // marginal MAP: argmax of the denoiser at the last cavity
     if (io.T_vamp > 0)
       MPQ_TRY(launch_vamp_row_scalar(p, W, mb, 0, 1, w.X1, w.R2, w.coef, w.kappa, w.gamma1,
                                      w.scale, w.offset, w.gamma1_0, nullptr, nullptr, nullptr, idx,
-                                     st));
+                                     st, nullptr, &fin));
   } else {
     const float* R1 = W;  // cavity r1_0 = w
     float* vblock = (p->d == 8) ? w.R2 : nullptr;  // R2 is free while the denoiser runs

@@ -196,7 +196,30 @@ mpq_status launch_extrinsic_d2l(const mpq_plan_s* p, const float* W, int64_t m, 
 // reads p' from P, writes the GEMM2 A operand (split, K = r)
 // M-step finisher after the projection GEMM's linear epilogue: per row, the
 // column tiles' sums in a fixed order, then alpha2, beta_hat, the damped
-// beta, gamma1', the l2d coefficients and the second GEMM's row scale.
+// beta, gamma1', the l2d coefficients and the second GEMM's row scale.  Its
+// inputs and outputs (the fused row kernel can run it in its prologue):
+struct LinFinish {
+  const float2* part;
+  int ntiles, e_bound;
+  int64_t m, n, r;
+  const float* a_unscale;
+  float* q_unscale;  // NULL: the expand GEMM takes its row scale from a_unscale
+  const double* gamma2;
+  const double* gamma1_0;
+  double* beta;
+  double damping, glo, ghi, amin, amax;
+  double* gamma1_out;
+  double* coef;
+  double* kappa;
+  double* alpha2_out;
+  double* beta_hat_out;
+  int32_t* clamps;
+};
+LinFinish make_lin_finish(const mpq_plan_s* p, int64_t m, const float2* part, int ntiles,
+                          int e_bound, const float* a_unscale, float* q_unscale,
+                          const double* gamma2, const double* gamma1_0, double* beta,
+                          double* gamma1_out, double* coef, double* kappa, double* alpha2,
+                          double* beta_hat, int32_t* clamps);
 mpq_status launch_linear_finish(const mpq_plan_s* p, int64_t m, const float2* part, int ntiles,
                                 int e_bound, const float* a_unscale, float* q_unscale,
                                 const double* gamma2, const double* gamma1_0, double* beta,
@@ -208,7 +231,9 @@ mpq_status launch_vamp_row_scalar(const mpq_plan_s* p, const float* W, int64_t m
                                   const double* kappa, const double* gamma1, const float* scale,
                                   const float* offset, const double* gamma1_0, SplitOperand* As,
                                   double* gamma2, int32_t* clamps, uint16_t* idx, cudaStream_t st,
-                                  float* R1o = nullptr);
+                                  float* R1o = nullptr, const LinFinish* fin = nullptr);
+// (fin: the previous linear step's M-step finish, run per row by the kernel
+// before it reads gamma1, coef and kappa)
 mpq_status launch_extrinsic_l2d(const mpq_plan_s* p, const float* W, int64_t m, const float* R2,
                                 const float* G, const double* coef, const double* kappa,
                                 float* R1_out, float* xhat2, cudaStream_t st);
