@@ -210,54 +210,57 @@ __global__ void __launch_bounds__(256)
   for (int e = t; e < BJ_P * BJ_P; e += blockDim.x) qo[e] = Q[e / BJ_P][e % BJ_P];
 }
 
-// 64 x 64 x 64 products in shared memory, Z = Xt^T Y (Xt holds X transposed,
-// so that both operands are read along rows): each of 128 threads owns an
-// 8 x 4 block of Z and reads 8 + 4 values per k as 16-byte loads (6 loads per
-// 32 FMAs).  With tout the block is stored transposed.
-constexpr int BJ_THREADS = 128;
+// 64 x 64 x 64 products in shared memory, acc = (Xt^T Y) block (Xt holds X
+// transposed, so that both operands are read along rows): each of 256
+// threads owns a 4 x 4 block of the result, rows ti.., columns tj.., and
+// reads 4 + 4 values per k as 16-byte loads.
+constexpr int BJ_THREADS = 256;
 __device__ __forceinline__ void bj_mm(const double (*Xt)[BJ_LD], const double (*Y)[BJ_LD],
-                                      double (*Z)[BJ_LD], bool tout) {
-  const int ti = (threadIdx.x / 16) * 8, tj = (threadIdx.x % 16) * 4;
-  double acc[8][4] = {};
+                                      double (&acc)[4][4]) {
+  const int ti = (threadIdx.x / 16) * 4, tj = (threadIdx.x % 16) * 4;
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) acc[a][b] = 0.0;
+#pragma unroll 4
   for (int kk = 0; kk < BJ_P; ++kk) {
-    double xv[8], yv[4];
+    const double2 x0 = *reinterpret_cast<const double2*>(&Xt[kk][ti]);
+    const double2 x1 = *reinterpret_cast<const double2*>(&Xt[kk][ti + 2]);
+    const double2 y0 = *reinterpret_cast<const double2*>(&Y[kk][tj]);
+    const double2 y1 = *reinterpret_cast<const double2*>(&Y[kk][tj + 2]);
+    const double xv[4] = {x0.x, x0.y, x1.x, x1.y}, yv[4] = {y0.x, y0.y, y1.x, y1.y};
 #pragma unroll
-    for (int a = 0; a < 8; a += 2) {
-      const double2 v = *reinterpret_cast<const double2*>(&Xt[kk][ti + a]);
-      xv[a] = v.x;
-      xv[a + 1] = v.y;
-    }
-#pragma unroll
-    for (int b = 0; b < 4; b += 2) {
-      const double2 v = *reinterpret_cast<const double2*>(&Y[kk][tj + b]);
-      yv[b] = v.x;
-      yv[b + 1] = v.y;
-    }
-#pragma unroll
-    for (int a = 0; a < 8; ++a)
+    for (int a = 0; a < 4; ++a)
 #pragma unroll
       for (int b = 0; b < 4; ++b) acc[a][b] = fma(xv[a], yv[b], acc[a][b]);
   }
-#pragma unroll
-  for (int a = 0; a < 8; ++a)
-#pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      if (tout) Z[tj + b][ti + a] = acc[a][b];
-      else Z[ti + a][tj + b] = acc[a][b];
-    }
 }
 
-constexpr int BJ_APPLY_SMEM = 4 * BJ_TILE * (int)sizeof(double);
+// a thread's 4 x 4 result block to rows gr[ti + a], columns gc[tj .. tj+3] of
+// M (the 4 columns lie in one 32-column block: two 16-byte stores per row)
+__device__ __forceinline__ void bj_store(double* __restrict__ M, int64_t N, const int* gr,
+                                         int64_t r0, const int* gc, const double (&acc)[4][4]) {
+  const int ti = (threadIdx.x / 16) * 4, tj = (threadIdx.x % 16) * 4;
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    double* dst = M + (gr ? (int64_t)gr[ti + a] : r0 + ti + a) * N + gc[tj];
+    *reinterpret_cast<double2*>(dst) = make_double2(acc[a][0], acc[a][1]);
+    *reinterpret_cast<double2*>(dst + 2) = make_double2(acc[a][2], acc[a][3]);
+  }
+}
 
-// A[rows of pair I, cols of pair J] <- Q_I^T A_IJ Q_J (the tiles partition A)
+// two tiles of shared memory per CTA: three CTAs (24 warps) fit an SM
+constexpr int BJ_APPLY_SMEM = 2 * BJ_TILE * (int)sizeof(double);
+
+// A[rows of pair I, cols of pair J] <- Q_I^T A_IJ Q_J (the tiles partition A):
+// U = Q_I^T T into registers, U^T over Q_I's tile, Q_J over T's, then U Q_J
+// straight to A
 __global__ void __launch_bounds__(BJ_THREADS)
     k_bj_apply_a(double* __restrict__ A, int64_t N, int64_t nb, int64_t k,
                  const double* __restrict__ Qall) {
   extern __shared__ __align__(16) double bj_sm[];
-  double(*T)[BJ_LD] = reinterpret_cast<double(*)[BJ_LD]>(bj_sm);
-  double(*QI)[BJ_LD] = reinterpret_cast<double(*)[BJ_LD]>(bj_sm + BJ_TILE);
-  double(*QJ)[BJ_LD] = reinterpret_cast<double(*)[BJ_LD]>(bj_sm + 2 * BJ_TILE);
-  double(*U)[BJ_LD] = reinterpret_cast<double(*)[BJ_LD]>(bj_sm + 3 * BJ_TILE);
+  double(*X)[BJ_LD] = reinterpret_cast<double(*)[BJ_LD]>(bj_sm);
+  double(*Y)[BJ_LD] = reinterpret_cast<double(*)[BJ_LD]>(bj_sm + BJ_TILE);
   __shared__ int gI[BJ_P], gJ[BJ_P];
   const int t = threadIdx.x;
   if (t == 0) {
@@ -269,19 +272,22 @@ __global__ void __launch_bounds__(BJ_THREADS)
   const double* qj = Qall + (int64_t)blockIdx.x * BJ_P * BJ_P;
   for (int e = t; e < BJ_P * BJ_P; e += blockDim.x) {
     const int i = e / BJ_P, j = e % BJ_P;
-    T[i][j] = A[(int64_t)gI[i] * N + gJ[j]];
-    QI[i][j] = qi[e];
-    QJ[i][j] = qj[e];
+    X[i][j] = qi[e];
+    Y[i][j] = A[(int64_t)gI[i] * N + gJ[j]];
   }
   __syncthreads();
-  bj_mm(QI, T, U, true);   // U^T with U = Q_I^T T
+  double acc[4][4];
+  bj_mm(X, Y, acc);  // U = Q_I^T T
   __syncthreads();
-  bj_mm(U, QJ, T, false);  // T = U Q_J
+  const int ti = (t / 16) * 4, tj = (t % 16) * 4;
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) X[tj + b][ti + a] = acc[a][b];  // U^T
+  for (int e = t; e < BJ_P * BJ_P; e += blockDim.x) Y[e / BJ_P][e % BJ_P] = qj[e];
   __syncthreads();
-  for (int e = t; e < BJ_P * BJ_P; e += blockDim.x) {
-    const int i = e / BJ_P, j = e % BJ_P;
-    A[(int64_t)gI[i] * N + gJ[j]] = T[i][j];
-  }
+  bj_mm(X, Y, acc);  // U Q_J
+  bj_store(A, N, gI, 0, gJ, acc);
 }
 
 // V[rows r0 .. r0+63, cols of pair J] <- V[.., pair J] Q_J
@@ -291,7 +297,6 @@ __global__ void __launch_bounds__(BJ_THREADS)
   extern __shared__ __align__(16) double bj_sm[];
   double(*Tt)[BJ_LD] = reinterpret_cast<double(*)[BJ_LD]>(bj_sm);
   double(*QJ)[BJ_LD] = reinterpret_cast<double(*)[BJ_LD]>(bj_sm + BJ_TILE);
-  double(*U)[BJ_LD] = reinterpret_cast<double(*)[BJ_LD]>(bj_sm + 2 * BJ_TILE);
   __shared__ int gJ[BJ_P];
   const int t = threadIdx.x;
   const int64_t r0 = (int64_t)blockIdx.y * BJ_P;
@@ -304,12 +309,9 @@ __global__ void __launch_bounds__(BJ_THREADS)
     QJ[i][j] = qj[e];
   }
   __syncthreads();
-  bj_mm(Tt, QJ, U, false);  // U = T Q_J
-  __syncthreads();
-  for (int e = t; e < BJ_P * BJ_P; e += blockDim.x) {
-    const int i = e / BJ_P, j = e % BJ_P;
-    V[(r0 + i) * N + gJ[j]] = U[i][j];
-  }
+  double acc[4][4];
+  bj_mm(Tt, QJ, acc);  // T Q_J
+  bj_store(V, N, nullptr, r0, gJ, acc);
 }
 
 __global__ void k_eye(double* V, int64_t N) {
@@ -503,7 +505,7 @@ mpq_status jacobi_eig_blocked(const double* G, int64_t N0, double* lam, double* 
   MPQ_CUDA(cudaFuncSetAttribute(k_bj_apply_a, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 BJ_APPLY_SMEM));
   MPQ_CUDA(cudaFuncSetAttribute(k_bj_apply_v, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                3 * BJ_TILE * (int)sizeof(double)));
+                                BJ_APPLY_SMEM));
   {
     ProfScope ps_("k_pad", st);
     k_pad<<<g1(N * N), 256, 0, st>>>(G, N0, N, A.p);
@@ -543,8 +545,8 @@ mpq_status jacobi_eig_blocked(const double* G, int64_t N0, double* lam, double* 
       }
       {
         ProfScope ps_("k_bj_apply_v", st);
-        k_bj_apply_v<<<dim3((unsigned)npairs, (unsigned)(N / BJ_P)), BJ_THREADS,
-                       3 * BJ_TILE * sizeof(double), st>>>(V.p, N, nb, k, Q.p);
+        k_bj_apply_v<<<dim3((unsigned)npairs, (unsigned)(N / BJ_P)), BJ_THREADS, BJ_APPLY_SMEM,
+                       st>>>(V.p, N, nb, k, Q.p);
       }
       count_launch(3);
     }

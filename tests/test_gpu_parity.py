@@ -536,7 +536,9 @@ def test_invalid_arguments_are_rejected_before_launch(mpq):
 
 # ----------------------------------------------------------------- setup ---
 
-@pytest.mark.parametrize("m,n", [(300, 200), (150, 200), (64, 64)])
+# (600, 320) and (300, 520): a smaller side of 320 and 300 (>= 256) takes the
+# blocked Jacobi, the second one with a zero-padded pair of blocks
+@pytest.mark.parametrize("m,n", [(300, 200), (150, 200), (64, 64), (600, 320), (300, 520)])
 def test_setup_from_x_matches_oracle_spectrum(mpq, m, n):
     g = np.random.default_rng(m + n)
     X = mi.heavy_tailed_x(g, g, m, n).astype(np.float32)
