@@ -72,7 +72,32 @@ def parse():
     ap.add_argument("--gram-rows", type=int, default=262144,
                     help="also time the streamed fp64 Gram accumulation of this many calibration "
                          "rows (chunks of 16384 through mpq_gram_accumulate; 0 = skip)")
+    ap.add_argument("--rht-rows", type=int, default=32768,
+                    help="also time the random Hadamard rotation (mpq_rht, in place) of this "
+                         "many rows of the config's width (0 = skip)")
     return ap.parse_args()
+
+
+def rht_timing(n, rows, dev, reps=5):
+    """Average milliseconds (CUDA events on the current stream) of one
+    in-place random Hadamard rotation of a rows x n fp32 matrix, after one
+    warm-up.  At 32768 x 4096 the matrix is 512 MiB, four times L2, so every
+    rotation reads and writes HBM."""
+    import torch
+    import post_weight_quantization_row_b200 as mpq
+    g = torch.Generator(device=dev)
+    g.manual_seed(20261300)
+    X = torch.randn(rows, n, generator=g, device=dev, dtype=torch.float32)
+    signs = torch.where(torch.rand(n, generator=g, device=dev) < 0.5, -1.0, 1.0).to(torch.float32)
+    mpq.rht(X, signs)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        mpq.rht(X, signs)
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
 
 
 def gram_timing(n, rows, dev):
@@ -402,6 +427,13 @@ def run_mpq(args, world, rank, local):
         gram_run = {"rows": args.gram_rows, "n": n, "s": round(gs, 3),
                     "fp64_tflops": round(2.0 * args.gram_rows * n * n / gs / 1e12, 2),
                     "what": "streamed X^T X in fp64 (mpq_gram_accumulate, 16384-row chunks)"}
+    rht_run = None
+    if args.rht_rows > 0 and rank == 0 and n & (n - 1) == 0:
+        rms = rht_timing(n, args.rht_rows, dev)
+        rgbs = 8.0 * args.rht_rows * n / (rms / 1e3) / 1e9  # one fp32 read + one write per element
+        rht_run = {"rows": args.rht_rows, "n": n, "ms": round(rms, 4), "gbs": round(rgbs, 1),
+                   "hbm_frac": round(rgbs / load_peaks()[0]["hbm_gbs"], 3),
+                   "what": "in-place x <- (x .* signs) H_n / sqrt(n) (mpq_rht), 8 B per element"}
     W = torch.from_numpy(p.W).to(dev)
     out = {"idx": torch.empty(m, plan.B, dtype=torch.int16, device=dev),
            "w_hat": torch.empty(m, n, dtype=torch.float32, device=dev),
@@ -545,7 +577,7 @@ def run_mpq(args, world, rank, local):
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
                 "data": "synthetic", "config": cfgd,
                 "run": {"setup_s": None if setup_s is None else round(setup_s, 3),
-                        "gram": gram_run, "rank": r,
+                        "gram": gram_run, "rht": rht_run, "rank": r,
                         "cd_panel": args.cd_panel or "auto",
                         "parallelism": f"rows sharded over {world} GPU(s)"},
                 "rows_per_s": world * m / (ms_per_step / 1e3),

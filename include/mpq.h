@@ -213,7 +213,10 @@ MPQ_API mpq_status mpq_plan_create_from_gram(mpq_gram_t gram, const mpq_params* 
  * (rows x n fp32, row-major, device) becomes x Q^T, Q = H_n diag(signs) /
  * sqrt(n) with H_n the Sylvester-Hadamard matrix; apply it to both W and X
  * and the objective ||(W - W_hat) X^T||^2 is unchanged.  signs: n floats,
- * each +1 or -1 (device).  n a power of two in [1, MPQ_RHT_MAX_N].
+ * each +1 or -1 (device).  n a power of two in [1, MPQ_RHT_MAX_N].  Any
+ * alignment is accepted; with X and signs 16-byte aligned and 512 <= n <=
+ * 8192 the rotation takes four butterfly stages per pass in registers, else
+ * one shared-memory pass per stage, with the same result bits either way.
  * Asynchronous on `stream`. */
 #define MPQ_RHT_MAX_N 32768
 MPQ_API mpq_status mpq_rht(float* X, int64_t rows, int64_t n, const float* signs, mpq_stream_t stream);

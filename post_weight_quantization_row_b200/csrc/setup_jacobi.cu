@@ -681,11 +681,14 @@ mpq_status setup_spectrum_from_x(mpq_plan_s* p, const float* X, int64_t m, int64
 // only through its eigenvalues).  Every row x of X becomes x Q^T with
 // Q = H_n diag(signs) / sqrt(n), H_n the Sylvester-Hadamard matrix
 // (H_1 = [1], H_2k = [[H_k, H_k], [H_k, -H_k]]; symmetric), so that
-// x Q^T = (x .* signs) H_n / sqrt(n).  One CTA per row (grid-stride): the row
-// sits in shared memory and takes log2(n) butterfly stages; pair i of the
-// stage with half-width h is (lo, lo + h), lo = 2h floor(i / h) + i mod h.
+// x Q^T = (x .* signs) H_n / sqrt(n): log2(n) butterfly stages, the stage of
+// half-width h taking every pair (lo, lo + h) with bit log2(h) of lo clear to
+// (a + b, a - b).  Both kernels run the stages in the order h = 1, 2, 4, ...,
+// so they give the same bits.
 namespace {
 
+// Any n (a power of two up to 32768; used outside 512..8192): one CTA per row, the row in shared
+// memory, one pass over it per stage.
 __global__ void __launch_bounds__(512)
     k_rht(float* __restrict__ X, int64_t rows, int n, const float* __restrict__ signs,
           float inv_sqrt_n) {
@@ -708,17 +711,144 @@ __global__ void __launch_bounds__(512)
   }
 }
 
+// 512 <= n <= 8192: n / 16 threads per row, 16 values each in registers.
+// The log2(n) index bits are taken in passes of up to four: in the pass over
+// bits [b0, b0 + nb) value v = (vh << nb) | vl of thread t is element
+//   j = (r mod 2^b0) | (vl << b0) | ((r >> b0) << (b0 + nb)),  r = vh T + t,
+// so its nb stages are butterflies between registers.  The first pass
+// (b0 = 0, nb = 4) is the thread's 16 consecutive elements (four float4
+// loads); between passes the row goes through shared memory once.  The
+// shared-memory word of element j is j with its quad bits (2..4) XORed by a
+// function of the 32-word line (j >> 5): line mod 8, and 4 more when bit 3 of
+// the line is set.  That keeps the float4 stores of the first pass and the
+// 32-lane scalar accesses of the later ones free of bank conflicts.
+constexpr int RHT_V = 16;
+constexpr int RHT_MIN_N = 512, RHT_MAX_N = 8192;
+
+__device__ __forceinline__ int rht_swz(int j) {
+  const int line = j >> 5;
+  const int g = (line & 7) ^ (((line >> 3) & 1) << 2);
+  return j ^ (g << 2);
+}
+
+__device__ __forceinline__ int rht_elem(int t, int v, int T, int b0, int nb) {
+  const int r = (v >> nb) * T + t;
+  return (r & ((1 << b0) - 1)) | ((v & ((1 << nb) - 1)) << b0) | ((r >> b0) << (b0 + nb));
+}
+
+template <int NB>
+__device__ __forceinline__ void rht_reg_stages(float (&a)[RHT_V]) {
+#pragma unroll
+  for (int s = 0; s < NB; ++s) {
+#pragma unroll
+    for (int v = 0; v < RHT_V; ++v) {
+      if (((v >> s) & 1) == 0) {
+        const float p = a[v], q = a[v + (1 << s)];
+        a[v] = p + q;
+        a[v + (1 << s)] = p - q;
+      }
+    }
+  }
+}
+
+// One pass over bits [B0, B0 + NB) after the previous pass over [PB0, B0):
+// hand the row over through shared memory, then NB register stages.
+template <int L, int PB0, int B0>
+__device__ __forceinline__ void rht_pass(float (&a)[RHT_V], float* sx, int t) {
+  constexpr int T = (1 << L) / RHT_V;
+  constexpr int NB = (L - B0) < 4 ? (L - B0) : 4;
+  if constexpr (B0 > 4) {
+#pragma unroll
+    for (int v = 0; v < RHT_V; ++v) sx[rht_swz(rht_elem(t, v, T, PB0, B0 - PB0))] = a[v];
+  }
+  __syncthreads();
+#pragma unroll
+  for (int v = 0; v < RHT_V; ++v) a[v] = sx[rht_swz(rht_elem(t, v, T, B0, NB))];
+  __syncthreads();  // every read done before the next hand-over or row
+  rht_reg_stages<NB>(a);
+  if constexpr (B0 + NB < L) rht_pass<L, B0, B0 + NB>(a, sx, t);
+}
+
+// At n = 4096 the register bound of 80 (three CTAs per SM) holds the 16
+// values and their addresses without spilling.
+template <int L>
+__global__ void __launch_bounds__((1 << L) / RHT_V, L == 12 ? 3 : 1)
+    k_rht_reg(float* __restrict__ X, int64_t rows, const float* __restrict__ signs,
+              float inv_sqrt_n) {
+  extern __shared__ float sx[];
+  constexpr int n = 1 << L;
+  constexpr int T = n / RHT_V;
+  constexpr int LB0 = 4 * ((L - 1) / 4), LNB = L - LB0;  // the last pass
+  const int t = threadIdx.x;
+  float a[RHT_V];
+  for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
+    float* x = X + row * (int64_t)n;
+#pragma unroll
+    for (int q = 0; q < RHT_V / 4; ++q) {
+      const float4 x4 = __ldcs(reinterpret_cast<const float4*>(x + RHT_V * t) + q);
+      const float4 s4 = __ldg(reinterpret_cast<const float4*>(signs + RHT_V * t) + q);
+      a[4 * q] = x4.x * s4.x;
+      a[4 * q + 1] = x4.y * s4.y;
+      a[4 * q + 2] = x4.z * s4.z;
+      a[4 * q + 3] = x4.w * s4.w;
+    }
+    rht_reg_stages<4>(a);
+    // first hand-over: the 16 consecutive elements as four float4 stores
+#pragma unroll
+    for (int q = 0; q < RHT_V / 4; ++q)
+      *reinterpret_cast<float4*>(sx + rht_swz(RHT_V * t + 4 * q)) =
+          make_float4(a[4 * q], a[4 * q + 1], a[4 * q + 2], a[4 * q + 3]);
+    rht_pass<L, 0, 4>(a, sx, t);
+    // last pass: its bits start at 8 or above, so a warp's 32 lanes store 32
+    // consecutive floats
+#pragma unroll
+    for (int v = 0; v < RHT_V; ++v) __stcs(x + rht_elem(t, v, T, LB0, LNB), a[v] * inv_sqrt_n);
+  }
+}
+
+template <int L>
+mpq_status launch_rht_reg(float* X, int64_t rows, const float* signs, float inv_sqrt_n, int sms,
+                          cudaStream_t st) {
+  constexpr int threads = (1 << L) / RHT_V;
+  constexpr size_t smem = sizeof(float) << L;
+  MPQ_CUDA(cudaFuncSetAttribute(k_rht_reg<L>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  int per_sm = 0;
+  MPQ_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_rht_reg<L>, threads, smem));
+  const unsigned grid = (unsigned)std::min<int64_t>(rows, (int64_t)sms * std::max(1, per_sm));
+  {
+    ProfScope ps_("k_rht", st);
+    k_rht_reg<L><<<grid, threads, smem, st>>>(X, rows, signs, inv_sqrt_n);
+  }
+  count_launch();
+  return check_launch("k_rht_reg");
+}
+
 }  // namespace
 
 mpq_status launch_rht(float* X, int64_t rows, int64_t n, const float* signs, cudaStream_t st) {
   if (rows == 0) return MPQ_OK;
-  const int threads = (int)std::min<int64_t>(512, std::max<int64_t>(32, n / 2));
+  const float inv_sqrt_n = (float)(1.0 / sqrt((double)n));
+  int dev = 0, sms = 0;
+  MPQ_CUDA(cudaGetDevice(&dev));
+  MPQ_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
   const size_t smem = sizeof(float) * (size_t)n;
+  if (n >= RHT_MIN_N && n <= RHT_MAX_N && (reinterpret_cast<uintptr_t>(X) & 15) == 0 &&
+      (reinterpret_cast<uintptr_t>(signs) & 15) == 0) {
+    switch (n) {
+      case 512: return launch_rht_reg<9>(X, rows, signs, inv_sqrt_n, sms, st);
+      case 1024: return launch_rht_reg<10>(X, rows, signs, inv_sqrt_n, sms, st);
+      case 2048: return launch_rht_reg<11>(X, rows, signs, inv_sqrt_n, sms, st);
+      case 4096: return launch_rht_reg<12>(X, rows, signs, inv_sqrt_n, sms, st);
+      case 8192: return launch_rht_reg<13>(X, rows, signs, inv_sqrt_n, sms, st);
+      default: break;
+    }
+  }
+  const int threads = (int)std::min<int64_t>(512, std::max<int64_t>(32, n / 2));
   MPQ_CUDA(cudaFuncSetAttribute(k_rht, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-  const unsigned grid = (unsigned)std::min<int64_t>(rows, 148 * 8);
+  const unsigned grid = (unsigned)std::min<int64_t>(rows, (int64_t)sms * 8);
   {
     ProfScope ps_("k_rht", st);
-    k_rht<<<grid, threads, smem, st>>>(X, rows, (int)n, signs, (float)(1.0 / sqrt((double)n)));
+    k_rht<<<grid, threads, smem, st>>>(X, rows, (int)n, signs, inv_sqrt_n);
   }
   count_launch();
   return check_launch("k_rht");

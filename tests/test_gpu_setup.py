@@ -159,7 +159,8 @@ def signs_of(seed, n):
     return np.where(np.random.default_rng(seed).random(n) < 0.5, -1.0, 1.0).astype(np.float32)
 
 
-@pytest.mark.parametrize("rows,n", [(5, 1), (7, 2), (37, 64), (2000, 64), (9, 1024), (3, 4096)])
+@pytest.mark.parametrize("rows,n", [(5, 1), (7, 2), (37, 64), (2000, 64), (11, 512), (9, 1024),
+                                    (300, 2048), (3, 4096), (5, 8192)])
 def test_rht_matches_dense_hadamard(mpq, rows, n):
     # 2000 rows: more rows than CTAs, so CTAs walk several rows
     g = np.random.default_rng(rows * 7 + n)
@@ -196,6 +197,34 @@ def test_rht_large_rows_kronecker_and_involution(mpq, n):
     mpq.rht(mpq.rht(Y, ones), ones)
     back = host(Y).astype(np.float64)
     assert np.abs(back - X).max() <= 1e-5 * np.abs(X).max()
+
+
+@pytest.mark.parametrize("n", [512, 4096, 8192])
+def test_rht_register_passes_match_the_stage_per_bit_kernel_bit_for_bit(mpq, n):
+    # widths 512..8192 on 16-byte aligned buffers take the kernel that runs
+    # four butterfly stages per pass in registers; a buffer one float off
+    # that alignment takes the kernel with one shared-memory pass per stage.
+    # Both run the stages in the order h = 1, 2, 4, ..., so the bits agree.
+    # 2000 rows at n = 4096 also walk several rows per CTA.
+    rows = 2000 if n == 4096 else 300
+    g = np.random.default_rng(n + 3)
+    X = g.standard_normal((rows, n)).astype(np.float32)
+    sg = cu(signs_of(n + 5, n))
+    A = cu(X.copy())
+    flat = torch.zeros(rows * n + 1, dtype=torch.float32, device="cuda")
+    B = flat[1:].view(rows, n)
+    B.copy_(A)
+    assert A.data_ptr() % 16 == 0 and B.data_ptr() % 16 == 4
+    mpq.rht(A, sg)
+    mpq.rht(B, sg)
+    assert torch.equal(A, B)
+    # and a sample of rows against the dense matrix
+    pick = np.arange(0, rows, rows // 8)
+    Q_T = (host(sg)[:, None].astype(np.float64) * scipy.linalg.hadamard(n)) / math.sqrt(n)
+    ref = X[pick].astype(np.float64) @ Q_T
+    got = host(A)[pick].astype(np.float64)
+    err = np.linalg.norm(got - ref, axis=1) / np.linalg.norm(ref, axis=1)
+    assert err.max() <= 4e-7 * math.log2(n)
 
 
 def test_rht_preserves_the_objective(mpq):
