@@ -63,6 +63,10 @@ def check_greedy(mpq, p, group=0, damp=0.01, cd_panel=0, sweeps=0, min_clean=0.5
     assert clean.mean() >= min_clean, f"only {clean.mean():.2f} of rows free of near-ties"
     assert np.array_equal(got[clean], ref.idx[clean])
     assert np.all(np.abs(e[clean] - ref.energy[clean]) <= ENERGY_TOL * ref.energy[clean])
+    # the layer's sum includes the tie-exempt rows, which may part from the
+    # oracle at a near-tie and end in another local minimum of the same
+    # objective: a sanity bound on their net drift, not the stated bar
+    # (that is the per-row check above)
     assert abs(e.sum() - ref.energy.sum()) <= 1e-2 * ref.energy.sum()
     return ref, out
 

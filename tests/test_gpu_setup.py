@@ -150,6 +150,10 @@ def test_solve_on_gram_plan_matches_oracle(mpq, d):
     assert np.array_equal(idx_np(out["idx"])[clean], ref.idx[clean])
     e = host(out["energy"]).astype(np.float64)
     assert np.all(np.abs(e[clean] - ref.energy[clean]) <= ENERGY_TOL * ref.energy[clean])
+    # the layer's sum includes the tie-exempt rows, which may part from the
+    # oracle at a near-tie and end in another local minimum of the same
+    # objective: a sanity bound on their net drift, not the stated bar
+    # (that is the per-row check above)
     assert abs(e.sum() - ref.energy.sum()) <= 1e-2 * ref.energy.sum()
 
 
